@@ -1,0 +1,10 @@
+"""CPU oracle of the sparse MoE layer forward pass (test infrastructure only).
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+use this package. The CUDA library never imports it.
+"""
+from .moe_oracle import *  # noqa: F401,F403
+from .moe_oracle import (capacity_from_factor, router_logits, softmax_over_experts,  # noqa: F401
+                         select_top_k, renormalise, assign_capacity_slots, route_from_logits,
+                         expert_permutation, silu, gelu, expert_ffn, combine,
+                         moe_layer_forward)

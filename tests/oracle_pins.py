@@ -1,0 +1,279 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each ``pin_*`` function takes the oracle module and raises AssertionError when
+the oracle disagrees with:
+
+* values printed on the pages (capacity limits and drop counts of the second
+  demo script, active-parameter counts of the first);
+* routing worked out by hand (a tie, renormalised weights, drops, row order);
+* expert outputs worked out by hand from textbook constants;
+* brute force on tiny inputs (all k-subsets; capacity slots by their rank
+  definition rather than the oracle's running counter);
+* the dense special case k = N with no capacity limit, which must equal the
+  softmax-weighted mixture of all experts;
+* invariants (weights sum to one, no expert above capacity, kept pairs precede
+  dropped pairs, a fully dropped token leaves the residual unchanged).
+
+They live in a plain module so ``test_oracle_mutations.py`` can plant mistakes
+in the oracle and check that some pin catches each one.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------- capacity / drops
+def pin_capacity_demo(o):
+    g = _golden("capacity_demo.json")
+    T, N = g["tokens"], g["experts"]
+    loads = g["collapsed_tokens_per_expert"]
+    assert sum(loads) == T
+    # a top-1 routing with exactly those per-expert loads, tokens interleaved
+    idx = []
+    remaining = list(loads)
+    while any(remaining):
+        for e in range(N):
+            if remaining[e]:
+                idx.append(e)
+                remaining[e] -= 1
+    topk_idx = np.array(idx, dtype=np.int64)[:, None]
+    for case in g["cases"]:
+        cap = o.capacity_from_factor(case["capacity_factor"], T, N)
+        assert cap == case["capacity"], (cap, case)
+        slot, kept = o.assign_capacity_slots(topk_idx, cap, N)
+        assert int((slot < 0).sum()) == case["dropped"], (int((slot < 0).sum()), case)
+        assert list(kept) == [min(c, cap) for c in loads]
+
+
+def pin_capacity_formula(o):
+    assert o.capacity_from_factor(1.25, 64, 8) == 10
+    assert o.capacity_from_factor(1.0, 4096, 64) == 64
+    assert o.capacity_from_factor(1.25, 16384, 256) == 80
+    assert o.capacity_from_factor(1.0, 3, 4) == 1          # rounds up
+    assert o.capacity_from_factor(1.0, 33, 8) == 5
+    assert o.capacity_from_factor(None, 17, 4) == 17      # unlimited
+    assert o.capacity_from_factor(float("inf"), 17, 4) == 17
+
+
+# ----------------------------------------------------------------- hand routing case
+def pin_hand_routing(o):
+    g = _golden("hand_case_top2_cap1.json")
+    L = np.array(g["logits"], dtype=np.float64)
+    T, N = L.shape
+    cap = o.capacity_from_factor(g["capacity_factor"], T, N)
+    assert cap == g["capacity"]
+    r = o.route_from_logits(L, g["top_k"], cap)
+    assert r["topk_idx"].tolist() == g["topk_idx"]
+    np.testing.assert_allclose(r["topk_w"], np.array(g["topk_w"]), rtol=0, atol=1e-15)
+    assert r["slot"].tolist() == g["slot"]
+    assert r["expert_count"].tolist() == g["expert_count"]
+    off, rop, por = o.expert_permutation(r["topk_idx"], r["slot"], r["expert_count"])
+    assert off.tolist() == g["expert_offset"]
+    assert rop.tolist() == g["row_of_pair"]
+    assert por.tolist() == g["pair_of_row"]
+    u = g["unlimited"]
+    r = o.route_from_logits(L, g["top_k"], u["capacity"])
+    assert r["slot"].tolist() == u["slot"]
+    assert r["expert_count"].tolist() == u["expert_count"]
+    off, rop, por = o.expert_permutation(r["topk_idx"], r["slot"], r["expert_count"])
+    assert off.tolist() == u["expert_offset"]
+    assert rop.tolist() == u["row_of_pair"]
+    assert por.tolist() == u["pair_of_row"]
+
+
+def pin_top1_weight_is_one(o):
+    rng = np.random.default_rng(7)
+    L = rng.normal(size=(20, 6))
+    r = o.route_from_logits(L, 1, 20)
+    assert np.all(r["topk_w"] == 1.0)
+    assert r["topk_idx"][:, 0].tolist() == np.argmax(L, axis=1).tolist()
+
+
+def pin_two_way_weights(o):
+    # k=2: w0 = logistic(a - b) for the two chosen logits a > b
+    L = np.array([[0.0, 1.0, -3.0, 0.5], [2.0, 2.0, 0.0, 1.0]])
+    r = o.route_from_logits(L, 2, 2)
+    assert r["topk_idx"].tolist() == [[1, 3], [0, 1]]
+    np.testing.assert_allclose(r["topk_w"][0], [0.6224593312018546, 0.3775406687981454], atol=1e-15)
+    np.testing.assert_allclose(r["topk_w"][1], [0.5, 0.5], atol=0)
+
+
+# ----------------------------------------------------------------- brute force
+def _brute_topk(row, k):
+    """The k-subset whose sorted logits are lexicographically largest; among equal
+    ones the lexicographically smallest sorted index tuple; best first."""
+    N = len(row)
+    best = None
+    for S in itertools.combinations(range(N), k):
+        vals = tuple(sorted((row[e] for e in S), reverse=True))
+        key = (vals, tuple(-e for e in S))
+        if best is None or key > best[0]:
+            best = (key, S)
+    S = best[1]
+    return sorted(S, key=lambda e: (-row[e], e))
+
+
+def _brute_slots(idx, cap):
+    """slot(t, j) = number of earlier pairs (in (choice, token) order) with the same expert."""
+    T, k = idx.shape
+    slot = np.full((T, k), -1)
+    for t in range(T):
+        for j in range(k):
+            e = idx[t, j]
+            rank = sum(1 for jj in range(k) for tt in range(T)
+                       if (jj, tt) < (j, t) and idx[tt, jj] == e)
+            slot[t, j] = rank if rank < cap else -1
+    return slot
+
+
+def pin_brute_force_routing(o):
+    rng = np.random.default_rng(1234)
+    for trial in range(60):
+        T = int(rng.integers(1, 9))
+        N = int(rng.integers(2, 7))
+        k = int(rng.integers(1, N + 1))
+        # small integers force many exact ties
+        L = rng.integers(-2, 3, size=(T, N)).astype(np.float64)
+        cap = int(rng.integers(0, T + 1))
+        r = o.route_from_logits(L, k, cap)
+        for t in range(T):
+            assert r["topk_idx"][t].tolist() == _brute_topk(L[t].tolist(), k), (L[t], k)
+        assert r["slot"].tolist() == _brute_slots(r["topk_idx"], cap).tolist()
+        for e in range(N):
+            c_e = int((r["topk_idx"] == e).sum())
+            assert r["expert_count"][e] == min(c_e, cap)
+        # weights: softmax of the chosen logits, computed directly
+        for t in range(T):
+            sel = L[t, r["topk_idx"][t]]
+            ex = [math.exp(v - sel.max()) for v in sel]
+            np.testing.assert_allclose(r["topk_w"][t], [v / sum(ex) for v in ex], rtol=1e-13, atol=0)
+
+
+# ----------------------------------------------------------------- expert FFN
+def pin_ffn_hand_cases(o):
+    g = _golden("ffn_hand_cases.json")
+    for act in ("swiglu", "gelu"):
+        c = g[act]
+        y = o.expert_ffn(np.array(c["x"], float), np.array(c["w_gate_up"], float),
+                         np.array(c["w_down"], float), act)
+        np.testing.assert_allclose(y, np.array(c["y"]), rtol=0, atol=2e-15)
+
+
+def pin_activation_limits(o):
+    z = np.array([0.0, 30.0, -30.0, 1.0, -1.0])
+    s = o.silu(z)
+    assert s[0] == 0.0 and abs(s[1] - 30.0) < 1e-11 and abs(s[2]) < 1e-11
+    np.testing.assert_allclose(s[3] - s[4], 1.0, atol=1e-15)        # silu(z) - silu(-z) = z
+    gl = o.gelu(z)
+    assert gl[0] == 0.0 and abs(gl[1] - 30.0) < 1e-12 and abs(gl[2]) < 1e-12
+    np.testing.assert_allclose(gl[3] - gl[4], 1.0, atol=1e-15)      # gelu(z) - gelu(-z) = z
+
+
+# ----------------------------------------------------------------- whole layer
+def _small_layer(rng, T, d, N, F, act):
+    x = rng.normal(size=(T, d))
+    wr = rng.normal(size=(N, d)) / math.sqrt(d)
+    rows = 2 * F if act == "swiglu" else F
+    wgu = rng.normal(size=(N, rows, d)) * 0.3
+    wd = rng.normal(size=(N, d, F)) * 0.3
+    return x, wr, wgu, wd
+
+
+def pin_dense_special_case(o):
+    """k = N with no capacity limit: sum_e softmax(L)_e * E_e(x) over every expert."""
+    rng = np.random.default_rng(99)
+    for act in ("swiglu", "gelu"):
+        T, d, N, F = 7, 5, 4, 3
+        x, wr, wgu, wd = _small_layer(rng, T, d, N, F, act)
+        res = rng.normal(size=(T, d))
+        got = o.moe_layer_forward(x, wr, wgu, wd, top_k=N, act=act, capacity=T, residual=res)["out"]
+        L = x @ wr.T
+        want = res.copy()
+        for t in range(T):
+            ex = np.array([math.exp(v - L[t].max()) for v in L[t]])
+            p = ex / ex.sum()
+            for e in range(N):
+                want[t] += p[e] * o.expert_ffn(x[t:t + 1], wgu[e], wd[e], act)[0]
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def pin_single_expert_layer(o):
+    """k = 1 with no limit: out[t] = res[t] + E_argmax(x[t]); token order irrelevant."""
+    rng = np.random.default_rng(5)
+    T, d, N, F = 9, 4, 3, 2
+    x, wr, wgu, wd = _small_layer(rng, T, d, N, F, "swiglu")
+    got = o.moe_layer_forward(x, wr, wgu, wd, top_k=1, act="swiglu", capacity=T, residual=x)["out"]
+    L = x @ wr.T
+    for t in range(T):
+        e = int(np.argmax(L[t]))
+        want = x[t] + o.expert_ffn(x[t:t + 1], wgu[e], wd[e], "swiglu")[0]
+        np.testing.assert_allclose(got[t], want, rtol=1e-13, atol=1e-13)
+
+
+def pin_invariants(o):
+    rng = np.random.default_rng(2024)
+    for trial in range(12):
+        T = int(rng.integers(4, 40))
+        N = int(rng.integers(2, 9))
+        k = int(rng.integers(1, min(N, 4) + 1))
+        d, F = 6, 4
+        x, wr, wgu, wd = _small_layer(rng, T, d, N, F, "swiglu")
+        cap = o.capacity_from_factor(float(rng.choice([0.5, 1.0, 1.25])), T, N)
+        r = o.moe_layer_forward(x, wr, wgu, wd, top_k=k, act="swiglu", capacity=cap, residual=x)
+        np.testing.assert_allclose(r["topk_w"].sum(axis=1), 1.0, rtol=0, atol=1e-14)
+        assert np.all(r["expert_count"] <= cap)
+        # per expert: kept pairs come before dropped pairs in (choice, token) order
+        for e in range(N):
+            seen_drop = False
+            for j in range(k):
+                for t in range(T):
+                    if r["topk_idx"][t, j] != e:
+                        continue
+                    if r["slot"][t, j] < 0:
+                        seen_drop = True
+                    else:
+                        assert not seen_drop
+        # a token with every choice dropped leaves the residual unchanged, bit for bit
+        all_dropped = np.all(r["slot"] < 0, axis=1)
+        assert np.array_equal(r["out"][all_dropped], x[all_dropped])
+        # the dropped-pair count obeys sum_e max(0, c_e - cap)
+        c = [int((r["topk_idx"] == e).sum()) for e in range(N)]
+        assert int((r["slot"] < 0).sum()) == sum(max(0, ce - cap) for ce in c)
+
+
+def pin_zero_down_weights(o):
+    rng = np.random.default_rng(3)
+    T, d, N, F = 6, 4, 3, 5
+    x, wr, wgu, wd = _small_layer(rng, T, d, N, F, "gelu")
+    out = o.moe_layer_forward(x, wr, wgu, np.zeros_like(wd), top_k=2, act="gelu",
+                              capacity=T, residual=x)["out"]
+    assert np.array_equal(out, x)
+
+
+def pin_active_params_demo(o_unused=None):
+    """The page's active/total parameter arithmetic (router + k experts; router + N experts)."""
+    g = _golden("active_params_demo.json")
+    d, h, N = g["d_model"], g["hidden"], g["experts"]
+    expert = d * h + h + h * d + d
+    router = d * N
+    assert router + 1 * expert == g["top1_active"]
+    assert router + 2 * expert == g["top2_active"]
+    assert router + N * expert == g["total"]
+
+
+ALL_PINS = [pin_capacity_demo, pin_capacity_formula, pin_hand_routing, pin_top1_weight_is_one,
+            pin_two_way_weights, pin_brute_force_routing, pin_ffn_hand_cases,
+            pin_activation_limits, pin_dense_special_case, pin_single_expert_layer,
+            pin_invariants, pin_zero_down_weights]

@@ -1,0 +1,120 @@
+"""Plant plausible mistakes in the CPU oracle and check that some pin catches each.
+
+The mistakes are planted in the oracle module on the CPU, for the duration of one
+test, with monkeypatch; nothing here touches the CUDA path.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle.moe_oracle as om
+from tests import oracle_pins
+
+
+def _silu_sign(z):
+    return z / (1.0 + np.exp(z))
+
+
+def _gelu_tanh(z):
+    return 0.5 * z * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (z + 0.044715 * z ** 3)))
+
+
+def _ffn_transposed_down(rows, wgu, wd, act):
+    if act == "swiglu":
+        F = wgu.shape[0] // 2
+        h = om.silu(rows @ wgu[:F].T) * (rows @ wgu[F:].T)
+    else:
+        h = om.gelu(rows @ wgu.T)
+    return h @ wd if wd.shape[0] == wd.shape[1] else h @ wd.T  # transposed when square
+
+
+def _ffn_gate_up_swapped(rows, wgu, wd, act):
+    if act == "swiglu":
+        F = wgu.shape[0] // 2
+        h = om.silu(rows @ wgu[F:].T) * (rows @ wgu[:F].T)
+    else:
+        h = om.gelu(rows @ wgu.T)
+    return h @ wd.T
+
+
+def _select_ties_high(logits, k):
+    T, N = logits.shape
+    idx = np.empty((T, k), dtype=np.int64)
+    for t in range(T):
+        order = np.lexsort((-np.arange(N), -logits[t]))
+        idx[t] = order[:k]
+    return idx
+
+
+def _no_renormalise(probs, idx):
+    return np.take_along_axis(probs, idx, axis=1)
+
+
+def _slots_token_major(idx, cap, n):
+    T, k = idx.shape
+    filled = np.zeros(n, dtype=np.int64)
+    slot = np.full((T, k), -1, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            if filled[e] < cap:
+                slot[t, j] = filled[e]
+                filled[e] += 1
+    return slot, filled
+
+
+def _capacity_floor(cf, T, n):
+    if cf is None or not math.isfinite(cf) or cf <= 0:
+        return T
+    return int(math.floor(cf * T / n))
+
+
+def _capacity_times_k(cf, T, n):
+    if cf is None or not math.isfinite(cf) or cf <= 0:
+        return T
+    return int(math.ceil(2 * cf * T / n))
+
+
+def _router_transposed_bias_sign(x, wr, b=None):
+    L = x @ wr.T
+    return L if b is None else L - b[None, :]
+
+
+def _softmax_no_shift_wrong_axis(logits):
+    ez = np.exp(logits)
+    return ez / ez.sum(axis=0, keepdims=True)
+
+
+def _combine_drops_residual(x, routing, wgu, wd, act, residual, tokens=None):
+    return _orig_combine(x, routing, wgu, wd, act, None, tokens)
+
+
+_orig_combine = om.combine
+
+MUTANTS = {
+    "silu_sign": ("silu", _silu_sign),
+    "gelu_tanh_approx": ("gelu", _gelu_tanh),
+    "down_transposed": ("expert_ffn", _ffn_transposed_down),
+    "gate_up_swapped": ("expert_ffn", _ffn_gate_up_swapped),
+    "ties_to_high_index": ("select_top_k", _select_ties_high),
+    "no_renormalise": ("renormalise", _no_renormalise),
+    "token_major_slots": ("assign_capacity_slots", _slots_token_major),
+    "capacity_floor": ("capacity_from_factor", _capacity_floor),
+    "capacity_times_k": ("capacity_from_factor", _capacity_times_k),
+    "softmax_wrong_axis": ("softmax_over_experts", _softmax_no_shift_wrong_axis),
+    "residual_dropped": ("combine", _combine_drops_residual),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_some_pin_catches(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(om, attr, fn)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(om)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, f"mutant {name} passed every pin"
