@@ -1,0 +1,479 @@
+#!/usr/bin/env python
+"""Benchmark: sparse MoE layer forward tokens/s on B200 (one JSON line on rank 0).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME[:T]] [--impl ours|reference]
+
+A step is one whole forward pass of the layer (route, permute, grouped expert FFN, combine)
+over one batch of synthetic tokens whose inputs already sit in HBM. Steps are timed one by one
+with CUDA events on the launching stream; L2 is flushed (a 256 MB write) before each step,
+outside the timed events. Under torchrun every rank runs its own replica of the workload
+(weak scaling, no collective on the data path). Rank 0 prints the line, with the time taken
+as the max over ranks.
+
+--impl reference times the CPU oracle (the plain float64 definition of the layer) on a bounded
+token sample of the same workload, on the host cores, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+DEFAULT_WORKLOAD = "switch_top1:4096"
+METRIC = "MoE-layer fwd tokens/s on 1 B200; % of bf16 tensor peak / % of HBM BW"
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SLOT_CHUNK = 4096  # (token, choice) pairs per block in the library's capacity pass
+
+
+# ----------------------------------------------------------------------------- workload model
+def parse_workload(spec: str):
+    name, _, t = spec.partition(":")
+    shape = synthetic.SHAPES[name]
+    T = int(t) if t else shape.token_counts[-1]
+    return shape, T
+
+
+def capacity_of(shape, T):
+    import sparse_mixture_experts_11_b200 as moe
+    return moe.capacity(shape.capacity_factor, T, shape.n_experts)
+
+
+def expert_params(d_model: int, d_ff: int, act: str, bias: bool = False) -> int:
+    """Parameters of one expert FFN: SwiGLU has gate, up and down projections; GELU up and down.
+    With bias=True each projection also carries a bias vector (the pages' demo expert)."""
+    if act == "swiglu":
+        n = 3 * d_model * d_ff
+        return n + (2 * d_ff + d_model if bias else 0)
+    n = 2 * d_model * d_ff
+    return n + (d_ff + d_model if bias else 0)
+
+
+def active_params(d_model: int, d_ff: int, n_experts: int, k: int, act: str, bias: bool) -> int:
+    """Parameters touched per token: the bias-free router plus k experts."""
+    return d_model * n_experts + k * expert_params(d_model, d_ff, act, bias)
+
+
+def algorithmic_bytes(shape, T: int, active_experts: int, R: int) -> dict:
+    """Bytes the layer must move (counting rules in the design notes).
+
+    layer: weights of every expert with at least one kept row, read once; router weight
+           (fp32); x read (bf16); out written (bf16). The residual is x itself.
+    ffn:   the same expert weights, plus x_perm read (bf16) and y_perm written (fp32).
+    """
+    d, F, N = shape.d_model, shape.d_ff, shape.n_experts
+    w = active_experts * expert_params(d, F, shape.act) * 2
+    layer = w + N * d * 4 + T * d * 2 + T * d * 2
+    ffn = w + R * d * 2 + R * d * 4
+    return {"layer": layer, "ffn": ffn, "weights": w}
+
+
+def ffn_flops(shape, R: int) -> int:
+    d, F = shape.d_model, shape.d_ff
+    return 2 * R * d * F * (3 if shape.act == "swiglu" else 2)
+
+
+def launches_per_step(T: int, k: int, R_max: int) -> int:
+    """Kernels one forward launches: router+top-k, capacity slots (1 pass, or 3 when the
+    arrivals span several chunks), permute, two grouped GEMMs (when rows can exist), combine."""
+    chunks = max(1, math.ceil(T * k / SLOT_CHUNK))
+    return 1 + (1 if chunks == 1 else 3) + 1 + (2 if R_max > 0 else 0) + 1
+
+
+def load_peaks():
+    if os.path.exists(MEASURED_PEAKS):
+        with open(MEASURED_PEAKS) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+class Layer:
+    """Device buffers of one layer invocation; stages called through the C ABI."""
+
+    def __init__(self, shape, T, device, seed=0):
+        import sparse_mixture_experts_11_b200 as moe
+        self.moe = moe
+        self.shape, self.T = shape, T
+        self.inp = synthetic.make_layer_inputs(shape, T, seed=seed, device=device)
+        cap = capacity_of(shape, T)
+        self.dims = moe.make_dims(T, shape.d_model, shape.n_experts, shape.top_k, shape.d_ff,
+                                  shape.act, cap)
+        self.R_max = moe.max_rows(self.dims)
+        self.fws = moe.new_workspace(self.dims, device, forward=True)
+        self.b = moe.forward_layout(self.dims, self.fws)
+        self.out = torch.empty((T, shape.d_model), dtype=torch.bfloat16, device=device)
+
+    def _view(self, ptr, n, dtype):
+        off = ptr - self.fws.data_ptr()
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return self.fws[off:off + nbytes].view(dtype)
+
+    def views(self):
+        s = self.shape
+        T, k, N = self.T, s.top_k, s.n_experts
+        b = self.b
+        return {"logits": self._view(b.logits, T * N, torch.float32).view(T, N),
+                "topk_idx": self._view(b.topk_idx, T * k, torch.int32).view(T, k),
+                "topk_w": self._view(b.topk_w, T * k, torch.float32).view(T, k),
+                "slot": self._view(b.slot, T * k, torch.int32).view(T, k),
+                "expert_count": self._view(b.expert_count, N, torch.int32),
+                "expert_offset": self._view(b.expert_offset, N + 1, torch.int32)}
+
+    def step_stages(self, ev):
+        """One forward as the four stage calls, with events between them (ev: 5 events)."""
+        moe, i, b, dims = self.moe, self.inp, self.b, self.dims
+        lib = moe._lib
+        d = moe.ctypes.byref(dims)
+        s = moe._stream(None)
+        P = moe.ctypes.c_void_p
+        ptr = lambda t: P(t.data_ptr()) if t is not None else None
+        ev[0].record()
+        moe._check(lib.moe_route(d, ptr(i["x"]), ptr(i["w_router"]), ptr(i["logit_bias"]),
+                                 P(b.logits), P(b.topk_idx), P(b.topk_w), P(b.slot),
+                                 P(b.expert_count), P(b.stage_ws), b.stage_ws_bytes, s), "route")
+        ev[1].record()
+        moe._check(lib.moe_permute(d, ptr(i["x"]), P(b.topk_idx), P(b.slot), P(b.expert_count),
+                                   P(b.expert_offset), P(b.row_of_pair), P(b.pair_of_row),
+                                   P(b.x_perm), P(b.stage_ws), b.stage_ws_bytes, s), "permute")
+        ev[2].record()
+        moe._check(lib.moe_grouped_ffn(d, P(b.x_perm), P(b.expert_offset), ptr(i["w_gate_up"]),
+                                       ptr(i["w_down"]), P(b.h), P(b.y_perm), P(b.stage_ws),
+                                       b.stage_ws_bytes, s), "grouped_ffn")
+        ev[3].record()
+        moe._check(lib.moe_unpermute_combine(d, P(b.y_perm), P(b.row_of_pair), P(b.topk_w),
+                                             ptr(i["x"]), ptr(self.out), 0, P(b.stage_ws),
+                                             b.stage_ws_bytes, s), "combine")
+        ev[4].record()
+
+    def forward_host(self, x_host, out_host):
+        """End to end through the public call: H2D of x, moe_forward, D2H of out."""
+        x = self.inp["x"]
+        x.copy_(x_host, non_blocking=True)
+        self.moe.forward_into(self.dims, x, self.inp["w_router"], self.inp["logit_bias"],
+                              self.inp["w_gate_up"], self.inp["w_down"], x, self.out, self.fws)
+        out_host.copy_(self.out, non_blocking=True)
+
+
+def flush_l2(buf):
+    buf.add_(1)  # 256 MB read-modify-write, larger than the 126 MB L2
+
+
+def run_gpu(args, rank, world, local_rank):
+    import sparse_mixture_experts_11_b200 as moe  # fails loudly without the CUDA library
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    shape, T = parse_workload(args.workload)
+    layer = Layer(shape, T, device)
+    flush = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    wev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+
+    for _ in range(args.warmup):
+        flush_l2(flush)
+        layer.step_stages(wev)
+    torch.cuda.synchronize()
+    err = moe.read_device_error(layer.fws, offset_bytes=layer.b.stage_ws - layer.fws.data_ptr())
+    if err != 0:
+        raise RuntimeError(f"device status after warm-up: {moe.status_string(err)}")
+
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(vis.split(",")[local_rank] if vis else local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for k in range(args.steps):
+        flush_l2(flush)
+        layer.step_stages(evs[k])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                for i, n in enumerate(["route", "permute", "grouped_ffn", "combine"])}
+    total_ms = sum(step_ms)
+    ffn_ms = stage_ms["grouped_ffn"]
+
+    # end to end through the public call with host buffers
+    x_host = layer.inp["x"].cpu().pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    for _ in range(args.warmup):
+        layer.forward_host(x_host, out_host)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record()
+    for _ in range(args.steps):
+        layer.forward_host(x_host, out_host)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    times = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    total_ms, e2e_ms = times.tolist()
+
+    v = layer.views()
+    counts = v["expert_count"].cpu()
+    R = int(counts.sum())
+    active = int((counts > 0).sum())
+    ab = algorithmic_bytes(shape, T, active, R)
+    peaks = load_peaks()
+    flops = ffn_flops(shape, R)
+    tensor_bound = flops / max(ab["ffn"], 1) > (peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9)
+    if tensor_bound:
+        ach = flops / (ffn_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(ach / peak, 4), "traffic": None,
+                "kernel": "moe_grouped_ffn (gate/up + down GEMM launches)",
+                "per_launch": f"{flops} FLOP", "peak_source": peaks["source"] + " sustained bf16"}
+    else:
+        ach = ab["ffn"] / (ffn_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "traffic": None,
+                "kernel": "moe_grouped_ffn (gate/up + down GEMM launches)",
+                "per_launch": f"{ab['ffn']} B", "peak_source": peaks["source"] + " copy"}
+
+    value = T * args.steps * world / (total_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; x~N(0,1) bf16, router W~N(0,1/d) fp32, expert W~N(0,0.02) bf16)",
+        "config": {"workload": shape.describe(T), "T": T, "d_model": shape.d_model,
+                   "n_experts": shape.n_experts, "top_k": shape.top_k, "d_ff": shape.d_ff,
+                   "act": shape.act, "capacity": layer.dims.capacity, "kept_rows": R,
+                   "active_experts": active,
+                   "l2": "flushed before every step (256 MB write outside the timed events); "
+                         "expert weights also exceed L2",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "stages_ms": {k: round(v_, 4) for k, v_ in stage_ms.items()},
+        "roofline": roof,
+        "layer_gbs": round(ab["layer"] / (total_ms / args.steps * 1e-3) / 1e9, 1),
+        "ffn_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 2),
+        "e2e": {"value": round(T * args.steps * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * shape.d_model * 2,
+                "d2h_bytes_per_step": T * shape.d_model * 2},
+        "gpu_launches": launches_per_step(T, shape.top_k, layer.R_max) * args.steps,
+        "clocks": clk,
+    }
+    return line, layer
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+def oracle_sample(shape, T, layer_inputs_cpu, n_tokens: int):
+    """Time the oracle's layer forward on the first n_tokens of the batch (routing over all T)."""
+    import numpy as np
+    import oracle
+    x = layer_inputs_cpu["x"]
+    cap = oracle.capacity_from_factor(shape.capacity_factor, T, shape.n_experts)
+    toks = np.arange(min(n_tokens, T))
+    t0 = time.perf_counter()
+    oracle.moe_layer_forward(x, layer_inputs_cpu["w_router"], layer_inputs_cpu["w_gate_up"],
+                             layer_inputs_cpu["w_down"], top_k=shape.top_k, act=shape.act,
+                             capacity=cap, logit_bias=layer_inputs_cpu["logit_bias"],
+                             residual=x, tokens=toks)
+    return time.perf_counter() - t0, len(toks)
+
+
+def cpu_inputs(shape, T, source: dict):
+    """float64 host copies of the inputs (weights converted one expert at a time, lazily)."""
+    import numpy as np
+    f = lambda t: None if t is None else t.detach().to("cpu", torch.float64).numpy()
+    wgu, wd = source["w_gate_up"], source["w_down"]
+    cache = {}
+
+    def lazy(w, tag):
+        def get(e):
+            key = (tag, e)
+            if key not in cache:
+                cache[key] = w[e].detach().to("cpu", torch.float64).numpy()
+            return cache[key]
+        return get
+    return {"x": f(source["x"]), "w_router": f(source["w_router"]), "logit_bias": f(source["logit_bias"]),
+            "w_gate_up": lazy(wgu, "gu"), "w_down": lazy(wd, "d"), "_cache": cache}
+
+
+def sample_tokens_for(shape, T) -> int:
+    """Tokens per oracle sample: a few seconds of float64 CPU work, and at most ~12 GB of
+    float64 expert weights touched (each token touches up to k experts)."""
+    p = expert_params(shape.d_model, shape.d_ff, shape.act)
+    by_flops = 4e10 // max(2 * shape.top_k * p, 1)
+    if min(shape.n_experts, T * shape.top_k) * p * 8 <= 12e9:
+        by_mem = T
+    else:
+        by_mem = 12e9 // (shape.top_k * p * 8)
+    return int(max(1, min(T, by_flops, by_mem)))
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(shape, T, source: dict) -> dict:
+    inp = cpu_inputs(shape, T, source)
+    n = sample_tokens_for(shape, T)
+    oracle_sample(shape, T, inp, n)   # converts the touched experts' weights to float64 once
+    dt, used = oracle_sample(shape, T, inp, n)
+    return {"value": round(used / dt, 2), "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"float64 oracle layer forward on the first {used} of {T} tokens "
+                      f"(routing and capacity over all {T}); {dt:.2f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    shape, T = parse_workload(args.workload)
+    src = synthetic.make_layer_inputs(shape, T, seed=0, device="cpu")
+    inp = cpu_inputs(shape, T, src)
+    n = sample_tokens_for(shape, T)
+    for _ in range(args.warmup):
+        oracle_sample(shape, T, inp, n)
+    dts = []
+    for _ in range(args.steps):
+        dt, used = oracle_sample(shape, T, inp, n)
+        dts.append(dt)
+    total = sum(dts)
+    value = used * args.steps / total
+    cores = blas_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": shape.describe(T), "T": T, "sample_tokens": used},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"float64 oracle on the first {used} of {T} tokens per step"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="shape[:T], shapes: " + ", ".join(synthetic.SHAPES))
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line, layer = run_gpu(args, rank, world, local_rank)
+        if rank == 0 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(layer.shape, layer.T, layer.inp)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,198 @@
+/*
+ * moe.h: C ABI of the sparse Mixture-of-Experts layer forward pass on NVIDIA B200 (sm_100a).
+ *
+ * The layer (page «Sparse Mixture-of-Experts», bigdataschool wiki):
+ *   1. router logits      L = x W_r^T (+ b), a linear layer without bias term
+ *                         (section «Роутер и top-k gating»; b is an optional per-expert
+ *                         additive logit bias used to skew loads);
+ *   2. softmax over the N experts, top-k experts per token, and the k probabilities
+ *      renormalised to sum to one (same section);
+ *   3. capacity: ceil(capacity_factor * T / N) slots per expert; a (token, choice) pair that
+ *      arrives at a full expert is dropped and contributes nothing, so a token whose every
+ *      choice is dropped leaves the layer unchanged through the residual
+ *      (section «Expert capacity и capacity factor»); arrival order is every token's first
+ *      choice in token order, then every token's second choice, and so on;
+ *   4. the kept pairs are sorted by expert id into expert-contiguous rows and every expert's
+ *      FFN runs as one grouped GEMM over packed expert weights (page «Что такое Mixture of
+ *      Experts (MoE) в трансформерах», aglamov.biz, sections «Бэкенд для экспертов»,
+ *      grouped_mm, and «Динамическая загрузка весов с WeightConverter», packed layouts);
+ *   5. the output is residual + the sum of the kept experts' outputs weighted by the
+ *      renormalised router probabilities (section «Роутер и top-k gating»).
+ *
+ * Conventions for every call:
+ *   - Every pointer is a DEVICE pointer, allocated and owned by the caller, 16-byte aligned.
+ *     The library allocates nothing and frees nothing. It keeps only two kinds of
+ *     process-wide state: a cached driver entry point and per-device attributes.
+ *   - "bf16" buffers hold bfloat16 bit patterns (uint16_t). All tensors are row-major and
+ *     contiguous.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *     default stream). No call synchronises with the host. The number of kept rows R lives
+ *     only on the device. Row buffers are sized for R_max = moe_max_rows().
+ *   - Host-side validation runs before any launch:
+ *       MOE_ERR_INVALID      null pointer where one is required, negative size, k > N, k < 1
+ *       MOE_ERR_UNSUPPORTED  d_model or d_ff not a multiple of 64, N > 256, k > 8, a pointer
+ *                            that is not 16-byte aligned, or a device that is not sm_100
+ *       MOE_ERR_WORKSPACE    ws_bytes below what moe_workspace_bytes() reports
+ *       MOE_ERR_CUDA         a CUDA runtime or driver call failed while launching
+ *     Nothing is launched when validation fails. T == 0 is valid and launches nothing.
+ *   - Faults found on the device are written into the workspace's status word, not trapped:
+ *       MOE_ERR_TIMEOUT      a bounded wait inside a kernel ran out (the kernel then stops)
+ *       MOE_ERR_BOUNDS       a row index computed from device data fell outside its buffer
+ *                            (the access is skipped)
+ *     moe_read_device_error() reads and clears that word.
+ *   - Inputs must be finite; results for NaN or Inf inputs are unspecified.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = -1,
+  MOE_ERR_UNSUPPORTED = -2,
+  MOE_ERR_CUDA = -3,
+  MOE_ERR_WORKSPACE = -4,
+  MOE_ERR_TIMEOUT = -5,
+  MOE_ERR_BOUNDS = -6
+} moe_status;
+
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_GELU = 1 } moe_act;
+
+/* Shape of one layer invocation. */
+typedef struct {
+  int32_t T;          /* tokens in the batch, >= 0 */
+  int32_t d_model;    /* hidden size d, multiple of 64 */
+  int32_t n_experts;  /* N, 1..256 */
+  int32_t top_k;      /* k, 1..min(8, N) */
+  int32_t d_ff;       /* expert FFN width F, multiple of 64 */
+  int32_t act;        /* moe_act: SwiGLU (gate/up/down) or GELU (up/down) */
+  int32_t capacity;   /* slots per expert, >= 0; a value >= T means no limit */
+} moe_dims;
+
+/* Slots per expert: ceil(capacity_factor * T / n_experts), computed as
+ * ceil((capacity_factor * T) / n_experts) in IEEE double.
+ * capacity_factor <= 0, NaN or infinite means no limit and returns T.
+ * Source: page «Sparse Mixture-of-Experts», section «Expert capacity и capacity factor».
+ * Returns -1 if T < 0 or n_experts < 1. Host-only; touches no device. */
+int32_t moe_capacity(double capacity_factor, int32_t T, int32_t n_experts);
+
+/* Upper bound on kept rows: R_max = min(T * k, N * min(capacity, T)).
+ * Row buffers (pair_of_row, x_perm, h, y_perm) must hold R_max rows. Returns -1 on bad dims. Host-only. */
+int64_t moe_max_rows(const moe_dims* dims);
+
+/* Bytes of the per-stage workspace `ws` taken by moe_route, moe_route_from_logits,
+ * moe_permute, moe_grouped_ffn and moe_unpermute_combine. Its first 256 bytes hold the device
+ * status word. The rest is scratch for the capacity scan. Host-only. */
+moe_status moe_workspace_bytes(const moe_dims* dims, size_t* bytes);
+
+/* Clear the status word of a fresh workspace (a 4-byte async memset on `stream`). */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Route: steps 1-3 above.
+ *   x            [T, d_model] bf16            hidden states
+ *   w_router     [N, d_model] fp32            router weight (linear, no bias term)
+ *   logit_bias   [N] fp32 or NULL             optional additive per-expert logit bias
+ *   logits       [T, N] fp32 (out)            x W_r^T (+ b), fp32 accumulation
+ *   topk_idx     [T, k] int32 (out)           chosen experts, best first; equal logits go
+ *                                             to the lower expert index
+ *   topk_w       [T, k] fp32 (out)            renormalised weights, sum to 1 per token:
+ *                                             exp(L_j - L_0) / sum_i exp(L_i - L_0)
+ *   slot         [T, k] int32 (out)           slot of each pair in its expert's buffer, -1 = dropped
+ *   expert_count [N] int32 (out)              kept pairs per expert = min(picks, capacity)
+ *   ws, ws_bytes                              per-stage workspace (moe_workspace_bytes)
+ */
+moe_status moe_route(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                     const float* logit_bias, float* logits, int32_t* topk_idx, float* topk_w,
+                     int32_t* slot, int32_t* expert_count, void* ws, size_t ws_bytes, void* stream);
+
+/* Route from given logits [T, N] fp32 (steps 2-3 only). Same outputs as moe_route.
+ * Lets a caller supply crafted logits (exact ties) or re-route stored logits. */
+moe_status moe_route_from_logits(const moe_dims* dims, const float* logits, int32_t* topk_idx,
+                                 float* topk_w, int32_t* slot, int32_t* expert_count, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/* Permute: step 4, sort by expert id.
+ *   expert_offset [N+1] int32 (out)  exclusive prefix sum of expert_count; expert e owns rows
+ *                                    [expert_offset[e], expert_offset[e+1]); R = expert_offset[N]
+ *   row_of_pair   [T, k] int32 (out) row of pair (t, j) = expert_offset[e] + slot, -1 if dropped
+ *   pair_of_row   [R_max] int32 (out) t * k + j for rows < R; rows >= R are not written
+ *   x_perm        [R_max, d_model] bf16 (out) x_perm[row_of_pair[t, j]] = x[t]; rows >= R not written
+ */
+moe_status moe_permute(const moe_dims* dims, const uint16_t* x, const int32_t* topk_idx,
+                       const int32_t* slot, const int32_t* expert_count, int32_t* expert_offset,
+                       int32_t* row_of_pair, int32_t* pair_of_row, uint16_t* x_perm, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Grouped expert FFN over the expert-contiguous rows (step 4), on tcgen05 tensor cores.
+ *   w_gate_up  SwiGLU: [N, 2F, d_model] bf16, rows 0..F-1 of expert e are the gate projection
+ *              and rows F..2F-1 the up projection (the packed gate_up_proj layout);
+ *              GELU:   [N, F, d_model] bf16
+ *   w_down     [N, d_model, F] bf16 (the packed down_proj layout)
+ *   h          [R_max, F] bf16 (out)   act(x_perm W_gu^T) in fp32, rounded once to bf16
+ *   y_perm     [R_max, d_model] fp32 (out)  h W_d^T with fp32 accumulation
+ * Rows >= R of h and y_perm are not written. Experts with no kept rows cost nothing. */
+moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
+                           const int32_t* expert_offset, const uint16_t* w_gate_up,
+                           const uint16_t* w_down, uint16_t* h, float* y_perm, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* Combine: step 5, back to token order.
+ *   out[t] = residual[t] + sum over kept j (ascending) of topk_w[t, j] * y_perm[row_of_pair[t, j]]
+ * summed in fp32 and rounded once. A token with no kept pair gets residual[t]'s bits
+ * unchanged (zeros if residual is NULL). out_f32 = 0: out is [T, d_model] bf16;
+ * out_f32 = 1: out is [T, d_model] fp32. `out` may alias `residual` (same dtype).
+ * ws may be NULL; if given, bounds faults are recorded in its status word. */
+moe_status moe_unpermute_combine(const moe_dims* dims, const float* y_perm,
+                                 const int32_t* row_of_pair, const float* topk_w,
+                                 const uint16_t* residual, void* out, int32_t out_f32, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/* Pointers into a moe_forward workspace (all device pointers; sizes as in the calls above). */
+typedef struct {
+  float* logits;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* slot;
+  int32_t* expert_count;
+  int32_t* expert_offset;
+  int32_t* row_of_pair;
+  int32_t* pair_of_row;
+  uint16_t* x_perm;
+  uint16_t* h;
+  float* y_perm;
+  void* stage_ws;
+  size_t stage_ws_bytes;
+} moe_forward_buffers;
+
+/* Bytes of workspace moe_forward needs: every intermediate plus the per-stage workspace. */
+moe_status moe_forward_workspace_bytes(const moe_dims* dims, size_t* bytes);
+
+/* Carve a moe_forward workspace into its intermediates (host arithmetic only). */
+moe_status moe_forward_layout(const moe_dims* dims, void* ws, size_t ws_bytes,
+                              moe_forward_buffers* bufs);
+
+/* The whole layer on one stream: route, permute, grouped FFN, combine.
+ *   out [T, d_model] bf16 (out). `residual` may be NULL (out = MoE part only) and may alias x;
+ *   out may alias residual. Intermediates stay in `ws` (see moe_forward_layout). */
+moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                       const float* logit_bias, const uint16_t* w_gate_up, const uint16_t* w_down,
+                       const uint16_t* residual, uint16_t* out, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Synchronise `stream`, read the status word of a per-stage workspace into *err and clear it.
+ * (For a moe_forward workspace pass moe_forward_buffers.stage_ws.) */
+moe_status moe_read_device_error(void* ws, void* stream, moe_status* err);
+
+/* Static description of a status code. */
+const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

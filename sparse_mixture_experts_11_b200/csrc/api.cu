@@ -1,0 +1,341 @@
+// C ABI of the MoE layer forward pass: host-side validation, workspace layout and the
+// launch sequence of each stage. The meaning of every call is documented in include/moe.h.
+#include <math.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+
+#include "launch.h"
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+constexpr int kMaxDevices = 64;
+DeviceInfo g_info[kMaxDevices];
+std::once_flag g_info_once[kMaxDevices];
+cudaError_t g_info_err[kMaxDevices];
+
+
+}  // namespace
+
+cudaError_t device_info(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_info_once[dev], [dev] {
+    DeviceInfo di{};
+    cudaError_t e = cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&di.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&di.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    g_info[dev] = di;
+    g_info_err[dev] = e;
+  });
+  *out = g_info[dev];
+  return g_info_err[dev];
+}
+
+}  // namespace moe
+
+using moe::DeviceInfo;
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+moe_status check_dims(const moe_dims* d) {
+  if (d == nullptr) return MOE_ERR_INVALID;
+  if (d->T < 0 || d->d_model <= 0 || d->n_experts <= 0 || d->top_k <= 0 || d->d_ff <= 0 ||
+      d->capacity < 0)
+    return MOE_ERR_INVALID;
+  if (d->top_k > d->n_experts) return MOE_ERR_INVALID;
+  if (d->act != MOE_ACT_SWIGLU && d->act != MOE_ACT_GELU) return MOE_ERR_INVALID;
+  if (d->n_experts > 256 || d->top_k > 8) return MOE_ERR_UNSUPPORTED;
+  if (d->d_model % 64 != 0 || d->d_ff % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->T) * d->top_k > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_device() {
+  DeviceInfo di;
+  if (moe::device_info(&di) != cudaSuccess) return MOE_ERR_CUDA;
+  if (di.cc_major != 10 || di.cc_minor != 0) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+int64_t max_rows(const moe_dims* d) {
+  const int64_t cap = std::min<int64_t>(d->capacity, d->T);
+  return std::min<int64_t>(static_cast<int64_t>(d->T) * d->top_k,
+                           static_cast<int64_t>(d->n_experts) * cap);
+}
+
+size_t stage_ws_bytes(const moe_dims* d) {
+  const int64_t chunks = moe::slot_chunks(static_cast<int64_t>(d->T) * d->top_k);
+  size_t b = moe::kStatusBytes;
+  if (chunks > 1) b += static_cast<size_t>(chunks) * d->n_experts * sizeof(int32_t);
+  return round_up(b, 256);
+}
+
+int* status_of(void* ws) { return static_cast<int*>(ws); }
+
+moe_status launch_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Shared by moe_route and moe_route_from_logits once top-k is written.
+moe_status route_slots(const moe_dims* d, int32_t* topk_idx, int32_t* slot, int32_t* expert_count,
+                       void* ws, cudaStream_t s) {
+  int32_t* scratch = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + moe::kStatusBytes);
+  const int cap = std::min(d->capacity, d->T);
+  return launch_status(moe::launch_capacity_slots(topk_idx, slot, expert_count, scratch, d->T,
+                                                  d->n_experts, d->top_k, cap, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_capacity(double capacity_factor, int32_t T, int32_t n_experts) {
+  if (T < 0 || n_experts < 1) return -1;
+  if (!(capacity_factor > 0.0) || isinf(capacity_factor)) return T;  // <= 0, NaN, inf: no limit
+  const double c = ceil((capacity_factor * static_cast<double>(T)) / static_cast<double>(n_experts));
+  return c >= static_cast<double>(INT32_MAX) ? INT32_MAX : static_cast<int32_t>(c);
+}
+
+int64_t moe_max_rows(const moe_dims* dims) {
+  if (check_dims(dims) != MOE_OK) return -1;
+  return max_rows(dims);
+}
+
+moe_status moe_workspace_bytes(const moe_dims* dims, size_t* bytes) {
+  const moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (bytes == nullptr) return MOE_ERR_INVALID;
+  *bytes = stage_ws_bytes(dims);
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < moe::kStatusBytes) return MOE_ERR_INVALID;
+  return launch_status(cudaMemsetAsync(ws, 0, sizeof(int32_t), as_stream(stream)));
+}
+
+moe_status moe_route(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                     const float* logit_bias, float* logits, int32_t* topk_idx, float* topk_w,
+                     int32_t* slot, int32_t* expert_count, void* ws, size_t ws_bytes,
+                     void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (dims->T == 0) return MOE_OK;
+  if (!x || !w_router || !logits || !topk_idx || !topk_w || !slot || !expert_count || !ws)
+    return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(logits) || !aligned16(topk_idx) ||
+      !aligned16(topk_w) || !aligned16(slot) || !aligned16(expert_count) || !aligned16(ws) ||
+      (logit_bias && !aligned16(logit_bias)))
+    return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < stage_ws_bytes(dims)) return MOE_ERR_WORKSPACE;
+  if ((st = check_device()) != MOE_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  st = launch_status(moe::launch_router_topk(x, w_router, logit_bias, logits, topk_idx, topk_w,
+                                             dims->T, dims->d_model, dims->n_experts,
+                                             dims->top_k, s));
+  if (st != MOE_OK) return st;
+  return route_slots(dims, topk_idx, slot, expert_count, ws, s);
+}
+
+moe_status moe_route_from_logits(const moe_dims* dims, const float* logits, int32_t* topk_idx,
+                                 float* topk_w, int32_t* slot, int32_t* expert_count, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (dims->T == 0) return MOE_OK;
+  if (!logits || !topk_idx || !topk_w || !slot || !expert_count || !ws) return MOE_ERR_INVALID;
+  if (!aligned16(logits) || !aligned16(topk_idx) || !aligned16(topk_w) || !aligned16(slot) ||
+      !aligned16(expert_count) || !aligned16(ws))
+    return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < stage_ws_bytes(dims)) return MOE_ERR_WORKSPACE;
+  if ((st = check_device()) != MOE_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  st = launch_status(moe::launch_topk_from_logits(logits, topk_idx, topk_w, dims->T,
+                                                  dims->n_experts, dims->top_k, s));
+  if (st != MOE_OK) return st;
+  return route_slots(dims, topk_idx, slot, expert_count, ws, s);
+}
+
+moe_status moe_permute(const moe_dims* dims, const uint16_t* x, const int32_t* topk_idx,
+                       const int32_t* slot, const int32_t* expert_count, int32_t* expert_offset,
+                       int32_t* row_of_pair, int32_t* pair_of_row, uint16_t* x_perm, void* ws,
+                       size_t ws_bytes, void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (dims->T == 0) return MOE_OK;
+  const int64_t rmax = max_rows(dims);
+  if (!x || !topk_idx || !slot || !expert_count || !expert_offset || !row_of_pair || !ws ||
+      (rmax > 0 && (!pair_of_row || !x_perm)))
+    return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(topk_idx) || !aligned16(slot) || !aligned16(expert_count) ||
+      !aligned16(expert_offset) || !aligned16(row_of_pair) || !aligned16(ws) ||
+      (pair_of_row && !aligned16(pair_of_row)) || (x_perm && !aligned16(x_perm)))
+    return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < moe::kStatusBytes) return MOE_ERR_WORKSPACE;
+  if ((st = check_device()) != MOE_OK) return st;
+  return launch_status(moe::launch_permute(x, topk_idx, slot, expert_count, expert_offset,
+                                           row_of_pair, pair_of_row, x_perm, dims->T,
+                                           dims->d_model, dims->n_experts, dims->top_k, rmax,
+                                           status_of(ws), as_stream(stream)));
+}
+
+moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
+                           const int32_t* expert_offset, const uint16_t* w_gate_up,
+                           const uint16_t* w_down, uint16_t* h, float* y_perm, void* ws,
+                           size_t ws_bytes, void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  const int64_t rmax = max_rows(dims);
+  if (dims->T == 0 || rmax == 0) return MOE_OK;
+  if (!x_perm || !expert_offset || !w_gate_up || !w_down || !h || !y_perm || !ws)
+    return MOE_ERR_INVALID;
+  if (!aligned16(x_perm) || !aligned16(expert_offset) || !aligned16(w_gate_up) ||
+      !aligned16(w_down) || !aligned16(h) || !aligned16(y_perm) || !aligned16(ws))
+    return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < moe::kStatusBytes) return MOE_ERR_WORKSPACE;
+  if ((st = check_device()) != MOE_OK) return st;
+  moe::GroupedFfnArgs a{};
+  a.x_perm = x_perm;
+  a.expert_offset = expert_offset;
+  a.w_gate_up = w_gate_up;
+  a.w_down = w_down;
+  a.h = h;
+  a.y_perm = y_perm;
+  a.N = dims->n_experts;
+  a.d = dims->d_model;
+  a.F = dims->d_ff;
+  a.act = dims->act;
+  a.r_max = rmax;
+  a.status = status_of(ws);
+  a.timeout_ns = moe::kDefaultWaitTimeoutNs;
+  return launch_status(moe::launch_grouped_ffn(a, as_stream(stream)));
+}
+
+moe_status moe_unpermute_combine(const moe_dims* dims, const float* y_perm,
+                                 const int32_t* row_of_pair, const float* topk_w,
+                                 const uint16_t* residual, void* out, int32_t out_f32, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (dims->T == 0) return MOE_OK;
+  const int64_t rmax = max_rows(dims);
+  if (!row_of_pair || !topk_w || !out || (rmax > 0 && !y_perm)) return MOE_ERR_INVALID;
+  if (out_f32 != 0 && out_f32 != 1) return MOE_ERR_INVALID;
+  if ((y_perm && !aligned16(y_perm)) || !aligned16(row_of_pair) || !aligned16(topk_w) ||
+      !aligned16(out) || (residual && !aligned16(residual)) || (ws && !aligned16(ws)))
+    return MOE_ERR_UNSUPPORTED;
+  if (ws && ws_bytes < moe::kStatusBytes) return MOE_ERR_WORKSPACE;
+  if ((st = check_device()) != MOE_OK) return st;
+  return launch_status(moe::launch_combine(y_perm, row_of_pair, topk_w, residual, out, out_f32,
+                                           dims->T, dims->d_model, dims->top_k, rmax,
+                                           ws ? status_of(ws) : nullptr, as_stream(stream)));
+}
+
+moe_status moe_forward_workspace_bytes(const moe_dims* dims, size_t* bytes) {
+  const moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (bytes == nullptr) return MOE_ERR_INVALID;
+  // lay the buffers out from address 0 to measure the total
+  size_t off = 0;
+  const int64_t T = dims->T, N = dims->n_experts, k = dims->top_k, d = dims->d_model,
+                F = dims->d_ff, R = max_rows(dims);
+  const size_t sizes[] = {size_t(T * N * 4), size_t(T * k * 4), size_t(T * k * 4), size_t(T * k * 4),
+                          size_t(N * 4),     size_t((N + 1) * 4), size_t(T * k * 4), size_t(R * 4),
+                          size_t(R * d * 2), size_t(R * F * 2),  size_t(R * d * 4),
+                          stage_ws_bytes(dims)};
+  for (size_t s : sizes) off += round_up(s, 256);
+  *bytes = off;
+  return MOE_OK;
+}
+
+moe_status moe_forward_layout(const moe_dims* dims, void* ws, size_t ws_bytes,
+                              moe_forward_buffers* bufs) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (ws == nullptr || bufs == nullptr) return MOE_ERR_INVALID;
+  if (!aligned16(ws)) return MOE_ERR_UNSUPPORTED;
+  size_t need = 0;
+  moe_forward_workspace_bytes(dims, &need);
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE;
+  const int64_t T = dims->T, N = dims->n_experts, k = dims->top_k, d = dims->d_model,
+                F = dims->d_ff, R = max_rows(dims);
+  char* p = static_cast<char*>(ws);
+  auto take = [&p](size_t bytes) {
+    char* q = p;
+    p += round_up(bytes, 256);
+    return q;
+  };
+  bufs->logits = reinterpret_cast<float*>(take(T * N * 4));
+  bufs->topk_idx = reinterpret_cast<int32_t*>(take(T * k * 4));
+  bufs->topk_w = reinterpret_cast<float*>(take(T * k * 4));
+  bufs->slot = reinterpret_cast<int32_t*>(take(T * k * 4));
+  bufs->expert_count = reinterpret_cast<int32_t*>(take(N * 4));
+  bufs->expert_offset = reinterpret_cast<int32_t*>(take((N + 1) * 4));
+  bufs->row_of_pair = reinterpret_cast<int32_t*>(take(T * k * 4));
+  bufs->pair_of_row = reinterpret_cast<int32_t*>(take(R * 4));
+  bufs->x_perm = reinterpret_cast<uint16_t*>(take(R * d * 2));
+  bufs->h = reinterpret_cast<uint16_t*>(take(R * F * 2));
+  bufs->y_perm = reinterpret_cast<float*>(take(R * d * 4));
+  bufs->stage_ws_bytes = stage_ws_bytes(dims);
+  bufs->stage_ws = take(bufs->stage_ws_bytes);
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                       const float* logit_bias, const uint16_t* w_gate_up, const uint16_t* w_down,
+                       const uint16_t* residual, uint16_t* out, void* ws, size_t ws_bytes,
+                       void* stream) {
+  moe_forward_buffers b;
+  moe_status st = moe_forward_layout(dims, ws, ws_bytes, &b);
+  if (st != MOE_OK) return st;
+  if (dims->T == 0) return MOE_OK;
+  if (!x || !w_router || !w_gate_up || !w_down || !out) return MOE_ERR_INVALID;
+  st = moe_route(dims, x, w_router, logit_bias, b.logits, b.topk_idx, b.topk_w, b.slot,
+                 b.expert_count, b.stage_ws, b.stage_ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  st = moe_permute(dims, x, b.topk_idx, b.slot, b.expert_count, b.expert_offset, b.row_of_pair,
+                   b.pair_of_row, b.x_perm, b.stage_ws, b.stage_ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  st = moe_grouped_ffn(dims, b.x_perm, b.expert_offset, w_gate_up, w_down, b.h, b.y_perm,
+                       b.stage_ws, b.stage_ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  return moe_unpermute_combine(dims, b.y_perm, b.row_of_pair, b.topk_w, residual, out, 0,
+                               b.stage_ws, b.stage_ws_bytes, stream);
+}
+
+moe_status moe_read_device_error(void* ws, void* stream, moe_status* err) {
+  if (ws == nullptr || err == nullptr) return MOE_ERR_INVALID;
+  const cudaStream_t s = as_stream(stream);
+  int v = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  *err = static_cast<moe_status>(v);
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape, alignment or device";
+    case MOE_ERR_CUDA: return "CUDA launch error";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_BOUNDS: return "device index out of bounds";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

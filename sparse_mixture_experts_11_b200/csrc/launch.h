@@ -1,0 +1,61 @@
+// Host-side launchers of the MoE kernels (internal to the library; the C ABI is in moe.h).
+// Each launcher only enqueues work on `stream` and returns the launch error, if any.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Per-stage workspace layout: [0, 256) status word (+ padding); [256, ...) capacity-scan scratch.
+constexpr size_t kStatusBytes = 256;
+constexpr int kSlotChunk = 4096;  // (token, choice) pairs ranked per block in the slot pass
+constexpr uint64_t kDefaultWaitTimeoutNs = 2000000000ull;  // limit of one mbarrier wait (2 s)
+
+inline int64_t slot_chunks(int64_t pairs) { return (pairs + kSlotChunk - 1) / kSlotChunk; }
+
+struct DeviceInfo {
+  int sm_count;
+  int cc_major;
+  int cc_minor;
+};
+cudaError_t device_info(DeviceInfo* out);
+
+// router: logits = x W_r^T (+ b), then top-k and renormalised weights
+cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const float* bias,
+                               float* logits, int32_t* topk_idx, float* topk_w, int T, int d,
+                               int N, int k, cudaStream_t s);
+// top-k and renormalised weights from given logits
+cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, float* topk_w, int T,
+                                    int N, int k, cudaStream_t s);
+// capacity slots in (choice, token) arrival order
+cudaError_t launch_capacity_slots(const int32_t* topk_idx, int32_t* slot, int32_t* expert_count,
+                                  int32_t* chunk_scratch, int T, int N, int k, int capacity,
+                                  cudaStream_t s);
+// sort kept pairs into expert-contiguous rows
+cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, const int32_t* slot,
+                           const int32_t* expert_count, int32_t* expert_offset,
+                           int32_t* row_of_pair, int32_t* pair_of_row, uint16_t* x_perm, int T,
+                           int d, int N, int k, int64_t r_max, int* status, cudaStream_t s);
+// weighted sum back in token order
+cudaError_t launch_combine(const float* y_perm, const int32_t* row_of_pair, const float* topk_w,
+                           const uint16_t* residual, void* out, int out_f32, int T, int d, int k,
+                           int64_t r_max, int* status, cudaStream_t s);
+
+// grouped expert GEMMs on tcgen05
+struct GroupedFfnArgs {
+  const uint16_t* x_perm;
+  const int32_t* expert_offset;
+  const uint16_t* w_gate_up;
+  const uint16_t* w_down;
+  uint16_t* h;
+  float* y_perm;
+  int N, d, F, act;
+  int64_t r_max;
+  int* status;
+  uint64_t timeout_ns;
+};
+cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,352 @@
+// Routing kernels: router logits, top-k with renormalised weights, capacity slots.
+//
+// Page «Sparse Mixture-of-Experts» (bigdataschool wiki):
+//   «Роутер и top-k gating»: logits from a linear layer without bias term, softmax over the
+//     experts, the k most probable experts per token, their probabilities renormalised to one;
+//   «Expert capacity и capacity factor»: ceil(capacity_factor * T / N) slots per expert, and a
+//     pair that arrives at a full expert is dropped (first come, first served in batch order).
+//
+// Selection is made on the fp32 logits (softmax is strictly increasing, so the chosen experts
+// are the same); equal logits go to the lower expert index. The renormalised weight of choice j
+// is exp(L_j - L_0) / sum_i exp(L_i - L_0) over the chosen logits, which equals p_j / sum p_i.
+// Arrival order for the capacity is (choice, token): all first choices in token order, then
+// all second choices, and so on.
+#include <math.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ bool better(float av, int ae, float bv, int be) {
+  return av > bv || (av == bv && ae < be);
+}
+
+// Best (value, expert) over the warp; every lane ends with the same pair.
+__device__ __forceinline__ void warp_best(float& v, int& e) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(kFull, v, o);
+    const int oe = __shfl_xor_sync(kFull, e, o);
+    if (better(ov, oe, v, e)) {
+      v = ov;
+      e = oe;
+    }
+  }
+}
+
+// Top-k of one token whose N logits are spread over the warp: lane l holds experts l + 32 j.
+// Lanes r < k write choice r. NaN logits are never preferred (unspecified input, but never
+// an out-of-range expert index).
+template <int EPT>
+__device__ __forceinline__ void warp_topk_write(const float (&val)[EPT], int N, int k, int t,
+                                                int32_t* topk_idx, float* topk_w) {
+  const int lane = static_cast<int>(lane_id());
+  uint32_t taken = 0;
+  float sel_v[8];
+  int sel_e[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    sel_v[r] = 0.f;
+    sel_e[r] = 0;
+    if (r < k) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < EPT; ++j) {
+        const int e = lane + 32 * j;
+        const float v = isnan(val[j]) ? -INFINITY : val[j];
+        if (e < N && !((taken >> j) & 1u) && better(v, e, bv, be)) {
+          bv = v;
+          be = e;
+        }
+      }
+      warp_best(bv, be);
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      sel_v[r] = bv;
+      sel_e[r] = be;
+    }
+  }
+  // renormalised weights: softmax over the chosen logits (the largest is sel_v[0])
+  float den = 0.f;
+  float num[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    num[r] = (r < k) ? expf(sel_v[r] - sel_v[0]) : 0.f;
+    den += num[r];
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (r < k && lane == r) {
+      topk_idx[static_cast<int64_t>(t) * k + r] = sel_e[r];
+      topk_w[static_cast<int64_t>(t) * k + r] = num[r] / den;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ router (SIMT fp32)
+constexpr int kRtTok = 32;      // tokens per block
+constexpr int kRtChunk = 32;    // d elements per shared-memory stage
+constexpr int kRtThreads = 256; // 8 warps; warp w owns tokens 4w..4w+3 of the block
+
+// logits[t, e] = sum_i x[t, i] * W_r[e, i] (+ b[e]) in fp32, summed in order of i;
+// then top-k and weights for each token of the block.
+template <int EPT>
+__global__ void __launch_bounds__(kRtThreads) router_topk_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias,
+    float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int T,
+    int d, int N, int k) {
+  __shared__ float xs[kRtTok][kRtChunk + 1];
+  __shared__ float ws[EPT * 32][kRtChunk + 1];
+  const int tid = threadIdx.x;
+  const int ty = tid >> 5, tx = tid & 31;
+  const int t0 = blockIdx.x * kRtTok;
+
+  for (int i = tid; i < EPT * 32 * (kRtChunk + 1); i += kRtThreads) (&ws[0][0])[i] = 0.f;
+
+  float acc[4][EPT];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) acc[i][j] = 0.f;
+
+  for (int c0 = 0; c0 < d; c0 += kRtChunk) {
+    __syncthreads();
+    {  // 32 tokens x 32 bf16: 4 elements per thread
+      const int tok = tid >> 3, c = (tid & 7) * 4;
+      float f[4] = {0.f, 0.f, 0.f, 0.f};
+      if (t0 + tok < T) {
+        const uint2 v = *reinterpret_cast<const uint2*>(x + static_cast<int64_t>(t0 + tok) * d + c0 + c);
+        f[0] = __uint_as_float(v.x << 16);
+        f[1] = __uint_as_float(v.x & 0xffff0000u);
+        f[2] = __uint_as_float(v.y << 16);
+        f[3] = __uint_as_float(v.y & 0xffff0000u);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) xs[tok][c + q] = f[q];
+    }
+    for (int f = tid; f < N * (kRtChunk / 4); f += kRtThreads) {
+      const int e = f / (kRtChunk / 4), c = (f % (kRtChunk / 4)) * 4;
+      const float4 v = *reinterpret_cast<const float4*>(w + static_cast<int64_t>(e) * d + c0 + c);
+      ws[e][c] = v.x;
+      ws[e][c + 1] = v.y;
+      ws[e][c + 2] = v.z;
+      ws[e][c + 3] = v.w;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < kRtChunk; ++c) {
+      float xv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[i] = xs[ty * 4 + i][c];
+#pragma unroll
+      for (int j = 0; j < EPT; ++j) {
+        const float wv = ws[tx + 32 * j][c];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(xv[i], wv, acc[i][j]);
+      }
+    }
+  }
+
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) break;  // warp-uniform
+    float val[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = tx + 32 * j;
+      val[j] = acc[i][j];
+      if (e < N) {
+        if (bias != nullptr) val[j] += bias[e];
+        logits[static_cast<int64_t>(t) * N + e] = val[j];
+      }
+    }
+    warp_topk_write<EPT>(val, N, k, t, topk_idx, topk_w);
+  }
+}
+
+template <int EPT>
+__global__ void __launch_bounds__(256) topk_from_logits_kernel(const float* __restrict__ logits,
+                                                               int32_t* __restrict__ topk_idx,
+                                                               float* __restrict__ topk_w, int T,
+                                                               int N, int k) {
+  const int warps = blockDim.x >> 5;
+  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
+    float val[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = static_cast<int>(lane_id()) + 32 * j;
+      val[j] = (e < N) ? logits[static_cast<int64_t>(t) * N + e] : -INFINITY;
+    }
+    warp_topk_write<EPT>(val, N, k, t, topk_idx, topk_w);
+  }
+}
+
+// ------------------------------------------------------------------ capacity slots
+// Pair p = j * T + t (choice-major) is the p-th arrival. Its slot is the number of earlier
+// arrivals with the same expert; it is kept iff that number is below the capacity.
+//
+// Pass 1 (one block per chunk of kSlotChunk arrivals): warp w ranks its 512 consecutive
+// arrivals 32 at a time with __match_any_sync, keeping per-warp running counts per expert in
+// shared memory; then the block turns the per-warp counts into exclusive offsets and either
+//   - (one chunk) writes final slots and kept counts directly, or
+//   - (several chunks) writes chunk-local ranks into `slot` and chunk totals into scratch.
+// Pass 2 (one block): per expert, exclusive scan of the chunk totals; kept counts.
+// Pass 3: slot = chunk-local rank + chunk base, or -1 when it reaches the capacity.
+constexpr int kSlThreads = 256;
+constexpr int kSlWarps = kSlThreads / 32;
+constexpr int kSlIters = kSlotChunk / kSlThreads;  // arrivals per lane
+
+__global__ void __launch_bounds__(kSlThreads) slot_rank_kernel(
+    const int32_t* __restrict__ topk_idx, int32_t* __restrict__ slot,
+    int32_t* __restrict__ chunk_hist, int32_t* __restrict__ expert_count, int T, int N, int k,
+    int cap, int single_chunk) {
+  __shared__ int s_cnt[kSlWarps][256];
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int64_t P = static_cast<int64_t>(T) * k;
+  for (int i = tid; i < kSlWarps * 256; i += kSlThreads) (&s_cnt[0][0])[i] = 0;
+  __syncthreads();
+
+  const int64_t p_base =
+      static_cast<int64_t>(blockIdx.x) * kSlotChunk + static_cast<int64_t>(w) * (kSlotChunk / kSlWarps);
+  int local[kSlIters];
+  int ex[kSlIters];
+#pragma unroll
+  for (int it = 0; it < kSlIters; ++it) {
+    const int64_t p = p_base + it * 32 + lane;
+    int e = -1;
+    if (p < P) {
+      const int j = static_cast<int>(p / T);
+      const int t = static_cast<int>(p - static_cast<int64_t>(j) * T);
+      e = topk_idx[static_cast<int64_t>(t) * k + j];
+      if (e < 0 || e >= N) e = -2;  // invalid expert id: never kept
+    }
+    ex[it] = e;
+    const unsigned peers = __match_any_sync(kFull, e);
+    const int rank = __popc(peers & lanemask_lt());
+    const int cnt = (e >= 0) ? s_cnt[w][e] : 0;
+    __syncwarp();
+    if (e >= 0 && rank == 0) s_cnt[w][e] = cnt + __popc(peers);
+    __syncwarp();
+    local[it] = cnt + rank;
+  }
+  __syncthreads();
+  for (int e = tid; e < N; e += kSlThreads) {
+    int run = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < kSlWarps; ++w2) {
+      const int v = s_cnt[w2][e];
+      s_cnt[w2][e] = run;
+      run += v;
+    }
+    if (single_chunk)
+      expert_count[e] = min(run, cap);
+    else
+      chunk_hist[static_cast<int64_t>(blockIdx.x) * N + e] = run;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int it = 0; it < kSlIters; ++it) {
+    const int64_t p = p_base + it * 32 + lane;
+    if (p >= P) break;
+    const int j = static_cast<int>(p / T);
+    const int t = static_cast<int>(p - static_cast<int64_t>(j) * T);
+    const int e = ex[it];
+    int out = -1;
+    if (e >= 0) {
+      const int r = local[it] + s_cnt[w][e];
+      out = single_chunk ? (r < cap ? r : -1) : r;
+    }
+    slot[static_cast<int64_t>(t) * k + j] = out;
+  }
+}
+
+__global__ void __launch_bounds__(256) slot_scan_kernel(int32_t* __restrict__ chunk_hist,
+                                                        int32_t* __restrict__ expert_count,
+                                                        int n_chunks, int N, int cap) {
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < n_chunks; ++c) {
+      const int v = chunk_hist[static_cast<int64_t>(c) * N + e];
+      chunk_hist[static_cast<int64_t>(c) * N + e] = run;
+      run += v;
+    }
+    expert_count[e] = min(run, cap);
+  }
+}
+
+__global__ void __launch_bounds__(256) slot_finalize_kernel(const int32_t* __restrict__ topk_idx,
+                                                            int32_t* __restrict__ slot,
+                                                            const int32_t* __restrict__ chunk_hist,
+                                                            int T, int N, int k, int cap) {
+  const int64_t P = static_cast<int64_t>(T) * k;
+  for (int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; p < P;
+       p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int j = static_cast<int>(p / T);
+    const int t = static_cast<int>(p - static_cast<int64_t>(j) * T);
+    const int64_t q = static_cast<int64_t>(t) * k + j;
+    const int e = topk_idx[q];
+    const int local = slot[q];
+    if (e < 0 || e >= N || local < 0) {
+      slot[q] = -1;
+      continue;
+    }
+    const int r = local + chunk_hist[(p / kSlotChunk) * N + e];
+    slot[q] = r < cap ? r : -1;
+  }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers
+cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const float* bias,
+                               float* logits, int32_t* topk_idx, float* topk_w, int T, int d,
+                               int N, int k, cudaStream_t s) {
+  const dim3 grid((T + kRtTok - 1) / kRtTok);
+  if (N <= 32)
+    router_topk_kernel<1><<<grid, kRtThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+  else if (N <= 64)
+    router_topk_kernel<2><<<grid, kRtThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+  else if (N <= 128)
+    router_topk_kernel<4><<<grid, kRtThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+  else
+    router_topk_kernel<8><<<grid, kRtThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, float* topk_w, int T,
+                                    int N, int k, cudaStream_t s) {
+  const int blocks = (T + 7) / 8;
+  if (N <= 32)
+    topk_from_logits_kernel<1><<<blocks, 256, 0, s>>>(logits, topk_idx, topk_w, T, N, k);
+  else if (N <= 64)
+    topk_from_logits_kernel<2><<<blocks, 256, 0, s>>>(logits, topk_idx, topk_w, T, N, k);
+  else if (N <= 128)
+    topk_from_logits_kernel<4><<<blocks, 256, 0, s>>>(logits, topk_idx, topk_w, T, N, k);
+  else
+    topk_from_logits_kernel<8><<<blocks, 256, 0, s>>>(logits, topk_idx, topk_w, T, N, k);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_capacity_slots(const int32_t* topk_idx, int32_t* slot, int32_t* expert_count,
+                                  int32_t* chunk_scratch, int T, int N, int k, int capacity,
+                                  cudaStream_t s) {
+  const int64_t P = static_cast<int64_t>(T) * k;
+  const int n_chunks = static_cast<int>(slot_chunks(P));
+  const int single = n_chunks == 1 ? 1 : 0;
+  slot_rank_kernel<<<n_chunks, kSlThreads, 0, s>>>(topk_idx, slot, chunk_scratch, expert_count, T,
+                                                   N, k, capacity, single);
+  if (single) return cudaGetLastError();
+  slot_scan_kernel<<<1, 256, 0, s>>>(chunk_scratch, expert_count, n_chunks, N, capacity);
+  const int blocks = static_cast<int>(std::min<int64_t>((P + 255) / 256, 148 * 8));
+  slot_finalize_kernel<<<blocks, 256, 0, s>>>(topk_idx, slot, chunk_scratch, T, N, k, capacity);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,43 @@
+"""The benchmark's counting model (CPU): parameter counts pinned to the pages' printed numbers,
+and the launch count and byte counts for the workloads."""
+import json
+import os
+
+import bench
+import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def test_active_params_reproduce_page_numbers():
+    g = json.load(open(os.path.join(GOLDEN, "active_params_demo.json")))
+    d, h, N = g["d_model"], g["hidden"], g["experts"]
+    # the demo expert is fc1 (d->h) and fc2 (h->d), each with bias: the GELU-shaped two-matrix FFN
+    assert bench.active_params(d, h, N, 1, "gelu", bias=True) == g["top1_active"]
+    assert bench.active_params(d, h, N, 2, "gelu", bias=True) == g["top2_active"]
+    assert N * bench.expert_params(d, h, "gelu", bias=True) + d * N == g["total"]
+
+
+def test_bandwidth_estimate_of_page():
+    # 800 GB/s over 3.6 B active params at 2 bytes each is about 111 tokens/s
+    assert round(800e9 / (3.6e9 * 2)) == 111
+
+
+def test_bytes_model_switch():
+    s = synthetic.SHAPES["switch_top1"]
+    b = bench.algorithmic_bytes(s, 4096, 64, 4096)
+    assert b["weights"] == 64 * 2 * 1024 * 4096 * 2
+    assert b["ffn"] == b["weights"] + 4096 * 1024 * 6
+
+
+def test_launch_counts():
+    assert bench.launches_per_step(4096, 1, 4096) == 6
+    assert bench.launches_per_step(16384, 8, 20480) == 8
+    assert bench.launches_per_step(5, 2, 0) == 4
+
+
+def test_workload_parsing():
+    s, T = bench.parse_workload("mixtral:512")
+    assert s.d_model == 4096 and T == 512
+    s, T = bench.parse_workload("switch_top1")
+    assert T == 4096

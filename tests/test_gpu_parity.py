@@ -1,0 +1,139 @@
+"""Parity of the CUDA path with the CPU oracle on small and ragged shapes (GPU)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from tests import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+# (name, T, d, N, k, F, act, capacity_factor, zipf)
+SMALL_CASES = [
+    ("tiny_top2_cfg", 64, 128, 8, 2, 256, "swiglu", 1.25, None),
+    ("ragged_multi_mtile", 600, 192, 4, 2, 320, "swiglu", None, None),
+    ("gelu_switch_small", 512, 256, 16, 1, 512, "gelu", 1.0, None),
+    ("gelu_ragged_n", 300, 320, 5, 3, 192, "gelu", 1.25, None),
+    ("many_experts_k8", 96, 128, 256, 8, 128, "swiglu", 1.25, 1.1),
+    ("gpt_oss_dims_small_T", 64, 2880, 32, 4, 2880, "swiglu", None, None),
+    ("single_token", 1, 256, 8, 2, 256, "swiglu", None, None),
+    ("k_equals_n", 40, 64, 4, 4, 64, "swiglu", None, None),
+    ("heavy_drop", 200, 128, 8, 2, 128, "swiglu", 0.25, 1.1),
+]
+
+
+def _inputs(T, d, N, F, act, zipf, seed=0):
+    inp = synthetic.make_custom_inputs(T, d, N, F, act, seed=seed, device="cuda", zipf_s=zipf)
+    return inp
+
+
+@pytest.mark.parametrize("case", SMALL_CASES, ids=lambda c: c[0])
+def test_stage_parity(case):
+    name, T, d, N, k, F, act, cf, zipf = case
+    inp = _inputs(T, d, N, F, act, zipf)
+    cap = oracle.capacity_from_factor(cf, T, N)
+    run = H.StageRun(inp, k, act, cap).run()
+    H.check_logits(H.f64(run.logits), H.f64(inp["x"]), H.f64(inp["w_router"]),
+                   None if inp["logit_bias"] is None else H.f64(inp["logit_bias"]))
+    routing, off, rop = H.check_routing(run, cap)
+    H.check_x_perm(run, rop)
+    R = int(off[-1])
+    if R:
+        H.check_expert_rows(run, routing, act, np.unique(np.linspace(0, R - 1, min(R, 24)).astype(np.int64)))
+    H.check_outputs(run, routing, act)
+    H.check_dropped_tokens_pass_through(run, routing["slot"])
+
+
+def test_no_residual_and_zero_capacity():
+    T, d, N, k, F = 48, 128, 8, 2, 128
+    inp = _inputs(T, d, N, F, "swiglu", None, seed=3)
+    run = H.StageRun(inp, k, "swiglu", 0).run(residual=True)
+    routing, off, _ = H.check_routing(run, 0)
+    assert int(off[-1]) == 0
+    assert torch.equal(run.out.view(torch.int16), inp["x"].view(torch.int16))
+    run = H.StageRun(inp, k, "swiglu", T).run(residual=False)
+    routing, _, _ = H.check_routing(run, T)
+    H.check_outputs(run, routing, "swiglu", residual=False)
+
+
+def _route_logits(L, k, cap):
+    import sparse_mixture_experts_11_b200 as moe
+    T, N = L.shape
+    dims = moe.make_dims(T, 64, N, k, 64, "swiglu", cap)
+    ws = moe.new_workspace(dims)
+    lg = torch.from_numpy(L).cuda()
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    slot = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((N,), dtype=torch.int32, device="cuda")
+    moe.route_from_logits(dims, lg, idx, w, slot, cnt, ws)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), w.cpu().numpy(), slot.cpu().numpy(), cnt.cpu().numpy()
+
+
+def test_route_from_logits_hand_case():
+    """The hand-worked case (a tie, drops at capacity 1) straight against its written values."""
+    import json, os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_case_top2_cap1.json")))
+    idx, w, slot, cnt = _route_logits(np.array(g["logits"], np.float32), g["top_k"], g["capacity"])
+    assert idx.tolist() == g["topk_idx"]
+    assert slot.tolist() == g["slot"]
+    assert cnt.tolist() == g["expert_count"]
+    np.testing.assert_allclose(w, np.array(g["topk_w"]), atol=H.WEIGHT_ATOL, rtol=0)
+
+
+@pytest.mark.parametrize("T,N,k", [(50, 8, 2), (33, 64, 4), (70, 256, 8), (9000, 16, 3), (20000, 8, 8)])
+def test_route_from_logits_ties(T, N, k):
+    """Crafted logits with many exact ties; several capacity-scan chunks for the large cases."""
+    rng = np.random.default_rng(T + N + k)
+    L = rng.integers(-3, 4, size=(T, N)).astype(np.float32) * 0.5
+    cap = int(np.ceil(1.0 * T / N))
+    idx, w, slot, cnt = _route_logits(L, k, cap)
+    r = oracle.route_from_logits(L.astype(np.float64), k, cap)
+    assert np.array_equal(idx, r["topk_idx"])
+    assert np.array_equal(slot, r["slot"])
+    assert np.array_equal(cnt, r["expert_count"])
+    np.testing.assert_allclose(w, r["topk_w"], atol=H.WEIGHT_ATOL, rtol=0)
+
+
+def test_forward_matches_stages_bitwise():
+    """moe_forward (one call) and the four stage calls produce identical bits."""
+    import sparse_mixture_experts_11_b200 as moe
+    T, d, N, k, F = 300, 192, 8, 2, 320
+    inp = _inputs(T, d, N, F, "swiglu", None, seed=5)
+    cap = oracle.capacity_from_factor(1.25, T, N)
+    run = H.StageRun(inp, k, "swiglu", cap).run()
+    dims = run.dims
+    ws = moe.new_workspace(dims, forward=True)
+    out = torch.empty_like(inp["x"])
+    for _ in range(2):
+        moe.forward_into(dims, inp["x"], inp["w_router"], None, inp["w_gate_up"], inp["w_down"],
+                         inp["x"], out, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), run.out.view(torch.int16))
+
+
+def test_repeat_runs_are_bitwise_identical():
+    T, d, N, k, F = 700, 256, 16, 2, 256
+    inp = _inputs(T, d, N, F, "swiglu", 1.1, seed=9)
+    cap = oracle.capacity_from_factor(1.0, T, N)
+    a = H.StageRun(inp, k, "swiglu", cap).run()
+    o1 = a.out.clone()
+    y1 = a.y_perm.clone()
+    a.run()
+    assert torch.equal(o1.view(torch.int16), a.out.view(torch.int16))
+    assert torch.equal(y1, a.y_perm)
+
+
+def test_empty_batch_is_a_no_op():
+    import sparse_mixture_experts_11_b200 as moe
+    dims = moe.make_dims(0, 128, 8, 2, 128, "swiglu", 0)
+    ws = moe.new_workspace(dims, forward=True)
+    x = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    wr = torch.zeros((8, 128), dtype=torch.float32, device="cuda")
+    wgu = torch.zeros((8, 256, 128), dtype=torch.bfloat16, device="cuda")
+    wd = torch.zeros((8, 128, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    moe.forward_into(dims, x, wr, None, wgu, wd, x, out, ws)
+    torch.cuda.synchronize()
