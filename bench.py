@@ -20,9 +20,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import torch
@@ -106,55 +104,75 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock, power and clock-event reasons of one GPU through NVML every ~1 ms
+    on a background thread while the timed region runs (the main thread spends that time in
+    CUDA synchronisation, which releases the GIL)."""
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
-        self.path = None
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
+
+    def __init__(self, torch_device_index: int, interval_s: float = 0.001):
+        self.interval = interval_s
+        self.samples = []
+        self.reasons = set()
+        self.err = None
+        self.nv = None
+        self.handle = None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.handle = nv.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = nv
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = f"nvml unavailable: {e}"
+
+    def _poll(self):
+        import threading  # noqa: F401
+        nv, h = self.nv, self.handle
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = get_reasons(h)
+                self.samples.append((sm, pw))
+                for name, const in self.REASONS.items():
+                    if rs & getattr(nv, const, 0):
+                        self.reasons.add(name)
+            except Exception as e:
+                self.err = str(e)
+                return
+            self._stop.wait(self.interval)
 
     def start(self):
-        try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        if self.nv is None:
+            return
+        import threading
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._poll, daemon=True)
+        self._t.start()
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, smax, reasons, power = [], [], set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    smax.append(float(parts[2]))
-                    power.append(float(parts[3]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "power_w_max": max(power) if power else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
+        self._stop.set()
+        self._t.join(timeout=5)
+        sm = [a for a, _ in self.samples]
+        pw = [b for _, b in self.samples]
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+               "power_w_max": max(pw) if pw else None, "samples": len(sm),
+               "reasons": sorted(self.reasons), "source": "nvml"}
+        if self.err:
+            out["note"] = self.err
+        return out
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -247,8 +265,7 @@ def run_gpu(args, rank, world, local_rank):
     if err != 0:
         raise RuntimeError(f"device status after warm-up: {moe.status_string(err)}")
 
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    clocks = ClockSampler(vis.split(",")[local_rank] if vis else local_rank)
+    clocks = ClockSampler(torch.cuda.current_device())
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
