@@ -185,6 +185,33 @@ moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_r
                        const uint16_t* residual, uint16_t* out, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* Size of the scratch array built into the library for moe_route_noalloc. */
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES 65536
+
+/* moe_route_noalloc: moe_route without a caller-provided workspace. The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device memory.
+ * Examples: an engine that hands out all device memory from its own arena up front; code on
+ * a real-time path where an allocation could synchronise the device or fail mid-run; a plugin
+ * whose host framework owns every allocation.
+ *
+ * Inputs, outputs, results and validation are those of moe_route. The capacity scan's scratch
+ * comes from a static array of MOE_ROUTE_NOALLOC_SCRATCH_BYTES in the library's own device
+ * memory. Every GPU that loads the library holds that array until the process exits.
+ *   - Limit: when T * k spans more than one capacity chunk (4096 pairs), the scan needs
+ *     ceil(T * k / 4096) * N int32 of scratch. A shape that needs more than the array holds
+ *     is rejected with MOE_ERR_WORKSPACE before anything is launched. With N = 256 the limit
+ *     is T * k <= 262144 pairs (64 chunks).
+ *   - The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current) and caches it. Make that first call before any stream capture.
+ *   - All calls share the one array, and it keeps the last call's contents. Each call writes
+ *     every scratch entry before reading it, so nothing has to start at zero. Calls that
+ *     overlap on the GPU (on concurrent streams) race on the array and must be serialised
+ *     by the caller. */
+moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                             const float* logit_bias, float* logits, int32_t* topk_idx,
+                             float* topk_w, int32_t* slot, int32_t* expert_count, void* stream);
+
 /* Synchronise `stream`, read the status word of a per-stage workspace into *err and clear it.
  * (For a moe_forward workspace pass moe_forward_buffers.stage_ws.) */
 moe_status moe_read_device_error(void* ws, void* stream, moe_status* err);

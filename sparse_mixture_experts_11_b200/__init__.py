@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m sparse_mixture_experts_11_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python sparse_mixture_experts_11_b200/build.py` "
         "(the MoE layer has no implementation other than this CUDA library)")
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -68,6 +68,7 @@ _SIGS = {
     "moe_forward_workspace_bytes": (ctypes.c_int, [_DIMS, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_forward_layout": (ctypes.c_int, [_DIMS, _P, ctypes.c_size_t, ctypes.POINTER(ForwardBuffers)]),
     "moe_forward": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_route_noalloc": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_read_device_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int)]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -179,6 +180,21 @@ def route(dims: Dims, x, w_router, logit_bias, logits, topk_idx, topk_w, slot, e
         _ptr(topk_w, "topk_w", torch.float32, (T, k)), _ptr(slot, "slot", torch.int32, (T, k)),
         _ptr(expert_count, "expert_count", torch.int32, (N,)), _ptr(ws, "ws", torch.uint8),
         _nbytes(ws), _stream(stream)), "moe_route")
+
+
+def route_noalloc(dims: Dims, x, w_router, logit_bias, logits, topk_idx, topk_w, slot,
+                  expert_count, stream=None) -> None:
+    """moe_route without a workspace argument: for callers that cannot allocate device memory.
+    Its scratch is a fixed array inside the library, shared by all calls. Calls that overlap
+    on the GPU race on it, and shapes beyond its size are rejected (MOE_ERR_WORKSPACE)."""
+    T, d, N, k = dims.T, dims.d_model, dims.n_experts, dims.top_k
+    _check(_lib.moe_route_noalloc(
+        ctypes.byref(dims), _ptr(x, "x", torch.bfloat16, (T, d)),
+        _ptr(w_router, "w_router", torch.float32, (N, d)),
+        _ptr(logit_bias, "logit_bias", torch.float32, (N,), allow_none=True),
+        _ptr(logits, "logits", torch.float32, (T, N)), _ptr(topk_idx, "topk_idx", torch.int32, (T, k)),
+        _ptr(topk_w, "topk_w", torch.float32, (T, k)), _ptr(slot, "slot", torch.int32, (T, k)),
+        _ptr(expert_count, "expert_count", torch.int32, (N,)), _stream(stream)), "moe_route_noalloc")
 
 
 def route_from_logits(dims: Dims, logits, topk_idx, topk_w, slot, expert_count, ws,

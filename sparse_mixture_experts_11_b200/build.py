@@ -1,6 +1,7 @@
 """Build the in-tree CUDA library ``libmoe.so`` for sm_100a with nvcc.
 
-Usage: ``python -m sparse_mixture_experts_11_b200.build [--verbose]``. The shared object is
+Usage: ``python sparse_mixture_experts_11_b200/build.py [--verbose] [--force]`` (run as a
+script: importing the package itself needs the built library). The shared object is
 written next to this file so it travels with the source tree.
 """
 from __future__ import annotations
@@ -14,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmoe.so")
-SOURCES = ["api.cu", "route.cu", "permute_combine.cu", "grouped_ffn.cu"]
+SOURCES = ["api.cu", "route.cu", "permute_combine.cu", "grouped_ffn.cu", "route_noalloc.cu"]
 GENCODE = "-gencode=arch=compute_100a,code=sm_100a"
 
 

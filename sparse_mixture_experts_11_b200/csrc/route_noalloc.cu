@@ -1,0 +1,90 @@
+// moe_route_noalloc: moe_route for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc, or have no allocator to ask. Examples: an inference
+// engine that hands out all device memory up front from its own arena; code on a real-time
+// path where an allocation could synchronise the device or fail mid-run; a plugin whose host
+// framework owns every allocation. moe_route needs a caller-provided workspace for its
+// capacity scan. This variant takes that scratch from a fixed array in the library's own
+// device memory instead, so its caller passes only inputs and outputs.
+//
+// The scratch lives in a file-scope __device__ array. Every GPU that loads the library holds
+// it until the process exits. In host code, the array's name is only a host-side stand-in
+// for the symbol: it is not a device address. A kernel given it would fault, or on a system
+// where the GPU can reach host memory, silently use the wrong memory. The device address is
+// therefore looked up once per device with cudaGetSymbolAddress (with that device current)
+// and then passed to the kernels.
+#include <mutex>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace {
+
+constexpr int kScratchInts = MOE_ROUTE_NOALLOC_SCRATCH_BYTES / 4;
+static_assert(MOE_ROUTE_NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch size");
+
+// Per-chunk expert histograms of the capacity scan: [n_chunks, N] int32. Each call writes
+// every entry it later reads, so nothing in it has to start at zero.
+static __device__ __align__(256) int32_t g_route_scratch[kScratchInts];
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_once[kMaxDevices];
+int32_t* g_scratch_ptr[kMaxDevices];
+cudaError_t g_scratch_err[kMaxDevices];
+
+// Device address of g_route_scratch on the current device; looked up on the first call per
+// device (with that device current) and cached.
+cudaError_t scratch_on_current_device(int32_t** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_once[dev], [dev] {
+    void* p = nullptr;
+    g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_route_scratch);
+    g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  });
+  *out = g_scratch_ptr[dev];
+  return g_scratch_err[dev];
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x,
+                                        const float* w_router, const float* logit_bias,
+                                        float* logits, int32_t* topk_idx, float* topk_w,
+                                        int32_t* slot, int32_t* expert_count, void* stream) {
+  if (dims == nullptr) return MOE_ERR_INVALID;
+  // Same shape rules as moe_route (moe_workspace_bytes validates and sizes).
+  size_t ws_bytes = 0;
+  const moe_status st = moe_workspace_bytes(dims, &ws_bytes);
+  if (st != MOE_OK) return st;
+  if (dims->T == 0) return MOE_OK;
+  const int64_t pairs = static_cast<int64_t>(dims->T) * dims->top_k;
+  const int64_t chunks = moe::slot_chunks(pairs);
+  const int64_t scratch_ints = chunks > 1 ? chunks * dims->n_experts : 0;
+  if (scratch_ints > kScratchInts) return MOE_ERR_WORKSPACE;  // beyond the built-in scratch
+  if (!x || !w_router || !logits || !topk_idx || !topk_w || !slot || !expert_count)
+    return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(logits) || !aligned16(topk_idx) ||
+      !aligned16(topk_w) || !aligned16(slot) || !aligned16(expert_count) ||
+      (logit_bias && !aligned16(logit_bias)))
+    return MOE_ERR_UNSUPPORTED;
+  moe::DeviceInfo di;
+  if (moe::device_info(&di) != cudaSuccess) return MOE_ERR_CUDA;
+  if (di.cc_major != 10 || di.cc_minor != 0) return MOE_ERR_UNSUPPORTED;
+  int32_t* scratch = nullptr;
+  if (scratch_on_current_device(&scratch) != cudaSuccess || scratch == nullptr) return MOE_ERR_CUDA;
+
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (moe::launch_router_topk(x, w_router, logit_bias, logits, topk_idx, topk_w, dims->T,
+                              dims->d_model, dims->n_experts, dims->top_k, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int cap = dims->capacity < dims->T ? dims->capacity : dims->T;
+  if (moe::launch_capacity_slots(topk_idx, slot, expert_count, scratch, dims->T, dims->n_experts,
+                                 dims->top_k, cap, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
