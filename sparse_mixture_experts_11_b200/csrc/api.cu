@@ -143,7 +143,8 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const float* w_rou
   const cudaStream_t s = as_stream(stream);
   st = launch_status(moe::launch_router_topk(x, w_router, logit_bias, logits, topk_idx, topk_w,
                                              dims->T, dims->d_model, dims->n_experts,
-                                             dims->top_k, s));
+                                             dims->top_k, status_of(ws), moe::kDefaultWaitTimeoutNs,
+                                             s));
   if (st != MOE_OK) return st;
   return route_slots(dims, topk_idx, slot, expert_count, ws, s);
 }

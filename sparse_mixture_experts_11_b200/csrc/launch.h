@@ -22,10 +22,14 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
-// router: logits = x W_r^T (+ b), then top-k and renormalised weights
+// router: logits = x W_r^T (+ b), then top-k and renormalised weights. Picks the per-token
+// SIMT kernel for small batches and the tensor-core kernel otherwise. status may be null.
 cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const float* bias,
                                float* logits, int32_t* topk_idx, float* topk_w, int T, int d,
-                               int N, int k, cudaStream_t s);
+                               int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s);
+cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const float* bias,
+                             float* logits, int32_t* topk_idx, float* topk_w, int T, int d, int N,
+                             int k, int* status, uint64_t timeout_ns, cudaStream_t s);
 // top-k and renormalised weights from given logits
 cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, float* topk_w, int T,
                                     int N, int k, cudaStream_t s);

@@ -90,82 +90,46 @@ __device__ __forceinline__ void warp_topk_write(const float (&val)[EPT], int N, 
 }
 
 // ------------------------------------------------------------------ router (SIMT fp32)
-constexpr int kRtTok = 32;      // tokens per block
-constexpr int kRtChunk = 32;    // d elements per shared-memory stage
-constexpr int kRtThreads = 256; // 8 warps; warp w owns tokens 4w..4w+3 of the block
-
-// logits[t, e] = sum_i x[t, i] * W_r[e, i] (+ b[e]) in fp32, summed in order of i;
-// then top-k and weights for each token of the block.
+// One block per token for small batches: warp w computes the logits of experts w, w+8, ...,
+// lanes splitting d (float4 of W_r and 4 bf16 of x per step), then a shuffle-tree sum; then
+// warp 0 takes the top-k of the token's N logits.
 template <int EPT>
-__global__ void __launch_bounds__(kRtThreads) router_topk_kernel(
+__global__ void __launch_bounds__(256) router_token_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias,
     float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int T,
     int d, int N, int k) {
-  __shared__ float xs[kRtTok][kRtChunk + 1];
-  __shared__ float ws[EPT * 32][kRtChunk + 1];
-  const int tid = threadIdx.x;
-  const int ty = tid >> 5, tx = tid & 31;
-  const int t0 = blockIdx.x * kRtTok;
-
-  for (int i = tid; i < EPT * 32 * (kRtChunk + 1); i += kRtThreads) (&ws[0][0])[i] = 0.f;
-
-  float acc[4][EPT];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < EPT; ++j) acc[i][j] = 0.f;
-
-  for (int c0 = 0; c0 < d; c0 += kRtChunk) {
-    __syncthreads();
-    {  // 32 tokens x 32 bf16: 4 elements per thread
-      const int tok = tid >> 3, c = (tid & 7) * 4;
-      float f[4] = {0.f, 0.f, 0.f, 0.f};
-      if (t0 + tok < T) {
-        const uint2 v = *reinterpret_cast<const uint2*>(x + static_cast<int64_t>(t0 + tok) * d + c0 + c);
-        f[0] = __uint_as_float(v.x << 16);
-        f[1] = __uint_as_float(v.x & 0xffff0000u);
-        f[2] = __uint_as_float(v.y << 16);
-        f[3] = __uint_as_float(v.y & 0xffff0000u);
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) xs[tok][c + q] = f[q];
+  __shared__ float s_logit[EPT * 32];
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint16_t* xr = x + static_cast<int64_t>(t) * d;
+  for (int e = warp; e < N; e += 8) {
+    const float* wr = w + static_cast<int64_t>(e) * d;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 4
+    for (int i = lane * 4; i < d; i += 128) {
+      const float4 wv = __ldg(reinterpret_cast<const float4*>(wr + i));
+      const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + i));
+      a0 = fmaf(__uint_as_float(xv.x << 16), wv.x, a0);
+      a1 = fmaf(__uint_as_float(xv.x & 0xffff0000u), wv.y, a1);
+      a2 = fmaf(__uint_as_float(xv.y << 16), wv.z, a2);
+      a3 = fmaf(__uint_as_float(xv.y & 0xffff0000u), wv.w, a3);
     }
-    for (int f = tid; f < N * (kRtChunk / 4); f += kRtThreads) {
-      const int e = f / (kRtChunk / 4), c = (f % (kRtChunk / 4)) * 4;
-      const float4 v = *reinterpret_cast<const float4*>(w + static_cast<int64_t>(e) * d + c0 + c);
-      ws[e][c] = v.x;
-      ws[e][c + 1] = v.y;
-      ws[e][c + 2] = v.z;
-      ws[e][c + 3] = v.w;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int c = 0; c < kRtChunk; ++c) {
-      float xv[4];
+    float acc = (a0 + a1) + (a2 + a3);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) xv[i] = xs[ty * 4 + i][c];
-#pragma unroll
-      for (int j = 0; j < EPT; ++j) {
-        const float wv = ws[tx + 32 * j][c];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(xv[i], wv, acc[i][j]);
-      }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+    if (lane == 0) {
+      const float L = acc + (bias != nullptr ? bias[e] : 0.f);
+      s_logit[e] = L;
+      logits[static_cast<int64_t>(t) * N + e] = L;
     }
   }
-
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
-    if (t >= T) break;  // warp-uniform
+  __syncthreads();
+  if (warp == 0) {
     float val[EPT];
 #pragma unroll
     for (int j = 0; j < EPT; ++j) {
-      const int e = tx + 32 * j;
-      val[j] = acc[i][j];
-      if (e < N) {
-        if (bias != nullptr) val[j] += bias[e];
-        logits[static_cast<int64_t>(t) * N + e] = val[j];
-      }
+      const int e = lane + 32 * j;
+      val[j] = (e < N) ? s_logit[e] : -INFINITY;
     }
     warp_topk_write<EPT>(val, N, k, t, topk_idx, topk_w);
   }
@@ -209,25 +173,32 @@ __global__ void __launch_bounds__(kSlThreads) slot_rank_kernel(
     int cap, int single_chunk) {
   __shared__ int s_cnt[kSlWarps][256];
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int64_t P = static_cast<int64_t>(T) * k;
+  const int P = T * k;  // < 2^31, checked on the host
   for (int i = tid; i < kSlWarps * 256; i += kSlThreads) (&s_cnt[0][0])[i] = 0;
-  __syncthreads();
 
-  const int64_t p_base =
-      static_cast<int64_t>(blockIdx.x) * kSlotChunk + static_cast<int64_t>(w) * (kSlotChunk / kSlWarps);
-  int local[kSlIters];
+  const int p_base = blockIdx.x * kSlotChunk + w * (kSlotChunk / kSlWarps);
   int ex[kSlIters];
+  int q_of[kSlIters];  // storage index t * k + j of each arrival
+  // all loads first, so their latencies overlap
 #pragma unroll
   for (int it = 0; it < kSlIters; ++it) {
-    const int64_t p = p_base + it * 32 + lane;
-    int e = -1;
+    const int p = p_base + it * 32 + lane;
+    int e = -1, q = -1;
     if (p < P) {
-      const int j = static_cast<int>(p / T);
-      const int t = static_cast<int>(p - static_cast<int64_t>(j) * T);
-      e = topk_idx[static_cast<int64_t>(t) * k + j];
+      const int j = p / T;
+      const int t = p - j * T;
+      q = t * k + j;
+      e = __ldg(topk_idx + q);
       if (e < 0 || e >= N) e = -2;  // invalid expert id: never kept
     }
     ex[it] = e;
+    q_of[it] = q;
+  }
+  __syncthreads();
+  int local[kSlIters];
+#pragma unroll
+  for (int it = 0; it < kSlIters; ++it) {
+    const int e = ex[it];
     const unsigned peers = __match_any_sync(kFull, e);
     const int rank = __popc(peers & lanemask_lt());
     const int cnt = (e >= 0) ? s_cnt[w][e] : 0;
@@ -253,17 +224,14 @@ __global__ void __launch_bounds__(kSlThreads) slot_rank_kernel(
   __syncthreads();
 #pragma unroll
   for (int it = 0; it < kSlIters; ++it) {
-    const int64_t p = p_base + it * 32 + lane;
-    if (p >= P) break;
-    const int j = static_cast<int>(p / T);
-    const int t = static_cast<int>(p - static_cast<int64_t>(j) * T);
+    if (q_of[it] < 0) continue;
     const int e = ex[it];
     int out = -1;
     if (e >= 0) {
       const int r = local[it] + s_cnt[w][e];
       out = single_chunk ? (r < cap ? r : -1) : r;
     }
-    slot[static_cast<int64_t>(t) * k + j] = out;
+    slot[q_of[it]] = out;
   }
 }
 
@@ -285,19 +253,18 @@ __global__ void __launch_bounds__(256) slot_finalize_kernel(const int32_t* __res
                                                             int32_t* __restrict__ slot,
                                                             const int32_t* __restrict__ chunk_hist,
                                                             int T, int N, int k, int cap) {
-  const int64_t P = static_cast<int64_t>(T) * k;
-  for (int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; p < P;
-       p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int j = static_cast<int>(p / T);
-    const int t = static_cast<int>(p - static_cast<int64_t>(j) * T);
-    const int64_t q = static_cast<int64_t>(t) * k + j;
+  const int P = T * k;
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < P; p += gridDim.x * blockDim.x) {
+    const int j = p / T;
+    const int t = p - j * T;
+    const int q = t * k + j;
     const int e = topk_idx[q];
     const int local = slot[q];
     if (e < 0 || e >= N || local < 0) {
       slot[q] = -1;
       continue;
     }
-    const int r = local + chunk_hist[(p / kSlotChunk) * N + e];
+    const int r = local + chunk_hist[static_cast<int64_t>(p / kSlotChunk) * N + e];
     slot[q] = r < cap ? r : -1;
   }
 }
@@ -307,16 +274,21 @@ __global__ void __launch_bounds__(256) slot_finalize_kernel(const int32_t* __res
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const float* bias,
                                float* logits, int32_t* topk_idx, float* topk_w, int T, int d,
-                               int N, int k, cudaStream_t s) {
-  const dim3 grid((T + kRtTok - 1) / kRtTok);
+                               int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
+  // Small batches: one block per token re-reads W_r from L2 per token. Once that re-read
+  // traffic would pass 256 MiB, the tensor-core router (W_r read once per 128 tokens) wins.
+  const double per_token_l2 = static_cast<double>(T) * N * d * 4.0;
+  if (per_token_l2 > 268435456.0)
+    return launch_router_tc(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status,
+                            timeout_ns, s);
   if (N <= 32)
-    router_topk_kernel<1><<<grid, kRtThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+    router_token_kernel<1><<<T, 256, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
   else if (N <= 64)
-    router_topk_kernel<2><<<grid, kRtThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+    router_token_kernel<2><<<T, 256, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
   else if (N <= 128)
-    router_topk_kernel<4><<<grid, kRtThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+    router_token_kernel<4><<<T, 256, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
   else
-    router_topk_kernel<8><<<grid, kRtThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+    router_token_kernel<8><<<T, 256, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
   return cudaGetLastError();
 }
 

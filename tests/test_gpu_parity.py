@@ -20,6 +20,13 @@ SMALL_CASES = [
     ("single_token", 1, 256, 8, 2, 256, "swiglu", None, None),
     ("k_equals_n", 40, 64, 4, 4, 64, "swiglu", None, None),
     ("heavy_drop", 200, 128, 8, 2, 128, "swiglu", 0.25, 1.1),
+    # large enough that the router runs on tensor cores (T*N*d*4 bytes > 256 MiB);
+    # expert counts padded to 16, 32, 64, 128 (N=100) and 256 tensor-core columns
+    ("tc_router_n8_bias", 20000, 512, 8, 2, 128, "swiglu", 1.25, 1.1),
+    ("tc_router_n32_ragged_T", 2200, 1024, 32, 4, 128, "swiglu", None, None),
+    ("tc_router_n64_gelu", 3000, 512, 64, 2, 256, "gelu", 1.0, None),
+    ("tc_router_n100", 2700, 256, 100, 3, 128, "swiglu", 1.25, None),
+    ("tc_router_n256_k8", 1100, 256, 256, 8, 64, "swiglu", 1.25, 1.1),
 ]
 
 
