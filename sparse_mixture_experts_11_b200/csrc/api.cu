@@ -76,11 +76,25 @@ int64_t max_rows(const moe_dims* d) {
                            static_cast<int64_t>(d->n_experts) * cap);
 }
 
-size_t stage_ws_bytes(const moe_dims* d) {
+// Per-stage workspace: [status word, 256 B][capacity-scan chunk totals][router weight split].
+size_t slot_scratch_bytes(const moe_dims* d) {
   const int64_t chunks = moe::slot_chunks(static_cast<int64_t>(d->T) * d->top_k);
-  size_t b = moe::kStatusBytes;
-  if (chunks > 1) b += static_cast<size_t>(chunks) * d->n_experts * sizeof(int32_t);
-  return round_up(b, 256);
+  return chunks > 1 ? round_up(static_cast<size_t>(chunks) * d->n_experts * sizeof(int32_t), 256) : 0;
+}
+
+size_t split_scratch_bytes(const moe_dims* d) {
+  return moe::router_uses_tensor_cores(d->T, d->n_experts, d->d_model)
+             ? round_up(moe::router_split_bytes(d->n_experts, d->d_model), 256)
+             : 0;
+}
+
+size_t stage_ws_bytes(const moe_dims* d) {
+  return moe::kStatusBytes + slot_scratch_bytes(d) + split_scratch_bytes(d);
+}
+
+uint16_t* split_scratch_of(const moe_dims* d, void* ws) {
+  if (split_scratch_bytes(d) == 0) return nullptr;
+  return reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + moe::kStatusBytes + slot_scratch_bytes(d));
 }
 
 int* status_of(void* ws) { return static_cast<int*>(ws); }
@@ -143,8 +157,8 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const float* w_rou
   const cudaStream_t s = as_stream(stream);
   st = launch_status(moe::launch_router_topk(x, w_router, logit_bias, logits, topk_idx, topk_w,
                                              dims->T, dims->d_model, dims->n_experts,
-                                             dims->top_k, status_of(ws), moe::kDefaultWaitTimeoutNs,
-                                             s));
+                                             dims->top_k, split_scratch_of(dims, ws), status_of(ws),
+                                             moe::kDefaultWaitTimeoutNs, s));
   if (st != MOE_OK) return st;
   return route_slots(dims, topk_idx, slot, expert_count, ws, s);
 }

@@ -22,14 +22,26 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
-// router: logits = x W_r^T (+ b), then top-k and renormalised weights. Picks the per-token
-// SIMT kernel for small batches and the tensor-core kernel otherwise. status may be null.
+// Router path choice. One block per token re-reads W_r from L2 for every token; once that
+// traffic (T * N * d * 4 bytes) passes 256 MiB the tensor-core router, which reads W_r once
+// per 128 tokens, is used instead.
+inline bool router_uses_tensor_cores(int64_t T, int64_t N, int64_t d) {
+  return static_cast<double>(T) * N * d * 4.0 > 268435456.0;
+}
+// Bytes of the [3][N][d] bf16 split of W_r the tensor-core router reads when given scratch.
+size_t router_split_bytes(int N, int d);
+
+// router: logits = x W_r^T (+ b), then top-k and renormalised weights. status may be null.
+// split_scratch: router_split_bytes() of device memory for the tensor-core path, or null to
+// split W_r inside the router kernel (same results, slower).
 cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const float* bias,
                                float* logits, int32_t* topk_idx, float* topk_w, int T, int d,
-                               int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s);
+                               int N, int k, uint16_t* split_scratch, int* status,
+                               uint64_t timeout_ns, cudaStream_t s);
 cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const float* bias,
                              float* logits, int32_t* topk_idx, float* topk_w, int T, int d, int N,
-                             int k, int* status, uint64_t timeout_ns, cudaStream_t s);
+                             int k, uint16_t* split_scratch, int* status, uint64_t timeout_ns,
+                             cudaStream_t s);
 // top-k and renormalised weights from given logits
 cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, float* topk_w, int T,
                                     int N, int k, cudaStream_t s);

@@ -274,13 +274,11 @@ __global__ void __launch_bounds__(256) slot_finalize_kernel(const int32_t* __res
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const float* bias,
                                float* logits, int32_t* topk_idx, float* topk_w, int T, int d,
-                               int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
-  // Small batches: one block per token re-reads W_r from L2 per token. Once that re-read
-  // traffic would pass 256 MiB, the tensor-core router (W_r read once per 128 tokens) wins.
-  const double per_token_l2 = static_cast<double>(T) * N * d * 4.0;
-  if (per_token_l2 > 268435456.0)
-    return launch_router_tc(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status,
-                            timeout_ns, s);
+                               int N, int k, uint16_t* split_scratch, int* status,
+                               uint64_t timeout_ns, cudaStream_t s) {
+  if (router_uses_tensor_cores(T, N, d))
+    return launch_router_tc(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k,
+                            split_scratch, status, timeout_ns, s);
   if (N <= 32)
     router_token_kernel<1><<<T, 256, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
   else if (N <= 64)

@@ -4,8 +4,10 @@
 // engine that hands out all device memory up front from its own arena; code on a real-time
 // path where an allocation could synchronise the device or fail mid-run; a plugin whose host
 // framework owns every allocation. moe_route needs a caller-provided workspace for its
-// capacity scan. This variant takes that scratch from a fixed array in the library's own
-// device memory instead, so its caller passes only inputs and outputs.
+// capacity scan (and, for large batches, for a bf16 split of the router weight). This variant
+// takes the capacity-scan scratch from a fixed array in the library's own device memory and
+// splits the router weight inside the router kernel instead, so its caller passes only inputs
+// and outputs. Its results are identical to moe_route's.
 //
 // The scratch lives in a file-scope __device__ array. Every GPU that loads the library holds
 // it until the process exits. In host code, the array's name is only a host-side stand-in
@@ -80,7 +82,7 @@ extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x,
 
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (moe::launch_router_topk(x, w_router, logit_bias, logits, topk_idx, topk_w, dims->T,
-                              dims->d_model, dims->n_experts, dims->top_k, nullptr,
+                              dims->d_model, dims->n_experts, dims->top_k, nullptr, nullptr,
                               moe::kDefaultWaitTimeoutNs, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   const int cap = dims->capacity < dims->T ? dims->capacity : dims->T;

@@ -11,17 +11,25 @@
 // dot product to within fp32 accumulation error. Every product of two bf16 values is exact
 // in fp32.
 //
+// Two ways to get the split terms, with identical results (same bf16 terms, same MMA order):
+//   PRESPLIT  a small kernel writes [3][N][d] bf16 into the caller's workspace once per call
+//             and the router kernel TMA-loads the three term tiles with each x tile;
+//   in-kernel for callers without a workspace: warps 4-7 read W_r[:, k block] in fp32 and
+//             write the three terms as K-major 128B-swizzled tiles into shared memory
+//             (double buffered), every CTA repeating the conversion.
+//
 // One CTA per 128-token tile, 256 threads:
-//   warp 0      TMA producer of the x tile [128 tokens x 64 k] (128B swizzle) into a ring;
+//   warp 0      TMA producer of the x tile [128 tokens x 64 k] (128B swizzle) into a ring
+//               (and of the three weight term tiles when PRESPLIT);
 //   warp 1      TMEM owner and MMA issuer: per k block 3 x 4 MMAs (M=128, N=NP, K=16) into one
 //               fp32 accumulator of NP columns;
-//   warps 4-7   split converters during the main loop: read W_r[:, k block] in fp32, write
-//               hi/mid/lo as K-major 128B-swizzled bf16 tiles (double buffered); then the
-//               epilogue: thread i owns token i's row of logits in TMEM, adds the bias,
-//               writes the logits, keeps a running top-k and writes indices and weights.
+//   warps 4-7   (in-kernel split only) the converters, then the epilogue: thread i owns token
+//               i's row of logits in TMEM, adds the bias, writes the logits, keeps a running
+//               top-8 and writes the first k indices and weights.
 // All mbarrier waits are bounded. A timeout records MOE_ERR_TIMEOUT, stops the CTA's work,
 // drains its own copies and MMAs, and frees TMEM.
 #include <math.h>
+#include <string.h>
 
 #include <algorithm>
 #include <mutex>
@@ -38,16 +46,20 @@ constexpr int kThreads = 256;
 constexpr int kConvThreads = 128;
 constexpr int kSmemLimit = 225 * 1024;
 
-template <int NP>
+template <int NP, bool PRESPLIT>
 struct RCfg {
-  static constexpr int A_BYTES = kTok * kBK * 2;           // 16 KB per x stage
+  static constexpr int A_BYTES = kTok * kBK * 2;           // 16 KB per x tile
   static constexpr int WT_BYTES = NP * kBK * 2;            // one split term tile
   static constexpr int WBUF_BYTES = 3 * WT_BYTES;          // hi, mid, lo
-  static constexpr int A_STAGES_FIT = (kSmemLimit - 1024 - 2 * WBUF_BYTES) / A_BYTES;
-  static constexpr int A_STAGES = A_STAGES_FIT > 8 ? 8 : A_STAGES_FIT;
+  // PRESPLIT: each ring stage holds the x tile and the three term tiles.
+  // in-kernel: a ring of x tiles plus two converter-written term buffers.
+  static constexpr int STAGE_BYTES = PRESPLIT ? A_BYTES + WBUF_BYTES : A_BYTES;
+  static constexpr int FIXED_BYTES = PRESPLIT ? 0 : 2 * WBUF_BYTES;
+  static constexpr int STAGES_FIT = (kSmemLimit - 1024 - FIXED_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int TMEM_COLS = NP < 32 ? 32 : NP;
-  static constexpr int SMEM_BYTES = 2 * WBUF_BYTES + A_STAGES * A_BYTES + 1024;
-  static_assert(A_STAGES >= 2, "router pipeline depth");
+  static constexpr int SMEM_BYTES = FIXED_BYTES + STAGES * STAGE_BYTES + 1024;
+  static_assert(STAGES >= 2, "router pipeline depth");
   static_assert(NP % 16 == 0 && NP >= 16 && NP <= 256, "UMMA N for M = 128");
 };
 
@@ -60,16 +72,57 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int NP>
+// Split 8 consecutive fp32 weights into three bf16 terms each (hi, mid, lo), packed in pairs.
+__device__ __forceinline__ void split3(const float4& v0, const float4& v1, uint4& hi, uint4& mid,
+                                       uint4& lo) {
+  const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  uint32_t h[4], m[4], l[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float r0 = f[2 * q], r1 = f[2 * q + 1];
+    const __nv_bfloat162 bh = __floats2bfloat162_rn(r0, r1);
+    r0 -= __low2float(bh);
+    r1 -= __high2float(bh);
+    const __nv_bfloat162 bm = __floats2bfloat162_rn(r0, r1);
+    r0 -= __low2float(bm);
+    r1 -= __high2float(bm);
+    const __nv_bfloat162 bl = __floats2bfloat162_rn(r0, r1);
+    h[q] = *reinterpret_cast<const uint32_t*>(&bh);
+    m[q] = *reinterpret_cast<const uint32_t*>(&bm);
+    l[q] = *reinterpret_cast<const uint32_t*>(&bl);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  mid = make_uint4(m[0], m[1], m[2], m[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// W_r [N, d] fp32 -> [3][N][d] bf16 terms (row-major per term).
+__global__ void __launch_bounds__(256) split_router_weights_kernel(const float* __restrict__ w,
+                                                                   uint16_t* __restrict__ out,
+                                                                   int64_t n_elems) {
+  const int64_t n8 = n_elems / 8;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4* src = reinterpret_cast<const float4*>(w) + 2 * i;
+    uint4 hi, mid, lo;
+    split3(__ldg(src), __ldg(src + 1), hi, mid, lo);
+    reinterpret_cast<uint4*>(out)[i] = hi;
+    reinterpret_cast<uint4*>(out + n_elems)[i] = mid;
+    reinterpret_cast<uint4*>(out + 2 * n_elems)[i] = lo;
+  }
+}
+
+template <int NP, bool PRESPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
-    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const float* __restrict__ w,
-                     const float* __restrict__ bias, float* __restrict__ logits,
-                     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int T, int d,
-                     int N, int k, int* status, uint64_t timeout_ns) {
-  using C = RCfg<NP>;
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const float* __restrict__ w, const float* __restrict__ bias,
+                     float* __restrict__ logits, int32_t* __restrict__ topk_idx,
+                     float* __restrict__ topk_w, int T, int d, int N, int k, int* status,
+                     uint64_t timeout_ns) {
+  using C = RCfg<NP, PRESPLIT>;
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
-  __shared__ __align__(8) uint64_t a_full[C::A_STAGES];
-  __shared__ __align__(8) uint64_t a_empty[C::A_STAGES];
+  __shared__ __align__(8) uint64_t a_full[C::STAGES];
+  __shared__ __align__(8) uint64_t a_empty[C::STAGES];
   __shared__ __align__(8) uint64_t w_full[2];
   __shared__ __align__(8) uint64_t w_empty[2];
   __shared__ __align__(8) uint64_t acc_full;
@@ -80,14 +133,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   uint8_t* gbase = dyn_smem + (base - smem_u32(dyn_smem));  // generic pointer of `base`
-  const uint32_t wbuf0 = base;                               // 2 x [3][NP][64] bf16
-  const uint32_t abuf0 = base + 2 * C::WBUF_BYTES;           // A_STAGES x [128][64] bf16
+  const uint32_t wbuf0 = base;                               // in-kernel: 2 x [3][NP][64] bf16
+  const uint32_t ring0 = base + C::FIXED_BYTES;              // ring of stages
   const int t0 = blockIdx.x * kTok;
   const int num_kb = d / kBK;
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmX);
-    for (int s = 0; s < C::A_STAGES; ++s) {
+    if (PRESPLIT) prefetch_tensormap(&tmW);
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_u32(&a_full[s]), 1);
       mbar_init(smem_u32(&a_empty[s]), 1);
     }
@@ -105,8 +159,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(&s_tmem), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp >= 4 && NP > N) {
-    // rows N..NP-1 of both split buffers stay zero for the whole kernel
+  if (!PRESPLIT && warp >= 4 && NP > N) {
+    // rows N..NP-1 of both term buffers stay zero for the whole kernel
     const int ct = threadIdx.x - 128;
     for (int b = 0; b < 2; ++b)
       for (int term = 0; term < 3; ++term)
@@ -123,42 +177,53 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s_tmem;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint64_t pol = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_first();
+      const uint64_t pol_w = l2_policy_evict_last();
       int kb = 0;
       bool ok = true;
       for (; kb < num_kb; ++kb) {
-        const int s = kb % C::A_STAGES;
-        if (!mbar_wait(smem_u32(&a_empty[s]), ((kb / C::A_STAGES) & 1) ^ 1u, timeout_ns, &s_abort)) {
+        const int s = kb % C::STAGES;
+        if (!mbar_wait(smem_u32(&a_empty[s]), ((kb / C::STAGES) & 1) ^ 1u, timeout_ns, &s_abort)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(smem_u32(&a_full[s]), C::A_BYTES);
-        tma_load_2d(abuf0 + s * C::A_BYTES, &tmX, smem_u32(&a_full[s]), kb * kBK, t0, pol);
+        const uint32_t st = ring0 + s * C::STAGE_BYTES;
+        const uint32_t fb = smem_u32(&a_full[s]);
+        mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+        tma_load_2d(st, &tmX, fb, kb * kBK, t0, pol_x);
+        if (PRESPLIT) {
+#pragma unroll
+          for (int term = 0; term < 3; ++term)
+            tma_load_3d(st + C::A_BYTES + term * C::WT_BYTES, &tmW, fb, kb * kBK, 0, term, pol_w);
+        }
       }
       if (!ok) {
         s_abort = 1;
         report_error(status, MOE_ERR_TIMEOUT);
       }
-      for (int i = max(0, kb - C::A_STAGES); i < kb; ++i)
-        mbar_wait(smem_u32(&a_full[i % C::A_STAGES]), (i / C::A_STAGES) & 1, timeout_ns, nullptr);
+      for (int i = max(0, kb - C::STAGES); i < kb; ++i)
+        mbar_wait(smem_u32(&a_full[i % C::STAGES]), (i / C::STAGES) & 1, timeout_ns, nullptr);
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kTok, NP);
       bool ok = true, issued = false;
       for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % C::A_STAGES, b = kb & 1;
-        if (!mbar_wait(smem_u32(&a_full[s]), (kb / C::A_STAGES) & 1, timeout_ns, &s_abort) ||
-            !mbar_wait(smem_u32(&w_full[b]), (kb >> 1) & 1, timeout_ns, &s_abort)) {
+        const int s = kb % C::STAGES, b = kb & 1;
+        if (!mbar_wait(smem_u32(&a_full[s]), (kb / C::STAGES) & 1, timeout_ns, &s_abort) ||
+            (!PRESPLIT && !mbar_wait(smem_u32(&w_full[b]), (kb >> 1) & 1, timeout_ns, &s_abort))) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t a = abuf0 + s * C::A_BYTES;
+        const uint32_t a = ring0 + s * C::STAGE_BYTES;
+        const uint32_t wt0 = PRESPLIT ? a + C::A_BYTES : wbuf0 + b * C::WBUF_BYTES;
 #pragma unroll
         for (int term = 0; term < 3; ++term) {
-          const uint32_t bt = wbuf0 + b * C::WBUF_BYTES + term * C::WT_BYTES;
+          const uint32_t bt = wt0 + term * C::WT_BYTES;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
             tc_mma_f16(tmem, smem_desc_k_sw128(a + kk * 32), smem_desc_k_sw128(bt + kk * 32), idesc,
@@ -166,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         issued = true;
         tc_commit(smem_u32(&a_empty[s]));
-        tc_commit(smem_u32(&w_empty[b]));
+        if (!PRESPLIT) tc_commit(smem_u32(&w_empty[b]));
       }
       if (ok) {
         tc_commit(smem_u32(&acc_full));
@@ -182,45 +247,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     const int ct = threadIdx.x - 128;  // 0..127
     bool ok = true;
-    // ---- main loop: split W_r[:, k block] into three bf16 terms, K-major swizzled tiles
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int b = kb & 1;
-      const bool got = mbar_wait(smem_u32(&w_empty[b]), ((kb >> 1) & 1) ^ 1u, timeout_ns, &s_abort);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after_sync();
-      uint8_t* buf = gbase + b * C::WBUF_BYTES;
-      for (int task = ct; task < N * 8; task += kConvThreads) {
-        const int row = task >> 3, chunk = task & 7;
-        const float4* src = reinterpret_cast<const float4*>(w + static_cast<int64_t>(row) * d + kb * kBK + chunk * 8);
-        const float4 v0 = __ldg(src), v1 = __ldg(src + 1);
-        const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        uint32_t hi[4], mid[4], lo[4];
+    if (!PRESPLIT) {
+      // -------------------------------------------------------- in-kernel split of W_r
+      constexpr int kTasks = (NP * 8 + kConvThreads - 1) / kConvThreads;  // <= 16
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const int b = kb & 1;
+        // issue every load of this k block before waiting, so their latencies overlap
+        float4 v[kTasks][2];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float r0 = f[2 * q], r1 = f[2 * q + 1];
-          const __nv_bfloat162 h = __floats2bfloat162_rn(r0, r1);
-          r0 -= __low2float(h);
-          r1 -= __high2float(h);
-          const __nv_bfloat162 m = __floats2bfloat162_rn(r0, r1);
-          r0 -= __low2float(m);
-          r1 -= __high2float(m);
-          const __nv_bfloat162 l = __floats2bfloat162_rn(r0, r1);
-          hi[q] = *reinterpret_cast<const uint32_t*>(&h);
-          mid[q] = *reinterpret_cast<const uint32_t*>(&m);
-          lo[q] = *reinterpret_cast<const uint32_t*>(&l);
+        for (int i = 0; i < kTasks; ++i) {
+          const int task = ct + i * kConvThreads;
+          if (task < N * 8) {
+            const float4* src = reinterpret_cast<const float4*>(
+                w + static_cast<int64_t>(task >> 3) * d + kb * kBK + (task & 7) * 8);
+            v[i][0] = __ldg(src);
+            v[i][1] = __ldg(src + 1);
+          }
         }
-        const uint32_t off = sw128_offset(row, chunk);
-        *reinterpret_cast<uint4*>(buf + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(buf + C::WT_BYTES + off) = make_uint4(mid[0], mid[1], mid[2], mid[3]);
-        *reinterpret_cast<uint4*>(buf + 2 * C::WT_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        const bool got = mbar_wait(smem_u32(&w_empty[b]), ((kb >> 1) & 1) ^ 1u, timeout_ns, &s_abort);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        uint8_t* buf = gbase + b * C::WBUF_BYTES;
+#pragma unroll
+        for (int i = 0; i < kTasks; ++i) {
+          const int task = ct + i * kConvThreads;
+          if (task < N * 8) {
+            uint4 hi, mid, lo;
+            split3(v[i][0], v[i][1], hi, mid, lo);
+            const uint32_t off = sw128_offset(task >> 3, task & 7);
+            *reinterpret_cast<uint4*>(buf + off) = hi;
+            *reinterpret_cast<uint4*>(buf + C::WT_BYTES + off) = mid;
+            *reinterpret_cast<uint4*>(buf + 2 * C::WT_BYTES + off) = lo;
+          }
+        }
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        mbar_arrive(smem_u32(&w_full[b]));
       }
-      fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-      mbar_arrive(smem_u32(&w_full[b]));
     }
-    // ---- epilogue: thread ct owns token t0 + ct
+    // ---------------------------------------------------------- epilogue: token t0 + ct
     if (ok) {
       const bool got = mbar_wait(smem_u32(&acc_full), 0, timeout_ns, &s_abort);
       ok = __all_sync(0xffffffffu, got);
@@ -231,6 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = t0 + ct;
       const bool valid = t < T;
       const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      // the best 8 are kept whatever k is (entry 7 is the admission threshold); the first k
+      // are written
       float best_v[8];
       int best_e[8];
 #pragma unroll
@@ -238,10 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         best_v[r] = -INFINITY;
         best_e[r] = 0x7fffffff;
       }
-      // the best 8 are kept whatever k is (entry 7 is the admission threshold); the first k
-      // are written
-      float thr_v = -INFINITY;
-      int thr_e = 0x7fffffff;
       for (int c0 = 0; c0 < N; c0 += 16) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(trow + c0, v);
@@ -254,20 +319,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (bias != nullptr) L += __ldg(bias + e);
           if (valid) logits[static_cast<int64_t>(t) * N + e] = L;
           const float key = isnan(L) ? -INFINITY : L;
-          // insert (key, e) into the sorted list best[0..7]
-          if (better(key, e, thr_v, thr_e)) {
+          if (better(key, e, best_v[7], best_e[7])) {
             // shift the entries the candidate beats down by one and drop it into place;
-            // from the last slot up, so best[r - 1] is still the old value when read
+            // from the last slot up, so entry r-1 is still the old value when read
 #pragma unroll
             for (int r = 7; r >= 0; --r) {
               if (better(key, e, best_v[r], best_e[r])) {
-                const bool above = (r == 0) || better(key, e, best_v[r > 0 ? r - 1 : 0], best_e[r > 0 ? r - 1 : 0]);
-                best_v[r] = above ? key : best_v[r > 0 ? r - 1 : 0];
-                best_e[r] = above ? e : best_e[r > 0 ? r - 1 : 0];
+                const int u = r > 0 ? r - 1 : 0;
+                const bool beats_prev = (r > 0) && better(key, e, best_v[u], best_e[u]);
+                best_v[r] = beats_prev ? best_v[u] : key;
+                best_e[r] = beats_prev ? best_e[u] : e;
               }
             }
-            thr_v = best_v[7];
-            thr_e = best_e[7];
           }
         }
       }
@@ -317,45 +380,83 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <int NP>
-cudaError_t launch_np(const CUtensorMap& mx, const float* w, const float* bias, float* logits,
-                      int32_t* topk_idx, float* topk_w, int T, int d, int N, int k, int* status,
-                      uint64_t timeout_ns, cudaStream_t s) {
-  using C = RCfg<NP>;
+template <int NP, bool PRESPLIT>
+cudaError_t launch_np(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
+                      const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
+                      int d, int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
+  using C = RCfg<NP, PRESPLIT>;
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(router_tc_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                C::SMEM_BYTES);
+    attr = cudaFuncSetAttribute(router_tc_kernel<NP, PRESPLIT>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr != cudaSuccess) return attr;
   const int grid = (T + kTok - 1) / kTok;
-  router_tc_kernel<NP><<<grid, kThreads, C::SMEM_BYTES, s>>>(mx, w, bias, logits, topk_idx, topk_w,
-                                                             T, d, N, k, status, timeout_ns);
+  router_tc_kernel<NP, PRESPLIT><<<grid, kThreads, C::SMEM_BYTES, s>>>(
+      mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns);
   return cudaGetLastError();
+}
+
+template <bool PRESPLIT>
+cudaError_t launch_tc(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
+                      const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
+                      int d, int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
+  if (N <= 16)
+    return launch_np<16, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+  if (N <= 32)
+    return launch_np<32, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+  if (N <= 64)
+    return launch_np<64, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+  if (N <= 128)
+    return launch_np<128, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+  return launch_np<256, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+}
+
+bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
+size_t router_split_bytes(int N, int d) { return static_cast<size_t>(3) * N * d * 2; }
+
 cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const float* bias,
                              float* logits, int32_t* topk_idx, float* topk_w, int T, int d, int N,
-                             int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return cudaErrorInvalidValue;
-  CUtensorMap mx;
-  const cuuint64_t gd[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T)};
-  const cuuint64_t gs[1] = {static_cast<cuuint64_t>(d) * 2};
-  const cuuint32_t box[2] = {kBK, kTok};
-  const cuuint32_t es[2] = {1, 1};
-  if (fn(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), gd, gs, box, es,
-         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  if (N <= 16) return launch_np<16>(mx, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
-  if (N <= 32) return launch_np<32>(mx, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
-  if (N <= 64) return launch_np<64>(mx, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
-  if (N <= 128) return launch_np<128>(mx, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
-  return launch_np<256>(mx, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+                             int k, uint16_t* split_scratch, int* status, uint64_t timeout_ns,
+                             cudaStream_t s) {
+  CUtensorMap mx, mw;
+  {
+    const cuuint64_t gd[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T)};
+    const cuuint64_t gs[1] = {static_cast<cuuint64_t>(d) * 2};
+    const cuuint32_t box[2] = {kBK, kTok};
+    if (!encode_bf16(&mx, x, 2, gd, gs, box)) return cudaErrorInvalidValue;
+  }
+  const int np = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+  if (split_scratch == nullptr) {
+    memset(&mw, 0, sizeof(mw));  // unused by the in-kernel split
+    return launch_tc<false>(mx, mw, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status,
+                            timeout_ns, s);
+  }
+  {
+    const cuuint64_t gd[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), 3};
+    const cuuint64_t gs[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+    const cuuint32_t box[3] = {kBK, static_cast<cuuint32_t>(np), 1};
+    if (!encode_bf16(&mw, split_scratch, 3, gd, gs, box)) return cudaErrorInvalidValue;
+  }
+  const int64_t n = static_cast<int64_t>(N) * d;
+  const int blocks = static_cast<int>(std::min<int64_t>((n / 8 + 255) / 256, 148 * 8));
+  split_router_weights_kernel<<<blocks, 256, 0, s>>>(w_router, split_scratch, n);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_tc<true>(mx, mw, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status,
+                         timeout_ns, s);
 }
 
 }  // namespace moe

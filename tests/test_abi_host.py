@@ -49,7 +49,9 @@ def test_workspace_sizes():
     small = moe.make_dims(64, 128, 8, 2, 256, "swiglu", 10)
     assert moe.workspace_bytes(small) == 256          # one capacity chunk: status word only
     big = moe.make_dims(16384, 7168, 256, 8, 2048, "swiglu", 80)
-    assert moe.workspace_bytes(big) == 256 + 32 * 256 * 4
+    # status word + capacity-scan chunk totals + the bf16 three-term split of W_r that the
+    # tensor-core router reads
+    assert moe.workspace_bytes(big) == 256 + 32 * 256 * 4 + 3 * 256 * 7168 * 2
     fb = moe.forward_workspace_bytes(big)
     assert fb > 20480 * 7168 * 6
 
