@@ -4,9 +4,11 @@
 python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME[:T]] [--impl ours|reference]
 
 A step is one whole forward pass of the layer (route, permute, grouped expert FFN, combine)
-over one batch of synthetic tokens whose inputs already sit in HBM. Steps are timed one by one
-with CUDA events on the launching stream; L2 is flushed (a 256 MB write) before each step,
-outside the timed events. Under torchrun every rank runs its own replica of the workload
+over one batch of synthetic tokens whose inputs already sit in HBM. Each stage is captured once
+as a CUDA graph; a timed step replays the four graphs with CUDA events between them on the
+launching stream. Steps are timed one by one; L2 is flushed (a 256 MB write) before each step,
+outside the timed events. The end-to-end figure (e2e) calls moe_forward eagerly, with the H2D
+copy of the tokens and the D2H copy of the output inside its timed region. Under torchrun every rank runs its own replica of the workload
 (weak scaling, no collective on the data path). Rank 0 prints the line, with the time taken
 as the max over ranks.
 
@@ -208,31 +210,59 @@ class Layer:
                 "expert_count": self._view(b.expert_count, N, torch.int32),
                 "expert_offset": self._view(b.expert_offset, N + 1, torch.int32)}
 
-    def step_stages(self, ev):
-        """One forward as the four stage calls, with events between them (ev: 5 events)."""
+    def stage_calls(self):
+        """The four stage calls of one forward (the calls moe_forward makes), as closures."""
         moe, i, b, dims = self.moe, self.inp, self.b, self.dims
         lib = moe._lib
         d = moe.ctypes.byref(dims)
-        s = moe._stream(None)
         P = moe.ctypes.c_void_p
         ptr = lambda t: P(t.data_ptr()) if t is not None else None
+
+        def route():
+            moe._check(lib.moe_route(d, ptr(i["x"]), ptr(i["w_router"]), ptr(i["logit_bias"]),
+                                     P(b.logits), P(b.topk_idx), P(b.topk_w), P(b.slot),
+                                     P(b.expert_count), P(b.stage_ws), b.stage_ws_bytes,
+                                     moe._stream(None)), "route")
+
+        def permute():
+            moe._check(lib.moe_permute(d, ptr(i["x"]), P(b.topk_idx), P(b.slot), P(b.expert_count),
+                                       P(b.expert_offset), P(b.row_of_pair), P(b.pair_of_row),
+                                       P(b.x_perm), P(b.stage_ws), b.stage_ws_bytes,
+                                       moe._stream(None)), "permute")
+
+        def ffn():
+            moe._check(lib.moe_grouped_ffn(d, P(b.x_perm), P(b.expert_offset), ptr(i["w_gate_up"]),
+                                           ptr(i["w_down"]), P(b.h), P(b.y_perm), P(b.stage_ws),
+                                           b.stage_ws_bytes, moe._stream(None)), "grouped_ffn")
+
+        def combine():
+            moe._check(lib.moe_unpermute_combine(d, P(b.y_perm), P(b.row_of_pair), P(b.topk_w),
+                                                 ptr(i["x"]), ptr(self.out), 0, P(b.stage_ws),
+                                                 b.stage_ws_bytes, moe._stream(None)), "combine")
+        return [route, permute, ffn, combine]
+
+    def capture_stage_graphs(self):
+        """Each stage captured once as a CUDA graph; a replay launches that stage's kernels
+        without host work in between."""
+        self.graphs = []
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for call in self.stage_calls():  # one eager pass on the capture stream first
+                call()
+        torch.cuda.current_stream().wait_stream(s)
+        for call in self.stage_calls():
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                call()
+            self.graphs.append(g)
+
+    def step_stages(self, ev):
+        """One forward: the four stage graphs replayed with events between them (5 events)."""
         ev[0].record()
-        moe._check(lib.moe_route(d, ptr(i["x"]), ptr(i["w_router"]), ptr(i["logit_bias"]),
-                                 P(b.logits), P(b.topk_idx), P(b.topk_w), P(b.slot),
-                                 P(b.expert_count), P(b.stage_ws), b.stage_ws_bytes, s), "route")
-        ev[1].record()
-        moe._check(lib.moe_permute(d, ptr(i["x"]), P(b.topk_idx), P(b.slot), P(b.expert_count),
-                                   P(b.expert_offset), P(b.row_of_pair), P(b.pair_of_row),
-                                   P(b.x_perm), P(b.stage_ws), b.stage_ws_bytes, s), "permute")
-        ev[2].record()
-        moe._check(lib.moe_grouped_ffn(d, P(b.x_perm), P(b.expert_offset), ptr(i["w_gate_up"]),
-                                       ptr(i["w_down"]), P(b.h), P(b.y_perm), P(b.stage_ws),
-                                       b.stage_ws_bytes, s), "grouped_ffn")
-        ev[3].record()
-        moe._check(lib.moe_unpermute_combine(d, P(b.y_perm), P(b.row_of_pair), P(b.topk_w),
-                                             ptr(i["x"]), ptr(self.out), 0, P(b.stage_ws),
-                                             b.stage_ws_bytes, s), "combine")
-        ev[4].record()
+        for n, g in enumerate(self.graphs):
+            g.replay()
+            ev[n + 1].record()
 
     def forward_host(self, x_host, out_host):
         """End to end through the public call: H2D of x, moe_forward, D2H of out."""
@@ -253,6 +283,10 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     shape, T = parse_workload(args.workload)
     layer = Layer(shape, T, device)
+    for call in layer.stage_calls():  # first calls set kernel attributes outside any capture
+        call()
+    torch.cuda.synchronize()
+    layer.capture_stage_graphs()
     flush = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     wev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
@@ -340,7 +374,8 @@ def run_gpu(args, rank, world, local_rank):
                    "active_experts": active,
                    "l2": "flushed before every step (256 MB write outside the timed events); "
                          "expert weights also exceed L2",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "launch": "each stage a captured CUDA graph, events between stages"},
         "stages_ms": {k: round(v_, 4) for k, v_ in stage_ms.items()},
         "roofline": roof,
         "layer_gbs": round(ab["layer"] / (total_ms / args.steps * 1e-3) / 1e9, 1),

@@ -87,11 +87,19 @@ int32_t moe_capacity(double capacity_factor, int32_t T, int32_t n_experts);
 int64_t moe_max_rows(const moe_dims* dims);
 
 /* Bytes of the per-stage workspace `ws` taken by moe_route, moe_route_from_logits,
- * moe_permute, moe_grouped_ffn and moe_unpermute_combine. Its first 256 bytes hold the device
- * status word. The rest is scratch for the capacity scan. Host-only. */
+ * moe_permute, moe_grouped_ffn and moe_unpermute_combine. Host-only. Its regions:
+ *   - the device status word (first 256 bytes);
+ *   - the grouped FFN's per-tile arrival counters for split-K. These are used only when
+ *     R_max <= 256 and must be zero between calls;
+ *   - one region shared by the stages, which run one after another on the stream:
+ *       - the capacity scan's chunk totals;
+ *       - the router's bf16 three-term split of W_r, on the tensor-core path;
+ *       - the grouped FFN's split-K partial tiles.
+ * Zero a workspace once before its first use, with moe_workspace_init or any memset to 0.
+ * Zero it again after a device error. */
 moe_status moe_workspace_bytes(const moe_dims* dims, size_t* bytes);
 
-/* Clear the status word of a fresh workspace (a 4-byte async memset on `stream`). */
+/* Zero a workspace (an async memset of ws_bytes on `stream`). */
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Route: steps 1-3 above.
@@ -136,7 +144,10 @@ moe_status moe_permute(const moe_dims* dims, const uint16_t* x, const int32_t* t
  *   w_down     [N, d_model, F] bf16 (the packed down_proj layout)
  *   h          [R_max, F] bf16 (out)   act(x_perm W_gu^T) in fp32, rounded once to bf16
  *   y_perm     [R_max, d_model] fp32 (out)  h W_d^T with fp32 accumulation
- * Rows >= R of h and y_perm are not written. Experts with no kept rows cost nothing. */
+ * Rows >= R of h and y_perm are not written. Experts with no kept rows cost nothing.
+ * Decode-sized batches (R_max <= 256) may split the K dimension of a GEMM across CTAs to use
+ * every SM. Each split's fp32 partial tile goes to the workspace. The last split to finish
+ * a tile adds the partials in a fixed order, so results are deterministic. */
 moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
                            const int32_t* expert_offset, const uint16_t* w_gate_up,
                            const uint16_t* w_down, uint16_t* h, float* y_perm, void* ws,

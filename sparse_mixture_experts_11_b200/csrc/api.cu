@@ -88,13 +88,31 @@ size_t split_scratch_bytes(const moe_dims* d) {
              : 0;
 }
 
+moe::FfnScratchPlan ffn_plan(const moe_dims* d) {
+  return moe::ffn_scratch_plan(d->n_experts, d->d_model, d->d_ff, d->act, max_rows(d));
+}
+
+// Per-stage workspace:
+//   [status word, 256 B][grouped-FFN tile counters, zero between calls]
+//   [shared region: routing scratch (capacity-scan chunk totals, router weight split) or,
+//    later on the stream, the grouped FFN's split-K partial tiles]
+size_t counters_bytes(const moe_dims* d) { return round_up(ffn_plan(d).counter_bytes, 256); }
+
+size_t shared_region_bytes(const moe_dims* d) {
+  return std::max(slot_scratch_bytes(d) + split_scratch_bytes(d), round_up(ffn_plan(d).part_bytes, 256));
+}
+
 size_t stage_ws_bytes(const moe_dims* d) {
-  return moe::kStatusBytes + slot_scratch_bytes(d) + split_scratch_bytes(d);
+  return moe::kStatusBytes + counters_bytes(d) + shared_region_bytes(d);
+}
+
+char* shared_region_of(const moe_dims* d, void* ws) {
+  return static_cast<char*>(ws) + moe::kStatusBytes + counters_bytes(d);
 }
 
 uint16_t* split_scratch_of(const moe_dims* d, void* ws) {
   if (split_scratch_bytes(d) == 0) return nullptr;
-  return reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + moe::kStatusBytes + slot_scratch_bytes(d));
+  return reinterpret_cast<uint16_t*>(shared_region_of(d, ws) + slot_scratch_bytes(d));
 }
 
 int* status_of(void* ws) { return static_cast<int*>(ws); }
@@ -104,7 +122,7 @@ moe_status launch_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
 // Shared by moe_route and moe_route_from_logits once top-k is written.
 moe_status route_slots(const moe_dims* d, int32_t* topk_idx, int32_t* slot, int32_t* expert_count,
                        void* ws, cudaStream_t s) {
-  int32_t* scratch = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + moe::kStatusBytes);
+  int32_t* scratch = reinterpret_cast<int32_t*>(shared_region_of(d, ws));
   const int cap = std::min(d->capacity, d->T);
   return launch_status(moe::launch_capacity_slots(topk_idx, slot, expert_count, scratch, d->T,
                                                   d->n_experts, d->top_k, cap, s));
@@ -136,7 +154,7 @@ moe_status moe_workspace_bytes(const moe_dims* dims, size_t* bytes) {
 
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (ws == nullptr || ws_bytes < moe::kStatusBytes) return MOE_ERR_INVALID;
-  return launch_status(cudaMemsetAsync(ws, 0, sizeof(int32_t), as_stream(stream)));
+  return launch_status(cudaMemsetAsync(ws, 0, ws_bytes, as_stream(stream)));
 }
 
 moe_status moe_route(const moe_dims* dims, const uint16_t* x, const float* w_router,
@@ -234,6 +252,11 @@ moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
   a.r_max = rmax;
   a.status = status_of(ws);
   a.timeout_ns = moe::kDefaultWaitTimeoutNs;
+  const moe::FfnScratchPlan plan = ffn_plan(dims);
+  if (plan.max_splits1 > 1 || plan.max_splits2 > 1) {
+    a.part = reinterpret_cast<float*>(shared_region_of(dims, ws));
+    a.tile_counters = reinterpret_cast<int*>(static_cast<char*>(ws) + moe::kStatusBytes);
+  }
   return launch_status(moe::launch_grouped_ffn(a, as_stream(stream)));
 }
 

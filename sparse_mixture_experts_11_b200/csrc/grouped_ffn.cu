@@ -59,6 +59,14 @@ struct GemmParams {
   int* status;
   uint64_t timeout_ns;
   int weight_policy;  // 0 evict_normal, 1 evict_first
+  // split-K (decode-sized batches): up to max_splits units per tile, each over a slice of K.
+  // Every unit stores its fp32 partial tile into part[split][row][col]; the CTA whose unit
+  // completes a tile last (per-tile arrival counter) adds the partials in order of split and
+  // writes the tile's output. The counters are zero between calls.
+  int max_splits;
+  float* part;
+  int part_ld;          // columns of a partial row: 2F (gate | up), F, or d
+  int* tile_counters;
 };
 
 constexpr int pow2_at_least(int v) {
@@ -123,9 +131,90 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, int N, int bn_out,
   return c;
 }
 
+// Number of K slices per tile. With equal units dealt out in turn to `grid` CTAs, the busiest
+// CTA runs ceil(units / grid) units of (num_kb / splits + kUnitOverheadKb) k-block times; the
+// count minimising that wins, a larger one only when it is at least 5 % faster. Units keep at
+// least 2 k blocks. The same pure function of (tiles, grid) on every CTA, so all agree.
+constexpr float kUnitOverheadKb = 2.0f;  // epilogue, partial round trip and pipeline refill
+
+__device__ __forceinline__ int choose_splits(int tiles, int grid, int num_kb, int max_splits) {
+  if (max_splits <= 1 || tiles <= 0) return 1;
+  auto cost = [=](int sp) {
+    const int waves = (tiles * sp + grid - 1) / grid;
+    return static_cast<float>(waves) * (static_cast<float>(num_kb) / sp + kUnitOverheadKb);
+  };
+  int best = 1;
+  float best_cost = cost(1);
+  for (int sp = 2; sp <= max_splits && num_kb / sp >= 2; ++sp) {
+    const float c = cost(sp);
+    if (c < 0.95f * best_cost) {
+      best = sp;
+      best_cost = c;
+    }
+  }
+  return best;
+}
+
+// Barrier of the 128 epilogue threads on a reusable mbarrier (count 128), bounded like every
+// other wait so that no thread can be left waiting for a warp that gave up.
+__device__ __forceinline__ bool epilogue_sync(uint32_t bar, uint32_t& phase, uint64_t timeout_ns,
+                                              const volatile int* abort) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase, timeout_ns, abort);
+  phase ^= 1u;
+  return ok;
+}
+
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 __device__ __forceinline__ float gelu_f(float z) {
   return 0.5f * z * (1.0f + erff(z * 0.7071067811865476f));
+}
+
+__device__ __forceinline__ void store_f32x16(float* dst, const float (&a)[16]) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = make_float4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+}
+
+// Final values of 4 consecutive output columns of one row (same rules as store_final16).
+template <int EPI>
+__device__ __forceinline__ void store_final4(const GemmParams& p, int64_t row, int col,
+                                             const float4& a, const float4& b) {
+  if (EPI == EPI_STORE_F32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ld_out + col) = a;
+  } else {
+    uint2 packed;
+    if (EPI == EPI_SWIGLU) {
+      packed.x = pack_bf16x2(silu_f(a.x) * b.x, silu_f(a.y) * b.y);
+      packed.y = pack_bf16x2(silu_f(a.z) * b.z, silu_f(a.w) * b.w);
+    } else {
+      packed.x = pack_bf16x2(gelu_f(a.x), gelu_f(a.y));
+      packed.y = pack_bf16x2(gelu_f(a.z), gelu_f(a.w));
+    }
+    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + row * p.ld_out + col) = packed;
+  }
+}
+
+// Final values of 16 consecutive output columns of one row: SwiGLU h = silu(g) * u and GELU
+// h = gelu(z) rounded once to bf16; the down projection stored as fp32.
+template <int EPI>
+__device__ __forceinline__ void store_final16(const GemmParams& p, int64_t row, int col,
+                                              const float (&a)[16], const float (&b)[16]) {
+  if (EPI == EPI_STORE_F32) {
+    store_f32x16(static_cast<float*>(p.out) + row * p.ld_out + col, a);
+  } else {
+    uint32_t packed[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (EPI == EPI_SWIGLU)
+        packed[i] = pack_bf16x2(silu_f(a[2 * i]) * b[2 * i], silu_f(a[2 * i + 1]) * b[2 * i + 1]);
+      else
+        packed[i] = pack_bf16x2(gelu_f(a[2 * i]), gelu_f(a[2 * i + 1]));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ld_out + col);
+    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+  }
 }
 
 template <int EPI, int BN_OUT>
@@ -139,10 +228,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t tfull_bar[2];
   __shared__ __align__(8) uint64_t tempty_bar[2];
   __shared__ __align__(8) uint64_t done_bar;
+  __shared__ __align__(8) uint64_t epi_bar;
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int s_abort;
   __shared__ int s_tile_start[257];
   __shared__ int s_off[257];
+  __shared__ int s_splits;
+  __shared__ int s_fixup;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -161,6 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&tempty_bar[b]), kEpiThreads);
     }
     mbar_init(smem_u32(&done_bar), 1);
+    mbar_init(smem_u32(&epi_bar), kEpiThreads);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -206,7 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         run += cnt[i];
       }
     }
-    if (lane == 31) s_tile_start[N] = incl;
+    if (lane == 31) {
+      s_tile_start[N] = incl;
+      s_splits = choose_splits(incl, gridDim.x, p.num_kb, p.max_splits);
+    }
     if (bad) report_error(p.status, MOE_ERR_BOUNDS);  // such an expert gets no tiles
   }
   tc_fence_before_sync();
@@ -215,6 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t tmem_base = s_tmem_base;
   const int total_tiles = s_tile_start[N];
+  const int splits = s_splits;
+  const int total_units = total_tiles * splits;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -223,9 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_b = make_policy(p.weight_policy);
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      for (int unit = blockIdx.x; ok && unit < total_units; unit += gridDim.x) {
+        const int tile = unit / splits, sp = unit - tile * splits;
         const TileCoord c = decode_tile(tile, N, BN_OUT, s_tile_start, s_off);
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        const int kb0 = sp * p.num_kb / splits, kb1 = (sp + 1) * p.num_kb / splits;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
           if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, p.timeout_ns, &s_abort)) {
@@ -260,7 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0, tc = 0;
       bool ok = true;
       bool issued = false;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++tc) {
+      for (int unit = blockIdx.x; ok && unit < total_units; unit += gridDim.x, ++tc) {
+        const int sp = unit % splits;
+        const int kb0 = sp * p.num_kb / splits, kb1 = (sp + 1) * p.num_kb / splits;
         const int buf = tc & 1;
         const uint32_t tph = (tc >> 1) & 1;
         if (!mbar_wait(smem_u32(&tempty_bar[buf]), tph ^ 1u, p.timeout_ns, &s_abort)) {
@@ -269,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::UMMA_N);
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
           if (!mbar_wait(smem_u32(&full_bar[s]), ph, p.timeout_ns, &s_abort)) {
@@ -282,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             tc_mma_f16(d_tmem, smem_desc_k_sw128(a_base + kk * 32), smem_desc_k_sw128(b_base + kk * 32),
-                       idesc, (kb | kk) != 0 ? 1u : 0u);
+                       idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
           }
           issued = true;
           tc_commit(smem_u32(&empty_bar[s]));
@@ -304,8 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int r_local = q * 32 + lane;
     int tc = 0;
+    uint32_t epi_phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tc) {
+    for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x, ++tc) {
+      const int tile = unit / splits, sp = unit - tile * splits;
       const TileCoord c = decode_tile(tile, N, BN_OUT, s_tile_start, s_off);
       const int buf = tc & 1;
       const uint32_t tph = (tc >> 1) & 1;
@@ -322,46 +426,76 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int cc = 0; cc < BN_OUT; cc += 16) {
         if (c.n0 + cc >= p.n_out) break;  // warp-uniform: ragged last n-tile
-        if (EPI == EPI_STORE_F32) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_row + cc, v);
+        float a[16], b[16];
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(t_row + cc, v);
+        if (EPI == EPI_SWIGLU) {
+          uint32_t u[16];
+          tmem_ld_32x32b_x16(t_row + BN_OUT + cc, u);
           tmem_ld_wait();
-          if (row_ok) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ld_out + c.n0 + cc);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-          }
+          for (int i = 0; i < 16; ++i) b[i] = __uint_as_float(u[i]);
         } else {
-          uint32_t g[16];
-          uint32_t packed[8];
-          tmem_ld_32x32b_x16(t_row + cc, g);
-          if (EPI == EPI_SWIGLU) {
-            uint32_t u[16];
-            tmem_ld_32x32b_x16(t_row + BN_OUT + cc, u);
-            tmem_ld_wait();
+          tmem_ld_wait();
+        }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-              const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-              packed[i] = pack_bf16x2(h0, h1);
-            }
-          } else {
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              packed[i] = pack_bf16x2(gelu_f(__uint_as_float(g[2 * i])), gelu_f(__uint_as_float(g[2 * i + 1])));
-          }
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ld_out + c.n0 + cc);
-            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-          }
+        for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(v[i]);
+        if (!row_ok) continue;
+        if (splits == 1) {
+          store_final16<EPI>(p, row, c.n0 + cc, a, b);
+        } else {  // this unit's partial tile
+          float* dst = p.part + (static_cast<int64_t>(sp) * p.r_max + row) * p.part_ld + c.n0 + cc;
+          store_f32x16(dst, a);
+          if (EPI == EPI_SWIGLU) store_f32x16(dst + p.n_out, b);
         }
       }
       tc_fence_before_sync();
-      mbar_arrive(smem_u32(&tempty_bar[buf]));
+      mbar_arrive(smem_u32(&tempty_bar[buf]));  // TMEM buffer free for the next unit
+
+      if (splits > 1) {
+        // publish this partial; the unit that completes the tile adds all partials in order
+        __threadfence();
+        if (!__all_sync(0xffffffffu, epilogue_sync(smem_u32(&epi_bar), epi_phase, p.timeout_ns, &s_abort))) {
+          ok = false;
+          break;
+        }
+        if (threadIdx.x == 64) {
+          const int prev = atomicAdd(p.tile_counters + tile, 1);
+          const int last = prev == splits - 1;
+          if (last) p.tile_counters[tile] = 0;  // every unit of the tile has arrived
+          s_fixup = last;
+        }
+        if (!__all_sync(0xffffffffu, epilogue_sync(smem_u32(&epi_bar), epi_phase, p.timeout_ns, &s_abort))) {
+          ok = false;
+          break;
+        }
+        if (s_fixup) {
+          // All 128 epilogue threads share the reduction: item i is (tile row i / G, float4
+          // column group i % G), so neighbouring threads touch neighbouring columns.
+          __threadfence();
+          constexpr int G = BN_OUT / 4;
+          const int cols = min(BN_OUT, p.n_out - c.n0);
+          const int et = threadIdx.x - 64;  // 0..127
+          for (int i = et; i < c.rows * G; i += kEpiThreads) {
+            const int r = i / G, c4 = (i - r * G) * 4;
+            if (c4 >= cols) continue;
+            const int64_t orow = static_cast<int64_t>(c.m0) + r;
+            const float* src = p.part + orow * p.part_ld + c.n0 + c4;
+            const int64_t sstride = p.r_max * p.part_ld;
+            float4 ga = make_float4(0.f, 0.f, 0.f, 0.f), ub = ga;
+#pragma unroll 4
+            for (int s2 = 0; s2 < splits; ++s2) {  // fixed order: deterministic sums
+              const float4 v = __ldcg(reinterpret_cast<const float4*>(src + s2 * sstride));
+              ga.x += v.x; ga.y += v.y; ga.z += v.z; ga.w += v.w;
+              if (EPI == EPI_SWIGLU) {
+                const float4 u = __ldcg(reinterpret_cast<const float4*>(src + s2 * sstride + p.n_out));
+                ub.x += u.x; ub.y += u.y; ub.z += u.z; ub.w += u.w;
+              }
+            }
+            store_final4<EPI>(p, orow, c.n0 + c4, ga, ub);
+          }
+        }
+      }
     }
     if (!ok) {
       s_abort = 1;
@@ -433,10 +567,26 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmP
   return cudaGetLastError();
 }
 
-int grid_for(int64_t r_max, int N, int n_tiles_n, int sm_count) {
+int64_t tiles_upper_bound(int64_t r_max, int N, int n_tiles_n) {
+  // sum_e ceil(m_e / BM) <= ceil(R / BM) + (experts with rows)
   const int64_t m_tiles_ub = (r_max + BM - 1) / BM + std::min<int64_t>(N, r_max);
-  const int64_t tiles_ub = m_tiles_ub * n_tiles_n;
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles_ub, sm_count)));
+  return m_tiles_ub * n_tiles_n;
+}
+
+int grid_for(int64_t r_max, int N, int n_tiles_n, int sm_count, int max_splits) {
+  const int64_t units_ub = tiles_upper_bound(r_max, N, n_tiles_n) * max_splits;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units_ub, sm_count)));
+}
+
+constexpr int64_t kSplitRowsMax = 256;                 // split-K only for decode-sized batches
+constexpr size_t kPartBudget = size_t(64) << 20;       // bytes of partial tiles per GEMM
+constexpr int kMaxSplits = 16;
+
+int max_splits_for(int64_t r_max, int num_kb, int part_ld) {
+  if (r_max > kSplitRowsMax) return 1;
+  int ms = std::min(kMaxSplits, num_kb / 2);
+  while (ms > 1 && static_cast<size_t>(ms) * r_max * part_ld * 4 > kPartBudget) --ms;
+  return std::max(1, ms);
 }
 
 constexpr int kGuBnSwiglu = 128;  // output columns per tile of the gate/up GEMM (UMMA N = 256)
@@ -444,6 +594,29 @@ constexpr int kGuBnGelu = 256;
 constexpr int kDnBn = 256;        // output columns per tile of the down GEMM
 
 }  // namespace
+
+FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max) {
+  FfnScratchPlan pl{1, 1, 0, 0};
+  if (r_max <= 0) return pl;
+  const bool swiglu = act == MOE_ACT_SWIGLU;
+  const int bn1 = swiglu ? kGuBnSwiglu : kGuBnGelu;
+  const int ld1 = swiglu ? 2 * F : F;
+  pl.max_splits1 = max_splits_for(r_max, d / BK, ld1);
+  pl.max_splits2 = max_splits_for(r_max, F / BK, d);
+  size_t part = 0;
+  int64_t tiles = 0;
+  if (pl.max_splits1 > 1) {
+    part = std::max(part, static_cast<size_t>(pl.max_splits1) * r_max * ld1 * 4);
+    tiles = std::max(tiles, tiles_upper_bound(r_max, N, (F + bn1 - 1) / bn1));
+  }
+  if (pl.max_splits2 > 1) {
+    part = std::max(part, static_cast<size_t>(pl.max_splits2) * r_max * d * 4);
+    tiles = std::max(tiles, tiles_upper_bound(r_max, N, (d + kDnBn - 1) / kDnBn));
+  }
+  pl.part_bytes = part;
+  pl.counter_bytes = static_cast<size_t>(tiles) * sizeof(int);
+  return pl;
+}
 
 cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   if (a.r_max <= 0) return cudaSuccess;
@@ -502,7 +675,13 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   g1.status = a.status;
   g1.timeout_ns = a.timeout_ns;
   g1.weight_policy = wpol;
-  const int grid1 = grid_for(a.r_max, a.N, g1.n_tiles_n, di.sm_count);
+  const FfnScratchPlan plan = ffn_scratch_plan(a.N, a.d, a.F, a.act, a.r_max);
+  const bool can_split = a.part != nullptr && a.tile_counters != nullptr;
+  g1.max_splits = can_split ? plan.max_splits1 : 1;
+  g1.part = a.part;
+  g1.part_ld = swiglu ? 2 * a.F : a.F;
+  g1.tile_counters = a.tile_counters;
+  const int grid1 = grid_for(a.r_max, a.N, g1.n_tiles_n, di.sm_count, g1.max_splits);
   err = swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu>(mA1, mB1, g1, grid1, s)
                : launch_one<EPI_GELU, kGuBnGelu>(mA1, mB1, g1, grid1, s);
   if (err != cudaSuccess) return err;
@@ -513,7 +692,9 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   g2.n_out = a.d;
   g2.n_tiles_n = (a.d + kDnBn - 1) / kDnBn;
   g2.num_kb = a.F / BK;
-  const int grid2 = grid_for(a.r_max, a.N, g2.n_tiles_n, di.sm_count);
+  g2.max_splits = can_split ? plan.max_splits2 : 1;
+  g2.part_ld = a.d;
+  const int grid2 = grid_for(a.r_max, a.N, g2.n_tiles_n, di.sm_count, g2.max_splits);
   return launch_one<EPI_STORE_F32, kDnBn>(mA2, mB2, g2, grid2, s);
 }
 

@@ -60,6 +60,16 @@ cudaError_t launch_combine(const float* y_perm, const int32_t* row_of_pair, cons
                            int64_t r_max, int* status, cudaStream_t s);
 
 // grouped expert GEMMs on tcgen05
+//
+// Scratch of the grouped FFN for split-K, used only for decode-sized batches (R_max <= 256):
+// fp32 partial tiles and one arrival counter per tile (zero between calls).
+struct FfnScratchPlan {
+  int max_splits1, max_splits2;  // gate/up GEMM, down GEMM (1 = no split)
+  size_t part_bytes;             // partial tiles (shared by the two GEMMs, which run in turn)
+  size_t counter_bytes;          // per-tile arrival counters
+};
+FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max);
+
 struct GroupedFfnArgs {
   const uint16_t* x_perm;
   const int32_t* expert_offset;
@@ -71,6 +81,8 @@ struct GroupedFfnArgs {
   int64_t r_max;
   int* status;
   uint64_t timeout_ns;
+  float* part;          // ffn_scratch_plan().part_bytes, or null when no split is planned
+  int* tile_counters;   // ffn_scratch_plan().counter_bytes, zeroed once before first use
 };
 cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s);
 

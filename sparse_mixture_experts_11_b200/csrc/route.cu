@@ -90,38 +90,60 @@ __device__ __forceinline__ void warp_topk_write(const float (&val)[EPT], int N, 
 }
 
 // ------------------------------------------------------------------ router (SIMT fp32)
-// One block per token for small batches: warp w computes the logits of experts w, w+8, ...,
-// lanes splitting d (float4 of W_r and 4 bf16 of x per step), then a shuffle-tree sum; then
-// warp 0 takes the top-k of the token's N logits.
+// One block of 1024 threads per token for small batches. g warps share each expert's dot
+// product (g = the largest power of two with g * N <= 32, at least 1), each taking every g-th
+// 128-element slice of d with
+// float4 loads of W_r and 4-bf16 loads of x; experts beyond 32 / g take further passes. Warp
+// partial sums meet in shared memory and are added in a fixed order, then warp 0 takes the
+// token's top-k.
+constexpr int kTokThreads = 1024;
+constexpr int kTokWarps = kTokThreads / 32;
+
 template <int EPT>
-__global__ void __launch_bounds__(256) router_token_kernel(
+__global__ void __launch_bounds__(kTokThreads) router_token_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias,
     float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int T,
     int d, int N, int k) {
+  __shared__ float s_part[kTokWarps][EPT];  // [warp][pass]: at most EPT passes of 32 experts
   __shared__ float s_logit[EPT * 32];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint16_t* xr = x + static_cast<int64_t>(t) * d;
-  for (int e = warp; e < N; e += 8) {
-    const float* wr = w + static_cast<int64_t>(e) * d;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 4
-    for (int i = lane * 4; i < d; i += 128) {
-      const float4 wv = __ldg(reinterpret_cast<const float4*>(wr + i));
-      const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + i));
-      a0 = fmaf(__uint_as_float(xv.x << 16), wv.x, a0);
-      a1 = fmaf(__uint_as_float(xv.x & 0xffff0000u), wv.y, a1);
-      a2 = fmaf(__uint_as_float(xv.y << 16), wv.z, a2);
-      a3 = fmaf(__uint_as_float(xv.y & 0xffff0000u), wv.w, a3);
-    }
-    float acc = (a0 + a1) + (a2 + a3);
+  int g = 1;  // warps per expert
+  while (g * 2 * N <= kTokWarps) g *= 2;
+  const int experts_per_pass = kTokWarps / g;
+  const int part = warp % g;
+  int pass = 0;
+  for (int e0 = 0; e0 < N; e0 += experts_per_pass, ++pass) {
+    const int e = e0 + warp / g;
+    float acc = 0.f;
+    if (e < N) {
+      const float* wr = w + static_cast<int64_t>(e) * d;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+      for (int i = (part * 32 + lane) * 4; i < d; i += 128 * g) {
+        const float4 wv = __ldg(reinterpret_cast<const float4*>(wr + i));
+        const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + i));
+        a0 = fmaf(__uint_as_float(xv.x << 16), wv.x, a0);
+        a1 = fmaf(__uint_as_float(xv.x & 0xffff0000u), wv.y, a1);
+        a2 = fmaf(__uint_as_float(xv.y << 16), wv.z, a2);
+        a3 = fmaf(__uint_as_float(xv.y & 0xffff0000u), wv.w, a3);
+      }
+      acc = (a0 + a1) + (a2 + a3);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-    if (lane == 0) {
-      const float L = acc + (bias != nullptr ? bias[e] : 0.f);
-      s_logit[e] = L;
-      logits[static_cast<int64_t>(t) * N + e] = L;
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
     }
+    if (lane == 0) s_part[warp][pass] = acc;
+  }
+  __syncthreads();
+  // the g partial sums of each expert, added in order of part
+  for (int e = threadIdx.x; e < N; e += kTokThreads) {
+    const int p = e / experts_per_pass, wbase = (e % experts_per_pass) * g;
+    float L = 0.f;
+    for (int q = 0; q < g; ++q) L += s_part[wbase + q][p];
+    if (bias != nullptr) L += bias[e];
+    s_logit[e] = L;
+    logits[static_cast<int64_t>(t) * N + e] = L;
   }
   __syncthreads();
   if (warp == 0) {
@@ -280,13 +302,13 @@ cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const f
     return launch_router_tc(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k,
                             split_scratch, status, timeout_ns, s);
   if (N <= 32)
-    router_token_kernel<1><<<T, 256, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+    router_token_kernel<1><<<T, kTokThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
   else if (N <= 64)
-    router_token_kernel<2><<<T, 256, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+    router_token_kernel<2><<<T, kTokThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
   else if (N <= 128)
-    router_token_kernel<4><<<T, 256, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+    router_token_kernel<4><<<T, kTokThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
   else
-    router_token_kernel<8><<<T, 256, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
+    router_token_kernel<8><<<T, kTokThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
   return cudaGetLastError();
 }
 

@@ -47,7 +47,9 @@ def test_max_rows():
 
 def test_workspace_sizes():
     small = moe.make_dims(64, 128, 8, 2, 256, "swiglu", 10)
-    assert moe.workspace_bytes(small) == 256          # one capacity chunk: status word only
+    # status word + split-K tile counters (9 tiles of the down GEMM, rounded to 256 B) +
+    # split-K partials of the down GEMM (2 splits x 80 rows x 128 fp32 columns)
+    assert moe.workspace_bytes(small) == 256 + 256 + 2 * 80 * 128 * 4
     big = moe.make_dims(16384, 7168, 256, 8, 2048, "swiglu", 80)
     # status word + capacity-scan chunk totals + the bf16 three-term split of W_r that the
     # tensor-core router reads

@@ -20,6 +20,11 @@ SMALL_CASES = [
     ("single_token", 1, 256, 8, 2, 256, "swiglu", None, None),
     ("k_equals_n", 40, 64, 4, 4, 64, "swiglu", None, None),
     ("heavy_drop", 200, 128, 8, 2, 128, "swiglu", 0.25, 1.1),
+    # decode-sized batches whose GEMMs split K across CTAs (last split adds the partials)
+    ("splitk_decode_swiglu", 3, 512, 8, 2, 1024, "swiglu", None, None),
+    ("splitk_decode_gelu", 5, 256, 16, 1, 2048, "gelu", None, None),
+    ("splitk_decode_deep_k", 2, 4096, 8, 2, 2048, "swiglu", None, None),
+    ("splitk_decode_ragged_n", 7, 2880, 32, 4, 2880, "swiglu", None, None),
     # large enough that the router runs on tensor cores (T*N*d*4 bytes > 256 MiB);
     # expert counts padded to 16, 32, 64, 128 (N=100) and 256 tensor-core columns
     ("tc_router_n8_bias", 20000, 512, 8, 2, 128, "swiglu", 1.25, 1.1),
