@@ -200,15 +200,21 @@ class Layer:
         return self.fws[off:off + nbytes].view(dtype)
 
     def views(self):
+        """Tensor views of the intermediates inside the forward workspace."""
         s = self.shape
-        T, k, N = self.T, s.top_k, s.n_experts
+        T, k, N, d, F, R = self.T, s.top_k, s.n_experts, s.d_model, s.d_ff, self.R_max
         b = self.b
         return {"logits": self._view(b.logits, T * N, torch.float32).view(T, N),
                 "topk_idx": self._view(b.topk_idx, T * k, torch.int32).view(T, k),
                 "topk_w": self._view(b.topk_w, T * k, torch.float32).view(T, k),
                 "slot": self._view(b.slot, T * k, torch.int32).view(T, k),
                 "expert_count": self._view(b.expert_count, N, torch.int32),
-                "expert_offset": self._view(b.expert_offset, N + 1, torch.int32)}
+                "expert_offset": self._view(b.expert_offset, N + 1, torch.int32),
+                "row_of_pair": self._view(b.row_of_pair, T * k, torch.int32).view(T, k),
+                "pair_of_row": self._view(b.pair_of_row, R, torch.int32),
+                "x_perm": self._view(b.x_perm, R * d, torch.bfloat16).view(R, d),
+                "y_perm": self._view(b.y_perm, R * d, torch.float32).view(R, d),
+                "stage_ws": self._view(b.stage_ws, b.stage_ws_bytes, torch.uint8)}
 
     def stage_calls(self):
         """The four stage calls of one forward (the calls moe_forward makes), as closures."""
@@ -273,6 +279,21 @@ class Layer:
         out_host.copy_(self.out, non_blocking=True)
 
 
+def reduce_max(values, world: int, device) -> list:
+    """Max over ranks of each timed duration (a no-op on one rank). Every rank calls it at the
+    same point, so the collective sequence is identical on all ranks."""
+    if world <= 1:
+        return list(values)
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def tokens_per_second(tokens_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * steps * world / (max_ms * 1e-3)
+
+
 def flush_l2(buf):
     buf.add_(1)  # 256 MB read-modify-write, larger than the 126 MB L2
 
@@ -334,10 +355,7 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    times = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    total_ms, e2e_ms = times.tolist()
+    total_ms, e2e_ms = reduce_max([total_ms, e2e_ms], world, device)
 
     v = layer.views()
     counts = v["expert_count"].cpu()
@@ -362,7 +380,7 @@ def run_gpu(args, rank, world, local_rank):
                 "kernel": "moe_grouped_ffn (gate/up + down GEMM launches)",
                 "per_launch": f"{ab['ffn']} B", "peak_source": peaks["source"] + " copy"}
 
-    value = T * args.steps * world / (total_ms * 1e-3)
+    value = tokens_per_second(T, args.steps, world, total_ms)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
@@ -380,7 +398,7 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": roof,
         "layer_gbs": round(ab["layer"] / (total_ms / args.steps * 1e-3) / 1e9, 1),
         "ffn_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 2),
-        "e2e": {"value": round(T * args.steps * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(tokens_per_second(T, args.steps, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * shape.d_model * 2,
                 "d2h_bytes_per_step": T * shape.d_model * 2},
         "gpu_launches": launches_per_step(T, shape.top_k, layer.R_max) * args.steps,

@@ -40,6 +40,13 @@ __device__ __forceinline__ void block_offsets_256(const int32_t* __restrict__ co
   __syncthreads();
 }
 
+// Block (token t, chunk c): the block's first warp turns token t's k (expert, slot) pairs
+// into rows; the token's chunk-0 block also records row_of_pair / pair_of_row. Then each
+// thread copies one 16-byte vector of x[t] (chunk c) into every kept row. Many blocks per
+// token keep small batches from being latency-bound; expert offsets are rebuilt per block
+// from the N <= 256 kept counts.
+constexpr int kVecPerBlock = 256;  // 16-byte vectors per block (4 KB of a bf16 row)
+
 __global__ void __launch_bounds__(256) permute_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx,
     const int32_t* __restrict__ slot, const int32_t* __restrict__ expert_count,
@@ -48,111 +55,126 @@ __global__ void __launch_bounds__(256) permute_kernel(
     int64_t r_max, int* status) {
   __shared__ int s_off[257];
   __shared__ int s_warp[8];
+  __shared__ int s_rows[8];
   block_offsets_256(expert_count, N, s_off, s_warp);
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i <= N; i += blockDim.x) expert_offset[i] = s_off[i];
 
-  const int lane = threadIdx.x & 31;
-  const int warps = blockDim.x >> 5;
   const int nv = d / 8;  // 16-byte vectors per row
-  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
-    int row = -1;
-    if (lane < k) {
-      const int64_t q = static_cast<int64_t>(t) * k + lane;
-      const int s = slot[q];
-      const int e = topk_idx[q];
-      if (s >= 0 && e >= 0 && e < N) {
-        row = s_off[e] + s;
-        if (row >= s_off[e + 1] || row >= r_max) {
-          report_error(status, MOE_ERR_BOUNDS);
-          row = -1;
+  const int chunks = (nv + kVecPerBlock - 1) / kVecPerBlock;
+  const int64_t items = static_cast<int64_t>(T) * chunks;
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    const int t = static_cast<int>(item / chunks);
+    const int c = static_cast<int>(item - static_cast<int64_t>(t) * chunks);
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      int row = -1;
+      if (lane < k) {
+        const int64_t q = static_cast<int64_t>(t) * k + lane;
+        const int sl = slot[q];
+        const int e = topk_idx[q];
+        if (sl >= 0 && e >= 0 && e < N) {
+          row = s_off[e] + sl;
+          if (row >= s_off[e + 1] || row >= r_max) {
+            report_error(status, MOE_ERR_BOUNDS);
+            row = -1;
+          }
         }
-      }
-      row_of_pair[q] = row;
-      if (row >= 0) pair_of_row[row] = static_cast<int32_t>(q);
-    }
-    int rows[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(kFull, row, j);
-    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * d);
-    for (int c = lane; c < nv; c += 32) {
-      const uint4 v = src[c];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < k && rows[j] >= 0)
-          reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(rows[j]) * d)[c] = v;
+        if (c == 0) {
+          row_of_pair[q] = row;
+          if (row >= 0) pair_of_row[row] = static_cast<int32_t>(q);
+        }
+        s_rows[lane] = row;
       }
     }
+    __syncthreads();
+    const int v = c * kVecPerBlock + threadIdx.x;
+    if (v < nv) {
+      const uint4 val = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * d)[v];
+      for (int j = 0; j < k; ++j) {
+        const int row = s_rows[j];
+        if (row >= 0) reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(row) * d)[v] = val;
+      }
+    }
+    __syncthreads();
   }
 }
+
+// Block (token t, chunk c of 1024 columns): thread i handles 4 columns (one float4 of each kept
+// expert row of y_perm and 4 bf16 of the residual). Weights and rows of the token come from its
+// k pairs.
+constexpr int kColsPerBlock = 1024;
 
 __global__ void __launch_bounds__(256) combine_kernel(
     const float* __restrict__ y, const int32_t* __restrict__ row_of_pair,
     const float* __restrict__ topk_w, const uint16_t* residual, void* out, int out_f32, int T,
     int d, int k, int64_t r_max, int* status) {
-  const int lane = threadIdx.x & 31;
-  const int warps = blockDim.x >> 5;
+  __shared__ int s_rows[8];
+  __shared__ float s_w[8];
+  __shared__ int s_any;
   const int nq = d / 4;  // groups of 4 columns
-  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
-    int row = -1;
-    float w = 0.f;
-    if (lane < k) {
-      const int64_t q = static_cast<int64_t>(t) * k + lane;
-      row = row_of_pair[q];
-      w = topk_w[q];
-      if (row >= r_max) {
-        report_error(status, MOE_ERR_BOUNDS);
-        row = -1;
+  const int chunks = (d + kColsPerBlock - 1) / kColsPerBlock;
+  const int64_t items = static_cast<int64_t>(T) * chunks;
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    const int t = static_cast<int>(item / chunks);
+    const int c = static_cast<int>(item - static_cast<int64_t>(t) * chunks);
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      int row = -1;
+      float w = 0.f;
+      if (lane < k) {
+        const int64_t q = static_cast<int64_t>(t) * k + lane;
+        row = row_of_pair[q];
+        w = topk_w[q];
+        if (row >= r_max) {
+          report_error(status, MOE_ERR_BOUNDS);
+          row = -1;
+        }
+        s_rows[lane] = row;
+        s_w[lane] = w;
       }
+      const unsigned any = __ballot_sync(kFull, row >= 0);
+      if (lane == 0) s_any = any != 0;
     }
-    const bool any_kept = __ballot_sync(kFull, row >= 0) != 0;
-    int rows[8];
-    float ws[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      rows[j] = __shfl_sync(kFull, row, j);
-      ws[j] = __shfl_sync(kFull, w, j);
-    }
-    const uint2* res = residual ? reinterpret_cast<const uint2*>(residual + static_cast<int64_t>(t) * d) : nullptr;
-    for (int c = lane; c < nq; c += 32) {
+    __syncthreads();
+    const int qi = c * (kColsPerBlock / 4) + threadIdx.x;
+    if (qi < nq) {
       uint2 rbits = make_uint2(0u, 0u);
-      if (res) rbits = res[c];
-      if (!any_kept) {  // residual passes through unchanged
+      if (residual != nullptr) rbits = reinterpret_cast<const uint2*>(residual + static_cast<int64_t>(t) * d)[qi];
+      if (!s_any) {  // every choice dropped: the residual passes through unchanged
         if (out_f32) {
-          float4 o;
-          o.x = __uint_as_float(rbits.x << 16);
-          o.y = __uint_as_float(rbits.x & 0xffff0000u);
-          o.z = __uint_as_float(rbits.y << 16);
-          o.w = __uint_as_float(rbits.y & 0xffff0000u);
-          reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<int64_t>(t) * d)[c] = o;
+          reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<int64_t>(t) * d)[qi] =
+              make_float4(__uint_as_float(rbits.x << 16), __uint_as_float(rbits.x & 0xffff0000u),
+                          __uint_as_float(rbits.y << 16), __uint_as_float(rbits.y & 0xffff0000u));
         } else {
-          reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + static_cast<int64_t>(t) * d)[c] = rbits;
+          reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + static_cast<int64_t>(t) * d)[qi] = rbits;
         }
-        continue;
-      }
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < k && rows[j] >= 0) {
-          const float4 v = reinterpret_cast<const float4*>(y + static_cast<int64_t>(rows[j]) * d)[c];
-          a0 = fmaf(ws[j], v.x, a0);
-          a1 = fmaf(ws[j], v.y, a1);
-          a2 = fmaf(ws[j], v.z, a2);
-          a3 = fmaf(ws[j], v.w, a3);
-        }
-      }
-      const float o0 = __uint_as_float(rbits.x << 16) + a0;
-      const float o1 = __uint_as_float(rbits.x & 0xffff0000u) + a1;
-      const float o2 = __uint_as_float(rbits.y << 16) + a2;
-      const float o3 = __uint_as_float(rbits.y & 0xffff0000u) + a3;
-      if (out_f32) {
-        reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<int64_t>(t) * d)[c] =
-            make_float4(o0, o1, o2, o3);
       } else {
-        reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + static_cast<int64_t>(t) * d)[c] =
-            make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        for (int j = 0; j < k; ++j) {  // ascending choice order
+          const int row = s_rows[j];
+          if (row < 0) continue;
+          const float wj = s_w[j];
+          const float4 v = reinterpret_cast<const float4*>(y + static_cast<int64_t>(row) * d)[qi];
+          a0 = fmaf(wj, v.x, a0);
+          a1 = fmaf(wj, v.y, a1);
+          a2 = fmaf(wj, v.z, a2);
+          a3 = fmaf(wj, v.w, a3);
+        }
+        const float o0 = __uint_as_float(rbits.x << 16) + a0;
+        const float o1 = __uint_as_float(rbits.x & 0xffff0000u) + a1;
+        const float o2 = __uint_as_float(rbits.y << 16) + a2;
+        const float o3 = __uint_as_float(rbits.y & 0xffff0000u) + a3;
+        if (out_f32) {
+          reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<int64_t>(t) * d)[qi] =
+              make_float4(o0, o1, o2, o3);
+        } else {
+          reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + static_cast<int64_t>(t) * d)[qi] =
+              make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+        }
       }
     }
+    __syncthreads();
   }
 }
 
@@ -165,7 +187,8 @@ cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, const int
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  const int blocks = std::max(1, std::min((T + 7) / 8, di.sm_count * 8));
+  const int64_t items = static_cast<int64_t>(T) * ((d / 8 + kVecPerBlock - 1) / kVecPerBlock);
+  const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(items, di.sm_count * 16)));
   permute_kernel<<<blocks, 256, 0, s>>>(x, topk_idx, slot, expert_count, expert_offset,
                                         row_of_pair, pair_of_row, x_perm, T, d, N, k, r_max, status);
   return cudaGetLastError();
@@ -177,7 +200,8 @@ cudaError_t launch_combine(const float* y_perm, const int32_t* row_of_pair, cons
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  const int blocks = std::max(1, std::min((T + 7) / 8, di.sm_count * 8));
+  const int64_t items = static_cast<int64_t>(T) * ((d + kColsPerBlock - 1) / kColsPerBlock);
+  const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(items, di.sm_count * 16)));
   combine_kernel<<<blocks, 256, 0, s>>>(y_perm, row_of_pair, topk_w, residual, out, out_f32, T, d,
                                         k, r_max, status);
   return cudaGetLastError();

@@ -179,12 +179,27 @@ __global__ void __launch_bounds__(256) topk_from_logits_kernel(const float* __re
 // arrivals with the same expert; it is kept iff that number is below the capacity.
 //
 // Pass 1 (one block per chunk of kSlotChunk arrivals): warp w ranks its 512 consecutive
-// arrivals 32 at a time with __match_any_sync, keeping per-warp running counts per expert in
+// arrivals 32 at a time (lanes with the same expert found by bit ballots), keeping per-warp
+// running counts per expert in
 // shared memory; then the block turns the per-warp counts into exclusive offsets and either
 //   - (one chunk) writes final slots and kept counts directly, or
 //   - (several chunks) writes chunk-local ranks into `slot` and chunk totals into scratch.
 // Pass 2 (one block): per expert, exclusive scan of the chunk totals; kept counts.
 // Pass 3: slot = chunk-local rank + chunk base, or -1 when it reaches the capacity.
+// Lanes of the warp whose key equals this lane's key (0 <= key < 512): the AND over the 9 key
+// bits of the ballot of lanes agreeing on that bit. Nine ballots, independent of how many
+// distinct keys the warp holds.
+__device__ __forceinline__ unsigned peers_with_same_key(int key) {
+  unsigned peers = kFull;
+#pragma unroll
+  for (int b = 0; b < 9; ++b) {
+    const bool bit = (key >> b) & 1;
+    const unsigned bal = __ballot_sync(kFull, bit);
+    peers &= bit ? bal : ~bal;
+  }
+  return peers;
+}
+
 constexpr int kSlThreads = 256;
 constexpr int kSlWarps = kSlThreads / 32;
 constexpr int kSlIters = kSlotChunk / kSlThreads;  // arrivals per lane
@@ -201,27 +216,28 @@ __global__ void __launch_bounds__(kSlThreads) slot_rank_kernel(
   const int p_base = blockIdx.x * kSlotChunk + w * (kSlotChunk / kSlWarps);
   int ex[kSlIters];
   int q_of[kSlIters];  // storage index t * k + j of each arrival
-  // all loads first, so their latencies overlap
+  // every load is issued before any is used, so their latencies overlap
 #pragma unroll
   for (int it = 0; it < kSlIters; ++it) {
     const int p = p_base + it * 32 + lane;
-    int e = -1, q = -1;
+    int q = -1;
     if (p < P) {
       const int j = p / T;
-      const int t = p - j * T;
-      q = t * k + j;
-      e = __ldg(topk_idx + q);
-      if (e < 0 || e >= N) e = -2;  // invalid expert id: never kept
+      q = (p - j * T) * k + j;
     }
-    ex[it] = e;
     q_of[it] = q;
   }
+#pragma unroll
+  for (int it = 0; it < kSlIters; ++it) ex[it] = q_of[it] >= 0 ? __ldg(topk_idx + q_of[it]) : -1;
+#pragma unroll
+  for (int it = 0; it < kSlIters; ++it)
+    if (q_of[it] >= 0 && (ex[it] < 0 || ex[it] >= N)) ex[it] = -2;  // invalid id: never kept
   __syncthreads();
   int local[kSlIters];
 #pragma unroll
   for (int it = 0; it < kSlIters; ++it) {
     const int e = ex[it];
-    const unsigned peers = __match_any_sync(kFull, e);
+    const unsigned peers = peers_with_same_key(e + 2);  // e + 2 in [0, 257]
     const int rank = __popc(peers & lanemask_lt());
     const int cnt = (e >= 0) ? s_cnt[w][e] : 0;
     __syncwarp();

@@ -24,8 +24,10 @@
 //   warp 1      TMEM owner and MMA issuer: per k block 3 x 4 MMAs (M=128, N=NP, K=16) into one
 //               fp32 accumulator of NP columns;
 //   warps 4-7   (in-kernel split only) the converters, then the epilogue: thread i owns token
-//               i's row of logits in TMEM, adds the bias, writes the logits, keeps a running
-//               top-8 and writes the first k indices and weights.
+//               i's row of logits in TMEM, adds the bias, keeps a running sorted top-KMAX
+//               (KMAX = k rounded up to 1, 2, 4 or 8) and writes the first k indices and
+//               weights; the [128][N] logits tile is staged in the idle
+//               pipeline shared memory and written out as one coalesced block.
 // All mbarrier waits are bounded. A timeout records MOE_ERR_TIMEOUT, stops the CTA's work,
 // drains its own copies and MMAs, and frees TMEM.
 #include <math.h>
@@ -61,6 +63,7 @@ struct RCfg {
   static constexpr int SMEM_BYTES = FIXED_BYTES + STAGES * STAGE_BYTES + 1024;
   static_assert(STAGES >= 2, "router pipeline depth");
   static_assert(NP % 16 == 0 && NP >= 16 && NP <= 256, "UMMA N for M = 128");
+  static_assert(kTok * (NP + 1) * 4 <= SMEM_BYTES - 1024, "logits staging fits the pipeline smem");
 };
 
 __device__ __forceinline__ bool better(float av, int ae, float bv, int be) {
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(256) split_router_weights_kernel(const float* 
   }
 }
 
-template <int NP, bool PRESPLIT>
+template <int NP, bool PRESPLIT, int KMAX>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ w, const float* __restrict__ bias,
@@ -127,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t w_empty[2];
   __shared__ __align__(8) uint64_t acc_full;
   __shared__ __align__(8) uint64_t done_bar;
+  __shared__ __align__(8) uint64_t epi_bar;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
 
@@ -151,6 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(&acc_full), 1);
     mbar_init(smem_u32(&done_bar), 1);
+    mbar_init(smem_u32(&epi_bar), kConvThreads);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -298,32 +303,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = t0 + ct;
       const bool valid = t < T;
       const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      // the best 8 are kept whatever k is (entry 7 is the admission threshold); the first k
-      // are written
-      float best_v[8];
-      int best_e[8];
+      // the pipeline's shared memory is idle now: it stages the [128][N] logits tile
+      float* stage = reinterpret_cast<float*>(gbase);
+      // a sorted list of the best KMAX (>= k) entries; entry KMAX-1 is the admission threshold
+      float best_v[KMAX];
+      int best_e[KMAX];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
+      for (int r = 0; r < KMAX; ++r) {
         best_v[r] = -INFINITY;
         best_e[r] = 0x7fffffff;
       }
-      for (int c0 = 0; c0 < N; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(trow + c0, v);
+      for (int c0 = 0; c0 < N; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(trow + c0, v);  // columns past NP are never used: c0 + 32 <= NP or N <= 16
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 32; ++i) {
           const int e = c0 + i;
           if (e >= N) continue;
           float L = __uint_as_float(v[i]);
           if (bias != nullptr) L += __ldg(bias + e);
-          if (valid) logits[static_cast<int64_t>(t) * N + e] = L;
+          stage[ct * (N + 1) + e] = L;  // padded rows: no bank conflicts
           const float key = isnan(L) ? -INFINITY : L;
-          if (better(key, e, best_v[7], best_e[7])) {
+          if (better(key, e, best_v[KMAX - 1], best_e[KMAX - 1])) {
             // shift the entries the candidate beats down by one and drop it into place;
-            // from the last slot up, so entry r-1 is still the old value when read
+            // every slot's update reads only the old list, so the slots update in parallel
 #pragma unroll
-            for (int r = 7; r >= 0; --r) {
+            for (int r = KMAX - 1; r >= 0; --r) {
               if (better(key, e, best_v[r], best_e[r])) {
                 const int u = r > 0 ? r - 1 : 0;
                 const bool beats_prev = (r > 0) && better(key, e, best_v[u], best_e[u]);
@@ -335,18 +341,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (valid) {
-        float num[8], den = 0.f;
+        float num[KMAX], den = 0.f;
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
+        for (int r = 0; r < KMAX; ++r) {
           num[r] = (r < k) ? expf(best_v[r] - best_v[0]) : 0.f;
           den += num[r];
         }
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int r = 0; r < KMAX; ++r)
           if (r < k) {
             topk_idx[static_cast<int64_t>(t) * k + r] = best_e[r];
             topk_w[static_cast<int64_t>(t) * k + r] = num[r] / den;
           }
+      }
+      // the tile's logits leave shared memory as one contiguous, coalesced block
+      mbar_arrive(smem_u32(&epi_bar));
+      const bool synced = mbar_wait(smem_u32(&epi_bar), 0, timeout_ns, &s_abort);
+      if (__all_sync(0xffffffffu, synced)) {
+        const int rows = min(kTok, T - t0);
+        float* dst = logits + static_cast<int64_t>(t0) * N;
+        for (int i = ct; i < rows * N; i += kConvThreads) {
+          const int r = i / N;
+          dst[i] = stage[r * (N + 1) + (i - r * N)];
+        }
+      } else {
+        s_abort = 1;
+        report_error(status, MOE_ERR_TIMEOUT);
       }
     } else {
       s_abort = 1;
@@ -380,22 +400,35 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <int NP, bool PRESPLIT>
-cudaError_t launch_np(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
-                      const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
-                      int d, int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
+template <int NP, bool PRESPLIT, int KMAX>
+cudaError_t launch_npk(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
+                       const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
+                       int d, int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
   using C = RCfg<NP, PRESPLIT>;
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(router_tc_kernel<NP, PRESPLIT>,
+    attr = cudaFuncSetAttribute(router_tc_kernel<NP, PRESPLIT, KMAX>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr != cudaSuccess) return attr;
   const int grid = (T + kTok - 1) / kTok;
-  router_tc_kernel<NP, PRESPLIT><<<grid, kThreads, C::SMEM_BYTES, s>>>(
+  router_tc_kernel<NP, PRESPLIT, KMAX><<<grid, kThreads, C::SMEM_BYTES, s>>>(
       mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns);
   return cudaGetLastError();
+}
+
+template <int NP, bool PRESPLIT>
+cudaError_t launch_np(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
+                      const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
+                      int d, int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
+  if (k <= 1)
+    return launch_npk<NP, PRESPLIT, 1>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+  if (k <= 2)
+    return launch_npk<NP, PRESPLIT, 2>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+  if (k <= 4)
+    return launch_npk<NP, PRESPLIT, 4>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+  return launch_npk<NP, PRESPLIT, 8>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
 }
 
 template <bool PRESPLIT>
