@@ -4,10 +4,11 @@
 python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME[:T]] [--impl ours|reference]
 
 A step is one whole forward pass of the layer (route, permute, grouped expert FFN, combine)
-over one batch of synthetic tokens whose inputs already sit in HBM. Each stage is captured once
-as a CUDA graph; a timed step replays the four graphs with CUDA events between them on the
-launching stream. Steps are timed one by one; L2 is flushed (a 256 MB write) before each step,
-outside the timed events. The end-to-end figure (e2e) calls moe_forward eagerly, with the H2D
+over one batch of synthetic tokens whose inputs already sit in HBM. The forward is captured
+once as a CUDA graph; a timed step replays it between two CUDA events on the launching stream.
+Steps are timed one by one; L2 is flushed (a 256 MB write) before each step, outside the
+timed events. A second pass replays the stages as separate graphs with events between them
+for the per-stage breakdown and the grouped FFN's roofline. The end-to-end figure (e2e) calls moe_forward eagerly, with the H2D
 copy of the tokens and the D2H copy of the output inside its timed region. Under torchrun every rank runs its own replica of the workload
 (weak scaling, no collective on the data path). Rank 0 prints the line, with the time taken
 as the max over ranks.
@@ -248,8 +249,8 @@ class Layer:
         return [route, permute, ffn, combine]
 
     def capture_stage_graphs(self):
-        """Each stage captured once as a CUDA graph; a replay launches that stage's kernels
-        without host work in between."""
+        """The forward captured as CUDA graphs: once whole (its kernels overlap through
+        programmatic dependent launch) and once per stage (for the stage breakdown)."""
         self.graphs = []
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
@@ -257,11 +258,21 @@ class Layer:
             for call in self.stage_calls():  # one eager pass on the capture stream first
                 call()
         torch.cuda.current_stream().wait_stream(s)
+        self.graph_full = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_full):
+            for call in self.stage_calls():
+                call()
         for call in self.stage_calls():
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 call()
             self.graphs.append(g)
+
+    def step_full(self, ev):
+        """One forward: the whole-forward graph between two events."""
+        ev[0].record()
+        self.graph_full.replay()
+        ev[1].record()
 
     def step_stages(self, ev):
         """One forward: the four stage graphs replayed with events between them (5 events)."""
@@ -314,6 +325,8 @@ def run_gpu(args, rank, world, local_rank):
 
     for _ in range(args.warmup):
         flush_l2(flush)
+        layer.step_full(wev)
+        flush_l2(flush)
         layer.step_stages(wev)
     torch.cuda.synchronize()
     err = moe.read_device_error(layer.fws, offset_bytes=layer.b.stage_ws - layer.fws.data_ptr())
@@ -327,16 +340,23 @@ def run_gpu(args, rank, world, local_rank):
     clocks.start()
     for k in range(args.steps):
         flush_l2(flush)
-        layer.step_stages(evs[k])
+        layer.step_full(evs[k])
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-
-    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
-    stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
-                for i, n in enumerate(["route", "permute", "grouped_ffn", "combine"])}
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_ms = sum(step_ms)
+
+    # stage breakdown: the same K steps replayed stage by stage, events between the stages
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush_l2(flush)
+        layer.step_stages(sev[k])
+    torch.cuda.synchronize()
+    stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in sev)
+                for i, n in enumerate(["route", "permute", "grouped_ffn", "combine"])}
     ffn_ms = stage_ms["grouped_ffn"]
 
     # end to end through the public call with host buffers
@@ -393,7 +413,9 @@ def run_gpu(args, rank, world, local_rank):
                    "l2": "flushed before every step (256 MB write outside the timed events); "
                          "expert weights also exceed L2",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "launch": "each stage a captured CUDA graph, events between stages"},
+                   "launch": "value: the whole forward as one captured CUDA graph (kernels chained "
+                             "by programmatic dependent launch); stages_ms and roofline: the same "
+                             "steps replayed as one graph per stage with events between stages"},
         "stages_ms": {k: round(v_, 4) for k, v_ in stage_ms.items()},
         "roofline": roof,
         "layer_gbs": round(ab["layer"] / (total_ms / args.steps * 1e-3) / 1e9, 1),

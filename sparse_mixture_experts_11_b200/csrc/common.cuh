@@ -48,6 +48,17 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream serialisation: it lets the
+// next kernel on the stream start launching (pdl_trigger) while this one still runs, and it
+// waits for the previous kernel's completion and memory (pdl_wait) before it reads anything
+// that kernel produced or writes any global memory. Setup that touches only shared memory,
+// TMEM and tensor-map prefetches runs before the wait, overlapping the previous kernel's tail.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

@@ -236,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int s_splits;
   __shared__ int s_fixup;
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int N = p.n_experts;
@@ -262,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(&s_tmem_base), C::TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_wait();  // below: reads of the previous kernels' outputs and writes to global memory
   if (warp == 2) {
     // Per-expert tile counts and their exclusive prefix (experts lane*per .. lane*per+per-1).
     const int per = (N + 31) / 32;
@@ -563,8 +565,8 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmP
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  grouped_gemm_kernel<EPI, BN_OUT><<<grid, kThreads, C::SMEM_BYTES, s>>>(ma, mb, gp);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_kernel<EPI, BN_OUT>, dim3(grid), dim3(kThreads), C::SMEM_BYTES, s,
+                    ma, mb, gp);
 }
 
 int64_t tiles_upper_bound(int64_t r_max, int N, int n_tiles_n) {

@@ -56,6 +56,8 @@ __global__ void __launch_bounds__(256) permute_kernel(
   __shared__ int s_off[257];
   __shared__ int s_warp[8];
   __shared__ int s_rows[8];
+  pdl_trigger();
+  pdl_wait();
   block_offsets_256(expert_count, N, s_off, s_warp);
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i <= N; i += blockDim.x) expert_offset[i] = s_off[i];
@@ -112,6 +114,8 @@ __global__ void __launch_bounds__(256) combine_kernel(
   __shared__ int s_rows[8];
   __shared__ float s_w[8];
   __shared__ int s_any;
+  pdl_trigger();
+  pdl_wait();
   const int nq = d / 4;  // groups of 4 columns
   const int chunks = (d + kColsPerBlock - 1) / kColsPerBlock;
   const int64_t items = static_cast<int64_t>(T) * chunks;
@@ -189,9 +193,8 @@ cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, const int
   if (err != cudaSuccess) return err;
   const int64_t items = static_cast<int64_t>(T) * ((d / 8 + kVecPerBlock - 1) / kVecPerBlock);
   const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(items, di.sm_count * 16)));
-  permute_kernel<<<blocks, 256, 0, s>>>(x, topk_idx, slot, expert_count, expert_offset,
-                                        row_of_pair, pair_of_row, x_perm, T, d, N, k, r_max, status);
-  return cudaGetLastError();
+  return launch_pdl(permute_kernel, dim3(blocks), dim3(256), 0, s, x, topk_idx, slot, expert_count,
+                    expert_offset, row_of_pair, pair_of_row, x_perm, T, d, N, k, r_max, status);
 }
 
 cudaError_t launch_combine(const float* y_perm, const int32_t* row_of_pair, const float* topk_w,
@@ -202,9 +205,8 @@ cudaError_t launch_combine(const float* y_perm, const int32_t* row_of_pair, cons
   if (err != cudaSuccess) return err;
   const int64_t items = static_cast<int64_t>(T) * ((d + kColsPerBlock - 1) / kColsPerBlock);
   const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(items, di.sm_count * 16)));
-  combine_kernel<<<blocks, 256, 0, s>>>(y_perm, row_of_pair, topk_w, residual, out, out_f32, T, d,
-                                        k, r_max, status);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(blocks), dim3(256), 0, s, y_perm, row_of_pair, topk_w,
+                    residual, out, out_f32, T, d, k, r_max, status);
 }
 
 }  // namespace moe

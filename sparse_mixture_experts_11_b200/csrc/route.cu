@@ -106,6 +106,8 @@ __global__ void __launch_bounds__(kTokThreads) router_token_kernel(
     int d, int N, int k) {
   __shared__ float s_part[kTokWarps][EPT];  // [warp][pass]: at most EPT passes of 32 experts
   __shared__ float s_logit[EPT * 32];
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint16_t* xr = x + static_cast<int64_t>(t) * d;
@@ -162,6 +164,8 @@ __global__ void __launch_bounds__(256) topk_from_logits_kernel(const float* __re
                                                                int32_t* __restrict__ topk_idx,
                                                                float* __restrict__ topk_w, int T,
                                                                int N, int k) {
+  pdl_trigger();
+  pdl_wait();
   const int warps = blockDim.x >> 5;
   for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
     float val[EPT];
@@ -209,9 +213,11 @@ __global__ void __launch_bounds__(kSlThreads) slot_rank_kernel(
     int32_t* __restrict__ chunk_hist, int32_t* __restrict__ expert_count, int T, int N, int k,
     int cap, int single_chunk) {
   __shared__ int s_cnt[kSlWarps][256];
+  pdl_trigger();
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int P = T * k;  // < 2^31, checked on the host
   for (int i = tid; i < kSlWarps * 256; i += kSlThreads) (&s_cnt[0][0])[i] = 0;
+  pdl_wait();
 
   const int p_base = blockIdx.x * kSlotChunk + w * (kSlotChunk / kSlWarps);
   int ex[kSlIters];
@@ -276,6 +282,8 @@ __global__ void __launch_bounds__(kSlThreads) slot_rank_kernel(
 __global__ void __launch_bounds__(256) slot_scan_kernel(int32_t* __restrict__ chunk_hist,
                                                         int32_t* __restrict__ expert_count,
                                                         int n_chunks, int N, int cap) {
+  pdl_trigger();
+  pdl_wait();
   for (int e = threadIdx.x; e < N; e += blockDim.x) {
     int run = 0;
     for (int c = 0; c < n_chunks; ++c) {
@@ -291,6 +299,8 @@ __global__ void __launch_bounds__(256) slot_finalize_kernel(const int32_t* __res
                                                             int32_t* __restrict__ slot,
                                                             const int32_t* __restrict__ chunk_hist,
                                                             int T, int N, int k, int cap) {
+  pdl_trigger();
+  pdl_wait();
   const int P = T * k;
   for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < P; p += gridDim.x * blockDim.x) {
     const int j = p / T;
@@ -317,29 +327,18 @@ cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const f
   if (router_uses_tensor_cores(T, N, d))
     return launch_router_tc(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k,
                             split_scratch, status, timeout_ns, s);
-  if (N <= 32)
-    router_token_kernel<1><<<T, kTokThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
-  else if (N <= 64)
-    router_token_kernel<2><<<T, kTokThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
-  else if (N <= 128)
-    router_token_kernel<4><<<T, kTokThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
-  else
-    router_token_kernel<8><<<T, kTokThreads, 0, s>>>(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k);
-  return cudaGetLastError();
+  auto kern = N <= 32 ? router_token_kernel<1> : N <= 64 ? router_token_kernel<2>
+             : N <= 128 ? router_token_kernel<4> : router_token_kernel<8>;
+  return launch_pdl(kern, dim3(T), dim3(kTokThreads), 0, s, x, w_router, bias, logits, topk_idx,
+                    topk_w, T, d, N, k);
 }
 
 cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, float* topk_w, int T,
                                     int N, int k, cudaStream_t s) {
   const int blocks = (T + 7) / 8;
-  if (N <= 32)
-    topk_from_logits_kernel<1><<<blocks, 256, 0, s>>>(logits, topk_idx, topk_w, T, N, k);
-  else if (N <= 64)
-    topk_from_logits_kernel<2><<<blocks, 256, 0, s>>>(logits, topk_idx, topk_w, T, N, k);
-  else if (N <= 128)
-    topk_from_logits_kernel<4><<<blocks, 256, 0, s>>>(logits, topk_idx, topk_w, T, N, k);
-  else
-    topk_from_logits_kernel<8><<<blocks, 256, 0, s>>>(logits, topk_idx, topk_w, T, N, k);
-  return cudaGetLastError();
+  auto kern = N <= 32 ? topk_from_logits_kernel<1> : N <= 64 ? topk_from_logits_kernel<2>
+             : N <= 128 ? topk_from_logits_kernel<4> : topk_from_logits_kernel<8>;
+  return launch_pdl(kern, dim3(blocks), dim3(256), 0, s, logits, topk_idx, topk_w, T, N, k);
 }
 
 cudaError_t launch_capacity_slots(const int32_t* topk_idx, int32_t* slot, int32_t* expert_count,
@@ -348,13 +347,15 @@ cudaError_t launch_capacity_slots(const int32_t* topk_idx, int32_t* slot, int32_
   const int64_t P = static_cast<int64_t>(T) * k;
   const int n_chunks = static_cast<int>(slot_chunks(P));
   const int single = n_chunks == 1 ? 1 : 0;
-  slot_rank_kernel<<<n_chunks, kSlThreads, 0, s>>>(topk_idx, slot, chunk_scratch, expert_count, T,
-                                                   N, k, capacity, single);
-  if (single) return cudaGetLastError();
-  slot_scan_kernel<<<1, 256, 0, s>>>(chunk_scratch, expert_count, n_chunks, N, capacity);
+  cudaError_t e = launch_pdl(slot_rank_kernel, dim3(n_chunks), dim3(kSlThreads), 0, s, topk_idx,
+                             slot, chunk_scratch, expert_count, T, N, k, capacity, single);
+  if (e != cudaSuccess || single) return e;
+  e = launch_pdl(slot_scan_kernel, dim3(1), dim3(256), 0, s, chunk_scratch, expert_count, n_chunks,
+                 N, capacity);
+  if (e != cudaSuccess) return e;
   const int blocks = static_cast<int>(std::min<int64_t>((P + 255) / 256, 148 * 8));
-  slot_finalize_kernel<<<blocks, 256, 0, s>>>(topk_idx, slot, chunk_scratch, T, N, k, capacity);
-  return cudaGetLastError();
+  return launch_pdl(slot_finalize_kernel, dim3(blocks), dim3(256), 0, s, topk_idx, slot,
+                    chunk_scratch, T, N, k, capacity);
 }
 
 }  // namespace moe

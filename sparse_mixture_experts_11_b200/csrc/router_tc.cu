@@ -103,6 +103,8 @@ __device__ __forceinline__ void split3(const float4& v0, const float4& v1, uint4
 __global__ void __launch_bounds__(256) split_router_weights_kernel(const float* __restrict__ w,
                                                                    uint16_t* __restrict__ out,
                                                                    int64_t n_elems) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t n8 = n_elems / 8;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -134,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   uint8_t* gbase = dyn_smem + (base - smem_u32(dyn_smem));  // generic pointer of `base`
@@ -176,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     fence_proxy_async_smem();
   }
+  pdl_wait();  // everything below reads the previous kernels' outputs or writes global memory
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -413,9 +417,8 @@ cudaError_t launch_npk(const CUtensorMap& mx, const CUtensorMap& mw, const float
   });
   if (attr != cudaSuccess) return attr;
   const int grid = (T + kTok - 1) / kTok;
-  router_tc_kernel<NP, PRESPLIT, KMAX><<<grid, kThreads, C::SMEM_BYTES, s>>>(
-      mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns);
-  return cudaGetLastError();
+  return launch_pdl(router_tc_kernel<NP, PRESPLIT, KMAX>, dim3(grid), dim3(kThreads), C::SMEM_BYTES,
+                    s, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns);
 }
 
 template <int NP, bool PRESPLIT>
@@ -485,8 +488,8 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const flo
   }
   const int64_t n = static_cast<int64_t>(N) * d;
   const int blocks = static_cast<int>(std::min<int64_t>((n / 8 + 255) / 256, 148 * 8));
-  split_router_weights_kernel<<<blocks, 256, 0, s>>>(w_router, split_scratch, n);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(split_router_weights_kernel, dim3(blocks), dim3(256), 0, s, w_router,
+                             split_scratch, n);
   if (e != cudaSuccess) return e;
   return launch_tc<true>(mx, mw, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status,
                          timeout_ns, s);
