@@ -89,7 +89,8 @@ size_t split_scratch_bytes(const moe_dims* d) {
 }
 
 moe::FfnScratchPlan ffn_plan(const moe_dims* d) {
-  return moe::ffn_scratch_plan(d->n_experts, d->d_model, d->d_ff, d->act, max_rows(d));
+  return moe::ffn_scratch_plan(d->n_experts, d->d_model, d->d_ff, d->act, max_rows(d),
+                               std::min(d->capacity, d->T));
 }
 
 // Per-stage workspace:
@@ -252,6 +253,7 @@ moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
   a.r_max = rmax;
   a.status = status_of(ws);
   a.timeout_ns = moe::kDefaultWaitTimeoutNs;
+  a.rows_per_expert = std::min(dims->capacity, dims->T);
   const moe::FfnScratchPlan plan = ffn_plan(dims);
   if (plan.max_splits1 > 1 || plan.max_splits2 > 1) {
     a.part = reinterpret_cast<float*>(shared_region_of(dims, ws));

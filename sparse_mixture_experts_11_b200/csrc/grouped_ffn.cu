@@ -39,7 +39,8 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;       // rows per tile (UMMA M)
+// Rows per tile (UMMA M) is a template parameter BM: 128, or 64 when no expert can hold more
+// than 64 rows. For M = 64 the accumulator's row 16q + i (i < 16) sits in TMEM lane 32q + i.
 constexpr int BK = 64;        // k per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
@@ -75,7 +76,7 @@ constexpr int pow2_at_least(int v) {
   return p;
 }
 
-template <int EPI, int BN_OUT>
+template <int EPI, int BN_OUT, int BM>
 struct Cfg {
   static constexpr int UMMA_N = (EPI == EPI_SWIGLU) ? 2 * BN_OUT : BN_OUT;
   static constexpr int A_BYTES = BM * BK * 2;
@@ -88,6 +89,7 @@ struct Cfg {
   static_assert(TMEM_COLS <= 512, "two accumulators must fit in TMEM");
   static_assert(BN_OUT % 16 == 0, "epilogue works in 16-column groups");
   static_assert(STAGES >= 2, "pipeline depth");
+  static_assert(BM == 64 || BM == 128, "UMMA M");
 };
 
 __device__ __forceinline__ uint64_t make_policy(int which) {
@@ -108,6 +110,7 @@ struct TileCoord {
   int n0;     // first output column
 };
 
+template <int BM>
 __device__ __forceinline__ TileCoord decode_tile(int tile, int N, int bn_out,
                                                  const int* s_tile_start, const int* s_off) {
   int lo = 0, hi = N - 1;  // largest e with s_tile_start[e] <= tile
@@ -217,11 +220,11 @@ __device__ __forceinline__ void store_final16(const GemmParams& p, int64_t row, 
   }
 }
 
-template <int EPI, int BN_OUT>
+template <int EPI, int BN_OUT, int BM>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
-  using C = Cfg<EPI, BN_OUT>;
+  using C = Cfg<EPI, BN_OUT, BM>;
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
   __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int unit = blockIdx.x; ok && unit < total_units; unit += gridDim.x) {
         const int tile = unit / splits, sp = unit - tile * splits;
-        const TileCoord c = decode_tile(tile, N, BN_OUT, s_tile_start, s_off);
+        const TileCoord c = decode_tile<BM>(tile, N, BN_OUT, s_tile_start, s_off);
         const int kb0 = sp * p.num_kb / splits, kb1 = (sp + 1) * p.num_kb / splits;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % C::STAGES;
@@ -406,13 +409,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const int r_local = q * 32 + lane;
+    // tile row held by this thread's TMEM lane (M = 64 uses lanes 0-15 of each quadrant)
+    const int r_local = BM == 128 ? q * 32 + lane : (lane < 16 ? q * 16 + lane : BM);
     int tc = 0;
     uint32_t epi_phase = 0;
     bool ok = true;
     for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x, ++tc) {
       const int tile = unit / splits, sp = unit - tile * splits;
-      const TileCoord c = decode_tile(tile, N, BN_OUT, s_tile_start, s_off);
+      const TileCoord c = decode_tile<BM>(tile, N, BN_OUT, s_tile_start, s_off);
       const int buf = tc & 1;
       const uint32_t tph = (tc >> 1) & 1;
       const bool got = mbar_wait(smem_u32(&tfull_bar[buf]), tph, p.timeout_ns, &s_abort);
@@ -554,29 +558,29 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
   return r == CUDA_SUCCESS;
 }
 
-template <int EPI, int BN_OUT>
+template <int EPI, int BN_OUT, int BM>
 cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& gp,
                        int grid, cudaStream_t s) {
-  using C = Cfg<EPI, BN_OUT>;
+  using C = Cfg<EPI, BN_OUT, BM>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN_OUT>,
+    attr_err = cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN_OUT, BM>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  return launch_pdl(grouped_gemm_kernel<EPI, BN_OUT>, dim3(grid), dim3(kThreads), C::SMEM_BYTES, s,
+  return launch_pdl(grouped_gemm_kernel<EPI, BN_OUT, BM>, dim3(grid), dim3(kThreads), C::SMEM_BYTES, s,
                     ma, mb, gp);
 }
 
-int64_t tiles_upper_bound(int64_t r_max, int N, int n_tiles_n) {
-  // sum_e ceil(m_e / BM) <= ceil(R / BM) + (experts with rows)
-  const int64_t m_tiles_ub = (r_max + BM - 1) / BM + std::min<int64_t>(N, r_max);
+int64_t tiles_upper_bound(int64_t r_max, int N, int n_tiles_n, int bm) {
+  // sum_e ceil(m_e / bm) <= ceil(R / bm) + (experts with rows)
+  const int64_t m_tiles_ub = (r_max + bm - 1) / bm + std::min<int64_t>(N, r_max);
   return m_tiles_ub * n_tiles_n;
 }
 
-int grid_for(int64_t r_max, int N, int n_tiles_n, int sm_count, int max_splits) {
-  const int64_t units_ub = tiles_upper_bound(r_max, N, n_tiles_n) * max_splits;
+int grid_for(int64_t r_max, int N, int n_tiles_n, int sm_count, int max_splits, int bm) {
+  const int64_t units_ub = tiles_upper_bound(r_max, N, n_tiles_n, bm) * max_splits;
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units_ub, sm_count)));
 }
 
@@ -597,9 +601,11 @@ constexpr int kDnBn = 256;        // output columns per tile of the down GEMM
 
 }  // namespace
 
-FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max) {
-  FfnScratchPlan pl{1, 1, 0, 0};
+FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max,
+                                int64_t rows_per_expert) {
+  FfnScratchPlan pl{1, 1, 0, 0, 128};
   if (r_max <= 0) return pl;
+  pl.bm = rows_per_expert <= 64 ? 64 : 128;
   const bool swiglu = act == MOE_ACT_SWIGLU;
   const int bn1 = swiglu ? kGuBnSwiglu : kGuBnGelu;
   const int ld1 = swiglu ? 2 * F : F;
@@ -609,11 +615,11 @@ FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max) {
   int64_t tiles = 0;
   if (pl.max_splits1 > 1) {
     part = std::max(part, static_cast<size_t>(pl.max_splits1) * r_max * ld1 * 4);
-    tiles = std::max(tiles, tiles_upper_bound(r_max, N, (F + bn1 - 1) / bn1));
+    tiles = std::max(tiles, tiles_upper_bound(r_max, N, (F + bn1 - 1) / bn1, pl.bm));
   }
   if (pl.max_splits2 > 1) {
     part = std::max(part, static_cast<size_t>(pl.max_splits2) * r_max * d * 4);
-    tiles = std::max(tiles, tiles_upper_bound(r_max, N, (d + kDnBn - 1) / kDnBn));
+    tiles = std::max(tiles, tiles_upper_bound(r_max, N, (d + kDnBn - 1) / kDnBn, pl.bm));
   }
   pl.part_bytes = part;
   pl.counter_bytes = static_cast<size_t>(tiles) * sizeof(int);
@@ -632,13 +638,16 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   const int bn_gu = swiglu ? kGuBnSwiglu : kGuBnGelu;
   // weights are read once per m-tile; when every expert has at most one m-tile (decode-sized
   // batches) they are pure streams and should not displace the activations in L2
-  const int wpol = (a.r_max <= BM) ? 1 : 0;
+  const FfnScratchPlan plan =
+      ffn_scratch_plan(a.N, a.d, a.F, a.act, a.r_max, a.rows_per_expert);
+  const int bm = plan.bm;
+  const int wpol = (a.rows_per_expert <= bm) ? 1 : 0;
 
   CUtensorMap mA1, mB1, mA2, mB2;
   {
     const uint64_t dims[2] = {d, R};
     const uint64_t str[1] = {d * 2};
-    const uint32_t box[2] = {BK, BM};
+    const uint32_t box[2] = {BK, static_cast<uint32_t>(bm)};
     if (!make_map(&mA1, a.x_perm, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   if (swiglu) {
@@ -655,7 +664,7 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   {
     const uint64_t dims[2] = {F, R};
     const uint64_t str[1] = {F * 2};
-    const uint32_t box[2] = {BK, BM};
+    const uint32_t box[2] = {BK, static_cast<uint32_t>(bm)};
     if (!make_map(&mA2, a.h, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   {
@@ -677,15 +686,18 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   g1.status = a.status;
   g1.timeout_ns = a.timeout_ns;
   g1.weight_policy = wpol;
-  const FfnScratchPlan plan = ffn_scratch_plan(a.N, a.d, a.F, a.act, a.r_max);
   const bool can_split = a.part != nullptr && a.tile_counters != nullptr;
   g1.max_splits = can_split ? plan.max_splits1 : 1;
   g1.part = a.part;
   g1.part_ld = swiglu ? 2 * a.F : a.F;
   g1.tile_counters = a.tile_counters;
-  const int grid1 = grid_for(a.r_max, a.N, g1.n_tiles_n, di.sm_count, g1.max_splits);
-  err = swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu>(mA1, mB1, g1, grid1, s)
-               : launch_one<EPI_GELU, kGuBnGelu>(mA1, mB1, g1, grid1, s);
+  const int grid1 = grid_for(a.r_max, a.N, g1.n_tiles_n, di.sm_count, g1.max_splits, bm);
+  if (bm == 64)
+    err = swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 64>(mA1, mB1, g1, grid1, s)
+                 : launch_one<EPI_GELU, kGuBnGelu, 64>(mA1, mB1, g1, grid1, s);
+  else
+    err = swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128>(mA1, mB1, g1, grid1, s)
+                 : launch_one<EPI_GELU, kGuBnGelu, 128>(mA1, mB1, g1, grid1, s);
   if (err != cudaSuccess) return err;
 
   GemmParams g2 = g1;
@@ -696,8 +708,9 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   g2.num_kb = a.F / BK;
   g2.max_splits = can_split ? plan.max_splits2 : 1;
   g2.part_ld = a.d;
-  const int grid2 = grid_for(a.r_max, a.N, g2.n_tiles_n, di.sm_count, g2.max_splits);
-  return launch_one<EPI_STORE_F32, kDnBn>(mA2, mB2, g2, grid2, s);
+  const int grid2 = grid_for(a.r_max, a.N, g2.n_tiles_n, di.sm_count, g2.max_splits, bm);
+  return bm == 64 ? launch_one<EPI_STORE_F32, kDnBn, 64>(mA2, mB2, g2, grid2, s)
+                  : launch_one<EPI_STORE_F32, kDnBn, 128>(mA2, mB2, g2, grid2, s);
 }
 
 }  // namespace moe

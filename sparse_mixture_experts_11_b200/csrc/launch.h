@@ -84,8 +84,11 @@ struct FfnScratchPlan {
   int max_splits1, max_splits2;  // gate/up GEMM, down GEMM (1 = no split)
   size_t part_bytes;             // partial tiles (shared by the two GEMMs, which run in turn)
   size_t counter_bytes;          // per-tile arrival counters
+  int bm;                        // rows per tile: 64 when no expert can hold more, else 128
 };
-FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max);
+// rows_per_expert: the most rows any one expert can receive, min(capacity, T).
+FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max,
+                                int64_t rows_per_expert);
 
 struct GroupedFfnArgs {
   const uint16_t* x_perm;
@@ -100,6 +103,7 @@ struct GroupedFfnArgs {
   uint64_t timeout_ns;
   float* part;          // ffn_scratch_plan().part_bytes, or null when no split is planned
   int* tile_counters;   // ffn_scratch_plan().counter_bytes, zeroed once before first use
+  int64_t rows_per_expert;  // min(capacity, T)
 };
 cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s);
 
