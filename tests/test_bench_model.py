@@ -31,8 +31,12 @@ def test_bytes_model_switch():
 
 
 def test_launch_counts():
-    assert bench.launches_per_step(4096, 1, 4096) == 6
-    assert bench.launches_per_step(16384, 8, 20480) == 8
+    # switch: W_r split + tensor-core router, one slot pass, permute, 2 GEMMs, combine
+    assert bench.launches_per_step(4096, 1, 4096, 64, 1024) == 7
+    # fine-grained: tensor-core router (2), three slot passes, permute, 2 GEMMs, combine
+    assert bench.launches_per_step(16384, 8, 20480, 256, 7168) == 9
+    # decode: per-token router, one slot pass, permute, 2 GEMMs, combine
+    assert bench.launches_per_step(1, 2, 2, 8, 4096) == 6
     assert bench.launches_per_step(5, 2, 0) == 4
 
 
