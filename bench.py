@@ -9,7 +9,8 @@ once as a CUDA graph; a timed step replays it between two CUDA events on the lau
 Steps are timed one by one; L2 is flushed (a 256 MB write) before each step, outside the
 timed events. A second pass replays the stages as separate graphs with events between them
 for the per-stage breakdown and the grouped FFN's roofline. The end-to-end figure (e2e) calls moe_forward eagerly, with the H2D
-copy of the tokens and the D2H copy of the output inside its timed region. Under torchrun every rank runs its own replica of the workload
+copy of the tokens and the D2H copy of the output of every step inside its timed region; the
+copies run on their own streams and overlap the neighbouring steps' compute. Under torchrun every rank runs its own replica of the workload
 (weak scaling, no collective on the data path). Rank 0 prints the line, with the time taken
 as the max over ranks.
 
@@ -299,13 +300,49 @@ class Layer:
             g.replay()
             ev[n + 1].record()
 
-    def forward_host(self, x_host, out_host):
-        """End to end through the public call: H2D of x, moe_forward, D2H of out."""
-        x = self.inp["x"]
-        x.copy_(x_host, non_blocking=True)
-        self.moe.forward_into(self.dims, x, self.inp["w_router"], self.inp["logit_bias"],
-                              self.inp["w_gate_up"], self.inp["w_down"], x, self.out, self.fws)
-        out_host.copy_(self.out, non_blocking=True)
+    def e2e_pipeline(self, steps: int, warmup: int):
+        """End to end through the public call, as a serving loop would run it: every step
+        copies its tokens from pinned host memory (H2D), runs moe_forward, and copies the
+        output back (D2H). H2D, compute and D2H use three streams and two device buffers, so
+        the copies of neighbouring steps overlap the compute. Returns the elapsed ms of
+        `steps` steps (after `warmup` untimed ones), measured from the first H2D to the last
+        D2H on the device."""
+        moe, i = self.moe, self.inp
+        T, d = self.T, self.shape.d_model
+        x_host = [i["x"].cpu().pin_memory() for _ in range(2)]
+        out_host = [torch.empty((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        x_dev = [torch.empty_like(i["x"]) for _ in range(2)]
+        out_dev = [torch.empty_like(i["x"]) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        s_comp = torch.cuda.current_stream()
+        ev = lambda: torch.cuda.Event()
+        h2d_done, comp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        for e in comp_done + d2h_done:
+            e.record(s_comp)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for n in range(warmup + steps):
+            b = n % 2
+            if n == warmup:
+                s_in.wait_stream(s_comp)
+                s_in.wait_stream(s_out)
+                t0.record(s_in)
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(comp_done[b])        # step n-2 no longer reads x_dev[b]
+                x_dev[b].copy_(x_host[b], non_blocking=True)
+                h2d_done[b].record(s_in)
+            s_comp.wait_event(h2d_done[b])
+            s_comp.wait_event(d2h_done[b])           # step n-2's output has left out_dev[b]
+            moe.forward_into(self.dims, x_dev[b], i["w_router"], i["logit_bias"], i["w_gate_up"],
+                             i["w_down"], x_dev[b], out_dev[b], self.fws, stream=s_comp)
+            comp_done[b].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[b])
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                d2h_done[b].record(s_out)
+        s_comp.wait_stream(s_out)
+        t1.record(s_comp)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
 
 
 def reduce_max(values, world: int, device) -> list:
@@ -377,21 +414,10 @@ def run_gpu(args, rank, world, local_rank):
                 for i, n in enumerate(["route", "permute", "grouped_ffn", "combine"])}
     ffn_ms = stage_ms["grouped_ffn"]
 
-    # end to end through the public call with host buffers
-    x_host = layer.inp["x"].cpu().pin_memory()
-    out_host = torch.empty_like(x_host).pin_memory()
-    for _ in range(args.warmup):
-        layer.forward_host(x_host, out_host)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # end to end through the public call with host buffers (copies overlap neighbouring steps)
     if world > 1:
         torch.distributed.barrier()
-    e0.record()
-    for _ in range(args.steps):
-        layer.forward_host(x_host, out_host)
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = layer.e2e_pipeline(args.steps, args.warmup)
 
     total_ms, e2e_ms = reduce_max([total_ms, e2e_ms], world, device)
 
