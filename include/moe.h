@@ -94,7 +94,8 @@ int64_t moe_max_rows(const moe_dims* dims);
  *   - one region shared by the stages, which run one after another on the stream:
  *       - the capacity scan's chunk totals;
  *       - the router's bf16 three-term split of W_r, on the tensor-core path;
- *       - the grouped FFN's split-K partial tiles.
+ *       - the grouped FFN's split-K partial tiles;
+ *       - moe_router_stats's partial sums.
  * Zero a workspace once before its first use, with moe_workspace_init or any memset to 0.
  * Zero it again after a device error. */
 moe_status moe_workspace_bytes(const moe_dims* dims, size_t* bytes);
@@ -163,6 +164,22 @@ moe_status moe_unpermute_combine(const moe_dims* dims, const float* y_perm,
                                  const int32_t* row_of_pair, const float* topk_w,
                                  const uint16_t* residual, void* out, int32_t out_f32, void* ws,
                                  size_t ws_bytes, void* stream);
+
+/* Router statistics and the auxiliary load-balancing loss (page «Sparse Mixture-of-Experts»,
+ * section «Маршрутизация токена и auxiliary loss»; the loss is alpha * N * sum_i f_i * P_i).
+ *   logits    [T, N] fp32            the router logits (from moe_route)
+ *   topk_idx  [T, k] int32, slot [T, k] int32   the routing (from moe_route)
+ *   alpha                             loss coefficient (the page reports 1e-2 as best)
+ *   picks     [N] int32 (out)         pairs that chose expert e, before the capacity limit
+ *   prob_mean [N] fp32 (out)          P_e: the mean over the batch of softmax(logits)_e
+ *   aux_loss  [1] fp32 (out)          alpha * N * sum_e (picks_e / T) * P_e; f_e counts a token
+ *                                     once for each of its chosen experts (sum_e f_e = k)
+ *   dropped   [1] int32 (out)         pairs with slot -1
+ * Deterministic: partial sums are added in a fixed order. Uses the per-stage workspace. */
+moe_status moe_router_stats(const moe_dims* dims, const float* logits, const int32_t* topk_idx,
+                            const int32_t* slot, float alpha, int32_t* picks, float* prob_mean,
+                            float* aux_loss, int32_t* dropped, void* ws, size_t ws_bytes,
+                            void* stream);
 
 /* Pointers into a moe_forward workspace (all device pointers; sizes as in the calls above). */
 typedef struct {

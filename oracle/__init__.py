@@ -7,4 +7,4 @@ from .moe_oracle import *  # noqa: F401,F403
 from .moe_oracle import (capacity_from_factor, router_logits, softmax_over_experts,  # noqa: F401
                          select_top_k, renormalise, assign_capacity_slots, route_from_logits,
                          expert_permutation, silu, gelu, expert_ffn, combine,
-                         moe_layer_forward)
+                         moe_layer_forward, router_statistics)

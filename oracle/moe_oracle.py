@@ -254,3 +254,31 @@ def moe_layer_forward(x: np.ndarray, w_router: np.ndarray, w_gate_up: ExpertWeig
     routing = route_from_logits(logits, top_k, capacity)
     out = combine(x, routing, w_gate_up, w_down, act, residual, tokens)
     return {"logits": logits, "out": out, **routing}
+
+
+# --------------------------------------------------------------------------
+# router statistics and the auxiliary load-balancing loss
+# (page «Sparse Mixture-of-Experts», section «Маршрутизация токена и auxiliary loss»;
+#  the auxiliary_loss function of the second demo script)
+# --------------------------------------------------------------------------
+def router_statistics(logits: np.ndarray, topk_idx: np.ndarray, slot: np.ndarray,
+                      alpha: float = 1e-2) -> dict:
+    """Per-expert load and router confidence over the batch, and the auxiliary loss.
+
+    picks[e]     number of (token, choice) pairs that chose expert e, before the capacity
+    prob_mean[e] P_e: mean over the batch of the router's softmax probability of expert e
+    f[e]         fraction of the batch's tokens sent to expert e: picks[e] / T
+    aux_loss     alpha * N * sum_e f[e] * P_e
+    dropped      number of pairs that found their expert full
+    """
+    T, N = logits.shape
+    probs = softmax_over_experts(logits)
+    picks = np.zeros(N, dtype=np.int64)
+    for t in range(T):
+        for e in topk_idx[t]:
+            picks[int(e)] += 1
+    prob_mean = probs.mean(axis=0)
+    f = picks / T
+    aux = alpha * N * float((f * prob_mean).sum())
+    return {"picks": picks, "prob_mean": prob_mean, "aux_loss": aux,
+            "dropped": int((np.asarray(slot) < 0).sum())}

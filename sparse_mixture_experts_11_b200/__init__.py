@@ -69,6 +69,8 @@ _SIGS = {
     "moe_forward_layout": (ctypes.c_int, [_DIMS, _P, ctypes.c_size_t, ctypes.POINTER(ForwardBuffers)]),
     "moe_forward": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_route_noalloc": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_router_stats": (ctypes.c_int, [_DIMS, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P,
+                                        ctypes.c_size_t, _P]),
     "moe_read_device_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int)]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -250,6 +252,20 @@ def unpermute_combine(dims: Dims, y_perm, row_of_pair, topk_w, residual, out, ws
         _ptr(out, "out", None, (T, d)), 1 if out.dtype == torch.float32 else 0,
         _ptr(ws, "ws", torch.uint8, allow_none=True), _nbytes(ws), _stream(stream)),
         "moe_unpermute_combine")
+
+
+def router_stats(dims: Dims, logits, topk_idx, slot, picks, prob_mean, aux_loss, dropped, ws,
+                 alpha: float = 1e-2, stream=None) -> None:
+    """Per-expert picks and mean router probability, dropped pairs, and the auxiliary loss
+    alpha * N * sum_e (picks_e / T) * P_e."""
+    T, N, k = dims.T, dims.n_experts, dims.top_k
+    _check(_lib.moe_router_stats(
+        ctypes.byref(dims), _ptr(logits, "logits", torch.float32, (T, N)),
+        _ptr(topk_idx, "topk_idx", torch.int32, (T, k)), _ptr(slot, "slot", torch.int32, (T, k)),
+        float(alpha), _ptr(picks, "picks", torch.int32, (N,)),
+        _ptr(prob_mean, "prob_mean", torch.float32, (N,)),
+        _ptr(aux_loss, "aux_loss", torch.float32, (1,)), _ptr(dropped, "dropped", torch.int32, (1,)),
+        _ptr(ws, "ws", torch.uint8), _nbytes(ws), _stream(stream)), "moe_router_stats")
 
 
 def forward_into(dims: Dims, x, w_router, logit_bias, w_gate_up, w_down, residual, out, ws,

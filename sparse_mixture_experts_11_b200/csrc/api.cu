@@ -100,7 +100,10 @@ moe::FfnScratchPlan ffn_plan(const moe_dims* d) {
 size_t counters_bytes(const moe_dims* d) { return round_up(ffn_plan(d).counter_bytes, 256); }
 
 size_t shared_region_bytes(const moe_dims* d) {
-  return std::max(slot_scratch_bytes(d) + split_scratch_bytes(d), round_up(ffn_plan(d).part_bytes, 256));
+  const size_t routing = slot_scratch_bytes(d) + split_scratch_bytes(d);
+  const size_t ffn = round_up(ffn_plan(d).part_bytes, 256);
+  const size_t stats = round_up(moe::router_stats_scratch_bytes(d->T, d->n_experts), 256);
+  return std::max(std::max(routing, ffn), stats);
 }
 
 size_t stage_ws_bytes(const moe_dims* d) {
@@ -280,6 +283,26 @@ moe_status moe_unpermute_combine(const moe_dims* dims, const float* y_perm,
   return launch_status(moe::launch_combine(y_perm, row_of_pair, topk_w, residual, out, out_f32,
                                            dims->T, dims->d_model, dims->top_k, rmax,
                                            ws ? status_of(ws) : nullptr, as_stream(stream)));
+}
+
+moe_status moe_router_stats(const moe_dims* dims, const float* logits, const int32_t* topk_idx,
+                            const int32_t* slot, float alpha, int32_t* picks, float* prob_mean,
+                            float* aux_loss, int32_t* dropped, void* ws, size_t ws_bytes,
+                            void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (dims->T == 0) return MOE_OK;
+  if (!logits || !topk_idx || !slot || !picks || !prob_mean || !aux_loss || !dropped || !ws)
+    return MOE_ERR_INVALID;
+  if (!aligned16(logits) || !aligned16(topk_idx) || !aligned16(slot) || !aligned16(picks) ||
+      !aligned16(prob_mean) || !aligned16(ws))
+    return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < stage_ws_bytes(dims)) return MOE_ERR_WORKSPACE;
+  if ((st = check_device()) != MOE_OK) return st;
+  return launch_status(moe::launch_router_stats(logits, topk_idx, slot, alpha, picks, prob_mean,
+                                                aux_loss, dropped, shared_region_of(dims, ws),
+                                                dims->T, dims->n_experts, dims->top_k,
+                                                as_stream(stream)));
 }
 
 moe_status moe_forward_workspace_bytes(const moe_dims* dims, size_t* bytes) {

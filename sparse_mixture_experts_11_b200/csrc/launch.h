@@ -76,6 +76,13 @@ cudaError_t launch_combine(const float* y_perm, const int32_t* row_of_pair, cons
                            const uint16_t* residual, void* out, int out_f32, int T, int d, int k,
                            int64_t r_max, int* status, cudaStream_t s);
 
+// router statistics and the auxiliary loss (two deterministic passes)
+size_t router_stats_scratch_bytes(int T, int N);
+cudaError_t launch_router_stats(const float* logits, const int32_t* topk_idx, const int32_t* slot,
+                                float alpha, int32_t* picks, float* prob_mean, float* aux_loss,
+                                int32_t* dropped, void* scratch, int T, int N, int k,
+                                cudaStream_t s);
+
 // grouped expert GEMMs on tcgen05
 //
 // Scratch of the grouped FFN for split-K, used only for decode-sized batches (R_max <= 256):

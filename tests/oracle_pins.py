@@ -273,7 +273,36 @@ def pin_active_params_demo(o_unused=None):
     assert router + N * expert == g["total"]
 
 
+# ----------------------------------------------------------------- router statistics
+def pin_aux_loss_closed_forms(o):
+    alpha = 0.01
+    # equal logits and a round-robin top-1 routing: f_i = P_i = 1/N, so the loss is alpha
+    T, N = 16, 8
+    L = np.zeros((T, N))
+    idx = (np.arange(T) % N)[:, None]
+    st = o.router_statistics(L, idx, np.zeros((T, 1)), alpha)
+    assert abs(st["aux_loss"] - alpha) < 1e-15
+    np.testing.assert_allclose(st["prob_mean"], 1.0 / N, atol=1e-15)
+    assert st["picks"].tolist() == [2] * N and st["dropped"] == 0
+    # collapse: every token sends to expert 0 with probability ~1: the loss tends to alpha * N
+    L = np.zeros((T, N))
+    L[:, 0] = 60.0
+    st = o.router_statistics(L, np.zeros((T, 1), dtype=np.int64), np.full((T, 1), -1), alpha)
+    assert abs(st["aux_loss"] - alpha * N) < 1e-12
+    assert st["dropped"] == T
+    # by hand: t0 = (0, 0) -> p = (1/2, 1/2); t1 = (ln 3, 0) -> p = (3/4, 1/4); both pick
+    # expert 0, so f = (1, 0), P = (5/8, 3/8) and the loss is alpha * 2 * 5/8 = 1.25 alpha
+    L = np.array([[0.0, 0.0], [math.log(3.0), 0.0]])
+    st = o.router_statistics(L, np.array([[0], [0]]), np.array([[0], [1]]), alpha)
+    np.testing.assert_allclose(st["prob_mean"], [0.625, 0.375], atol=1e-15)
+    assert abs(st["aux_loss"] - 1.25 * alpha) < 1e-15
+    # top-2 counts each chosen expert once per token
+    st = o.router_statistics(np.zeros((3, 4)), np.array([[0, 1], [1, 2], [3, 0]]),
+                             np.array([[0, -1], [0, 0], [0, -1]]), alpha)
+    assert st["picks"].tolist() == [2, 2, 1, 1] and st["dropped"] == 2
+
+
 ALL_PINS = [pin_capacity_demo, pin_capacity_formula, pin_hand_routing, pin_top1_weight_is_one,
             pin_two_way_weights, pin_brute_force_routing, pin_ffn_hand_cases,
             pin_activation_limits, pin_dense_special_case, pin_single_expert_layer,
-            pin_invariants, pin_zero_down_weights]
+            pin_invariants, pin_zero_down_weights, pin_aux_loss_closed_forms]

@@ -90,6 +90,22 @@ def _combine_drops_residual(x, routing, wgu, wd, act, residual, tokens=None):
     return _orig_combine(x, routing, wgu, wd, act, None, tokens)
 
 
+def _aux_without_n(logits, topk_idx, slot, alpha=1e-2):
+    st = _orig_stats(logits, topk_idx, slot, alpha)
+    st["aux_loss"] /= logits.shape[1]
+    return st
+
+
+def _aux_f_over_tk(logits, topk_idx, slot, alpha=1e-2):
+    st = _orig_stats(logits, topk_idx, slot, alpha)
+    st["aux_loss"] /= topk_idx.shape[1]
+    st["picks"] = st["picks"] // topk_idx.shape[1]
+    return st
+
+
+_orig_stats = om.router_statistics
+
+
 _orig_combine = om.combine
 
 MUTANTS = {
@@ -104,6 +120,8 @@ MUTANTS = {
     "capacity_times_k": ("capacity_from_factor", _capacity_times_k),
     "softmax_wrong_axis": ("softmax_over_experts", _softmax_no_shift_wrong_axis),
     "residual_dropped": ("combine", _combine_drops_residual),
+    "aux_without_N": ("router_statistics", _aux_without_n),
+    "aux_f_over_Tk": ("router_statistics", _aux_f_over_tk),
 }
 
 
@@ -118,3 +136,4 @@ def test_some_pin_catches(name, monkeypatch):
         except (AssertionError, ValueError, IndexError):
             caught.append(pin.__name__)
     assert caught, f"mutant {name} passed every pin"
+
