@@ -236,6 +236,36 @@ class Layer:
                 "y_perm": self._view(b.y_perm, R * d, torch.float32).view(R, d),
                 "stage_ws": self._view(b.stage_ws, b.stage_ws_bytes, torch.uint8)}
 
+    def stats_timing(self, steps: int, flush) -> dict:
+        """moe_router_stats on the step's logits and routing: mean ms per call and its
+        algorithmic bandwidth (logits, indices and slots read once)."""
+        moe, v = self.moe, self.views()
+        N, k, T = self.shape.n_experts, self.shape.top_k, self.T
+        picks = torch.empty((N,), dtype=torch.int32, device=v["logits"].device)
+        pm = torch.empty((N,), dtype=torch.float32, device=picks.device)
+        aux = torch.empty((1,), dtype=torch.float32, device=picks.device)
+        dropped = torch.empty((1,), dtype=torch.int32, device=picks.device)
+        call = lambda: moe.router_stats(self.dims, v["logits"], v["topk_idx"], v["slot"], picks, pm,
+                                        aux, dropped, v["stage_ws"], alpha=0.01)
+        call()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for e0, e1 in evs:
+            flush_l2(flush)
+            e0.record()
+            g.replay()
+            e1.record()
+        torch.cuda.synchronize()
+        ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+        nbytes = T * N * 4 + 2 * T * k * 4
+        return {"ms": round(ms, 4), "aux_loss": round(float(aux.item()), 6),
+                "dropped_pairs": int(dropped.item()), "algorithmic_bytes": nbytes,
+                "achieved_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+
     def stage_calls(self):
         """The four stage calls of one forward (the calls moe_forward makes), as closures."""
         moe, i, b, dims = self.moe, self.inp, self.b, self.dims
@@ -414,6 +444,10 @@ def run_gpu(args, rank, world, local_rank):
                 for i, n in enumerate(["route", "permute", "grouped_ffn", "combine"])}
     ffn_ms = stage_ms["grouped_ffn"]
 
+    # router statistics and the auxiliary loss over this step's routing (a "next" row),
+    # replayed as a graph K times between events
+    stats = layer.stats_timing(args.steps, flush)
+
     # end to end through the public call with host buffers (copies overlap neighbouring steps)
     if world > 1:
         torch.distributed.barrier()
@@ -462,6 +496,7 @@ def run_gpu(args, rank, world, local_rank):
                              "by programmatic dependent launch); stages_ms and roofline: the same "
                              "steps replayed as one graph per stage with events between stages"},
         "stages_ms": {k: round(v_, 4) for k, v_ in stage_ms.items()},
+        "router_stats": stats,
         "roofline": roof,
         "layer_gbs": round(ab["layer"] / (total_ms / args.steps * 1e-3) / 1e9, 1),
         "ffn_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 2),

@@ -102,7 +102,23 @@ __global__ void __launch_bounds__(256) stats_final_kernel(
   for (int e = threadIdx.x; e < N; e += blockDim.x) {
     float s = 0.f;
     int c = 0;
-    for (int b = 0; b < n_parts; ++b) {  // block order: deterministic
+    // block order (deterministic); eight independent loads in flight per step
+    int b = 0;
+    for (; b + 8 <= n_parts; b += 8) {
+      float v[8];
+      int u[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[i] = part_prob[static_cast<int64_t>(b + i) * N + e];
+        u[i] = part_picks[static_cast<int64_t>(b + i) * N + e];
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        s += v[i];
+        c += u[i];
+      }
+    }
+    for (; b < n_parts; ++b) {
       s += part_prob[static_cast<int64_t>(b) * N + e];
       c += part_picks[static_cast<int64_t>(b) * N + e];
     }
@@ -116,7 +132,7 @@ __global__ void __launch_bounds__(256) stats_final_kernel(
     float total = 0.f;
     for (int e = 0; e < N; ++e) total += s_term[e];
     int d = 0;
-    for (int b = 0; b < n_parts; ++b) d += part_dropped[b];
+    for (int b2 = 0; b2 < n_parts; ++b2) d += part_dropped[b2];
     *aux_loss = alpha * static_cast<float>(N) * total;
     *dropped = d;
   }
