@@ -244,6 +244,15 @@ moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x, const floa
  * (For a moe_forward workspace pass moe_forward_buffers.stage_ws.) */
 moe_status moe_read_device_error(void* ws, void* stream, moe_status* err);
 
+/* Diagnostics: set the limit, in nanoseconds, of every bounded wait inside the library's
+ * tensor-core kernels, for calls made afterwards in this process; 0 restores the default of
+ * 2 s. Returns the previous limit. A limit too short for the work makes the kernels stop
+ * early and record MOE_ERR_TIMEOUT in the workspace status word. Their outputs are then
+ * undefined, and the workspace must be zeroed again (moe_workspace_init). Copies and MMAs
+ * already in flight are still waited for, under a separate 1 s limit, before a CTA exits.
+ * Meant for testing the error path. */
+uint64_t moe_debug_set_wait_timeout_ns(uint64_t ns);
+
 /* Static description of a status code. */
 const char* moe_status_string(moe_status s);
 

@@ -72,6 +72,7 @@ _SIGS = {
     "moe_router_stats": (ctypes.c_int, [_DIMS, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P,
                                         ctypes.c_size_t, _P]),
     "moe_read_device_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int)]),
+    "moe_debug_set_wait_timeout_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -113,6 +114,11 @@ def _nbytes(t: Optional[torch.Tensor]) -> int:
 
 
 # ----------------------------------------------------------------------------- host helpers
+def debug_set_wait_timeout_ns(ns: int) -> int:
+    """Limit of the kernels' bounded waits for later calls (0 = default 2 s); returns the old one."""
+    return int(_lib.moe_debug_set_wait_timeout_ns(int(ns)))
+
+
 def status_string(status: int) -> str:
     return _lib.moe_status_string(int(status)).decode()
 

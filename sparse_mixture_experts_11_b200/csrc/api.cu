@@ -12,6 +12,8 @@
 
 namespace moe {
 
+std::atomic<uint64_t> g_wait_timeout_ns{kDefaultWaitTimeoutNs};
+
 namespace {
 constexpr int kMaxDevices = 64;
 DeviceInfo g_info[kMaxDevices];
@@ -20,6 +22,8 @@ cudaError_t g_info_err[kMaxDevices];
 
 
 }  // namespace
+
+uint64_t wait_timeout_ns() { return g_wait_timeout_ns.load(std::memory_order_relaxed); }
 
 cudaError_t device_info(DeviceInfo* out) {
   int dev = 0;
@@ -180,7 +184,7 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const float* w_rou
   st = launch_status(moe::launch_router_topk(x, w_router, logit_bias, logits, topk_idx, topk_w,
                                              dims->T, dims->d_model, dims->n_experts,
                                              dims->top_k, split_scratch_of(dims, ws), status_of(ws),
-                                             moe::kDefaultWaitTimeoutNs, s));
+                                             moe::wait_timeout_ns(), s));
   if (st != MOE_OK) return st;
   return route_slots(dims, topk_idx, slot, expert_count, ws, s);
 }
@@ -255,7 +259,7 @@ moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
   a.act = dims->act;
   a.r_max = rmax;
   a.status = status_of(ws);
-  a.timeout_ns = moe::kDefaultWaitTimeoutNs;
+  a.timeout_ns = moe::wait_timeout_ns();
   a.rows_per_expert = std::min(dims->capacity, dims->T);
   const moe::FfnScratchPlan plan = ffn_plan(dims);
   if (plan.max_splits1 > 1 || plan.max_splits2 > 1) {
@@ -386,6 +390,10 @@ moe_status moe_read_device_error(void* ws, void* stream, moe_status* err) {
   if (cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
   *err = static_cast<moe_status>(v);
   return MOE_OK;
+}
+
+uint64_t moe_debug_set_wait_timeout_ns(uint64_t ns) {
+  return moe::g_wait_timeout_ns.exchange(ns == 0 ? moe::kDefaultWaitTimeoutNs : ns);
 }
 
 const char* moe_status_string(moe_status s) {

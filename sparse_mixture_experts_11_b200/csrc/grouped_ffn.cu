@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // No TMA write may still be landing in shared memory when the CTA exits.
       for (int i = max(0, it - C::STAGES); i < it; ++i)
-        mbar_wait(smem_u32(&full_bar[i % C::STAGES]), (i / C::STAGES) & 1, p.timeout_ns, nullptr);
+        mbar_wait(smem_u32(&full_bar[i % C::STAGES]), (i / C::STAGES) & 1, kDrainTimeoutNs, nullptr);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -402,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         report_error(p.status, MOE_ERR_TIMEOUT);
         if (issued) {  // let every issued MMA finish before TMEM is freed
           tc_commit(smem_u32(&done_bar));
-          mbar_wait(smem_u32(&done_bar), 0, p.timeout_ns, nullptr);
+          mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
         }
       }
     }

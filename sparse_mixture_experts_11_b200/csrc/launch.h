@@ -29,6 +29,11 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 constexpr size_t kStatusBytes = 256;
 constexpr int kSlotChunk = 4096;  // (token, choice) pairs ranked per block in the slot pass
 constexpr uint64_t kDefaultWaitTimeoutNs = 2000000000ull;  // limit of one mbarrier wait (2 s)
+// Limit of the waits a CTA makes, after giving up, for its own TMA copies and MMAs still in
+// flight (independent of the wait limit above, so a short limit never cuts the drain short).
+constexpr uint64_t kDrainTimeoutNs = 1000000000ull;
+// The wait limit the entry points pass to the kernels (moe_debug_set_wait_timeout_ns).
+uint64_t wait_timeout_ns();
 
 inline int64_t slot_chunks(int64_t pairs) { return (pairs + kSlotChunk - 1) / kSlotChunk; }
 

@@ -83,7 +83,7 @@ extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x,
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (moe::launch_router_topk(x, w_router, logit_bias, logits, topk_idx, topk_w, dims->T,
                               dims->d_model, dims->n_experts, dims->top_k, nullptr, nullptr,
-                              moe::kDefaultWaitTimeoutNs, s) != cudaSuccess)
+                              moe::wait_timeout_ns(), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   const int cap = dims->capacity < dims->T ? dims->capacity : dims->T;
   if (moe::launch_capacity_slots(topk_idx, slot, expert_count, scratch, dims->T, dims->n_experts,

@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         report_error(status, MOE_ERR_TIMEOUT);
       }
       for (int i = max(0, kb - C::STAGES); i < kb; ++i)
-        mbar_wait(smem_u32(&a_full[i % C::STAGES]), (i / C::STAGES) & 1, timeout_ns, nullptr);
+        mbar_wait(smem_u32(&a_full[i % C::STAGES]), (i / C::STAGES) & 1, kDrainTimeoutNs, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         report_error(status, MOE_ERR_TIMEOUT);
         if (issued) {
           tc_commit(smem_u32(&done_bar));
-          mbar_wait(smem_u32(&done_bar), 0, timeout_ns, nullptr);
+          mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
         }
       }
     }
