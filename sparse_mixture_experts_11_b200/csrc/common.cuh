@@ -96,16 +96,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase with the given parity has completed. Gives up (returns false) when
 // `timeout_ns` of wall-clock time pass, or when *abort becomes non-zero (abort may be null).
+// try_wait itself suspends the thread for a while before reporting failure, so the clock and
+// the abort flag are checked after every failed attempt.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
                                           const volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t n = 1;; ++n) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 31u) == 0) {
-      if (abort != nullptr && *abort != 0) return false;
-      if (globaltimer_ns() - t0 > timeout_ns) return false;
-    }
+    if (abort != nullptr && *abort != 0) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
   }
 }
 
