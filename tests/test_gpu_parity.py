@@ -149,3 +149,18 @@ def test_empty_batch_is_a_no_op():
     out = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
     moe.forward_into(dims, x, wr, None, wgu, wd, x, out, ws)
     torch.cuda.synchronize()
+
+
+def test_k_scaled_capacity():
+    """Overflow-policy variant: capacity scaled by k, ceil(cf * k * T / N), passed through the
+    capacity field (fine-grained-like shape: N=256, k=8, Zipf-skewed loads)."""
+    import math
+    T, d, N, k, F = 600, 256, 256, 8, 128
+    inp = _inputs(T, d, N, F, "swiglu", 1.1, seed=21)
+    cap = int(math.ceil(1.25 * k * T / N))
+    run = H.StageRun(inp, k, "swiglu", cap).run()
+    routing, off, rop = H.check_routing(run, cap)
+    H.check_x_perm(run, rop)
+    H.check_outputs(run, routing, "swiglu")
+    H.check_dropped_tokens_pass_through(run, routing["slot"])
+    assert int((routing["slot"] < 0).sum()) > 0  # the Zipf skew still overflows hot experts
