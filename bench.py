@@ -95,19 +95,29 @@ def router_on_tensor_cores(T: int, n_experts: int, d_model: int) -> bool:
     return T * n_experts * d_model * 4 > 268435456
 
 
+DECODE_ROUTE_MAX_T = 16           # batches routed (and, when small, sorted) in one launch
+DECODE_PERMUTE_MAX_BYTES = 512 * 1024
+
+
 def launches_per_step(T: int, k: int, R_max: int, n_experts: int = 1, d_model: int = 1) -> int:
-    """Kernels one forward launches: router + top-k (plus the W_r split kernel on the
-    tensor-core path), capacity slots (1 pass, or 3 when the arrivals span several chunks),
-    permute, two grouped GEMMs (when rows can exist), combine."""
+    """Kernels one forward (moe_forward) launches. Decode-sized batches (T <= 16): one routing
+    launch (router, top-k and slots), which also sorts by expert while x_perm is at most
+    512 KB, else a permute launch. Larger batches: router + top-k (plus the W_r split kernel
+    on the tensor-core path), capacity slots (1 pass, or 3 when the arrivals span several
+    chunks), permute. Then the grouped FFN (both GEMMs in one launch, when rows can exist)
+    and the combine."""
+    ffn = (1 if R_max > 0 else 0) + 1
+    if 1 <= T <= DECODE_ROUTE_MAX_T:
+        return 1 + (0 if R_max * d_model * 2 <= DECODE_PERMUTE_MAX_BYTES else 1) + ffn
     chunks = max(1, math.ceil(T * k / SLOT_CHUNK))
     router = 2 if router_on_tensor_cores(T, n_experts, d_model) else 1
-    return router + (1 if chunks == 1 else 3) + 1 + (2 if R_max > 0 else 0) + 1
+    return router + (1 if chunks == 1 else 3) + 1 + ffn
 
 
 # DRAM traffic of the grouped-FFN stage per forward (dram__bytes_read.sum +
-# dram__bytes_write.sum of its two GEMM launches) from one ncu capture of the current kernels;
-# workloads without a capture report null.
-MEASURED_FFN_TRAFFIC = {("switch_top1", 4096): 1124.6e6, ("mixtral", 1): 721.1e6}
+# dram__bytes_write.sum of its launch) from one ncu capture of the current kernel; workloads
+# without a capture of the current kernel report null.
+MEASURED_FFN_TRAFFIC = {}
 
 
 def load_peaks():
@@ -297,20 +307,28 @@ class Layer:
                                                  b.stage_ws_bytes, moe._stream(None)), "combine")
         return [route, permute, ffn, combine]
 
+    def forward_call(self):
+        """moe_forward on the layer's inputs (the public call; decode-sized batches route and
+        sort in one launch there, which the stage calls do not)."""
+        i = self.inp
+        self.moe.forward_into(self.dims, i["x"], i["w_router"], i["logit_bias"], i["w_gate_up"],
+                              i["w_down"], i["x"], self.out, self.fws)
+
     def capture_stage_graphs(self):
-        """The forward captured as CUDA graphs: once whole (its kernels overlap through
-        programmatic dependent launch) and once per stage (for the stage breakdown)."""
+        """The forward captured as CUDA graphs: once whole (moe_forward; its kernels overlap
+        through programmatic dependent launch) and once per stage (the four stage calls, for
+        the stage breakdown)."""
         self.graphs = []
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             for call in self.stage_calls():  # one eager pass on the capture stream first
                 call()
+            self.forward_call()
         torch.cuda.current_stream().wait_stream(s)
         self.graph_full = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph_full):
-            for call in self.stage_calls():
-                call()
+            self.forward_call()
         for call in self.stage_calls():
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
@@ -468,7 +486,7 @@ def run_gpu(args, rank, world, local_rank):
         peak = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(ach / peak, 4), "traffic": None,
-                "kernel": "moe_grouped_ffn (gate/up + down GEMM launches)",
+                "kernel": "grouped_ffn_kernel (gate/up and down GEMMs in one launch)",
                 "per_launch": f"{flops} FLOP", "peak_source": peaks["source"] + " sustained bf16"}
     else:
         ach = ab["ffn"] / (ffn_ms * 1e-3) / 1e9
@@ -476,7 +494,7 @@ def run_gpu(args, rank, world, local_rank):
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(ach / peak, 4),
                 "traffic": MEASURED_FFN_TRAFFIC.get((shape.name, T)),
-                "kernel": "moe_grouped_ffn (gate/up + down GEMM launches)",
+                "kernel": "grouped_ffn_kernel (gate/up and down GEMMs in one launch)",
                 "per_launch": f"{ab['ffn']} B", "peak_source": peaks["source"] + " copy"}
 
     value = tokens_per_second(T, args.steps, world, total_ms)

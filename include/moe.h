@@ -89,12 +89,12 @@ int64_t moe_max_rows(const moe_dims* dims);
 /* Bytes of the per-stage workspace `ws` taken by moe_route, moe_route_from_logits,
  * moe_permute, moe_grouped_ffn and moe_unpermute_combine. Host-only. Its regions:
  *   - the device status word (first 256 bytes);
- *   - the grouped FFN's per-tile arrival counters for split-K. These are used only when
- *     R_max <= 256 and must be zero between calls;
+ *   - the grouped FFN's per-tile arrival counters for its stream-K schedule. They must be
+ *     zero between calls (each call leaves them zero);
  *   - one region shared by the stages, which run one after another on the stream:
  *       - the capacity scan's chunk totals;
  *       - the router's bf16 three-term split of W_r, on the tensor-core path;
- *       - the grouped FFN's split-K partial tiles;
+ *       - the grouped FFN's stream-K partial tiles (two per CTA);
  *       - moe_router_stats's partial sums.
  * Zero a workspace once before its first use, with moe_workspace_init or any memset to 0.
  * Zero it again after a device error. */
@@ -146,9 +146,11 @@ moe_status moe_permute(const moe_dims* dims, const uint16_t* x, const int32_t* t
  *   h          [R_max, F] bf16 (out)   act(x_perm W_gu^T) in fp32, rounded once to bf16
  *   y_perm     [R_max, d_model] fp32 (out)  h W_d^T with fp32 accumulation
  * Rows >= R of h and y_perm are not written. Experts with no kept rows cost nothing.
- * Decode-sized batches (R_max <= 256) may split the K dimension of a GEMM across CTAs to use
- * every SM. Each split's fp32 partial tile goes to the workspace. The last split to finish
- * a tile adds the partials in a fixed order, so results are deterministic. */
+ * When the tiles do not fill the SMs evenly (decode-sized and mid-sized batches), a GEMM runs
+ * stream-K: its tiles' K blocks, end to end, are cut into one equal range per CTA. A tile
+ * cut by a range boundary gets fp32 partial tiles in the workspace, and the last CTA to finish
+ * it adds them in order of CTA index, so results are deterministic for a given device.
+ * ws_bytes must be at least moe_workspace_bytes(). */
 moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
                            const int32_t* expert_offset, const uint16_t* w_gate_up,
                            const uint16_t* w_down, uint16_t* h, float* y_perm, void* ws,

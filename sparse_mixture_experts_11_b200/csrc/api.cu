@@ -92,19 +92,27 @@ size_t split_scratch_bytes(const moe_dims* d) {
              : 0;
 }
 
+// Partial dot products of the one-launch router of decode-sized batches.
+size_t decode_scratch_bytes(const moe_dims* d) {
+  return moe::use_decode_route(d->T)
+             ? round_up(moe::decode_route_scratch_bytes(d->T, d->n_experts, d->d_model), 256)
+             : 0;
+}
+
 moe::FfnScratchPlan ffn_plan(const moe_dims* d) {
   return moe::ffn_scratch_plan(d->n_experts, d->d_model, d->d_ff, d->act, max_rows(d),
                                std::min(d->capacity, d->T));
 }
 
 // Per-stage workspace:
-//   [status word, 256 B][grouped-FFN tile counters, zero between calls]
-//   [shared region: routing scratch (capacity-scan chunk totals, router weight split) or,
-//    later on the stream, the grouped FFN's split-K partial tiles]
+//   [status word, 256 B][grouped-FFN counters, zero between calls]
+//   [shared region: routing scratch (capacity-scan chunk totals, router weight split, the
+//    decode router's partial dot products) or,
+//    later on the stream, the grouped FFN's stream-K partial tiles]
 size_t counters_bytes(const moe_dims* d) { return round_up(ffn_plan(d).counter_bytes, 256); }
 
 size_t shared_region_bytes(const moe_dims* d) {
-  const size_t routing = slot_scratch_bytes(d) + split_scratch_bytes(d);
+  const size_t routing = slot_scratch_bytes(d) + split_scratch_bytes(d) + decode_scratch_bytes(d);
   const size_t ffn = round_up(ffn_plan(d).part_bytes, 256);
   const size_t stats = round_up(moe::router_stats_scratch_bytes(d->T, d->n_experts), 256);
   return std::max(std::max(routing, ffn), stats);
@@ -124,6 +132,32 @@ uint16_t* split_scratch_of(const moe_dims* d, void* ws) {
 }
 
 int* status_of(void* ws) { return static_cast<int*>(ws); }
+
+// One-launch routing of a decode-sized batch (moe::use_decode_route); the four permute
+// outputs are null unless the same launch also sorts by expert.
+moe::DecodeRouteArgs decode_route_args(const moe_dims* d, const uint16_t* x, const float* w_router,
+                                       const float* bias, float* logits, int32_t* topk_idx,
+                                       float* topk_w, int32_t* slot, int32_t* expert_count,
+                                       void* ws) {
+  moe::DecodeRouteArgs a{};
+  a.x = x;
+  a.w_router = w_router;
+  a.bias = bias;
+  a.logits = logits;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.slot = slot;
+  a.expert_count = expert_count;
+  a.part = reinterpret_cast<float*>(shared_region_of(d, ws) + slot_scratch_bytes(d) +
+                                    split_scratch_bytes(d));
+  a.counter = reinterpret_cast<int*>(static_cast<char*>(ws) + moe::kDecodeCounterOffset);
+  a.T = d->T;
+  a.d = d->d_model;
+  a.N = d->n_experts;
+  a.k = d->top_k;
+  a.cap = std::min(d->capacity, d->T);
+  return a;
+}
 
 moe_status launch_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -181,6 +215,11 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const float* w_rou
   if (ws_bytes < stage_ws_bytes(dims)) return MOE_ERR_WORKSPACE;
   if ((st = check_device()) != MOE_OK) return st;
   const cudaStream_t s = as_stream(stream);
+  if (moe::use_decode_route(dims->T))
+    return launch_status(moe::launch_decode_route(
+        decode_route_args(dims, x, w_router, logit_bias, logits, topk_idx, topk_w, slot,
+                          expert_count, ws),
+        s));
   st = launch_status(moe::launch_router_topk(x, w_router, logit_bias, logits, topk_idx, topk_w,
                                              dims->T, dims->d_model, dims->n_experts,
                                              dims->top_k, split_scratch_of(dims, ws), status_of(ws),
@@ -244,7 +283,7 @@ moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
   if (!aligned16(x_perm) || !aligned16(expert_offset) || !aligned16(w_gate_up) ||
       !aligned16(w_down) || !aligned16(h) || !aligned16(y_perm) || !aligned16(ws))
     return MOE_ERR_UNSUPPORTED;
-  if (ws_bytes < moe::kStatusBytes) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < stage_ws_bytes(dims)) return MOE_ERR_WORKSPACE;
   if ((st = check_device()) != MOE_OK) return st;
   moe::GroupedFfnArgs a{};
   a.x_perm = x_perm;
@@ -262,10 +301,8 @@ moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
   a.timeout_ns = moe::wait_timeout_ns();
   a.rows_per_expert = std::min(dims->capacity, dims->T);
   const moe::FfnScratchPlan plan = ffn_plan(dims);
-  if (plan.max_splits1 > 1 || plan.max_splits2 > 1) {
-    a.part = reinterpret_cast<float*>(shared_region_of(dims, ws));
-    a.tile_counters = reinterpret_cast<int*>(static_cast<char*>(ws) + moe::kStatusBytes);
-  }
+  a.counters = reinterpret_cast<int*>(static_cast<char*>(ws) + moe::kStatusBytes);
+  if (plan.part_bytes > 0) a.part = reinterpret_cast<float*>(shared_region_of(dims, ws));
   return launch_status(moe::launch_grouped_ffn(a, as_stream(stream)));
 }
 
@@ -368,11 +405,28 @@ moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_r
   if (st != MOE_OK) return st;
   if (dims->T == 0) return MOE_OK;
   if (!x || !w_router || !w_gate_up || !w_down || !out) return MOE_ERR_INVALID;
-  st = moe_route(dims, x, w_router, logit_bias, b.logits, b.topk_idx, b.topk_w, b.slot,
-                 b.expert_count, b.stage_ws, b.stage_ws_bytes, stream);
-  if (st != MOE_OK) return st;
-  st = moe_permute(dims, x, b.topk_idx, b.slot, b.expert_count, b.expert_offset, b.row_of_pair,
-                   b.pair_of_row, b.x_perm, b.stage_ws, b.stage_ws_bytes, stream);
+  const int64_t rmax = max_rows(dims);
+  if (moe::use_decode_route(dims->T) &&
+      rmax * dims->d_model * 2 <= moe::kDecodePermuteMaxBytes) {
+    // decode-sized batch: routing and the sort by expert in one launch
+    if (!aligned16(x) || !aligned16(w_router) || (logit_bias && !aligned16(logit_bias)))
+      return MOE_ERR_UNSUPPORTED;
+    if ((st = check_device()) != MOE_OK) return st;
+    moe::DecodeRouteArgs a = decode_route_args(dims, x, w_router, logit_bias, b.logits,
+                                               b.topk_idx, b.topk_w, b.slot, b.expert_count,
+                                               b.stage_ws);
+    a.expert_offset = b.expert_offset;
+    a.row_of_pair = b.row_of_pair;
+    a.pair_of_row = b.pair_of_row;
+    a.x_perm = b.x_perm;
+    st = launch_status(moe::launch_decode_route(a, as_stream(stream)));
+  } else {
+    st = moe_route(dims, x, w_router, logit_bias, b.logits, b.topk_idx, b.topk_w, b.slot,
+                   b.expert_count, b.stage_ws, b.stage_ws_bytes, stream);
+    if (st != MOE_OK) return st;
+    st = moe_permute(dims, x, b.topk_idx, b.slot, b.expert_count, b.expert_offset, b.row_of_pair,
+                     b.pair_of_row, b.x_perm, b.stage_ws, b.stage_ws_bytes, stream);
+  }
   if (st != MOE_OK) return st;
   st = moe_grouped_ffn(dims, b.x_perm, b.expert_offset, w_gate_up, w_down, b.h, b.y_perm,
                        b.stage_ws, b.stage_ws_bytes, stream);

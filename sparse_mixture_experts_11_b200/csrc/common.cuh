@@ -72,6 +72,31 @@ __device__ __forceinline__ void fence_barrier_init() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Orders this thread's generic-proxy global accesses with its async-proxy (TMA) ones: used
+// around data that one CTA stores with plain stores and another reads with a TMA load.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.global.acquire.gpu.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait until *counter >= target (acquire); false on timeout or when *abort is set.
+__device__ __forceinline__ bool wait_counter_at_least(const int* counter, int target,
+                                                      uint64_t timeout_ns,
+                                                      const volatile int* abort) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (ld_acquire_gpu(counter) >= target) return true;
+    if (abort != nullptr && *abort != 0) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+    __nanosleep(32);
+  }
+}
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");

@@ -8,28 +8,45 @@
 // Page «Sparse Mixture-of-Experts», «Архитектура и ключевые особенности»: an expert is an
 // ordinary transformer FFN.
 //
-// Two launches of one persistent kernel template:
-//   1. h = act(x_perm W_gu^T) per expert: SwiGLU silu(x W_g^T) * (x W_u^T), or GELU (erf form);
-//      bf16 inputs, fp32 accumulation in TMEM, activation in fp32, h rounded once to bf16.
-//   2. y_perm = h W_d^T per expert, fp32 out.
+// One persistent launch runs both GEMMs, one phase after the other on every CTA:
+//   phase 0  h = act(x_perm W_gu^T) per expert: SwiGLU silu(x W_g^T) * (x W_u^T), or GELU (erf
+//            form); bf16 inputs, fp32 accumulation in TMEM, activation in fp32, h rounded once
+//            to bf16;
+//   phase 1  y_perm = h W_d^T per expert, fp32 out.
+// A down-projection tile needs its rows of h complete, that is every phase-0 tile of the same
+// expert and m-tile. Each finished phase-0 tile adds one to its m-tile's counter (after its h
+// stores); the producer of a phase-1 tile streams the tile's W_d blocks into the shared-memory
+// ring at once and issues the h loads when the counter is full. So the down projection's
+// weight stream starts as soon as a CTA runs out of phase-0 work, instead of after the whole
+// first GEMM, its kernel boundary and the second kernel's start. Every CTA must be resident at
+// the same time (one CTA per SM, at most one per SM of the grid); each wait is bounded.
 //
 // Kernel structure (one CTA per SM, 192 threads):
-//   warp 0      TMA producer: A tile [128 rows x 64 k] of the expert's rows and the weight tile
-//               [UMMA_N rows x 64 k] into a STAGES-deep ring of 128B-swizzled shared-memory
+//   warp 0      TMA producer: A tile [BM rows x 64 k] of the expert's rows and the weight tile
+//               [256 rows x 64 k] into a STAGES-deep ring of 128B-swizzled shared-memory
 //               stages (mbarrier full/empty pairs). For SwiGLU one B tile is the gate rows
-//               [f0, f0+BN) stacked on the up rows [f0, f0+BN) of the same expert, so one MMA
+//               [f0, f0+128) stacked on the up rows [f0, f0+128) of the same expert, so one MMA
 //               chain produces both halves of the activation's input side by side.
-//   warp 1      allocates TMEM (two accumulator buffers) and issues tcgen05.mma (M=128,
-//               N=UMMA_N, K=16, four per stage) from one thread; tcgen05.commit frees smem
-//               stages and publishes finished accumulators.
+//   warp 1      allocates TMEM (two accumulator buffers) and issues tcgen05.mma (M=BM, N=256,
+//               K=16, four per stage) from one thread; tcgen05.commit frees smem stages and
+//               publishes finished accumulators.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (thread i owns row i of the tile),
 //               activation, conversion and masked global stores; then hand the TMEM buffer
-//               back, so the epilogue of tile i overlaps the mainloop of tile i+1.
+//               back, so the epilogue of one tile overlaps the mainloop of the next.
 // Tile scheduler: tiles are (expert, n-tile, m-tile) with m fastest, numbered expert by
-// expert; the per-expert tile counts come from expert_offset on the device (no host sync),
-// and CTAs stride through the tile list. Experts without rows produce no tiles.
-// Every mbarrier wait is bounded; on timeout the CTA records MOE_ERR_TIMEOUT, stops issuing
-// work, waits (bounded) for its own TMA copies and MMAs, frees TMEM and exits.
+// expert; the per-expert m-tile counts come from expert_offset on the device (no host sync).
+// Experts without rows produce no tiles. Each phase has one of two schedules, chosen on the
+// device from its tile count by a cost model that every CTA evaluates alike:
+//   whole tiles   CTAs stride through the tile list;
+//   stream-K      the tiles' k blocks, laid end to end, are cut into one equal contiguous range
+//                 per CTA, so no CTA idles in a last, partly filled wave. A tile that a range
+//                 boundary cuts gets fp32 partial sums from each CTA that covers part of it;
+//                 its owner (the CTA holding its first k blocks, which it reaches last) waits
+//                 for the others' arrival count and adds the partials in order of CTA index.
+//                 Each CTA holds at most two such partial tiles per phase (its first and its
+//                 last), so the partials take two slots.
+// Every wait is bounded; on timeout the CTA records MOE_ERR_TIMEOUT, stops issuing work, waits
+// (bounded) for its own TMA copies and MMAs, frees TMEM and exits.
 #include <algorithm>
 #include <mutex>
 
@@ -41,53 +58,52 @@ namespace {
 
 // Rows per tile (UMMA M) is a template parameter BM: 128, or 64 when no expert can hold more
 // than 64 rows. For M = 64 the accumulator's row 16q + i (i < 16) sits in TMEM lane 32q + i.
-constexpr int BK = 64;        // k per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int BK = 64;         // k per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int kUmmaN = 256;    // UMMA N of both phases (SwiGLU: 128 gate + 128 up columns)
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr int kSmemBudget = 200 * 1024;
+constexpr int kDnBn = 256;     // output columns per tile of the down projection
 
 enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_STORE_F32 = 2 };
 
-struct GemmParams {
-  const int32_t* expert_offset;  // [N+1]
-  void* out;                     // h (bf16) or y_perm (fp32)
-  int64_t ld_out;                // row stride of out, elements
-  int64_t r_max;
-  int n_experts;
-  int n_out;       // valid output columns per expert (multiple of 16)
-  int n_tiles_n;   // ceil(n_out / BN_OUT)
-  int num_kb;      // K / BK
-  int* status;
-  uint64_t timeout_ns;
-  int weight_policy;  // 0 evict_normal, 1 evict_first
-  // split-K (decode-sized batches): up to max_splits units per tile, each over a slice of K.
-  // Every unit stores its fp32 partial tile into part[split][row][col]; the CTA whose unit
-  // completes a tile last (per-tile arrival counter) adds the partials in order of split and
-  // writes the tile's output. The counters are zero between calls.
-  int max_splits;
+struct PhaseParams {
+  void* out;        // h (bf16) or y_perm (fp32)
+  int64_t ld_out;   // row stride of out, elements
+  int n_out;        // valid output columns per expert (multiple of 16)
+  int n_tiles_n;    // ceil(n_out / BN)
+  int num_kb;       // K / BK
+  // stream-K: 0 disables it; else at most this many CTAs take ranges, each with two partial
+  // slots part[cta][slot][row][kUmmaN] of slot_rows rows. The counters are zero between calls.
+  int sk_ctas;
   float* part;
-  int part_ld;          // columns of a partial row: 2F (gate | up), F, or d
   int* tile_counters;
 };
 
-constexpr int pow2_at_least(int v) {
-  int p = 32;
-  while (p < v) p <<= 1;
-  return p;
-}
+struct FfnParams {
+  const int32_t* expert_offset;  // [N+1]
+  int64_t r_max;
+  int64_t rows_per_expert;       // no expert may hold more rows (partial slots are this tall)
+  int n_experts;
+  int slot_rows;
+  PhaseParams ph[2];
+  int* h_ready;    // per m-tile: phase-0 tiles finished; zero between calls
+  int m_tiles_cap; // entries of h_ready (tile counters hold m_tiles_cap * n_tiles_n)
+  int* done_ctas;  // CTAs finished; the last one zeroes h_ready
+  int* status;
+  uint64_t timeout_ns;
+  int weight_policy;  // 0 evict_normal, 1 evict_first
+};
 
-template <int EPI, int BN_OUT, int BM>
+template <int BM>
 struct Cfg {
-  static constexpr int UMMA_N = (EPI == EPI_SWIGLU) ? 2 * BN_OUT : BN_OUT;
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = UMMA_N * BK * 2;
+  static constexpr int B_BYTES = kUmmaN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (kSmemBudget / STAGE_BYTES) > 8 ? 8 : (kSmemBudget / STAGE_BYTES);
-  static constexpr int TMEM_COLS = pow2_at_least(2 * UMMA_N);
+  static constexpr int TMEM_COLS = 2 * kUmmaN;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
-  static_assert(UMMA_N % 16 == 0 && UMMA_N >= 16 && UMMA_N <= 256, "UMMA N for M=128");
   static_assert(TMEM_COLS <= 512, "two accumulators must fit in TMEM");
-  static_assert(BN_OUT % 16 == 0, "epilogue works in 16-column groups");
   static_assert(STAGES >= 2, "pipeline depth");
   static_assert(BM == 64 || BM == 128, "UMMA M");
 };
@@ -108,55 +124,112 @@ struct TileCoord {
   int m0;     // first row of the tile (global row in x_perm / h)
   int rows;   // valid rows in the tile (<= BM)
   int n0;     // first output column
+  int gm;     // global m-tile index (counter of the rows' h)
 };
 
+// Tile `tile` of a phase with `ntn` n-tiles per m-tile; s_mt[e] = first m-tile of expert e.
 template <int BM>
-__device__ __forceinline__ TileCoord decode_tile(int tile, int N, int bn_out,
-                                                 const int* s_tile_start, const int* s_off) {
-  int lo = 0, hi = N - 1;  // largest e with s_tile_start[e] <= tile
+__device__ __forceinline__ TileCoord decode_tile(int tile, int N, int bn, int ntn,
+                                                 const int* s_mt, const int* s_off) {
+  int lo = 0, hi = N - 1;  // largest e with s_mt[e] * ntn <= tile
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (s_tile_start[mid] <= tile)
+    if (s_mt[mid] * ntn <= tile)
       lo = mid;
     else
       hi = mid - 1;
   }
   TileCoord c;
   c.e = lo;
-  const int local = tile - s_tile_start[lo];
-  const int m_e = s_off[lo + 1] - s_off[lo];
-  const int mt = (m_e + BM - 1) / BM;
+  const int local = tile - s_mt[lo] * ntn;
+  const int mt = s_mt[lo + 1] - s_mt[lo];
   const int nt = local / mt;
   const int mi = local - nt * mt;
   c.m0 = s_off[lo] + mi * BM;
   c.rows = min(BM, s_off[lo + 1] - c.m0);
-  c.n0 = nt * bn_out;
+  c.n0 = nt * bn;
+  c.gm = s_mt[lo] + mi;
   return c;
 }
 
-// Number of K slices per tile. With equal units dealt out in turn to `grid` CTAs, the busiest
-// CTA runs ceil(units / grid) units of (num_kb / splits + kUnitOverheadKb) k-block times; the
-// count minimising that wins, a larger one only when it is at least 5 % faster. Units keep at
-// least 2 k blocks. The same pure function of (tiles, grid) on every CTA, so all agree.
-constexpr float kUnitOverheadKb = 2.0f;  // epilogue, partial round trip and pipeline refill
+// Schedule of one phase. Stream-K gives CTA b < g the k-block iterations
+// [b * total / g, (b + 1) * total / g) of the tiles laid end to end (num_kb per tile).
+struct Sched {
+  int sk;         // 1: stream-K, 0: whole tiles
+  int g;          // CTAs with a stream-K range
+  int tiles;
+  int num_kb;
+  int64_t total;  // tiles * num_kb
+};
 
-__device__ __forceinline__ int choose_splits(int tiles, int grid, int num_kb, int max_splits) {
-  if (max_splits <= 1 || tiles <= 0) return 1;
-  auto cost = [=](int sp) {
-    const int waves = (tiles * sp + grid - 1) / grid;
-    return static_cast<float>(waves) * (static_cast<float>(num_kb) / sp + kUnitOverheadKb);
-  };
-  int best = 1;
-  float best_cost = cost(1);
-  for (int sp = 2; sp <= max_splits && num_kb / sp >= 2; ++sp) {
-    const float c = cost(sp);
-    if (c < 0.95f * best_cost) {
-      best = sp;
-      best_cost = c;
+__device__ __forceinline__ int64_t sk_begin(const Sched& s, int b) {
+  return static_cast<int64_t>(b) * s.total / s.g;
+}
+// The CTA whose range holds iteration i: the largest b with sk_begin(b) <= i.
+__device__ __forceinline__ int sk_cta_of(const Sched& s, int64_t i) {
+  return static_cast<int>(((i + 1) * s.g + s.total - 1) / s.total) - 1;
+}
+
+// Cost, in k-block times, of the busiest CTA: whole tiles take ceil(tiles / grid) waves of
+// num_kb; stream-K takes ceil(total / g) plus the partial round trip of the tile finished
+// last (latency, and a k block's worth of traffic per 32 partial rows). Stream-K is chosen
+// when at least 5 % faster. Ranges keep at least kSkMinKb k blocks.
+constexpr int kSkMinKb = 4;
+constexpr float kTailKb = 2.0f;  // epilogue of the last tile and pipeline refill
+
+__device__ __forceinline__ Sched choose_schedule(int tiles, int grid, int num_kb, int sk_ctas,
+                                                 int slot_rows) {
+  Sched s{0, 0, tiles, num_kb, static_cast<int64_t>(tiles) * num_kb};
+  if (sk_ctas <= 0 || tiles <= 0) return s;
+  const int min_kb = min(kSkMinKb, num_kb);
+  const int64_t by_size = s.total / min_kb;
+  const int64_t g = by_size < min(grid, sk_ctas) ? by_size : min(grid, sk_ctas);
+  if (g < 2) return s;
+  const float dp = static_cast<float>((tiles + grid - 1) / grid) * num_kb + kTailKb;
+  const float fixup = 2.0f + slot_rows / 32.0f;
+  const float sk = static_cast<float>((s.total + g - 1) / g) + kTailKb + fixup;
+  if (sk < 0.95f * dp) {
+    s.sk = 1;
+    s.g = static_cast<int>(g);
+  }
+  return s;
+}
+
+struct Seg {
+  int tile, kb0, kb1;
+};
+
+// Walks this CTA's segments (a tile and a k-block range of it) of one phase in order; the
+// producer, the MMA issuer and the epilogue each run their own copy and see the same sequence.
+struct SegCursor {
+  int64_t it, end;
+  __device__ __forceinline__ SegCursor(const Sched& s) {
+    if (s.sk) {
+      const int b = static_cast<int>(blockIdx.x);
+      it = b < s.g ? sk_begin(s, b) : 0;
+      end = b < s.g ? sk_begin(s, b + 1) : 0;
+    } else {
+      it = blockIdx.x;
+      end = s.tiles;
     }
   }
-  return best;
-}
+  __device__ __forceinline__ bool next(const Sched& s, Seg& g) {
+    if (it >= end) return false;
+    if (s.sk) {
+      g.tile = static_cast<int>(it / s.num_kb);
+      g.kb0 = static_cast<int>(it - static_cast<int64_t>(g.tile) * s.num_kb);
+      const int64_t left = end - it;
+      g.kb1 = left < s.num_kb - g.kb0 ? g.kb0 + static_cast<int>(left) : s.num_kb;
+      it += g.kb1 - g.kb0;
+    } else {
+      g.tile = static_cast<int>(it);
+      g.kb0 = 0;
+      g.kb1 = s.num_kb;
+      it += gridDim.x;
+    }
+    return true;
+  }
+};
 
 // Barrier of the 128 epilogue threads on a reusable mbarrier (count 128), bounded like every
 // other wait so that no thread can be left waiting for a warp that gave up.
@@ -181,7 +254,7 @@ __device__ __forceinline__ void store_f32x16(float* dst, const float (&a)[16]) {
 
 // Final values of 4 consecutive output columns of one row (same rules as store_final16).
 template <int EPI>
-__device__ __forceinline__ void store_final4(const GemmParams& p, int64_t row, int col,
+__device__ __forceinline__ void store_final4(const PhaseParams& p, int64_t row, int col,
                                              const float4& a, const float4& b) {
   if (EPI == EPI_STORE_F32) {
     *reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ld_out + col) = a;
@@ -201,7 +274,7 @@ __device__ __forceinline__ void store_final4(const GemmParams& p, int64_t row, i
 // Final values of 16 consecutive output columns of one row: SwiGLU h = silu(g) * u and GELU
 // h = gelu(z) rounded once to bf16; the down projection stored as fp32.
 template <int EPI>
-__device__ __forceinline__ void store_final16(const GemmParams& p, int64_t row, int col,
+__device__ __forceinline__ void store_final16(const PhaseParams& p, int64_t row, int col,
                                               const float (&a)[16], const float (&b)[16]) {
   if (EPI == EPI_STORE_F32) {
     store_f32x16(static_cast<float*>(p.out) + row * p.ld_out + col, a);
@@ -220,11 +293,129 @@ __device__ __forceinline__ void store_final16(const GemmParams& p, int64_t row, 
   }
 }
 
-template <int EPI, int BN_OUT, int BM>
+// Epilogue of one segment (all 128 epilogue threads): read the accumulator from TMEM, store
+// the final tile or this segment's partial, hand the TMEM buffer back; for a partial, count the
+// arrival and, if last, add the partials in order and store the tile. Returns whether this CTA
+// wrote the tile's final values in *finished; false on a timed-out wait.
+template <int EPI, int BN, int BM>
+__device__ __forceinline__ bool epilogue_segment(const FfnParams& fp, const PhaseParams& p,
+                                                 const Sched& sched, const Seg& sg,
+                                                 const TileCoord& c, uint32_t tmem_base, int tc,
+                                                 uint32_t tfull, uint32_t tempty, uint32_t ebar,
+                                                 uint32_t& epi_phase, volatile int* s_abort,
+                                                 int* s_fixup, bool* finished) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3;  // TMEM lane quadrant this warp may access
+  // tile row held by this thread's TMEM lane (M = 64 uses lanes 0-15 of each quadrant)
+  const int r_local = BM == 128 ? q * 32 + lane : (lane < 16 ? q * 16 + lane : BM);
+  const int buf = tc & 1;
+  const uint32_t tph = (tc >> 1) & 1;
+  const bool got = mbar_wait(tfull, tph, fp.timeout_ns, s_abort);
+  if (!__all_sync(0xffffffffu, got)) return false;
+  tc_fence_after_sync();
+  const bool whole = sg.kb0 == 0 && sg.kb1 == sched.num_kb;
+  // partial slot of this segment: 0 when the CTA's range starts inside this tile
+  const int64_t t_it0 = static_cast<int64_t>(sg.tile) * sched.num_kb;
+  const int slot = whole ? 0 : (sk_begin(sched, blockIdx.x) >= t_it0 ? 0 : 1);
+  float* const my_part =
+      p.part + (static_cast<int64_t>(blockIdx.x * 2 + slot) * fp.slot_rows) * kUmmaN;
+  const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                         static_cast<uint32_t>(buf * kUmmaN);
+  const bool row_ok = r_local < c.rows;
+  const int64_t row = static_cast<int64_t>(c.m0) + r_local;
+#pragma unroll 1
+  for (int cc = 0; cc < BN; cc += 16) {
+    if (c.n0 + cc >= p.n_out) break;  // warp-uniform: ragged last n-tile
+    float a[16], b[16];
+    uint32_t v[16];
+    tmem_ld_32x32b_x16(t_row + cc, v);
+    if (EPI == EPI_SWIGLU) {
+      uint32_t u[16];
+      tmem_ld_32x32b_x16(t_row + BN + cc, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) b[i] = __uint_as_float(u[i]);
+    } else {
+      tmem_ld_wait();
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(v[i]);
+    if (!row_ok) continue;
+    if (whole) {
+      store_final16<EPI>(p, row, c.n0 + cc, a, b);
+    } else {  // this segment's partial tile
+      float* dst = my_part + static_cast<int64_t>(r_local) * kUmmaN + cc;
+      store_f32x16(dst, a);
+      if (EPI == EPI_SWIGLU) store_f32x16(dst + BN, b);
+    }
+  }
+  tc_fence_before_sync();
+  mbar_arrive(tempty);  // TMEM buffer free for the next segment
+  *finished = whole;
+  if (whole) return true;
+
+  // A tile cut by range boundaries is finished by its owner: the first CTA of its range,
+  // whose segment (the tile's first k blocks) ends its range, so it is done last. The others
+  // publish their partials with one release increment of the tile's counter (after a barrier
+  // of the 128 epilogue threads, one fenced thread releases them all); the owner waits for
+  // that count, then adds every partial in order of CTA index.
+  const int first_cta = sk_cta_of(sched, t_it0);
+  const int n_seg = sk_cta_of(sched, t_it0 + sched.num_kb - 1) - first_cta + 1;
+  const bool owner = static_cast<int>(blockIdx.x) == first_cta;
+  if (!__all_sync(0xffffffffu, epilogue_sync(ebar, epi_phase, fp.timeout_ns, s_abort))) return false;
+  if (!owner) {
+    if (threadIdx.x == 64) {
+      __threadfence();
+      atomicAdd(p.tile_counters + sg.tile, 1);  // result unused: a fire-and-forget reduction
+    }
+    return true;
+  }
+  if (threadIdx.x == 64) {
+    const bool arrived =
+        wait_counter_at_least(p.tile_counters + sg.tile, n_seg - 1, fp.timeout_ns, s_abort);
+    if (arrived) p.tile_counters[sg.tile] = 0;  // every other segment has arrived
+    *s_fixup = arrived;
+  }
+  if (!__all_sync(0xffffffffu, epilogue_sync(ebar, epi_phase, fp.timeout_ns, s_abort))) return false;
+  if (!*s_fixup) return false;
+  // All 128 epilogue threads share the reduction: item i is (tile row i / G, float4 column
+  // group i % G), so neighbouring threads touch neighbouring columns.
+  constexpr int G = BN / 4;
+  const int cols = min(BN, p.n_out - c.n0);
+  const int et = threadIdx.x - 64;  // 0..127
+  for (int i = et; i < c.rows * G; i += kEpiThreads) {
+    const int r = i / G, c4 = (i - r * G) * 4;
+    if (c4 >= cols) continue;
+    const int64_t orow = static_cast<int64_t>(c.m0) + r;
+    float4 ga = make_float4(0.f, 0.f, 0.f, 0.f), ub = ga;
+#pragma unroll 2
+    for (int j = 0; j < n_seg; ++j) {  // fixed order (CTA index): deterministic sums
+      const int b2 = first_cta + j;
+      const int slot2 = sk_begin(sched, b2) >= t_it0 ? 0 : 1;
+      const float* src =
+          p.part + (static_cast<int64_t>(b2 * 2 + slot2) * fp.slot_rows + r) * kUmmaN + c4;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+      ga.x += v.x; ga.y += v.y; ga.z += v.z; ga.w += v.w;
+      if (EPI == EPI_SWIGLU) {
+        const float4 u = __ldcg(reinterpret_cast<const float4*>(src + BN));
+        ub.x += u.x; ub.y += u.y; ub.z += u.z; ub.w += u.w;
+      }
+    }
+    store_final4<EPI>(p, orow, c.n0 + c4, ga, ub);
+  }
+  *finished = true;
+  return true;
+}
+
+template <int EPI1, int BN1, int BM>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
-  using C = Cfg<EPI, BN_OUT, BM>;
+    grouped_ffn_kernel(const __grid_constant__ CUtensorMap tmA1,
+                       const __grid_constant__ CUtensorMap tmB1,
+                       const __grid_constant__ CUtensorMap tmA2,
+                       const __grid_constant__ CUtensorMap tmB2, const FfnParams p) {
+  using C = Cfg<BM>;
+  static_assert(EPI1 != EPI_SWIGLU || 2 * BN1 == kUmmaN, "SwiGLU tile: gate | up halves");
+  static_assert(EPI1 == EPI_SWIGLU || BN1 == kUmmaN, "GELU tile");
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
   __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
@@ -234,10 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t epi_bar;
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int s_abort;
-  __shared__ int s_tile_start[257];
+  __shared__ int s_mt[257];   // first m-tile of each expert; s_mt[N] = m-tiles in all
   __shared__ int s_off[257];
-  __shared__ int s_splits;
+  __shared__ Sched s_sched[2];
   __shared__ int s_fixup;
+  __shared__ int s_last_cta;
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5;
@@ -246,8 +438,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tiles = (smem_u32(dyn_smem) + 1023u) & ~1023u;
 
   if (threadIdx.x == 0) {
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmA1);
+    prefetch_tensormap(&tmB1);
+    prefetch_tensormap(&tmA2);
+    prefetch_tensormap(&tmB2);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
@@ -268,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   pdl_wait();  // below: reads of the previous kernels' outputs and writes to global memory
   if (warp == 2) {
-    // Per-expert tile counts and their exclusive prefix (experts lane*per .. lane*per+per-1).
+    // Per-expert m-tile counts and their exclusive prefix (experts lane*per .. lane*per+per-1).
     const int per = (N + 31) / 32;
     int cnt[8];
     int sum = 0;
@@ -280,11 +474,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i < per && e < N) {
         const int a = p.expert_offset[e], b = p.expert_offset[e + 1];
         s_off[e] = a;
-        if (a < 0 || b < a || b > p.r_max) {
+        if (a < 0 || b < a || b > p.r_max || b - a > p.rows_per_expert)
           bad = true;
-        } else {
-          cnt[i] = ((b - a + BM - 1) / BM) * p.n_tiles_n;
-        }
+        else
+          cnt[i] = (b - a + BM - 1) / BM;
         sum += cnt[i];
       }
     }
@@ -300,13 +493,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 8; ++i) {
       const int e = lane * per + i;
       if (i < per && e < N) {
-        s_tile_start[e] = run;
+        s_mt[e] = run;
         run += cnt[i];
       }
     }
+    if (__shfl_sync(0xffffffffu, incl, 31) > p.m_tiles_cap) {  // overlapping offsets: no tiles
+      bad = true;
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane * per + i;
+        if (i < per && e < N) s_mt[e] = 0;
+      }
+      incl = 0;
+    }
     if (lane == 31) {
-      s_tile_start[N] = incl;
-      s_splits = choose_splits(incl, gridDim.x, p.num_kb, p.max_splits);
+      s_mt[N] = incl;
+      for (int ph = 0; ph < 2; ++ph)
+        s_sched[ph] = choose_schedule(incl * p.ph[ph].n_tiles_n, gridDim.x, p.ph[ph].num_kb,
+                                      p.ph[ph].sk_ctas, p.slot_rows);
     }
     if (bad) report_error(p.status, MOE_ERR_BOUNDS);  // such an expert gets no tiles
   }
@@ -315,9 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
 
   const uint32_t tmem_base = s_tmem_base;
-  const int total_tiles = s_tile_start[N];
-  const int splits = s_splits;
-  const int total_units = total_tiles * splits;
+  const int h_target = p.ph[0].n_tiles_n;  // phase-0 tiles per m-tile
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -326,27 +527,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_b = make_policy(p.weight_policy);
       int it = 0;
       bool ok = true;
-      for (int unit = blockIdx.x; ok && unit < total_units; unit += gridDim.x) {
-        const int tile = unit / splits, sp = unit - tile * splits;
-        const TileCoord c = decode_tile<BM>(tile, N, BN_OUT, s_tile_start, s_off);
-        const int kb0 = sp * p.num_kb / splits, kb1 = (sp + 1) * p.num_kb / splits;
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1;
-          if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, p.timeout_ns, &s_abort)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fb = smem_u32(&full_bar[s]);
-          const uint32_t a_dst = tiles + s * C::STAGE_BYTES;
-          const uint32_t b_dst = a_dst + C::A_BYTES;
-          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-          tma_load_2d(a_dst, &tmA, fb, kb * BK, c.m0, pol_a);
-          if (EPI == EPI_SWIGLU) {
-            tma_load_4d(b_dst, &tmB, fb, kb * BK, c.n0, 0, c.e, pol_b);
-            tma_load_4d(b_dst + BN_OUT * BK * 2, &tmB, fb, kb * BK, c.n0, 1, c.e, pol_b);
-          } else {
-            tma_load_3d(b_dst, &tmB, fb, kb * BK, c.n0, c.e, pol_b);
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        const Sched sc = s_sched[ph];
+        const int bn = ph == 0 ? BN1 : kDnBn;
+        const CUtensorMap* tA = ph == 0 ? &tmA1 : &tmA2;
+        SegCursor cur(sc);
+        Seg sg;
+        while (ok && cur.next(sc, sg)) {
+          const TileCoord c = decode_tile<BM>(sg.tile, N, bn, p.ph[ph].n_tiles_n, s_mt, s_off);
+          // phase 1: the W_d blocks go out at once; the h blocks once the rows' h is complete
+          // (one poll here: an acquire load stalls this thread for an L2 round trip)
+          bool ready = ph == 0 || ld_acquire_gpu(p.h_ready + c.gm) >= h_target;
+          int pend_from = -1;  // first iteration whose stage holds its B block but not its A
+          const int seg_it0 = it;
+          for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+            const int s = it % C::STAGES;
+            const uint32_t par = (it / C::STAGES) & 1;
+            if (!mbar_wait(smem_u32(&empty_bar[s]), par ^ 1u, p.timeout_ns, &s_abort)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = smem_u32(&full_bar[s]);
+            const uint32_t a_dst = tiles + s * C::STAGE_BYTES;
+            const uint32_t b_dst = a_dst + C::A_BYTES;
+            mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+            if (ph == 0) {
+              if (EPI1 == EPI_SWIGLU) {
+                tma_load_4d(b_dst, &tmB1, fb, kb * BK, c.n0, 0, c.e, pol_b);
+                tma_load_4d(b_dst + BN1 * BK * 2, &tmB1, fb, kb * BK, c.n0, 1, c.e, pol_b);
+              } else {
+                tma_load_3d(b_dst, &tmB1, fb, kb * BK, c.n0, c.e, pol_b);
+              }
+            } else {
+              tma_load_3d(b_dst, &tmB2, fb, kb * BK, c.n0, c.e, pol_b);
+            }
+            if (ready) {
+              tma_load_2d(a_dst, tA, fb, kb * BK, c.m0, pol_a);
+              ++it;
+              continue;
+            }
+            if (pend_from < 0) pend_from = it;
+            if (it - pend_from + 1 == C::STAGES || kb + 1 == sg.kb1) {
+              // every stage holds a W_d block (or the segment ends): wait for the rows' h
+              if (!wait_counter_at_least(p.h_ready + c.gm, h_target, p.timeout_ns, &s_abort))
+                ok = false;  // the h loads below still complete the armed stages
+              fence_proxy_async_global();
+              for (int j = pend_from; j <= it; ++j) {
+                const int sj = j % C::STAGES;
+                tma_load_2d(tiles + sj * C::STAGE_BYTES, tA, smem_u32(&full_bar[sj]),
+                            (sg.kb0 + (j - seg_it0)) * BK, c.m0, pol_a);
+              }
+              pend_from = -1;
+              ready = true;
+            }
+            ++it;
+            if (!ok) break;
           }
         }
       }
@@ -361,41 +596,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, C::UMMA_N);
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, kUmmaN);
       int it = 0, tc = 0;
       bool ok = true;
       bool issued = false;
-      for (int unit = blockIdx.x; ok && unit < total_units; unit += gridDim.x, ++tc) {
-        const int sp = unit % splits;
-        const int kb0 = sp * p.num_kb / splits, kb1 = (sp + 1) * p.num_kb / splits;
-        const int buf = tc & 1;
-        const uint32_t tph = (tc >> 1) & 1;
-        if (!mbar_wait(smem_u32(&tempty_bar[buf]), tph ^ 1u, p.timeout_ns, &s_abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::UMMA_N);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1;
-          if (!mbar_wait(smem_u32(&full_bar[s]), ph, p.timeout_ns, &s_abort)) {
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        const Sched sc = s_sched[ph];
+        SegCursor cur(sc);
+        Seg sg;
+        for (; ok && cur.next(sc, sg); ++tc) {
+          const int buf = tc & 1;
+          const uint32_t tph = (tc >> 1) & 1;
+          if (!mbar_wait(smem_u32(&tempty_bar[buf]), tph ^ 1u, p.timeout_ns, &s_abort)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_base = tiles + s * C::STAGE_BYTES;
-          const uint32_t b_base = a_base + C::A_BYTES;
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kUmmaN);
+          for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+            const int s = it % C::STAGES;
+            const uint32_t par = (it / C::STAGES) & 1;
+            if (!mbar_wait(smem_u32(&full_bar[s]), par, p.timeout_ns, &s_abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+            const uint32_t a_base = tiles + s * C::STAGE_BYTES;
+            const uint32_t b_base = a_base + C::A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            tc_mma_f16(d_tmem, smem_desc_k_sw128(a_base + kk * 32), smem_desc_k_sw128(b_base + kk * 32),
-                       idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              tc_mma_f16(d_tmem, smem_desc_k_sw128(a_base + kk * 32),
+                         smem_desc_k_sw128(b_base + kk * 32), idesc,
+                         (kb != sg.kb0 || kk != 0) ? 1u : 0u);
+            }
+            issued = true;
+            tc_commit(smem_u32(&empty_bar[s]));
           }
-          issued = true;
-          tc_commit(smem_u32(&empty_bar[s]));
+          if (!ok) break;
+          tc_commit(smem_u32(&tfull_bar[buf]));
         }
-        if (!ok) break;
-        tc_commit(smem_u32(&tfull_bar[buf]));
       }
       if (!ok) {
         s_abort = 1;
@@ -408,97 +647,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- epilogue (warps 2..5)
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    // tile row held by this thread's TMEM lane (M = 64 uses lanes 0-15 of each quadrant)
-    const int r_local = BM == 128 ? q * 32 + lane : (lane < 16 ? q * 16 + lane : BM);
     int tc = 0;
     uint32_t epi_phase = 0;
     bool ok = true;
-    for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x, ++tc) {
-      const int tile = unit / splits, sp = unit - tile * splits;
-      const TileCoord c = decode_tile<BM>(tile, N, BN_OUT, s_tile_start, s_off);
-      const int buf = tc & 1;
-      const uint32_t tph = (tc >> 1) & 1;
-      const bool got = mbar_wait(smem_u32(&tfull_bar[buf]), tph, p.timeout_ns, &s_abort);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after_sync();
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(buf * C::UMMA_N);
-      const bool row_ok = r_local < c.rows;
-      const int64_t row = static_cast<int64_t>(c.m0) + r_local;
-#pragma unroll 1
-      for (int cc = 0; cc < BN_OUT; cc += 16) {
-        if (c.n0 + cc >= p.n_out) break;  // warp-uniform: ragged last n-tile
-        float a[16], b[16];
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(t_row + cc, v);
-        if (EPI == EPI_SWIGLU) {
-          uint32_t u[16];
-          tmem_ld_32x32b_x16(t_row + BN_OUT + cc, u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) b[i] = __uint_as_float(u[i]);
-        } else {
-          tmem_ld_wait();
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(v[i]);
-        if (!row_ok) continue;
-        if (splits == 1) {
-          store_final16<EPI>(p, row, c.n0 + cc, a, b);
-        } else {  // this unit's partial tile
-          float* dst = p.part + (static_cast<int64_t>(sp) * p.r_max + row) * p.part_ld + c.n0 + cc;
-          store_f32x16(dst, a);
-          if (EPI == EPI_SWIGLU) store_f32x16(dst + p.n_out, b);
-        }
-      }
-      tc_fence_before_sync();
-      mbar_arrive(smem_u32(&tempty_bar[buf]));  // TMEM buffer free for the next unit
-
-      if (splits > 1) {
-        // publish this partial; the unit that completes the tile adds all partials in order
-        __threadfence();
-        if (!__all_sync(0xffffffffu, epilogue_sync(smem_u32(&epi_bar), epi_phase, p.timeout_ns, &s_abort))) {
-          ok = false;
-          break;
-        }
-        if (threadIdx.x == 64) {
-          const int prev = atomicAdd(p.tile_counters + tile, 1);
-          const int last = prev == splits - 1;
-          if (last) p.tile_counters[tile] = 0;  // every unit of the tile has arrived
-          s_fixup = last;
-        }
-        if (!__all_sync(0xffffffffu, epilogue_sync(smem_u32(&epi_bar), epi_phase, p.timeout_ns, &s_abort))) {
-          ok = false;
-          break;
-        }
-        if (s_fixup) {
-          // All 128 epilogue threads share the reduction: item i is (tile row i / G, float4
-          // column group i % G), so neighbouring threads touch neighbouring columns.
-          __threadfence();
-          constexpr int G = BN_OUT / 4;
-          const int cols = min(BN_OUT, p.n_out - c.n0);
-          const int et = threadIdx.x - 64;  // 0..127
-          for (int i = et; i < c.rows * G; i += kEpiThreads) {
-            const int r = i / G, c4 = (i - r * G) * 4;
-            if (c4 >= cols) continue;
-            const int64_t orow = static_cast<int64_t>(c.m0) + r;
-            const float* src = p.part + orow * p.part_ld + c.n0 + c4;
-            const int64_t sstride = p.r_max * p.part_ld;
-            float4 ga = make_float4(0.f, 0.f, 0.f, 0.f), ub = ga;
-#pragma unroll 4
-            for (int s2 = 0; s2 < splits; ++s2) {  // fixed order: deterministic sums
-              const float4 v = __ldcg(reinterpret_cast<const float4*>(src + s2 * sstride));
-              ga.x += v.x; ga.y += v.y; ga.z += v.z; ga.w += v.w;
-              if (EPI == EPI_SWIGLU) {
-                const float4 u = __ldcg(reinterpret_cast<const float4*>(src + s2 * sstride + p.n_out));
-                ub.x += u.x; ub.y += u.y; ub.z += u.z; ub.w += u.w;
-              }
-            }
-            store_final4<EPI>(p, orow, c.n0 + c4, ga, ub);
+    for (int ph = 0; ph < 2 && ok; ++ph) {
+      const Sched sc = s_sched[ph];
+      const int bn = ph == 0 ? BN1 : kDnBn;
+      SegCursor cur(sc);
+      Seg sg;
+      for (; cur.next(sc, sg); ++tc) {
+        const TileCoord c = decode_tile<BM>(sg.tile, N, bn, p.ph[ph].n_tiles_n, s_mt, s_off);
+        const uint32_t tf = smem_u32(&tfull_bar[tc & 1]), te = smem_u32(&tempty_bar[tc & 1]);
+        bool finished = false;
+        if (ph == 0)
+          ok = epilogue_segment<EPI1, BN1, BM>(p, p.ph[0], sc, sg, c, tmem_base, tc, tf, te,
+                                               smem_u32(&epi_bar), epi_phase, &s_abort,
+                                               &s_fixup, &finished);
+        else
+          ok = epilogue_segment<EPI_STORE_F32, kDnBn, BM>(p, p.ph[1], sc, sg, c, tmem_base, tc,
+                                                          tf, te, smem_u32(&epi_bar), epi_phase,
+                                                          &s_abort, &s_fixup, &finished);
+        if (!ok) break;
+        if (ph == 0 && finished) {
+          // this CTA wrote the tile's h: order it before TMA loads, then count it (one fenced
+          // thread after the barrier releases every epilogue thread's stores)
+          fence_proxy_async_global();
+          if (!__all_sync(0xffffffffu, epilogue_sync(smem_u32(&epi_bar), epi_phase, p.timeout_ns, &s_abort))) {
+            ok = false;
+            break;
+          }
+          if (threadIdx.x == 64) {
+            __threadfence();
+            atomicAdd(p.h_ready + c.gm, 1);
           }
         }
       }
@@ -514,6 +694,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+  // the last CTA to finish zeroes the m-tile counters for the next call
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last_cta = atomicAdd(p.done_ctas, 1) == static_cast<int>(gridDim.x) - 1;
+  }
+  __syncthreads();
+  if (s_last_cta) {
+    __threadfence();
+    for (int i = threadIdx.x; i < s_mt[N]; i += kThreads) p.h_ready[i] = 0;
+    if (threadIdx.x == 0) *p.done_ctas = 0;
   }
 }
 
@@ -558,76 +749,71 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
   return r == CUDA_SUCCESS;
 }
 
-template <int EPI, int BN_OUT, int BM>
-cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& gp,
-                       int grid, cudaStream_t s) {
-  using C = Cfg<EPI, BN_OUT, BM>;
+template <int EPI1, int BN1, int BM>
+cudaError_t launch_one(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
+                       const CUtensorMap& b2, const FfnParams& fp, int grid, cudaStream_t s) {
+  using C = Cfg<BM>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(grouped_gemm_kernel<EPI, BN_OUT, BM>,
+    attr_err = cudaFuncSetAttribute(grouped_ffn_kernel<EPI1, BN1, BM>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  return launch_pdl(grouped_gemm_kernel<EPI, BN_OUT, BM>, dim3(grid), dim3(kThreads), C::SMEM_BYTES, s,
-                    ma, mb, gp);
+  return launch_pdl(grouped_ffn_kernel<EPI1, BN1, BM>, dim3(grid), dim3(kThreads), C::SMEM_BYTES,
+                    s, a1, b1, a2, b2, fp);
 }
 
-int64_t tiles_upper_bound(int64_t r_max, int N, int n_tiles_n, int bm) {
-  // sum_e ceil(m_e / bm) <= ceil(R / bm) + (experts with rows)
-  const int64_t m_tiles_ub = (r_max + bm - 1) / bm + std::min<int64_t>(N, r_max);
-  return m_tiles_ub * n_tiles_n;
+// sum_e ceil(m_e / bm) <= ceil(R / bm) + (experts with rows)
+int64_t m_tiles_upper_bound(int64_t r_max, int N, int bm) {
+  return (r_max + bm - 1) / bm + std::min<int64_t>(N, r_max);
 }
 
-int grid_for(int64_t r_max, int N, int n_tiles_n, int sm_count, int max_splits, int bm) {
-  const int64_t units_ub = tiles_upper_bound(r_max, N, n_tiles_n, bm) * max_splits;
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units_ub, sm_count)));
-}
+constexpr int kSkMaxCtas = 148;  // CTAs that hold stream-K partial slots (one per B200 SM)
+// Stream-K only while a partial tile is at most this many rows: the last CTA of a tile adds the
+// partials through L2 at latency-bound speed, which costs more than a last, partly filled wave
+// of whole tiles once partial tiles reach 64 rows (measured on B200).
+constexpr int kSkMaxSlotRows = 32;
 
-constexpr int64_t kSplitRowsMax = 256;                 // split-K only for decode-sized batches
-constexpr size_t kPartBudget = size_t(64) << 20;       // bytes of partial tiles per GEMM
-constexpr int kMaxSplits = 16;
-
-int max_splits_for(int64_t r_max, int num_kb, int part_ld) {
-  if (r_max > kSplitRowsMax) return 1;
-  int ms = std::min(kMaxSplits, num_kb / 2);
-  while (ms > 1 && static_cast<size_t>(ms) * r_max * part_ld * 4 > kPartBudget) --ms;
-  return std::max(1, ms);
+// CTAs that can have work: whole tiles, or stream-K ranges of at least kSkMinKb k blocks.
+int64_t useful_ctas(int64_t tiles_ub, int num_kb, int sk_ctas) {
+  const int64_t sk = tiles_ub * num_kb / std::min(kSkMinKb, num_kb);
+  return std::max<int64_t>(tiles_ub, std::min<int64_t>(sk_ctas, sk));
 }
 
 constexpr int kGuBnSwiglu = 128;  // output columns per tile of the gate/up GEMM (UMMA N = 256)
 constexpr int kGuBnGelu = 256;
-constexpr int kDnBn = 256;        // output columns per tile of the down GEMM
 
 }  // namespace
 
 FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max,
                                 int64_t rows_per_expert) {
-  FfnScratchPlan pl{1, 1, 0, 0, 128};
+  FfnScratchPlan pl{};
+  pl.bm = 128;
   if (r_max <= 0) return pl;
   pl.bm = rows_per_expert <= 64 ? 64 : 128;
-  const bool swiglu = act == MOE_ACT_SWIGLU;
-  const int bn1 = swiglu ? kGuBnSwiglu : kGuBnGelu;
-  const int ld1 = swiglu ? 2 * F : F;
-  pl.max_splits1 = max_splits_for(r_max, d / BK, ld1);
-  pl.max_splits2 = max_splits_for(r_max, F / BK, d);
-  size_t part = 0;
-  int64_t tiles = 0;
-  if (pl.max_splits1 > 1) {
-    part = std::max(part, static_cast<size_t>(pl.max_splits1) * r_max * ld1 * 4);
-    tiles = std::max(tiles, tiles_upper_bound(r_max, N, (F + bn1 - 1) / bn1, pl.bm));
+  pl.slot_rows = static_cast<int>(std::min<int64_t>(pl.bm, std::max<int64_t>(1, rows_per_expert)));
+  const int bn1 = act == MOE_ACT_SWIGLU ? kGuBnSwiglu : kGuBnGelu;
+  pl.m_tiles_ub = m_tiles_upper_bound(r_max, N, pl.bm);
+  pl.tiles1_ub = pl.m_tiles_ub * ((F + bn1 - 1) / bn1);
+  pl.tiles2_ub = pl.m_tiles_ub * ((d + kDnBn - 1) / kDnBn);
+  if (pl.slot_rows <= kSkMaxSlotRows) {
+    const int64_t by1 = pl.tiles1_ub * (d / BK) / std::min(kSkMinKb, d / BK);
+    const int64_t by2 = pl.tiles2_ub * (F / BK) / std::min(kSkMinKb, F / BK);
+    pl.sk_ctas1 = static_cast<int>(std::min<int64_t>(kSkMaxCtas, by1));
+    pl.sk_ctas2 = static_cast<int>(std::min<int64_t>(kSkMaxCtas, by2));
   }
-  if (pl.max_splits2 > 1) {
-    part = std::max(part, static_cast<size_t>(pl.max_splits2) * r_max * d * 4);
-    tiles = std::max(tiles, tiles_upper_bound(r_max, N, (d + kDnBn - 1) / kDnBn, pl.bm));
-  }
-  pl.part_bytes = part;
-  pl.counter_bytes = static_cast<size_t>(tiles) * sizeof(int);
+  const int64_t ints = pl.m_tiles_ub + 1 + (pl.sk_ctas1 > 0 ? pl.tiles1_ub : 0) +
+                       (pl.sk_ctas2 > 0 ? pl.tiles2_ub : 0);
+  pl.counter_bytes = static_cast<size_t>(ints) * sizeof(int);
+  pl.part_bytes = static_cast<size_t>(pl.sk_ctas1 + pl.sk_ctas2) * 2 * pl.slot_rows * kUmmaN *
+                  sizeof(float);
   return pl;
 }
 
 cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   if (a.r_max <= 0) return cudaSuccess;
+  if (a.counters == nullptr) return cudaErrorInvalidValue;
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
@@ -636,11 +822,11 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   const uint64_t N = static_cast<uint64_t>(a.N), R = static_cast<uint64_t>(a.r_max);
   const bool swiglu = a.act == MOE_ACT_SWIGLU;
   const int bn_gu = swiglu ? kGuBnSwiglu : kGuBnGelu;
-  // weights are read once per m-tile; when every expert has at most one m-tile (decode-sized
-  // batches) they are pure streams and should not displace the activations in L2
   const FfnScratchPlan plan =
       ffn_scratch_plan(a.N, a.d, a.F, a.act, a.r_max, a.rows_per_expert);
   const int bm = plan.bm;
+  // weights are read once per m-tile; when every expert has at most one m-tile (decode-sized
+  // batches) they are pure streams and should not displace the activations in L2
   const int wpol = (a.rows_per_expert <= bm) ? 1 : 0;
 
   CUtensorMap mA1, mB1, mA2, mB2;
@@ -674,43 +860,53 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
     if (!make_map(&mB2, a.w_down, 3, dims, str, box)) return cudaErrorInvalidValue;
   }
 
-  GemmParams g1{};
-  g1.expert_offset = a.expert_offset;
-  g1.out = a.h;
-  g1.ld_out = a.F;
-  g1.r_max = a.r_max;
-  g1.n_experts = a.N;
-  g1.n_out = a.F;
-  g1.n_tiles_n = (a.F + bn_gu - 1) / bn_gu;
-  g1.num_kb = a.d / BK;
-  g1.status = a.status;
-  g1.timeout_ns = a.timeout_ns;
-  g1.weight_policy = wpol;
-  const bool can_split = a.part != nullptr && a.tile_counters != nullptr;
-  g1.max_splits = can_split ? plan.max_splits1 : 1;
-  g1.part = a.part;
-  g1.part_ld = swiglu ? 2 * a.F : a.F;
-  g1.tile_counters = a.tile_counters;
-  const int grid1 = grid_for(a.r_max, a.N, g1.n_tiles_n, di.sm_count, g1.max_splits, bm);
-  if (bm == 64)
-    err = swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 64>(mA1, mB1, g1, grid1, s)
-                 : launch_one<EPI_GELU, kGuBnGelu, 64>(mA1, mB1, g1, grid1, s);
-  else
-    err = swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128>(mA1, mB1, g1, grid1, s)
-                 : launch_one<EPI_GELU, kGuBnGelu, 128>(mA1, mB1, g1, grid1, s);
-  if (err != cudaSuccess) return err;
+  const bool stream_k = a.part != nullptr;
+  FfnParams fp{};
+  fp.expert_offset = a.expert_offset;
+  fp.r_max = a.r_max;
+  fp.rows_per_expert = a.rows_per_expert;
+  fp.n_experts = a.N;
+  fp.slot_rows = plan.slot_rows;
+  int* cnt = a.counters;
+  fp.h_ready = cnt;
+  fp.m_tiles_cap = static_cast<int>(plan.m_tiles_ub);
+  cnt += plan.m_tiles_ub;
+  fp.done_ctas = cnt;
+  cnt += 1;
+  fp.status = a.status;
+  fp.timeout_ns = a.timeout_ns;
+  fp.weight_policy = wpol;
 
-  GemmParams g2 = g1;
-  g2.out = a.y_perm;
-  g2.ld_out = a.d;
-  g2.n_out = a.d;
-  g2.n_tiles_n = (a.d + kDnBn - 1) / kDnBn;
-  g2.num_kb = a.F / BK;
-  g2.max_splits = can_split ? plan.max_splits2 : 1;
-  g2.part_ld = a.d;
-  const int grid2 = grid_for(a.r_max, a.N, g2.n_tiles_n, di.sm_count, g2.max_splits, bm);
-  return bm == 64 ? launch_one<EPI_STORE_F32, kDnBn, 64>(mA2, mB2, g2, grid2, s)
-                  : launch_one<EPI_STORE_F32, kDnBn, 128>(mA2, mB2, g2, grid2, s);
+  PhaseParams& p1 = fp.ph[0];
+  p1.out = a.h;
+  p1.ld_out = a.F;
+  p1.n_out = a.F;
+  p1.n_tiles_n = (a.F + bn_gu - 1) / bn_gu;
+  p1.num_kb = a.d / BK;
+  p1.sk_ctas = stream_k ? plan.sk_ctas1 : 0;
+  p1.part = a.part;
+  p1.tile_counters = cnt;
+  if (plan.sk_ctas1 > 0) cnt += plan.tiles1_ub;
+
+  PhaseParams& p2 = fp.ph[1];
+  p2.out = a.y_perm;
+  p2.ld_out = a.d;
+  p2.n_out = a.d;
+  p2.n_tiles_n = (a.d + kDnBn - 1) / kDnBn;
+  p2.num_kb = a.F / BK;
+  p2.sk_ctas = stream_k ? plan.sk_ctas2 : 0;
+  p2.part = stream_k ? a.part + static_cast<size_t>(plan.sk_ctas1) * 2 * plan.slot_rows * kUmmaN
+                     : nullptr;
+  p2.tile_counters = cnt;
+
+  const int64_t useful = std::max(useful_ctas(plan.tiles1_ub, p1.num_kb, p1.sk_ctas),
+                                  useful_ctas(plan.tiles2_ub, p2.num_kb, p2.sk_ctas));
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(useful, di.sm_count)));
+  if (bm == 64)
+    return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 64>(mA1, mB1, mA2, mB2, fp, grid, s)
+                  : launch_one<EPI_GELU, kGuBnGelu, 64>(mA1, mB1, mA2, mB2, fp, grid, s);
+  return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128>(mA1, mB1, mA2, mB2, fp, grid, s)
+                : launch_one<EPI_GELU, kGuBnGelu, 128>(mA1, mB1, mA2, mB2, fp, grid, s);
 }
 
 }  // namespace moe

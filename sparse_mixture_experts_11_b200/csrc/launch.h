@@ -64,6 +64,38 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const flo
                              float* logits, int32_t* topk_idx, float* topk_w, int T, int d, int N,
                              int k, uint16_t* split_scratch, int* status, uint64_t timeout_ns,
                              cudaStream_t s);
+// Decode-sized batches (T <= kDecodeRouteMaxT) route in one launch: CTA c takes columns
+// [128 c, 128 c + 128) of d for every token and expert and stores partial dot products; the
+// last CTA to finish (arrival counter, zero between calls) adds them in order of c, then takes
+// top-k, the capacity slots and, when given the permute outputs, the sort by expert and the
+// x_perm copy. Scratch: decode_route_scratch_bytes(); the counter lives in the status region.
+constexpr int kDecodeRouteMaxT = 16;
+constexpr int kDecodeSlice = 128;
+constexpr size_t kDecodeCounterOffset = 128;  // bytes into the workspace's status region
+// the last CTA copies x_perm only while it is this small
+constexpr int64_t kDecodePermuteMaxBytes = 512 * 1024;
+inline bool use_decode_route(int64_t T) { return T >= 1 && T <= kDecodeRouteMaxT; }
+inline size_t decode_route_scratch_bytes(int T, int N, int d) {
+  return static_cast<size_t>((d + kDecodeSlice - 1) / kDecodeSlice) * T * N * sizeof(float);
+}
+struct DecodeRouteArgs {
+  const uint16_t* x;
+  const float* w_router;
+  const float* bias;
+  float* logits;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* slot;
+  int32_t* expert_count;
+  int32_t* expert_offset;  // these four null: no permutation
+  int32_t* row_of_pair;
+  int32_t* pair_of_row;
+  uint16_t* x_perm;
+  float* part;    // decode_route_scratch_bytes()
+  int* counter;   // zero between calls
+  int T, d, N, k, cap;
+};
+cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t s);
 // top-k and renormalised weights from given logits
 cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, float* topk_w, int T,
                                     int N, int k, cudaStream_t s);
@@ -90,13 +122,17 @@ cudaError_t launch_router_stats(const float* logits, const int32_t* topk_idx, co
 
 // grouped expert GEMMs on tcgen05
 //
-// Scratch of the grouped FFN for split-K, used only for decode-sized batches (R_max <= 256):
-// fp32 partial tiles and one arrival counter per tile (zero between calls).
+// Scratch of the grouped FFN (one launch for both GEMMs). Counters, zero between calls (each
+// call leaves them zero), as ints: [per m-tile: finished gate/up tiles][CTAs done][stream-K
+// arrival counters of the gate/up tiles][... of the down tiles]. Partial slots, as floats:
+// [gate/up: sk_ctas1 x 2 x slot_rows x 256][down: sk_ctas2 x 2 x slot_rows x 256].
 struct FfnScratchPlan {
-  int max_splits1, max_splits2;  // gate/up GEMM, down GEMM (1 = no split)
-  size_t part_bytes;             // partial tiles (shared by the two GEMMs, which run in turn)
-  size_t counter_bytes;          // per-tile arrival counters
-  int bm;                        // rows per tile: 64 when no expert can hold more, else 128
+  int bm;                  // rows per tile: 64 when no expert can hold more, else 128
+  int slot_rows;           // rows of a partial slot: min(bm, rows_per_expert)
+  int sk_ctas1, sk_ctas2;  // CTAs with stream-K partial slots per GEMM (0: whole tiles only)
+  int64_t m_tiles_ub, tiles1_ub, tiles2_ub;
+  size_t counter_bytes;
+  size_t part_bytes;       // shares the workspace region with the routing scratch
 };
 // rows_per_expert: the most rows any one expert can receive, min(capacity, T).
 FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max,
@@ -113,8 +149,8 @@ struct GroupedFfnArgs {
   int64_t r_max;
   int* status;
   uint64_t timeout_ns;
-  float* part;          // ffn_scratch_plan().part_bytes, or null when no split is planned
-  int* tile_counters;   // ffn_scratch_plan().counter_bytes, zeroed once before first use
+  int* counters;            // ffn_scratch_plan().counter_bytes, zero between calls
+  float* part;              // ffn_scratch_plan().part_bytes, or null: whole tiles only
   int64_t rows_per_expert;  // min(capacity, T)
 };
 cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s);

@@ -46,14 +46,28 @@ def test_max_rows():
 
 
 def test_workspace_sizes():
+    def counters(m_tiles, tiles1, tiles2):
+        # FFN counters: finished gate/up tiles per m-tile, CTAs done, stream-K arrival
+        # counters of both GEMMs' tiles; rounded to 256 B
+        return -(-((m_tiles + 1 + tiles1 + tiles2) * 4) // 256) * 256
+
     small = moe.make_dims(64, 128, 8, 2, 256, "swiglu", 10)
-    # status word + split-K tile counters (9 tiles of the down GEMM, rounded to 256 B) +
-    # split-K partials of the down GEMM (2 splits x 80 rows x 128 fp32 columns)
-    assert moe.workspace_bytes(small) == 256 + 256 + 2 * 80 * 128 * 4
+    # status word + counters (at most 10 m-tiles of 64 rows: 20 gate/up and 10 down tiles) +
+    # two partial slots of 10 rows x 256 fp32 columns for each CTA that can hold a stream-K
+    # range of either GEMM (20 and 10)
+    assert moe.workspace_bytes(small) == 256 + counters(10, 20, 10) + (20 + 10) * 2 * 10 * 256 * 4
     big = moe.make_dims(16384, 7168, 256, 8, 2048, "swiglu", 80)
-    # status word + capacity-scan chunk totals + the bf16 three-term split of W_r that the
-    # tensor-core router reads
-    assert moe.workspace_bytes(big) == 256 + 32 * 256 * 4 + 3 * 256 * 7168 * 2
+    # 80-row partial tiles: whole tiles only; status word + per-m-tile counters (at most
+    # 160 + 256 m-tiles) + the routing scratch: capacity-scan chunk totals + the bf16
+    # three-term split of W_r that the tensor-core router reads
+    assert moe.workspace_bytes(big) == 256 + counters(416, 0, 0) + 32 * 256 * 4 + 3 * 256 * 7168 * 2
+    decode = moe.make_dims(4, 2880, 32, 4, 2880, "swiglu", 4)
+    # status word (+ the decode router's arrival counter) + counters (at most 1 + 16 m-tiles:
+    # 17 x 23 gate/up and 17 x 12 down tiles) + the larger of the decode router's partial dot
+    # products (23 slices x 4 tokens x 32 experts) and two 4-row partial slots per CTA for each
+    # GEMM (148 + 148 CTAs)
+    assert moe.workspace_bytes(decode) == (256 + counters(17, 17 * 23, 17 * 12)
+                                           + max(23 * 4 * 32 * 4, 296 * 2 * 4 * 256 * 4))
     fb = moe.forward_workspace_bytes(big)
     assert fb > 20480 * 7168 * 6
 

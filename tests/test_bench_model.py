@@ -31,13 +31,18 @@ def test_bytes_model_switch():
 
 
 def test_launch_counts():
-    # switch: W_r split + tensor-core router, one slot pass, permute, 2 GEMMs, combine
-    assert bench.launches_per_step(4096, 1, 4096, 64, 1024) == 7
-    # fine-grained: tensor-core router (2), three slot passes, permute, 2 GEMMs, combine
-    assert bench.launches_per_step(16384, 8, 20480, 256, 7168) == 9
-    # decode: per-token router, one slot pass, permute, 2 GEMMs, combine
-    assert bench.launches_per_step(1, 2, 2, 8, 4096) == 6
-    assert bench.launches_per_step(5, 2, 0) == 4
+    # switch: W_r split + tensor-core router, one slot pass, permute, grouped FFN, combine
+    assert bench.launches_per_step(4096, 1, 4096, 64, 1024) == 6
+    # fine-grained: tensor-core router (2), three slot passes, permute, grouped FFN, combine
+    assert bench.launches_per_step(16384, 8, 20480, 256, 7168) == 8
+    # mid-size: per-token router, one slot pass, permute, grouped FFN, combine
+    assert bench.launches_per_step(64, 4, 256, 32, 2880) == 5
+    # decode: one launch routes and sorts (x_perm 16 KB), grouped FFN, combine
+    assert bench.launches_per_step(1, 2, 2, 8, 4096) == 3
+    # decode with an x_perm above 512 KB (16 tokens x 8 choices x 7168): separate permute
+    assert bench.launches_per_step(16, 8, 128, 256, 7168) == 4
+    # no rows can be kept: routing (and sort) and the combine only
+    assert bench.launches_per_step(5, 2, 0) == 2
 
 
 def test_workload_parsing():

@@ -26,10 +26,16 @@ def _replay_forward(spec):
         call()
     torch.cuda.synchronize()
     layer.capture_stage_graphs()
+    # the whole-forward graph (moe_forward) and the stage graphs give the same bits
+    layer.out.fill_(0)
+    layer.graph_full.replay()
+    torch.cuda.synchronize()
+    full = layer.out.clone()
     layer.out.fill_(0)
     for g in layer.graphs:
         g.replay()
     torch.cuda.synchronize()
+    assert torch.equal(full.view(torch.int16), layer.out.view(torch.int16))
     return shape, T, layer
 
 

@@ -164,3 +164,40 @@ def test_k_scaled_capacity():
     H.check_outputs(run, routing, "swiglu")
     H.check_dropped_tokens_pass_through(run, routing["slot"])
     assert int((routing["slot"] < 0).sum()) > 0  # the Zipf skew still overflows hot experts
+
+
+# Decode-sized batches route in one launch (router split over d across CTAs; the last CTA
+# adds the partial dot products, takes top-k and the capacity slots) and, in moe_forward,
+# also sort by expert while x_perm is at most 512 KB.
+# (T, d, N, k, F, act, capacity_factor, zipf)
+DECODE_CASES = [
+    (1, 2880, 32, 4, 256, "swiglu", None, None),
+    (16, 512, 256, 8, 128, "swiglu", 1.25, 1.1),
+    (16, 7168, 8, 2, 128, "gelu", None, None),
+    (12, 4096, 64, 8, 128, "swiglu", 0.5, 1.1),  # x_perm 768 KB: separate permute launch
+    (5, 320, 100, 3, 192, "gelu", 1.0, None),
+    (2, 64, 4, 4, 64, "swiglu", None, None),     # one d slice, k = N
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=lambda c: f"T{c[0]}_d{c[1]}_N{c[2]}_k{c[3]}")
+def test_decode_route_and_forward(case):
+    import sparse_mixture_experts_11_b200 as moe
+    T, d, N, k, F, act, cf, zipf = case
+    inp = _inputs(T, d, N, F, act, zipf, seed=31)
+    cap = oracle.capacity_from_factor(cf, T, N)
+    run = H.StageRun(inp, k, act, cap).run()
+    H.check_logits(H.f64(run.logits), H.f64(inp["x"]), H.f64(inp["w_router"]),
+                   None if inp["logit_bias"] is None else H.f64(inp["logit_bias"]))
+    routing, off, rop = H.check_routing(run, cap)
+    H.check_x_perm(run, rop)
+    H.check_outputs(run, routing, act)
+    H.check_dropped_tokens_pass_through(run, routing["slot"])
+    ws = moe.new_workspace(run.dims, forward=True)
+    out = torch.empty_like(inp["x"])
+    for _ in range(2):  # the arrival counter is back at zero after each call
+        out.fill_(0)
+        moe.forward_into(run.dims, inp["x"], inp["w_router"], inp["logit_bias"], inp["w_gate_up"],
+                         inp["w_down"], inp["x"], out, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), run.out.view(torch.int16))
