@@ -4,13 +4,15 @@
 python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME[:T]] [--impl ours|reference]
 
 A step is one whole forward pass of the layer (route, permute, grouped expert FFN, combine)
-over one batch of synthetic tokens whose inputs already sit in HBM. The forward is captured
-once as a CUDA graph; a timed step replays it between two CUDA events on the launching stream.
-Steps are timed one by one; L2 is flushed (a 256 MB write) before each step, outside the
-timed events. A second pass replays the stages as separate graphs with events between them
-for the per-stage breakdown and the grouped FFN's roofline. The end-to-end figure (e2e) calls moe_forward eagerly, with the H2D
-copy of the tokens and the D2H copy of the output of every step inside its timed region; the
-copies run on their own streams and overlap the neighbouring steps' compute. Under torchrun every rank runs its own replica of the workload
+over one batch of synthetic tokens whose inputs already sit in HBM. The forward (moe_forward)
+is captured once as a CUDA graph; a timed step replays it between two CUDA events on the
+launching stream. Steps are timed one by one; before each step, outside the timed events, L2
+is flushed: a 256 MB write, then a 256 MB read of a second buffer that takes the write's
+write-back. A second pass replays the stages as separate graphs with events between them for
+the per-stage breakdown and the grouped FFN's roofline. The end-to-end figure (e2e) calls
+moe_forward eagerly, with the H2D copy of the tokens and the D2H copy of the output of every
+step inside its timed region; the copies run on their own streams and overlap the
+neighbouring steps' compute. Under torchrun every rank runs its own replica of the workload
 (weak scaling, no collective on the data path). Rank 0 prints the line, with the time taken
 as the max over ranks.
 
@@ -96,18 +98,25 @@ def router_on_tensor_cores(T: int, n_experts: int, d_model: int) -> bool:
 
 
 DECODE_ROUTE_MAX_T = 16           # batches routed (and, when small, sorted) in one launch
+DECODE_ROUTE_MAX_SCRATCH = 1 << 20  # ... while their partial dot products fit this
 DECODE_PERMUTE_MAX_BYTES = 512 * 1024
 
 
+def decode_route(T: int, n_experts: int, d_model: int) -> bool:
+    """The library's rule for the one-launch routing of decode-sized batches."""
+    return 1 <= T <= DECODE_ROUTE_MAX_T and \
+        math.ceil(d_model / 128) * T * n_experts * 4 <= DECODE_ROUTE_MAX_SCRATCH
+
+
 def launches_per_step(T: int, k: int, R_max: int, n_experts: int = 1, d_model: int = 1) -> int:
-    """Kernels one forward (moe_forward) launches. Decode-sized batches (T <= 16): one routing
+    """Kernels one forward (moe_forward) launches. Decode-sized batches (decode_route): one routing
     launch (router, top-k and slots), which also sorts by expert while x_perm is at most
     512 KB, else a permute launch. Larger batches: router + top-k (plus the W_r split kernel
     on the tensor-core path), capacity slots (1 pass, or 3 when the arrivals span several
     chunks), permute. Then the grouped FFN (both GEMMs in one launch, when rows can exist)
     and the combine."""
     ffn = (1 if R_max > 0 else 0) + 1
-    if 1 <= T <= DECODE_ROUTE_MAX_T:
+    if decode_route(T, n_experts, d_model):
         return 1 + (0 if R_max * d_model * 2 <= DECODE_PERMUTE_MAX_BYTES else 1) + ffn
     chunks = max(1, math.ceil(T * k / SLOT_CHUNK))
     router = 2 if router_on_tensor_cores(T, n_experts, d_model) else 1
@@ -117,7 +126,7 @@ def launches_per_step(T: int, k: int, R_max: int, n_experts: int = 1, d_model: i
 # DRAM traffic of the grouped-FFN stage per forward (dram__bytes_read.sum +
 # dram__bytes_write.sum of its launch) from one ncu capture of the current kernel; workloads
 # without a capture of the current kernel report null.
-MEASURED_FFN_TRAFFIC = {}
+MEASURED_FFN_TRAFFIC = {("switch_top1", 4096): 1097.5e6, ("gpt_oss", 1): 205.2e6}
 
 
 def load_peaks():
@@ -409,7 +418,13 @@ def tokens_per_second(tokens_per_rank: int, steps: int, world: int, max_ms: floa
 
 
 def flush_l2(buf):
-    buf.add_(1)  # 256 MB read-modify-write, larger than the 126 MB L2
+    """Evict L2 before a step: a 256 MB write (larger than the 126 MB L2), then a 256 MB read
+    of a second buffer, so the write's dirty lines go back to HBM here, outside the timed
+    region, instead of during the step, and the step starts with no line of its own data
+    in L2."""
+    w, r = buf
+    w.add_(1)
+    torch.sum(r, dtype=torch.float32)
 
 
 def run_gpu(args, rank, world, local_rank):
@@ -422,7 +437,8 @@ def run_gpu(args, rank, world, local_rank):
         call()
     torch.cuda.synchronize()
     layer.capture_stage_graphs()
-    flush = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device)
+    flush = (torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device),
+             torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     wev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
 
@@ -507,7 +523,7 @@ def run_gpu(args, rank, world, local_rank):
                    "n_experts": shape.n_experts, "top_k": shape.top_k, "d_ff": shape.d_ff,
                    "act": shape.act, "capacity": layer.dims.capacity, "kept_rows": R,
                    "active_experts": active,
-                   "l2": "flushed before every step (256 MB write outside the timed events); "
+                   "l2": "flushed before every step (256 MB write, then 256 MB read of another buffer, outside the timed events); "
                          "expert weights also exceed L2",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "launch": "value: the whole forward as one captured CUDA graph (kernels chained "

@@ -103,7 +103,12 @@ moe_status moe_workspace_bytes(const moe_dims* dims, size_t* bytes);
 /* Zero a workspace (an async memset of ws_bytes on `stream`). */
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
-/* Route: steps 1-3 above.
+/* Route: steps 1-3 above. Decode-sized batches (1 <= T <= 16, with ceil(d_model / 128) * T * N
+ * fp32 partial sums of at most 1 MiB) route in one launch: CTA c takes d columns
+ * [128 c, 128 c + 128) of every dot product; the last CTA to finish adds the partials in
+ * order of c, then takes top-k and the slots. Larger batches run the router, then the slot
+ * pass(es). The results follow the same rules either way; the logits' rounding follows the
+ * path's summation order.
  *   x            [T, d_model] bf16            hidden states
  *   w_router     [N, d_model] fp32            router weight (linear, no bias term)
  *   logit_bias   [N] fp32 or NULL             optional additive per-expert logit bias
@@ -234,9 +239,12 @@ moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_r
  *   - The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
  *     with that device current) and caches it. Make that first call before any stream capture.
- *   - All calls share the one array, and it keeps the last call's contents. Each call writes
+ *   - Decode-sized batches (the one-launch routing of moe_route, below) take their partial
+ *     dot products from a second static array of 1 MiB and their arrival counter from a
+ *     third; the counter is zero when the library loads and every call leaves it zero.
+ *   - All calls share the arrays, and they keep the last call's contents. Each call writes
  *     every scratch entry before reading it, so nothing has to start at zero. Calls that
- *     overlap on the GPU (on concurrent streams) race on the array and must be serialised
+ *     overlap on the GPU (on concurrent streams) race on the arrays and must be serialised
  *     by the caller. */
 moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x, const float* w_router,
                              const float* logit_bias, float* logits, int32_t* topk_idx,

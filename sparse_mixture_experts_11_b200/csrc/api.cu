@@ -94,7 +94,7 @@ size_t split_scratch_bytes(const moe_dims* d) {
 
 // Partial dot products of the one-launch router of decode-sized batches.
 size_t decode_scratch_bytes(const moe_dims* d) {
-  return moe::use_decode_route(d->T)
+  return moe::use_decode_route(d->T, d->n_experts, d->d_model)
              ? round_up(moe::decode_route_scratch_bytes(d->T, d->n_experts, d->d_model), 256)
              : 0;
 }
@@ -215,7 +215,7 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const float* w_rou
   if (ws_bytes < stage_ws_bytes(dims)) return MOE_ERR_WORKSPACE;
   if ((st = check_device()) != MOE_OK) return st;
   const cudaStream_t s = as_stream(stream);
-  if (moe::use_decode_route(dims->T))
+  if (moe::use_decode_route(dims->T, dims->n_experts, dims->d_model))
     return launch_status(moe::launch_decode_route(
         decode_route_args(dims, x, w_router, logit_bias, logits, topk_idx, topk_w, slot,
                           expert_count, ws),
@@ -406,7 +406,7 @@ moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_r
   if (dims->T == 0) return MOE_OK;
   if (!x || !w_router || !w_gate_up || !w_down || !out) return MOE_ERR_INVALID;
   const int64_t rmax = max_rows(dims);
-  if (moe::use_decode_route(dims->T) &&
+  if (moe::use_decode_route(dims->T, dims->n_experts, dims->d_model) &&
       rmax * dims->d_model * 2 <= moe::kDecodePermuteMaxBytes) {
     // decode-sized batch: routing and the sort by expert in one launch
     if (!aligned16(x) || !aligned16(w_router) || (logit_bias && !aligned16(logit_bias)))

@@ -72,11 +72,16 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const flo
 constexpr int kDecodeRouteMaxT = 16;
 constexpr int kDecodeSlice = 128;
 constexpr size_t kDecodeCounterOffset = 128;  // bytes into the workspace's status region
+constexpr size_t kDecodeMaxScratch = size_t(1) << 20;  // partial dot products, at most
 // the last CTA copies x_perm only while it is this small
 constexpr int64_t kDecodePermuteMaxBytes = 512 * 1024;
-inline bool use_decode_route(int64_t T) { return T >= 1 && T <= kDecodeRouteMaxT; }
-inline size_t decode_route_scratch_bytes(int T, int N, int d) {
+inline size_t decode_route_scratch_bytes(int64_t T, int64_t N, int64_t d) {
   return static_cast<size_t>((d + kDecodeSlice - 1) / kDecodeSlice) * T * N * sizeof(float);
+}
+// moe_route, moe_forward and moe_route_noalloc all take this path under the same rule, so
+// their routing agrees bit for bit.
+inline bool use_decode_route(int64_t T, int64_t N, int64_t d) {
+  return T >= 1 && T <= kDecodeRouteMaxT && decode_route_scratch_bytes(T, N, d) <= kDecodeMaxScratch;
 }
 struct DecodeRouteArgs {
   const uint16_t* x;

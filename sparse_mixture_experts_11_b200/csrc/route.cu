@@ -487,7 +487,7 @@ cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const f
 }
 
 cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t s) {
-  if (!use_decode_route(a.T) || a.N > 256 || a.k > 8) return cudaErrorInvalidValue;
+  if (!use_decode_route(a.T, a.N, a.d) || a.N > 256 || a.k > 8) return cudaErrorInvalidValue;
   const int ctas = (a.d + kDecodeSlice - 1) / kDecodeSlice;
   const int ept = a.N <= 32 ? 1 : a.N <= 64 ? 2 : a.N <= 128 ? 4 : 8;
   auto pick = [&](auto k1, auto k2, auto k4, auto k8) {

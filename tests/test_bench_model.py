@@ -43,6 +43,9 @@ def test_launch_counts():
     assert bench.launches_per_step(16, 8, 128, 256, 7168) == 4
     # no rows can be kept: routing (and sort) and the combine only
     assert bench.launches_per_step(5, 2, 0) == 2
+    # 16 tokens, N = 256, d = 16384: partial dot products above 1 MiB, so per-token router,
+    # slot pass, permute, grouped FFN, combine
+    assert bench.launches_per_step(16, 8, 128, 256, 16384) == 5
 
 
 def test_workload_parsing():

@@ -87,3 +87,12 @@ def test_noalloc_refuses_shapes_beyond_its_scratch():
     r = moe._lib.moe_route_noalloc(ctypes.byref(dims), None, P(16), None, P(16), P(16), P(16),
                                    P(16), P(16), None)
     assert r == moe.ERR_INVALID
+
+
+@pytest.mark.parametrize("T,d,N,k,cap", [(1, 2880, 32, 4, 1), (16, 512, 256, 8, 1), (7, 4096, 8, 2, 2)])
+def test_noalloc_matches_route_decode_sized(T, d, N, k, cap):
+    """Decode-sized batches take the one-launch router in both calls (same partial sums)."""
+    for _ in range(2):  # the static arrival counter is back at zero after each call
+        ref, got = _route_both(T, d, N, k, cap, 3, 1.1)
+        _assert_same_routing(ref, got)
+        assert torch.equal(ref["logits"], got["logits"])
