@@ -18,7 +18,11 @@
 //             write the three terms as K-major 128B-swizzled tiles into shared memory
 //             (double buffered), every CTA repeating the conversion.
 //
-// One CTA per 128-token tile, 256 threads:
+// One CTA per 128-token tile, 256 threads. When the tiles leave SMs idle, a cluster of 2 or 4
+// CTAs shares a tile, each taking an equal range of the k blocks into its own TMEM
+// accumulator; the non-leaders stage their partial logits in shared memory and the leader
+// adds them through distributed shared memory in rank order (deterministic), then runs the
+// epilogue below. Per CTA:
 //   warp 0      TMA producer of the x tile [128 tokens x 64 k] (128B swizzle) into a ring
 //               (and of the three weight term tiles when PRESPLIT);
 //   warp 1      TMEM owner and MMA issuer: per k block 3 x 4 MMAs (M=128, N=NP, K=16) into one
@@ -63,7 +67,10 @@ struct RCfg {
   static constexpr int SMEM_BYTES = FIXED_BYTES + STAGES * STAGE_BYTES + 1024;
   static_assert(STAGES >= 2, "router pipeline depth");
   static_assert(NP % 16 == 0 && NP >= 16 && NP <= 256, "UMMA N for M = 128");
-  static_assert(kTok * (NP + 1) * 4 <= SMEM_BYTES - 1024, "logits staging fits the pipeline smem");
+  static_assert(kTok * (NP + 4) * 4 <= SMEM_BYTES - 1024, "logits staging fits the pipeline smem");
+  // with a k split: the staged partials plus the final rows of this CTA (at most 64)
+  static_assert((kTok + kTok / 2) * (NP + 4) * 4 <= SMEM_BYTES - 1024,
+                "k-split staging (partials + final rows) fits the pipeline smem");
 };
 
 __device__ __forceinline__ bool better(float av, int ae, float bv, int be) {
@@ -117,13 +124,87 @@ __global__ void __launch_bounds__(256) split_router_weights_kernel(const float* 
   }
 }
 
+// A sorted list of the best KMAX (>= k) (logit, expert) entries; entry KMAX-1 is the
+// admission threshold. NaN logits rank below every number; equal logits go to the lower index.
+template <int KMAX>
+struct TopK {
+  float v[KMAX];
+  int e[KMAX];
+  __device__ __forceinline__ TopK() {
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r) {
+      v[r] = -INFINITY;
+      e[r] = 0x7fffffff;
+    }
+  }
+  // drop the best entry (the list moves up by one; the last slot empties)
+  __device__ __forceinline__ void pop() {
+#pragma unroll
+    for (int r = 0; r + 1 < KMAX; ++r) {
+      v[r] = v[r + 1];
+      e[r] = e[r + 1];
+    }
+    v[KMAX - 1] = -INFINITY;
+    e[KMAX - 1] = 0x7fffffff;
+  }
+  __device__ __forceinline__ void offer(float L, int ex) {
+    const float key = isnan(L) ? -INFINITY : L;
+    if (!better(key, ex, v[KMAX - 1], e[KMAX - 1])) return;
+    // shift the entries the candidate beats down by one and drop it into place; every
+    // slot's update reads only the old list, so the slots update in parallel
+#pragma unroll
+    for (int r = KMAX - 1; r >= 0; --r) {
+      if (better(key, ex, v[r], e[r])) {
+        const int u = r > 0 ? r - 1 : 0;
+        const bool beats_prev = (r > 0) && better(key, ex, v[u], e[u]);
+        v[r] = beats_prev ? v[u] : key;
+        e[r] = beats_prev ? e[u] : ex;
+      }
+    }
+  }
+};
+
+// Token t0 + ct's top-k indices and renormalised weights, then (after a barrier of the 128
+// epilogue threads) the tile's logits out of the staging rows as one coalesced block.
+template <int KMAX>
+__device__ __forceinline__ bool finish_tile(const TopK<KMAX>& best, const float* stage, int t0,
+                                            int ct, int T, int N, int NS, int k, float* logits,
+                                            int32_t* topk_idx, float* topk_w, uint32_t epi_bar,
+                                            uint64_t timeout_ns, const volatile int* abort) {
+  const int t = t0 + ct;
+  if (t < T) {
+    float num[KMAX], den = 0.f;
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r) {
+      num[r] = (r < k) ? expf(best.v[r] - best.v[0]) : 0.f;
+      den += num[r];
+    }
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r)
+      if (r < k) {
+        topk_idx[static_cast<int64_t>(t) * k + r] = best.e[r];
+        topk_w[static_cast<int64_t>(t) * k + r] = num[r] / den;
+      }
+  }
+  mbar_arrive(epi_bar);
+  const bool synced = mbar_wait(epi_bar, 0, timeout_ns, abort);
+  if (!__all_sync(0xffffffffu, synced)) return false;
+  const int rows = min(kTok, T - t0);
+  float* dst = logits + static_cast<int64_t>(t0) * N;
+  for (int i = ct; i < rows * N; i += kConvThreads) {
+    const int r = i / N;
+    dst[i] = stage[r * NS + (i - r * N)];
+  }
+  return true;
+}
+
 template <int NP, bool PRESPLIT, int KMAX>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ w, const float* __restrict__ bias,
                      float* __restrict__ logits, int32_t* __restrict__ topk_idx,
                      float* __restrict__ topk_w, int T, int d, int N, int k, int* status,
-                     uint64_t timeout_ns) {
+                     uint64_t timeout_ns, int ksplit) {
   using C = RCfg<NP, PRESPLIT>;
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t a_full[C::STAGES];
@@ -142,8 +223,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = dyn_smem + (base - smem_u32(dyn_smem));  // generic pointer of `base`
   const uint32_t wbuf0 = base;                               // in-kernel: 2 x [3][NP][64] bf16
   const uint32_t ring0 = base + C::FIXED_BYTES;              // ring of stages
-  const int t0 = blockIdx.x * kTok;
+  // ksplit > 1: a cluster of ksplit CTAs shares one token tile, CTA `rank` taking k blocks
+  // [kb_lo, kb_hi); the leader (rank 0) adds the partial logits in rank order
+  const int rank = ksplit > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int t0 = (blockIdx.x / ksplit) * kTok;
   const int num_kb = d / kBK;
+  const int kb_lo = rank * num_kb / ksplit, kb_hi = (rank + 1) * num_kb / ksplit;
+  const int n_it = kb_hi - kb_lo;
+  // staged logits rows: N4 = N rounded up to 4 columns, stride NS (16-byte aligned rows)
+  const int N4 = (N + 3) & ~3;
+  const int NS = ksplit > 1 ? N4 + 4 : N + 1;  // N + 1: no bank conflicts in the 1-CTA path
+  bool epi_ok = false;
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmX);
@@ -190,11 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint64_t pol_x = l2_policy_evict_first();
       const uint64_t pol_w = l2_policy_evict_last();
-      int kb = 0;
+      int i = 0;
       bool ok = true;
-      for (; kb < num_kb; ++kb) {
-        const int s = kb % C::STAGES;
-        if (!mbar_wait(smem_u32(&a_empty[s]), ((kb / C::STAGES) & 1) ^ 1u, timeout_ns, &s_abort)) {
+      for (; i < n_it; ++i) {
+        const int kb = kb_lo + i;
+        const int s = i % C::STAGES;
+        if (!mbar_wait(smem_u32(&a_empty[s]), ((i / C::STAGES) & 1) ^ 1u, timeout_ns, &s_abort)) {
           ok = false;
           break;
         }
@@ -212,18 +303,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         s_abort = 1;
         report_error(status, MOE_ERR_TIMEOUT);
       }
-      for (int i = max(0, kb - C::STAGES); i < kb; ++i)
-        mbar_wait(smem_u32(&a_full[i % C::STAGES]), (i / C::STAGES) & 1, kDrainTimeoutNs, nullptr);
+      for (int j = max(0, i - C::STAGES); j < i; ++j)
+        mbar_wait(smem_u32(&a_full[j % C::STAGES]), (j / C::STAGES) & 1, kDrainTimeoutNs, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kTok, NP);
       bool ok = true, issued = false;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % C::STAGES, b = kb & 1;
-        if (!mbar_wait(smem_u32(&a_full[s]), (kb / C::STAGES) & 1, timeout_ns, &s_abort) ||
-            (!PRESPLIT && !mbar_wait(smem_u32(&w_full[b]), (kb >> 1) & 1, timeout_ns, &s_abort))) {
+      for (int i = 0; i < n_it; ++i) {
+        const int s = i % C::STAGES, b = i & 1;
+        if (!mbar_wait(smem_u32(&a_full[s]), (i / C::STAGES) & 1, timeout_ns, &s_abort) ||
+            (!PRESPLIT && !mbar_wait(smem_u32(&w_full[b]), (i >> 1) & 1, timeout_ns, &s_abort))) {
           ok = false;
           break;
         }
@@ -236,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
             tc_mma_f16(tmem, smem_desc_k_sw128(a + kk * 32), smem_desc_k_sw128(bt + kk * 32), idesc,
-                       (kb | term | kk) != 0 ? 1u : 0u);
+                       (i | term | kk) != 0 ? 1u : 0u);
         }
         issued = true;
         tc_commit(smem_u32(&a_empty[s]));
@@ -259,8 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!PRESPLIT) {
       // -------------------------------------------------------- in-kernel split of W_r
       constexpr int kTasks = (NP * 8 + kConvThreads - 1) / kConvThreads;  // <= 16
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int b = kb & 1;
+      for (int i = 0; i < n_it; ++i) {
+        const int kb = kb_lo + i;
+        const int b = i & 1;
         // issue every load of this k block before waiting, so their latencies overlap
         float4 v[kTasks][2];
 #pragma unroll
@@ -273,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             v[i][1] = __ldg(src + 1);
           }
         }
-        const bool got = mbar_wait(smem_u32(&w_empty[b]), ((kb >> 1) & 1) ^ 1u, timeout_ns, &s_abort);
+        const bool got = mbar_wait(smem_u32(&w_empty[b]), ((i >> 1) & 1) ^ 1u, timeout_ns, &s_abort);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
@@ -304,78 +396,155 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after_sync();
       const int q = warp & 3;
-      const int t = t0 + ct;
-      const bool valid = t < T;
       const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
       // the pipeline's shared memory is idle now: it stages the [128][N] logits tile
       float* stage = reinterpret_cast<float*>(gbase);
-      // a sorted list of the best KMAX (>= k) entries; entry KMAX-1 is the admission threshold
-      float best_v[KMAX];
-      int best_e[KMAX];
+      if (ksplit > 1) {
+        // this CTA's partial sums (its k range), raw, for the leader to add up
+        for (int c0 = 0; c0 < N; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(trow + c0, v);  // columns past NP are never used (see below)
+          tmem_ld_wait();
 #pragma unroll
-      for (int r = 0; r < KMAX; ++r) {
-        best_v[r] = -INFINITY;
-        best_e[r] = 0x7fffffff;
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i < N4) stage[ct * NS + c0 + i] = __uint_as_float(v[i]);
+        }
+      } else {
+        TopK<KMAX> best;
+        for (int c0 = 0; c0 < N; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(trow + c0, v);  // columns past NP are never used: c0 + 32 <= NP or N <= 16
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int e = c0 + i;
+            if (e >= N) continue;
+            float L = __uint_as_float(v[i]);
+            if (bias != nullptr) L += __ldg(bias + e);
+            stage[ct * NS + e] = L;
+            best.offer(L, e);
+          }
+        }
+        ok = finish_tile<KMAX>(best, stage, t0, ct, T, N, NS, k, logits, topk_idx, topk_w,
+                               smem_u32(&epi_bar), timeout_ns, &s_abort);
       }
-      for (int c0 = 0; c0 < N; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(trow + c0, v);  // columns past NP are never used: c0 + 32 <= NP or N <= 16
-        tmem_ld_wait();
+    }
+    epi_ok = ok;
+    if (!ok) {
+      s_abort = 1;
+      report_error(status, MOE_ERR_TIMEOUT);
+    }
+  }
+
+  if (ksplit > 1) {
+    __syncwarp();
+    cluster_sync_all();  // every CTA's partial tile is in its shared memory
+    if (warp >= 4 && epi_ok) {
+      // CTA `rank` finishes rows [rank * R, rank * R + R) of the tile: ksplit threads per row,
+      // each adding the partials of its float4 column groups in rank order (all loads in
+      // flight at once), then the row's top-k is merged across the row's threads by shuffles
+      const int ct = threadIdx.x - 128;
+      const int R = kTok / ksplit;
+      const int lr = ct / ksplit, part = ct - lr * ksplit;  // local row, thread within the row
+      const int row = rank * R + lr;
+      float* stage = reinterpret_cast<float*>(gbase);
+      float* fin = stage + kTok * NS;  // [R][NS] final logits of this CTA's rows
+      const uint32_t src = smem_u32(stage + row * NS);
+      uint32_t base_r[4];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int e = c0 + i;
-          if (e >= N) continue;
-          float L = __uint_as_float(v[i]);
-          if (bias != nullptr) L += __ldg(bias + e);
-          stage[ct * (N + 1) + e] = L;  // padded rows: no bank conflicts
-          const float key = isnan(L) ? -INFINITY : L;
-          if (better(key, e, best_v[KMAX - 1], best_e[KMAX - 1])) {
-            // shift the entries the candidate beats down by one and drop it into place;
-            // every slot's update reads only the old list, so the slots update in parallel
+      for (int r = 0; r < 4; ++r) base_r[r] = r < ksplit ? map_smem_to_rank(src, r) : 0u;
+      TopK<KMAX> best;
+      constexpr int kGroups = (NP / 4 + 1) / 2;  // column groups per thread (ksplit >= 2)
+      for (int g0 = 0; g0 < kGroups; g0 += 4) {
+        float4 v[4][4];
 #pragma unroll
-            for (int r = KMAX - 1; r >= 0; --r) {
-              if (better(key, e, best_v[r], best_e[r])) {
-                const int u = r > 0 ? r - 1 : 0;
-                const bool beats_prev = (r > 0) && better(key, e, best_v[u], best_e[u]);
-                best_v[r] = beats_prev ? best_v[u] : key;
-                best_e[r] = beats_prev ? best_e[u] : e;
-              }
+        for (int j = 0; j < 4; ++j) {
+          const int g = (g0 + j) * ksplit + part;
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            if (r < ksplit && g * 4 < N4) v[j][r] = ld_dsmem_f32x4(base_r[r] + g * 16);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int g = (g0 + j) * ksplit + part;
+          if (g * 4 >= N4) continue;
+          float4 acc = v[j][0];
+#pragma unroll
+          for (int r = 1; r < 4; ++r) {
+            if (r < ksplit) {
+              acc.x += v[j][r].x;
+              acc.y += v[j][r].y;
+              acc.z += v[j][r].z;
+              acc.w += v[j][r].w;
             }
+          }
+          const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int e = g * 4 + i;
+            if (e >= N) continue;
+            float L = a4[i];
+            if (bias != nullptr) L += __ldg(bias + e);
+            fin[lr * NS + e] = L;
+            best.offer(L, e);
           }
         }
       }
-      if (valid) {
+      // merge the row's ksplit sorted lists (neighbouring lanes): KMAX rounds of "best head
+      // wins and is popped"; equal logits go to the lower expert index as everywhere else
+      float sel_v[KMAX];
+      int sel_e[KMAX];
+#pragma unroll
+      for (int r = 0; r < KMAX; ++r) {
+        float bv = best.v[0];
+        int be = best.e[0];
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+          if (o < ksplit) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (better(ov, oe, bv, be)) {
+              bv = ov;
+              be = oe;
+            }
+          }
+        }
+        sel_v[r] = bv;
+        sel_e[r] = be;
+        if (best.e[0] == be && best.v[0] == bv) best.pop();  // this lane's head won
+      }
+      const int t = t0 + row;
+      if (part == 0 && t < T) {
         float num[KMAX], den = 0.f;
 #pragma unroll
         for (int r = 0; r < KMAX; ++r) {
-          num[r] = (r < k) ? expf(best_v[r] - best_v[0]) : 0.f;
+          num[r] = (r < k) ? expf(sel_v[r] - sel_v[0]) : 0.f;
           den += num[r];
         }
 #pragma unroll
         for (int r = 0; r < KMAX; ++r)
           if (r < k) {
-            topk_idx[static_cast<int64_t>(t) * k + r] = best_e[r];
+            topk_idx[static_cast<int64_t>(t) * k + r] = sel_e[r];
             topk_w[static_cast<int64_t>(t) * k + r] = num[r] / den;
           }
       }
-      // the tile's logits leave shared memory as one contiguous, coalesced block
+      // this CTA's rows of logits leave shared memory as one coalesced block
       mbar_arrive(smem_u32(&epi_bar));
       const bool synced = mbar_wait(smem_u32(&epi_bar), 0, timeout_ns, &s_abort);
       if (__all_sync(0xffffffffu, synced)) {
-        const int rows = min(kTok, T - t0);
-        float* dst = logits + static_cast<int64_t>(t0) * N;
+        const int rows = max(0, min(R, T - (t0 + rank * R)));
+        float* dst = logits + static_cast<int64_t>(t0 + rank * R) * N;
         for (int i = ct; i < rows * N; i += kConvThreads) {
           const int r = i / N;
-          dst[i] = stage[r * (N + 1) + (i - r * N)];
+          dst[i] = fin[r * NS + (i - r * N)];
         }
       } else {
         s_abort = 1;
         report_error(status, MOE_ERR_TIMEOUT);
       }
-    } else {
-      s_abort = 1;
-      report_error(status, MOE_ERR_TIMEOUT);
     }
+    __syncwarp();
+    cluster_sync_all();  // every CTA has read the others' shared memory; they may exit
   }
 
   tc_fence_before_sync();
@@ -404,6 +573,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// CTAs per 128-token tile: the k blocks are split over a cluster of 2 or 4 CTAs while the
+// tiles leave SMs idle and every CTA keeps at least 2 k blocks. A function of the shape only
+// (SM count of a B200), so the workspace and in-kernel-split variants cut K alike and give
+// identical logits.
+int router_ksplit(int tiles, int num_kb) {
+  constexpr int kSms = 148;
+  int ks = 1;
+  while (ks < 4 && static_cast<int64_t>(tiles) * ks * 2 <= kSms && num_kb >= ks * 4) ks *= 2;
+  return ks;
+}
+
 template <int NP, bool PRESPLIT, int KMAX>
 cudaError_t launch_npk(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
                        const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
@@ -416,9 +596,16 @@ cudaError_t launch_npk(const CUtensorMap& mx, const CUtensorMap& mw, const float
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr != cudaSuccess) return attr;
-  const int grid = (T + kTok - 1) / kTok;
-  return launch_pdl(router_tc_kernel<NP, PRESPLIT, KMAX>, dim3(grid), dim3(kThreads), C::SMEM_BYTES,
-                    s, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns);
+  const int tiles = (T + kTok - 1) / kTok;
+  const int ksplit = router_ksplit(tiles, d / kBK);
+  if (ksplit == 1)
+    return launch_pdl(router_tc_kernel<NP, PRESPLIT, KMAX>, dim3(tiles), dim3(kThreads),
+                      C::SMEM_BYTES, s, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k,
+                      status, timeout_ns, 1);
+  return launch_pdl_cluster(router_tc_kernel<NP, PRESPLIT, KMAX>, dim3(tiles * ksplit),
+                            dim3(kThreads), C::SMEM_BYTES, s, static_cast<unsigned>(ksplit), mx, mw,
+                            w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns,
+                            ksplit);
 }
 
 template <int NP, bool PRESPLIT>
