@@ -64,6 +64,14 @@ typedef enum {
 
 typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_GELU = 1 } moe_act;
 
+/* Storage of the expert weights. MX formats follow the OCP Microscaling (MX) Specification
+ * v1.0: every block of 32 consecutive elements along the reduction axis K shares one E8M0
+ * scale X = 2^(s - 127) (s = 255: NaN), and an element's value is X times its own value.
+ *   MOE_WFMT_MXFP8  elements FP8 E4M3 (bias 7, subnormals, max 448, S.1111.111 NaN), 1 byte
+ *   MOE_WFMT_MXFP4  elements FP4 E2M1 (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), 2 per byte,
+ *                   element 2i in the low nibble of byte i */
+typedef enum { MOE_WFMT_BF16 = 0, MOE_WFMT_MXFP8 = 1, MOE_WFMT_MXFP4 = 2 } moe_wfmt;
+
 /* Shape of one layer invocation. */
 typedef struct {
   int32_t T;          /* tokens in the batch, >= 0 */
@@ -219,6 +227,38 @@ moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_r
                        const float* logit_bias, const uint16_t* w_gate_up, const uint16_t* w_down,
                        const uint16_t* residual, uint16_t* out, void* ws, size_t ws_bytes,
                        void* stream);
+
+/* Expert weights in an MX format (device pointers, 16-byte aligned):
+ *   fmt             MOE_WFMT_MXFP8 or MOE_WFMT_MXFP4
+ *   gate_up         elements of the packed gate_up rows, [N, 2F, d_model] (SwiGLU: gate rows
+ *                   then up rows) or [N, F, d_model] (GELU): d_model bytes a row (MXFP8) or
+ *                   d_model / 2 (MXFP4)
+ *   gate_up_scales  [N, d_model / 32, 2F (or F)] uint8 E8M0: block b of row r at [e][b][r]
+ *   down            elements of [N, d_model, d_ff]: d_ff (MXFP8) or d_ff / 2 (MXFP4) bytes a row
+ *   down_scales     [N, d_ff / 32, d_model] uint8 E8M0
+ * The scale axis order (K blocks outer, rows inner) lets one TMA box carry a tile's scales. */
+typedef struct {
+  int32_t fmt;
+  const void* gate_up;
+  const uint8_t* gate_up_scales;
+  const void* down;
+  const uint8_t* down_scales;
+} moe_mx_weights;
+
+/* moe_grouped_ffn with MX weights. The weights stream from HBM in their packed form (1/2 or
+ * 1/4 of the bf16 bytes) and are decoded in shared memory, exactly, into bf16 (a power-of-two
+ * scale times an FP8/FP4 value is a bf16 value while it stays in bf16's normal range); the
+ * tensor-core arithmetic, h, y_perm and their rounding rules are those of moe_grouped_ffn on
+ * the decoded weights. Same workspace. MOE_ERR_INVALID for a bad fmt or a NULL pointer. */
+moe_status moe_grouped_ffn_mx(const moe_dims* dims, const uint16_t* x_perm,
+                              const int32_t* expert_offset, const moe_mx_weights* w, uint16_t* h,
+                              float* y_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_forward with MX expert weights (same workspace, layout and routing). */
+moe_status moe_forward_mx(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                          const float* logit_bias, const moe_mx_weights* w,
+                          const uint16_t* residual, uint16_t* out, void* ws, size_t ws_bytes,
+                          void* stream);
 
 /* Size of the scratch array built into the library for moe_route_noalloc. */
 #define MOE_ROUTE_NOALLOC_SCRATCH_BYTES 65536

@@ -8,3 +8,5 @@ from .moe_oracle import (capacity_from_factor, router_logits, softmax_over_exper
                          select_top_k, renormalise, assign_capacity_slots, route_from_logits,
                          expert_permutation, silu, gelu, expert_ffn, combine,
                          moe_layer_forward, router_statistics)
+from .mx_oracle import (MX_BLOCK, decode_e8m0, decode_e4m3, decode_e2m1,  # noqa: F401
+                        unpack_fp4, dequantize_mx)

@@ -52,8 +52,20 @@ class ForwardBuffers(ctypes.Structure):
         "pair_of_row", "x_perm", "h", "y_perm", "stage_ws")] + [("stage_ws_bytes", ctypes.c_size_t)]
 
 
+WFMT_BF16, WFMT_MXFP8, WFMT_MXFP4 = 0, 1, 2
+_WFMT = {"mxfp8": WFMT_MXFP8, "mxfp4": WFMT_MXFP4}
+
+
+class MxWeights(ctypes.Structure):
+    """``moe_mx_weights``: expert weights in an MX format (device pointers)."""
+    _fields_ = [("fmt", ctypes.c_int32), ("gate_up", ctypes.c_void_p),
+                ("gate_up_scales", ctypes.c_void_p), ("down", ctypes.c_void_p),
+                ("down_scales", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _DIMS = ctypes.POINTER(Dims)
+_MXW = ctypes.POINTER(MxWeights)
 _SIGS = {
     "moe_capacity": (ctypes.c_int32, [ctypes.c_double, ctypes.c_int32, ctypes.c_int32]),
     "moe_max_rows": (ctypes.c_int64, [_DIMS]),
@@ -69,6 +81,8 @@ _SIGS = {
     "moe_forward_layout": (ctypes.c_int, [_DIMS, _P, ctypes.c_size_t, ctypes.POINTER(ForwardBuffers)]),
     "moe_forward": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_route_noalloc": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_grouped_ffn_mx": (ctypes.c_int, [_DIMS, _P, _P, _MXW, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_forward_mx": (ctypes.c_int, [_DIMS, _P, _P, _P, _MXW, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_router_stats": (ctypes.c_int, [_DIMS, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P,
                                         ctypes.c_size_t, _P]),
     "moe_read_device_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int)]),
@@ -242,6 +256,44 @@ def grouped_ffn(dims: Dims, x_perm, expert_offset, w_gate_up, w_down, h, y_perm,
         _ptr(w_down, "w_down", torch.bfloat16, (N, d, F)), _ptr(h, "h", torch.bfloat16, (R, F)),
         _ptr(y_perm, "y_perm", torch.float32, (R, d)), _ptr(ws, "ws", torch.uint8), _nbytes(ws),
         _stream(stream)), "moe_grouped_ffn")
+
+
+def mx_weights(dims: Dims, fmt: str, gate_up, gate_up_scales, down, down_scales) -> MxWeights:
+    """Check shapes and dtypes of MX expert weights and describe them for the C ABI.
+    gate_up [N, rows, d_model or d_model/2] uint8, gate_up_scales [N, d_model/32, rows] uint8,
+    down [N, d_model, d_ff or d_ff/2] uint8, down_scales [N, d_ff/32, d_model] uint8."""
+    d, N, F = dims.d_model, dims.n_experts, dims.d_ff
+    rows = 2 * F if dims.act == ACT_SWIGLU else F
+    per = 1 if fmt == "mxfp8" else 2
+    return MxWeights(_WFMT[fmt],
+                     _ptr(gate_up, "gate_up", torch.uint8, (N, rows, d // per)),
+                     _ptr(gate_up_scales, "gate_up_scales", torch.uint8, (N, d // 32, rows)),
+                     _ptr(down, "down", torch.uint8, (N, d, F // per)),
+                     _ptr(down_scales, "down_scales", torch.uint8, (N, F // 32, d)))
+
+
+def grouped_ffn_mx(dims: Dims, x_perm, expert_offset, w: MxWeights, h, y_perm, ws,
+                   stream=None) -> None:
+    d, N, F = dims.d_model, dims.n_experts, dims.d_ff
+    R = max_rows(dims)
+    _check(_lib.moe_grouped_ffn_mx(
+        ctypes.byref(dims), _ptr(x_perm, "x_perm", torch.bfloat16, (R, d)),
+        _ptr(expert_offset, "expert_offset", torch.int32, (N + 1,)), ctypes.byref(w),
+        _ptr(h, "h", torch.bfloat16, (R, F)), _ptr(y_perm, "y_perm", torch.float32, (R, d)),
+        _ptr(ws, "ws", torch.uint8), _nbytes(ws), _stream(stream)), "moe_grouped_ffn_mx")
+
+
+def forward_mx_into(dims: Dims, x, w_router, logit_bias, w: MxWeights, residual, out, ws,
+                    stream=None) -> None:
+    """moe_forward_mx with caller-provided output and workspace (no allocation)."""
+    T, d, N = dims.T, dims.d_model, dims.n_experts
+    _check(_lib.moe_forward_mx(
+        ctypes.byref(dims), _ptr(x, "x", torch.bfloat16, (T, d)),
+        _ptr(w_router, "w_router", torch.float32, (N, d)),
+        _ptr(logit_bias, "logit_bias", torch.float32, (N,), allow_none=True), ctypes.byref(w),
+        _ptr(residual, "residual", torch.bfloat16, (T, d), allow_none=True),
+        _ptr(out, "out", torch.bfloat16, (T, d)), _ptr(ws, "ws", torch.uint8), _nbytes(ws),
+        _stream(stream)), "moe_forward_mx")
 
 
 def unpermute_combine(dims: Dims, y_perm, row_of_pair, topk_w, residual, out, ws=None,

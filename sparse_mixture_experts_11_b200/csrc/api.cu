@@ -270,26 +270,54 @@ moe_status moe_permute(const moe_dims* dims, const uint16_t* x, const int32_t* t
                                            status_of(ws), as_stream(stream)));
 }
 
-moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
-                           const int32_t* expert_offset, const uint16_t* w_gate_up,
-                           const uint16_t* w_down, uint16_t* h, float* y_perm, void* ws,
-                           size_t ws_bytes, void* stream) {
+namespace {
+// Expert weights of either storage: bf16 (scales null) or an MX format.
+struct Weights {
+  int fmt;
+  const void* gate_up;
+  const uint8_t* gate_up_scales;
+  const void* down;
+  const uint8_t* down_scales;
+};
+
+moe_status check_weights(const Weights& w) {
+  if (w.fmt != MOE_WFMT_BF16 && w.fmt != MOE_WFMT_MXFP8 && w.fmt != MOE_WFMT_MXFP4)
+    return MOE_ERR_INVALID;
+  if (!w.gate_up || !w.down) return MOE_ERR_INVALID;
+  if (w.fmt != MOE_WFMT_BF16 && (!w.gate_up_scales || !w.down_scales)) return MOE_ERR_INVALID;
+  if (!aligned16(w.gate_up) || !aligned16(w.down) ||
+      (w.gate_up_scales && !aligned16(w.gate_up_scales)) ||
+      (w.down_scales && !aligned16(w.down_scales)))
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+Weights weights_of(const moe_mx_weights* w) {
+  return Weights{w->fmt, w->gate_up, w->gate_up_scales, w->down, w->down_scales};
+}
+
+moe_status grouped_ffn_impl(const moe_dims* dims, const uint16_t* x_perm,
+                            const int32_t* expert_offset, const Weights& w, uint16_t* h,
+                            float* y_perm, void* ws, size_t ws_bytes, void* stream) {
   moe_status st = check_dims(dims);
   if (st != MOE_OK) return st;
   const int64_t rmax = max_rows(dims);
   if (dims->T == 0 || rmax == 0) return MOE_OK;
-  if (!x_perm || !expert_offset || !w_gate_up || !w_down || !h || !y_perm || !ws)
-    return MOE_ERR_INVALID;
-  if (!aligned16(x_perm) || !aligned16(expert_offset) || !aligned16(w_gate_up) ||
-      !aligned16(w_down) || !aligned16(h) || !aligned16(y_perm) || !aligned16(ws))
+  if ((st = check_weights(w)) != MOE_OK) return st;
+  if (!x_perm || !expert_offset || !h || !y_perm || !ws) return MOE_ERR_INVALID;
+  if (!aligned16(x_perm) || !aligned16(expert_offset) || !aligned16(h) || !aligned16(y_perm) ||
+      !aligned16(ws))
     return MOE_ERR_UNSUPPORTED;
   if (ws_bytes < stage_ws_bytes(dims)) return MOE_ERR_WORKSPACE;
   if ((st = check_device()) != MOE_OK) return st;
   moe::GroupedFfnArgs a{};
   a.x_perm = x_perm;
   a.expert_offset = expert_offset;
-  a.w_gate_up = w_gate_up;
-  a.w_down = w_down;
+  a.wfmt = w.fmt;
+  a.w_gate_up = w.gate_up;
+  a.w_down = w.down;
+  a.w_gate_up_scales = w.gate_up_scales;
+  a.w_down_scales = w.down_scales;
   a.h = h;
   a.y_perm = y_perm;
   a.N = dims->n_experts;
@@ -304,6 +332,24 @@ moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
   a.counters = reinterpret_cast<int*>(static_cast<char*>(ws) + moe::kStatusBytes);
   if (plan.part_bytes > 0) a.part = reinterpret_cast<float*>(shared_region_of(dims, ws));
   return launch_status(moe::launch_grouped_ffn(a, as_stream(stream)));
+}
+}  // namespace
+
+moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
+                           const int32_t* expert_offset, const uint16_t* w_gate_up,
+                           const uint16_t* w_down, uint16_t* h, float* y_perm, void* ws,
+                           size_t ws_bytes, void* stream) {
+  return grouped_ffn_impl(dims, x_perm, expert_offset,
+                          Weights{MOE_WFMT_BF16, w_gate_up, nullptr, w_down, nullptr}, h, y_perm,
+                          ws, ws_bytes, stream);
+}
+
+moe_status moe_grouped_ffn_mx(const moe_dims* dims, const uint16_t* x_perm,
+                              const int32_t* expert_offset, const moe_mx_weights* w, uint16_t* h,
+                              float* y_perm, void* ws, size_t ws_bytes, void* stream) {
+  if (w == nullptr || w->fmt == MOE_WFMT_BF16) return MOE_ERR_INVALID;
+  return grouped_ffn_impl(dims, x_perm, expert_offset, weights_of(w), h, y_perm, ws, ws_bytes,
+                          stream);
 }
 
 moe_status moe_unpermute_combine(const moe_dims* dims, const float* y_perm,
@@ -396,15 +442,16 @@ moe_status moe_forward_layout(const moe_dims* dims, void* ws, size_t ws_bytes,
   return MOE_OK;
 }
 
-moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_router,
-                       const float* logit_bias, const uint16_t* w_gate_up, const uint16_t* w_down,
-                       const uint16_t* residual, uint16_t* out, void* ws, size_t ws_bytes,
-                       void* stream) {
+namespace {
+moe_status forward_impl(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                        const float* logit_bias, const Weights& w, const uint16_t* residual,
+                        uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
   moe_forward_buffers b;
   moe_status st = moe_forward_layout(dims, ws, ws_bytes, &b);
   if (st != MOE_OK) return st;
   if (dims->T == 0) return MOE_OK;
-  if (!x || !w_router || !w_gate_up || !w_down || !out) return MOE_ERR_INVALID;
+  if (!x || !w_router || !out) return MOE_ERR_INVALID;
+  if ((st = check_weights(w)) != MOE_OK) return st;
   const int64_t rmax = max_rows(dims);
   if (moe::use_decode_route(dims->T, dims->n_experts, dims->d_model) &&
       rmax * dims->d_model * 2 <= moe::kDecodePermuteMaxBytes) {
@@ -428,11 +475,30 @@ moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_r
                      b.pair_of_row, b.x_perm, b.stage_ws, b.stage_ws_bytes, stream);
   }
   if (st != MOE_OK) return st;
-  st = moe_grouped_ffn(dims, b.x_perm, b.expert_offset, w_gate_up, w_down, b.h, b.y_perm,
-                       b.stage_ws, b.stage_ws_bytes, stream);
+  st = grouped_ffn_impl(dims, b.x_perm, b.expert_offset, w, b.h, b.y_perm, b.stage_ws,
+                        b.stage_ws_bytes, stream);
   if (st != MOE_OK) return st;
   return moe_unpermute_combine(dims, b.y_perm, b.row_of_pair, b.topk_w, residual, out, 0,
                                b.stage_ws, b.stage_ws_bytes, stream);
+}
+}  // namespace
+
+moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                       const float* logit_bias, const uint16_t* w_gate_up, const uint16_t* w_down,
+                       const uint16_t* residual, uint16_t* out, void* ws, size_t ws_bytes,
+                       void* stream) {
+  return forward_impl(dims, x, w_router, logit_bias,
+                      Weights{MOE_WFMT_BF16, w_gate_up, nullptr, w_down, nullptr}, residual, out,
+                      ws, ws_bytes, stream);
+}
+
+moe_status moe_forward_mx(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                          const float* logit_bias, const moe_mx_weights* w,
+                          const uint16_t* residual, uint16_t* out, void* ws, size_t ws_bytes,
+                          void* stream) {
+  if (w == nullptr || w->fmt == MOE_WFMT_BF16) return MOE_ERR_INVALID;
+  return forward_impl(dims, x, w_router, logit_bias, weights_of(w), residual, out, ws, ws_bytes,
+                      stream);
 }
 
 moe_status moe_read_device_error(void* ws, void* stream, moe_status* err) {

@@ -47,8 +47,13 @@
 //                 last), so the partials take two slots.
 // Every wait is bounded; on timeout the CTA records MOE_ERR_TIMEOUT, stops issuing work, waits
 // (bounded) for its own TMA copies and MMAs, frees TMEM and exits.
+#include <string.h>
+
 #include <algorithm>
 #include <mutex>
+
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "launch.h"
@@ -95,18 +100,71 @@ struct FfnParams {
   int weight_policy;  // 0 evict_normal, 1 evict_first
 };
 
-template <int BM>
+// Weight storage: bf16, or an MX format (blocks of 32 elements along K sharing one E8M0
+// scale) with E4M3 or E2M1 elements, decoded exactly to bf16 in shared memory.
+enum { WFMT_BF16 = 0, WFMT_MXFP8 = 1, WFMT_MXFP4 = 2 };
+constexpr int kConvThreads = 256;  // MX decoders (warps 7-14)
+
+template <int BM, int WFMT>
 struct Cfg {
+  static constexpr bool MX = WFMT != WFMT_BF16;
+  static constexpr int THREADS = MX ? kThreads + 32 + kConvThreads : kThreads;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = kUmmaN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (kSmemBudget / STAGE_BYTES) > 8 ? 8 : (kSmemBudget / STAGE_BYTES);
+  // MX: two bf16 stages (decoded from shared memory, not waiting on HBM) and a deeper ring of
+  // packed stages: 256 rows of 64 elements (64 or 32 bytes a row) plus 2 x 256 scale bytes
+  static constexpr int ROW_BYTES = WFMT == WFMT_MXFP8 ? BK : BK / 2;
+  static constexpr int STG_BYTES = MX ? kUmmaN * ROW_BYTES + 2 * kUmmaN : 0;
+  static constexpr int STAGES_FIT = (kSmemBudget / STAGE_BYTES) > 8 ? 8 : (kSmemBudget / STAGE_BYTES);
+  static constexpr int STAGES = MX ? 2 : STAGES_FIT;
+  static constexpr int SST_FIT = MX ? (kSmemBudget - STAGES * STAGE_BYTES) / STG_BYTES : 0;
+  static constexpr int SST = SST_FIT > 16 ? 16 : SST_FIT;
   static constexpr int TMEM_COLS = 2 * kUmmaN;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SST * STG_BYTES + 1024;  // + alignment slack
   static_assert(TMEM_COLS <= 512, "two accumulators must fit in TMEM");
   static_assert(STAGES >= 2, "pipeline depth");
+  static_assert(!MX || SST >= 4, "MX staging depth");
   static_assert(BM == 64 || BM == 128, "UMMA M");
 };
+
+// Decoders of one MX row segment: 8 elements and the block scale X = 2^(s - 127) -> 8 bf16
+// (one 16-byte chunk). Elements convert exactly to fp16 (CUDA's FP8/FP4 conversions), then
+// to fp32; the product with a power of two and the final bf16 rounding are exact while the
+// result stays in bf16's normal range.
+__device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
+  if (s == 255u) return __uint_as_float(0x7fc00000u);
+  if (s == 0u) return __uint_as_float(0x00400000u);  // 2^-127
+  return __uint_as_float(s << 23);
+}
+
+__device__ __forceinline__ uint32_t half2raw_to_bf16x2(__half2_raw h, float x) {
+  __half_raw lo, hi;
+  lo.x = h.x;
+  hi.x = h.y;
+  return pack_bf16x2(__half2float(__half(lo)) * x, __half2float(__half(hi)) * x);
+}
+
+__device__ __forceinline__ uint4 decode8_e4m3(uint2 w, float x) {
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t word = i < 2 ? w.x : w.y;
+    const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>(word >> (16 * (i & 1)));
+    o[i] = half2raw_to_bf16x2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3), x);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ uint4 decode8_e2m1(uint32_t w, float x) {
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // byte i holds elements 2i (low nibble) and 2i + 1
+    const __nv_fp4x2_storage_t pair = static_cast<__nv_fp4x2_storage_t>(w >> (8 * i));
+    o[i] = half2raw_to_bf16x2(__nv_cvt_fp4x2_to_halfraw2(pair, __NV_E2M1), x);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
 
 __device__ __forceinline__ uint64_t make_policy(int which) {
   uint64_t p;
@@ -407,13 +465,18 @@ __device__ __forceinline__ bool epilogue_segment(const FfnParams& fp, const Phas
   return true;
 }
 
-template <int EPI1, int BN1, int BM>
-__global__ void __launch_bounds__(kThreads, 1)
+// MX weights (WFMT != 0): tmB1 / tmB2 map the packed elements (uint8) and tmS1 / tmS2 the
+// scales; warp 6 streams both into the packed ring and warps 7-14 decode each stage into
+// the B half of a bf16 stage, which the MMA then reads as for bf16 weights.
+template <int EPI1, int BN1, int BM, int WFMT>
+__global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
     grouped_ffn_kernel(const __grid_constant__ CUtensorMap tmA1,
                        const __grid_constant__ CUtensorMap tmB1,
                        const __grid_constant__ CUtensorMap tmA2,
-                       const __grid_constant__ CUtensorMap tmB2, const FfnParams p) {
-  using C = Cfg<BM>;
+                       const __grid_constant__ CUtensorMap tmB2,
+                       const __grid_constant__ CUtensorMap tmS1,
+                       const __grid_constant__ CUtensorMap tmS2, const FfnParams p) {
+  using C = Cfg<BM, WFMT>;
   static_assert(EPI1 != EPI_SWIGLU || 2 * BN1 == kUmmaN, "SwiGLU tile: gate | up halves");
   static_assert(EPI1 == EPI_SWIGLU || BN1 == kUmmaN, "GELU tile");
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
@@ -430,20 +493,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ Sched s_sched[2];
   __shared__ int s_fixup;
   __shared__ int s_last_cta;
+  __shared__ __align__(8) uint64_t sfull_bar[C::MX ? C::SST : 1];
+  __shared__ __align__(8) uint64_t sempty_bar[C::MX ? C::SST : 1];
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int N = p.n_experts;
   const uint32_t tiles = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  const uint32_t stg0 = tiles + C::STAGES * C::STAGE_BYTES;  // MX: packed ring
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmA1);
     prefetch_tensormap(&tmB1);
     prefetch_tensormap(&tmA2);
     prefetch_tensormap(&tmB2);
+    if (C::MX) {
+      prefetch_tensormap(&tmS1);
+      prefetch_tensormap(&tmS2);
+      for (int s = 0; s < C::SST; ++s) {
+        mbar_init(smem_u32(&sfull_bar[s]), 1);
+        mbar_init(smem_u32(&sempty_bar[s]), kConvThreads);
+      }
+    }
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_u32(&full_bar[s]), 1);
+      // MX: the A copy's transaction bytes plus one arrival per decoder thread
+      mbar_init(smem_u32(&full_bar[s]), C::MX ? 1 + kConvThreads : 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -550,16 +625,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t fb = smem_u32(&full_bar[s]);
             const uint32_t a_dst = tiles + s * C::STAGE_BYTES;
             const uint32_t b_dst = a_dst + C::A_BYTES;
-            mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-            if (ph == 0) {
-              if (EPI1 == EPI_SWIGLU) {
-                tma_load_4d(b_dst, &tmB1, fb, kb * BK, c.n0, 0, c.e, pol_b);
-                tma_load_4d(b_dst + BN1 * BK * 2, &tmB1, fb, kb * BK, c.n0, 1, c.e, pol_b);
+            mbar_arrive_expect_tx(fb, C::MX ? C::A_BYTES : C::STAGE_BYTES);
+            if (!C::MX) {  // MX: the decoders fill the B half
+              if (ph == 0) {
+                if (EPI1 == EPI_SWIGLU) {
+                  tma_load_4d(b_dst, &tmB1, fb, kb * BK, c.n0, 0, c.e, pol_b);
+                  tma_load_4d(b_dst + BN1 * BK * 2, &tmB1, fb, kb * BK, c.n0, 1, c.e, pol_b);
+                } else {
+                  tma_load_3d(b_dst, &tmB1, fb, kb * BK, c.n0, c.e, pol_b);
+                }
               } else {
-                tma_load_3d(b_dst, &tmB1, fb, kb * BK, c.n0, c.e, pol_b);
+                tma_load_3d(b_dst, &tmB2, fb, kb * BK, c.n0, c.e, pol_b);
               }
-            } else {
-              tma_load_3d(b_dst, &tmB2, fb, kb * BK, c.n0, c.e, pol_b);
             }
             if (ready) {
               tma_load_2d(a_dst, tA, fb, kb * BK, c.m0, pol_a);
@@ -645,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else {
+  } else if (warp < 6) {
     // ---------------------------------------------------------------- epilogue (warps 2..5)
     int tc = 0;
     uint32_t epi_phase = 0;
@@ -687,6 +764,104 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_abort = 1;
       report_error(p.status, MOE_ERR_TIMEOUT);
     }
+  } else if (C::MX && warp == 6) {
+    // ---------------------------------------------------------------- MX packed-ring producer
+    if (lane == 0) {
+      const uint64_t pol_b = make_policy(p.weight_policy);
+      int it = 0;
+      bool ok = true;
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        const Sched sc = s_sched[ph];
+        const int bn = ph == 0 ? BN1 : kDnBn;
+        SegCursor cur(sc);
+        Seg sg;
+        while (ok && cur.next(sc, sg)) {
+          const TileCoord c = decode_tile<BM>(sg.tile, N, bn, p.ph[ph].n_tiles_n, s_mt, s_off);
+          for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+            const int s = it % C::SST;
+            if (!mbar_wait(smem_u32(&sempty_bar[s]), ((it / C::SST) & 1) ^ 1u, p.timeout_ns, &s_abort)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = smem_u32(&sfull_bar[s]);
+            const uint32_t dst = stg0 + s * C::STG_BYTES;
+            const uint32_t sc_dst = dst + kUmmaN * C::ROW_BYTES;  // [2 blocks][256 rows] scales
+            mbar_arrive_expect_tx(fb, C::STG_BYTES);
+            const int kx = kb * C::ROW_BYTES;  // byte column of this k block's elements
+            if (ph == 0 && EPI1 == EPI_SWIGLU) {
+              tma_load_4d(dst, &tmB1, fb, kx, c.n0, 0, c.e, pol_b);  // gate rows
+              tma_load_4d(dst + BN1 * C::ROW_BYTES, &tmB1, fb, kx, c.n0, 1, c.e, pol_b);  // up rows
+              tma_load_4d(sc_dst, &tmS1, fb, c.n0, 0, 2 * kb, c.e, pol_b);  // [2][128] gate
+              tma_load_4d(sc_dst + 2 * BN1, &tmS1, fb, c.n0, 1, 2 * kb, c.e, pol_b);  // [2][128] up
+            } else if (ph == 0) {
+              tma_load_3d(dst, &tmB1, fb, kx, c.n0, c.e, pol_b);
+              tma_load_3d(sc_dst, &tmS1, fb, c.n0, 2 * kb, c.e, pol_b);
+            } else {
+              tma_load_3d(dst, &tmB2, fb, kx, c.n0, c.e, pol_b);
+              tma_load_3d(sc_dst, &tmS2, fb, c.n0, 2 * kb, c.e, pol_b);
+            }
+          }
+        }
+      }
+      if (!ok) {
+        s_abort = 1;
+        report_error(p.status, MOE_ERR_TIMEOUT);
+      }
+      for (int i = max(0, it - C::SST); i < it; ++i)
+        mbar_wait(smem_u32(&sfull_bar[i % C::SST]), (i / C::SST) & 1, kDrainTimeoutNs, nullptr);
+    }
+  } else if (C::MX) {
+    // ---------------------------------------------------------------- MX decoders (warps 7..14)
+    // Thread r decodes row r of every stage: 64 elements (8 chunks of 8) with the row's two
+    // block scales, into the 128B-swizzled K-major layout the MMA reads (chunk c of row r at
+    // 16 * (c ^ (r & 7))).
+    const int r = threadIdx.x - (kThreads + 32);  // 0..255
+    int it = 0;
+    bool ok = true;
+    for (int ph = 0; ph < 2 && ok; ++ph) {
+      const Sched sc = s_sched[ph];
+      // scale layout of this phase's stages: SwiGLU gate/up halves, or one [2][256] block
+      const bool halves = ph == 0 && EPI1 == EPI_SWIGLU;
+      const int sc_idx0 = halves ? (r >> 7) * 256 + (r & 127) : r;
+      const int sc_step = halves ? 128 : 256;
+      SegCursor cur(sc);
+      Seg sg;
+      while (ok && cur.next(sc, sg)) {
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+          const int s2 = it % C::SST, s = it % C::STAGES;
+          const bool got = mbar_wait(smem_u32(&sfull_bar[s2]), (it / C::SST) & 1, p.timeout_ns, &s_abort) &&
+                           mbar_wait(smem_u32(&empty_bar[s]), ((it / C::STAGES) & 1) ^ 1u, p.timeout_ns, &s_abort);
+          if (!got) {
+            ok = false;
+            break;
+          }
+          const uint8_t* stg = dyn_smem + (stg0 - smem_u32(dyn_smem)) + s2 * C::STG_BYTES;
+          const uint8_t* row = stg + r * C::ROW_BYTES;
+          const uint8_t* scl = stg + kUmmaN * C::ROW_BYTES;
+          const float x0 = e8m0_to_f32(scl[sc_idx0]);
+          const float x1 = e8m0_to_f32(scl[sc_idx0 + sc_step]);
+          uint8_t* bdst = dyn_smem + (tiles - smem_u32(dyn_smem)) + s * C::STAGE_BYTES + C::A_BYTES +
+                          r * 128;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const float x = ch < 4 ? x0 : x1;  // elements 0..31: block 0; 32..63: block 1
+            uint4 v;
+            if (WFMT == WFMT_MXFP8)
+              v = decode8_e4m3(*reinterpret_cast<const uint2*>(row + ch * 8), x);
+            else
+              v = decode8_e2m1(*reinterpret_cast<const uint32_t*>(row + ch * 4), x);
+            *reinterpret_cast<uint4*>(bdst + ((ch ^ (r & 7)) << 4)) = v;
+          }
+          fence_proxy_async_smem();  // generic stores -> visible to the tensor core
+          mbar_arrive(smem_u32(&full_bar[s]));
+          mbar_arrive(smem_u32(&sempty_bar[s2]));
+        }
+      }
+    }
+    if (!ok) {
+      s_abort = 1;
+      report_error(p.status, MOE_ERR_TIMEOUT);
+    }
   }
 
   tc_fence_before_sync();
@@ -703,7 +878,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (s_last_cta) {
     __threadfence();
-    for (int i = threadIdx.x; i < s_mt[N]; i += kThreads) p.h_ready[i] = 0;
+    for (int i = threadIdx.x; i < s_mt[N]; i += C::THREADS) p.h_ready[i] = 0;
     if (threadIdx.x == 0) *p.done_ctas = 0;
   }
 }
@@ -749,20 +924,48 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
   return r == CUDA_SUCCESS;
 }
 
-template <int EPI1, int BN1, int BM>
+// uint8 tensor map without swizzle (MX elements and scales; dims[0] contiguous).
+bool make_map_u8(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t gd[5];
+  cuuint64_t gs[4];
+  cuuint32_t bx[5];
+  cuuint32_t es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) gs[i] = strides_bytes[i];
+  }
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank),
+                        const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int EPI1, int BN1, int BM, int WFMT>
 cudaError_t launch_one(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
-                       const CUtensorMap& b2, const FfnParams& fp, int grid, cudaStream_t s) {
-  using C = Cfg<BM>;
+                       const CUtensorMap& b2, const CUtensorMap& s1, const CUtensorMap& s2,
+                       const FfnParams& fp, int grid, cudaStream_t s) {
+  using C = Cfg<BM, WFMT>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(grouped_ffn_kernel<EPI1, BN1, BM>,
+    attr_err = cudaFuncSetAttribute(grouped_ffn_kernel<EPI1, BN1, BM, WFMT>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  return launch_pdl(grouped_ffn_kernel<EPI1, BN1, BM>, dim3(grid), dim3(kThreads), C::SMEM_BYTES,
-                    s, a1, b1, a2, b2, fp);
+  return launch_pdl(grouped_ffn_kernel<EPI1, BN1, BM, WFMT>, dim3(grid), dim3(C::THREADS),
+                    C::SMEM_BYTES, s, a1, b1, a2, b2, s1, s2, fp);
 }
+
+template <int WFMT>
+cudaError_t launch_fmt(bool swiglu, int bm, const CUtensorMap& a1, const CUtensorMap& b1,
+                       const CUtensorMap& a2, const CUtensorMap& b2, const CUtensorMap& s1,
+                       const CUtensorMap& s2, const FfnParams& fp, int grid, cudaStream_t s);
 
 // sum_e ceil(m_e / bm) <= ceil(R / bm) + (experts with rows)
 int64_t m_tiles_upper_bound(int64_t r_max, int N, int bm) {
@@ -829,14 +1032,49 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   // batches) they are pure streams and should not displace the activations in L2
   const int wpol = (a.rows_per_expert <= bm) ? 1 : 0;
 
-  CUtensorMap mA1, mB1, mA2, mB2;
+  CUtensorMap mA1, mB1, mA2, mB2, mS1, mS2;
+  memset(&mS1, 0, sizeof(mS1));  // bf16 weights: the scale maps are not read
+  memset(&mS2, 0, sizeof(mS2));
   {
     const uint64_t dims[2] = {d, R};
     const uint64_t str[1] = {d * 2};
     const uint32_t box[2] = {BK, static_cast<uint32_t>(bm)};
     if (!make_map(&mA1, a.x_perm, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
-  if (swiglu) {
+  if (a.wfmt != MOE_WFMT_BF16) {
+    // packed elements: [N][rows][K * rb / 64] bytes, no swizzle; scales: [N][K/32][rows] bytes
+    const uint64_t rb = a.wfmt == MOE_WFMT_MXFP8 ? BK : BK / 2;  // bytes per row and k block
+    const uint64_t db = d * rb / BK, fb = F * rb / BK;
+    if (swiglu) {
+      const uint64_t dims[4] = {db, F, 2, N};
+      const uint64_t str[3] = {db, F * db, 2 * F * db};
+      const uint32_t box[4] = {static_cast<uint32_t>(rb), static_cast<uint32_t>(bn_gu), 1, 1};
+      if (!make_map_u8(&mB1, a.w_gate_up, 4, dims, str, box)) return cudaErrorInvalidValue;
+      const uint64_t sd[4] = {F, 2, d / 32, N};
+      const uint64_t ss[3] = {F, 2 * F, (d / 32) * 2 * F};
+      const uint32_t sb[4] = {static_cast<uint32_t>(bn_gu), 1, 2, 1};
+      if (!make_map_u8(&mS1, a.w_gate_up_scales, 4, sd, ss, sb)) return cudaErrorInvalidValue;
+    } else {
+      const uint64_t dims[3] = {db, F, N};
+      const uint64_t str[2] = {db, F * db};
+      const uint32_t box[3] = {static_cast<uint32_t>(rb), static_cast<uint32_t>(bn_gu), 1};
+      if (!make_map_u8(&mB1, a.w_gate_up, 3, dims, str, box)) return cudaErrorInvalidValue;
+      const uint64_t sd[3] = {F, d / 32, N};
+      const uint64_t ss[2] = {F, (d / 32) * F};
+      const uint32_t sb[3] = {static_cast<uint32_t>(bn_gu), 2, 1};
+      if (!make_map_u8(&mS1, a.w_gate_up_scales, 3, sd, ss, sb)) return cudaErrorInvalidValue;
+    }
+    {
+      const uint64_t dims[3] = {fb, d, N};
+      const uint64_t str[2] = {fb, d * fb};
+      const uint32_t box[3] = {static_cast<uint32_t>(rb), static_cast<uint32_t>(kDnBn), 1};
+      if (!make_map_u8(&mB2, a.w_down, 3, dims, str, box)) return cudaErrorInvalidValue;
+      const uint64_t sd[3] = {d, F / 32, N};
+      const uint64_t ss[2] = {d, (F / 32) * d};
+      const uint32_t sb[3] = {static_cast<uint32_t>(kDnBn), 2, 1};
+      if (!make_map_u8(&mS2, a.w_down_scales, 3, sd, ss, sb)) return cudaErrorInvalidValue;
+    }
+  } else if (swiglu) {
     const uint64_t dims[4] = {d, F, 2, N};
     const uint64_t str[3] = {d * 2, F * d * 2, 2 * F * d * 2};
     const uint32_t box[4] = {BK, static_cast<uint32_t>(bn_gu), 1, 1};
@@ -853,7 +1091,7 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
     const uint32_t box[2] = {BK, static_cast<uint32_t>(bm)};
     if (!make_map(&mA2, a.h, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
-  {
+  if (a.wfmt == MOE_WFMT_BF16) {
     const uint64_t dims[3] = {F, d, N};
     const uint64_t str[2] = {F * 2, d * F * 2};
     const uint32_t box[3] = {BK, static_cast<uint32_t>(kDnBn), 1};
@@ -902,11 +1140,24 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   const int64_t useful = std::max(useful_ctas(plan.tiles1_ub, p1.num_kb, p1.sk_ctas),
                                   useful_ctas(plan.tiles2_ub, p2.num_kb, p2.sk_ctas));
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(useful, di.sm_count)));
-  if (bm == 64)
-    return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 64>(mA1, mB1, mA2, mB2, fp, grid, s)
-                  : launch_one<EPI_GELU, kGuBnGelu, 64>(mA1, mB1, mA2, mB2, fp, grid, s);
-  return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128>(mA1, mB1, mA2, mB2, fp, grid, s)
-                : launch_one<EPI_GELU, kGuBnGelu, 128>(mA1, mB1, mA2, mB2, fp, grid, s);
+  if (a.wfmt == MOE_WFMT_MXFP8)
+    return launch_fmt<WFMT_MXFP8>(swiglu, bm, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
+  if (a.wfmt == MOE_WFMT_MXFP4)
+    return launch_fmt<WFMT_MXFP4>(swiglu, bm, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
+  return launch_fmt<WFMT_BF16>(swiglu, bm, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
 }
+
+namespace {
+template <int WFMT>
+cudaError_t launch_fmt(bool swiglu, int bm, const CUtensorMap& a1, const CUtensorMap& b1,
+                       const CUtensorMap& a2, const CUtensorMap& b2, const CUtensorMap& s1,
+                       const CUtensorMap& s2, const FfnParams& fp, int grid, cudaStream_t s) {
+  if (bm == 64)
+    return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 64, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s)
+                  : launch_one<EPI_GELU, kGuBnGelu, 64, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s);
+  return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s)
+                : launch_one<EPI_GELU, kGuBnGelu, 128, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s);
+}
+}  // namespace
 
 }  // namespace moe

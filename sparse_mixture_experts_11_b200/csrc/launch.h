@@ -168,8 +168,11 @@ FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max,
 struct GroupedFfnArgs {
   const uint16_t* x_perm;
   const int32_t* expert_offset;
-  const uint16_t* w_gate_up;
-  const uint16_t* w_down;
+  int wfmt;                    // moe_wfmt: bf16 or an MX format
+  const void* w_gate_up;       // bf16 weights, or MX packed elements
+  const void* w_down;
+  const uint8_t* w_gate_up_scales;  // MX only: E8M0 scales [N][K/32][rows]
+  const uint8_t* w_down_scales;
   uint16_t* h;
   float* y_perm;
   int N, d, F, act;

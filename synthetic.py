@@ -67,6 +67,7 @@ SHAPES = {
 
 # tensor ids for per-tensor generator streams
 _X, _WR, _WGU, _WD = 1, 2, 3, 4
+_WGU_Q, _WGU_S, _WD_Q, _WD_S = 5, 6, 7, 8
 
 
 def _gen(device: torch.device, seed: int, tensor_id: int, sub: int = 0) -> torch.Generator:
@@ -138,3 +139,60 @@ def make_custom_inputs(T: int, d_model: int, n_experts: int, d_ff: int, act: str
     if router_std is not None:
         out["w_router"] = _normal((n_experts, d_model), router_std, torch.device(device), seed, _WR)
     return out
+
+
+# ---------------------------------------------------------------- MX-format expert weights
+# Expert weights stored in an MX format are drawn as codes directly (no quantisation step):
+#   element codes: "mxfp8" E4M3 codes uniform over the 254 non-NaN codes; "mxfp4" E2M1 codes
+#                  uniform over all 16 codes, two per byte;
+#   scale codes:   E8M0 codes 127 + scale_exp + U{-1, 0, 1} per block of 32 elements.
+# scale_exp is chosen so that the decoded weights have magnitudes like the bf16 recipe's
+# (E4M3 codes reach 448, E2M1 codes 6).
+MX_SCALE_EXP = {"mxfp8": -13, "mxfp4": -8}
+
+
+def _mx_codes(shape, fmt: str, g: torch.Generator, device) -> torch.Tensor:
+    if fmt == "mxfp8":
+        c = torch.randint(0, 254, shape, generator=g, device=device, dtype=torch.int32)
+        c = c + (c >= 127).to(torch.int32)  # skip 0x7F; 0xFF is never drawn
+        return c.to(torch.uint8)
+    if fmt == "mxfp4":
+        packed = shape[:-1] + (shape[-1] // 2,)
+        return torch.randint(0, 256, packed, generator=g, device=device, dtype=torch.int32).to(torch.uint8)
+    raise ValueError(fmt)
+
+
+def make_mx_matrix_stack(n_experts: int, rows: int, K: int, fmt: str, *, seed: int, tensor_id: int,
+                         scale_tensor_id: int, device="cpu") -> Tuple[torch.Tensor, torch.Tensor]:
+    """elements [N, rows, K] (mxfp8) or [N, rows, K/2] (mxfp4) uint8, scales [N, K/32, rows] uint8."""
+    dev = torch.device(device)
+    kb = K if fmt == "mxfp8" else K // 2
+    el = torch.empty((n_experts, rows, kb), dtype=torch.uint8, device=dev)
+    sc = torch.empty((n_experts, K // 32, rows), dtype=torch.uint8, device=dev)
+    for e in range(n_experts):
+        el[e].copy_(_mx_codes((rows, K), fmt, _gen(dev, seed, tensor_id, e), dev))
+        j = torch.randint(-1, 2, (K // 32, rows), generator=_gen(dev, seed, scale_tensor_id, e),
+                          device=dev, dtype=torch.int32)
+        sc[e].copy_((127 + MX_SCALE_EXP[fmt] + j).to(torch.uint8))
+    return el, sc
+
+
+def make_mx_layer_inputs(shape: LayerShape, T: int, fmt: str, *, seed: int = 0, device="cpu") -> dict:
+    """Hidden states and router as in make_layer_inputs; expert weights in an MX format:
+    w_gate_up_q/_s for the packed gate_up rows ([N, 2F or F, d]) and w_down_q/_s ([N, d, F])."""
+    dev = torch.device(device)
+    N, d, F = shape.n_experts, shape.d_model, shape.d_ff
+    w_router = _normal((N, d), 1.0 / math.sqrt(d), dev, seed, _WR)
+    bias = zipf_logit_bias(N, shape.zipf_s).to(dev) if shape.zipf_s is not None else None
+    gq, gs = make_mx_matrix_stack(N, shape.gate_up_rows(), d, fmt, seed=seed, tensor_id=_WGU_Q,
+                                  scale_tensor_id=_WGU_S, device=dev)
+    dq, ds = make_mx_matrix_stack(N, d, F, fmt, seed=seed, tensor_id=_WD_Q, scale_tensor_id=_WD_S,
+                                  device=dev)
+    return {"x": make_hidden(T, d, seed=seed, device=dev), "w_router": w_router, "logit_bias": bias,
+            "wfmt": fmt, "w_gate_up_q": gq, "w_gate_up_s": gs, "w_down_q": dq, "w_down_s": ds}
+
+
+def make_mx_custom_inputs(T: int, d_model: int, n_experts: int, d_ff: int, act: str, fmt: str, *,
+                          seed: int = 0, device="cpu", zipf_s: Optional[float] = None) -> dict:
+    shape = LayerShape("custom", d_model, n_experts, 1, d_ff, act, None, (T,), zipf_s)
+    return make_mx_layer_inputs(shape, T, fmt, seed=seed, device=device)

@@ -52,7 +52,8 @@ class StageRun:
         x = inp["x"]
         T, d = x.shape
         N = inp["w_router"].shape[0]
-        F = inp["w_down"].shape[2]
+        # MX weights: [N, F/32, d] down-projection scales give F
+        F = inp["w_down"].shape[2] if "w_down" in inp else 32 * inp["w_down_s"].shape[1]
         self.dims = moe.make_dims(T, d, N, top_k, F, act, cap)
         R = moe.max_rows(self.dims)
         self.R_max = R
@@ -74,6 +75,13 @@ class StageRun:
         self.out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
         self.out32 = torch.empty((T, d), dtype=torch.float32, device=dev)
         self.inp = inp
+        if "wfmt" in inp:
+            self.mx = moe.mx_weights(self.dims, inp["wfmt"], inp["w_gate_up_q"], inp["w_gate_up_s"],
+                                     inp["w_down_q"], inp["w_down_s"])
+            self.gu, self.dn = mx_weight_getters(inp)
+        else:
+            self.mx = None
+            self.gu, self.dn = expert_weights_f64(inp["w_gate_up"]), expert_weights_f64(inp["w_down"])
 
     def run(self, residual=True):
         i = self.inp
@@ -82,8 +90,12 @@ class StageRun:
                   self.topk_w, self.slot, self.expert_count, self.ws)
         moe.permute(self.dims, i["x"], self.topk_idx, self.slot, self.expert_count,
                     self.expert_offset, self.row_of_pair, self.pair_of_row, self.x_perm, self.ws)
-        moe.grouped_ffn(self.dims, self.x_perm, self.expert_offset, i["w_gate_up"], i["w_down"],
-                        self.h, self.y_perm, self.ws)
+        if self.mx is not None:
+            moe.grouped_ffn_mx(self.dims, self.x_perm, self.expert_offset, self.mx, self.h,
+                               self.y_perm, self.ws)
+        else:
+            moe.grouped_ffn(self.dims, self.x_perm, self.expert_offset, i["w_gate_up"],
+                            i["w_down"], self.h, self.y_perm, self.ws)
         moe.unpermute_combine(self.dims, self.y_perm, self.row_of_pair, self.topk_w, res, self.out,
                               self.ws)
         moe.unpermute_combine(self.dims, self.y_perm, self.row_of_pair, self.topk_w, res, self.out32,
@@ -142,12 +154,26 @@ def expert_weights_f64(w: torch.Tensor):
     return get
 
 
+def mx_weight_getters(inp):
+    """Lazy per-expert float64 weights decoded from MX storage by the oracle."""
+    fmt = inp["wfmt"]
+
+    def make(q, sc):
+        cache = {}
+
+        def get(e):
+            if e not in cache:
+                cache[e] = oracle.dequantize_mx(q[e].cpu().numpy(), sc[e].cpu().numpy(), fmt)
+            return cache[e]
+        return get
+    return make(inp["w_gate_up_q"], inp["w_gate_up_s"]), make(inp["w_down_q"], inp["w_down_s"])
+
+
 def check_outputs(run: StageRun, routing: dict, act: str, tokens=None, residual=True):
     i = run.inp
     x = f64(i["x"])
     res = x if residual else None
-    want = oracle.combine(x, routing, expert_weights_f64(i["w_gate_up"]),
-                          expert_weights_f64(i["w_down"]), act, res, tokens)
+    want = oracle.combine(x, routing, run.gu, run.dn, act, res, tokens)
     sel = slice(None) if tokens is None else torch.from_numpy(np.asarray(tokens)).long().cuda()
     g32 = f64(run.out32[sel])
     g16 = f64(run.out[sel])
@@ -189,8 +215,7 @@ def check_expert_rows(run: StageRun, routing: dict, act: str, rows: np.ndarray):
     por = run.pair_of_row.cpu().numpy()
     k = run.dims.top_k
     x = run.inp["x"]
-    gu = expert_weights_f64(run.inp["w_gate_up"])
-    dn = expert_weights_f64(run.inp["w_down"])
+    gu, dn = run.gu, run.dn
     y = f64(run.y_perm[torch.from_numpy(rows).long().cuda()])
     for n, r in enumerate(rows):
         e = int(np.searchsorted(off, r, side="right") - 1)

@@ -306,3 +306,58 @@ ALL_PINS = [pin_capacity_demo, pin_capacity_formula, pin_hand_routing, pin_top1_
             pin_two_way_weights, pin_brute_force_routing, pin_ffn_hand_cases,
             pin_activation_limits, pin_dense_special_case, pin_single_expert_layer,
             pin_invariants, pin_zero_down_weights, pin_aux_loss_closed_forms]
+
+
+# ---------------------------------------------------------------- MX weight formats
+# Pins of oracle/mx_oracle.py against the OCP Microscaling (MX) v1.0 definitions (closed
+# forms of the scale and element encodings) and against torch's own float8_e4m3fn cast.
+def pin_e8m0_closed_forms(m):
+    v = m.decode_e8m0(np.array([127, 128, 126, 0, 254, 255]))
+    assert v[:5].tolist() == [1.0, 2.0, 0.5, 2.0 ** -127, 2.0 ** 127]
+    assert math.isnan(v[5])
+
+
+def pin_e4m3_closed_forms(m):
+    codes = np.array([0x00, 0x80, 0x38, 0xB8, 0x40, 0x7E, 0xFE, 0x08, 0x01, 0x07, 0x3C])
+    want = [0.0, -0.0, 1.0, -1.0, 2.0, 448.0, -448.0, 2.0 ** -6, 2.0 ** -9, 7 / 8 * 2.0 ** -6, 1.5]
+    assert m.decode_e4m3(codes).tolist() == want
+    assert np.isnan(m.decode_e4m3(np.array([0x7F, 0xFF]))).all()
+
+
+def pin_e4m3_against_torch(m):
+    import torch
+    codes = np.arange(256)
+    got = m.decode_e4m3(codes)
+    ref = torch.tensor(codes, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+
+
+def pin_e2m1_table(m):
+    # the spec's FP4 E2M1 magnitudes for codes 0..7; codes 8..15 are their negatives
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    v = m.decode_e2m1(np.arange(16))
+    assert v[:8].tolist() == mags
+    assert (-v[8:]).tolist() == mags and np.signbit(v[8])
+
+
+def pin_fp4_nibble_order(m):
+    # element 2i is the low nibble of byte i
+    assert m.unpack_fp4(np.array([[0x21, 0xF0]])).tolist() == [[1, 2, 0, 15]]
+
+
+def pin_dequantize_blocks(m):
+    # scales are [K/32, rows]: row 0 gets 2^0 then 2^3, row 1 gets 2^2 then 2^-1
+    scales = np.array([[127, 129], [130, 126]], dtype=np.uint8)
+    w8 = m.dequantize_mx(np.full((2, 64), 0x38, dtype=np.uint8), scales, "mxfp8")  # all 1.0
+    assert w8[0].tolist() == [1.0] * 32 + [8.0] * 32
+    assert w8[1].tolist() == [4.0] * 32 + [0.5] * 32
+    # FP4: byte 0x72 holds codes 2 (1.0, low nibble) and 7 (6.0, high nibble)
+    w4 = m.dequantize_mx(np.full((2, 32), 0x72, dtype=np.uint8), scales, "mxfp4")
+    assert w4[0].tolist() == [1.0, 6.0] * 16 + [8.0, 48.0] * 16
+    assert w4[1].tolist() == [4.0, 24.0] * 16 + [0.5, 3.0] * 16
+
+
+MX_PINS = [pin_e8m0_closed_forms, pin_e4m3_closed_forms, pin_e4m3_against_torch, pin_e2m1_table,
+           pin_fp4_nibble_order, pin_dequantize_blocks]

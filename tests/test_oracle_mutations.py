@@ -137,3 +137,63 @@ def test_some_pin_catches(name, monkeypatch):
             caught.append(pin.__name__)
     assert caught, f"mutant {name} passed every pin"
 
+
+
+# ---------------------------------------------------------------- MX decoding mutants
+import oracle.mx_oracle as mxo  # noqa: E402
+
+
+def _unpack_high_first(packed):
+    b = np.asarray(packed, dtype=np.int64)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.int64)
+    out[..., 0::2] = b >> 4
+    out[..., 1::2] = b & 15
+    return out
+
+
+def _e4m3_bias8(codes):
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where((c >> 7) & 1, -1.0, 1.0)
+    e, mm = (c >> 3) & 15, c & 7
+    v = sign * np.where(e == 0, np.ldexp(mm / 8.0, -7), np.ldexp(1.0 + mm / 8.0, e - 8))
+    return np.where((c & 0x7F) == 0x7F, np.nan, v)
+
+
+def _e2m1_no_subnormal(codes):
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where((c >> 3) & 1, -1.0, 1.0)
+    e, mm = (c >> 1) & 3, c & 1
+    return sign * np.ldexp(1.0 + mm / 2.0, e - 1)
+
+
+def _e8m0_bias128(codes):
+    c = np.asarray(codes, dtype=np.int64)
+    return np.where(c == 255, np.nan, np.ldexp(1.0, c - 128))
+
+
+def _dequant_scales_not_transposed(elements, scales, fmt):
+    vals = mxo.decode_e4m3(elements) if fmt == "mxfp8" else mxo.decode_e2m1(mxo.unpack_fp4(elements))
+    x = mxo.decode_e8m0(scales)  # read as [rows, K/32]
+    return vals * np.repeat(x, mxo.MX_BLOCK, axis=1)
+
+
+MX_MUTANTS = {
+    "fp4_high_nibble_first": ("unpack_fp4", _unpack_high_first),
+    "e4m3_bias_8": ("decode_e4m3", _e4m3_bias8),
+    "e2m1_no_subnormal": ("decode_e2m1", _e2m1_no_subnormal),
+    "e8m0_bias_128": ("decode_e8m0", _e8m0_bias128),
+    "scales_not_transposed": ("dequantize_mx", _dequant_scales_not_transposed),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MX_MUTANTS))
+def test_some_mx_pin_catches(name, monkeypatch):
+    attr, fn = MX_MUTANTS[name]
+    monkeypatch.setattr(mxo, attr, fn)
+    caught = []
+    for pin in oracle_pins.MX_PINS:
+        try:
+            pin(mxo)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, f"mutant {name} passed every pin"

@@ -64,3 +64,8 @@ def test_token_subset_matches_full():
     part = oracle.moe_layer_forward(x, wr, wgu, wd, top_k=2, act="swiglu", capacity=9,
                                     residual=x, tokens=sub)
     np.testing.assert_allclose(part["out"], full["out"][sub], rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("pin", oracle_pins.MX_PINS, ids=lambda f: f.__name__)
+def test_mx_pin(pin):
+    pin(oracle.mx_oracle)
