@@ -72,7 +72,15 @@ def active_params(d_model: int, d_ff: int, n_experts: int, k: int, act: str, bia
     return d_model * n_experts + k * expert_params(d_model, d_ff, act, bias)
 
 
-def algorithmic_bytes(shape, T: int, active_experts: int, R: int) -> dict:
+def weight_bytes(params: int, wfmt: str = "bf16") -> int:
+    """Bytes of `params` expert weights in storage: bf16 2 B each; MX formats one E8M0 scale
+    byte per 32 elements plus 1 B (MXFP8) or 1/2 B (MXFP4) per element."""
+    if wfmt == "bf16":
+        return params * 2
+    return (params if wfmt == "mxfp8" else params // 2) + params // 32
+
+
+def algorithmic_bytes(shape, T: int, active_experts: int, R: int, wfmt: str = "bf16") -> dict:
     """Bytes the layer must move (counting rules in the design notes).
 
     layer: weights of every expert with at least one kept row, read once; router weight
@@ -80,7 +88,7 @@ def algorithmic_bytes(shape, T: int, active_experts: int, R: int) -> dict:
     ffn:   the same expert weights, plus x_perm read (bf16) and y_perm written (fp32).
     """
     d, F, N = shape.d_model, shape.d_ff, shape.n_experts
-    w = active_experts * expert_params(d, F, shape.act) * 2
+    w = active_experts * weight_bytes(expert_params(d, F, shape.act), wfmt)
     layer = w + N * d * 4 + T * d * 2 + T * d * 2
     ffn = w + R * d * 2 + R * d * 4
     return {"layer": layer, "ffn": ffn, "weights": w}
@@ -220,14 +228,20 @@ class ClockSampler:
 class Layer:
     """Device buffers of one layer invocation; stages called through the C ABI."""
 
-    def __init__(self, shape, T, device, seed=0):
+    def __init__(self, shape, T, device, seed=0, wfmt="bf16"):
         import sparse_mixture_experts_11_b200 as moe
         self.moe = moe
-        self.shape, self.T = shape, T
-        self.inp = synthetic.make_layer_inputs(shape, T, seed=seed, device=device)
+        self.shape, self.T, self.wfmt = shape, T, wfmt
+        if wfmt == "bf16":
+            self.inp = synthetic.make_layer_inputs(shape, T, seed=seed, device=device)
+        else:
+            self.inp = synthetic.make_mx_layer_inputs(shape, T, wfmt, seed=seed, device=device)
         cap = capacity_of(shape, T)
         self.dims = moe.make_dims(T, shape.d_model, shape.n_experts, shape.top_k, shape.d_ff,
                                   shape.act, cap)
+        i = self.inp
+        self.mx = None if wfmt == "bf16" else moe.mx_weights(
+            self.dims, wfmt, i["w_gate_up_q"], i["w_gate_up_s"], i["w_down_q"], i["w_down_s"])
         self.R_max = moe.max_rows(self.dims)
         self.fws = moe.new_workspace(self.dims, device, forward=True)
         self.b = moe.forward_layout(self.dims, self.fws)
@@ -306,6 +320,12 @@ class Layer:
                                        moe._stream(None)), "permute")
 
         def ffn():
+            if self.mx is not None:
+                moe._check(lib.moe_grouped_ffn_mx(d, P(b.x_perm), P(b.expert_offset),
+                                                  moe.ctypes.byref(self.mx), P(b.h), P(b.y_perm),
+                                                  P(b.stage_ws), b.stage_ws_bytes,
+                                                  moe._stream(None)), "grouped_ffn_mx")
+                return
             moe._check(lib.moe_grouped_ffn(d, P(b.x_perm), P(b.expert_offset), ptr(i["w_gate_up"]),
                                            ptr(i["w_down"]), P(b.h), P(b.y_perm), P(b.stage_ws),
                                            b.stage_ws_bytes, moe._stream(None)), "grouped_ffn")
@@ -319,9 +339,17 @@ class Layer:
     def forward_call(self):
         """moe_forward on the layer's inputs (the public call; decode-sized batches route and
         sort in one launch there, which the stage calls do not)."""
+        self.forward_on(self.inp["x"], self.out)
+
+    def forward_on(self, x, out, stream=None):
+        """moe_forward (bf16 or MX weights) of tokens x into out, residual x."""
         i = self.inp
-        self.moe.forward_into(self.dims, i["x"], i["w_router"], i["logit_bias"], i["w_gate_up"],
-                              i["w_down"], i["x"], self.out, self.fws)
+        if self.mx is not None:
+            self.moe.forward_mx_into(self.dims, x, i["w_router"], i["logit_bias"], self.mx, x, out,
+                                     self.fws, stream=stream)
+        else:
+            self.moe.forward_into(self.dims, x, i["w_router"], i["logit_bias"], i["w_gate_up"],
+                                  i["w_down"], x, out, self.fws, stream=stream)
 
     def capture_stage_graphs(self):
         """The forward captured as CUDA graphs: once whole (moe_forward; its kernels overlap
@@ -389,8 +417,7 @@ class Layer:
                 h2d_done[b].record(s_in)
             s_comp.wait_event(h2d_done[b])
             s_comp.wait_event(d2h_done[b])           # step n-2's output has left out_dev[b]
-            moe.forward_into(self.dims, x_dev[b], i["w_router"], i["logit_bias"], i["w_gate_up"],
-                             i["w_down"], x_dev[b], out_dev[b], self.fws, stream=s_comp)
+            self.forward_on(x_dev[b], out_dev[b], stream=s_comp)
             comp_done[b].record(s_comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(comp_done[b])
@@ -432,7 +459,7 @@ def run_gpu(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     shape, T = parse_workload(args.workload)
-    layer = Layer(shape, T, device)
+    layer = Layer(shape, T, device, wfmt=args.wfmt)
     for call in layer.stage_calls():  # first calls set kernel attributes outside any capture
         call()
     torch.cuda.synchronize()
@@ -493,7 +520,7 @@ def run_gpu(args, rank, world, local_rank):
     counts = v["expert_count"].cpu()
     R = int(counts.sum())
     active = int((counts > 0).sum())
-    ab = algorithmic_bytes(shape, T, active, R)
+    ab = algorithmic_bytes(shape, T, active, R, args.wfmt)
     peaks = load_peaks()
     flops = ffn_flops(shape, R)
     tensor_bound = flops / max(ab["ffn"], 1) > (peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9)
@@ -518,8 +545,12 @@ def run_gpu(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded; x~N(0,1) bf16, router W~N(0,1/d) fp32, expert W~N(0,0.02) bf16)",
-        "config": {"workload": shape.describe(T), "T": T, "d_model": shape.d_model,
+        "data": ("synthetic (seeded; x~N(0,1) bf16, router W~N(0,1/d) fp32, expert W~N(0,0.02) bf16)"
+                 if args.wfmt == "bf16" else
+                 f"synthetic (seeded; x~N(0,1) bf16, router W~N(0,1/d) fp32, expert weights "
+                 f"{args.wfmt}: random element codes, E8M0 scales per 32 elements)"),
+        "config": {"workload": shape.describe(T) + ("" if args.wfmt == "bf16" else f" weights={args.wfmt}"),
+                   "T": T, "d_model": shape.d_model, "expert_weights": args.wfmt,
                    "n_experts": shape.n_experts, "top_k": shape.top_k, "d_ff": shape.d_ff,
                    "act": shape.act, "capacity": layer.dims.capacity, "kept_rows": R,
                    "active_experts": active,
@@ -650,6 +681,8 @@ def main(argv=None):
                     help="shape[:T], shapes: " + ", ".join(synthetic.SHAPES))
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--wfmt", choices=["bf16", "mxfp8", "mxfp4"], default="bf16",
+                    help="expert weight storage (MX formats: OCP microscaling, E8M0 block scales)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -671,7 +704,7 @@ def main(argv=None):
                                              device_id=torch.device("cuda", local_rank))
     try:
         line, layer = run_gpu(args, rank, world, local_rank)
-        if rank == 0 and not args.no_cpu_baseline:
+        if rank == 0 and not args.no_cpu_baseline and args.wfmt == "bf16":
             line["cpu_baseline"] = cpu_baseline(layer.shape, layer.T, layer.inp)
         if rank == 0:
             print(json.dumps(line), flush=True)

@@ -104,6 +104,7 @@ struct FfnParams {
 // scale) with E4M3 or E2M1 elements, decoded exactly to bf16 in shared memory.
 enum { WFMT_BF16 = 0, WFMT_MXFP8 = 1, WFMT_MXFP4 = 2 };
 constexpr int kConvThreads = 256;  // MX decoders (warps 7-14)
+constexpr int kConvWarps = kConvThreads / 32;
 
 template <int BM, int WFMT>
 struct Cfg {
@@ -112,19 +113,31 @@ struct Cfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = kUmmaN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  // MX: two bf16 stages (decoded from shared memory, not waiting on HBM) and a deeper ring of
-  // packed stages: 256 rows of 64 elements (64 or 32 bytes a row) plus 2 x 256 scale bytes
-  static constexpr int ROW_BYTES = WFMT == WFMT_MXFP8 ? BK : BK / 2;
-  static constexpr int STG_BYTES = MX ? kUmmaN * ROW_BYTES + 2 * kUmmaN : 0;
+  // MX: bf16 stages (decoded from shared memory, not waiting on HBM) and a ring of packed
+  // stages, each 256 rows of one 128-byte segment (KG k blocks: 2 of E4M3, 4 of E2M1; one
+  // TMA row request then carries 2x or 4x the elements of a bf16 one) plus 2 KG x 256 scales
+  static constexpr int ROW_BYTES = WFMT == WFMT_MXFP8 ? BK : BK / 2;  // per row and k block
+  static constexpr int KG = MX ? 128 / ROW_BYTES : 1;
+  static constexpr int STG_BYTES = MX ? kUmmaN * 128 + 2 * KG * kUmmaN : 0;
   static constexpr int STAGES_FIT = (kSmemBudget / STAGE_BYTES) > 8 ? 8 : (kSmemBudget / STAGE_BYTES);
+  // MX: three bf16 stages, so the decoders run a stage ahead of the MMA's round trip
+  // (decode, MMA, commit, stage free), and the rest of 224 KB for packed stages
+  // MX: two bf16 B stages (decoded from shared memory), a separate ring of SA A stages
+  // (token rows, loaded ahead of the decoders: an A copy waits on L2 for about 1.7 us when
+  // the weight streams load it), and the rest of 224 KB for packed stages
+  static constexpr int kMxBudget = 224 * 1024;
   static constexpr int STAGES = MX ? 2 : STAGES_FIT;
-  static constexpr int SST_FIT = MX ? (kSmemBudget - STAGES * STAGE_BYTES) / STG_BYTES : 0;
+  static constexpr int SA = MX ? (BM == 64 ? 6 : 3) : 0;
+  static constexpr int B_RING = MX ? STAGES * B_BYTES : STAGES * STAGE_BYTES;  // bytes
+  static constexpr int A_RING = SA * A_BYTES;
+  static constexpr int SST_FIT = MX ? (kMxBudget - B_RING - A_RING) / STG_BYTES : 0;
   static constexpr int SST = SST_FIT > 16 ? 16 : SST_FIT;
   static constexpr int TMEM_COLS = 2 * kUmmaN;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SST * STG_BYTES + 1024;  // + alignment slack
+  static constexpr int SMEM_BYTES = B_RING + A_RING + SST * STG_BYTES + 1024;  // + alignment slack
   static_assert(TMEM_COLS <= 512, "two accumulators must fit in TMEM");
   static_assert(STAGES >= 2, "pipeline depth");
-  static_assert(!MX || SST >= 4, "MX staging depth");
+  static_assert(!MX || SST >= 2, "MX staging depth");
+  static_assert(!MX || STG_BYTES % 1024 == 0, "packed stages stay 1024-byte aligned (swizzle)");
   static_assert(BM == 64 || BM == 128, "UMMA M");
 };
 
@@ -210,42 +223,47 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, int N, int bn, int nt
   return c;
 }
 
-// Schedule of one phase. Stream-K gives CTA b < g the k-block iterations
-// [b * total / g, (b + 1) * total / g) of the tiles laid end to end (num_kb per tile).
+// Schedule of one phase in units of kg k blocks (kg = 1 for bf16 weights; MX weights stream
+// 128-byte row segments, 2 or 4 k blocks, per copy, so their units are those groups). Stream-K
+// gives CTA b < g the units [b * total / g, (b + 1) * total / g) of the tiles laid end to end
+// (upt = ceil(num_kb / kg) per tile); a tile's last unit may hold fewer than kg k blocks.
 struct Sched {
   int sk;         // 1: stream-K, 0: whole tiles
   int g;          // CTAs with a stream-K range
   int tiles;
-  int num_kb;
-  int64_t total;  // tiles * num_kb
+  int num_kb;     // k blocks per tile
+  int kg;         // k blocks per unit
+  int upt;        // units per tile
+  int64_t total;  // tiles * upt
 };
 
 __device__ __forceinline__ int64_t sk_begin(const Sched& s, int b) {
   return static_cast<int64_t>(b) * s.total / s.g;
 }
-// The CTA whose range holds iteration i: the largest b with sk_begin(b) <= i.
+// The CTA whose range holds unit i: the largest b with sk_begin(b) <= i.
 __device__ __forceinline__ int sk_cta_of(const Sched& s, int64_t i) {
   return static_cast<int>(((i + 1) * s.g + s.total - 1) / s.total) - 1;
 }
 
 // Cost, in k-block times, of the busiest CTA: whole tiles take ceil(tiles / grid) waves of
-// num_kb; stream-K takes ceil(total / g) plus the partial round trip of the tile finished
-// last (latency, and a k block's worth of traffic per 32 partial rows). Stream-K is chosen
-// when at least 5 % faster. Ranges keep at least kSkMinKb k blocks.
+// num_kb; stream-K takes ceil(total / g) units plus the partial round trip of the tile
+// finished last (latency, and a k block's worth of traffic per 32 partial rows). Stream-K is
+// chosen when at least 5 % faster. Ranges keep at least kSkMinKb k blocks.
 constexpr int kSkMinKb = 4;
 constexpr float kTailKb = 2.0f;  // epilogue of the last tile and pipeline refill
 
-__device__ __forceinline__ Sched choose_schedule(int tiles, int grid, int num_kb, int sk_ctas,
-                                                 int slot_rows) {
-  Sched s{0, 0, tiles, num_kb, static_cast<int64_t>(tiles) * num_kb};
+__device__ __forceinline__ Sched choose_schedule(int tiles, int grid, int num_kb, int kg,
+                                                 int sk_ctas, int slot_rows) {
+  const int upt = (num_kb + kg - 1) / kg;
+  Sched s{0, 0, tiles, num_kb, kg, upt, static_cast<int64_t>(tiles) * upt};
   if (sk_ctas <= 0 || tiles <= 0) return s;
-  const int min_kb = min(kSkMinKb, num_kb);
-  const int64_t by_size = s.total / min_kb;
+  const int min_u = max(1, min(kSkMinKb, num_kb) / kg);
+  const int64_t by_size = s.total / min_u;
   const int64_t g = by_size < min(grid, sk_ctas) ? by_size : min(grid, sk_ctas);
   if (g < 2) return s;
   const float dp = static_cast<float>((tiles + grid - 1) / grid) * num_kb + kTailKb;
   const float fixup = 2.0f + slot_rows / 32.0f;
-  const float sk = static_cast<float>((s.total + g - 1) / g) + kTailKb + fixup;
+  const float sk = static_cast<float>((s.total + g - 1) / g) * kg + kTailKb + fixup;
   if (sk < 0.95f * dp) {
     s.sk = 1;
     s.g = static_cast<int>(g);
@@ -254,11 +272,12 @@ __device__ __forceinline__ Sched choose_schedule(int tiles, int grid, int num_kb
 }
 
 struct Seg {
-  int tile, kb0, kb1;
+  int tile, kb0, kb1;  // k blocks [kb0, kb1) of tile; kb0 is a multiple of the unit size
 };
 
 // Walks this CTA's segments (a tile and a k-block range of it) of one phase in order; the
-// producer, the MMA issuer and the epilogue each run their own copy and see the same sequence.
+// producers, the MMA issuer, the decoders and the epilogue each run their own copy and see
+// the same sequence.
 struct SegCursor {
   int64_t it, end;
   __device__ __forceinline__ SegCursor(const Sched& s) {
@@ -274,11 +293,13 @@ struct SegCursor {
   __device__ __forceinline__ bool next(const Sched& s, Seg& g) {
     if (it >= end) return false;
     if (s.sk) {
-      g.tile = static_cast<int>(it / s.num_kb);
-      g.kb0 = static_cast<int>(it - static_cast<int64_t>(g.tile) * s.num_kb);
+      g.tile = static_cast<int>(it / s.upt);
+      const int u0 = static_cast<int>(it - static_cast<int64_t>(g.tile) * s.upt);
       const int64_t left = end - it;
-      g.kb1 = left < s.num_kb - g.kb0 ? g.kb0 + static_cast<int>(left) : s.num_kb;
-      it += g.kb1 - g.kb0;
+      const int u1 = left < s.upt - u0 ? u0 + static_cast<int>(left) : s.upt;
+      g.kb0 = u0 * s.kg;
+      g.kb1 = min(u1 * s.kg, s.num_kb);
+      it += u1 - u0;
     } else {
       g.tile = static_cast<int>(it);
       g.kb0 = 0;
@@ -373,7 +394,7 @@ __device__ __forceinline__ bool epilogue_segment(const FfnParams& fp, const Phas
   tc_fence_after_sync();
   const bool whole = sg.kb0 == 0 && sg.kb1 == sched.num_kb;
   // partial slot of this segment: 0 when the CTA's range starts inside this tile
-  const int64_t t_it0 = static_cast<int64_t>(sg.tile) * sched.num_kb;
+  const int64_t t_it0 = static_cast<int64_t>(sg.tile) * sched.upt;  // the tile's first unit
   const int slot = whole ? 0 : (sk_begin(sched, blockIdx.x) >= t_it0 ? 0 : 1);
   float* const my_part =
       p.part + (static_cast<int64_t>(blockIdx.x * 2 + slot) * fp.slot_rows) * kUmmaN;
@@ -418,7 +439,7 @@ __device__ __forceinline__ bool epilogue_segment(const FfnParams& fp, const Phas
   // of the 128 epilogue threads, one fenced thread releases them all); the owner waits for
   // that count, then adds every partial in order of CTA index.
   const int first_cta = sk_cta_of(sched, t_it0);
-  const int n_seg = sk_cta_of(sched, t_it0 + sched.num_kb - 1) - first_cta + 1;
+  const int n_seg = sk_cta_of(sched, t_it0 + sched.upt - 1) - first_cta + 1;
   const bool owner = static_cast<int>(blockIdx.x) == first_cta;
   if (!__all_sync(0xffffffffu, epilogue_sync(ebar, epi_phase, fp.timeout_ns, s_abort))) return false;
   if (!owner) {
@@ -495,13 +516,25 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
   __shared__ int s_last_cta;
   __shared__ __align__(8) uint64_t sfull_bar[C::MX ? C::SST : 1];
   __shared__ __align__(8) uint64_t sempty_bar[C::MX ? C::SST : 1];
+  __shared__ __align__(8) uint64_t afull_bar[C::MX ? C::SA : 1];
+  __shared__ __align__(8) uint64_t aempty_bar[C::MX ? C::SA : 1];
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int N = p.n_experts;
   const uint32_t tiles = (smem_u32(dyn_smem) + 1023u) & ~1023u;
-  const uint32_t stg0 = tiles + C::STAGES * C::STAGE_BYTES;  // MX: packed ring
+  // bf16: stage s = [A | B]; MX: B stages, then the A ring, then the packed ring
+  const uint32_t stg0 = tiles + C::B_RING + C::A_RING;
+  auto a_addr = [&](int i) -> uint32_t {
+    return C::MX ? tiles + C::B_RING + i * C::A_BYTES : tiles + i * C::STAGE_BYTES;
+  };
+  auto b_addr = [&](int i) -> uint32_t {
+    return C::MX ? tiles + i * C::B_BYTES : tiles + i * C::STAGE_BYTES + C::A_BYTES;
+  };
+  constexpr int AST = C::MX ? C::SA : C::STAGES;  // stages of the A operand's ring
+  uint64_t* const a_full = C::MX ? afull_bar : full_bar;
+  uint64_t* const a_empty = C::MX ? aempty_bar : empty_bar;
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmA1);
@@ -513,13 +546,17 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
       prefetch_tensormap(&tmS2);
       for (int s = 0; s < C::SST; ++s) {
         mbar_init(smem_u32(&sfull_bar[s]), 1);
-        mbar_init(smem_u32(&sempty_bar[s]), kConvThreads);
+        mbar_init(smem_u32(&sempty_bar[s]), kConvWarps);
       }
     }
     for (int s = 0; s < C::STAGES; ++s) {
-      // MX: the A copy's transaction bytes plus one arrival per decoder thread
-      mbar_init(smem_u32(&full_bar[s]), C::MX ? 1 + kConvThreads : 1);
+      // MX: B stages filled by the decoders, one arrival per decoder warp
+      mbar_init(smem_u32(&full_bar[s]), C::MX ? kConvWarps : 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int s = 0; s < C::SA; ++s) {
+      mbar_init(smem_u32(&afull_bar[s]), 1);
+      mbar_init(smem_u32(&aempty_bar[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tfull_bar[b]), 1);
@@ -584,7 +621,7 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
       s_mt[N] = incl;
       for (int ph = 0; ph < 2; ++ph)
         s_sched[ph] = choose_schedule(incl * p.ph[ph].n_tiles_n, gridDim.x, p.ph[ph].num_kb,
-                                      p.ph[ph].sk_ctas, p.slot_rows);
+                                      C::KG, p.ph[ph].sk_ctas, p.slot_rows);
     }
     if (bad) report_error(p.status, MOE_ERR_BOUNDS);  // such an expert gets no tiles
   }
@@ -616,15 +653,15 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
           int pend_from = -1;  // first iteration whose stage holds its B block but not its A
           const int seg_it0 = it;
           for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
-            const int s = it % C::STAGES;
-            const uint32_t par = (it / C::STAGES) & 1;
-            if (!mbar_wait(smem_u32(&empty_bar[s]), par ^ 1u, p.timeout_ns, &s_abort)) {
+            const int s = it % AST;
+            const uint32_t par = (it / AST) & 1;
+            if (!mbar_wait(smem_u32(&a_empty[s]), par ^ 1u, p.timeout_ns, &s_abort)) {
               ok = false;
               break;
             }
-            const uint32_t fb = smem_u32(&full_bar[s]);
-            const uint32_t a_dst = tiles + s * C::STAGE_BYTES;
-            const uint32_t b_dst = a_dst + C::A_BYTES;
+            const uint32_t fb = smem_u32(&a_full[s]);
+            const uint32_t a_dst = a_addr(s);
+            const uint32_t b_dst = b_addr(s);
             mbar_arrive_expect_tx(fb, C::MX ? C::A_BYTES : C::STAGE_BYTES);
             if (!C::MX) {  // MX: the decoders fill the B half
               if (ph == 0) {
@@ -644,14 +681,14 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
               continue;
             }
             if (pend_from < 0) pend_from = it;
-            if (it - pend_from + 1 == C::STAGES || kb + 1 == sg.kb1) {
+            if (it - pend_from + 1 == AST || kb + 1 == sg.kb1) {
               // every stage holds a W_d block (or the segment ends): wait for the rows' h
               if (!wait_counter_at_least(p.h_ready + c.gm, h_target, p.timeout_ns, &s_abort))
                 ok = false;  // the h loads below still complete the armed stages
               fence_proxy_async_global();
               for (int j = pend_from; j <= it; ++j) {
-                const int sj = j % C::STAGES;
-                tma_load_2d(tiles + sj * C::STAGE_BYTES, tA, smem_u32(&full_bar[sj]),
+                const int sj = j % AST;
+                tma_load_2d(a_addr(sj), tA, smem_u32(&a_full[sj]),
                             (sg.kb0 + (j - seg_it0)) * BK, c.m0, pol_a);
               }
               pend_from = -1;
@@ -667,8 +704,8 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
         report_error(p.status, MOE_ERR_TIMEOUT);
       }
       // No TMA write may still be landing in shared memory when the CTA exits.
-      for (int i = max(0, it - C::STAGES); i < it; ++i)
-        mbar_wait(smem_u32(&full_bar[i % C::STAGES]), (i / C::STAGES) & 1, kDrainTimeoutNs, nullptr);
+      for (int i = max(0, it - AST); i < it; ++i)
+        mbar_wait(smem_u32(&a_full[i % AST]), (i / AST) & 1, kDrainTimeoutNs, nullptr);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -691,15 +728,16 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
           tc_fence_after_sync();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kUmmaN);
           for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
-            const int s = it % C::STAGES;
+            const int s = it % C::STAGES, sa = it % AST;
             const uint32_t par = (it / C::STAGES) & 1;
-            if (!mbar_wait(smem_u32(&full_bar[s]), par, p.timeout_ns, &s_abort)) {
+            if (!mbar_wait(smem_u32(&full_bar[s]), par, p.timeout_ns, &s_abort) ||
+                (C::MX && !mbar_wait(smem_u32(&afull_bar[sa]), (it / AST) & 1, p.timeout_ns, &s_abort))) {
               ok = false;
               break;
             }
             tc_fence_after_sync();
-            const uint32_t a_base = tiles + s * C::STAGE_BYTES;
-            const uint32_t b_base = a_base + C::A_BYTES;
+            const uint32_t a_base = a_addr(C::MX ? sa : s);
+            const uint32_t b_base = b_addr(s);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
               tc_mma_f16(d_tmem, smem_desc_k_sw128(a_base + kk * 32),
@@ -708,6 +746,7 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
             }
             issued = true;
             tc_commit(smem_u32(&empty_bar[s]));
+            if (C::MX) tc_commit(smem_u32(&aempty_bar[sa]));
           }
           if (!ok) break;
           tc_commit(smem_u32(&tfull_bar[buf]));
@@ -766,9 +805,11 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
     }
   } else if (C::MX && warp == 6) {
     // ---------------------------------------------------------------- MX packed-ring producer
+    // One packed stage per unit of KG k blocks: 256 rows x 128 bytes (128B-swizzled) and the
+    // rows' 2 KG block scales.
     if (lane == 0) {
       const uint64_t pol_b = make_policy(p.weight_policy);
-      int it = 0;
+      int su = 0;
       bool ok = true;
       for (int ph = 0; ph < 2 && ok; ++ph) {
         const Sched sc = s_sched[ph];
@@ -777,25 +818,25 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
         Seg sg;
         while (ok && cur.next(sc, sg)) {
           const TileCoord c = decode_tile<BM>(sg.tile, N, bn, p.ph[ph].n_tiles_n, s_mt, s_off);
-          for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
-            const int s = it % C::SST;
-            if (!mbar_wait(smem_u32(&sempty_bar[s]), ((it / C::SST) & 1) ^ 1u, p.timeout_ns, &s_abort)) {
+          for (int kb = sg.kb0; kb < sg.kb1; kb += C::KG, ++su) {
+            const int s = su % C::SST;
+            if (!mbar_wait(smem_u32(&sempty_bar[s]), ((su / C::SST) & 1) ^ 1u, p.timeout_ns, &s_abort)) {
               ok = false;
               break;
             }
             const uint32_t fb = smem_u32(&sfull_bar[s]);
             const uint32_t dst = stg0 + s * C::STG_BYTES;
-            const uint32_t sc_dst = dst + kUmmaN * C::ROW_BYTES;  // [2 blocks][256 rows] scales
+            const uint32_t sc_dst = dst + kUmmaN * 128;  // scales after the 32 KB of elements
             mbar_arrive_expect_tx(fb, C::STG_BYTES);
-            const int kx = kb * C::ROW_BYTES;  // byte column of this k block's elements
+            const int kx = kb * C::ROW_BYTES;  // byte column of the unit's first k block
             if (ph == 0 && EPI1 == EPI_SWIGLU) {
-              tma_load_4d(dst, &tmB1, fb, kx, c.n0, 0, c.e, pol_b);  // gate rows
-              tma_load_4d(dst + BN1 * C::ROW_BYTES, &tmB1, fb, kx, c.n0, 1, c.e, pol_b);  // up rows
-              tma_load_4d(sc_dst, &tmS1, fb, c.n0, 0, 2 * kb, c.e, pol_b);  // [2][128] gate
-              tma_load_4d(sc_dst + 2 * BN1, &tmS1, fb, c.n0, 1, 2 * kb, c.e, pol_b);  // [2][128] up
+              tma_load_4d(dst, &tmB1, fb, kx, c.n0, 0, c.e, pol_b);              // gate rows
+              tma_load_4d(dst + BN1 * 128, &tmB1, fb, kx, c.n0, 1, c.e, pol_b);  // up rows
+              tma_load_4d(sc_dst, &tmS1, fb, c.n0, 0, 2 * kb, c.e, pol_b);       // [2KG][128] gate
+              tma_load_4d(sc_dst + 2 * C::KG * BN1, &tmS1, fb, c.n0, 1, 2 * kb, c.e, pol_b);
             } else if (ph == 0) {
               tma_load_3d(dst, &tmB1, fb, kx, c.n0, c.e, pol_b);
-              tma_load_3d(sc_dst, &tmS1, fb, c.n0, 2 * kb, c.e, pol_b);
+              tma_load_3d(sc_dst, &tmS1, fb, c.n0, 2 * kb, c.e, pol_b);  // [2KG][256]
             } else {
               tma_load_3d(dst, &tmB2, fb, kx, c.n0, c.e, pol_b);
               tma_load_3d(sc_dst, &tmS2, fb, c.n0, 2 * kb, c.e, pol_b);
@@ -807,54 +848,67 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
         s_abort = 1;
         report_error(p.status, MOE_ERR_TIMEOUT);
       }
-      for (int i = max(0, it - C::SST); i < it; ++i)
+      for (int i = max(0, su - C::SST); i < su; ++i)
         mbar_wait(smem_u32(&sfull_bar[i % C::SST]), (i / C::SST) & 1, kDrainTimeoutNs, nullptr);
     }
   } else if (C::MX) {
     // ---------------------------------------------------------------- MX decoders (warps 7..14)
-    // Thread r decodes row r of every stage: 64 elements (8 chunks of 8) with the row's two
-    // block scales, into the 128B-swizzled K-major layout the MMA reads (chunk c of row r at
-    // 16 * (c ^ (r & 7))).
+    // Thread r decodes row r of every k block: 64 elements (8 chunks of 8) from its 128-byte
+    // packed row segment (128B-swizzled: 16-byte chunk q at 16 * (q ^ (r & 7))) with the
+    // row's two block scales, into the 128B-swizzled K-major bf16 layout the MMA reads (chunk
+    // c of row r at 16 * (c ^ (r & 7))). A packed stage is released after its last k block.
     const int r = threadIdx.x - (kThreads + 32);  // 0..255
-    int it = 0;
+    int it = 0, su = 0;
     bool ok = true;
     for (int ph = 0; ph < 2 && ok; ++ph) {
       const Sched sc = s_sched[ph];
-      // scale layout of this phase's stages: SwiGLU gate/up halves, or one [2][256] block
+      // scale layout of this phase's stages: SwiGLU gate/up halves, or one [2KG][256] block
       const bool halves = ph == 0 && EPI1 == EPI_SWIGLU;
-      const int sc_idx0 = halves ? (r >> 7) * 256 + (r & 127) : r;
+      const int sc_base = halves ? (r >> 7) * (2 * C::KG * 128) + (r & 127) : r;
       const int sc_step = halves ? 128 : 256;
       SegCursor cur(sc);
       Seg sg;
       while (ok && cur.next(sc, sg)) {
         for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
-          const int s2 = it % C::SST, s = it % C::STAGES;
-          const bool got = mbar_wait(smem_u32(&sfull_bar[s2]), (it / C::SST) & 1, p.timeout_ns, &s_abort) &&
-                           mbar_wait(smem_u32(&empty_bar[s]), ((it / C::STAGES) & 1) ^ 1u, p.timeout_ns, &s_abort);
+          const int j = (kb - sg.kb0) % C::KG;  // k block within the packed stage
+          const int s2 = su % C::SST, s = it % C::STAGES;
+          bool got = true;
+          if (j == 0) got = mbar_wait(smem_u32(&sfull_bar[s2]), (su / C::SST) & 1, p.timeout_ns, &s_abort);
+          got = got && mbar_wait(smem_u32(&empty_bar[s]), ((it / C::STAGES) & 1) ^ 1u, p.timeout_ns, &s_abort);
           if (!got) {
             ok = false;
             break;
           }
           const uint8_t* stg = dyn_smem + (stg0 - smem_u32(dyn_smem)) + s2 * C::STG_BYTES;
-          const uint8_t* row = stg + r * C::ROW_BYTES;
-          const uint8_t* scl = stg + kUmmaN * C::ROW_BYTES;
-          const float x0 = e8m0_to_f32(scl[sc_idx0]);
-          const float x1 = e8m0_to_f32(scl[sc_idx0 + sc_step]);
-          uint8_t* bdst = dyn_smem + (tiles - smem_u32(dyn_smem)) + s * C::STAGE_BYTES + C::A_BYTES +
-                          r * 128;
+          const uint8_t* scl = stg + kUmmaN * 128;
+          const float x0 = e8m0_to_f32(scl[sc_base + (2 * j) * sc_step]);
+          const float x1 = e8m0_to_f32(scl[sc_base + (2 * j + 1) * sc_step]);
+          // this k block's part of the packed row (64 or 32 bytes), then the eight chunks
+          constexpr int kQ = C::ROW_BYTES / 16;
+          uint4 raw[kQ];
+#pragma unroll
+          for (int q = 0; q < kQ; ++q)
+            raw[q] = *reinterpret_cast<const uint4*>(stg + r * 128 + (((j * kQ + q) ^ (r & 7)) << 4));
+          const uint32_t* wd = reinterpret_cast<const uint32_t*>(raw);
+          uint8_t* bdst = dyn_smem + (b_addr(s) - smem_u32(dyn_smem)) + r * 128;
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             const float x = ch < 4 ? x0 : x1;  // elements 0..31: block 0; 32..63: block 1
             uint4 v;
             if (WFMT == WFMT_MXFP8)
-              v = decode8_e4m3(*reinterpret_cast<const uint2*>(row + ch * 8), x);
+              v = decode8_e4m3(make_uint2(wd[2 * ch], wd[2 * ch + 1]), x);
             else
-              v = decode8_e2m1(*reinterpret_cast<const uint32_t*>(row + ch * 4), x);
+              v = decode8_e2m1(wd[ch], x);
             *reinterpret_cast<uint4*>(bdst + ((ch ^ (r & 7)) << 4)) = v;
           }
           fence_proxy_async_smem();  // generic stores -> visible to the tensor core
-          mbar_arrive(smem_u32(&full_bar[s]));
-          mbar_arrive(smem_u32(&sempty_bar[s2]));
+          __syncwarp();
+          const bool last = j == C::KG - 1 || kb + 1 == sg.kb1;
+          if (lane == 0) {  // one arrival per warp on each barrier
+            mbar_arrive(smem_u32(&full_bar[s]));
+            if (last) mbar_arrive(smem_u32(&sempty_bar[s2]));
+          }
+          if (last) ++su;
         }
       }
     }
@@ -924,9 +978,9 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
   return r == CUDA_SUCCESS;
 }
 
-// uint8 tensor map without swizzle (MX elements and scales; dims[0] contiguous).
+// uint8 tensor map (MX elements: 128B swizzle, 128-byte boxes; scales: no swizzle).
 bool make_map_u8(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                 const uint64_t* strides_bytes, const uint32_t* box) {
+                 const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t gd[5];
@@ -941,7 +995,8 @@ bool make_map_u8(CUtensorMap* m, const void* base, int rank, const uint64_t* dim
   }
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank),
                         const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -1042,37 +1097,39 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
     if (!make_map(&mA1, a.x_perm, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   if (a.wfmt != MOE_WFMT_BF16) {
-    // packed elements: [N][rows][K * rb / 64] bytes, no swizzle; scales: [N][K/32][rows] bytes
+    // packed elements: [N][rows][K * rb / 64] bytes, 128-byte boxes (2 or 4 k blocks) with
+    // 128B swizzle; scales: [N][K/32][rows] bytes, boxes of 2 KG blocks
     const uint64_t rb = a.wfmt == MOE_WFMT_MXFP8 ? BK : BK / 2;  // bytes per row and k block
+    const uint32_t kg2 = static_cast<uint32_t>(2 * (128 / rb));    // scale blocks per box
     const uint64_t db = d * rb / BK, fb = F * rb / BK;
     if (swiglu) {
       const uint64_t dims[4] = {db, F, 2, N};
       const uint64_t str[3] = {db, F * db, 2 * F * db};
-      const uint32_t box[4] = {static_cast<uint32_t>(rb), static_cast<uint32_t>(bn_gu), 1, 1};
-      if (!make_map_u8(&mB1, a.w_gate_up, 4, dims, str, box)) return cudaErrorInvalidValue;
+      const uint32_t box[4] = {128, static_cast<uint32_t>(bn_gu), 1, 1};
+      if (!make_map_u8(&mB1, a.w_gate_up, 4, dims, str, box, true)) return cudaErrorInvalidValue;
       const uint64_t sd[4] = {F, 2, d / 32, N};
       const uint64_t ss[3] = {F, 2 * F, (d / 32) * 2 * F};
-      const uint32_t sb[4] = {static_cast<uint32_t>(bn_gu), 1, 2, 1};
-      if (!make_map_u8(&mS1, a.w_gate_up_scales, 4, sd, ss, sb)) return cudaErrorInvalidValue;
+      const uint32_t sb[4] = {static_cast<uint32_t>(bn_gu), 1, kg2, 1};
+      if (!make_map_u8(&mS1, a.w_gate_up_scales, 4, sd, ss, sb, false)) return cudaErrorInvalidValue;
     } else {
       const uint64_t dims[3] = {db, F, N};
       const uint64_t str[2] = {db, F * db};
-      const uint32_t box[3] = {static_cast<uint32_t>(rb), static_cast<uint32_t>(bn_gu), 1};
-      if (!make_map_u8(&mB1, a.w_gate_up, 3, dims, str, box)) return cudaErrorInvalidValue;
+      const uint32_t box[3] = {128, static_cast<uint32_t>(bn_gu), 1};
+      if (!make_map_u8(&mB1, a.w_gate_up, 3, dims, str, box, true)) return cudaErrorInvalidValue;
       const uint64_t sd[3] = {F, d / 32, N};
       const uint64_t ss[2] = {F, (d / 32) * F};
-      const uint32_t sb[3] = {static_cast<uint32_t>(bn_gu), 2, 1};
-      if (!make_map_u8(&mS1, a.w_gate_up_scales, 3, sd, ss, sb)) return cudaErrorInvalidValue;
+      const uint32_t sb[3] = {static_cast<uint32_t>(bn_gu), kg2, 1};
+      if (!make_map_u8(&mS1, a.w_gate_up_scales, 3, sd, ss, sb, false)) return cudaErrorInvalidValue;
     }
     {
       const uint64_t dims[3] = {fb, d, N};
       const uint64_t str[2] = {fb, d * fb};
-      const uint32_t box[3] = {static_cast<uint32_t>(rb), static_cast<uint32_t>(kDnBn), 1};
-      if (!make_map_u8(&mB2, a.w_down, 3, dims, str, box)) return cudaErrorInvalidValue;
+      const uint32_t box[3] = {128, static_cast<uint32_t>(kDnBn), 1};
+      if (!make_map_u8(&mB2, a.w_down, 3, dims, str, box, true)) return cudaErrorInvalidValue;
       const uint64_t sd[3] = {d, F / 32, N};
       const uint64_t ss[2] = {d, (F / 32) * d};
-      const uint32_t sb[3] = {static_cast<uint32_t>(kDnBn), 2, 1};
-      if (!make_map_u8(&mS2, a.w_down_scales, 3, sd, ss, sb)) return cudaErrorInvalidValue;
+      const uint32_t sb[3] = {static_cast<uint32_t>(kDnBn), kg2, 1};
+      if (!make_map_u8(&mS2, a.w_down_scales, 3, sd, ss, sb, false)) return cudaErrorInvalidValue;
     }
   } else if (swiglu) {
     const uint64_t dims[4] = {d, F, 2, N};

@@ -53,3 +53,14 @@ def test_workload_parsing():
     assert s.d_model == 4096 and T == 512
     s, T = bench.parse_workload("switch_top1")
     assert T == 4096
+
+
+def test_mx_weight_bytes():
+    # one E8M0 scale byte per 32 elements; 1 byte (MXFP8) or half a byte (MXFP4) per element
+    assert bench.weight_bytes(1024, "bf16") == 2048
+    assert bench.weight_bytes(1024, "mxfp8") == 1024 + 32
+    assert bench.weight_bytes(1024, "mxfp4") == 512 + 32
+    s = synthetic.SHAPES["gpt_oss"]
+    b = bench.algorithmic_bytes(s, 1, 4, 4, "mxfp4")
+    params = 3 * 2880 * 2880
+    assert b["weights"] == 4 * (params // 2 + params // 32)
