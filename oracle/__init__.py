@@ -5,7 +5,8 @@ use this package. The CUDA library never imports it.
 """
 from .moe_oracle import *  # noqa: F401,F403
 from .moe_oracle import (capacity_from_factor, router_logits, softmax_over_experts,  # noqa: F401
-                         select_top_k, renormalise, assign_capacity_slots, route_from_logits,
+                         select_top_k, renormalise, assign_capacity_slots,
+                         assign_capacity_slots_reroute, route_from_logits,
                          expert_permutation, silu, gelu, expert_ffn, combine,
                          moe_layer_forward, router_statistics)
 from .mx_oracle import (MX_BLOCK, decode_e8m0, decode_e4m3, decode_e2m1,  # noqa: F401

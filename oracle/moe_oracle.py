@@ -132,13 +132,56 @@ def assign_capacity_slots(topk_idx: np.ndarray, capacity: int, n_experts: int):
     return slot, filled
 
 
-def route_from_logits(logits: np.ndarray, k: int, capacity: int) -> dict:
-    """Softmax, top-k, renormalise and capacity assignment for given logits."""
+def assign_capacity_slots_reroute(topk_idx: np.ndarray, logits: np.ndarray, capacity: int):
+    """Overflow policy "redirect to the next most suitable expert" (page «Архитектура MoE в
+    больших языковых моделях — кто такие «эксперты»?» (gerwin.io), section «Как работает MoE:
+    принцип маршрутизации», the load-balancing list: exceeding an expert's capacity may drop
+    tokens or redirect them to the next most suitable expert).
+
+    Reading (the page names the policy only): pairs arrive in the same order as for
+    dropping (choice 0 of every token in token order, then choice 1, ...). A pair whose
+    expert is full goes instead to the token's most probable expert (largest logit, equal
+    logits to the lower index) that has a free slot and that the token does not already
+    use: neither another of its top-k choices nor an earlier redirect. If no expert
+    qualifies, the pair is dropped. A redirected pair keeps its router weight.
+    Returns (expert [T, k] serving each pair, slot [T, k], kept_count [N]).
+    """
+    T, k = topk_idx.shape
+    n_experts = logits.shape[1]
+    expert = np.array(topk_idx, dtype=np.int64, copy=True)
+    filled = np.zeros(n_experts, dtype=np.int64)
+    slot = np.full((T, k), -1, dtype=np.int64)
+    for j in range(k):
+        for t in range(T):
+            e = int(expert[t, j])
+            if filled[e] < capacity:
+                slot[t, j] = filled[e]
+                filled[e] += 1
+                continue
+            used = {int(u) for u in expert[t]}
+            # candidates in the token's order of preference
+            order = sorted(range(n_experts), key=lambda c: (-logits[t, c], c))
+            for c in order:
+                if c not in used and filled[c] < capacity:
+                    expert[t, j] = c
+                    slot[t, j] = filled[c]
+                    filled[c] += 1
+                    break
+    return expert, slot, filled
+
+
+def route_from_logits(logits: np.ndarray, k: int, capacity: int, reroute: bool = False) -> dict:
+    """Softmax, top-k, renormalise and capacity assignment for given logits. With reroute,
+    overflowing pairs go to the next most suitable expert (topk_idx then holds the expert
+    serving each pair; the weights are the router's)."""
     n_experts = logits.shape[1]
     probs = softmax_over_experts(logits)
     topk_idx = select_top_k(logits, k)
     topk_w = renormalise(probs, topk_idx)
-    slot, kept = assign_capacity_slots(topk_idx, capacity, n_experts)
+    if reroute:
+        topk_idx, slot, kept = assign_capacity_slots_reroute(topk_idx, logits, capacity)
+    else:
+        slot, kept = assign_capacity_slots(topk_idx, capacity, n_experts)
     return {"topk_idx": topk_idx, "topk_w": topk_w, "slot": slot, "expert_count": kept}
 
 

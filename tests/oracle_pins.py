@@ -361,3 +361,78 @@ def pin_dequantize_blocks(m):
 
 MX_PINS = [pin_e8m0_closed_forms, pin_e4m3_closed_forms, pin_e4m3_against_torch, pin_e2m1_table,
            pin_fp4_nibble_order, pin_dequantize_blocks]
+
+
+# ---------------------------------------------------------------- reroute overflow policy
+def pin_reroute_hand_case(o):
+    # N = 3, k = 1, capacity 1. Token 0 takes expert 0; token 1 overflows expert 0 and goes to
+    # its next best expert 2; token 2 overflows expert 0, its next best (1) has room.
+    logits = np.array([[3.0, 1.0, 2.0], [3.0, 1.0, 2.0], [3.0, 2.0, 1.0]])
+    top = o.select_top_k(logits, 1)
+    expert, slot, kept = o.assign_capacity_slots_reroute(top, logits, 1)
+    assert expert.tolist() == [[0], [2], [1]]
+    assert slot.tolist() == [[0], [0], [0]] and kept.tolist() == [1, 1, 1]
+    # a fourth token finds every expert full: dropped, and keeps its own choice
+    logits4 = np.vstack([logits, [[0.0, 5.0, 4.0]]])
+    expert, slot, kept = o.assign_capacity_slots_reroute(o.select_top_k(logits4, 1), logits4, 1)
+    assert expert[3].tolist() == [1] and slot[3].tolist() == [-1]
+
+
+def pin_reroute_skips_own_choices(o):
+    # k = 2, capacity 1, N = 4: token 1's choices are experts 0 and 1 (both taken by token 0
+    # in choice order); its redirects skip its own choices and each other: experts 2, then 3.
+    logits = np.array([[9.0, 8.0, 1.0, 0.0], [9.0, 8.0, 2.0, 3.0]])
+    top = o.select_top_k(logits, 2)
+    expert, slot, kept = o.assign_capacity_slots_reroute(top, logits, 1)
+    # arrivals: (t0, j0)->0, (t1, j0)->0 full->best free not used {3 (3.0), 2 (2.0)} = 3,
+    # (t0, j1)->1, (t1, j1)->1 full-> free and unused: 2
+    assert expert.tolist() == [[0, 1], [3, 2]]
+    assert slot.tolist() == [[0, 0], [0, 0]] and kept.tolist() == [1, 1, 1, 1]
+
+
+def pin_reroute_properties(o):
+    rng = np.random.default_rng(5)
+    for trial in range(40):
+        T, N = int(rng.integers(1, 12)), int(rng.integers(2, 7))
+        k = int(rng.integers(1, N + 1))
+        cap = int(rng.integers(0, 4))
+        logits = rng.integers(-3, 4, size=(T, N)).astype(np.float64)  # many ties
+        top = o.select_top_k(logits, k)
+        expert, slot, kept = o.assign_capacity_slots_reroute(top, logits, cap)
+        # without overflow the policy equals dropping
+        s0, k0 = o.assign_capacity_slots(top, max(cap, T), N)
+        e1, s1, k1 = o.assign_capacity_slots_reroute(top, logits, max(cap, T))
+        assert np.array_equal(e1, top) and np.array_equal(s1, s0) and np.array_equal(k1, k0)
+        for t in range(T):
+            assert len(set(expert[t].tolist())) == k, "a token's pairs use distinct experts"
+        assert (kept <= cap).all()
+        for e in range(N):  # slots of each expert are 0..kept-1 exactly once
+            got = sorted(int(slot[t, j]) for t in range(T) for j in range(k)
+                         if expert[t, j] == e and slot[t, j] >= 0)
+            assert got == list(range(kept[e]))
+        # a dropped pair's token already uses every expert that still has room at the end
+        for t in range(T):
+            for j in range(k):
+                if slot[t, j] < 0:
+                    free = {e for e in range(N) if kept[e] < cap}
+                    assert free <= set(expert[t].tolist())
+        # brute force: replay the arrivals with the "best free unused expert" rule written as
+        # an argmax (equal logits to the lower index) instead of a sorted scan
+        ex = top.copy()
+        cnt = np.zeros(N, dtype=np.int64)
+        for j in range(k):
+            for t in range(T):
+                e = ex[t, j]
+                if cnt[e] < cap:
+                    cnt[e] += 1
+                    continue
+                cands = [c for c in range(N) if cnt[c] < cap and c not in set(ex[t].tolist())]
+                if cands:
+                    best = max(cands, key=lambda c: (logits[t, c], -c))
+                    ex[t, j] = best
+                    cnt[best] += 1
+        assert np.array_equal(ex, expert) and np.array_equal(cnt, kept)
+
+
+REROUTE_PINS = [pin_reroute_hand_case, pin_reroute_skips_own_choices, pin_reroute_properties]
+ALL_PINS = ALL_PINS + REROUTE_PINS

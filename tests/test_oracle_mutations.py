@@ -197,3 +197,89 @@ def test_some_mx_pin_catches(name, monkeypatch):
         except (AssertionError, ValueError, IndexError):
             caught.append(pin.__name__)
     assert caught, f"mutant {name} passed every pin"
+
+
+# ---------------------------------------------------------------- reroute policy mutants
+def _reroute_allows_reuse(topk_idx, logits, capacity):
+    T, k = topk_idx.shape
+    N = logits.shape[1]
+    expert = np.array(topk_idx, dtype=np.int64, copy=True)
+    filled = np.zeros(N, dtype=np.int64)
+    slot = np.full((T, k), -1, dtype=np.int64)
+    for j in range(k):
+        for t in range(T):
+            e = int(expert[t, j])
+            if filled[e] < capacity:
+                slot[t, j] = filled[e]
+                filled[e] += 1
+                continue
+            for c in sorted(range(N), key=lambda c: (-logits[t, c], c)):
+                if filled[c] < capacity:  # mistake: may pick an expert the token already uses
+                    expert[t, j], slot[t, j] = c, filled[c]
+                    filled[c] += 1
+                    break
+    return expert, slot, filled
+
+
+def _reroute_token_major(topk_idx, logits, capacity):
+    T, k = topk_idx.shape
+    N = logits.shape[1]
+    expert = np.array(topk_idx, dtype=np.int64, copy=True)
+    filled = np.zeros(N, dtype=np.int64)
+    slot = np.full((T, k), -1, dtype=np.int64)
+    for t in range(T):  # mistake: token-major arrivals
+        for j in range(k):
+            e = int(expert[t, j])
+            if filled[e] < capacity:
+                slot[t, j] = filled[e]
+                filled[e] += 1
+                continue
+            used = set(expert[t].tolist())
+            for c in sorted(range(N), key=lambda c: (-logits[t, c], c)):
+                if c not in used and filled[c] < capacity:
+                    expert[t, j], slot[t, j] = c, filled[c]
+                    filled[c] += 1
+                    break
+    return expert, slot, filled
+
+
+def _reroute_worst_first(topk_idx, logits, capacity):
+    T, k = topk_idx.shape
+    N = logits.shape[1]
+    expert = np.array(topk_idx, dtype=np.int64, copy=True)
+    filled = np.zeros(N, dtype=np.int64)
+    slot = np.full((T, k), -1, dtype=np.int64)
+    for j in range(k):
+        for t in range(T):
+            e = int(expert[t, j])
+            if filled[e] < capacity:
+                slot[t, j] = filled[e]
+                filled[e] += 1
+                continue
+            used = set(expert[t].tolist())
+            for c in sorted(range(N), key=lambda c: (logits[t, c], c)):  # mistake: least suitable
+                if c not in used and filled[c] < capacity:
+                    expert[t, j], slot[t, j] = c, filled[c]
+                    filled[c] += 1
+                    break
+    return expert, slot, filled
+
+
+REROUTE_MUTANTS = {
+    "reroute_reuses_own_expert": ("assign_capacity_slots_reroute", _reroute_allows_reuse),
+    "reroute_token_major": ("assign_capacity_slots_reroute", _reroute_token_major),
+    "reroute_least_suitable": ("assign_capacity_slots_reroute", _reroute_worst_first),
+}
+
+
+@pytest.mark.parametrize("name", sorted(REROUTE_MUTANTS))
+def test_some_reroute_pin_catches(name, monkeypatch):
+    attr, fn = REROUTE_MUTANTS[name]
+    monkeypatch.setattr(om, attr, fn)
+    caught = []
+    for pin in oracle_pins.REROUTE_PINS:
+        try:
+            pin(om)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, f"mutant {name} passed every pin"
