@@ -299,6 +299,41 @@ class Layer:
                 "dropped_pairs": int(dropped.item()), "algorithmic_bytes": nbytes,
                 "achieved_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
 
+    def redirect_timing(self, steps: int, flush) -> dict:
+        """moe_redirect_overflow (overflow policy "redirect") on the step's logits and top-k,
+        into separate buffers: mean ms per call of a graph that restores the router's top-k
+        (a T*k*4-byte device copy) and redirects. Pairs kept and redirected, against dropping."""
+        moe, v = self.moe, self.views()
+        N, k, T = self.shape.n_experts, self.shape.top_k, self.T
+        dev = v["logits"].device
+        idx0 = v["topk_idx"].clone()
+        idx = torch.empty_like(idx0)
+        slot = torch.empty((T, k), dtype=torch.int32, device=dev)
+        cnt = torch.empty((N,), dtype=torch.int32, device=dev)
+
+        def call():
+            idx.copy_(idx0)
+            moe.redirect_overflow(self.dims, v["logits"], idx, slot, cnt, v["stage_ws"])
+        call()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for e0, e1 in evs:
+            flush_l2(flush)
+            e0.record()
+            g.replay()
+            e1.record()
+        torch.cuda.synchronize()
+        ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+        kept = int((slot >= 0).sum())
+        return {"ms": round(ms, 4), "pairs": T * k, "kept_pairs": kept,
+                "kept_pairs_drop_policy": int((v["slot"] >= 0).sum()),
+                "redirected_pairs": int((idx != idx0).sum()),
+                "ns_per_pair": round(ms * 1e6 / (T * k), 2)}
+
     def stage_calls(self):
         """The four stage calls of one forward (the calls moe_forward makes), as closures."""
         moe, i, b, dims = self.moe, self.inp, self.b, self.dims
@@ -508,6 +543,9 @@ def run_gpu(args, rank, world, local_rank):
     # router statistics and the auxiliary loss over this step's routing (a "next" row),
     # replayed as a graph K times between events
     stats = layer.stats_timing(args.steps, flush)
+    # overflow policy "redirect" on the same routing (a "next" row), where the batch allows it
+    redirect = (layer.redirect_timing(args.steps, flush)
+                if T * shape.top_k <= moe.REDIRECT_MAX_PAIRS else None)
 
     # end to end through the public call with host buffers (copies overlap neighbouring steps)
     if world > 1:
@@ -562,6 +600,7 @@ def run_gpu(args, rank, world, local_rank):
                              "steps replayed as one graph per stage with events between stages"},
         "stages_ms": {k: round(v_, 4) for k, v_ in stage_ms.items()},
         "router_stats": stats,
+        "overflow_redirect": redirect,
         "roofline": roof,
         "layer_gbs": round(ab["layer"] / (total_ms / args.steps * 1e-3) / 1e9, 1),
         "ffn_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 2),

@@ -103,7 +103,8 @@ int64_t moe_max_rows(const moe_dims* dims);
  *       - the capacity scan's chunk totals;
  *       - the router's bf16 three-term split of W_r, on the tensor-core path;
  *       - the grouped FFN's stream-K partial tiles (two per CTA);
- *       - moe_router_stats's partial sums.
+ *       - moe_router_stats's partial sums;
+ *       - moe_redirect_overflow's per-token lists of next experts.
  * Zero a workspace once before its first use, with moe_workspace_init or any memset to 0.
  * Zero it again after a device error. */
 moe_status moe_workspace_bytes(const moe_dims* dims, size_t* bytes);
@@ -138,6 +139,29 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const float* w_rou
 moe_status moe_route_from_logits(const moe_dims* dims, const float* logits, int32_t* topk_idx,
                                  float* topk_w, int32_t* slot, int32_t* expert_count, void* ws,
                                  size_t ws_bytes, void* stream);
+
+/* Overflow policy "redirect": a pair that arrives at a full expert goes to the next most
+ * suitable expert instead of being dropped (page «Архитектура MoE в больших языковых моделях —
+ * кто такие «эксперты»?», section «Как работает MoE: принцип маршрутизации», which names
+ * dropping and redirecting as the two ways to handle an expert over capacity).
+ * Call after moe_route or moe_route_from_logits; it replaces their drop-policy slots. Pairs
+ * arrive in the same (choice, token) order. A pair whose expert is full goes to the token's
+ * expert with the largest logit (equal logits: lower index; NaN counts as -inf) that has a
+ * free slot and that the token does not already use (another of its top-k choices or an
+ * earlier redirect); with none, it is dropped (slot -1, topk_idx unchanged). A redirected
+ * pair keeps its router weight topk_w.
+ *   logits       [T, N] fp32            the router logits (from moe_route)
+ *   topk_idx     [T, k] int32 (in/out)  the router's choices in; the expert serving each pair out
+ *   slot         [T, k] int32 (out)     slot in the serving expert's buffer, -1 = dropped
+ *   expert_count [N] int32 (out)        kept pairs per expert, <= capacity
+ * topk_idx must be the top-k of these logits as moe_route writes them: a list of each token's
+ * next 16 experts after its top-k (written into the workspace by a first launch over all SMs)
+ * stands in for a scan of its logits, which only runs when all 16 fail. The decisions depend
+ * on each other in arrival order, so one warp then takes them in sequence (second launch).
+ * MOE_ERR_UNSUPPORTED when T * k > 32768. Uses the per-stage workspace (T * 16 bytes). */
+moe_status moe_redirect_overflow(const moe_dims* dims, const float* logits, int32_t* topk_idx,
+                                 int32_t* slot, int32_t* expert_count, void* ws, size_t ws_bytes,
+                                 void* stream);
 
 /* Permute: step 4, sort by expert id.
  *   expert_offset [N+1] int32 (out)  exclusive prefix sum of expert_count; expert e owns rows

@@ -73,6 +73,7 @@ _SIGS = {
     "moe_workspace_init": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "moe_route": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_route_from_logits": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_redirect_overflow": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_permute": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_grouped_ffn": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_unpermute_combine": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, ctypes.c_int32, _P,
@@ -227,6 +228,19 @@ def route_from_logits(dims: Dims, logits, topk_idx, topk_w, slot, expert_count, 
         _ptr(topk_idx, "topk_idx", torch.int32, (T, k)), _ptr(topk_w, "topk_w", torch.float32, (T, k)),
         _ptr(slot, "slot", torch.int32, (T, k)), _ptr(expert_count, "expert_count", torch.int32, (N,)),
         _ptr(ws, "ws", torch.uint8), _nbytes(ws), _stream(stream)), "moe_route_from_logits")
+
+
+REDIRECT_MAX_PAIRS = 32768  # T * k limit of moe_redirect_overflow
+
+
+def redirect_overflow(dims: Dims, logits, topk_idx, slot, expert_count, ws, stream=None) -> None:
+    """Overflow policy "redirect" after route(): topk_idx is rewritten with the serving expert."""
+    T, N, k = dims.T, dims.n_experts, dims.top_k
+    _check(_lib.moe_redirect_overflow(
+        ctypes.byref(dims), _ptr(logits, "logits", torch.float32, (T, N)),
+        _ptr(topk_idx, "topk_idx", torch.int32, (T, k)), _ptr(slot, "slot", torch.int32, (T, k)),
+        _ptr(expert_count, "expert_count", torch.int32, (N,)),
+        _ptr(ws, "ws", torch.uint8), _nbytes(ws), _stream(stream)), "moe_redirect_overflow")
 
 
 def permute(dims: Dims, x, topk_idx, slot, expert_count, expert_offset, row_of_pair,

@@ -115,7 +115,8 @@ size_t shared_region_bytes(const moe_dims* d) {
   const size_t routing = slot_scratch_bytes(d) + split_scratch_bytes(d) + decode_scratch_bytes(d);
   const size_t ffn = round_up(ffn_plan(d).part_bytes, 256);
   const size_t stats = round_up(moe::router_stats_scratch_bytes(d->T, d->n_experts), 256);
-  return std::max(std::max(routing, ffn), stats);
+  const size_t redirect = round_up(moe::redirect_scratch_bytes(d->T, d->top_k), 256);
+  return std::max(std::max(std::max(routing, ffn), stats), redirect);
 }
 
 size_t stage_ws_bytes(const moe_dims* d) {
@@ -245,6 +246,27 @@ moe_status moe_route_from_logits(const moe_dims* dims, const float* logits, int3
                                                   dims->n_experts, dims->top_k, s));
   if (st != MOE_OK) return st;
   return route_slots(dims, topk_idx, slot, expert_count, ws, s);
+}
+
+moe_status moe_redirect_overflow(const moe_dims* dims, const float* logits, int32_t* topk_idx,
+                                 int32_t* slot, int32_t* expert_count, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (dims->T == 0) return MOE_OK;
+  if (!logits || !topk_idx || !slot || !expert_count || !ws) return MOE_ERR_INVALID;
+  if (static_cast<int64_t>(dims->T) * dims->top_k > moe::kRerouteMaxPairs)
+    return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(logits) || !aligned16(topk_idx) || !aligned16(slot) || !aligned16(expert_count) ||
+      !aligned16(ws))
+    return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < stage_ws_bytes(dims)) return MOE_ERR_WORKSPACE;
+  if ((st = check_device()) != MOE_OK) return st;
+  uint8_t* prefs = reinterpret_cast<uint8_t*>(shared_region_of(dims, ws));
+  return launch_status(moe::launch_reroute_slots(logits, prefs, topk_idx, slot, expert_count,
+                                                 dims->T, dims->n_experts, dims->top_k,
+                                                 std::min(dims->capacity, dims->T),
+                                                 as_stream(stream)));
 }
 
 moe_status moe_permute(const moe_dims* dims, const uint16_t* x, const int32_t* topk_idx,

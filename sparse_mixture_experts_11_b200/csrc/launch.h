@@ -123,6 +123,17 @@ struct DecodeRouteArgs {
   int T, d, N, k, cap;
 };
 cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t s);
+// Overflow policy "redirect to the next most suitable expert" (see route.cu): slots and the
+// serving experts from the router's top-k and logits, for at most kRerouteMaxPairs pairs.
+// prefs: T * kRedirectPrefs bytes of scratch, 16-byte aligned.
+constexpr int64_t kRerouteMaxPairs = 32768;
+constexpr int kRedirectPrefs = 16;
+inline size_t redirect_scratch_bytes(int64_t T, int k) {
+  return T * k <= kRerouteMaxPairs ? static_cast<size_t>(T) * kRedirectPrefs : 0;
+}
+cudaError_t launch_reroute_slots(const float* logits, uint8_t* prefs, int32_t* topk_idx,
+                                int32_t* slot, int32_t* expert_count, int T, int N, int k,
+                                int capacity, cudaStream_t s);
 // top-k and renormalised weights from given logits
 cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, float* topk_w, int T,
                                     int N, int k, cudaStream_t s);

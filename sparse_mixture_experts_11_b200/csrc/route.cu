@@ -317,6 +317,291 @@ __global__ void __launch_bounds__(256) slot_finalize_kernel(const int32_t* __res
   }
 }
 
+// ------------------------------------------------------------------ overflow: redirect
+// Page «Архитектура MoE в больших языковых моделях — кто такие «эксперты»?», section «Как
+// работает MoE: принцип маршрутизации»: a pair over its expert's capacity may be dropped or
+// redirected to the next most suitable expert. Reading: arrivals in (choice, token) order; a
+// pair whose expert is full goes to the token's best expert (largest logit, equal logits to
+// the lower index) that has a free slot and that the token does not use yet; with none, it is
+// dropped. topk_idx is rewritten with the serving expert; the router weights stay.
+//
+// Two launches. redirect_prefs_kernel (one warp per token, all SMs) writes each token's next
+// kRedirectPrefs experts after its top-k, best first, as bytes (255 = none). The experts of
+// the top-k never qualify later: each is either still the token's or was full when its pair
+// arrived, and counts only grow. So the best qualifying expert is the first qualifying entry
+// of the list, unless every entry fails and the list does not cover all the token's other
+// experts; only then are the token's logits scanned.
+//
+// reroute_slots_kernel: each decision depends on all earlier ones, so one warp walks the
+// arrivals in order, 32 at a time (lane l takes arrival a0 + l), and decides every pair of the
+// window from the counts at its start: a pair whose expert has room targets it; otherwise
+// the pair targets the first qualifying entry of its token's list (or is dropped). Lanes that
+// target the same expert take consecutive slots in lane order. A lane's decision is the one
+// the sequential rule makes as long as its target still has room after the earlier lanes'
+// slots: experts that were full stay full, and a token's other pairs only change in the same
+// window when T < 32, which also ends the window. So the window commits every lane before the
+// first one whose slot is past the capacity (or that needs the full scan, or whose token is
+// already in the window), and the next window starts there. A window's first lane always
+// commits; when it needs the scan, the warp scans the token's logits for it alone. Once no
+// expert has a free slot, the rest are dropped. The pairs come into shared memory with
+// cp.async, and the lists stream through a ring of kRedirectRing rows refilled half a ring
+// ahead of the walk, so the sequential path does not wait on global memory.
+constexpr int kRedirectRing = 2048;
+
+struct RerouteSmem {
+  static __host__ __device__ size_t bytes(int P) {
+    return static_cast<size_t>(kRedirectRing) * kRedirectPrefs + 256 * 4 +
+           static_cast<size_t>(P) * 4;
+  }
+};
+
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_newest_pending() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
+// Lanes holding the same value v (0 <= v < 256) among the lanes where `on` holds.
+__device__ __forceinline__ unsigned lanes_with_same(int v, bool on) {
+  unsigned same = __ballot_sync(kFull, on);
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    const bool bit = (v >> b) & 1;
+    const unsigned m = __ballot_sync(kFull, bit);
+    same &= bit ? m : ~m;
+  }
+  return same;
+}
+
+// Experts ranked k .. k + kRedirectPrefs - 1 in the token's order (logit descending, equal
+// logits to the lower index, NaN as -inf), as bytes; 255 past the last expert.
+__global__ void __launch_bounds__(256) redirect_prefs_kernel(const float* __restrict__ logits,
+                                                             uint8_t* __restrict__ prefs, int T,
+                                                             int N, int k) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = static_cast<int>(lane_id());
+  const int warps = gridDim.x * (blockDim.x / 32);
+  const int rounds = min(N, k + kRedirectPrefs);
+  for (int t = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; t < T; t += warps) {
+    float val[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      const float v = e < N ? logits[static_cast<int64_t>(t) * N + e] : -INFINITY;
+      val[i] = isnan(v) ? -INFINITY : v;
+    }
+    uint32_t taken = 0;
+    int mine = 255;  // lane r < kRedirectPrefs keeps the expert of rank k + r
+    for (int r = 0; r < rounds; ++r) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        if (e < N && !((taken >> i) & 1u) && better(val[i], e, bv, be)) {
+          bv = val[i];
+          be = e;
+        }
+      }
+      warp_best(bv, be);
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      if (r >= k && lane == r - k) mine = be;
+    }
+    if (lane < kRedirectPrefs)
+      prefs[static_cast<int64_t>(t) * kRedirectPrefs + lane] = static_cast<uint8_t>(mine);
+  }
+}
+
+// Lists of stream positions [from, to) (position a is token a mod T) into ring rows a mod
+// kRedirectRing, one cp.async group.
+__device__ __forceinline__ void stage_prefs(const uint8_t* prefs, uint8_t* ring, int from, int to,
+                                            int T, int lane) {
+  for (int a = from + lane; a < to; a += 32)
+    cp_async_16(smem_u32(ring + (a % kRedirectRing) * kRedirectPrefs),
+                prefs + static_cast<int64_t>(a % T) * kRedirectPrefs);
+  cp_async_commit();
+}
+
+__global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restrict__ logits,
+                                                           const uint8_t* __restrict__ prefs,
+                                                           int32_t* __restrict__ topk_idx,
+                                                           int32_t* __restrict__ slot,
+                                                           int32_t* __restrict__ expert_count,
+                                                           int T, int N, int k, int cap) {
+  extern __shared__ __align__(16) int r_sm[];
+  const int P = T * k;
+  uint8_t* ring = reinterpret_cast<uint8_t*>(r_sm);      // [ring][prefs]
+  int* cnt = r_sm + kRedirectRing * kRedirectPrefs / 4;  // [256] filled slots
+  int* ex = cnt + 256;                                   // [P] serving experts
+  pdl_trigger();
+  pdl_wait();
+  const int lane = static_cast<int>(lane_id());
+  {  // the pairs (ex and topk_idx are 16-byte aligned)
+    const int p4 = P / 4;
+    for (int i = lane; i < p4; i += 32) cp_async_16(smem_u32(ex + 4 * i), topk_idx + 4 * i);
+    for (int q = 4 * p4 + lane; q < P; q += 32) cp_async_4(smem_u32(ex + q), topk_idx + q);
+    cp_async_commit();
+  }
+  constexpr int kHalf = kRedirectRing / 2;
+  int filled = min(P, kHalf);  // lists of positions below `filled` are requested
+  stage_prefs(prefs, ring, 0, filled, T, lane);
+  int newest = 0;  // first position of the newest group
+  if (filled < P) {
+    newest = filled;
+    stage_prefs(prefs, ring, filled, min(P, 2 * kHalf), T, lane);
+    filled = min(P, 2 * kHalf);
+  }
+  for (int e = lane; e < 256; e += 32) cnt[e] = 0;
+  const bool whole_list = N - k <= kRedirectPrefs;  // the list holds every other expert
+  int room = cap > 0 ? N : 0;                       // experts with a free slot
+  cp_async_wait_all();
+  __syncwarp();
+  int waited = filled;  // lists of positions below `waited` have landed
+  int t = lane % T;     // token and choice of arrival a0 + lane
+  int j = lane / T;
+  int a0 = 0;           // first arrival not decided yet
+  while (a0 < P) {
+    if (room == 0) {  // no free slot anywhere: the rest are dropped
+      for (int a = a0 + lane; a < P; a += 32) {
+        const int jj = a / T;
+        slot[(a - jj * T) * k + jj] = -1;
+      }
+      break;
+    }
+    if (filled < P && a0 >= filled - kHalf) {
+      // the walk is past the older half: refill it with the next positions
+      cp_async_wait_newest_pending();  // the group that last wrote those rows has landed
+      waited = max(waited, newest);
+      __syncwarp();
+      newest = filled;
+      stage_prefs(prefs, ring, filled, min(P, filled + kHalf), T, lane);
+      filled = min(P, filled + kHalf);
+    }
+    const int n_act = min(32, P - a0);
+    const bool act = lane < n_act;
+    const int q = t * k + j;
+    const int e = act ? ex[q] : -1;
+    const bool valid = act && e >= 0 && e < N;
+    const bool need = act && (!valid || cnt[e] >= cap);  // own expert full: search the list
+    if (__any_sync(kFull, need) && a0 + n_act - 1 >= waited) {
+      if (a0 + n_act - 1 >= newest) {
+        cp_async_wait_all();
+        waited = filled;
+      } else {
+        cp_async_wait_newest_pending();
+        waited = newest;
+      }
+      __syncwarp();
+    }
+    int target = (act && !need) ? e : -1;
+    bool scan = false;
+    if (need && room > 0) {
+      const uint4 row =
+          *reinterpret_cast<const uint4*>(ring + ((a0 + lane) % kRedirectRing) * kRedirectPrefs);
+      int own[8];  // the token's current experts
+#pragma unroll
+      for (int j2 = 0; j2 < 8; ++j2) own[j2] = j2 < k ? ex[t * k + j2] : -1;
+      const uint32_t w4[4] = {row.x, row.y, row.z, row.w};
+#pragma unroll
+      for (int r = 0; r < kRedirectPrefs; ++r) {
+        const int cand = (w4[r >> 2] >> (8 * (r & 3))) & 0xff;
+        bool ok = cand < N && cnt[cand] < cap;
+#pragma unroll
+        for (int j2 = 0; j2 < 8; ++j2) ok &= own[j2] != cand;
+        if (ok && target < 0) target = cand;
+      }
+      scan = target < 0 && !whole_list;
+    }
+    const unsigned same = lanes_with_same(target, target >= 0);
+    const int c = target >= 0 ? cnt[target] + __popc(same & lanemask_lt()) : -1;
+    bool dup = false;  // the token already has an earlier lane in this window
+    if (T < 32) {
+      const unsigned st = lanes_with_same(t, act);
+      dup = (st & lanemask_lt()) != 0;
+    }
+    const unsigned bad = __ballot_sync(kFull, act && ((target >= 0 && c >= cap) || scan || dup));
+    const int first = bad ? __ffs(bad) - 1 : n_act;
+    __syncwarp();  // every lane has read cnt and ex before they change
+    if (first == 0) {
+      // the window's first pair needs a scan of its token's logits
+      const int t0 = __shfl_sync(kFull, t, 0);
+      const int q0 = __shfl_sync(kFull, q, 0);
+      const float* lrow = logits + static_cast<int64_t>(t0) * N;
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = (lane + 32 * i < N) ? lrow[lane + 32 * i] : -INFINITY;
+      int used = 0;  // bit i: expert lane + 32 i is already one of the token's
+      for (int j2 = 0; j2 < k; ++j2) {
+        const int e2 = ex[t0 * k + j2];
+        if (e2 >= 0 && e2 < N && (e2 & 31) == lane) used |= 1 << (e2 >> 5);
+      }
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c2 = lane + 32 * i;
+        if (c2 < N && !((used >> i) & 1) && cnt[c2] < cap) {
+          const float vi = isnan(v[i]) ? -INFINITY : v[i];
+          if (better(vi, c2, bv, bi)) {
+            bv = vi;
+            bi = c2;
+          }
+        }
+      }
+      warp_best(bv, bi);
+      const int out = bi != 0x7fffffff ? cnt[bi] : -1;
+      if (out >= 0 && out + 1 == cap) --room;
+      __syncwarp();
+      if (lane == 0) {
+        slot[q0] = out;
+        if (out >= 0) {
+          cnt[bi] = out + 1;
+          ex[q0] = bi;
+        }
+      }
+      __syncwarp();
+      a0 += 1;
+      t += 1;
+      while (t >= T) {
+        t -= T;
+        ++j;
+      }
+      continue;
+    }
+    const unsigned commit = first >= 32 ? kFull : ((1u << first) - 1);
+    const bool mine = lane < first;
+    const bool last = target >= 0 && ((same & commit) >> lane) == 1u;  // last lane on target
+    if (mine) {
+      slot[q] = target >= 0 ? c : -1;
+      if (target >= 0 && target != e) ex[q] = target;
+      if (last) cnt[target] = c + 1;
+    }
+    room -= __popc(__ballot_sync(kFull, mine && last && c + 1 == cap));
+    __syncwarp();
+    a0 += first;
+    t += first;
+    while (t >= T) {
+      t -= T;
+      ++j;
+    }
+  }
+  cp_async_wait_all();
+  __syncwarp();
+  for (int qq = lane; qq < P; qq += 32) topk_idx[qq] = ex[qq];
+  for (int e = lane; e < N; e += 32) expert_count[e] = cnt[e];
+}
+
 // ------------------------------------------------------------------ decode-sized batches
 // One launch for T <= kDecodeRouteMaxT tokens. CTA c owns d columns [128 c, 128 c + 128): lane
 // l holds 4 of them of every token's x, and warp w takes experts w, w + 8, ... one float4 of
@@ -500,6 +785,23 @@ cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t s) {
   return launch_pdl(pick(decode_route_kernel<16, 1>, decode_route_kernel<16, 2>,
                          decode_route_kernel<16, 4>, decode_route_kernel<16, 8>),
                     dim3(ctas), dim3(kDrThreads), 0, s, a);
+}
+
+cudaError_t launch_reroute_slots(const float* logits, uint8_t* prefs, int32_t* topk_idx,
+                                int32_t* slot, int32_t* expert_count, int T, int N, int k,
+                                int capacity, cudaStream_t s) {
+  if (static_cast<int64_t>(T) * k > kRerouteMaxPairs || N > 256) return cudaErrorInvalidValue;
+  static cudaError_t attr = cudaFuncSetAttribute(
+      reroute_slots_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      static_cast<int>(RerouteSmem::bytes(static_cast<int>(kRerouteMaxPairs))));
+  if (attr != cudaSuccess) return attr;
+  const int blocks = std::max(1, std::min((T + 7) / 8, 4 * 148));
+  cudaError_t e = launch_pdl(redirect_prefs_kernel, dim3(blocks), dim3(256), 0, s, logits, prefs,
+                             T, N, k);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(reroute_slots_kernel, dim3(1), dim3(32), RerouteSmem::bytes(T * k), s, logits,
+                    static_cast<const uint8_t*>(prefs), topk_idx, slot, expert_count, T, N, k,
+                    capacity);
 }
 
 cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, float* topk_w, int T,

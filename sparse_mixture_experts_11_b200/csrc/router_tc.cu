@@ -356,13 +356,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // issue every load of this k block before waiting, so their latencies overlap
         float4 v[kTasks][2];
 #pragma unroll
-        for (int i = 0; i < kTasks; ++i) {
-          const int task = ct + i * kConvThreads;
+        for (int u = 0; u < kTasks; ++u) {
+          const int task = ct + u * kConvThreads;
           if (task < N * 8) {
             const float4* src = reinterpret_cast<const float4*>(
                 w + static_cast<int64_t>(task >> 3) * d + kb * kBK + (task & 7) * 8);
-            v[i][0] = __ldg(src);
-            v[i][1] = __ldg(src + 1);
+            v[u][0] = __ldg(src);
+            v[u][1] = __ldg(src + 1);
           }
         }
         const bool got = mbar_wait(smem_u32(&w_empty[b]), ((i >> 1) & 1) ^ 1u, timeout_ns, &s_abort);
@@ -373,11 +373,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after_sync();
         uint8_t* buf = gbase + b * C::WBUF_BYTES;
 #pragma unroll
-        for (int i = 0; i < kTasks; ++i) {
-          const int task = ct + i * kConvThreads;
+        for (int u = 0; u < kTasks; ++u) {
+          const int task = ct + u * kConvThreads;
           if (task < N * 8) {
             uint4 hi, mid, lo;
-            split3(v[i][0], v[i][1], hi, mid, lo);
+            split3(v[u][0], v[u][1], hi, mid, lo);
             const uint32_t off = sw128_offset(task >> 3, task & 7);
             *reinterpret_cast<uint4*>(buf + off) = hi;
             *reinterpret_cast<uint4*>(buf + C::WT_BYTES + off) = mid;

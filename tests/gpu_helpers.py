@@ -83,11 +83,14 @@ class StageRun:
             self.mx = None
             self.gu, self.dn = expert_weights_f64(inp["w_gate_up"]), expert_weights_f64(inp["w_down"])
 
-    def run(self, residual=True):
+    def run(self, residual=True, redirect=False):
         i = self.inp
         res = i["x"] if residual else None
         moe.route(self.dims, i["x"], i["w_router"], i.get("logit_bias"), self.logits, self.topk_idx,
                   self.topk_w, self.slot, self.expert_count, self.ws)
+        if redirect:
+            moe.redirect_overflow(self.dims, self.logits, self.topk_idx, self.slot,
+                                  self.expert_count, self.ws)
         moe.permute(self.dims, i["x"], self.topk_idx, self.slot, self.expert_count,
                     self.expert_offset, self.row_of_pair, self.pair_of_row, self.x_perm, self.ws)
         if self.mx is not None:
@@ -114,11 +117,11 @@ def check_logits(gpu_logits: np.ndarray, x: np.ndarray, w_router: np.ndarray, bi
     assert not bad.any(), f"{bad.sum()} logits off; worst {np.abs(got - want).max()}"
 
 
-def check_routing(run: StageRun, cap: int):
+def check_routing(run: StageRun, cap: int, reroute=False):
     """Routing bit-exact against the oracle re-run on the GPU's own logits."""
     L = f64(run.logits)
     k = run.dims.top_k
-    r = oracle.route_from_logits(L, k, cap)
+    r = oracle.route_from_logits(L, k, cap, reroute=reroute)
     g_idx = run.topk_idx.cpu().numpy()
     assert np.array_equal(g_idx, r["topk_idx"]), "expert ids differ"
     np.testing.assert_allclose(f64(run.topk_w), r["topk_w"], rtol=0, atol=WEIGHT_ATOL)

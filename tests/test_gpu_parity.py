@@ -201,3 +201,83 @@ def test_decode_route_and_forward(case):
                          inp["w_down"], inp["x"], out, ws)
         torch.cuda.synchronize()
         assert torch.equal(out.view(torch.int16), run.out.view(torch.int16))
+
+
+# Overflow policy "redirect": pairs at a full expert go to the token's next most suitable
+# expert with a free slot (the oracle re-run on the GPU's own logits decides every pair).
+def _redirect_logits(L, k, cap):
+    import sparse_mixture_experts_11_b200 as moe
+    T, N = L.shape
+    dims = moe.make_dims(T, 64, N, k, 64, "swiglu", cap)
+    ws = moe.new_workspace(dims)
+    lg = torch.from_numpy(L).cuda()
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    slot = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((N,), -7, dtype=torch.int32, device="cuda")
+    moe.route_from_logits(dims, lg, idx, w, slot, cnt, ws)
+    moe.redirect_overflow(dims, lg, idx, slot, cnt, ws)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), w.cpu().numpy(), slot.cpu().numpy(), cnt.cpu().numpy()
+
+
+def test_redirect_hand_case():
+    """Worked by hand: one slot per expert, top-1. Token 0 keeps expert 0; token 1 prefers 0
+    (full), then 2 (logit 2 > 1); token 2 prefers 0 (full), then 1 (2 > 1, expert 2 full)."""
+    L = np.array([[3, 1, 2], [3, 1, 2], [3, 2, 1]], np.float32)
+    idx, w, slot, cnt = _redirect_logits(L, 1, 1)
+    assert idx.tolist() == [[0], [2], [1]]
+    assert slot.tolist() == [[0], [0], [0]]
+    assert cnt.tolist() == [1, 1, 1]
+    np.testing.assert_allclose(w, np.ones((3, 1)), atol=H.WEIGHT_ATOL, rtol=0)
+
+
+@pytest.mark.parametrize("T,N,k,cf", [(50, 8, 2, 1.0), (33, 64, 4, 0.5), (70, 256, 8, 1.0),
+                                      (2000, 16, 3, 1.0), (4096, 256, 8, 0.75), (4096, 256, 8, 8.0),
+                                      (300, 4, 4, 0.5),
+                                      (64, 8, 2, 0.0)])
+def test_redirect_ties(T, N, k, cf):
+    """Crafted logits with many exact ties; at T * k = 32768 the largest supported batch."""
+    rng = np.random.default_rng(7 * T + N + k)
+    L = rng.integers(-3, 4, size=(T, N)).astype(np.float32) * 0.5
+    cap = oracle.capacity_from_factor(cf, T, N) if cf > 0 else 0
+    idx, w, slot, cnt = _redirect_logits(L, k, cap)
+    r = oracle.route_from_logits(L.astype(np.float64), k, cap, reroute=True)
+    assert np.array_equal(idx, r["topk_idx"])
+    assert np.array_equal(slot, r["slot"])
+    assert np.array_equal(cnt, r["expert_count"])
+    np.testing.assert_allclose(w, r["topk_w"], atol=H.WEIGHT_ATOL, rtol=0)
+
+
+@pytest.mark.parametrize("T,d,N,k,F,act,cf,zipf", [
+    (600, 256, 16, 2, 256, "swiglu", 1.0, 1.1),
+    (200, 128, 8, 2, 128, "gelu", 0.5, 1.1),
+    (96, 128, 256, 8, 128, "swiglu", 1.25, 1.1),
+], ids=["switchlike_zipf", "gelu_heavy_overflow", "fine_grained_k8"])
+def test_redirect_full_pipeline(T, d, N, k, F, act, cf, zipf):
+    """route -> redirect -> permute -> grouped FFN -> combine against the oracle."""
+    inp = _inputs(T, d, N, F, act, zipf, seed=41)
+    cap = oracle.capacity_from_factor(cf, T, N)
+    run = H.StageRun(inp, k, act, cap).run(redirect=True)
+    routing, off, rop = H.check_routing(run, cap, reroute=True)
+    H.check_x_perm(run, rop)
+    H.check_outputs(run, routing, act)
+    H.check_dropped_tokens_pass_through(run, routing["slot"])
+    drop = oracle.route_from_logits(H.f64(run.logits), k, cap)
+    # the policy keeps pairs that dropping loses
+    assert int((routing["slot"] >= 0).sum()) > int((drop["slot"] >= 0).sum())
+
+
+def test_redirect_switch_size_gaussian_logits():
+    """The default switch-like batch (T=4096, N=64, top-1, capacity factor 1.0) with Gaussian
+    logits skewed towards a few experts, as the router produces them."""
+    rng = np.random.default_rng(11)
+    T, N, k = 4096, 64, 1
+    L = (rng.standard_normal((T, N)) + np.linspace(0.0, 1.5, N)[None, :]).astype(np.float32)
+    cap = oracle.capacity_from_factor(1.0, T, N)
+    idx, w, slot, cnt = _redirect_logits(L, k, cap)
+    r = oracle.route_from_logits(L.astype(np.float64), k, cap, reroute=True)
+    assert np.array_equal(idx, r["topk_idx"])
+    assert np.array_equal(slot, r["slot"])
+    assert np.array_equal(cnt, r["expert_count"])
+    assert int((slot >= 0).sum()) == min(T * k, N * cap)  # nothing is dropped while room is left
