@@ -1,4 +1,4 @@
-"""CPU oracle of the sparse MoE layer forward pass (test infrastructure only).
+"""CPU oracle of the sparse MoE layer forward and backward passes (test infrastructure only).
 
 Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
 use this package. The CUDA library never imports it.
@@ -11,3 +11,6 @@ from .moe_oracle import (capacity_from_factor, router_logits, softmax_over_exper
                          moe_layer_forward, router_statistics)
 from .mx_oracle import (MX_BLOCK, decode_e8m0, decode_e4m3, decode_e2m1,  # noqa: F401
                         unpack_fp4, dequantize_mx)
+from .moe_backward import (logistic, silu_derivative, gelu_derivative,  # noqa: F401
+                           combine_backward, renormalise_backward, expert_backward,
+                           moe_layer_backward)
