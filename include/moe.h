@@ -252,6 +252,35 @@ moe_status moe_forward(const moe_dims* dims, const uint16_t* x, const float* w_r
                        const uint16_t* residual, uint16_t* out, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* Backward pass of the layer (bf16 expert weights), after moe_forward on the same inputs.
+ * The pages discuss training MoE layers (page «Что такое Mixture of Experts (MoE) в
+ * трансформерах», section «Обучение MoE с помощью Transformers») without formulas; this is
+ * the chain rule of the forward pass. The choice of experts and the capacity slots pass no
+ * gradient; a dropped pair's weight gets none, but it still takes part in the softmax over
+ * the chosen logits.
+ *   x, w_router, w_gate_up, w_down   the forward's inputs (residual excluded)
+ *   fwd_ws, fwd_ws_bytes   the moe_forward workspace holding that forward's intermediates
+ *                          (routing, x_perm, y_perm; see moe_forward_layout), read only
+ *   d_out        [T, d_model] bf16      gradient of the layer output
+ *   d_x          [T, d_model] fp32 (out) gradient through the router and the experts; the
+ *                                       residual's own gradient is d_out and is not added
+ *   d_w_router   [N, d_model] fp32 (out)  dL^T x, dL the logits' gradient
+ *   d_logit_bias [N] fp32 (out) or NULL   sum over tokens of dL
+ *   d_w_gate_up  [N, 2F, d_model] (SwiGLU) or [N, F, d_model] (GELU) fp32 (out)
+ *   d_w_down     [N, d_model, d_ff] fp32 (out); experts with no kept rows get zeros
+ *   ws, ws_bytes  backward workspace (moe_backward_workspace_bytes), no zeroing needed
+ * Precision: the expert GEMMs take bf16 operands (d_out * w and the activation's gradient
+ * are rounded once to bf16) with fp32 accumulation on tensor cores; the router's gradients
+ * are fp32 throughout. Deterministic for a given device. The status word of the backward
+ * workspace (its first int32) records MOE_ERR_TIMEOUT or MOE_ERR_BOUNDS like the forward's;
+ * read it with moe_read_device_error(ws). */
+moe_status moe_backward_workspace_bytes(const moe_dims* dims, size_t* bytes);
+moe_status moe_backward(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                        const uint16_t* w_gate_up, const uint16_t* w_down, const void* fwd_ws,
+                        size_t fwd_ws_bytes, const uint16_t* d_out, float* d_x, float* d_w_router,
+                        float* d_logit_bias, float* d_w_gate_up, float* d_w_down, void* ws,
+                        size_t ws_bytes, void* stream);
+
 /* Expert weights in an MX format (device pointers, 16-byte aligned):
  *   fmt             MOE_WFMT_MXFP8 or MOE_WFMT_MXFP4
  *   gate_up         elements of the packed gate_up rows, [N, 2F, d_model] (SwiGLU: gate rows

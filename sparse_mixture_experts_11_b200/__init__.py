@@ -86,6 +86,9 @@ _SIGS = {
     "moe_forward_mx": (ctypes.c_int, [_DIMS, _P, _P, _P, _MXW, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_router_stats": (ctypes.c_int, [_DIMS, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P,
                                         ctypes.c_size_t, _P]),
+    "moe_backward_workspace_bytes": (ctypes.c_int, [_DIMS, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_backward": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P, _P,
+                                    _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_read_device_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int)]),
     "moe_debug_set_wait_timeout_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -385,3 +388,34 @@ def exported_symbols() -> list:
     with open(hdr) as f:
         text = f.read()
     return sorted(set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+# ----------------------------------------------------------------------------- backward
+def backward_workspace_bytes(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.moe_backward_workspace_bytes(ctypes.byref(dims), ctypes.byref(n)),
+           "moe_backward_workspace_bytes")
+    return int(n.value)
+
+
+def new_backward_workspace(dims: Dims, device=None) -> torch.Tensor:
+    return torch.zeros(backward_workspace_bytes(dims), dtype=torch.uint8, device=device or "cuda")
+
+
+def backward_into(dims: Dims, x, w_router, w_gate_up, w_down, fwd_ws, d_out, d_x, d_w_router,
+                  d_logit_bias, d_w_gate_up, d_w_down, ws, stream=None) -> None:
+    """moe_backward after moe_forward (whose workspace is fwd_ws) on the same inputs."""
+    T, d, N, F = dims.T, dims.d_model, dims.n_experts, dims.d_ff
+    rows = 2 * F if dims.act == ACT_SWIGLU else F
+    _check(_lib.moe_backward(
+        ctypes.byref(dims), _ptr(x, "x", torch.bfloat16, (T, d)),
+        _ptr(w_router, "w_router", torch.float32, (N, d)),
+        _ptr(w_gate_up, "w_gate_up", torch.bfloat16, (N, rows, d)),
+        _ptr(w_down, "w_down", torch.bfloat16, (N, d, F)),
+        _ptr(fwd_ws, "fwd_ws", torch.uint8), _nbytes(fwd_ws),
+        _ptr(d_out, "d_out", torch.bfloat16, (T, d)), _ptr(d_x, "d_x", torch.float32, (T, d)),
+        _ptr(d_w_router, "d_w_router", torch.float32, (N, d)),
+        _ptr(d_logit_bias, "d_logit_bias", torch.float32, (N,), allow_none=True),
+        _ptr(d_w_gate_up, "d_w_gate_up", torch.float32, (N, rows, d)),
+        _ptr(d_w_down, "d_w_down", torch.float32, (N, d, F)),
+        _ptr(ws, "ws", torch.uint8), _nbytes(ws), _stream(stream)), "moe_backward")

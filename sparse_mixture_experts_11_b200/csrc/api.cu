@@ -465,6 +465,100 @@ moe_status moe_forward_layout(const moe_dims* dims, void* ws, size_t ws_bytes,
 }
 
 namespace {
+// Regions of a backward workspace, in order (each rounded up to 256 bytes).
+struct BackwardLayout {
+  size_t sizes[9];
+};
+BackwardLayout backward_layout(const moe_dims* dims) {
+  const int64_t T = dims->T, N = dims->n_experts, d = dims->d_model, F = dims->d_ff,
+                R = max_rows(dims);
+  const int64_t n_gu = dims->act == MOE_ACT_SWIGLU ? 2 * F : F;
+  const int64_t chunk = static_cast<int64_t>(moe::backward_router_chunk(static_cast<int>(T)));
+  const int64_t chunks = T > 0 ? (T + chunk - 1) / chunk : 0;
+  BackwardLayout l{{moe::kStatusBytes, size_t(T * N * 4), size_t(R * d * 2), size_t(R * n_gu * 4),
+                    size_t(R * F * 4), size_t(R * n_gu * 2), size_t(R * F * 2), size_t(R * d * 4),
+                    size_t(chunks * N * d * 4)}};
+  return l;
+}
+}  // namespace
+
+moe_status moe_backward_workspace_bytes(const moe_dims* dims, size_t* bytes) {
+  const moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (bytes == nullptr) return MOE_ERR_INVALID;
+  size_t off = 0;
+  for (size_t s : backward_layout(dims).sizes) off += round_up(s, 256);
+  *bytes = off;
+  return MOE_OK;
+}
+
+moe_status moe_backward(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                        const uint16_t* w_gate_up, const uint16_t* w_down, const void* fwd_ws,
+                        size_t fwd_ws_bytes, const uint16_t* d_out, float* d_x, float* d_w_router,
+                        float* d_logit_bias, float* d_w_gate_up, float* d_w_down, void* ws,
+                        size_t ws_bytes, void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (dims->T == 0) return MOE_OK;
+  if (!x || !w_router || !w_gate_up || !w_down || !fwd_ws || !d_out || !d_x || !d_w_router ||
+      !d_w_gate_up || !d_w_down || !ws)
+    return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w_gate_up) || !aligned16(w_down) ||
+      !aligned16(d_out) || !aligned16(d_x) || !aligned16(d_w_router) || !aligned16(d_w_gate_up) ||
+      !aligned16(d_w_down) || !aligned16(ws) || (d_logit_bias && !aligned16(d_logit_bias)))
+    return MOE_ERR_UNSUPPORTED;
+  size_t need = 0;
+  moe_backward_workspace_bytes(dims, &need);
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE;
+  moe_forward_buffers fb;
+  if ((st = moe_forward_layout(dims, const_cast<void*>(fwd_ws), fwd_ws_bytes, &fb)) != MOE_OK)
+    return st;
+  if ((st = check_device()) != MOE_OK) return st;
+  const BackwardLayout l = backward_layout(dims);
+  char* regions[9];
+  char* p = static_cast<char*>(ws);
+  for (int i = 0; i < 9; ++i) {
+    regions[i] = p;
+    p += round_up(l.sizes[i], 256);
+  }
+  moe::BackwardArgs a{};
+  a.d_out = d_out;
+  a.x = x;
+  a.w_router = w_router;
+  a.w_gate_up = w_gate_up;
+  a.w_down = w_down;
+  a.topk_w = fb.topk_w;
+  a.topk_idx = fb.topk_idx;
+  a.row_of_pair = fb.row_of_pair;
+  a.expert_offset = fb.expert_offset;
+  a.x_perm = fb.x_perm;
+  a.y_perm = fb.y_perm;
+  a.status = reinterpret_cast<int*>(regions[0]);
+  a.d_logits = reinterpret_cast<float*>(regions[1]);
+  a.dy_perm = reinterpret_cast<uint16_t*>(regions[2]);
+  a.pre = reinterpret_cast<float*>(regions[3]);
+  a.dh = reinterpret_cast<float*>(regions[4]);
+  a.d_pre = reinterpret_cast<uint16_t*>(regions[5]);
+  a.h = reinterpret_cast<uint16_t*>(regions[6]);
+  a.dx_rows = reinterpret_cast<float*>(regions[7]);
+  a.router_part = reinterpret_cast<float*>(regions[8]);
+  a.d_x = d_x;
+  a.d_w_router = d_w_router;
+  a.d_logit_bias = d_logit_bias;
+  a.d_w_gate_up = d_w_gate_up;
+  a.d_w_down = d_w_down;
+  a.T = dims->T;
+  a.d = dims->d_model;
+  a.N = dims->n_experts;
+  a.k = dims->top_k;
+  a.F = dims->d_ff;
+  a.act = dims->act;
+  a.r_max = max_rows(dims);
+  a.timeout_ns = moe::wait_timeout_ns();
+  return launch_status(moe::launch_backward(a, as_stream(stream)));
+}
+
+namespace {
 moe_status forward_impl(const moe_dims* dims, const uint16_t* x, const float* w_router,
                         const float* logit_bias, const Weights& w, const uint16_t* residual,
                         uint16_t* out, void* ws, size_t ws_bytes, void* stream) {

@@ -1,0 +1,732 @@
+// Backward pass of the sparse MoE layer on sm_100a.
+//
+// The pages discuss training MoE layers with grouped-GEMM kernels (page «Что такое Mixture of
+// Experts (MoE) в трансформерах», section «Обучение MoE с помощью Transformers») and print no
+// gradient formulas; these kernels compute the chain rule of the forward pass:
+//   out[t] = residual[t] + sum over kept j of w[t, j] y[row(t, j)],   y = h W_d^T,
+//   h = silu(x W_g^T) (x W_u^T) (SwiGLU) or gelu(x W_1^T) (GELU),
+//   w[t] = softmax of the chosen logits, L = x W_r^T (+ b).
+// The choice of experts and the capacity slots pass no gradient. Steps, on one stream:
+//   1 bwd_pairs_kernel      dy[row] = w[t, j] d_out[t] (bf16), dw[t, j] = <d_out[t], y[row]>,
+//                           dL[t, i] = w_i (dw_i - sum_j w_j dw_j) on the chosen experts
+//   2 bwd_gemm (rows)       pre = x_perm W_gu^T                (fp32, recomputed)
+//   3 bwd_gemm (rows)       dh = dy W_d                        (W_d read MN-major)
+//   4 act_bwd_kernel        d_pre = dh * act'(pre) (bf16), h = act(pre) (bf16)
+//   5 bwd_gemm (rows)       dx_rows = d_pre W_gu               (W_gu read MN-major)
+//   6 bwd_gemm (wgrad)      dW_d[e] = dy_e^T h_e               (both operands MN-major)
+//   7 bwd_gemm (wgrad)      dW_gu[e] = d_pre_e^T x_e           (both operands MN-major)
+//   8 router_wgrad kernels  dW_r = dL^T x, db = sum_t dL[t]    (fp32, fixed summation order)
+//   9 bwd_dx_kernel         dx[t] = sum over kept j of dx_rows[row] + sum_j dL[t, idx_j] W_r[idx_j]
+//
+// bwd_gemm_kernel is one 128 x 256 output tile per CTA on tcgen05 (192 threads: TMA producer,
+// MMA issuer, four epilogue warps; four 48 KB stages; fp32 accumulator in TMEM). Each operand
+// is K-major (the contiguous axis is the reduction axis) or MN-major (the contiguous axis is
+// the output's row or column axis), so the transposed products read the weights and the
+// activations where they lie: an MN-major operand comes as 64 x 64 TMA boxes (128 bytes of
+// the MN axis by 64 k rows, 128B-swizzled) and the MMA reads it through an MN-major shared
+// memory descriptor with the instruction's transpose bit set. Rows mode: the tile's rows are
+// an expert's rows of the permuted batch and K is fixed. Weight-gradient mode: the tile is a
+// block of an expert's [M, n_out] gradient and K runs over the expert's rows; the last k block
+// is cut at the expert's end by zeroing the rows past it in shared memory. Every wait is
+// bounded; on timeout the CTA records MOE_ERR_TIMEOUT and drains what it issued.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "launch.h"
+#include "tma_host.h"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;  // UMMA M
+constexpr int kBN = 256;  // UMMA N
+constexpr int kBK = 64;   // k per stage: 64 bf16, one 128-byte swizzle row
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;
+constexpr int kBBytes = kBN * kBK * 2;
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kGemmThreads = 192;
+constexpr int kGemmSmem = kStages * kStageBytes + 1024;
+constexpr int kBox = 64 * 64 * 2;  // one MN-major TMA box: 64 MN x 64 k rows, 8 KB
+
+enum { GEMM_ROWS = 0, GEMM_WGRAD = 1 };
+
+struct BwdGemmParams {
+  const int32_t* expert_offset;  // [N + 1]
+  int n_experts;
+  int M;          // weight-gradient mode: rows of each expert's output block
+  int n_out;      // output columns (a multiple of 16)
+  int num_kb;     // rows mode: K / 64
+  int r_max;      // rows of the permuted batch's buffers
+  float* out;     // rows mode: [r_max, n_out]; weight-gradient mode: [N, M, n_out]
+  int* status;
+  uint64_t timeout_ns;
+};
+
+// Shared-memory descriptor of a 128B-swizzled MN-major operand: 8 k rows of 128 bytes (64 MN
+// elements) form a 1024-byte group (stride-dimension offset); successive 64-element MN blocks
+// are one TMA box (8 KB) apart (leading-dimension offset).
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(kBox >> 4) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+template <bool A_MN, bool B_MN, int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const BwdGemmParams p) {
+  extern __shared__ __align__(1024) uint8_t dyn_smem[];
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ __align__(8) uint64_t tfull_bar;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+  __shared__ int s_tile[4];  // expert (-1: no tile), first row or m0, rows, first row of K
+
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t tiles = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  const int N = p.n_experts;
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    mbar_init(smem_u32(&tfull_bar), 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  pdl_wait();
+  if (warp == 0) {
+    if (lane == 0) s_tile[0] = -1;
+    __syncwarp();
+    if (MODE == GEMM_ROWS) {
+      // m-tile blockIdx.y of the experts' m-tiles in expert order
+      const int per = (N + 31) / 32;
+      int cnt[8], lo[8], hi[8];
+      int sum = 0;
+      bool bad = false;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cnt[i] = 0;
+        lo[i] = hi[i] = 0;
+        const int e = lane * per + i;
+        if (i < per && e < N) {
+          lo[i] = p.expert_offset[e];
+          hi[i] = p.expert_offset[e + 1];
+          if (lo[i] < 0 || hi[i] < lo[i] || hi[i] > p.r_max) bad = true;
+          else cnt[i] = (hi[i] - lo[i] + kBM - 1) / kBM;
+          sum += cnt[i];
+        }
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (__any_sync(0xffffffffu, bad)) {
+        if (lane == 0) report_error(p.status, MOE_ERR_BOUNDS);
+      } else {
+        int run = incl - sum;
+        const int y = static_cast<int>(blockIdx.y);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (cnt[i] > 0 && y >= run && y < run + cnt[i]) {
+            const int m0 = lo[i] + (y - run) * kBM;
+            s_tile[0] = lane * per + i;
+            s_tile[1] = m0;
+            s_tile[2] = min(kBM, hi[i] - m0);
+            s_tile[3] = 0;
+          }
+          run += cnt[i];
+        }
+      }
+    } else if (lane == 0) {
+      const int e = blockIdx.z;
+      const int a = p.expert_offset[e], b = p.expert_offset[e + 1];
+      if (a < 0 || b < a || b > p.r_max) {
+        report_error(p.status, MOE_ERR_BOUNDS);
+      } else {
+        s_tile[0] = e;
+        s_tile[1] = static_cast<int>(blockIdx.y) * kBM;
+        s_tile[2] = b - a;  // K rows
+        s_tile[3] = a;
+      }
+    }
+  }
+  __syncthreads();
+  if (s_tile[0] < 0) return;  // whole CTA: no tile here
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&s_tmem), kBN);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+
+  const int e = s_tile[0], m0 = s_tile[1], rows = s_tile[2], k0 = s_tile[3];
+  const int n0 = static_cast<int>(blockIdx.x) * kBN;
+  const int nkb = MODE == GEMM_ROWS ? p.num_kb : (rows + kBK - 1) / kBK;
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_last();
+      bool ok = true;
+      int kb = 0;
+      for (; kb < nkb; ++kb) {
+        const int s = kb % kStages;
+        if (!mbar_wait(smem_u32(&empty_bar[s]), ((kb / kStages) & 1) ^ 1u, p.timeout_ns, &s_abort)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = smem_u32(&full_bar[s]);
+        const uint32_t a_dst = tiles + s * kStageBytes, b_dst = a_dst + kABytes;
+        mbar_arrive_expect_tx(fb, kStageBytes);
+        if (!A_MN) {
+          tma_load_2d(a_dst, &tmA, fb, kb * kBK, m0, pol);
+        } else {
+#pragma unroll
+          for (int i = 0; i < kBM / 64; ++i)
+            tma_load_2d(a_dst + i * kBox, &tmA, fb, m0 + 64 * i, k0 + kb * kBK, pol);
+        }
+        if (!B_MN) {
+          tma_load_3d(b_dst, &tmB, fb, kb * kBK, n0, e, pol);
+        } else if (MODE == GEMM_ROWS) {
+#pragma unroll
+          for (int i = 0; i < kBN / 64; ++i)
+            tma_load_3d(b_dst + i * kBox, &tmB, fb, n0 + 64 * i, kb * kBK, e, pol);
+        } else {
+#pragma unroll
+          for (int i = 0; i < kBN / 64; ++i)
+            tma_load_2d(b_dst + i * kBox, &tmB, fb, n0 + 64 * i, k0 + kb * kBK, pol);
+        }
+      }
+      if (!ok) {
+        s_abort = 1;
+        report_error(p.status, MOE_ERR_TIMEOUT);
+      }
+      // no TMA write may still be landing in shared memory when the CTA exits
+      for (int i = max(0, kb - kStages); i < kb; ++i)
+        mbar_wait(smem_u32(&full_bar[i % kStages]), (i / kStages) & 1, kDrainTimeoutNs, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN) | (A_MN ? (1u << 15) : 0u) |
+                               (B_MN ? (1u << 16) : 0u);
+    bool ok = true;
+    bool issued = false;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % kStages;
+      const bool got = mbar_wait(smem_u32(&full_bar[s]), (kb / kStages) & 1, p.timeout_ns, &s_abort);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      const uint32_t a_base = tiles + s * kStageBytes, b_base = a_base + kABytes;
+      const int valid = rows - kb * kBK;
+      if (MODE == GEMM_WGRAD && valid < kBK) {
+        // the expert's rows end inside this k block: zero k rows [valid, 64) of every box
+        uint8_t* st = dyn_smem + (a_base - smem_u32(dyn_smem));
+        const int lines = kBK - valid;
+        const int boxes = kBM / 64 + kBN / 64;
+        for (int i = lane; i < boxes * lines * 8; i += 32) {
+          const int box = i / (lines * 8), rem = i - box * lines * 8;
+          const int line = valid + rem / 8, chunk = rem & 7;
+          const uint32_t off = (box < kBM / 64 ? box * kBox : kABytes + (box - kBM / 64) * kBox) +
+                               line * 128 + chunk * 16;
+          *reinterpret_cast<uint4*>(st + off) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();  // generic stores -> visible to the tensor core
+        __syncwarp();
+      }
+      tc_fence_after_sync();
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t da = A_MN ? smem_desc_mn_sw128(a_base + kk * 2048)
+                                   : smem_desc_k_sw128(a_base + kk * 32);
+          const uint64_t db = B_MN ? smem_desc_mn_sw128(b_base + kk * 2048)
+                                   : smem_desc_k_sw128(b_base + kk * 32);
+          tc_mma_f16(tmem, da, db, idesc, (kb != 0 || kk != 0) ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&empty_bar[s]));
+      }
+      issued = true;
+      __syncwarp();
+    }
+    if (lane == 0) {
+      if (ok && nkb > 0) {
+        tc_commit(smem_u32(&tfull_bar));
+      } else if (!ok) {
+        s_abort = 1;
+        report_error(p.status, MOE_ERR_TIMEOUT);
+        if (issued) {  // let every issued MMA finish before TMEM is freed
+          tc_commit(smem_u32(&tfull_bar));
+          mbar_wait(smem_u32(&tfull_bar), 0, kDrainTimeoutNs, nullptr);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quadrant of this warp
+    const int r_local = q * 32 + lane;
+    bool have = nkb > 0;
+    if (have) {
+      const bool got = mbar_wait(smem_u32(&tfull_bar), 0, p.timeout_ns, &s_abort);
+      if (!__all_sync(0xffffffffu, got)) {
+        s_abort = 1;
+        report_error(p.status, MOE_ERR_TIMEOUT);
+        have = false;
+      } else {
+        tc_fence_after_sync();
+      }
+    }
+    if (have || nkb == 0) {
+      bool row_ok;
+      float* dst;
+      if (MODE == GEMM_ROWS) {
+        row_ok = r_local < rows;
+        dst = p.out + (static_cast<int64_t>(m0) + r_local) * p.n_out;
+      } else {
+        row_ok = m0 + r_local < p.M;
+        dst = p.out + (static_cast<int64_t>(e) * p.M + m0 + r_local) * p.n_out;
+      }
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int cc = 0; cc < kBN; cc += 16) {
+        if (n0 + cc >= p.n_out) break;  // warp-uniform: ragged last n-tile
+        uint32_t v[16];
+        if (have) {
+          tmem_ld_32x32b_x16(t_row + cc, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = 0u;  // an expert with no rows: zero gradient
+        }
+        if (!row_ok) continue;
+        float4* d4 = reinterpret_cast<float4*>(dst + n0 + cc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                              __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kBN);
+  }
+}
+
+// ------------------------------------------------------------------ combine and router step
+// Warp per token. For each kept choice j: dy[row] = bf16(w_j d_out[t]) and
+// dw_j = <d_out[t], y[row]> (fp32); dropped choices have dw_j = 0. Then the renormalised
+// softmax's gradient on the chosen logits, dL_i = w_i (dw_i - sum_j w_j dw_j); the row of dL
+// is written whole (zeros on the other experts).
+__global__ void __launch_bounds__(256) bwd_pairs_kernel(
+    const uint16_t* __restrict__ d_out, const float* __restrict__ y_perm,
+    const float* __restrict__ topk_w, const int32_t* __restrict__ topk_idx,
+    const int32_t* __restrict__ row_of_pair, uint16_t* __restrict__ dy_perm,
+    float* __restrict__ d_logits, int T, int d, int N, int k, int r_max, int* status) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = static_cast<int>(lane_id());
+  const int warps = gridDim.x * (blockDim.x / 32);
+  for (int t = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; t < T; t += warps) {
+    int row[8], idx[8];
+    float w[8], acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      row[j] = -1;
+      idx[j] = -1;
+      w[j] = 0.f;
+      acc[j] = 0.f;
+      if (j < k) {
+        row[j] = row_of_pair[t * k + j];
+        idx[j] = topk_idx[t * k + j];
+        w[j] = topk_w[t * k + j];
+        if (row[j] >= r_max) {
+          if (lane == 0) report_error(status, MOE_ERR_BOUNDS);
+          row[j] = -1;
+        }
+      }
+    }
+    for (int c = lane * 8; c < d; c += 256) {
+      const uint4 g4 = *reinterpret_cast<const uint4*>(d_out + static_cast<int64_t>(t) * d + c);
+      const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+      float g[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        g[2 * i] = __uint_as_float(gw[i] << 16);
+        g[2 * i + 1] = __uint_as_float(gw[i] & 0xffff0000u);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (row[j] < 0) continue;
+        const float4* yr = reinterpret_cast<const float4*>(y_perm + static_cast<int64_t>(row[j]) * d + c);
+        const float4 y0 = yr[0], y1 = yr[1];
+        acc[j] += g[0] * y0.x + g[1] * y0.y + g[2] * y0.z + g[3] * y0.w + g[4] * y1.x +
+                  g[5] * y1.y + g[6] * y1.z + g[7] * y1.w;
+        uint4 o;
+        o.x = pack_bf16x2(w[j] * g[0], w[j] * g[1]);
+        o.y = pack_bf16x2(w[j] * g[2], w[j] * g[3]);
+        o.z = pack_bf16x2(w[j] * g[4], w[j] * g[5]);
+        o.w = pack_bf16x2(w[j] * g[6], w[j] * g[7]);
+        *reinterpret_cast<uint4*>(dy_perm + static_cast<int64_t>(row[j]) * d + c) = o;
+      }
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+      s += w[j] * acc[j];  // w[j] = 0 past k
+    }
+    for (int n = lane; n < N; n += 32) {
+      float v = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (idx[j] == n) v = w[j] * (acc[j] - s);
+      d_logits[static_cast<int64_t>(t) * N + n] = v;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ activation backward
+// Row r of the permuted batch (r < R = expert_offset[N]), 4 columns per thread:
+//   SwiGLU  pre = [g | u]: h = silu(g) u, d_pre = [dh u silu'(g) | dh silu(g)],
+//           silu'(g) = s (1 + g (1 - s)), s = 1 / (1 + exp(-g));
+//   GELU    h = z Phi(z), d_pre = dh (Phi(z) + z phi(z)) (exact erf form).
+// h and d_pre are rounded once to bf16 (operands of the weight-gradient GEMMs).
+__global__ void __launch_bounds__(256) act_bwd_kernel(const float* __restrict__ pre,
+                                                      const float* __restrict__ dh,
+                                                      const int32_t* __restrict__ expert_offset,
+                                                      uint16_t* __restrict__ d_pre,
+                                                      uint16_t* __restrict__ h, int N, int F,
+                                                      int swiglu) {
+  pdl_wait();
+  pdl_trigger();
+  const int R = expert_offset[N];
+  const int n_gu = swiglu ? 2 * F : F;
+  const int64_t items = static_cast<int64_t>(R) * (F / 4);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < items;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / (F / 4);
+    const int c = static_cast<int>(i - r * (F / 4)) * 4;
+    const float4 d4 = *reinterpret_cast<const float4*>(dh + r * F + c);
+    const float4 z4 = *reinterpret_cast<const float4*>(pre + r * n_gu + c);
+    const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+    const float zv[4] = {z4.x, z4.y, z4.z, z4.w};
+    float hv[4], da[4], du[4];
+    if (swiglu) {
+      const float4 u4 = *reinterpret_cast<const float4*>(pre + r * n_gu + F + c);
+      const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float sg = 1.0f / (1.0f + expf(-zv[q]));
+        const float sl = zv[q] * sg;
+        hv[q] = sl * uv[q];
+        da[q] = dv[q] * uv[q] * (sg * (1.0f + zv[q] * (1.0f - sg)));
+        du[q] = dv[q] * sl;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float Phi = 0.5f * (1.0f + erff(zv[q] * 0.7071067811865476f));
+        const float phi = expf(-0.5f * zv[q] * zv[q]) * 0.3989422804014327f;
+        hv[q] = zv[q] * Phi;
+        da[q] = dv[q] * (Phi + zv[q] * phi);
+        du[q] = 0.f;
+      }
+    }
+    *reinterpret_cast<uint2*>(h + r * F + c) = make_uint2(pack_bf16x2(hv[0], hv[1]), pack_bf16x2(hv[2], hv[3]));
+    *reinterpret_cast<uint2*>(d_pre + r * n_gu + c) =
+        make_uint2(pack_bf16x2(da[0], da[1]), pack_bf16x2(da[2], da[3]));
+    if (swiglu)
+      *reinterpret_cast<uint2*>(d_pre + r * n_gu + F + c) =
+          make_uint2(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]));
+  }
+}
+
+// ------------------------------------------------------------------ router weight gradient
+// dW_r = dL^T x in fp32, in two passes with a fixed summation order: chunk c of the tokens
+// adds its tokens in order into part[c][n][col] (thread = column, 16 experts a block), then
+// the chunks are added in order. db[n] = sum_t dL[t, n]: warp w of a block adds tokens
+// t = w mod 32 in order for 32 experts, and the 32 warp sums are added in warp order.
+constexpr int kRwExperts = 16;
+constexpr int kRwTokens = 64;
+
+__global__ void __launch_bounds__(256) router_wgrad_partial_kernel(
+    const float* __restrict__ d_logits, const uint16_t* __restrict__ x, float* __restrict__ part,
+    int T, int d, int N, int chunk) {
+  __shared__ float s_dl[kRwTokens][kRwExperts];
+  pdl_wait();
+  pdl_trigger();
+  const int col = blockIdx.x * 256 + threadIdx.x;
+  const int n0 = blockIdx.y * kRwExperts;
+  const int t0 = blockIdx.z * chunk, t1 = min(T, t0 + chunk);
+  float acc[kRwExperts];
+#pragma unroll
+  for (int i = 0; i < kRwExperts; ++i) acc[i] = 0.f;
+  for (int tb = t0; tb < t1; tb += kRwTokens) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < kRwTokens * kRwExperts; i += 256) {
+      const int tt = tb + i / kRwExperts, n = n0 + i % kRwExperts;
+      s_dl[i / kRwExperts][i % kRwExperts] =
+          (tt < t1 && n < N) ? d_logits[static_cast<int64_t>(tt) * N + n] : 0.f;
+    }
+    __syncthreads();
+    if (col < d) {
+      const int nt = min(kRwTokens, t1 - tb);
+      for (int tt = 0; tt < nt; ++tt) {
+        const float xv = bf16_bits_to_float(x[static_cast<int64_t>(tb + tt) * d + col]);
+#pragma unroll
+        for (int i = 0; i < kRwExperts; ++i) acc[i] += s_dl[tt][i] * xv;
+      }
+    }
+  }
+  if (col < d) {
+#pragma unroll
+    for (int i = 0; i < kRwExperts; ++i)
+      if (n0 + i < N)
+        part[(static_cast<int64_t>(blockIdx.z) * N + n0 + i) * d + col] = acc[i];
+  }
+}
+
+__global__ void __launch_bounds__(256) router_wgrad_final_kernel(const float* __restrict__ part,
+                                                                 float* __restrict__ d_w_router,
+                                                                 int d, int N, int chunks) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t items = static_cast<int64_t>(N) * d;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < items;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = 0.f;
+    for (int c = 0; c < chunks; ++c) s += part[c * items + i];
+    d_w_router[i] = s;
+  }
+}
+
+__global__ void __launch_bounds__(1024) router_bias_grad_kernel(const float* __restrict__ d_logits,
+                                                                float* __restrict__ d_bias, int T,
+                                                                int N) {
+  __shared__ float s_sum[32][33];
+  pdl_wait();
+  pdl_trigger();
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * 32 + lane;
+  float acc = 0.f;
+  if (n < N)
+    for (int t = w; t < T; t += 32) acc += d_logits[static_cast<int64_t>(t) * N + n];
+  s_sum[w][lane] = acc;
+  __syncthreads();
+  if (w == 0 && n < N) {
+    float s = 0.f;
+    for (int i = 0; i < 32; ++i) s += s_sum[i][lane];
+    d_bias[n] = s;
+  }
+}
+
+// ------------------------------------------------------------------ back to token order
+// dx[t] = sum over kept j (in choice order) of dx_rows[row(t, j)] + sum over j of
+// dL[t, idx_j] W_r[idx_j] (dL is zero on the experts not chosen). Block per (token, 1024
+// columns; tokens strided over grid.y), 4 columns a thread.
+__global__ void __launch_bounds__(256) bwd_dx_kernel(
+    const float* __restrict__ dx_rows, const int32_t* __restrict__ row_of_pair,
+    const int32_t* __restrict__ topk_idx, const float* __restrict__ d_logits,
+    const float* __restrict__ w_router, float* __restrict__ dx, int T, int d, int N, int k,
+    int r_max) {
+  pdl_wait();
+  pdl_trigger();
+  const int c = (blockIdx.x * 256 + threadIdx.x) * 4;
+  if (c >= d) return;
+  for (int t = blockIdx.y; t < T; t += gridDim.y) {
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < k; ++j) {
+    const int r = row_of_pair[t * k + j];
+    if (r < 0 || r >= r_max) continue;
+    const float4 v = *reinterpret_cast<const float4*>(dx_rows + static_cast<int64_t>(r) * d + c);
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  for (int j = 0; j < k; ++j) {
+    const int e = topk_idx[t * k + j];
+    if (e < 0 || e >= N) continue;
+    const float g = d_logits[static_cast<int64_t>(t) * N + e];
+    const float4 wr = *reinterpret_cast<const float4*>(w_router + static_cast<int64_t>(e) * d + c);
+    acc.x += g * wr.x;
+    acc.y += g * wr.y;
+    acc.z += g * wr.z;
+    acc.w += g * wr.w;
+  }
+  *reinterpret_cast<float4*>(dx + static_cast<int64_t>(t) * d + c) = acc;
+  }
+}
+
+// ------------------------------------------------------------------ host side
+template <bool A_MN, bool B_MN, int MODE>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const BwdGemmParams& p,
+                        dim3 grid, cudaStream_t s) {
+  auto kern = bwd_gemm_kernel<A_MN, B_MN, MODE>;
+  static cudaError_t attr =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  if (attr != cudaSuccess) return attr;
+  return launch_pdl(kern, grid, dim3(kGemmThreads), kGemmSmem, s, a, b, p);
+}
+
+// K-major operand [outer][K] bf16: boxes of 64 k x `rows`.
+bool map_k_major_2d(CUtensorMap* m, const void* base, uint64_t K, uint64_t outer, uint32_t rows) {
+  const uint64_t dims[2] = {K, outer};
+  const uint64_t str[1] = {K * 2};
+  const uint32_t box[2] = {static_cast<uint32_t>(kBK), rows};
+  return make_map(m, base, 2, dims, str, box);
+}
+// MN-major operand [K rows][MN] bf16 (2-D): boxes of 64 MN x 64 k.
+bool map_mn_major_2d(CUtensorMap* m, const void* base, uint64_t MN, uint64_t krows) {
+  const uint64_t dims[2] = {MN, krows};
+  const uint64_t str[1] = {MN * 2};
+  const uint32_t box[2] = {64, static_cast<uint32_t>(kBK)};
+  return make_map(m, base, 2, dims, str, box);
+}
+
+}  // namespace
+
+size_t backward_router_chunk(int T) { return static_cast<size_t>(std::max(256, (T + 15) / 16)); }
+
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {
+  const int T = a.T, d = a.d, N = a.N, k = a.k, F = a.F;
+  const bool swiglu = a.act == MOE_ACT_SWIGLU;
+  const int n_gu = swiglu ? 2 * F : F;
+  const uint64_t R = static_cast<uint64_t>(a.r_max);
+  cudaError_t e;
+  // 1: dy, dL
+  {
+    const int blocks = std::max(1, std::min((T + 7) / 8, 8 * 148));
+    e = launch_pdl(bwd_pairs_kernel, dim3(blocks), dim3(256), 0, s, a.d_out, a.y_perm, a.topk_w,
+                   a.topk_idx, a.row_of_pair, a.dy_perm, a.d_logits, T, d, N, k,
+                   static_cast<int>(a.r_max), a.status);
+    if (e != cudaSuccess) return e;
+  }
+  if (R > 0) {
+    BwdGemmParams p{};
+    p.expert_offset = a.expert_offset;
+    p.n_experts = N;
+    p.r_max = static_cast<int>(a.r_max);
+    p.status = a.status;
+    p.timeout_ns = a.timeout_ns;
+    const unsigned m_tiles = static_cast<unsigned>((R + kBM - 1) / kBM + N);
+    CUtensorMap mA, mB;
+    // 2: pre = x_perm W_gu^T
+    if (!map_k_major_2d(&mA, a.x_perm, d, R, kBM)) return cudaErrorInvalidValue;
+    {
+      const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_gu), static_cast<uint64_t>(N)};
+      const uint64_t str[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(n_gu) * d * 2};
+      const uint32_t box[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBN), 1};
+      if (!make_map(&mB, a.w_gate_up, 3, dims, str, box)) return cudaErrorInvalidValue;
+    }
+    p.n_out = n_gu;
+    p.num_kb = d / kBK;
+    p.out = a.pre;
+    e = launch_gemm<false, false, GEMM_ROWS>(mA, mB, p, dim3((n_gu + kBN - 1) / kBN, m_tiles), s);
+    if (e != cudaSuccess) return e;
+    // 3: dh = dy W_d (W_d [N][d][F] read MN-major: F is the output axis)
+    if (!map_k_major_2d(&mA, a.dy_perm, d, R, kBM)) return cudaErrorInvalidValue;
+    {
+      const uint64_t dims[3] = {static_cast<uint64_t>(F), static_cast<uint64_t>(d), static_cast<uint64_t>(N)};
+      const uint64_t str[2] = {static_cast<uint64_t>(F) * 2, static_cast<uint64_t>(d) * F * 2};
+      const uint32_t box[3] = {64, static_cast<uint32_t>(kBK), 1};
+      if (!make_map(&mB, a.w_down, 3, dims, str, box)) return cudaErrorInvalidValue;
+    }
+    p.n_out = F;
+    p.num_kb = d / kBK;
+    p.out = a.dh;
+    e = launch_gemm<false, true, GEMM_ROWS>(mA, mB, p, dim3((F + kBN - 1) / kBN, m_tiles), s);
+    if (e != cudaSuccess) return e;
+    // 4: d_pre, h
+    {
+      const int64_t items = static_cast<int64_t>(R) * (F / 4);
+      const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((items + 255) / 256, 16 * 148)));
+      e = launch_pdl(act_bwd_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const float*>(a.pre),
+                     static_cast<const float*>(a.dh), a.expert_offset, a.d_pre, a.h, N, F,
+                     swiglu ? 1 : 0);
+      if (e != cudaSuccess) return e;
+    }
+    // 5: dx_rows = d_pre W_gu (W_gu [N][n_gu][d] read MN-major: d is the output axis)
+    if (!map_k_major_2d(&mA, a.d_pre, n_gu, R, kBM)) return cudaErrorInvalidValue;
+    {
+      const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_gu), static_cast<uint64_t>(N)};
+      const uint64_t str[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(n_gu) * d * 2};
+      const uint32_t box[3] = {64, static_cast<uint32_t>(kBK), 1};
+      if (!make_map(&mB, a.w_gate_up, 3, dims, str, box)) return cudaErrorInvalidValue;
+    }
+    p.n_out = d;
+    p.num_kb = n_gu / kBK;
+    p.out = a.dx_rows;
+    e = launch_gemm<false, true, GEMM_ROWS>(mA, mB, p, dim3((d + kBN - 1) / kBN, m_tiles), s);
+    if (e != cudaSuccess) return e;
+    // 6: dW_d[e] = dy_e^T h_e  ([d, F] per expert)
+    if (!map_mn_major_2d(&mA, a.dy_perm, d, R)) return cudaErrorInvalidValue;
+    if (!map_mn_major_2d(&mB, a.h, F, R)) return cudaErrorInvalidValue;
+    p.M = d;
+    p.n_out = F;
+    p.out = a.d_w_down;
+    e = launch_gemm<true, true, GEMM_WGRAD>(mA, mB, p, dim3((F + kBN - 1) / kBN, (d + kBM - 1) / kBM, N), s);
+    if (e != cudaSuccess) return e;
+    // 7: dW_gu[e] = d_pre_e^T x_e  ([n_gu, d] per expert)
+    if (!map_mn_major_2d(&mA, a.d_pre, n_gu, R)) return cudaErrorInvalidValue;
+    if (!map_mn_major_2d(&mB, a.x_perm, d, R)) return cudaErrorInvalidValue;
+    p.M = n_gu;
+    p.n_out = d;
+    p.out = a.d_w_gate_up;
+    e = launch_gemm<true, true, GEMM_WGRAD>(mA, mB, p, dim3((d + kBN - 1) / kBN, (n_gu + kBM - 1) / kBM, N), s);
+    if (e != cudaSuccess) return e;
+  } else {
+    // no kept rows: the experts' gradients are zero
+    e = cudaMemsetAsync(a.d_w_gate_up, 0, static_cast<size_t>(N) * n_gu * d * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a.d_w_down, 0, static_cast<size_t>(N) * d * F * 4, s);
+    if (e != cudaSuccess) return e;
+  }
+  // 8: router weight (and bias) gradient
+  {
+    const int chunk = static_cast<int>(backward_router_chunk(T));
+    const int chunks = (T + chunk - 1) / chunk;
+    e = launch_pdl(router_wgrad_partial_kernel,
+                   dim3((d + 255) / 256, (N + kRwExperts - 1) / kRwExperts, chunks), dim3(256), 0, s,
+                   static_cast<const float*>(a.d_logits), a.x, a.router_part, T, d, N, chunk);
+    if (e != cudaSuccess) return e;
+    const int64_t items = static_cast<int64_t>(N) * d;
+    const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((items + 255) / 256, 8 * 148)));
+    e = launch_pdl(router_wgrad_final_kernel, dim3(blocks), dim3(256), 0, s,
+                   static_cast<const float*>(a.router_part), a.d_w_router, d, N, chunks);
+    if (e != cudaSuccess) return e;
+    if (a.d_logit_bias != nullptr) {
+      e = launch_pdl(router_bias_grad_kernel, dim3((N + 31) / 32), dim3(1024), 0, s,
+                     static_cast<const float*>(a.d_logits), a.d_logit_bias, T, N);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  // 9: dx
+  return launch_pdl(bwd_dx_kernel, dim3((d + 1023) / 1024, std::min(T, 65535)), dim3(256), 0, s,
+                    static_cast<const float*>(a.dx_rows), a.row_of_pair, a.topk_idx,
+                    static_cast<const float*>(a.d_logits), a.w_router, a.d_x, T, d, N, k,
+                    static_cast<int>(a.r_max));
+}
+
+}  // namespace moe

@@ -196,4 +196,40 @@ struct GroupedFfnArgs {
 };
 cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s);
 
+// Backward pass (backward.cu). Saved from the forward: the routing, x_perm and y_perm.
+struct BackwardArgs {
+  const uint16_t* d_out;          // [T, d] bf16
+  const uint16_t* x;              // [T, d] bf16
+  const float* w_router;          // [N, d]
+  const uint16_t* w_gate_up;      // [N, n_gu, d]
+  const uint16_t* w_down;         // [N, d, F]
+  const float* topk_w;            // [T, k]
+  const int32_t* topk_idx;        // [T, k]
+  const int32_t* row_of_pair;     // [T, k]
+  const int32_t* expert_offset;   // [N + 1]
+  const uint16_t* x_perm;         // [r_max, d]
+  const float* y_perm;            // [r_max, d]
+  // workspace
+  float* d_logits;                // [T, N]
+  uint16_t* dy_perm;              // [r_max, d]
+  float* pre;                     // [r_max, n_gu]
+  float* dh;                      // [r_max, F]
+  uint16_t* d_pre;                // [r_max, n_gu]
+  uint16_t* h;                    // [r_max, F]
+  float* dx_rows;                 // [r_max, d]
+  float* router_part;             // [chunks, N, d], chunks = ceil(T / backward_router_chunk(T))
+  // outputs
+  float* d_x;                     // [T, d]
+  float* d_w_router;              // [N, d]
+  float* d_logit_bias;            // [N] or null
+  float* d_w_gate_up;             // [N, n_gu, d]
+  float* d_w_down;                // [N, d, F]
+  int T, d, N, k, F, act;
+  int64_t r_max;
+  int* status;
+  uint64_t timeout_ns;
+};
+size_t backward_router_chunk(int T);
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s);
+
 }  // namespace moe

@@ -68,6 +68,7 @@ SHAPES = {
 # tensor ids for per-tensor generator streams
 _X, _WR, _WGU, _WD = 1, 2, 3, 4
 _WGU_Q, _WGU_S, _WD_Q, _WD_S = 5, 6, 7, 8
+_DOUT = 9
 
 
 def _gen(device: torch.device, seed: int, tensor_id: int, sub: int = 0) -> torch.Generator:
@@ -97,6 +98,11 @@ def zipf_logit_bias(n_experts: int, s: float) -> torch.Tensor:
 def make_hidden(T: int, d_model: int, *, seed: int = 0, device="cpu") -> torch.Tensor:
     """x ~ N(0,1) rounded to bf16, shape [T, d_model]."""
     return _normal((T, d_model), 1.0, torch.device(device), seed, _X).to(torch.bfloat16)
+
+
+def make_grad_output(T: int, d_model: int, *, seed: int = 0, device="cpu") -> torch.Tensor:
+    """Gradient of the layer output for the backward pass: N(0,1) rounded to bf16, [T, d_model]."""
+    return _normal((T, d_model), 1.0, torch.device(device), seed, _DOUT).to(torch.bfloat16)
 
 
 def make_layer_weights(shape: LayerShape, *, seed: int = 0, device="cpu",
