@@ -299,6 +299,63 @@ class Layer:
                 "dropped_pairs": int(dropped.item()), "algorithmic_bytes": nbytes,
                 "achieved_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
 
+    def backward_timing(self, steps: int, flush, peaks: dict) -> dict:
+        """moe_backward after this layer's forward (bf16 weights): mean ms per call of the
+        captured backward between events, with L2 flushed before each call. FLOPs are the five
+        expert GEMMs (pre recomputed, dh, dx_rows, dW_d, dW_gu); algorithmic bytes are the
+        expert weights read once, the fp32 weight gradients written, the saved rows read
+        (x_perm, y_perm), d_out and x read, dx and the router's gradient written."""
+        moe, i, s = self.moe, self.inp, self.shape
+        T, d, N, F = self.T, s.d_model, s.n_experts, s.d_ff
+        dev = i["x"].device
+        n_gu = 2 * F if s.act == "swiglu" else F
+        g = synthetic.make_grad_output(T, d, seed=1, device=dev)
+        out = {"dx": torch.empty((T, d), dtype=torch.float32, device=dev),
+               "d_w_router": torch.empty((N, d), dtype=torch.float32, device=dev),
+               "d_logit_bias": torch.empty((N,), dtype=torch.float32, device=dev),
+               "d_w_gate_up": torch.empty((N, n_gu, d), dtype=torch.float32, device=dev),
+               "d_w_down": torch.empty((N, d, F), dtype=torch.float32, device=dev)}
+        bws = moe.new_backward_workspace(self.dims, dev)
+
+        def call():
+            moe.backward_into(self.dims, i["x"], i["w_router"], i["w_gate_up"], i["w_down"],
+                              self.fws, g, out["dx"], out["d_w_router"], out["d_logit_bias"],
+                              out["d_w_gate_up"], out["d_w_down"], bws)
+        self.forward_call()
+        call()
+        torch.cuda.synchronize()
+        err = moe.read_device_error(bws)
+        if err != 0:
+            raise RuntimeError(f"backward device status: {moe.status_string(err)}")
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            call()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for e0, e1 in evs:
+            flush_l2(flush)
+            e0.record()
+            gr.replay()
+            e1.record()
+        torch.cuda.synchronize()
+        ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+        counts = self.views()["expert_count"].cpu()
+        R, active = int(counts.sum()), int((counts > 0).sum())
+        flops = 6 * R * d * n_gu + 4 * R * d * F
+        per_expert = n_gu * d + d * F
+        nbytes = (active * per_expert * 2 + N * per_expert * 4 + R * d * (2 + 4)
+                  + T * d * (2 + 2 + 4) + N * d * 4)
+        tensor = flops / nbytes > (peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9)
+        if tensor:
+            ach, peak, unit = flops / (ms * 1e-3) / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+        else:
+            ach, peak, unit = nbytes / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        return {"ms": round(ms, 4), "tokens_per_s": round(T / (ms * 1e-3), 1),
+                "flops": flops, "algorithmic_bytes": nbytes,
+                "bound": "tensor" if tensor else "hbm", "achieved": round(ach, 1), "peak": peak,
+                "unit": unit, "frac": round(ach / peak, 4),
+                "launches": 11 if R > 0 else 5}
+
     def redirect_timing(self, steps: int, flush) -> dict:
         """moe_redirect_overflow (overflow policy "redirect") on the step's logits and top-k,
         into separate buffers: mean ms per call of a graph that restores the router's top-k
@@ -543,6 +600,8 @@ def run_gpu(args, rank, world, local_rank):
     # router statistics and the auxiliary loss over this step's routing (a "next" row),
     # replayed as a graph K times between events
     stats = layer.stats_timing(args.steps, flush)
+    # backward pass after this forward (a "next" row); bf16 expert weights only
+    backward = layer.backward_timing(args.steps, flush, load_peaks()) if args.wfmt == "bf16" else None
     # overflow policy "redirect" on the same routing (a "next" row), where the batch allows it
     redirect = (layer.redirect_timing(args.steps, flush)
                 if T * shape.top_k <= moe.REDIRECT_MAX_PAIRS else None)
@@ -601,6 +660,7 @@ def run_gpu(args, rank, world, local_rank):
         "stages_ms": {k: round(v_, 4) for k, v_ in stage_ms.items()},
         "router_stats": stats,
         "overflow_redirect": redirect,
+        "backward": backward,
         "roofline": roof,
         "layer_gbs": round(ab["layer"] / (total_ms / args.steps * 1e-3) / 1e9, 1),
         "ffn_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 2),
