@@ -18,8 +18,10 @@
 //   8 router_wgrad kernels  dW_r = dL^T x, db = sum_t dL[t]    (fp32, fixed summation order)
 //   9 bwd_dx_kernel         dx[t] = sum over kept j of dx_rows[row] + sum_j dL[t, idx_j] W_r[idx_j]
 //
-// bwd_gemm_kernel is one 128 x 256 output tile per CTA on tcgen05 (192 threads: TMA producer,
-// MMA issuer, four epilogue warps; four 48 KB stages; fp32 accumulator in TMEM). Each operand
+// bwd_gemm_kernel is persistent, one CTA per SM striding through 128 x 256 output tiles on
+// tcgen05 (192 threads: TMA producer, MMA issuer, four epilogue warps; four 48 KB stages;
+// two fp32 accumulators in TMEM, so one tile's epilogue overlaps the next one's loads and
+// MMAs). Each operand
 // is K-major (the contiguous axis is the reduction axis) or MN-major (the contiguous axis is
 // the output's row or column axis), so the transposed products read the weights and the
 // activations where they lie: an MN-major operand comes as 64 x 64 TMA boxes (128 bytes of
@@ -79,6 +81,49 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t smem_addr) {
   return d;
 }
 
+struct GemmTile {
+  int e;     // expert
+  int m0;    // rows mode: first row of the permuted batch; weight-gradient mode: first output row
+  int rows;  // rows mode: valid rows of the tile; weight-gradient mode: the expert's rows (K)
+  int k0;    // weight-gradient mode: the expert's first row (start of K)
+  int n0;    // first output column
+  int nkb;   // k blocks
+};
+
+// Tile t of the CTA-strided list. Rows mode: t = m-tile * n_tiles_n + n-tile, m-tiles numbered
+// expert by expert (s_mt: each expert's first m-tile, s_off: its first row). Weight-gradient
+// mode: t = (expert * m_tiles + m-tile) * n_tiles_n + n-tile.
+template <int MODE>
+__device__ __forceinline__ GemmTile decode_gemm_tile(int t, const BwdGemmParams& p, int n_tiles_n,
+                                                     int m_tiles, const int* s_mt,
+                                                     const int* s_off) {
+  GemmTile c;
+  const int nt = t % n_tiles_n;
+  c.n0 = nt * kBN;
+  if (MODE == GEMM_ROWS) {
+    const int gm = t / n_tiles_n;
+    int lo = 0, hi = p.n_experts;  // last e with s_mt[e] <= gm
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_mt[mid] <= gm) lo = mid;
+      else hi = mid;
+    }
+    c.e = lo;
+    c.m0 = s_off[lo] + (gm - s_mt[lo]) * kBM;
+    c.rows = min(kBM, s_off[lo + 1] - c.m0);
+    c.k0 = 0;
+    c.nkb = p.num_kb;
+  } else {
+    const int em = t / n_tiles_n;
+    c.e = em / m_tiles;
+    c.m0 = (em - c.e * m_tiles) * kBM;
+    c.k0 = s_off[c.e];
+    c.rows = s_off[c.e + 1] - c.k0;
+    c.nkb = (c.rows + kBK - 1) / kBK;
+  }
+  return c;
+}
+
 template <bool A_MN, bool B_MN, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -86,10 +131,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
-  __shared__ __align__(8) uint64_t tfull_bar;
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t done_bar;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
-  __shared__ int s_tile[4];  // expert (-1: no tile), first row or m0, rows, first row of K
+  __shared__ int s_mt[257];  // rows mode: first m-tile of each expert; s_mt[N] = all m-tiles
+  __shared__ int s_off[257];
+  __shared__ int s_tiles;
+  __shared__ float s_stage[4][32][33];  // epilogue: one 32 x 32 fp32 block per warp
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,82 +152,67 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
-    mbar_init(smem_u32(&tfull_bar), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&tfull_bar[b]), 1);
+      mbar_init(smem_u32(&tempty_bar[b]), kGemmThreads - 64);
+    }
+    mbar_init(smem_u32(&done_bar), 1);
     s_abort = 0;
     fence_barrier_init();
   }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&s_tmem), 2 * kBN);
+    tmem_relinquish();
+  }
   pdl_wait();
+  const int n_tiles_n = (p.n_out + kBN - 1) / kBN;
+  const int m_tiles = (p.M + kBM - 1) / kBM;  // weight-gradient mode
   if (warp == 0) {
-    if (lane == 0) s_tile[0] = -1;
-    __syncwarp();
-    if (MODE == GEMM_ROWS) {
-      // m-tile blockIdx.y of the experts' m-tiles in expert order
-      const int per = (N + 31) / 32;
-      int cnt[8], lo[8], hi[8];
-      int sum = 0;
-      bool bad = false;
+    // per-expert offsets (and, rows mode, m-tile counts and their prefix); experts
+    // lane * per .. lane * per + per - 1 on this lane
+    const int per = (N + 31) / 32;
+    int cnt[8];
+    int sum = 0;
+    bool bad = false;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        cnt[i] = 0;
-        lo[i] = hi[i] = 0;
-        const int e = lane * per + i;
-        if (i < per && e < N) {
-          lo[i] = p.expert_offset[e];
-          hi[i] = p.expert_offset[e + 1];
-          if (lo[i] < 0 || hi[i] < lo[i] || hi[i] > p.r_max) bad = true;
-          else cnt[i] = (hi[i] - lo[i] + kBM - 1) / kBM;
-          sum += cnt[i];
-        }
-      }
-      int incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-      }
-      if (__any_sync(0xffffffffu, bad)) {
-        if (lane == 0) report_error(p.status, MOE_ERR_BOUNDS);
-      } else {
-        int run = incl - sum;
-        const int y = static_cast<int>(blockIdx.y);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (cnt[i] > 0 && y >= run && y < run + cnt[i]) {
-            const int m0 = lo[i] + (y - run) * kBM;
-            s_tile[0] = lane * per + i;
-            s_tile[1] = m0;
-            s_tile[2] = min(kBM, hi[i] - m0);
-            s_tile[3] = 0;
-          }
-          run += cnt[i];
-        }
-      }
-    } else if (lane == 0) {
-      const int e = blockIdx.z;
-      const int a = p.expert_offset[e], b = p.expert_offset[e + 1];
-      if (a < 0 || b < a || b > p.r_max) {
-        report_error(p.status, MOE_ERR_BOUNDS);
-      } else {
-        s_tile[0] = e;
-        s_tile[1] = static_cast<int>(blockIdx.y) * kBM;
-        s_tile[2] = b - a;  // K rows
-        s_tile[3] = a;
+    for (int i = 0; i < 8; ++i) {
+      cnt[i] = 0;
+      const int e = lane * per + i;
+      if (i < per && e < N) {
+        const int a = p.expert_offset[e], b = p.expert_offset[e + 1];
+        s_off[e] = a;
+        if (a < 0 || b < a || b > p.r_max) bad = true;
+        else cnt[i] = (b - a + kBM - 1) / kBM;
+        sum += cnt[i];
       }
     }
-  }
-  __syncthreads();
-  if (s_tile[0] < 0) return;  // whole CTA: no tile here
-  if (warp == 1) {
-    tmem_alloc(smem_u32(&s_tmem), kBN);
-    tmem_relinquish();
+    if (lane == 31) s_off[N] = p.expert_offset[N];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * per + i;
+      if (i < per && e < N) {
+        s_mt[e] = run;
+        run += cnt[i];
+      }
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 31) {
+      s_mt[N] = incl;
+      s_tiles = bad ? 0 : (MODE == GEMM_ROWS ? incl * n_tiles_n : N * m_tiles * n_tiles_n);
+      if (bad) report_error(p.status, MOE_ERR_BOUNDS);
+    }
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-
-  const int e = s_tile[0], m0 = s_tile[1], rows = s_tile[2], k0 = s_tile[3];
-  const int n0 = static_cast<int>(blockIdx.x) * kBN;
-  const int nkb = MODE == GEMM_ROWS ? p.num_kb : (rows + kBK - 1) / kBK;
+  const int total = s_tiles;
   const uint32_t tmem = s_tmem;
 
   if (warp == 0) {
@@ -185,33 +220,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_last();
       bool ok = true;
-      int kb = 0;
-      for (; kb < nkb; ++kb) {
-        const int s = kb % kStages;
-        if (!mbar_wait(smem_u32(&empty_bar[s]), ((kb / kStages) & 1) ^ 1u, p.timeout_ns, &s_abort)) {
-          ok = false;
-          break;
-        }
-        const uint32_t fb = smem_u32(&full_bar[s]);
-        const uint32_t a_dst = tiles + s * kStageBytes, b_dst = a_dst + kABytes;
-        mbar_arrive_expect_tx(fb, kStageBytes);
-        if (!A_MN) {
-          tma_load_2d(a_dst, &tmA, fb, kb * kBK, m0, pol);
-        } else {
+      int it = 0;
+      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        const GemmTile c = decode_gemm_tile<MODE>(t, p, n_tiles_n, m_tiles, s_mt, s_off);
+        for (int kb = 0; kb < c.nkb; ++kb, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(smem_u32(&empty_bar[s]), ((it / kStages) & 1) ^ 1u, p.timeout_ns, &s_abort)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full_bar[s]);
+          const uint32_t a_dst = tiles + s * kStageBytes, b_dst = a_dst + kABytes;
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          if (!A_MN) {
+            tma_load_2d(a_dst, &tmA, fb, kb * kBK, c.m0, pol);
+          } else {
 #pragma unroll
-          for (int i = 0; i < kBM / 64; ++i)
-            tma_load_2d(a_dst + i * kBox, &tmA, fb, m0 + 64 * i, k0 + kb * kBK, pol);
-        }
-        if (!B_MN) {
-          tma_load_3d(b_dst, &tmB, fb, kb * kBK, n0, e, pol);
-        } else if (MODE == GEMM_ROWS) {
+            for (int i = 0; i < kBM / 64; ++i)
+              tma_load_2d(a_dst + i * kBox, &tmA, fb, c.m0 + 64 * i, c.k0 + kb * kBK, pol);
+          }
+          if (!B_MN) {
+            tma_load_3d(b_dst, &tmB, fb, kb * kBK, c.n0, c.e, pol);
+          } else if (MODE == GEMM_ROWS) {
 #pragma unroll
-          for (int i = 0; i < kBN / 64; ++i)
-            tma_load_3d(b_dst + i * kBox, &tmB, fb, n0 + 64 * i, kb * kBK, e, pol);
-        } else {
+            for (int i = 0; i < kBN / 64; ++i)
+              tma_load_3d(b_dst + i * kBox, &tmB, fb, c.n0 + 64 * i, kb * kBK, c.e, pol);
+          } else {
 #pragma unroll
-          for (int i = 0; i < kBN / 64; ++i)
-            tma_load_2d(b_dst + i * kBox, &tmB, fb, n0 + 64 * i, k0 + kb * kBK, pol);
+            for (int i = 0; i < kBN / 64; ++i)
+              tma_load_2d(b_dst + i * kBox, &tmB, fb, c.n0 + 64 * i, c.k0 + kb * kBK, pol);
+          }
         }
       }
       if (!ok) {
@@ -219,7 +257,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         report_error(p.status, MOE_ERR_TIMEOUT);
       }
       // no TMA write may still be landing in shared memory when the CTA exits
-      for (int i = max(0, kb - kStages); i < kb; ++i)
+      for (int i = max(0, it - kStages); i < it; ++i)
         mbar_wait(smem_u32(&full_bar[i % kStages]), (i / kStages) & 1, kDrainTimeoutNs, nullptr);
     }
   } else if (warp == 1) {
@@ -228,100 +266,122 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                (B_MN ? (1u << 16) : 0u);
     bool ok = true;
     bool issued = false;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % kStages;
-      const bool got = mbar_wait(smem_u32(&full_bar[s]), (kb / kStages) & 1, p.timeout_ns, &s_abort);
-      if (!__all_sync(0xffffffffu, got)) {
+    int it = 0, uc = 0;
+    for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+      const GemmTile c = decode_gemm_tile<MODE>(t, p, n_tiles_n, m_tiles, s_mt, s_off);
+      if (c.nkb == 0) continue;  // no rows: the epilogue writes zeros
+      const int buf = uc & 1;
+      const bool free_buf = mbar_wait(smem_u32(&tempty_bar[buf]), ((uc >> 1) & 1) ^ 1u, p.timeout_ns, &s_abort);
+      if (!__all_sync(0xffffffffu, free_buf)) {
         ok = false;
         break;
       }
-      const uint32_t a_base = tiles + s * kStageBytes, b_base = a_base + kABytes;
-      const int valid = rows - kb * kBK;
-      if (MODE == GEMM_WGRAD && valid < kBK) {
-        // the expert's rows end inside this k block: zero k rows [valid, 64) of every box
-        uint8_t* st = dyn_smem + (a_base - smem_u32(dyn_smem));
-        const int lines = kBK - valid;
-        const int boxes = kBM / 64 + kBN / 64;
-        for (int i = lane; i < boxes * lines * 8; i += 32) {
-          const int box = i / (lines * 8), rem = i - box * lines * 8;
-          const int line = valid + rem / 8, chunk = rem & 7;
-          const uint32_t off = (box < kBM / 64 ? box * kBox : kABytes + (box - kBM / 64) * kBox) +
-                               line * 128 + chunk * 16;
-          *reinterpret_cast<uint4*>(st + off) = make_uint4(0u, 0u, 0u, 0u);
+      tc_fence_after_sync();
+      const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * kBN);
+      for (int kb = 0; kb < c.nkb; ++kb, ++it) {
+        const int s = it % kStages;
+        const bool got = mbar_wait(smem_u32(&full_bar[s]), (it / kStages) & 1, p.timeout_ns, &s_abort);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
         }
-        fence_proxy_async_smem();  // generic stores -> visible to the tensor core
+        const uint32_t a_base = tiles + s * kStageBytes, b_base = a_base + kABytes;
+        const int valid = c.rows - kb * kBK;
+        if (MODE == GEMM_WGRAD && valid < kBK) {
+          // the expert's rows end inside this k block: zero k rows [valid, 64) of every box
+          uint8_t* st = dyn_smem + (a_base - smem_u32(dyn_smem));
+          const int lines = kBK - valid;
+          const int boxes = kBM / 64 + kBN / 64;
+          for (int i = lane; i < boxes * lines * 8; i += 32) {
+            const int box = i / (lines * 8), rem = i - box * lines * 8;
+            const int line = valid + rem / 8, chunk = rem & 7;
+            const uint32_t off = (box < kBM / 64 ? box * kBox : kABytes + (box - kBM / 64) * kBox) +
+                                 line * 128 + chunk * 16;
+            *reinterpret_cast<uint4*>(st + off) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();  // generic stores -> visible to the tensor core
+          __syncwarp();
+        }
+        tc_fence_after_sync();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t da = A_MN ? smem_desc_mn_sw128(a_base + kk * 2048)
+                                     : smem_desc_k_sw128(a_base + kk * 32);
+            const uint64_t db = B_MN ? smem_desc_mn_sw128(b_base + kk * 2048)
+                                     : smem_desc_k_sw128(b_base + kk * 32);
+            tc_mma_f16(d_tmem, da, db, idesc, (kb != 0 || kk != 0) ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&empty_bar[s]));
+        }
+        issued = true;
         __syncwarp();
       }
-      tc_fence_after_sync();
-      if (lane == 0) {
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          const uint64_t da = A_MN ? smem_desc_mn_sw128(a_base + kk * 2048)
-                                   : smem_desc_k_sw128(a_base + kk * 32);
-          const uint64_t db = B_MN ? smem_desc_mn_sw128(b_base + kk * 2048)
-                                   : smem_desc_k_sw128(b_base + kk * 32);
-          tc_mma_f16(tmem, da, db, idesc, (kb != 0 || kk != 0) ? 1u : 0u);
-        }
-        tc_commit(smem_u32(&empty_bar[s]));
-      }
-      issued = true;
-      __syncwarp();
+      if (!ok) break;
+      if (lane == 0) tc_commit(smem_u32(&tfull_bar[buf]));
+      ++uc;
     }
-    if (lane == 0) {
-      if (ok && nkb > 0) {
-        tc_commit(smem_u32(&tfull_bar));
-      } else if (!ok) {
-        s_abort = 1;
-        report_error(p.status, MOE_ERR_TIMEOUT);
-        if (issued) {  // let every issued MMA finish before TMEM is freed
-          tc_commit(smem_u32(&tfull_bar));
-          mbar_wait(smem_u32(&tfull_bar), 0, kDrainTimeoutNs, nullptr);
-        }
+    if (!ok && lane == 0) {
+      s_abort = 1;
+      report_error(p.status, MOE_ERR_TIMEOUT);
+      if (issued) {  // let every issued MMA finish before TMEM is freed
+        tc_commit(smem_u32(&done_bar));
+        mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
       }
     }
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lane quadrant of this warp
-    const int r_local = q * 32 + lane;
-    bool have = nkb > 0;
-    if (have) {
-      const bool got = mbar_wait(smem_u32(&tfull_bar), 0, p.timeout_ns, &s_abort);
-      if (!__all_sync(0xffffffffu, got)) {
-        s_abort = 1;
-        report_error(p.status, MOE_ERR_TIMEOUT);
-        have = false;
-      } else {
+    int uc = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const GemmTile c = decode_gemm_tile<MODE>(t, p, n_tiles_n, m_tiles, s_mt, s_off);
+      const bool have = c.nkb > 0;
+      const int buf = uc & 1;
+      if (have) {
+        const bool got = mbar_wait(smem_u32(&tfull_bar[buf]), (uc >> 1) & 1, p.timeout_ns, &s_abort);
+        if (!__all_sync(0xffffffffu, got)) {
+          s_abort = 1;
+          report_error(p.status, MOE_ERR_TIMEOUT);
+          break;
+        }
         tc_fence_after_sync();
       }
-    }
-    if (have || nkb == 0) {
-      bool row_ok;
-      float* dst;
+      // rows q*32 .. q*32+31 of the tile: 32 columns at a time go through this warp's
+      // shared-memory block, so that each store instruction writes one row's 128 bytes
+      int row_lim;  // rows of this warp's 32 that exist
+      float* base;  // row q*32 of the tile
       if (MODE == GEMM_ROWS) {
-        row_ok = r_local < rows;
-        dst = p.out + (static_cast<int64_t>(m0) + r_local) * p.n_out;
+        row_lim = min(32, c.rows - q * 32);
+        base = p.out + (static_cast<int64_t>(c.m0) + q * 32) * p.n_out;
       } else {
-        row_ok = m0 + r_local < p.M;
-        dst = p.out + (static_cast<int64_t>(e) * p.M + m0 + r_local) * p.n_out;
+        row_lim = min(32, p.M - c.m0 - q * 32);
+        base = p.out + (static_cast<int64_t>(c.e) * p.M + c.m0 + q * 32) * p.n_out;
       }
-      const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      float (*stage)[33] = s_stage[warp - 2];
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kBN);
 #pragma unroll 1
-      for (int cc = 0; cc < kBN; cc += 16) {
-        if (n0 + cc >= p.n_out) break;  // warp-uniform: ragged last n-tile
-        uint32_t v[16];
+      for (int cc = 0; cc < kBN; cc += 32) {
+        if (c.n0 + cc >= p.n_out) break;  // warp-uniform: ragged last n-tile
+        uint32_t v[32];
         if (have) {
-          tmem_ld_32x32b_x16(t_row + cc, v);
+          tmem_ld_32x32b_x32(t_row + cc, v);
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = 0u;  // an expert with no rows: zero gradient
+          for (int i = 0; i < 32; ++i) v[i] = 0u;  // an expert with no rows: zero gradient
         }
-        if (!row_ok) continue;
-        float4* d4 = reinterpret_cast<float4*>(dst + n0 + cc);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                              __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        for (int i = 0; i < 32; ++i) stage[lane][i] = __uint_as_float(v[i]);
+        __syncwarp();
+        const int col = c.n0 + cc + lane;
+        if (col < p.n_out)
+          for (int r = 0; r < row_lim; ++r) base[static_cast<int64_t>(r) * p.n_out + col] = stage[r][lane];
+        __syncwarp();
+      }
+      if (have) {
+        tc_fence_before_sync();
+        mbar_arrive(smem_u32(&tempty_bar[buf]));  // TMEM buffer free for the tile after next
+        ++uc;
       }
     }
   }
@@ -329,7 +389,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem, kBN);
+    tmem_dealloc(tmem, 2 * kBN);
   }
 }
 
@@ -631,7 +691,18 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {
     p.r_max = static_cast<int>(a.r_max);
     p.status = a.status;
     p.timeout_ns = a.timeout_ns;
-    const unsigned m_tiles = static_cast<unsigned>((R + kBM - 1) / kBM + N);
+    int sms = 148;
+    {
+      int dev = 0;
+      if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    // rows mode: the tile count depends on expert_offset, so every SM gets a CTA
+    const dim3 rows_grid(static_cast<unsigned>(sms));
+    auto wgrad_grid = [&](int M, int n_out) {
+      const int64_t t = static_cast<int64_t>(N) * ((M + kBM - 1) / kBM) * ((n_out + kBN - 1) / kBN);
+      return dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(t, sms))));
+    };
     CUtensorMap mA, mB;
     // 2: pre = x_perm W_gu^T
     if (!map_k_major_2d(&mA, a.x_perm, d, R, kBM)) return cudaErrorInvalidValue;
@@ -644,7 +715,7 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {
     p.n_out = n_gu;
     p.num_kb = d / kBK;
     p.out = a.pre;
-    e = launch_gemm<false, false, GEMM_ROWS>(mA, mB, p, dim3((n_gu + kBN - 1) / kBN, m_tiles), s);
+    e = launch_gemm<false, false, GEMM_ROWS>(mA, mB, p, rows_grid, s);
     if (e != cudaSuccess) return e;
     // 3: dh = dy W_d (W_d [N][d][F] read MN-major: F is the output axis)
     if (!map_k_major_2d(&mA, a.dy_perm, d, R, kBM)) return cudaErrorInvalidValue;
@@ -657,7 +728,7 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {
     p.n_out = F;
     p.num_kb = d / kBK;
     p.out = a.dh;
-    e = launch_gemm<false, true, GEMM_ROWS>(mA, mB, p, dim3((F + kBN - 1) / kBN, m_tiles), s);
+    e = launch_gemm<false, true, GEMM_ROWS>(mA, mB, p, rows_grid, s);
     if (e != cudaSuccess) return e;
     // 4: d_pre, h
     {
@@ -679,7 +750,7 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {
     p.n_out = d;
     p.num_kb = n_gu / kBK;
     p.out = a.dx_rows;
-    e = launch_gemm<false, true, GEMM_ROWS>(mA, mB, p, dim3((d + kBN - 1) / kBN, m_tiles), s);
+    e = launch_gemm<false, true, GEMM_ROWS>(mA, mB, p, rows_grid, s);
     if (e != cudaSuccess) return e;
     // 6: dW_d[e] = dy_e^T h_e  ([d, F] per expert)
     if (!map_mn_major_2d(&mA, a.dy_perm, d, R)) return cudaErrorInvalidValue;
@@ -687,7 +758,7 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {
     p.M = d;
     p.n_out = F;
     p.out = a.d_w_down;
-    e = launch_gemm<true, true, GEMM_WGRAD>(mA, mB, p, dim3((F + kBN - 1) / kBN, (d + kBM - 1) / kBM, N), s);
+    e = launch_gemm<true, true, GEMM_WGRAD>(mA, mB, p, wgrad_grid(d, F), s);
     if (e != cudaSuccess) return e;
     // 7: dW_gu[e] = d_pre_e^T x_e  ([n_gu, d] per expert)
     if (!map_mn_major_2d(&mA, a.d_pre, n_gu, R)) return cudaErrorInvalidValue;
@@ -695,7 +766,7 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {
     p.M = n_gu;
     p.n_out = d;
     p.out = a.d_w_gate_up;
-    e = launch_gemm<true, true, GEMM_WGRAD>(mA, mB, p, dim3((d + kBN - 1) / kBN, (n_gu + kBM - 1) / kBM, N), s);
+    e = launch_gemm<true, true, GEMM_WGRAD>(mA, mB, p, wgrad_grid(n_gu, d), s);
     if (e != cudaSuccess) return e;
   } else {
     // no kept rows: the experts' gradients are zero
