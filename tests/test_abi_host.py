@@ -134,3 +134,56 @@ def test_forward_layout_is_disjoint_and_aligned():
 def test_status_strings():
     for s in (0, -1, -2, -3, -4, -5, -6):
         assert moe.status_string(s)
+
+
+def _r256(n):
+    return (n + 255) // 256 * 256
+
+
+def test_backward_workspace_bytes():
+    """Regions: status word, dL, dy, pre, dh, d_pre, h, dx_rows, router partial sums."""
+    for T, d, N, k, F, act, cap in [(300, 192, 8, 2, 320, "swiglu", 75), (4096, 1024, 64, 1, 4096, "gelu", 64),
+                                    (40000, 128, 4, 2, 64, "gelu", 40000)]:
+        dims = moe.make_dims(T, d, N, k, F, act, cap)
+        R = moe.max_rows(dims)
+        n_gu = 2 * F if act == "swiglu" else F
+        chunk = max(256, (T + 15) // 16)
+        chunks = (T + chunk - 1) // chunk
+        sizes = [256, T * N * 4, R * d * 2, R * n_gu * 4, R * F * 4, R * n_gu * 2, R * F * 2,
+                 R * d * 4, chunks * N * d * 4]
+        assert moe.backward_workspace_bytes(dims) == sum(_r256(s) for s in sizes)
+
+
+def test_backward_validation_precedes_device_use():
+    d = moe.make_dims(16, 128, 8, 2, 128, "swiglu", 16)
+    P = ctypes.c_void_p
+    lib = moe._lib
+    big = 1 << 30
+    fw = moe.forward_workspace_bytes(d)
+    args = lambda x=P(16), ws_bytes=big, fwd_bytes=fw, d_bias=None: (
+        ctypes.byref(d), x, P(16), P(16), P(16), P(16), fwd_bytes, P(16), P(16), P(16), d_bias,
+        P(16), P(16), P(16), ws_bytes, None)
+    assert lib.moe_backward(*args(x=None)) == moe.ERR_INVALID
+    assert lib.moe_backward(*args(x=P(24))) == moe.ERR_UNSUPPORTED
+    assert lib.moe_backward(*args(d_bias=P(8))) == moe.ERR_UNSUPPORTED
+    assert lib.moe_backward(*args(ws_bytes=64)) == moe.ERR_WORKSPACE
+    assert lib.moe_backward(*args(fwd_bytes=64)) == moe.ERR_WORKSPACE
+    e = moe.make_dims(0, 128, 8, 2, 128, "swiglu", 0)
+    assert lib.moe_backward(ctypes.byref(e), None, None, None, None, None, 0, None, None, None,
+                            None, None, None, None, 0, None) == moe.OK
+
+
+def test_redirect_validation_precedes_device_use():
+    P = ctypes.c_void_p
+    lib = moe._lib
+    d = moe.make_dims(16, 128, 8, 2, 128, "swiglu", 4)
+    assert lib.moe_redirect_overflow(ctypes.byref(d), None, P(16), P(16), P(16), P(16), 1 << 20,
+                                     None) == moe.ERR_INVALID
+    assert lib.moe_redirect_overflow(ctypes.byref(d), P(16), P(20), P(16), P(16), P(16), 1 << 20,
+                                     None) == moe.ERR_UNSUPPORTED
+    assert lib.moe_redirect_overflow(ctypes.byref(d), P(16), P(16), P(16), P(16), P(16), 8,
+                                     None) == moe.ERR_WORKSPACE
+    big = moe.make_dims(16385, 128, 8, 2, 128, "swiglu", 4)  # T * k = 32770 pairs
+    assert lib.moe_redirect_overflow(ctypes.byref(big), P(16), P(16), P(16), P(16), P(16), 1 << 30,
+                                     None) == moe.ERR_UNSUPPORTED
+    assert moe.REDIRECT_MAX_PAIRS == 32768
