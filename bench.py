@@ -94,6 +94,24 @@ def algorithmic_bytes(shape, T: int, active_experts: int, R: int, wfmt: str = "b
     return {"layer": layer, "ffn": ffn, "weights": w}
 
 
+def backward_model(shape, T: int, R: int, active_experts: int):
+    """(FLOPs, algorithmic bytes) of one backward pass with R kept rows.
+
+    FLOPs: the five expert GEMMs, pre = x W_gu^T (recomputed) and dx_rows = d_pre W_gu and
+    dW_gu = d_pre^T x (2 R d n_gu each), dh = dy W_d and dW_d = dy^T h (2 R d F each).
+    Bytes: the active experts' bf16 weights read once, every expert's fp32 weight gradients
+    written, x_perm (bf16) and y_perm (fp32) read, d_out and x read (bf16), dx written
+    (fp32), and the router's fp32 gradient written.
+    """
+    d, N, F = shape.d_model, shape.n_experts, shape.d_ff
+    n_gu = 2 * F if shape.act == "swiglu" else F
+    flops = 6 * R * d * n_gu + 4 * R * d * F
+    per_expert = n_gu * d + d * F
+    nbytes = (active_experts * per_expert * 2 + N * per_expert * 4 + R * d * (2 + 4)
+              + T * d * (2 + 2 + 4) + N * d * 4)
+    return flops, nbytes
+
+
 def ffn_flops(shape, R: int) -> int:
     d, F = shape.d_model, shape.d_ff
     return 2 * R * d * F * (3 if shape.act == "swiglu" else 2)
@@ -341,10 +359,7 @@ class Layer:
         ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
         counts = self.views()["expert_count"].cpu()
         R, active = int(counts.sum()), int((counts > 0).sum())
-        flops = 6 * R * d * n_gu + 4 * R * d * F
-        per_expert = n_gu * d + d * F
-        nbytes = (active * per_expert * 2 + N * per_expert * 4 + R * d * (2 + 4)
-                  + T * d * (2 + 2 + 4) + N * d * 4)
+        flops, nbytes = backward_model(s, T, R, active)
         tensor = flops / nbytes > (peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9)
         if tensor:
             ach, peak, unit = flops / (ms * 1e-3) / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"

@@ -64,3 +64,16 @@ def test_mx_weight_bytes():
     b = bench.algorithmic_bytes(s, 1, 4, 4, "mxfp4")
     params = 3 * 2880 * 2880
     assert b["weights"] == 4 * (params // 2 + params // 32)
+
+
+def test_backward_model_hand_numbers():
+    """Backward FLOPs and bytes for a hand-sized GELU and SwiGLU layer."""
+    import synthetic
+    gelu = synthetic.LayerShape("t", 8, 2, 1, 4, "gelu", None, (3,))
+    flops, nbytes = bench.backward_model(gelu, T=3, R=3, active_experts=2)
+    assert flops == 10 * 3 * 8 * 4                        # 6 R d F + 4 R d F
+    per = 4 * 8 + 8 * 4                                    # W_1 and W_2 of one expert
+    assert nbytes == 2 * per * 2 + 2 * per * 4 + 3 * 8 * 6 + 3 * 8 * 8 + 2 * 8 * 4
+    swiglu = synthetic.LayerShape("t", 8, 2, 1, 4, "swiglu", None, (3,))
+    flops, _ = bench.backward_model(swiglu, T=3, R=3, active_experts=2)
+    assert flops == 6 * 3 * 8 * 8 + 4 * 3 * 8 * 4
