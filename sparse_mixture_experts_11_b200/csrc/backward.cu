@@ -51,7 +51,8 @@ constexpr int kABytes = kBM * kBK * 2;
 constexpr int kBBytes = kBN * kBK * 2;
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kGemmThreads = 192;
-constexpr int kGemmSmem = kStages * kStageBytes + 1024;
+constexpr int kStoreStage = 32 * 32 * 4;  // one epilogue warp's 32 x 32 fp32 block
+constexpr int kGemmSmem = kStages * kStageBytes + 4 * kStoreStage + 1024;
 constexpr int kBox = 64 * 64 * 2;  // one MN-major TMA box: 64 MN x 64 k rows, 8 KB
 
 enum { GEMM_ROWS = 0, GEMM_WGRAD = 1 };
@@ -127,7 +128,7 @@ __device__ __forceinline__ GemmTile decode_gemm_tile(int t, const BwdGemmParams&
 template <bool A_MN, bool B_MN, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const BwdGemmParams p) {
+                    const __grid_constant__ CUtensorMap tmC, const BwdGemmParams p) {
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
@@ -139,7 +140,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __shared__ int s_mt[257];  // rows mode: first m-tile of each expert; s_mt[N] = all m-tiles
   __shared__ int s_off[257];
   __shared__ int s_tiles;
-  __shared__ float s_stage[4][32][33];  // epilogue: one 32 x 32 fp32 block per warp
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmC);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
@@ -332,6 +333,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lane quadrant of this warp
+    const uint32_t stg_addr = tiles + kStages * kStageBytes + (warp - 2) * kStoreStage;
+    uint8_t* const stg = dyn_smem + (stg_addr - smem_u32(dyn_smem));
     int uc = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const GemmTile c = decode_gemm_tile<MODE>(t, p, n_tiles_n, m_tiles, s_mt, s_off);
@@ -346,8 +349,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after_sync();
       }
-      // rows q*32 .. q*32+31 of the tile: 32 columns at a time go through this warp's
-      // shared-memory block, so that each store instruction writes one row's 128 bytes
+      // rows q*32 .. q*32+31 of the tile, 32 columns at a time through this warp's block of
+      // shared memory. A block whose 32 rows all exist leaves as one TMA store (128B-swizzled:
+      // row r's 16-byte chunk j sits at chunk j ^ (r & 7)); the rows of an expert's last, partial
+      // m-tile go out as plain stores, each instruction one row's 128 bytes.
       int row_lim;  // rows of this warp's 32 that exist
       float* base;  // row q*32 of the tile
       if (MODE == GEMM_ROWS) {
@@ -357,7 +362,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         row_lim = min(32, p.M - c.m0 - q * 32);
         base = p.out + (static_cast<int64_t>(c.e) * p.M + c.m0 + q * 32) * p.n_out;
       }
-      float (*stage)[33] = s_stage[warp - 2];
       const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kBN);
 #pragma unroll 1
       for (int cc = 0; cc < kBN; cc += 32) {
@@ -370,13 +374,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0u;  // an expert with no rows: zero gradient
         }
+        if (lane == 0) tma_store_wait_read();  // the last store has read this warp's block
+        __syncwarp();
+        if (row_lim >= 32) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) stage[lane][i] = __uint_as_float(v[i]);
-        __syncwarp();
-        const int col = c.n0 + cc + lane;
-        if (col < p.n_out)
-          for (int r = 0; r < row_lim; ++r) base[static_cast<int64_t>(r) * p.n_out + col] = stage[r][lane];
-        __syncwarp();
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          fence_proxy_async_smem();  // generic stores -> visible to the TMA engine
+          __syncwarp();
+          if (lane == 0) {
+            if (MODE == GEMM_ROWS) tma_store_2d(&tmC, stg_addr, c.n0 + cc, c.m0 + q * 32);
+            else tma_store_3d(&tmC, stg_addr, c.n0 + cc, c.m0 + q * 32, c.e);
+            tma_store_commit();
+          }
+        } else if (row_lim > 0) {
+          // element i of row r at r * 32 + (i ^ r): conflict-free both ways
+          float* f = reinterpret_cast<float*>(stg);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[lane * 32 + (i ^ lane)] = __uint_as_float(v[i]);
+          __syncwarp();
+          const int col = c.n0 + cc + lane;
+          if (col < p.n_out)
+            for (int r = 0; r < row_lim; ++r) base[static_cast<int64_t>(r) * p.n_out + col] = f[r * 32 + (lane ^ r)];
+          __syncwarp();
+        }
       }
       if (have) {
         tc_fence_before_sync();
@@ -384,6 +406,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ++uc;
       }
     }
+    if (lane == 0) tma_store_wait_all();  // every store of this warp has landed
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -644,11 +667,26 @@ __global__ void __launch_bounds__(256) bwd_dx_kernel(
 template <bool A_MN, bool B_MN, int MODE>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const BwdGemmParams& p,
                         dim3 grid, cudaStream_t s) {
+  // the output as fp32 32 x 32 store boxes: [r_max, n_out] (rows mode) or [N, M, n_out]
+  CUtensorMap c;
+  if (MODE == GEMM_ROWS) {
+    const uint64_t dims[2] = {static_cast<uint64_t>(p.n_out), static_cast<uint64_t>(p.r_max)};
+    const uint64_t str[1] = {static_cast<uint64_t>(p.n_out) * 4};
+    const uint32_t box[2] = {32, 32};
+    if (!make_map_f32(&c, p.out, 2, dims, str, box)) return cudaErrorInvalidValue;
+  } else {
+    const uint64_t dims[3] = {static_cast<uint64_t>(p.n_out), static_cast<uint64_t>(p.M),
+                              static_cast<uint64_t>(p.n_experts)};
+    const uint64_t str[2] = {static_cast<uint64_t>(p.n_out) * 4,
+                             static_cast<uint64_t>(p.M) * p.n_out * 4};
+    const uint32_t box[3] = {32, 32, 1};
+    if (!make_map_f32(&c, p.out, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
   auto kern = bwd_gemm_kernel<A_MN, B_MN, MODE>;
   static cudaError_t attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
   if (attr != cudaSuccess) return attr;
-  return launch_pdl(kern, grid, dim3(kGemmThreads), kGemmSmem, s, a, b, p);
+  return launch_pdl(kern, grid, dim3(kGemmThreads), kGemmSmem, s, a, b, c, p);
 }
 
 // K-major operand [outer][K] bf16: boxes of 64 k x `rows`.
