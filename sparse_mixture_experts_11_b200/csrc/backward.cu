@@ -21,15 +21,15 @@
 // bwd_gemm_kernel is persistent, one CTA per SM striding through 128 x 256 output tiles on
 // tcgen05 (192 threads: TMA producer, MMA issuer, four epilogue warps; four 48 KB stages;
 // two fp32 accumulators in TMEM, so one tile's epilogue overlaps the next one's loads and
-// MMAs). Each operand
-// is K-major (the contiguous axis is the reduction axis) or MN-major (the contiguous axis is
-// the output's row or column axis), so the transposed products read the weights and the
-// activations where they lie: an MN-major operand comes as 64 x 64 TMA boxes (128 bytes of
-// the MN axis by 64 k rows, 128B-swizzled) and the MMA reads it through an MN-major shared
-// memory descriptor with the instruction's transpose bit set. Rows mode: the tile's rows are
-// an expert's rows of the permuted batch and K is fixed. Weight-gradient mode: the tile is a
-// block of an expert's [M, n_out] gradient and K runs over the expert's rows; the last k block
-// is cut at the expert's end by zeroing the rows past it in shared memory. Every wait is
+// MMAs). Each operand is K-major (the contiguous axis is the reduction axis) or MN-major (the
+// contiguous axis is the output's row or column axis), so the transposed products read the
+// weights and the activations where they lie: an MN-major operand comes as 64 x 64 TMA boxes
+// (128 bytes of the MN axis by 64 k rows, 128B-swizzled) and the MMA reads it through an
+// MN-major shared-memory descriptor with the instruction's transpose bit set. Rows mode: the
+// tile's rows are an expert's rows of the permuted batch and K is fixed. Weight-gradient mode:
+// the tile is a block of an expert's [M, n_out] gradient and K runs over the expert's rows;
+// the last k block is cut at the expert's end by zeroing the rows past it in shared memory.
+// The epilogue sends each warp's 32 x 32 fp32 block out as one TMA store. Every wait is
 // bounded; on timeout the CTA records MOE_ERR_TIMEOUT and drains what it issued.
 #include <math.h>
 #include <string.h>
