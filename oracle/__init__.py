@@ -12,5 +12,5 @@ from .moe_oracle import (capacity_from_factor, router_logits, softmax_over_exper
 from .mx_oracle import (MX_BLOCK, decode_e8m0, decode_e4m3, decode_e2m1,  # noqa: F401
                         unpack_fp4, dequantize_mx)
 from .moe_backward import (logistic, silu_derivative, gelu_derivative,  # noqa: F401
-                           combine_backward, renormalise_backward, expert_backward,
+                           combine_backward, renormalise_backward, expert_backward, aux_loss_backward,
                            moe_layer_backward)

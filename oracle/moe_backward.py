@@ -85,6 +85,28 @@ def renormalise_backward(topk_w: np.ndarray, dw: np.ndarray, topk_idx: np.ndarra
     return dL
 
 
+def aux_loss_backward(logits: np.ndarray, topk_idx: np.ndarray, alpha: float = 1e-2,
+                      d_aux: float = 1.0) -> np.ndarray:
+    """Gradient of the auxiliary loss with respect to the logits (page «Sparse
+    Mixture-of-Experts», section «Маршрутизация токена и auxiliary loss»: aux =
+    alpha * N * sum_e f_e * P_e, f_e the fraction of the batch's tokens sent to expert e, P_e
+    the batch mean of the router probability).
+
+    f comes from the choice of experts and passes no gradient. P_e = (1/T) sum_t p_te and
+    dp_te/dL_ti = p_te (delta_ei - p_ti), so
+    dL_ti = d_aux * alpha * N / T * p_ti * (f_i - sum_e f_e p_te).
+    """
+    T, N = logits.shape
+    z = logits - logits.max(axis=1, keepdims=True)
+    p = np.exp(z)
+    p /= p.sum(axis=1, keepdims=True)
+    f = np.zeros(N)
+    for t in range(T):
+        for e in topk_idx[t]:
+            f[int(e)] += 1.0 / T
+    return d_aux * alpha * N / T * p * (f[None, :] - (p * f[None, :]).sum(axis=1, keepdims=True))
+
+
 def expert_backward(rows: np.ndarray, dy: np.ndarray, w_gate_up: np.ndarray,
                     w_down: np.ndarray, act: str):
     """One expert's rows: y = act-FFN(rows). Returns (d_rows, d_w_gate_up, d_w_down, pre, h).

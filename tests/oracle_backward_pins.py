@@ -134,5 +134,37 @@ def pin_dense_mixture(bwd):
         np.testing.assert_allclose(got[name], ref.numpy(), rtol=1e-10, atol=1e-12, err_msg=name)
 
 
+def pin_aux_loss_gradient(bwd):
+    """Finite differences of the forward oracle's auxiliary loss (routing held fixed by a
+    margin check), and two closed forms: a batch that loads every expert equally, and a single
+    expert, both have a zero gradient (sum_e p_te = 1)."""
+    rng = np.random.default_rng(41)
+    for T, N, k in ((9, 5, 2), (12, 4, 1)):
+        L = rng.normal(size=(T, N)) * 2.0
+        assert _margin(L, k) > 1e-3
+        idx = fwd.select_top_k(L, k)
+        got = bwd.aux_loss_backward(L, idx, alpha=0.01)
+        slot = np.zeros_like(idx)
+        eps = 1e-6
+        num = np.zeros_like(L)
+        for t in range(T):
+            for i in range(N):
+                keep = L[t, i]
+                L[t, i] = keep + eps
+                lp = fwd.router_statistics(L, idx, slot, alpha=0.01)["aux_loss"]
+                L[t, i] = keep - eps
+                lm = fwd.router_statistics(L, idx, slot, alpha=0.01)["aux_loss"]
+                L[t, i] = keep
+                num[t, i] = (lp - lm) / (2 * eps)
+        assert np.abs(got - num).max() <= 1e-8 * max(1.0, np.abs(num).max())
+    # every expert picked equally often: f_e = k / N, and the gradient vanishes
+    T, N, k = 8, 4, 2
+    idx = np.array([[t % N, (t + 1) % N] for t in range(T)])
+    g = bwd.aux_loss_backward(rng.normal(size=(T, N)), idx, alpha=0.5)
+    assert np.abs(g).max() < 1e-15
+    g1 = bwd.aux_loss_backward(rng.normal(size=(5, 1)), np.zeros((5, 1), dtype=np.int64))
+    assert np.abs(g1).max() == 0.0
+
+
 BACKWARD_PINS = [pin_fd_swiglu_top2_drops, pin_fd_gelu_top1, pin_fd_swiglu_top3_no_limit,
-                 pin_single_expert_is_plain_ffn, pin_dense_mixture]
+                 pin_single_expert_is_plain_ffn, pin_dense_mixture, pin_aux_loss_gradient]

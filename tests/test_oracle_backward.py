@@ -59,7 +59,25 @@ def _expert_backward_swapped_gate_up(rows, dy, wgu, wd, act):
     return d_rows, dgu, dd, pre, h
 
 
+def _aux_backward_without_mean_term(logits, topk_idx, alpha=1e-2, d_aux=1.0):
+    T, N = logits.shape
+    z = np.exp(logits - logits.max(axis=1, keepdims=True))
+    p = z / z.sum(axis=1, keepdims=True)
+    f = np.zeros(N)
+    for t in range(T):
+        for e in topk_idx[t]:
+            f[int(e)] += 1.0 / T
+    return d_aux * alpha * N / T * p * f[None, :]
+
+
+def _aux_backward_per_pair_f(logits, topk_idx, alpha=1e-2, d_aux=1.0):
+    k = topk_idx.shape[1]
+    return bwd.__dict__["_orig_aux_loss_backward"](logits, topk_idx, alpha, d_aux) / k
+
+
 MUTANTS = {
+    "aux_backward_without_mean_term": ("aux_loss_backward", _aux_backward_without_mean_term),
+    "aux_backward_f_over_pairs": ("aux_loss_backward", _aux_backward_per_pair_f),
     "silu_derivative_without_z_term": ("silu_derivative", _silu_derivative_no_second_term),
     "gelu_derivative_without_z_phi": ("gelu_derivative", _gelu_derivative_cdf_only),
     "renormalise_backward_missing_sum": ("renormalise_backward",
