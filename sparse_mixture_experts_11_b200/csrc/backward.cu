@@ -576,10 +576,17 @@ __global__ void __launch_bounds__(256) router_wgrad_partial_kernel(
     __syncthreads();
     if (col < d) {
       const int nt = min(kRwTokens, t1 - tb);
-      for (int tt = 0; tt < nt; ++tt) {
-        const float xv = bf16_bits_to_float(x[static_cast<int64_t>(tb + tt) * d + col]);
+      // eight tokens' loads in flight at once; the additions keep token order (staged dL rows
+      // past the chunk's end are zero)
+      for (int tt = 0; tt < nt; tt += 8) {
+        float xv[8];
 #pragma unroll
-        for (int i = 0; i < kRwExperts; ++i) acc[i] += s_dl[tt][i] * xv;
+        for (int u = 0; u < 8; ++u)
+          xv[u] = tt + u < nt ? bf16_bits_to_float(x[static_cast<int64_t>(tb + tt + u) * d + col]) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+          for (int i = 0; i < kRwExperts; ++i) acc[i] += s_dl[tt + u][i] * xv[u];
       }
     }
   }
