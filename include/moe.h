@@ -1,5 +1,7 @@
 /*
- * moe.h: C ABI of the sparse Mixture-of-Experts layer forward pass on NVIDIA B200 (sm_100a).
+ * moe.h: C ABI of the sparse Mixture-of-Experts layer on NVIDIA B200 (sm_100a): the forward
+ * pass, its router statistics, expert weights in MX formats, the redirect overflow policy and
+ * the backward pass.
  *
  * The layer (page «Sparse Mixture-of-Experts», bigdataschool wiki):
  *   1. router logits      L = x W_r^T (+ b), a linear layer without bias term
@@ -18,6 +20,8 @@
  *      grouped_mm, and «Динамическая загрузка весов с WeightConverter», packed layouts);
  *   5. the output is residual + the sum of the kept experts' outputs weighted by the
  *      renormalised router probabilities (section «Роутер и top-k gating»).
+ * moe_backward differentiates these steps (the choice of experts and the slots pass no
+ * gradient); moe_redirect_overflow replaces step 3's dropping by redirection.
  *
  * Conventions for every call:
  *   - Every pointer is a DEVICE pointer, allocated and owned by the caller, 16-byte aligned.
