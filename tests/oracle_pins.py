@@ -93,6 +93,29 @@ def pin_hand_routing(o):
     assert por.tolist() == u["pair_of_row"]
 
 
+def pin_logit_bias_hand_case(o):
+    """The per-expert logit bias, worked by hand: it enters every token's logits per expert
+    (not per token), with a plus sign, before selection and before the weights."""
+    g = _golden("hand_case_logit_bias.json")
+    x = np.array(g["x"], dtype=np.float64)
+    wr = np.array(g["w_router"], dtype=np.float64)
+    b = np.array(g["logit_bias"], dtype=np.float64)
+    L = o.router_logits(x, wr, b)
+    assert L.tolist() == g["logits"], L.tolist()
+    T, N = L.shape
+    r = o.route_from_logits(L, g["top_k"], T)
+    assert r["topk_idx"].tolist() == g["topk_idx"]
+    np.testing.assert_allclose(r["topk_w"], np.array(g["topk_w"]), rtol=0, atol=1e-15)
+    assert o.route_from_logits(L, 1, T)["topk_idx"].tolist() == g["top1_idx"]
+    c1 = g["capacity_1"]
+    r = o.route_from_logits(L, g["top_k"], 1)
+    assert r["slot"].tolist() == c1["slot"] and r["expert_count"].tolist() == c1["expert_count"]
+    # the whole layer routes on the biased logits as well
+    out = o.moe_layer_forward(x, wr, np.zeros((N, 2, 2)), np.zeros((N, 2, 1)), top_k=g["top_k"],
+                              act="swiglu", capacity=T, logit_bias=b, residual=x)
+    assert out["topk_idx"].tolist() == g["topk_idx"]
+
+
 def pin_top1_weight_is_one(o):
     rng = np.random.default_rng(7)
     L = rng.normal(size=(20, 6))
@@ -209,6 +232,24 @@ def pin_dense_special_case(o):
         np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
 
 
+def pin_dense_with_logit_bias(o):
+    """k = N, no limit, with a per-expert logit bias b: out = r + sum_e softmax(L + b)_e E_e(x),
+    the softmax written out term by term from the logits and the bias."""
+    rng = np.random.default_rng(41)
+    T, d, N, F = 5, 4, 3, 2
+    x, wr, wgu, wd = _small_layer(rng, T, d, N, F, "swiglu")
+    b = np.array([1.5, -0.75, 0.25])
+    got = o.moe_layer_forward(x, wr, wgu, wd, top_k=N, act="swiglu", capacity=T,
+                              logit_bias=b, residual=x)["out"]
+    want = x.copy()
+    for t in range(T):
+        z = [sum(x[t, i] * wr[e, i] for i in range(d)) + b[e] for e in range(N)]
+        ex = [math.exp(v - max(z)) for v in z]
+        for e in range(N):
+            want[t] += ex[e] / sum(ex) * o.expert_ffn(x[t:t + 1], wgu[e], wd[e], "swiglu")[0]
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
 def pin_single_expert_layer(o):
     """k = 1 with no limit: out[t] = res[t] + E_argmax(x[t]); token order irrelevant."""
     rng = np.random.default_rng(5)
@@ -302,9 +343,11 @@ def pin_aux_loss_closed_forms(o):
     assert st["picks"].tolist() == [2, 2, 1, 1] and st["dropped"] == 2
 
 
-ALL_PINS = [pin_capacity_demo, pin_capacity_formula, pin_hand_routing, pin_top1_weight_is_one,
+ALL_PINS = [pin_capacity_demo, pin_capacity_formula, pin_hand_routing, pin_logit_bias_hand_case,
+            pin_top1_weight_is_one,
             pin_two_way_weights, pin_brute_force_routing, pin_ffn_hand_cases,
-            pin_activation_limits, pin_dense_special_case, pin_single_expert_layer,
+            pin_activation_limits, pin_dense_special_case, pin_dense_with_logit_bias,
+            pin_single_expert_layer,
             pin_invariants, pin_zero_down_weights, pin_aux_loss_closed_forms]
 
 

@@ -81,6 +81,15 @@ def _router_transposed_bias_sign(x, wr, b=None):
     return L if b is None else L - b[None, :]
 
 
+def _router_bias_ignored(x, wr, b=None):
+    return x @ wr.T
+
+
+def _router_bias_per_token(x, wr, b=None):
+    L = x @ wr.T
+    return L if b is None else L + b[:L.shape[0], None]
+
+
 def _softmax_no_shift_wrong_axis(logits):
     ez = np.exp(logits)
     return ez / ez.sum(axis=0, keepdims=True)
@@ -122,6 +131,9 @@ MUTANTS = {
     "residual_dropped": ("combine", _combine_drops_residual),
     "aux_without_N": ("router_statistics", _aux_without_n),
     "aux_f_over_Tk": ("router_statistics", _aux_f_over_tk),
+    "bias_sign": ("router_logits", _router_transposed_bias_sign),
+    "bias_ignored": ("router_logits", _router_bias_ignored),
+    "bias_per_token": ("router_logits", _router_bias_per_token),
 }
 
 
