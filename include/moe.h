@@ -25,8 +25,11 @@
  *
  * Conventions for every call:
  *   - Every pointer is a DEVICE pointer, allocated and owned by the caller, 16-byte aligned.
- *     The library allocates nothing and frees nothing. It keeps only two kinds of
- *     process-wide state: a cached driver entry point and per-device attributes.
+ *     The library allocates nothing and frees nothing. Its process-wide state is: a cached
+ *     driver entry point; per-device kernel attributes and device properties, set or read
+ *     once per device; the wait limit of moe_debug_set_wait_timeout_ns; and, for
+ *     moe_route_noalloc only, static scratch arrays in device memory with their cached
+ *     device addresses.
  *   - "bf16" buffers hold bfloat16 bit patterns (uint16_t). All tensors are row-major and
  *     contiguous.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
@@ -342,7 +345,13 @@ moe_status moe_forward_mx(const moe_dims* dims, const uint16_t* x, const float* 
  *   - All calls share the arrays, and they keep the last call's contents. Each call writes
  *     every scratch entry before reading it, so nothing has to start at zero. Calls that
  *     overlap on the GPU (on concurrent streams) race on the arrays and must be serialised
- *     by the caller. */
+ *     by the caller.
+ *   - Device-side faults are not reported. moe_route keeps its status word in the caller's
+ *     workspace; this call has none. Its kernels bound their waits as moe_route's do. A wait
+ *     that runs out (which only a limit far below the default 2 s makes happen, see
+ *     moe_debug_set_wait_timeout_ns) stops the kernel early: the outputs of that call are
+ *     then undefined and the call has still returned MOE_OK. Expert ids outside [0, N) that
+ *     such a call may leave behind are never given a slot. The next call is unaffected. */
 moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x, const float* w_router,
                              const float* logit_bias, float* logits, int32_t* topk_idx,
                              float* topk_w, int32_t* slot, int32_t* expert_count, void* stream);

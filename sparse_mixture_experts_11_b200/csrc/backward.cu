@@ -325,10 +325,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (!ok && lane == 0) {
       s_abort = 1;
       report_error(p.status, MOE_ERR_TIMEOUT);
-      if (issued) {  // let every issued MMA finish before TMEM is freed
-        tc_commit(smem_u32(&done_bar));
-        mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
-      }
+    }
+    // every issued MMA has finished before TMEM is freed, also when the epilogue gave up on
+    // a tile whose MMAs this warp had already issued
+    if (issued && lane == 0) {
+      tc_commit(smem_u32(&done_bar));
+      mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
     }
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
@@ -690,8 +692,9 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const BwdGem
     if (!make_map_f32(&c, p.out, 3, dims, str, box)) return cudaErrorInvalidValue;
   }
   auto kern = bwd_gemm_kernel<A_MN, B_MN, MODE>;
-  static cudaError_t attr =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  static PerDeviceOnce once;
+  const cudaError_t attr = once.run(
+      [kern] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem); });
   if (attr != cudaSuccess) return attr;
   return launch_pdl(kern, grid, dim3(kGemmThreads), kGemmSmem, s, a, b, c, p);
 }

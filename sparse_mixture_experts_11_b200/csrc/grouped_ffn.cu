@@ -756,10 +756,12 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
       if (!ok) {
         s_abort = 1;
         report_error(p.status, MOE_ERR_TIMEOUT);
-        if (issued) {  // let every issued MMA finish before TMEM is freed
-          tc_commit(smem_u32(&done_bar));
-          mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
-        }
+      }
+      // every issued MMA has finished before TMEM is freed, also when the epilogue gave up
+      // on a tile whose MMAs this thread had already issued
+      if (issued) {
+        tc_commit(smem_u32(&done_bar));
+        mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
       }
     }
   } else if (warp < 6) {
@@ -944,11 +946,10 @@ cudaError_t launch_one(const CUtensorMap& a1, const CUtensorMap& b1, const CUten
                        const CUtensorMap& b2, const CUtensorMap& s1, const CUtensorMap& s2,
                        const FfnParams& fp, int grid, cudaStream_t s) {
   using C = Cfg<BM, WFMT>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(grouped_ffn_kernel<EPI1, BN1, BM, WFMT>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  static PerDeviceOnce once;
+  const cudaError_t attr_err = once.run([] {
+    return cudaFuncSetAttribute(grouped_ffn_kernel<EPI1, BN1, BM, WFMT>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
   return launch_pdl(grouped_ffn_kernel<EPI1, BN1, BM, WFMT>, dim3(grid), dim3(C::THREADS),

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace moe {
 
 // Launch a library kernel with programmatic stream serialisation (see pdl_wait/pdl_trigger).
@@ -46,6 +48,27 @@ inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
+
+// Runs a set-up step (a kernel attribute such as the dynamic shared-memory limit, which the
+// runtime keeps per device) once on each device it is called on, the current device at the
+// time of the call, and returns that device's cached result afterwards.
+class PerDeviceOnce {
+ public:
+  static constexpr int kDevices = 64;
+  template <typename Fn>
+  cudaError_t run(Fn fn) {
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kDevices) return cudaErrorInvalidDevice;
+    std::call_once(flag_[dev], [&] { err_[dev] = fn(); });
+    return err_[dev];
+  }
+
+ private:
+  std::once_flag flag_[kDevices];
+  cudaError_t err_[kDevices] = {};
+};
 
 // Per-stage workspace layout: [0, 256) status word (+ padding); [256, ...) capacity-scan scratch.
 constexpr size_t kStatusBytes = 256;

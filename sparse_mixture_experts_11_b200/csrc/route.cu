@@ -791,9 +791,12 @@ cudaError_t launch_reroute_slots(const float* logits, uint8_t* prefs, int32_t* t
                                 int32_t* slot, int32_t* expert_count, int T, int N, int k,
                                 int capacity, cudaStream_t s) {
   if (static_cast<int64_t>(T) * k > kRerouteMaxPairs || N > 256) return cudaErrorInvalidValue;
-  static cudaError_t attr = cudaFuncSetAttribute(
-      reroute_slots_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-      static_cast<int>(RerouteSmem::bytes(static_cast<int>(kRerouteMaxPairs))));
+  static PerDeviceOnce once;
+  const cudaError_t attr = once.run([] {
+    return cudaFuncSetAttribute(
+        reroute_slots_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        static_cast<int>(RerouteSmem::bytes(static_cast<int>(kRerouteMaxPairs))));
+  });
   if (attr != cudaSuccess) return attr;
   const int blocks = std::max(1, std::min((T + 7) / 8, 4 * 148));
   cudaError_t e = launch_pdl(redirect_prefs_kernel, dim3(blocks), dim3(256), 0, s, logits, prefs,

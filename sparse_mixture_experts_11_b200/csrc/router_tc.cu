@@ -339,10 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         s_abort = 1;
         report_error(status, MOE_ERR_TIMEOUT);
-        if (issued) {
-          tc_commit(smem_u32(&done_bar));
-          mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
-        }
+      }
+      // every issued MMA has finished before TMEM is freed, also when the epilogue gave up
+      // waiting for the accumulator
+      if (issued) {
+        tc_commit(smem_u32(&done_bar));
+        mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
       }
     }
   } else if (warp >= 4) {
@@ -572,10 +574,9 @@ cudaError_t launch_npk(const CUtensorMap& mx, const CUtensorMap& mw, const float
                        const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
                        int d, int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
   using C = RCfg<NP, PRESPLIT>;
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(router_tc_kernel<NP, PRESPLIT, KMAX>,
+  static PerDeviceOnce once;
+  const cudaError_t attr = once.run([] {
+    return cudaFuncSetAttribute(router_tc_kernel<NP, PRESPLIT, KMAX>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr != cudaSuccess) return attr;

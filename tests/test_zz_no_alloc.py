@@ -96,3 +96,25 @@ def test_noalloc_matches_route_decode_sized(T, d, N, k, cap):
         ref, got = _route_both(T, d, N, k, cap, 3, 1.1)
         _assert_same_routing(ref, got)
         assert torch.equal(ref["logits"], got["logits"])
+
+
+def test_noalloc_survives_a_timed_out_call():
+    """This call has no status word, so a wait that runs out is not reported. With a limit far
+    below the default, the tensor-core router (this shape's path) stops early; the context
+    stays usable and the next call, with the default limit, matches moe_route again."""
+    import sparse_mixture_experts_11_b200 as moe
+    T, d, N, k, cap = 9000, 256, 64, 2, 160
+    inp = synthetic.make_custom_inputs(T, d, N, 64, "swiglu", seed=1, device="cuda")
+    dims = moe.make_dims(T, d, N, k, 64, "swiglu", cap)
+    got = _buffers(T, N, k)
+    old = moe.debug_set_wait_timeout_ns(1)
+    try:
+        moe.route_noalloc(dims, inp["x"], inp["w_router"], inp["logit_bias"], got["logits"],
+                          got["topk_idx"], got["topk_w"], got["slot"], got["expert_count"])
+        torch.cuda.synchronize()  # raises if the early stop had faulted
+    finally:
+        moe.debug_set_wait_timeout_ns(0)
+    assert old == 2_000_000_000
+    for _ in range(2):
+        ref, got = _route_both(T, d, N, k, cap, 1)
+        _assert_same_routing(ref, got)
