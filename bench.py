@@ -37,7 +37,12 @@ if ROOT not in sys.path:
 
 import synthetic  # noqa: E402
 
-DEFAULT_WORKLOAD = "switch_top1:4096"
+DEFAULT_WORKLOAD = "fine_grained:16384"   # the largest workload that fits one GPU
+# every workload point of the five layer shapes, measured in one run (the "sweep" key)
+SWEEP = ("tiny_top2:64", "switch_top1:4096", "mixtral:1", "mixtral:16", "mixtral:512",
+         "mixtral:8192", "gpt_oss:1", "gpt_oss:8", "gpt_oss:64", "gpt_oss:16384",
+         "fine_grained:16384")
+DECODE_MIN_STEPS = 100  # sweep points with T <= 64 time at least this many steps
 METRIC = "MoE-layer fwd tokens/s on 1 B200; % of bf16 tensor peak / % of HBM BW"
 MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -83,15 +88,17 @@ def weight_bytes(params: int, wfmt: str = "bf16") -> int:
 def algorithmic_bytes(shape, T: int, active_experts: int, R: int, wfmt: str = "bf16") -> dict:
     """Bytes the layer must move (counting rules in the design notes).
 
-    layer: weights of every expert with at least one kept row, read once; router weight
-           (fp32); x read (bf16); out written (bf16). The residual is x itself.
-    ffn:   the same expert weights, plus x_perm read (bf16) and y_perm written (fp32).
+    weights: every expert with at least one kept row, read once (idle experts cost nothing).
+             This is the grouped FFN's algorithmic traffic: its intermediates (x_perm, h,
+             y_perm) are implementation overhead and are measured by ncu, not counted.
+    layer:   the same expert weights; router weight (fp32); x read (bf16); out written (bf16).
+             The residual is x itself.
+    rows:    the FFN's intermediate rows, for reference: x_perm read (bf16), y_perm written (fp32).
     """
     d, F, N = shape.d_model, shape.d_ff, shape.n_experts
     w = active_experts * weight_bytes(expert_params(d, F, shape.act), wfmt)
     layer = w + N * d * 4 + T * d * 2 + T * d * 2
-    ffn = w + R * d * 2 + R * d * 4
-    return {"layer": layer, "ffn": ffn, "weights": w}
+    return {"layer": layer, "weights": w, "rows": R * d * (2 + 4)}
 
 
 def backward_model(shape, T: int, R: int, active_experts: int):
@@ -115,6 +122,41 @@ def backward_model(shape, T: int, R: int, active_experts: int):
 def ffn_flops(shape, R: int) -> int:
     d, F = shape.d_model, shape.d_ff
     return 2 * R * d * F * (3 if shape.act == "swiglu" else 2)
+
+
+def roofline_of(shape, T: int, R: int, active: int, ffn_ms: float, step_ms: float, peaks: dict,
+                wfmt: str = "bf16", traffic=None) -> dict:
+    """Roofline of the grouped FFN (the dominant kernel) and of the whole layer.
+
+    The FFN is tensor-bound when its FLOPs (measured R) per algorithmic byte (active expert
+    weights) exceed the machine ridge, measured bf16 burst TFLOP/s over measured copy GB/s.
+    Its fraction is taken against the burst bf16 peak (the FFN stage is timed alone, between
+    L2 flushes) or the copy peak. The layer's fraction is its algorithmic bytes (weights, W_r,
+    x, out) over the whole step time against the copy peak; it is the figure the decode
+    targets are stated on. Tensor-bound points also report the layer's TFLOP/s."""
+    ab = algorithmic_bytes(shape, T, active, R, wfmt)
+    flops = ffn_flops(shape, R)
+    ridge = (peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9)
+    tensor = ab["weights"] > 0 and flops / ab["weights"] > ridge
+    ffn_s, step_s = ffn_ms * 1e-3, step_ms * 1e-3
+    if tensor:
+        ach, peak, unit = flops / ffn_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        per_launch, src = f"{flops} FLOP", peaks["source"] + " bf16 burst"
+    else:
+        ach, peak, unit = ab["weights"] / ffn_s / 1e9, peaks["hbm_gbs"], "GB/s"
+        per_launch, src = f"{ab['weights']} B", peaks["source"] + " copy"
+    ffn = {"bound": "tensor" if tensor else "hbm", "achieved": round(ach, 1), "peak": peak,
+           "unit": unit, "frac": round(ach / peak, 4), "per_launch": per_launch,
+           "peak_source": src, "traffic": traffic,
+           "traffic_over_algorithmic": (round(traffic / ab["weights"], 3)
+                                        if traffic and not tensor else None)}
+    layer_gbs = ab["layer"] / step_s / 1e9
+    layer = {"achieved_gbs": round(layer_gbs, 1), "frac_hbm": round(layer_gbs / peaks["hbm_gbs"], 4),
+             "algorithmic_bytes": ab["layer"]}
+    if tensor:
+        layer["achieved_tflops"] = round((flops + 2 * T * shape.d_model * shape.n_experts)
+                                         / step_s / 1e12, 1)
+    return {"ffn": ffn, "layer": layer, "weights_bytes": ab["weights"], "ffn_flops": flops}
 
 
 def router_on_tensor_cores(T: int, n_experts: int, d_model: int) -> bool:
@@ -152,7 +194,7 @@ def launches_per_step(T: int, k: int, R_max: int, n_experts: int = 1, d_model: i
 # DRAM traffic of the grouped-FFN stage per forward (dram__bytes_read.sum +
 # dram__bytes_write.sum of its launch) from one ncu capture of the current kernel; workloads
 # without a capture of the current kernel report null.
-MEASURED_FFN_TRAFFIC = {("switch_top1", 4096): 1097.1e6}
+MEASURED_FFN_TRAFFIC = {}
 
 
 def load_peaks():
@@ -246,11 +288,16 @@ class ClockSampler:
 class Layer:
     """Device buffers of one layer invocation; stages called through the C ABI."""
 
-    def __init__(self, shape, T, device, seed=0, wfmt="bf16"):
+    def __init__(self, shape, T, device, seed=0, wfmt="bf16", weights=None):
+        """weights: the weights (and router) of an earlier Layer of the same shape to reuse;
+        only the tokens are drawn then."""
         import sparse_mixture_experts_11_b200 as moe
         self.moe = moe
         self.shape, self.T, self.wfmt = shape, T, wfmt
-        if wfmt == "bf16":
+        if weights is not None:
+            self.inp = {k: v for k, v in weights.items() if k != "x"}
+            self.inp["x"] = synthetic.make_hidden(T, shape.d_model, seed=seed, device=device)
+        elif wfmt == "bf16":
             self.inp = synthetic.make_layer_inputs(shape, T, seed=seed, device=device)
         else:
             self.inp = synthetic.make_mx_layer_inputs(shape, T, wfmt, seed=seed, device=device)
@@ -561,22 +608,17 @@ def flush_l2(buf):
     torch.sum(r, dtype=torch.float32)
 
 
-def run_gpu(args, rank, world, local_rank):
-    import sparse_mixture_experts_11_b200 as moe  # fails loudly without the CUDA library
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    shape, T = parse_workload(args.workload)
-    layer = Layer(shape, T, device, wfmt=args.wfmt)
+def measure_forward(layer, steps: int, warmup: int, flush, world: int = 1, clocks=None):
+    """Warm-up, then `steps` timed whole-forward steps (one captured graph each, L2 flushed
+    before every step outside the events) and `steps` stage-by-stage steps for the breakdown.
+    Returns (per-step ms of the whole forward, mean ms per stage)."""
+    moe = layer.moe
     for call in layer.stage_calls():  # first calls set kernel attributes outside any capture
         call()
     torch.cuda.synchronize()
     layer.capture_stage_graphs()
-    flush = (torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device),
-             torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     wev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
-
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush_l2(flush)
         layer.step_full(wev)
         flush_l2(flush)
@@ -585,41 +627,112 @@ def run_gpu(args, rank, world, local_rank):
     err = moe.read_device_error(layer.fws, offset_bytes=layer.b.stage_ws - layer.fws.data_ptr())
     if err != 0:
         raise RuntimeError(f"device status after warm-up: {moe.status_string(err)}")
-
-    clocks = ClockSampler(torch.cuda.current_device())
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    for k in range(args.steps):
+    if clocks is not None:
+        clocks.start()
+    for k in range(steps):
         flush_l2(flush)
         layer.step_full(evs[k])
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    clk = clocks.stop()
+    clk = clocks.stop() if clocks is not None else None
     step_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    total_ms = sum(step_ms)
-
-    # stage breakdown: the same K steps replayed stage by stage, events between the stages
-    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    for k in range(args.steps):
+    # stage breakdown: the same number of steps replayed stage by stage, events between stages
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for k in range(steps):
         flush_l2(flush)
         layer.step_stages(sev[k])
     torch.cuda.synchronize()
     stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in sev)
                 for i, n in enumerate(["route", "permute", "grouped_ffn", "combine"])}
+    err = moe.read_device_error(layer.fws, offset_bytes=layer.b.stage_ws - layer.fws.data_ptr())
+    if err != 0:
+        raise RuntimeError(f"device status after the timed steps: {moe.status_string(err)}")
+    return step_ms, stage_ms, clk
+
+
+def routing_counts(layer):
+    counts = layer.views()["expert_count"].cpu()
+    return int(counts.sum()), int((counts > 0).sum())
+
+
+def sweep_entry(layer, spec: str, step_ms: list, stage_ms: dict, peaks: dict) -> dict:
+    shape, T = layer.shape, layer.T
+    R, active = routing_counts(layer)
+    mean_ms = statistics.mean(step_ms)
+    roof = roofline_of(shape, T, R, active, stage_ms["grouped_ffn"], mean_ms, peaks, layer.wfmt,
+                       MEASURED_FFN_TRAFFIC.get((shape.name, T)) if layer.wfmt == "bf16" else None)
+    return {"workload": spec, "T": T, "steps": len(step_ms), "ms_per_step": round(mean_ms, 4),
+            "ms_median": round(statistics.median(step_ms), 4),
+            "tokens_per_s": round(T / (mean_ms * 1e-3), 1),
+            "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "kept_rows": R, "active_experts": active, "capacity": layer.dims.capacity,
+            "ffn": roof["ffn"], "layer": roof["layer"],
+            "gpu_launches_per_step": launches_per_step(T, shape.top_k, layer.R_max,
+                                                       shape.n_experts, shape.d_model)}
+
+
+def run_sweep(args, device, flush, peaks, headline=None) -> dict:
+    """Every workload point of the five shapes (bf16 or the --wfmt expert weights), each timed
+    like the headline line; points of one shape share its weights. The headline's own entry is
+    reused. Clocks are sampled over the whole sweep."""
+    specs = SWEEP if args.sweep == "all" else tuple(x for x in args.sweep.split(",") if x)
+    out = []
+    cache = {}
+    for spec in specs:
+        shape, T = parse_workload(spec)
+        if headline is not None and (shape.name, T) == (headline[0].shape.name, headline[0].T):
+            out.append(headline[1])
+            continue
+        if cache.get("name") != shape.name:
+            cache.clear()
+            torch.cuda.empty_cache()
+            cache["name"] = shape.name
+        steps = max(args.steps, DECODE_MIN_STEPS) if T <= 64 else args.steps
+        layer = Layer(shape, T, device, wfmt=args.wfmt, weights=cache.get("weights"))
+        cache["weights"] = layer.inp
+        clocks = ClockSampler(torch.cuda.current_device())
+        step_ms, stage_ms, clk = measure_forward(layer, steps, args.warmup, flush, clocks=clocks)
+        entry = sweep_entry(layer, spec, step_ms, stage_ms, peaks)
+        entry["clocks"] = {key: clk.get(key) for key in ("sm_mhz", "sm_max_mhz", "reasons", "samples")}
+        out.append(entry)
+        del layer
+    cache.clear()
+    torch.cuda.empty_cache()
+    return {"points": out,
+            "timing": "per point: the whole forward as one captured graph, L2 flushed before "
+                      "every step; mean (and median) of the timed steps; grouped FFN from the "
+                      "stage-by-stage pass; clocks sampled over each point's timed steps"}
+
+
+def run_gpu(args, rank, world, local_rank):
+    import sparse_mixture_experts_11_b200 as moe  # fails loudly without the CUDA library
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    shape, T = parse_workload(args.workload)
+    peaks = load_peaks()
+    layer = Layer(shape, T, device, wfmt=args.wfmt)
+    flush = (torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device),
+             torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device))
+    clocks = ClockSampler(torch.cuda.current_device())
+    step_ms, stage_ms, clk = measure_forward(layer, args.steps, args.warmup, flush, world, clocks)
+    total_ms = sum(step_ms)
     ffn_ms = stage_ms["grouped_ffn"]
 
+    extras = not args.no_extras
     # router statistics and the auxiliary loss over this step's routing (a "next" row),
     # replayed as a graph K times between events
-    stats = layer.stats_timing(args.steps, flush)
+    stats = layer.stats_timing(args.steps, flush) if extras else None
     # backward pass after this forward (a "next" row); bf16 expert weights only
-    backward = layer.backward_timing(args.steps, flush, load_peaks()) if args.wfmt == "bf16" else None
+    backward = (layer.backward_timing(args.steps, flush, peaks)
+                if extras and args.wfmt == "bf16" else None)
     # overflow policy "redirect" on the same routing (a "next" row), where the batch allows it
     redirect = (layer.redirect_timing(args.steps, flush)
-                if T * shape.top_k <= moe.REDIRECT_MAX_PAIRS else None)
+                if extras and T * shape.top_k <= moe.REDIRECT_MAX_PAIRS else None)
 
     # end to end through the public call with host buffers (copies overlap neighbouring steps)
     if world > 1:
@@ -628,29 +741,14 @@ def run_gpu(args, rank, world, local_rank):
 
     total_ms, e2e_ms = reduce_max([total_ms, e2e_ms], world, device)
 
-    v = layer.views()
-    counts = v["expert_count"].cpu()
-    R = int(counts.sum())
-    active = int((counts > 0).sum())
-    ab = algorithmic_bytes(shape, T, active, R, args.wfmt)
-    peaks = load_peaks()
-    flops = ffn_flops(shape, R)
-    tensor_bound = flops / max(ab["ffn"], 1) > (peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9)
-    if tensor_bound:
-        ach = flops / (ffn_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(ach / peak, 4), "traffic": None,
-                "kernel": "grouped_ffn_kernel (gate/up and down GEMMs in one launch)",
-                "per_launch": f"{flops} FLOP", "peak_source": peaks["source"] + " sustained bf16"}
-    else:
-        ach = ab["ffn"] / (ffn_ms * 1e-3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(ach / peak, 4),
-                "traffic": MEASURED_FFN_TRAFFIC.get((shape.name, T)),
-                "kernel": "grouped_ffn_kernel (gate/up and down GEMMs in one launch)",
-                "per_launch": f"{ab['ffn']} B", "peak_source": peaks["source"] + " copy"}
+    R, active = routing_counts(layer)
+    traffic = MEASURED_FFN_TRAFFIC.get((shape.name, T)) if args.wfmt == "bf16" else None
+    roof_all = roofline_of(shape, T, R, active, ffn_ms, total_ms / args.steps, peaks, args.wfmt,
+                           traffic)
+    roof = dict(roof_all["ffn"])
+    roof["kernel"] = "grouped_ffn_kernel (gate/up and down GEMMs in one launch)"
+    headline_entry = sweep_entry(layer, f"{shape.name}:{T}", step_ms, stage_ms, peaks)
+    headline_entry["clocks"] = {key: clk.get(key) for key in ("sm_mhz", "sm_max_mhz", "reasons", "samples")}
 
     value = tokens_per_second(T, args.steps, world, total_ms)
     line = {
@@ -677,8 +775,7 @@ def run_gpu(args, rank, world, local_rank):
         "overflow_redirect": redirect,
         "backward": backward,
         "roofline": roof,
-        "layer_gbs": round(ab["layer"] / (total_ms / args.steps * 1e-3) / 1e9, 1),
-        "ffn_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 2),
+        "layer": roof_all["layer"],
         "e2e": {"value": round(tokens_per_second(T, args.steps, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * shape.d_model * 2,
                 "d2h_bytes_per_step": T * shape.d_model * 2},
@@ -686,6 +783,8 @@ def run_gpu(args, rank, world, local_rank):
                                           shape.d_model) * args.steps,
         "clocks": clk,
     }
+    if args.sweep != "none" and world == 1:
+        line["sweep"] = run_sweep(args, device, flush, peaks, headline=(layer, headline_entry))
     return line, layer
 
 
@@ -706,32 +805,33 @@ def oracle_sample(shape, T, layer_inputs_cpu, n_tokens: int):
 
 
 def cpu_inputs(shape, T, source: dict):
-    """float64 host copies of the inputs (weights converted one expert at a time, lazily)."""
-    import numpy as np
+    """float64 host copies of the inputs; expert weights converted one expert at a time, on
+    first use. source holds x, w_router, logit_bias and either the stacked expert weights
+    (w_gate_up, w_down: device or host tensors) or `expert`, a function e -> (gate_up, down)."""
     f = lambda t: None if t is None else t.detach().to("cpu", torch.float64).numpy()
-    wgu, wd = source["w_gate_up"], source["w_down"]
     cache = {}
 
-    def lazy(w, tag):
-        def get(e):
-            key = (tag, e)
-            if key not in cache:
-                cache[key] = w[e].detach().to("cpu", torch.float64).numpy()
-            return cache[key]
-        return get
+    def get(e):
+        if e not in cache:
+            if "expert" in source:
+                gu, dn = source["expert"](e)
+            else:
+                gu, dn = source["w_gate_up"][e], source["w_down"][e]
+            cache[e] = (f(gu), f(dn))
+        return cache[e]
     return {"x": f(source["x"]), "w_router": f(source["w_router"]), "logit_bias": f(source["logit_bias"]),
-            "w_gate_up": lazy(wgu, "gu"), "w_down": lazy(wd, "d"), "_cache": cache}
+            "w_gate_up": lambda e: get(e)[0], "w_down": lambda e: get(e)[1], "_cache": cache}
 
 
 def sample_tokens_for(shape, T) -> int:
-    """Tokens per oracle sample: a few seconds of float64 CPU work, and at most ~12 GB of
+    """Tokens per oracle sample: a few seconds of float64 CPU work, and at most ~6 GB of
     float64 expert weights touched (each token touches up to k experts)."""
     p = expert_params(shape.d_model, shape.d_ff, shape.act)
     by_flops = 4e10 // max(2 * shape.top_k * p, 1)
-    if min(shape.n_experts, T * shape.top_k) * p * 8 <= 12e9:
+    if min(shape.n_experts, T * shape.top_k) * p * 8 <= 6e9:
         by_mem = T
     else:
-        by_mem = 12e9 // (shape.top_k * p * 8)
+        by_mem = 6e9 // (shape.top_k * p * 8)
     return int(max(1, min(T, by_flops, by_mem)))
 
 
@@ -759,7 +859,10 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     shape, T = parse_workload(args.workload)
-    src = synthetic.make_layer_inputs(shape, T, seed=0, device="cpu")
+    # tokens and router drawn whole; each expert's weights drawn when the sample first uses it
+    src = dict(synthetic.make_router_weights(shape, seed=0, device="cpu"),
+               x=synthetic.make_hidden(T, shape.d_model, seed=0, device="cpu"),
+               expert=lambda e: synthetic.make_expert_weights(shape, e, seed=0, device="cpu"))
     inp = cpu_inputs(shape, T, src)
     n = sample_tokens_for(shape, T)
     for _ in range(args.warmup):
@@ -779,7 +882,8 @@ def run_reference(args, rank, world):
         "config": {"workload": shape.describe(T), "T": T, "sample_tokens": used},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
                          "kind": "oracle",
-                         "sample": f"float64 oracle on the first {used} of {T} tokens per step"},
+                         "sample": f"float64 oracle layer forward on the first {used} of {T} tokens "
+                                   f"per step (routing and capacity over all {T})"},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -797,6 +901,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--wfmt", choices=["bf16", "mxfp8", "mxfp4"], default="bf16",
                     help="expert weight storage (MX formats: OCP microscaling, E8M0 block scales)")
+    ap.add_argument("--sweep", default="all",
+                    help="'all' (every workload point), 'none', or a comma list of shape:T")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the router-statistics, backward and redirect timings")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -116,17 +116,35 @@ def make_layer_weights(shape: LayerShape, *, seed: int = 0, device="cpu",
     """
     dev = torch.device(device)
     N, d, F = shape.n_experts, shape.d_model, shape.d_ff
-    w_router = _normal((N, d), 1.0 / math.sqrt(d), dev, seed, _WR)
     rows = shape.gate_up_rows()
     w_gate_up = torch.empty((N, rows, d), dtype=torch.bfloat16, device=dev)
     w_down = torch.empty((N, d, F), dtype=torch.bfloat16, device=dev)
     for e in range(N):  # one expert at a time keeps the fp32 temporaries small
-        w_gate_up[e].copy_(_normal((rows, d), expert_std, dev, seed, _WGU, e))
-        w_down[e].copy_(_normal((d, F), expert_std, dev, seed, _WD, e))
-    bias = None
-    if shape.zipf_s is not None:
-        bias = zipf_logit_bias(N, shape.zipf_s).to(dev)
-    return {"w_router": w_router, "logit_bias": bias, "w_gate_up": w_gate_up, "w_down": w_down}
+        gu, dn = make_expert_weights(shape, e, seed=seed, device=dev, expert_std=expert_std)
+        w_gate_up[e].copy_(gu)
+        w_down[e].copy_(dn)
+    return {**make_router_weights(shape, seed=seed, device=dev), "w_gate_up": w_gate_up,
+            "w_down": w_down}
+
+
+def make_router_weights(shape: LayerShape, *, seed: int = 0, device="cpu") -> dict:
+    """w_router [N, d] fp32 N(0, 1/d) and the logit bias ([N] fp32 for skewed shapes, else None)."""
+    dev = torch.device(device)
+    N, d = shape.n_experts, shape.d_model
+    w_router = _normal((N, d), 1.0 / math.sqrt(d), dev, seed, _WR)
+    bias = zipf_logit_bias(N, shape.zipf_s).to(dev) if shape.zipf_s is not None else None
+    return {"w_router": w_router, "logit_bias": bias}
+
+
+def make_expert_weights(shape: LayerShape, e: int, *, seed: int = 0, device="cpu",
+                        expert_std: float = 0.02) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Expert e's packed weights alone, bf16: gate_up [2F or F, d] and down [d, F]. The same
+    values as expert e of make_layer_weights on the same device type."""
+    dev = torch.device(device)
+    d, F = shape.d_model, shape.d_ff
+    gu = _normal((shape.gate_up_rows(), d), expert_std, dev, seed, _WGU, e).to(torch.bfloat16)
+    dn = _normal((d, F), expert_std, dev, seed, _WD, e).to(torch.bfloat16)
+    return gu, dn
 
 
 def make_layer_inputs(shape: LayerShape, T: int, *, seed: int = 0, device="cpu",

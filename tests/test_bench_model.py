@@ -27,7 +27,27 @@ def test_bytes_model_switch():
     s = synthetic.SHAPES["switch_top1"]
     b = bench.algorithmic_bytes(s, 4096, 64, 4096)
     assert b["weights"] == 64 * 2 * 1024 * 4096 * 2
-    assert b["ffn"] == b["weights"] + 4096 * 1024 * 6
+    assert b["layer"] == b["weights"] + 64 * 1024 * 4 + 2 * 4096 * 1024 * 2
+    assert b["rows"] == 4096 * 1024 * 6
+
+
+def test_roofline_counting():
+    """The FFN's numerator is the active experts' weights (HBM-bound points) or the FLOPs of
+    the kept rows (tensor-bound points), against the burst bf16 peak or the copy peak."""
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1300.0,
+             "source": "test"}
+    s = synthetic.SHAPES["gpt_oss"]
+    w = 4 * 3 * 2880 * 2880 * 2
+    r = bench.roofline_of(s, 1, 4, 4, 0.05, 0.06, peaks)
+    assert r["ffn"]["bound"] == "hbm" and r["ffn"]["per_launch"] == f"{w} B"
+    assert abs(r["ffn"]["frac"] - w / 0.05e-3 / 6000e9) < 1e-4
+    lb = w + 32 * 2880 * 4 + 2 * 2880 * 2
+    assert abs(r["layer"]["frac_hbm"] - lb / 0.06e-3 / 6000e9) < 1e-4
+    m = synthetic.SHAPES["mixtral"]
+    fl = 2 * 16384 * 4096 * 14336 * 3
+    r = bench.roofline_of(m, 8192, 16384, 8, 5.0, 5.5, peaks)
+    assert r["ffn"]["bound"] == "tensor" and r["ffn"]["peak"] == 1500.0
+    assert abs(r["ffn"]["frac"] - fl / 5e-3 / 1500e12) < 1e-4
 
 
 def test_launch_counts():
