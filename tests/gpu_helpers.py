@@ -11,7 +11,13 @@ Matching rules (tolerances are written here once and used by every parity test):
   bf16 output within 2e-2 + half a bf16 ulp of the oracle value (the bf16 rounding of the exact
   answer alone can exceed 2e-2 once |out| >= 8) and mean-rel 1e-2; the MoE contribution
   (out - residual, fp32 mode) within mean-rel 1e-2 of the oracle's;
-* tokens with every choice dropped: output bits equal to the residual's bits.
+* tokens with every choice dropped: output bits equal to the residual's bits;
+* expert rows (y_perm, an fp32 intermediate the target states no bar for): max-abs within
+  2e-2 * max(1, rms of the oracle's row) and mean-rel 1e-2. The kernels round h to bf16 once
+  (2^-9 relative); summed over d_ff terms that leaves an error of about 0.17 % of the row's rms
+  (Mixtral-shaped expert, d_ff = 14336: rms(y) 2.4, largest error per 4096-element row 0.013 to
+  0.017 in a float64 simulation of that rounding alone), which a fixed 2e-2 does not cover
+  once rms(y) > 1.
 """
 from __future__ import annotations
 
@@ -31,6 +37,11 @@ OUT_MEAN_REL = 1e-2
 
 def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
+
+
+def y_row_max_abs(want_row: np.ndarray) -> float:
+    """Max-abs bar of one expert output row (see the module notes)."""
+    return OUT_MAX_ABS * max(1.0, float(np.sqrt(np.mean(np.square(want_row)))))
 
 
 def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
@@ -225,7 +236,7 @@ def check_expert_rows(run: StageRun, routing: dict, act: str, rows: np.ndarray):
         t = int(por[r]) // k
         want = oracle.expert_ffn(f64(x[t:t + 1]), gu(e), dn(e), act)[0]
         err = np.abs(y[n] - want)
-        assert err.max() <= OUT_MAX_ABS, f"row {r} (expert {e}, token {t}) max-abs {err.max()}"
+        assert err.max() <= y_row_max_abs(want), f"row {r} (expert {e}, token {t}) max-abs {err.max()}"
         assert mean_rel(y[n], want) <= OUT_MEAN_REL
 
 
