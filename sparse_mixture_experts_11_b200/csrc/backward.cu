@@ -693,8 +693,10 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const BwdGem
   }
   auto kern = bwd_gemm_kernel<A_MN, B_MN, MODE>;
   static PerDeviceOnce once;
-  const cudaError_t attr = once.run(
-      [kern] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem); });
+  const cudaError_t attr = once.run([] {
+    return cudaFuncSetAttribute(bwd_gemm_kernel<A_MN, B_MN, MODE>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  });
   if (attr != cudaSuccess) return attr;
   return launch_pdl(kern, grid, dim3(kGemmThreads), kGemmSmem, s, a, b, c, p);
 }

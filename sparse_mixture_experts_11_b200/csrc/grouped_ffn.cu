@@ -952,6 +952,15 @@ cudaError_t launch_one(const CUtensorMap& a1, const CUtensorMap& b1, const CUten
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
+  // down tiles wait for other CTAs' h counters: every CTA of the grid must be resident at once
+  int per_sm = 0;
+  const cudaError_t occ = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+      &per_sm, grouped_ffn_kernel<EPI1, BN1, BM, WFMT>, C::THREADS, C::SMEM_BYTES);
+  if (occ != cudaSuccess) return occ;
+  DeviceInfo di;
+  const cudaError_t de = device_info(&di);
+  if (de != cudaSuccess) return de;
+  if (static_cast<int64_t>(per_sm) * di.sm_count < grid) return cudaErrorInvalidConfiguration;
   return launch_pdl(grouped_ffn_kernel<EPI1, BN1, BM, WFMT>, dim3(grid), dim3(C::THREADS),
                     C::SMEM_BYTES, s, a1, b1, a2, b2, s1, s2, fp);
 }

@@ -8,6 +8,8 @@
 
 #include <mutex>
 
+#include "moe.h"
+
 namespace moe {
 
 // Launch a library kernel with programmatic stream serialisation (see pdl_wait/pdl_trigger).
@@ -218,6 +220,49 @@ struct GroupedFfnArgs {
   int64_t rows_per_expert;  // min(capacity, T)
 };
 cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s);
+
+// Expert FFN of decode-sized batches (SwiGLU, bf16 weights, T <= kDecodeFfnMaxT, so an expert
+// holds at most that many rows): the work is cut into slices of 64 columns of d_ff, each slice
+// computed whole by one CTA (its gate/up rows, the activation and its columns of W_d), and y is
+// the sum of the slices' fp32 partials, added in a fixed order after a grid-wide barrier.
+// Optionally the same launch first routes (the decode router, as moe_route does) and finally
+// combines with the residual. Every CTA of the grid must be resident at once (one per SM).
+constexpr int kDecodeFfnMaxT = 8;
+constexpr int kDecodeFfnSlice = 64;  // d_ff columns per slice
+inline bool use_decode_ffn(int64_t T, int act, int64_t r_max) {
+  return act == MOE_ACT_SWIGLU && T >= 1 && T <= kDecodeFfnMaxT && r_max > 0;
+}
+// fp32 partials: [F / 64][r_max][d]
+inline size_t decode_ffn_part_bytes(int64_t r_max, int64_t d, int64_t F) {
+  return static_cast<size_t>(F / kDecodeFfnSlice) * r_max * d * sizeof(float);
+}
+constexpr int kDecodeFfnSyncInts = 4;  // zero between calls
+
+struct DecodeFfnArgs {
+  const uint16_t* x_perm;        // [r_max, d]
+  const int32_t* expert_offset;  // [N + 1]
+  const uint16_t* w_gate_up;     // [N, 2F, d]
+  const uint16_t* w_down;        // [N, d, F]
+  uint16_t* h;                   // [r_max, F]
+  float* y_perm;                 // [r_max, d]
+  float* part;                   // decode_ffn_part_bytes()
+  int* sync;                     // kDecodeFfnSyncInts, zero between calls
+  int N, d, F, T, k;
+  int64_t r_max;
+  int* status;
+  uint64_t timeout_ns;
+  // combine (out non-null): out = residual + sum_j w_j y[row(t, j)], as moe_unpermute_combine
+  const int32_t* row_of_pair;
+  const float* topk_w;
+  const uint16_t* residual;  // may be null
+  void* out;
+  int out_f32;
+  // routing in the same launch (route_in_kernel): the decode router with its permute outputs;
+  // then x_perm and expert_offset above are the router's outputs
+  bool route_in_kernel;
+  DecodeRouteArgs route;
+};
+cudaError_t launch_decode_ffn(const DecodeFfnArgs& a, cudaStream_t s);
 
 // Backward pass (backward.cu). Saved from the forward: the routing, x_perm and y_perm.
 struct BackwardArgs {

@@ -16,78 +16,16 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "decode_route.cuh"
 #include "launch.h"
 
 namespace moe {
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
-
-__device__ __forceinline__ bool better(float av, int ae, float bv, int be) {
-  return av > bv || (av == bv && ae < be);
-}
-
-// Best (value, expert) over the warp; every lane ends with the same pair.
-__device__ __forceinline__ void warp_best(float& v, int& e) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float ov = __shfl_xor_sync(kFull, v, o);
-    const int oe = __shfl_xor_sync(kFull, e, o);
-    if (better(ov, oe, v, e)) {
-      v = ov;
-      e = oe;
-    }
-  }
-}
-
-// Top-k of one token whose N logits are spread over the warp: lane l holds experts l + 32 j.
-// Lanes r < k write choice r. NaN logits are never preferred (unspecified input, but never
-// an out-of-range expert index).
-template <int EPT>
-__device__ __forceinline__ void warp_topk_write(const float (&val)[EPT], int N, int k, int t,
-                                                int32_t* topk_idx, float* topk_w) {
-  const int lane = static_cast<int>(lane_id());
-  uint32_t taken = 0;
-  float sel_v[8];
-  int sel_e[8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    sel_v[r] = 0.f;
-    sel_e[r] = 0;
-    if (r < k) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < EPT; ++j) {
-        const int e = lane + 32 * j;
-        const float v = isnan(val[j]) ? -INFINITY : val[j];
-        if (e < N && !((taken >> j) & 1u) && better(v, e, bv, be)) {
-          bv = v;
-          be = e;
-        }
-      }
-      warp_best(bv, be);
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      sel_v[r] = bv;
-      sel_e[r] = be;
-    }
-  }
-  // renormalised weights: softmax over the chosen logits (the largest is sel_v[0])
-  float den = 0.f;
-  float num[8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    num[r] = (r < k) ? expf(sel_v[r] - sel_v[0]) : 0.f;
-    den += num[r];
-  }
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    if (r < k && lane == r) {
-      topk_idx[static_cast<int64_t>(t) * k + r] = sel_e[r];
-      topk_w[static_cast<int64_t>(t) * k + r] = num[r] / den;
-    }
-  }
-}
+using dr::better;
+using dr::kFull;
+using dr::warp_best;
+using dr::warp_topk_write;
 
 // ------------------------------------------------------------------ router (SIMT fp32)
 // One block of 1024 threads per token for small batches. g warps share each expert's dot
@@ -603,156 +541,13 @@ __global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restri
 }
 
 // ------------------------------------------------------------------ decode-sized batches
-// One launch for T <= kDecodeRouteMaxT tokens. CTA c owns d columns [128 c, 128 c + 128): lane
-// l holds 4 of them of every token's x, and warp w takes experts w, w + 8, ... one float4 of
-// W_r per lane, so W_r is read once over all CTAs. Per (token, expert) the warp adds its
-// lanes' products by a butterfly and stores the slice's partial dot product. The last CTA to
-// arrive adds the partials in order of slice (deterministic), then runs top-k per token, the
-// capacity slots in (choice, token) order and, if asked, the permutation.
-constexpr int kDrThreads = 256;
-constexpr int kDrWarps = kDrThreads / 32;
-
+// One launch for T <= kDecodeRouteMaxT tokens (see dr::decode_route_body).
 template <int TMAX, int EPT>
-__global__ void __launch_bounds__(kDrThreads) decode_route_kernel(const DecodeRouteArgs a) {
-  __shared__ float s_logit[TMAX][EPT * 32];
-  __shared__ int s_pe[TMAX * 8];    // expert of arrival p = j * T + t
-  __shared__ int s_row[TMAX * 8];   // row of arrival p, -1 if dropped
-  __shared__ int s_cnt[256];
-  __shared__ int s_off[257];
-  __shared__ int s_warp[kDrWarps];
-  __shared__ int s_last;
+__global__ void __launch_bounds__(dr::kDrThreads) decode_route_kernel(const DecodeRouteArgs a) {
+  __shared__ dr::DecodeRouteSmem<TMAX, EPT> sm;
   pdl_trigger();
   pdl_wait();
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int T = a.T, N = a.N, d = a.d, k = a.k;
-  const int c0 = blockIdx.x * kDecodeSlice + lane * 4;
-  const bool col_ok = c0 < d;
-
-  float xv[TMAX][4];
-#pragma unroll
-  for (int t = 0; t < TMAX; ++t) {
-    uint2 u = make_uint2(0u, 0u);
-    if (t < T && col_ok) u = __ldg(reinterpret_cast<const uint2*>(a.x + static_cast<int64_t>(t) * d + c0));
-    xv[t][0] = __uint_as_float(u.x << 16);
-    xv[t][1] = __uint_as_float(u.x & 0xffff0000u);
-    xv[t][2] = __uint_as_float(u.y << 16);
-    xv[t][3] = __uint_as_float(u.y & 0xffff0000u);
-  }
-  float* part = a.part + static_cast<int64_t>(blockIdx.x) * T * N;
-  for (int e0 = warp; e0 < N; e0 += 4 * kDrWarps) {
-    float4 w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {  // four experts' loads in flight before any is used
-      const int e = e0 + i * kDrWarps;
-      w[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < N && col_ok) w[i] = __ldg(reinterpret_cast<const float4*>(a.w_router + static_cast<int64_t>(e) * d + c0));
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = e0 + i * kDrWarps;
-      if (e >= N) break;  // warp-uniform
-#pragma unroll
-      for (int t = 0; t < TMAX; ++t) {
-        if (t >= T) break;  // warp-uniform
-        float acc = xv[t][0] * w[i].x;
-        acc = fmaf(xv[t][1], w[i].y, acc);
-        acc = fmaf(xv[t][2], w[i].z, acc);
-        acc = fmaf(xv[t][3], w[i].w, acc);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-        if (lane == 0) part[t * N + e] = acc;
-      }
-    }
-  }
-
-  // the last CTA to arrive finishes the routing
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(a.counter, 1) == static_cast<int>(gridDim.x) - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  const int S = gridDim.x;
-  for (int i = tid; i < T * N; i += kDrThreads) {
-    const int t = i / N, e = i - t * N;
-    float L = 0.f;
-    for (int c = 0; c < S; ++c) L += __ldcg(a.part + (static_cast<int64_t>(c) * T + t) * N + e);
-    if (a.bias != nullptr) L += a.bias[e];
-    s_logit[t][e] = L;
-    a.logits[static_cast<int64_t>(t) * N + e] = L;
-  }
-  __syncthreads();
-  for (int t = warp; t < T; t += kDrWarps) {
-    float val[EPT];
-#pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-      const int e = lane + 32 * j;
-      val[j] = (e < N) ? s_logit[t][e] : -INFINITY;
-    }
-    warp_topk_write<EPT>(val, N, k, t, a.topk_idx, a.topk_w);
-  }
-  __syncthreads();  // this block's top-k stores are visible to the whole block
-
-  const int P = T * k;  // <= 128 arrivals
-  if (tid < P) {
-    const int j = tid / T, t = tid - j * T;
-    s_pe[tid] = a.topk_idx[t * k + j];
-  }
-  __syncthreads();
-  int my_slot = -1, my_e = -1, my_q = 0;
-  if (tid < P) {
-    const int j = tid / T, t = tid - j * T;
-    my_q = t * k + j;
-    my_e = s_pe[tid];
-    int r = 0;
-    for (int p2 = 0; p2 < tid; ++p2) r += s_pe[p2] == my_e;
-    my_slot = r < a.cap ? r : -1;
-    a.slot[my_q] = my_slot;
-  }
-  for (int e = tid; e < N; e += kDrThreads) {
-    int c = 0;
-    for (int p2 = 0; p2 < P; ++p2) c += s_pe[p2] == e;
-    c = min(c, a.cap);
-    s_cnt[e] = c;
-    a.expert_count[e] = c;
-  }
-  if (a.x_perm != nullptr) {
-    __syncthreads();
-    // exclusive prefix of the kept counts (N <= 256 = blockDim.x)
-    const int v = tid < N ? s_cnt[tid] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += u;
-    }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    int base = 0;
-    for (int i = 0; i < warp; ++i) base += s_warp[i];
-    s_off[tid + 1] = base + incl;
-    if (tid == 0) s_off[0] = 0;
-    __syncthreads();
-    for (int i = tid; i <= N; i += kDrThreads) a.expert_offset[i] = s_off[i];
-    if (tid < P) {
-      const int row = my_slot >= 0 ? s_off[my_e] + my_slot : -1;
-      a.row_of_pair[my_q] = row;
-      if (row >= 0) a.pair_of_row[row] = my_q;
-      s_row[tid] = row;
-    }
-    __syncthreads();
-    const int nv = d / 8;  // 16-byte vectors per row
-    for (int i = tid; i < P * nv; i += kDrThreads) {
-      const int p2 = i / nv, vv = i - p2 * nv;
-      const int row = s_row[p2];
-      if (row < 0) continue;
-      const int t = p2 % T;
-      const uint4 val = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(t) * d)[vv];
-      reinterpret_cast<uint4*>(a.x_perm + static_cast<int64_t>(row) * d)[vv] = val;
-    }
-  }
-  if (tid == 0) *a.counter = 0;  // every CTA has arrived
+  dr::decode_route_body<TMAX, EPT>(a, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), sm);
 }
 
 }  // namespace
@@ -781,10 +576,10 @@ cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t s) {
   if (a.T <= 4)
     return launch_pdl(pick(decode_route_kernel<4, 1>, decode_route_kernel<4, 2>,
                            decode_route_kernel<4, 4>, decode_route_kernel<4, 8>),
-                      dim3(ctas), dim3(kDrThreads), 0, s, a);
+                      dim3(ctas), dim3(dr::kDrThreads), 0, s, a);
   return launch_pdl(pick(decode_route_kernel<16, 1>, decode_route_kernel<16, 2>,
                          decode_route_kernel<16, 4>, decode_route_kernel<16, 8>),
-                    dim3(ctas), dim3(kDrThreads), 0, s, a);
+                    dim3(ctas), dim3(dr::kDrThreads), 0, s, a);
 }
 
 cudaError_t launch_reroute_slots(const float* logits, uint8_t* prefs, int32_t* topk_idx,

@@ -63,11 +63,13 @@ def test_workspace_sizes():
     assert moe.workspace_bytes(big) == 256 + counters(416, 0, 0) + 32 * 256 * 4 + 3 * 256 * 7168 * 2
     decode = moe.make_dims(4, 2880, 32, 4, 2880, "swiglu", 4)
     # status word (+ the decode router's arrival counter) + counters (at most 1 + 16 m-tiles:
-    # 17 x 23 gate/up and 17 x 12 down tiles) + the larger of the decode router's partial dot
-    # products (23 slices x 4 tokens x 32 experts) and two 4-row partial slots per CTA for each
-    # GEMM (148 + 148 CTAs)
+    # 17 x 23 gate/up and 17 x 12 down tiles) + the largest of the decode router's partial dot
+    # products (23 slices x 4 tokens x 32 experts), two 4-row partial slots per CTA for each
+    # GEMM (148 + 148 CTAs) and the decode FFN's fp32 partials (45 slices of 64 d_ff columns x
+    # 16 rows x 2880)
     assert moe.workspace_bytes(decode) == (256 + counters(17, 17 * 23, 17 * 12)
-                                           + max(23 * 4 * 32 * 4, 296 * 2 * 4 * 256 * 4))
+                                           + max(23 * 4 * 32 * 4, 296 * 2 * 4 * 256 * 4,
+                                                 45 * 16 * 2880 * 4))
     fb = moe.forward_workspace_bytes(big)
     assert fb > 20480 * 7168 * 6
 
