@@ -166,8 +166,13 @@ moe_status moe_route_from_logits(const moe_dims* dims, const float* logits, int3
  * topk_idx must be the top-k of these logits as moe_route writes them: a list of each token's
  * next 16 experts after its top-k (written into the workspace by a first launch over all SMs)
  * stands in for a scan of its logits, which only runs when all 16 fail. The decisions depend
- * on each other in arrival order, so one warp then takes them in sequence (second launch).
- * MOE_ERR_UNSUPPORTED when T * k > 32768. Uses the per-stage workspace (T * 16 bytes). */
+ * on each other in arrival order, so one warp then takes them in sequence (second launch);
+ * it stops once no expert has a free slot, and every later pair stays dropped.
+ * An expert id in topk_idx outside [0, N) is reported as MOE_ERR_BOUNDS in the workspace's
+ * status word; such a pair holds no expert and may be redirected like an overflowing one.
+ * MOE_ERR_UNSUPPORTED when T * k > 163840 (every pair's serving expert is held as a byte in
+ * shared memory). Uses the per-stage workspace: T * 16 bytes of lists, T * k bytes of experts
+ * and T * k / 8 bytes of flags. */
 moe_status moe_redirect_overflow(const moe_dims* dims, const float* logits, int32_t* topk_idx,
                                  int32_t* slot, int32_t* expert_count, void* ws, size_t ws_bytes,
                                  void* stream);

@@ -233,7 +233,7 @@ def route_from_logits(dims: Dims, logits, topk_idx, topk_w, slot, expert_count, 
         _ptr(ws, "ws", torch.uint8), _nbytes(ws), _stream(stream)), "moe_route_from_logits")
 
 
-REDIRECT_MAX_PAIRS = 32768  # T * k limit of moe_redirect_overflow
+REDIRECT_MAX_PAIRS = 163840  # T * k limit of moe_redirect_overflow
 
 
 def redirect_overflow(dims: Dims, logits, topk_idx, slot, expert_count, ws, stream=None) -> None:

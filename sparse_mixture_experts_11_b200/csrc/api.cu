@@ -276,11 +276,11 @@ moe_status moe_redirect_overflow(const moe_dims* dims, const float* logits, int3
     return MOE_ERR_UNSUPPORTED;
   if (ws_bytes < stage_ws_bytes(dims)) return MOE_ERR_WORKSPACE;
   if ((st = check_device()) != MOE_OK) return st;
-  uint8_t* prefs = reinterpret_cast<uint8_t*>(shared_region_of(dims, ws));
-  return launch_status(moe::launch_reroute_slots(logits, prefs, topk_idx, slot, expert_count,
+  uint8_t* scratch = reinterpret_cast<uint8_t*>(shared_region_of(dims, ws));
+  return launch_status(moe::launch_reroute_slots(logits, scratch, topk_idx, slot, expert_count,
                                                  dims->T, dims->n_experts, dims->top_k,
                                                  std::min(dims->capacity, dims->T),
-                                                 as_stream(stream)));
+                                                 status_of(ws), as_stream(stream)));
 }
 
 moe_status moe_permute(const moe_dims* dims, const uint16_t* x, const int32_t* topk_idx,

@@ -149,16 +149,22 @@ struct DecodeRouteArgs {
 };
 cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t s);
 // Overflow policy "redirect to the next most suitable expert" (see route.cu): slots and the
-// serving experts from the router's top-k and logits, for at most kRerouteMaxPairs pairs.
-// prefs: T * kRedirectPrefs bytes of scratch, 16-byte aligned.
-constexpr int64_t kRerouteMaxPairs = 32768;
+// serving experts from the router's top-k and logits, for at most kRerouteMaxPairs pairs (the
+// sequential pass holds every pair's expert as a byte in shared memory).
+// Scratch (16-byte aligned pieces): the preference lists, T * kRedirectPrefs bytes; the pairs'
+// experts as bytes, P rounded up to 32; a bit per pair marking an expert id outside [0, N).
+constexpr int64_t kRerouteMaxPairs = 163840;
 constexpr int kRedirectPrefs = 16;
+inline size_t redirect_round16(int64_t b) { return static_cast<size_t>((b + 15) / 16 * 16); }
 inline size_t redirect_scratch_bytes(int64_t T, int k) {
-  return T * k <= kRerouteMaxPairs ? static_cast<size_t>(T) * kRedirectPrefs : 0;
+  const int64_t P = T * k;
+  if (P > kRerouteMaxPairs) return 0;
+  return redirect_round16(T * kRedirectPrefs) + static_cast<size_t>((P + 31) / 32 * 32) +
+         redirect_round16((P + 31) / 32 * 4);
 }
-cudaError_t launch_reroute_slots(const float* logits, uint8_t* prefs, int32_t* topk_idx,
+cudaError_t launch_reroute_slots(const float* logits, uint8_t* scratch, int32_t* topk_idx,
                                 int32_t* slot, int32_t* expert_count, int T, int N, int k,
-                                int capacity, cudaStream_t s);
+                                int capacity, int* status, cudaStream_t s);
 // top-k and renormalised weights from given logits
 cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, float* topk_w, int T,
                                     int N, int k, cudaStream_t s);

@@ -286,10 +286,15 @@ __global__ void __launch_bounds__(256) slot_finalize_kernel(const int32_t* __res
 // ahead of the walk, so the sequential path does not wait on global memory.
 constexpr int kRedirectRing = 2048;
 
+// Shared memory of the sequential pass: the list ring, the per-expert counts, every pair's
+// serving expert as a byte (padded to 32) and a bit per pair for ids outside [0, N).
 struct RerouteSmem {
+  static __host__ __device__ size_t ex_bytes(int P) { return static_cast<size_t>((P + 31) / 32) * 32; }
+  static __host__ __device__ size_t inv_bytes(int P) {
+    return (static_cast<size_t>((P + 31) / 32) * 4 + 15) / 16 * 16;
+  }
   static __host__ __device__ size_t bytes(int P) {
-    return static_cast<size_t>(kRedirectRing) * kRedirectPrefs + 256 * 4 +
-           static_cast<size_t>(P) * 4;
+    return static_cast<size_t>(kRedirectRing) * kRedirectPrefs + 256 * 4 + ex_bytes(P) + inv_bytes(P);
   }
 };
 
@@ -323,13 +328,47 @@ __device__ __forceinline__ unsigned lanes_with_same(int v, bool on) {
 
 // Experts ranked k .. k + kRedirectPrefs - 1 in the token's order (logit descending, equal
 // logits to the lower index, NaN as -inf), as bytes; 255 past the last expert.
+// Also, for the sequential pass: every pair's expert as a byte (ex8) with a bit per pair for
+// ids outside [0, N) (inv; such a pair is reported as MOE_ERR_BOUNDS and holds no expert), and
+// every slot set to -1, so that the pass writes only the pairs it decides.
 __global__ void __launch_bounds__(256) redirect_prefs_kernel(const float* __restrict__ logits,
-                                                             uint8_t* __restrict__ prefs, int T,
-                                                             int N, int k) {
+                                                             uint8_t* __restrict__ prefs,
+                                                             const int32_t* __restrict__ topk_idx,
+                                                             uint8_t* __restrict__ ex8,
+                                                             uint32_t* __restrict__ inv,
+                                                             int32_t* __restrict__ slot, int T,
+                                                             int N, int k, int* status) {
   pdl_wait();
   pdl_trigger();
   const int lane = static_cast<int>(lane_id());
   const int warps = gridDim.x * (blockDim.x / 32);
+  {
+    const int P = T * k;
+    const int words = (P + 31) / 32;
+    bool bad = false;
+    for (int w = blockIdx.x * blockDim.x + threadIdx.x; w < words; w += gridDim.x * blockDim.x) {
+      uint32_t bits = 0;
+      uint32_t packed[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) packed[i] = 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int q = w * 32 + i;
+        if (q >= P) break;
+        const int e = topk_idx[q];
+        const bool ok = e >= 0 && e < N;
+        bad |= !ok;
+        if (!ok) bits |= 1u << i;
+        packed[i >> 2] |= static_cast<uint32_t>(ok ? e : 0) << (8 * (i & 3));
+        slot[q] = -1;
+      }
+      uint4* dst = reinterpret_cast<uint4*>(ex8 + static_cast<int64_t>(w) * 32);
+      dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      inv[w] = bits;
+    }
+    if (bad) report_error(status, MOE_ERR_BOUNDS);
+  }
   const int rounds = min(N, k + kRedirectPrefs);
   for (int t = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; t < T; t += warps) {
     float val[8];
@@ -373,6 +412,8 @@ __device__ __forceinline__ void stage_prefs(const uint8_t* prefs, uint8_t* ring,
 
 __global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restrict__ logits,
                                                            const uint8_t* __restrict__ prefs,
+                                                           const uint8_t* __restrict__ ex8_g,
+                                                           const uint32_t* __restrict__ inv_g,
                                                            int32_t* __restrict__ topk_idx,
                                                            int32_t* __restrict__ slot,
                                                            int32_t* __restrict__ expert_count,
@@ -381,16 +422,23 @@ __global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restri
   const int P = T * k;
   uint8_t* ring = reinterpret_cast<uint8_t*>(r_sm);      // [ring][prefs]
   int* cnt = r_sm + kRedirectRing * kRedirectPrefs / 4;  // [256] filled slots
-  int* ex = cnt + 256;                                   // [P] serving experts
+  uint8_t* ex8 = reinterpret_cast<uint8_t*>(cnt + 256);  // [P] serving experts, as bytes
+  uint32_t* inv = reinterpret_cast<uint32_t*>(ex8 + RerouteSmem::ex_bytes(P));  // id outside [0, N)
   pdl_trigger();
   pdl_wait();
   const int lane = static_cast<int>(lane_id());
-  {  // the pairs (ex and topk_idx are 16-byte aligned)
-    const int p4 = P / 4;
-    for (int i = lane; i < p4; i += 32) cp_async_16(smem_u32(ex + 4 * i), topk_idx + 4 * i);
-    for (int q = 4 * p4 + lane; q < P; q += 32) cp_async_4(smem_u32(ex + q), topk_idx + q);
+  {  // the pairs' experts and invalid bits (16-byte pieces, padded in global memory alike)
+    const int n16 = static_cast<int>(RerouteSmem::ex_bytes(P) / 16);
+    for (int i = lane; i < n16; i += 32) cp_async_16(smem_u32(ex8 + 16 * i), ex8_g + 16 * i);
+    const int m16 = static_cast<int>(RerouteSmem::inv_bytes(P) / 16);
+    const uint8_t* inv_src = reinterpret_cast<const uint8_t*>(inv_g);
+    for (int i = lane; i < m16; i += 32) cp_async_16(smem_u32(inv) + 16 * i, inv_src + 16 * i);
     cp_async_commit();
   }
+  // expert serving pair q, or -1 for an id outside [0, N)
+  auto expert_of = [&](int q) -> int {
+    return ((inv[q >> 5] >> (q & 31)) & 1u) ? -1 : static_cast<int>(ex8[q]);
+  };
   constexpr int kHalf = kRedirectRing / 2;
   int filled = min(P, kHalf);  // lists of positions below `filled` are requested
   stage_prefs(prefs, ring, 0, filled, T, lane);
@@ -410,13 +458,7 @@ __global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restri
   int j = lane / T;
   int a0 = 0;           // first arrival not decided yet
   while (a0 < P) {
-    if (room == 0) {  // no free slot anywhere: the rest are dropped
-      for (int a = a0 + lane; a < P; a += 32) {
-        const int jj = a / T;
-        slot[(a - jj * T) * k + jj] = -1;
-      }
-      break;
-    }
+    if (room == 0) break;  // no free slot anywhere: the rest stay dropped (slot -1)
     if (filled < P && a0 >= filled - kHalf) {
       // the walk is past the older half: refill it with the next positions
       cp_async_wait_newest_pending();  // the group that last wrote those rows has landed
@@ -429,7 +471,7 @@ __global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restri
     const int n_act = min(32, P - a0);
     const bool act = lane < n_act;
     const int q = t * k + j;
-    const int e = act ? ex[q] : -1;
+    const int e = act ? expert_of(q) : -1;
     const bool valid = act && e >= 0 && e < N;
     const bool need = act && (!valid || cnt[e] >= cap);  // own expert full: search the list
     if (__any_sync(kFull, need) && a0 + n_act - 1 >= waited) {
@@ -449,7 +491,7 @@ __global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restri
           *reinterpret_cast<const uint4*>(ring + ((a0 + lane) % kRedirectRing) * kRedirectPrefs);
       int own[8];  // the token's current experts
 #pragma unroll
-      for (int j2 = 0; j2 < 8; ++j2) own[j2] = j2 < k ? ex[t * k + j2] : -1;
+      for (int j2 = 0; j2 < 8; ++j2) own[j2] = j2 < k ? expert_of(t * k + j2) : -1;
       const uint32_t w4[4] = {row.x, row.y, row.z, row.w};
 #pragma unroll
       for (int r = 0; r < kRedirectPrefs; ++r) {
@@ -481,7 +523,7 @@ __global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restri
       for (int i = 0; i < 8; ++i) v[i] = (lane + 32 * i < N) ? lrow[lane + 32 * i] : -INFINITY;
       int used = 0;  // bit i: expert lane + 32 i is already one of the token's
       for (int j2 = 0; j2 < k; ++j2) {
-        const int e2 = ex[t0 * k + j2];
+        const int e2 = expert_of(t0 * k + j2);
         if (e2 >= 0 && e2 < N && (e2 & 31) == lane) used |= 1 << (e2 >> 5);
       }
       float bv = -INFINITY;
@@ -505,7 +547,9 @@ __global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restri
         slot[q0] = out;
         if (out >= 0) {
           cnt[bi] = out + 1;
-          ex[q0] = bi;
+          ex8[q0] = static_cast<uint8_t>(bi);
+          inv[q0 >> 5] &= ~(1u << (q0 & 31));
+          topk_idx[q0] = bi;
         }
       }
       __syncwarp();
@@ -522,7 +566,11 @@ __global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restri
     const bool last = target >= 0 && ((same & commit) >> lane) == 1u;  // last lane on target
     if (mine) {
       slot[q] = target >= 0 ? c : -1;
-      if (target >= 0 && target != e) ex[q] = target;
+      if (target >= 0 && target != e) {  // redirected: the serving expert changes
+        ex8[q] = static_cast<uint8_t>(target);
+        if (e < 0) atomicAnd(&inv[q >> 5], ~(1u << (q & 31)));
+        topk_idx[q] = target;
+      }
       if (last) cnt[target] = c + 1;
     }
     room -= __popc(__ballot_sync(kFull, mine && last && c + 1 == cap));
@@ -536,7 +584,6 @@ __global__ void __launch_bounds__(32) reroute_slots_kernel(const float* __restri
   }
   cp_async_wait_all();
   __syncwarp();
-  for (int qq = lane; qq < P; qq += 32) topk_idx[qq] = ex[qq];
   for (int e = lane; e < N; e += 32) expert_count[e] = cnt[e];
 }
 
@@ -582,9 +629,9 @@ cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t s) {
                     dim3(ctas), dim3(dr::kDrThreads), 0, s, a);
 }
 
-cudaError_t launch_reroute_slots(const float* logits, uint8_t* prefs, int32_t* topk_idx,
+cudaError_t launch_reroute_slots(const float* logits, uint8_t* scratch, int32_t* topk_idx,
                                 int32_t* slot, int32_t* expert_count, int T, int N, int k,
-                                int capacity, cudaStream_t s) {
+                                int capacity, int* status, cudaStream_t s) {
   if (static_cast<int64_t>(T) * k > kRerouteMaxPairs || N > 256) return cudaErrorInvalidValue;
   static PerDeviceOnce once;
   const cudaError_t attr = once.run([] {
@@ -593,12 +640,17 @@ cudaError_t launch_reroute_slots(const float* logits, uint8_t* prefs, int32_t* t
         static_cast<int>(RerouteSmem::bytes(static_cast<int>(kRerouteMaxPairs))));
   });
   if (attr != cudaSuccess) return attr;
+  const int P = T * k;
+  uint8_t* prefs = scratch;
+  uint8_t* ex8 = prefs + redirect_round16(static_cast<int64_t>(T) * kRedirectPrefs);
+  uint32_t* inv = reinterpret_cast<uint32_t*>(ex8 + RerouteSmem::ex_bytes(P));
   const int blocks = std::max(1, std::min((T + 7) / 8, 4 * 148));
   cudaError_t e = launch_pdl(redirect_prefs_kernel, dim3(blocks), dim3(256), 0, s, logits, prefs,
-                             T, N, k);
+                             static_cast<const int32_t*>(topk_idx), ex8, inv, slot, T, N, k, status);
   if (e != cudaSuccess) return e;
-  return launch_pdl(reroute_slots_kernel, dim3(1), dim3(32), RerouteSmem::bytes(T * k), s, logits,
-                    static_cast<const uint8_t*>(prefs), topk_idx, slot, expert_count, T, N, k,
+  return launch_pdl(reroute_slots_kernel, dim3(1), dim3(32), RerouteSmem::bytes(P), s, logits,
+                    static_cast<const uint8_t*>(prefs), static_cast<const uint8_t*>(ex8),
+                    static_cast<const uint32_t*>(inv), topk_idx, slot, expert_count, T, N, k,
                     capacity);
 }
 

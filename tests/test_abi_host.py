@@ -185,7 +185,7 @@ def test_redirect_validation_precedes_device_use():
                                      None) == moe.ERR_UNSUPPORTED
     assert lib.moe_redirect_overflow(ctypes.byref(d), P(16), P(16), P(16), P(16), P(16), 8,
                                      None) == moe.ERR_WORKSPACE
-    big = moe.make_dims(16385, 128, 8, 2, 128, "swiglu", 4)  # T * k = 32770 pairs
+    big = moe.make_dims(20481, 128, 256, 8, 128, "swiglu", 4)  # T * k = 163848 pairs
     assert lib.moe_redirect_overflow(ctypes.byref(big), P(16), P(16), P(16), P(16), P(16), 1 << 30,
                                      None) == moe.ERR_UNSUPPORTED
-    assert moe.REDIRECT_MAX_PAIRS == 32768
+    assert moe.REDIRECT_MAX_PAIRS == 163840

@@ -235,9 +235,12 @@ def test_redirect_hand_case():
 @pytest.mark.parametrize("T,N,k,cf", [(50, 8, 2, 1.0), (33, 64, 4, 0.5), (70, 256, 8, 1.0),
                                       (2000, 16, 3, 1.0), (4096, 256, 8, 0.75), (4096, 256, 8, 8.0),
                                       (300, 4, 4, 0.5),
-                                      (64, 8, 2, 0.0)])
+                                      (64, 8, 2, 0.0),
+                                      (16384, 256, 8, 1.25), (20480, 256, 8, 40.0)])
 def test_redirect_ties(T, N, k, cf):
-    """Crafted logits with many exact ties; at T * k = 32768 the largest supported batch."""
+    """Crafted logits with many exact ties. (16384, 256, 8): the fine-grained layer's 131072
+    pairs; (20480, 256, 8) with room for every pair: 163840 pairs, the largest supported batch,
+    walked to its end."""
     rng = np.random.default_rng(7 * T + N + k)
     L = rng.integers(-3, 4, size=(T, N)).astype(np.float32) * 0.5
     cap = oracle.capacity_from_factor(cf, T, N) if cf > 0 else 0
