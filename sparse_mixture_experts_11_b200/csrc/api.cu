@@ -109,20 +109,31 @@ moe::FfnScratchPlan ffn_plan(const moe_dims* d) {
 //   [shared region: routing scratch (capacity-scan chunk totals, router weight split, the
 //    decode router's partial dot products) or,
 //    later on the stream, the grouped FFN's stream-K partial tiles]
+bool decode_ffn_for(const moe_dims* d) { return moe::use_decode_ffn(d->T, d->act, max_rows(d)); }
+
 size_t counters_bytes(const moe_dims* d) {
-  return round_up(std::max<size_t>(ffn_plan(d).counter_bytes, moe::kDecodeFfnSyncInts * sizeof(int)),
-                  256);
+  const size_t decode =
+      decode_ffn_for(d) ? moe::decode_ffn_counter_bytes(d->n_experts, d->T, d->top_k, d->d_ff) : 0;
+  return round_up(std::max(ffn_plan(d).counter_bytes, decode), 256);
 }
 
-bool decode_ffn_for(const moe_dims* d) { return moe::use_decode_ffn(d->T, d->act, max_rows(d)); }
+// The decode FFN's scratch in the shared region: after the decode router's partial dot products
+// (the launch that also routes reads them while other CTAs already store FFN partials), the
+// fp32 partials of y, then the gate/up partials passed between CTAs.
+size_t decode_ffn_part_offset(const moe_dims* d) { return decode_scratch_bytes(d); }
+size_t decode_ffn_part_gu_offset(const moe_dims* d) {
+  return decode_ffn_part_offset(d) +
+         round_up(moe::decode_ffn_part_bytes(max_rows(d), d->d_model, d->d_ff), 256);
+}
+size_t decode_ffn_scratch_bytes(const moe_dims* d) {
+  if (!decode_ffn_for(d)) return 0;
+  return decode_ffn_part_gu_offset(d) +
+         round_up(moe::decode_ffn_part_gu_bytes(d->n_experts, d->T, d->top_k, d->d_ff), 256);
+}
 
 size_t shared_region_bytes(const moe_dims* d) {
   const size_t routing = slot_scratch_bytes(d) + split_scratch_bytes(d) + decode_scratch_bytes(d);
-  const size_t ffn = round_up(std::max(ffn_plan(d).part_bytes,
-                                       decode_ffn_for(d) ? moe::decode_ffn_part_bytes(
-                                                               max_rows(d), d->d_model, d->d_ff)
-                                                         : size_t(0)),
-                              256);
+  const size_t ffn = round_up(std::max(ffn_plan(d).part_bytes, decode_ffn_scratch_bytes(d)), 256);
   const size_t stats = round_up(moe::router_stats_scratch_bytes(d->T, d->n_experts), 256);
   const size_t redirect = round_up(moe::redirect_scratch_bytes(d->T, d->top_k), 256);
   return std::max(std::max(std::max(routing, ffn), stats), redirect);
@@ -343,8 +354,11 @@ moe::DecodeFfnArgs decode_ffn_args(const moe_dims* dims, const uint16_t* x_perm,
   a.w_down = static_cast<const uint16_t*>(w.down);
   a.h = h;
   a.y_perm = y_perm;
-  a.part = reinterpret_cast<float*>(shared_region_of(dims, ws));
+  char* region = shared_region_of(dims, ws);
+  a.part = reinterpret_cast<float*>(region + decode_ffn_part_offset(dims));
+  a.part_gu = reinterpret_cast<float*>(region + decode_ffn_part_gu_offset(dims));
   a.sync = reinterpret_cast<int*>(static_cast<char*>(ws) + moe::kStatusBytes);
+  a.flags = a.sync + moe::kDecodeFfnSyncInts;
   a.N = dims->n_experts;
   a.d = dims->d_model;
   a.F = dims->d_ff;

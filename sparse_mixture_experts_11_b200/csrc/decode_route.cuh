@@ -96,22 +96,24 @@ constexpr int kDrWarps = kDrThreads / 32;
 template <int TMAX, int EPT>
 struct DecodeRouteSmem {
   float logit[TMAX][EPT * 32];
-  int pe[TMAX * 8];   // expert of arrival p = j * T + t
-  int row[TMAX * 8];  // row of arrival p, -1 if dropped
+  int tidx[TMAX * 8];  // top-k, storage order t * k + j
+  float tw[TMAX * 8];
+  int pe[TMAX * 8];    // expert of arrival p = j * T + t
+  int row[TMAX * 8];   // row of arrival p, -1 if dropped
   int cnt[256];
   int off[257];
   int warp[kDrWarps];
   int last;
 };
 
-// The work of CTA `cta` of the `ctas` CTAs that split d (all kDrThreads threads of the CTA take
-// part). Returns true in the CTA that arrived last and finished the routing; the routing's
-// outputs are then written (by this CTA's threads).
+// Phase 1: CTA `cta` of the `ctas` CTAs that split d stores its slice's partial dot products
+// and counts its arrival (all kDrThreads threads of the CTA take part). Returns true in the CTA
+// that arrived last.
 template <int TMAX, int EPT>
-__device__ __forceinline__ bool decode_route_body(const DecodeRouteArgs& a, int cta, int ctas,
-                                                  DecodeRouteSmem<TMAX, EPT>& sm) {
+__device__ __forceinline__ bool decode_route_partials(const DecodeRouteArgs& a, int cta, int ctas,
+                                                      DecodeRouteSmem<TMAX, EPT>& sm) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int T = a.T, N = a.N, d = a.d, k = a.k;
+  const int T = a.T, N = a.N, d = a.d;
   const int c0 = cta * kDecodeSlice + lane * 4;
   const bool col_ok = c0 < d;
 
@@ -151,15 +153,25 @@ __device__ __forceinline__ bool decode_route_body(const DecodeRouteArgs& a, int 
       }
     }
   }
-
-  // the last CTA to arrive finishes the routing
   __threadfence();
   __syncthreads();
   if (tid == 0) sm.last = atomicAdd(a.counter, 1) == ctas - 1;
   __syncthreads();
-  if (!sm.last) return false;
-  __threadfence();
+  return sm.last != 0;
+}
 
+// Phase 2, once every slice's partial dot products are stored: the logits (slices added in
+// order), top-k with the renormalised weights, the capacity slots in (choice, token) order, the
+// kept counts, the expert offsets and the rows of the kept pairs; all of it in shared memory
+// (sm). With `write` the CTA also stores the routing's outputs to global memory, and when the
+// permute outputs are given the offsets and row maps as well, with the x_perm copy unless
+// copy_rows is false.
+template <int TMAX, int EPT>
+__device__ __forceinline__ void decode_route_finish(const DecodeRouteArgs& a, int ctas,
+                                                    DecodeRouteSmem<TMAX, EPT>& sm, bool write,
+                                                    bool copy_rows = true) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = a.T, N = a.N, d = a.d, k = a.k;
   const int S = ctas;
   for (int i = tid; i < T * N; i += kDrThreads) {
     const int t = i / N, e = i - t * N;
@@ -186,7 +198,7 @@ __device__ __forceinline__ bool decode_route_body(const DecodeRouteArgs& a, int 
     }
     if (a.bias != nullptr) L += a.bias[e];
     sm.logit[t][e] = L;
-    a.logits[static_cast<int64_t>(t) * N + e] = L;
+    if (write) a.logits[static_cast<int64_t>(t) * N + e] = L;
   }
   __syncthreads();
   for (int t = warp; t < T; t += kDrWarps) {
@@ -196,14 +208,18 @@ __device__ __forceinline__ bool decode_route_body(const DecodeRouteArgs& a, int 
       const int e = lane + 32 * j;
       val[j] = (e < N) ? sm.logit[t][e] : -INFINITY;
     }
-    warp_topk_write<EPT>(val, N, k, t, a.topk_idx, a.topk_w);
+    warp_topk_write<EPT>(val, N, k, t, sm.tidx, sm.tw);
   }
-  __syncthreads();  // this block's top-k stores are visible to the whole block
+  __syncthreads();
 
-  const int P = T * k;  // <= 128 arrivals
+  const int P = T * k;  // <= 8 * TMAX arrivals
   if (tid < P) {
     const int j = tid / T, t = tid - j * T;
-    sm.pe[tid] = a.topk_idx[t * k + j];
+    sm.pe[tid] = sm.tidx[t * k + j];
+    if (write) {
+      a.topk_idx[t * k + j] = sm.tidx[t * k + j];
+      a.topk_w[t * k + j] = sm.tw[t * k + j];
+    }
   }
   __syncthreads();
   int my_slot = -1, my_e = -1, my_q = 0;
@@ -214,40 +230,44 @@ __device__ __forceinline__ bool decode_route_body(const DecodeRouteArgs& a, int 
     int r = 0;
     for (int p2 = 0; p2 < tid; ++p2) r += sm.pe[p2] == my_e;
     my_slot = r < a.cap ? r : -1;
-    a.slot[my_q] = my_slot;
+    if (write) a.slot[my_q] = my_slot;
   }
   for (int e = tid; e < N; e += kDrThreads) {
     int c = 0;
     for (int p2 = 0; p2 < P; ++p2) c += sm.pe[p2] == e;
     c = min(c, a.cap);
     sm.cnt[e] = c;
-    a.expert_count[e] = c;
+    if (write) a.expert_count[e] = c;
   }
-  if (a.x_perm != nullptr) {
-    __syncthreads();
-    // exclusive prefix of the kept counts (N <= 256 = blockDim.x)
-    const int v = tid < N ? sm.cnt[tid] : 0;
-    int incl = v;
+  __syncthreads();
+  // exclusive prefix of the kept counts (N <= 256 = blockDim.x)
+  const int v = tid < N ? sm.cnt[tid] : 0;
+  int incl = v;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += u;
-    }
-    if (lane == 31) sm.warp[warp] = incl;
-    __syncthreads();
-    int base = 0;
-    for (int i = 0; i < warp; ++i) base += sm.warp[i];
-    sm.off[tid + 1] = base + incl;
-    if (tid == 0) sm.off[0] = 0;
-    __syncthreads();
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) sm.warp[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int i = 0; i < warp; ++i) base += sm.warp[i];
+  sm.off[tid + 1] = base + incl;
+  if (tid == 0) sm.off[0] = 0;
+  __syncthreads();
+  const bool permute = write && a.x_perm != nullptr;
+  if (permute)
     for (int i = tid; i <= N; i += kDrThreads) a.expert_offset[i] = sm.off[i];
-    if (tid < P) {
-      const int row = my_slot >= 0 ? sm.off[my_e] + my_slot : -1;
+  if (tid < P) {
+    const int row = my_slot >= 0 ? sm.off[my_e] + my_slot : -1;
+    if (permute) {
       a.row_of_pair[my_q] = row;
       if (row >= 0) a.pair_of_row[row] = my_q;
-      sm.row[tid] = row;
     }
-    __syncthreads();
+    sm.row[tid] = row;
+  }
+  __syncthreads();
+  if (permute && copy_rows) {
     const int nv = d / 8;  // 16-byte vectors per row
     for (int i = tid; i < P * nv; i += kDrThreads) {
       const int p2 = i / nv, vv = i - p2 * nv;
@@ -258,10 +278,7 @@ __device__ __forceinline__ bool decode_route_body(const DecodeRouteArgs& a, int 
       reinterpret_cast<uint4*>(a.x_perm + static_cast<int64_t>(row) * d)[vv] = val;
     }
   }
-  if (tid == 0) *a.counter = 0;  // every CTA has arrived
-  return true;
 }
-
 
 }  // namespace dr
 }  // namespace moe

@@ -234,15 +234,28 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s);
 // Optionally the same launch first routes (the decode router, as moe_route does) and finally
 // combines with the residual. Every CTA of the grid must be resident at once (one per SM).
 constexpr int kDecodeFfnMaxT = 8;
-constexpr int kDecodeFfnSlice = 64;  // d_ff columns per slice
+constexpr int kDecodeFfnMaxRows = 8;  // rows per expert: at most T
+constexpr int kDecodeFfnSlice = 64;   // d_ff columns per slice
 inline bool use_decode_ffn(int64_t T, int act, int64_t r_max) {
   return act == MOE_ACT_SWIGLU && T >= 1 && T <= kDecodeFfnMaxT && r_max > 0;
 }
-// fp32 partials: [F / 64][r_max][d]
+// slices at most: the experts that can hold rows times F / 64
+inline int64_t decode_ffn_max_slices(int64_t N, int64_t T, int64_t k, int64_t F) {
+  return (N < T * k ? N : T * k) * (F / kDecodeFfnSlice);
+}
+// Scratch: fp32 partials of y [F / 64][r_max][d], then the gate/up partials a slice's owner
+// receives from the CTA before it [max slices][8][128] fp32 (one per slice)
 inline size_t decode_ffn_part_bytes(int64_t r_max, int64_t d, int64_t F) {
   return static_cast<size_t>(F / kDecodeFfnSlice) * r_max * d * sizeof(float);
 }
-constexpr int kDecodeFfnSyncInts = 4;  // zero between calls
+inline size_t decode_ffn_part_gu_bytes(int64_t N, int64_t T, int64_t k, int64_t F) {
+  return static_cast<size_t>(decode_ffn_max_slices(N, T, k, F)) * kDecodeFfnMaxRows * 128 * sizeof(float);
+}
+// Counters, zero between calls: grid-barrier arrivals and departures, then two flags per slice
+constexpr int kDecodeFfnSyncInts = 4;
+inline size_t decode_ffn_counter_bytes(int64_t N, int64_t T, int64_t k, int64_t F) {
+  return static_cast<size_t>(kDecodeFfnSyncInts + 2 * decode_ffn_max_slices(N, T, k, F)) * sizeof(int);
+}
 
 struct DecodeFfnArgs {
   const uint16_t* x_perm;        // [r_max, d]
@@ -252,7 +265,9 @@ struct DecodeFfnArgs {
   uint16_t* h;                   // [r_max, F]
   float* y_perm;                 // [r_max, d]
   float* part;                   // decode_ffn_part_bytes()
+  float* part_gu;                // decode_ffn_part_gu_bytes()
   int* sync;                     // kDecodeFfnSyncInts, zero between calls
+  int* flags;                    // 2 * decode_ffn_max_slices(), zero between calls
   int N, d, F, T, k;
   int64_t r_max;
   int* status;

@@ -594,7 +594,11 @@ __global__ void __launch_bounds__(dr::kDrThreads) decode_route_kernel(const Deco
   __shared__ dr::DecodeRouteSmem<TMAX, EPT> sm;
   pdl_trigger();
   pdl_wait();
-  dr::decode_route_body<TMAX, EPT>(a, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), sm);
+  const int ctas = static_cast<int>(gridDim.x);
+  if (!dr::decode_route_partials<TMAX, EPT>(a, static_cast<int>(blockIdx.x), ctas, sm)) return;
+  __threadfence();
+  dr::decode_route_finish<TMAX, EPT>(a, ctas, sm, true);  // the last CTA to arrive
+  if (threadIdx.x == 0) *a.counter = 0;  // every CTA has arrived
 }
 
 }  // namespace

@@ -62,14 +62,18 @@ def test_workspace_sizes():
     # three-term split of W_r that the tensor-core router reads
     assert moe.workspace_bytes(big) == 256 + counters(416, 0, 0) + 32 * 256 * 4 + 3 * 256 * 7168 * 2
     decode = moe.make_dims(4, 2880, 32, 4, 2880, "swiglu", 4)
-    # status word (+ the decode router's arrival counter) + counters (at most 1 + 16 m-tiles:
-    # 17 x 23 gate/up and 17 x 12 down tiles) + the largest of the decode router's partial dot
-    # products (23 slices x 4 tokens x 32 experts), two 4-row partial slots per CTA for each
-    # GEMM (148 + 148 CTAs) and the decode FFN's fp32 partials (45 slices of 64 d_ff columns x
-    # 16 rows x 2880)
-    assert moe.workspace_bytes(decode) == (256 + counters(17, 17 * 23, 17 * 12)
-                                           + max(23 * 4 * 32 * 4, 296 * 2 * 4 * 256 * 4,
-                                                 45 * 16 * 2880 * 4))
+    # status word (+ the decode router's arrival counter) + the larger of the grouped FFN's
+    # counters (at most 1 + 16 m-tiles: 17 x 23 gate/up and 17 x 12 down tiles) and the decode
+    # FFN's (4 + two flags for each of 16 experts x 45 slices) + the larger of the grouped FFN's
+    # two 4-row partial slots per CTA for each GEMM (148 + 148 CTAs) and the decode FFN's
+    # scratch: the decode router's partial dot products (23 slices x 4 tokens x 32 experts), the
+    # fp32 partials of y (45 slices of 64 d_ff columns x 16 rows x 2880) and a gate/up partial
+    # of 8 x 128 fp32 per slice
+    decode_counters = -(-((4 + 2 * 16 * 45) * 4) // 256) * 256
+    assert moe.workspace_bytes(decode) == (256 + max(counters(17, 17 * 23, 17 * 12), decode_counters)
+                                           + max(296 * 2 * 4 * 256 * 4,
+                                                 23 * 4 * 32 * 4 + 45 * 16 * 2880 * 4
+                                                 + 16 * 45 * 8 * 128 * 4))
     fb = moe.forward_workspace_bytes(big)
     assert fb > 20480 * 7168 * 6
 
