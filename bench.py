@@ -373,6 +373,43 @@ class Layer:
                 "dropped_pairs": int(dropped.item()), "algorithmic_bytes": nbytes,
                 "achieved_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
 
+    def route_stats_timing(self, steps: int, flush) -> dict:
+        """The route stage alone (moe_route) and with the router statistics emitted by the
+        routing launches (moe_route_with_stats), each a captured graph replayed between events
+        with L2 flushed before every call: mean ms of each and the difference."""
+        moe, i, b, v = self.moe, self.inp, self.b, self.views()
+        N = self.shape.n_experts
+        dev = i["x"].device
+        picks = torch.empty((N,), dtype=torch.int32, device=dev)
+        pm = torch.empty((N,), dtype=torch.float32, device=dev)
+        aux = torch.empty((1,), dtype=torch.float32, device=dev)
+        dropped = torch.empty((1,), dtype=torch.int32, device=dev)
+        plain = self.stage_calls()[0]
+
+        def fused():
+            moe.route_with_stats(self.dims, i["x"], i["w_router"], i["logit_bias"], v["logits"],
+                                 v["topk_idx"], v["topk_w"], v["slot"], v["expert_count"], picks,
+                                 pm, aux, dropped, v["stage_ws"], alpha=0.01)
+        out = {}
+        for name, call in (("route_ms", plain), ("route_with_stats_ms", fused)):
+            call()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                call()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)]
+            for e0, e1 in evs:
+                flush_l2(flush)
+                e0.record()
+                g.replay()
+                e1.record()
+            torch.cuda.synchronize()
+            out[name] = round(statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs), 4)
+        out["added_us"] = round((out["route_with_stats_ms"] - out["route_ms"]) * 1e3, 2)
+        out["aux_loss"] = round(float(aux.item()), 6)
+        return out
+
     def backward_timing(self, steps: int, flush, peaks: dict) -> dict:
         """moe_backward after this layer's forward (bf16 weights): mean ms per call of the
         captured backward between events, with L2 flushed before each call. FLOPs are the five
@@ -736,6 +773,8 @@ def run_gpu(args, rank, world, local_rank):
     # router statistics and the auxiliary loss over this step's routing (a "next" row),
     # replayed as a graph K times between events
     stats = layer.stats_timing(args.steps, flush) if extras else None
+    # the same statistics emitted by the routing launches themselves
+    fused_stats = layer.route_stats_timing(args.steps, flush) if extras else None
     # backward pass after this forward (a "next" row); bf16 expert weights only
     backward = (layer.backward_timing(args.steps, flush, peaks)
                 if extras and args.wfmt == "bf16" else None)
@@ -781,6 +820,7 @@ def run_gpu(args, rank, world, local_rank):
                              "steps replayed as one graph per stage with events between stages"},
         "stages_ms": {k: round(v_, 4) for k, v_ in stage_ms.items()},
         "router_stats": stats,
+        "route_with_stats": fused_stats,
         "overflow_redirect": redirect,
         "backward": backward,
         "roofline": roof,

@@ -149,6 +149,25 @@ moe_status moe_route_from_logits(const moe_dims* dims, const float* logits, int3
                                  float* topk_w, int32_t* slot, int32_t* expert_count, void* ws,
                                  size_t ws_bytes, void* stream);
 
+/* moe_route_with_stats: moe_route that also emits the router statistics of moe_router_stats
+ * from the routing launches themselves (page «Sparse Mixture-of-Experts», section «Маршрутизация
+ * токена и auxiliary loss»): the router writes per-tile sums of its softmax probabilities while
+ * the logits are still on chip, and the capacity pass, which counts each expert's picks, adds
+ * them in a fixed order. Decode-sized batches form the statistics in the one routing launch.
+ * Inputs and routing outputs are those of moe_route; the statistics are those of
+ * moe_router_stats:
+ *   picks      [N] int32    (token, choice) pairs that chose expert e, before the capacity
+ *   prob_mean  [N] fp32     P_e, the batch mean of the router's softmax probability of e
+ *   aux_loss   [1] fp32     alpha * N * sum_e (picks_e / T) * P_e (alpha = 1e-2 on the page)
+ *   dropped    [1] int32    pairs over the capacity
+ * The sums are deterministic; their order differs from moe_router_stats', so the fp32 results
+ * may differ from it in the last bits. Uses the per-stage workspace (moe_workspace_bytes). */
+moe_status moe_route_with_stats(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                                const float* logit_bias, float* logits, int32_t* topk_idx,
+                                float* topk_w, int32_t* slot, int32_t* expert_count, float alpha,
+                                int32_t* picks, float* prob_mean, float* aux_loss,
+                                int32_t* dropped, void* ws, size_t ws_bytes, void* stream);
+
 /* Overflow policy "redirect": a pair that arrives at a full expert goes to the next most
  * suitable expert instead of being dropped (page «Архитектура MoE в больших языковых моделях —
  * кто такие «эксперты»?», section «Как работает MoE: принцип маршрутизации», which names

@@ -73,6 +73,8 @@ _SIGS = {
     "moe_workspace_init": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "moe_route": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_route_from_logits": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_route_with_stats": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float,
+                                            _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_redirect_overflow": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_permute": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_grouped_ffn": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -221,6 +223,23 @@ def route_noalloc(dims: Dims, x, w_router, logit_bias, logits, topk_idx, topk_w,
         _ptr(logits, "logits", torch.float32, (T, N)), _ptr(topk_idx, "topk_idx", torch.int32, (T, k)),
         _ptr(topk_w, "topk_w", torch.float32, (T, k)), _ptr(slot, "slot", torch.int32, (T, k)),
         _ptr(expert_count, "expert_count", torch.int32, (N,)), _stream(stream)), "moe_route_noalloc")
+
+
+def route_with_stats(dims: Dims, x, w_router, logit_bias, logits, topk_idx, topk_w, slot,
+                     expert_count, picks, prob_mean, aux_loss, dropped, ws, alpha=0.01,
+                     stream=None) -> None:
+    """moe_route with the router statistics emitted by the routing launches."""
+    T, d, N, k = dims.T, dims.d_model, dims.n_experts, dims.top_k
+    _check(_lib.moe_route_with_stats(
+        ctypes.byref(dims), _ptr(x, "x", torch.bfloat16, (T, d)),
+        _ptr(w_router, "w_router", torch.float32, (N, d)),
+        _ptr(logit_bias, "logit_bias", torch.float32, (N,), allow_none=True),
+        _ptr(logits, "logits", torch.float32, (T, N)), _ptr(topk_idx, "topk_idx", torch.int32, (T, k)),
+        _ptr(topk_w, "topk_w", torch.float32, (T, k)), _ptr(slot, "slot", torch.int32, (T, k)),
+        _ptr(expert_count, "expert_count", torch.int32, (N,)), ctypes.c_float(alpha),
+        _ptr(picks, "picks", torch.int32, (N,)), _ptr(prob_mean, "prob_mean", torch.float32, (N,)),
+        _ptr(aux_loss, "aux_loss", torch.float32, (1,)), _ptr(dropped, "dropped", torch.int32, (1,)),
+        _ptr(ws, "ws", torch.uint8), _nbytes(ws), _stream(stream)), "moe_route_with_stats")
 
 
 def route_from_logits(dims: Dims, logits, topk_idx, topk_w, slot, expert_count, ws,

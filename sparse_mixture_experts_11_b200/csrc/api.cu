@@ -131,8 +131,18 @@ size_t decode_ffn_scratch_bytes(const moe_dims* d) {
          round_up(moe::decode_ffn_part_gu_bytes(d->n_experts, d->T, d->top_k, d->d_ff), 256);
 }
 
+// Router statistics emitted by the routing launches: the router's per-tile probability sums,
+// after the routing scratch (both are live during the same call).
+size_t route_stats_bytes(const moe_dims* d) {
+  if (d->T == 0 || moe::use_decode_route(d->T, d->n_experts, d->d_model)) return 0;
+  return round_up(static_cast<size_t>(moe::route_stats_parts(d->T, d->n_experts, d->d_model)) *
+                      d->n_experts * sizeof(float),
+                  256);
+}
+
 size_t shared_region_bytes(const moe_dims* d) {
-  const size_t routing = slot_scratch_bytes(d) + split_scratch_bytes(d) + decode_scratch_bytes(d);
+  const size_t routing = slot_scratch_bytes(d) + split_scratch_bytes(d) + decode_scratch_bytes(d) +
+                         route_stats_bytes(d);
   const size_t ffn = round_up(std::max(ffn_plan(d).part_bytes, decode_ffn_scratch_bytes(d)), 256);
   const size_t stats = round_up(moe::router_stats_scratch_bytes(d->T, d->n_experts), 256);
   const size_t redirect = round_up(moe::redirect_scratch_bytes(d->T, d->top_k), 256);
@@ -252,6 +262,54 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const float* w_rou
                                              moe::wait_timeout_ns(), s));
   if (st != MOE_OK) return st;
   return route_slots(dims, topk_idx, slot, expert_count, ws, s);
+}
+
+moe_status moe_route_with_stats(const moe_dims* dims, const uint16_t* x, const float* w_router,
+                                const float* logit_bias, float* logits, int32_t* topk_idx,
+                                float* topk_w, int32_t* slot, int32_t* expert_count, float alpha,
+                                int32_t* picks, float* prob_mean, float* aux_loss,
+                                int32_t* dropped, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (dims->T == 0) return MOE_OK;
+  if (!x || !w_router || !logits || !topk_idx || !topk_w || !slot || !expert_count || !ws ||
+      !picks || !prob_mean || !aux_loss || !dropped)
+    return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(logits) || !aligned16(topk_idx) ||
+      !aligned16(topk_w) || !aligned16(slot) || !aligned16(expert_count) || !aligned16(ws) ||
+      !aligned16(picks) || !aligned16(prob_mean) || (logit_bias && !aligned16(logit_bias)))
+    return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < stage_ws_bytes(dims)) return MOE_ERR_WORKSPACE;
+  if ((st = check_device()) != MOE_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  if (moe::use_decode_route(dims->T, dims->n_experts, dims->d_model)) {
+    moe::DecodeRouteArgs a = decode_route_args(dims, x, w_router, logit_bias, logits, topk_idx,
+                                               topk_w, slot, expert_count, ws);
+    a.st_picks = picks;
+    a.st_prob_mean = prob_mean;
+    a.st_aux_loss = aux_loss;
+    a.st_dropped = dropped;
+    a.st_alpha = alpha;
+    return launch_status(moe::launch_decode_route(a, s));
+  }
+  moe::RouteStats rs{};
+  rs.prob_part = reinterpret_cast<float*>(shared_region_of(dims, ws) + slot_scratch_bytes(dims) +
+                                          split_scratch_bytes(dims) + decode_scratch_bytes(dims));
+  rs.n_parts = moe::route_stats_parts(dims->T, dims->n_experts, dims->d_model);
+  rs.alpha = alpha;
+  rs.picks = picks;
+  rs.prob_mean = prob_mean;
+  rs.aux_loss = aux_loss;
+  rs.dropped = dropped;
+  st = launch_status(moe::launch_router_topk(x, w_router, logit_bias, logits, topk_idx, topk_w,
+                                             dims->T, dims->d_model, dims->n_experts,
+                                             dims->top_k, split_scratch_of(dims, ws), status_of(ws),
+                                             moe::wait_timeout_ns(), s, rs.prob_part));
+  if (st != MOE_OK) return st;
+  int32_t* scratch = reinterpret_cast<int32_t*>(shared_region_of(dims, ws));
+  return launch_status(moe::launch_capacity_slots(topk_idx, slot, expert_count, scratch, dims->T,
+                                                  dims->n_experts, dims->top_k,
+                                                  std::min(dims->capacity, dims->T), s, &rs));
 }
 
 moe_status moe_route_from_logits(const moe_dims* dims, const float* logits, int32_t* topk_idx,

@@ -104,6 +104,7 @@ struct DecodeRouteSmem {
   int off[257];
   int warp[kDrWarps];
   int last;
+  float term[256];  // router statistics: (picks_e / T) * P_e
 };
 
 // Phase 1: CTA `cta` of the `ctas` CTAs that split d stores its slice's partial dot products
@@ -232,14 +233,62 @@ __device__ __forceinline__ void decode_route_finish(const DecodeRouteArgs& a, in
     my_slot = r < a.cap ? r : -1;
     if (write) a.slot[my_q] = my_slot;
   }
+  const bool stats = write && a.st_picks != nullptr;
+  if (stats) {
+    // router statistics: each token's softmax over the experts, in place of its logits (they
+    // are stored and no longer needed), warp per token
+    for (int t = warp; t < T; t += kDrWarps) {
+      float v[EPT];
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < EPT; ++j) {
+        const int e = lane + 32 * j;
+        v[j] = e < N ? sm.logit[t][e] : -INFINITY;
+        m = fmaxf(m, v[j]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < EPT; ++j) {
+        v[j] = (lane + 32 * j) < N ? expf(v[j] - m) : 0.f;
+        sum += v[j];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
+      const float inv = 1.0f / sum;
+#pragma unroll
+      for (int j = 0; j < EPT; ++j)
+        if (lane + 32 * j < N) sm.logit[t][lane + 32 * j] = v[j] * inv;
+    }
+    __syncthreads();
+  }
   for (int e = tid; e < N; e += kDrThreads) {
     int c = 0;
     for (int p2 = 0; p2 < P; ++p2) c += sm.pe[p2] == e;
+    if (stats) {  // picks before the capacity; P_e, the batch mean of the probability
+      float sum = 0.f;
+      for (int t = 0; t < T; ++t) sum += sm.logit[t][e];
+      const float Pe = sum / static_cast<float>(T);
+      a.st_picks[e] = c;
+      a.st_prob_mean[e] = Pe;
+      sm.term[e] = (static_cast<float>(c) / static_cast<float>(T)) * Pe;
+    }
     c = min(c, a.cap);
     sm.cnt[e] = c;
     if (write) a.expert_count[e] = c;
   }
   __syncthreads();
+  if (stats && tid == 0) {
+    float total = 0.f;
+    int kept = 0;
+    for (int e = 0; e < N; ++e) {
+      total += sm.term[e];
+      kept += sm.cnt[e];
+    }
+    *a.st_aux_loss = a.st_alpha * static_cast<float>(N) * total;
+    *a.st_dropped = P - kept;
+  }
   // exclusive prefix of the kept counts (N <= 256 = blockDim.x)
   const int v = tid < N ? sm.cnt[tid] : 0;
   int incl = v;

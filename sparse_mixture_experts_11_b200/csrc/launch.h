@@ -100,17 +100,38 @@ inline bool router_uses_tensor_cores(int64_t T, int64_t N, int64_t d) {
 // Bytes of the [3][N][d] bf16 split of W_r the tensor-core router reads when given scratch.
 size_t router_split_bytes(int N, int d);
 
+// Router statistics emitted by the routing launches (moe_route_with_stats). The router writes
+// per-tile sums of its softmax probabilities, prob_part [n_parts][N] (the tensor-core router:
+// one row per 128-token tile, or per CTA of a tile split over a cluster; the per-token router:
+// one row per token); the capacity pass, which counts each expert's picks before the
+// capacity, adds the rows in order and forms the outputs. prob_part null: no statistics.
+struct RouteStats {
+  float* prob_part;
+  int n_parts;
+  float alpha;
+  int32_t* picks;     // [N] pairs that chose each expert
+  float* prob_mean;   // [N] mean router probability
+  float* aux_loss;    // alpha * N * sum_e (picks_e / T) * prob_mean_e
+  int32_t* dropped;   // pairs over the capacity
+};
+// partial rows the router writes: the tensor-core router's (tiles x cluster size) or T
+int router_tc_parts(int T, int d);
+inline int route_stats_parts(int64_t T, int64_t N, int64_t d) {
+  return router_uses_tensor_cores(T, N, d) ? router_tc_parts(static_cast<int>(T), static_cast<int>(d))
+                                           : static_cast<int>(T);
+}
+
 // router: logits = x W_r^T (+ b), then top-k and renormalised weights. status may be null.
 // split_scratch: router_split_bytes() of device memory for the tensor-core path, or null to
-// split W_r inside the router kernel (same results, slower).
+// split W_r inside the router kernel (same results, slower). prob_part: see RouteStats.
 cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const float* bias,
                                float* logits, int32_t* topk_idx, float* topk_w, int T, int d,
                                int N, int k, uint16_t* split_scratch, int* status,
-                               uint64_t timeout_ns, cudaStream_t s);
+                               uint64_t timeout_ns, cudaStream_t s, float* prob_part = nullptr);
 cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const float* bias,
                              float* logits, int32_t* topk_idx, float* topk_w, int T, int d, int N,
                              int k, uint16_t* split_scratch, int* status, uint64_t timeout_ns,
-                             cudaStream_t s);
+                             float* prob_part, cudaStream_t s);
 // Decode-sized batches (T <= kDecodeRouteMaxT) route in one launch: CTA c takes columns
 // [128 c, 128 c + 128) of d for every token and expert and stores partial dot products; the
 // last CTA to finish (arrival counter, zero between calls) adds them in order of c, then takes
@@ -146,6 +167,13 @@ struct DecodeRouteArgs {
   float* part;    // decode_route_scratch_bytes()
   int* counter;   // zero between calls
   int T, d, N, k, cap;
+  // router statistics (moe_route_with_stats), formed by the CTA that finishes the routing;
+  // picks null: none
+  int32_t* st_picks;
+  float* st_prob_mean;
+  float* st_aux_loss;
+  int32_t* st_dropped;
+  float st_alpha;
 };
 cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t s);
 // Overflow policy "redirect to the next most suitable expert" (see route.cu): slots and the
@@ -171,7 +199,7 @@ cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, floa
 // capacity slots in (choice, token) arrival order
 cudaError_t launch_capacity_slots(const int32_t* topk_idx, int32_t* slot, int32_t* expert_count,
                                   int32_t* chunk_scratch, int T, int N, int k, int capacity,
-                                  cudaStream_t s);
+                                  cudaStream_t s, const RouteStats* stats = nullptr);
 // sort kept pairs into expert-contiguous rows
 cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, const int32_t* slot,
                            const int32_t* expert_count, int32_t* expert_offset,

@@ -41,7 +41,7 @@ template <int EPT>
 __global__ void __launch_bounds__(kTokThreads) router_token_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias,
     float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int T,
-    int d, int N, int k) {
+    int d, int N, int k, float* __restrict__ prob_part) {
   __shared__ float s_part[kTokWarps][EPT];  // [warp][pass]: at most EPT passes of 32 experts
   __shared__ float s_logit[EPT * 32];
   pdl_trigger();
@@ -94,6 +94,32 @@ __global__ void __launch_bounds__(kTokThreads) router_token_kernel(
       val[j] = (e < N) ? s_logit[e] : -INFINITY;
     }
     warp_topk_write<EPT>(val, N, k, t, topk_idx, topk_w);
+  } else if (warp == 1 && prob_part != nullptr) {
+    // router statistics: this token's softmax over the experts, one row per token
+    float v[EPT];
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = lane + 32 * j;
+      v[j] = e < N ? s_logit[e] : -INFINITY;
+      m = fmaxf(m, v[j]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      v[j] = (lane + 32 * j) < N ? expf(v[j] - m) : 0.f;
+      sum += v[j];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
+    const float inv = 1.0f / sum;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = lane + 32 * j;
+      if (e < N) prob_part[static_cast<int64_t>(t) * N + e] = v[j] * inv;
+    }
   }
 }
 
@@ -146,11 +172,50 @@ constexpr int kSlThreads = 256;
 constexpr int kSlWarps = kSlThreads / 32;
 constexpr int kSlIters = kSlotChunk / kSlThreads;  // arrivals per lane
 
+// Router statistics from the picks each expert got before the capacity (run, shared memory) and
+// the router's partial rows of probability sums, added in row order (page «Sparse
+// Mixture-of-Experts», «Маршрутизация токена и auxiliary loss»: alpha * N * sum_i f_i * P_i with
+// f_i = picks_i / T and P_i the batch mean of the router's probability for expert i). One block;
+// s_term holds 256 floats of shared memory.
+__device__ __forceinline__ void route_stats_finish(const RouteStats& st, const int* run, int T,
+                                                   int N, int cap, float* s_term) {
+  for (int e = threadIdx.x; e < 256; e += blockDim.x) s_term[e] = 0.f;
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    float sum = 0.f;
+    int b = 0;
+    for (; b + 8 <= st.n_parts; b += 8) {  // eight independent loads in flight per step
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __ldcg(st.prob_part + static_cast<int64_t>(b + i) * N + e);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum += v[i];
+    }
+    for (; b < st.n_parts; ++b) sum += __ldcg(st.prob_part + static_cast<int64_t>(b) * N + e);
+    const float P = sum / static_cast<float>(T);
+    st.prob_mean[e] = P;
+    st.picks[e] = run[e];
+    s_term[e] = (static_cast<float>(run[e]) / static_cast<float>(T)) * P;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float total = 0.f;
+    int dropped = 0;
+    for (int e = 0; e < N; ++e) {
+      total += s_term[e];
+      dropped += max(0, run[e] - cap);
+    }
+    *st.aux_loss = st.alpha * static_cast<float>(N) * total;
+    *st.dropped = dropped;
+  }
+}
+
 __global__ void __launch_bounds__(kSlThreads) slot_rank_kernel(
     const int32_t* __restrict__ topk_idx, int32_t* __restrict__ slot,
     int32_t* __restrict__ chunk_hist, int32_t* __restrict__ expert_count, int T, int N, int k,
-    int cap, int single_chunk) {
+    int cap, int single_chunk, const RouteStats st) {
   __shared__ int s_cnt[kSlWarps][256];
+  __shared__ int s_run[256];
+  __shared__ float s_term[256];
   pdl_trigger();
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int P = T * k;  // < 2^31, checked on the host
@@ -202,6 +267,7 @@ __global__ void __launch_bounds__(kSlThreads) slot_rank_kernel(
       expert_count[e] = min(run, cap);
     else
       chunk_hist[static_cast<int64_t>(blockIdx.x) * N + e] = run;
+    s_run[e] = run;
   }
   __syncthreads();
 #pragma unroll
@@ -215,11 +281,15 @@ __global__ void __launch_bounds__(kSlThreads) slot_rank_kernel(
     }
     slot[q_of[it]] = out;
   }
+  if (single_chunk && st.prob_part != nullptr) route_stats_finish(st, s_run, T, N, cap, s_term);
 }
 
 __global__ void __launch_bounds__(256) slot_scan_kernel(int32_t* __restrict__ chunk_hist,
                                                         int32_t* __restrict__ expert_count,
-                                                        int n_chunks, int N, int cap) {
+                                                        int n_chunks, int T, int N, int cap,
+                                                        const RouteStats st) {
+  __shared__ int s_run[256];
+  __shared__ float s_term[256];
   pdl_trigger();
   pdl_wait();
   for (int e = threadIdx.x; e < N; e += blockDim.x) {
@@ -230,7 +300,10 @@ __global__ void __launch_bounds__(256) slot_scan_kernel(int32_t* __restrict__ ch
       run += v;
     }
     expert_count[e] = min(run, cap);
+    s_run[e] = run;
   }
+  __syncthreads();
+  if (st.prob_part != nullptr) route_stats_finish(st, s_run, T, N, cap, s_term);
 }
 
 __global__ void __launch_bounds__(256) slot_finalize_kernel(const int32_t* __restrict__ topk_idx,
@@ -607,14 +680,14 @@ __global__ void __launch_bounds__(dr::kDrThreads) decode_route_kernel(const Deco
 cudaError_t launch_router_topk(const uint16_t* x, const float* w_router, const float* bias,
                                float* logits, int32_t* topk_idx, float* topk_w, int T, int d,
                                int N, int k, uint16_t* split_scratch, int* status,
-                               uint64_t timeout_ns, cudaStream_t s) {
+                               uint64_t timeout_ns, cudaStream_t s, float* prob_part) {
   if (router_uses_tensor_cores(T, N, d))
     return launch_router_tc(x, w_router, bias, logits, topk_idx, topk_w, T, d, N, k,
-                            split_scratch, status, timeout_ns, s);
+                            split_scratch, status, timeout_ns, prob_part, s);
   auto kern = N <= 32 ? router_token_kernel<1> : N <= 64 ? router_token_kernel<2>
              : N <= 128 ? router_token_kernel<4> : router_token_kernel<8>;
   return launch_pdl(kern, dim3(T), dim3(kTokThreads), 0, s, x, w_router, bias, logits, topk_idx,
-                    topk_w, T, d, N, k);
+                    topk_w, T, d, N, k, prob_part);
 }
 
 cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t s) {
@@ -668,15 +741,17 @@ cudaError_t launch_topk_from_logits(const float* logits, int32_t* topk_idx, floa
 
 cudaError_t launch_capacity_slots(const int32_t* topk_idx, int32_t* slot, int32_t* expert_count,
                                   int32_t* chunk_scratch, int T, int N, int k, int capacity,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, const RouteStats* stats) {
+  RouteStats st{};
+  if (stats != nullptr) st = *stats;
   const int64_t P = static_cast<int64_t>(T) * k;
   const int n_chunks = static_cast<int>(slot_chunks(P));
   const int single = n_chunks == 1 ? 1 : 0;
   cudaError_t e = launch_pdl(slot_rank_kernel, dim3(n_chunks), dim3(kSlThreads), 0, s, topk_idx,
-                             slot, chunk_scratch, expert_count, T, N, k, capacity, single);
+                             slot, chunk_scratch, expert_count, T, N, k, capacity, single, st);
   if (e != cudaSuccess || single) return e;
   e = launch_pdl(slot_scan_kernel, dim3(1), dim3(256), 0, s, chunk_scratch, expert_count, n_chunks,
-                 N, capacity);
+                 T, N, capacity, st);
   if (e != cudaSuccess) return e;
   const int blocks = static_cast<int>(std::min<int64_t>((P + 255) / 256, 148 * 8));
   return launch_pdl(slot_finalize_kernel, dim3(blocks), dim3(256), 0, s, topk_idx, slot,

@@ -199,13 +199,52 @@ __device__ __forceinline__ bool finish_tile(const TopK<KMAX>& best, const float*
   return true;
 }
 
+// For the router statistics: the tile's router probabilities summed per expert over its
+// tokens. The staged rows of logits (rows valid ones of the buffer's, stride NS; ks threads per
+// row, neighbouring lanes, ks = 1, 2 or 4) become their softmax in place, using m, the row's
+// largest logit; after a barrier thread ct adds columns ct, ct + 128, ... over the rows in row
+// order. Each barrier is a phase of the epilogue threads' mbarrier, starting at `parity`.
+__device__ __forceinline__ bool tile_prob_sums(float m, float* buf, int rows, int NS, int N, int ks,
+                                               int ct, float* out_row, uint32_t epi_bar,
+                                               uint32_t parity, uint64_t timeout_ns,
+                                               const volatile int* abort) {
+  mbar_arrive(epi_bar);  // every thread has finished reading the staged logits
+  bool ok = mbar_wait(epi_bar, parity, timeout_ns, abort);
+  if (!__all_sync(0xffffffffu, ok)) return false;
+  const int lr = ct / ks, part = ct - lr * ks;
+  float sum = 0.f;
+  if (lr < rows) {
+    float* row = buf + lr * NS;
+    for (int e = part; e < N; e += ks) {
+      const float v = expf(row[e] - m);
+      row[e] = v;
+      sum += v;
+    }
+  }
+  for (int o = 1; o < ks; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lr < rows) {
+    const float inv = 1.0f / sum;
+    float* row = buf + lr * NS;
+    for (int e = part; e < N; e += ks) row[e] *= inv;
+  }
+  mbar_arrive(epi_bar);
+  ok = mbar_wait(epi_bar, parity ^ 1u, timeout_ns, abort);
+  if (!__all_sync(0xffffffffu, ok)) return false;
+  for (int e = ct; e < N; e += kConvThreads) {
+    float acc = 0.f;
+    for (int r = 0; r < rows; ++r) acc += buf[r * NS + e];
+    out_row[e] = acc;
+  }
+  return true;
+}
+
 template <int NP, bool PRESPLIT, int KMAX>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ w, const float* __restrict__ bias,
                      float* __restrict__ logits, int32_t* __restrict__ topk_idx,
                      float* __restrict__ topk_w, int T, int d, int N, int k, int* status,
-                     uint64_t timeout_ns, int ksplit) {
+                     uint64_t timeout_ns, float* __restrict__ prob_part, int ksplit) {
   using C = RCfg<NP, PRESPLIT>;
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t a_full[C::STAGES];
@@ -430,6 +469,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ok = finish_tile<KMAX>(best, stage, t0, ct, T, N, NS, k, logits, topk_idx, topk_w,
                                smem_u32(&epi_bar), timeout_ns, &s_abort);
+        if (ok && prob_part != nullptr)
+          ok = tile_prob_sums(best.v[0], stage, min(kTok, T - t0), NS, N, 1, ct,
+                              prob_part + static_cast<int64_t>(blockIdx.x) * N, smem_u32(&epi_bar),
+                              1u, timeout_ns, &s_abort);
       }
     }
     epi_ok = ok;
@@ -541,6 +584,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int r = i / N;
           dst[i] = fin[r * NS + (i - r * N)];
         }
+        if (prob_part != nullptr &&
+            !tile_prob_sums(sel_v[0], fin, rows, NS, N, ksplit, ct,
+                            prob_part + static_cast<int64_t>(blockIdx.x) * N, smem_u32(&epi_bar),
+                            1u, timeout_ns, &s_abort)) {
+          s_abort = 1;
+          report_error(status, MOE_ERR_TIMEOUT);
+        }
       } else {
         s_abort = 1;
         report_error(status, MOE_ERR_TIMEOUT);
@@ -572,7 +622,7 @@ int router_ksplit(int tiles, int num_kb) {
 template <int NP, bool PRESPLIT, int KMAX>
 cudaError_t launch_npk(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
                        const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
-                       int d, int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
+                       int d, int N, int k, int* status, uint64_t timeout_ns, float* prob_part, cudaStream_t s) {
   using C = RCfg<NP, PRESPLIT>;
   static PerDeviceOnce once;
   const cudaError_t attr = once.run([] {
@@ -585,39 +635,39 @@ cudaError_t launch_npk(const CUtensorMap& mx, const CUtensorMap& mw, const float
   if (ksplit == 1)
     return launch_pdl(router_tc_kernel<NP, PRESPLIT, KMAX>, dim3(tiles), dim3(kThreads),
                       C::SMEM_BYTES, s, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k,
-                      status, timeout_ns, 1);
+                      status, timeout_ns, prob_part, 1);
   return launch_pdl_cluster(router_tc_kernel<NP, PRESPLIT, KMAX>, dim3(tiles * ksplit),
                             dim3(kThreads), C::SMEM_BYTES, s, static_cast<unsigned>(ksplit), mx, mw,
-                            w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns,
+                            w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part,
                             ksplit);
 }
 
 template <int NP, bool PRESPLIT>
 cudaError_t launch_np(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
                       const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
-                      int d, int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
+                      int d, int N, int k, int* status, uint64_t timeout_ns, float* prob_part, cudaStream_t s) {
   if (k <= 1)
-    return launch_npk<NP, PRESPLIT, 1>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+    return launch_npk<NP, PRESPLIT, 1>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
   if (k <= 2)
-    return launch_npk<NP, PRESPLIT, 2>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+    return launch_npk<NP, PRESPLIT, 2>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
   if (k <= 4)
-    return launch_npk<NP, PRESPLIT, 4>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
-  return launch_npk<NP, PRESPLIT, 8>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+    return launch_npk<NP, PRESPLIT, 4>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+  return launch_npk<NP, PRESPLIT, 8>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
 }
 
 template <bool PRESPLIT>
 cudaError_t launch_tc(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
                       const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
-                      int d, int N, int k, int* status, uint64_t timeout_ns, cudaStream_t s) {
+                      int d, int N, int k, int* status, uint64_t timeout_ns, float* prob_part, cudaStream_t s) {
   if (N <= 16)
-    return launch_np<16, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+    return launch_np<16, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
   if (N <= 32)
-    return launch_np<32, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+    return launch_np<32, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
   if (N <= 64)
-    return launch_np<64, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+    return launch_np<64, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
   if (N <= 128)
-    return launch_np<128, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
-  return launch_np<256, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, s);
+    return launch_np<128, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+  return launch_np<256, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
 }
 
 bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
@@ -634,9 +684,14 @@ bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* d
 
 size_t router_split_bytes(int N, int d) { return static_cast<size_t>(3) * N * d * 2; }
 
+int router_tc_parts(int T, int d) {
+  const int tiles = (T + kTok - 1) / kTok;
+  return tiles * router_ksplit(tiles, d / kBK);
+}
+
 cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const float* bias,
                              float* logits, int32_t* topk_idx, float* topk_w, int T, int d, int N,
-                             int k, uint16_t* split_scratch, int* status, uint64_t timeout_ns,
+                             int k, uint16_t* split_scratch, int* status, uint64_t timeout_ns, float* prob_part,
                              cudaStream_t s) {
   CUtensorMap mx, mw;
   {
@@ -649,7 +704,7 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const flo
   if (split_scratch == nullptr) {
     memset(&mw, 0, sizeof(mw));  // unused by the in-kernel split
     return launch_tc<false>(mx, mw, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status,
-                            timeout_ns, s);
+                            timeout_ns, prob_part, s);
   }
   {
     const cuuint64_t gd[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), 3};
@@ -663,7 +718,7 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const flo
                              split_scratch, n);
   if (e != cudaSuccess) return e;
   return launch_tc<true>(mx, mw, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status,
-                         timeout_ns, s);
+                         timeout_ns, prob_part, s);
 }
 
 }  // namespace moe

@@ -59,8 +59,10 @@ def test_workspace_sizes():
     big = moe.make_dims(16384, 7168, 256, 8, 2048, "swiglu", 80)
     # 80-row partial tiles: whole tiles only; status word + per-m-tile counters (at most
     # 160 + 256 m-tiles) + the routing scratch: capacity-scan chunk totals + the bf16
-    # three-term split of W_r that the tensor-core router reads
-    assert moe.workspace_bytes(big) == 256 + counters(416, 0, 0) + 32 * 256 * 4 + 3 * 256 * 7168 * 2
+    # three-term split of W_r that the tensor-core router reads + the router's probability sums
+    # for moe_route_with_stats (one row of 256 per 128-token tile)
+    assert moe.workspace_bytes(big) == (256 + counters(416, 0, 0) + 32 * 256 * 4
+                                        + 3 * 256 * 7168 * 2 + 128 * 256 * 4)
     decode = moe.make_dims(4, 2880, 32, 4, 2880, "swiglu", 4)
     # status word (+ the decode router's arrival counter) + the larger of the grouped FFN's
     # counters (at most 1 + 16 m-tiles: 17 x 23 gate/up and 17 x 12 down tiles) and the decode
