@@ -90,8 +90,10 @@ __global__ void __launch_bounds__(256) permute_kernel(
       }
     }
     __syncthreads();
+    bool any = false;  // a token whose every pair was dropped has nothing to copy
+    for (int j = 0; j < k; ++j) any |= s_rows[j] >= 0;
     const int v = c * kVecPerBlock + threadIdx.x;
-    if (v < nv) {
+    if (any && v < nv) {
       const uint4 val = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * d)[v];
       for (int j = 0; j < k; ++j) {
         const int row = s_rows[j];
@@ -102,83 +104,98 @@ __global__ void __launch_bounds__(256) permute_kernel(
   }
 }
 
-// Block (token t, chunk c of 1024 columns): thread i handles 4 columns (one float4 of each kept
-// expert row of y_perm and 4 bf16 of the residual). Weights and rows of the token come from its
-// k pairs.
-constexpr int kColsPerBlock = 1024;
+// Warp per item (token t, group g of 512 columns), grid-stride: lanes j < k read the token's
+// pair j (its y_perm row and router weight; a row at or past R_max is skipped and reported),
+// shared with the warp by shuffles, and each lane then handles 16 columns, one float4 of each
+// kept row of y_perm and 4 bf16 of the residual for each of four 128-column steps (coalesced
+// across the warp). The next item's pairs are read before this item's rows, so the dependent
+// loads of consecutive items overlap; warps need no block-wide barrier. Per column the sum is
+// the kept choices' w_j * y in ascending j (fp32 fma from zero), then plus the residual, rounded
+// once; a token with no kept pair passes the residual's bits through.
+constexpr int kCombCols = 512;
 
-__global__ void __launch_bounds__(256) combine_kernel(
+__device__ __forceinline__ void combine_pair(const int32_t* __restrict__ row_of_pair,
+                                             const float* __restrict__ topk_w, int64_t t, int k,
+                                             int64_t r_max, int lane, int* status, int& row,
+                                             float& w) {
+  row = -1;
+  w = 0.f;
+  if (lane < k) {
+    const int64_t q = t * k + lane;
+    row = row_of_pair[q];
+    w = topk_w[q];
+    if (row >= r_max) {
+      report_error(status, MOE_ERR_BOUNDS);
+      row = -1;
+    }
+  }
+}
+
+constexpr int kCombBlocksPerSm = 4;
+
+__global__ void __launch_bounds__(256, kCombBlocksPerSm) combine_kernel(
     const float* __restrict__ y, const int32_t* __restrict__ row_of_pair,
     const float* __restrict__ topk_w, const uint16_t* residual, void* out, int out_f32, int T,
     int d, int k, int64_t r_max, int* status) {
-  __shared__ int s_rows[8];
-  __shared__ float s_w[8];
-  __shared__ int s_any;
   pdl_trigger();
   pdl_wait();
-  const int nq = d / 4;  // groups of 4 columns
-  const int chunks = (d + kColsPerBlock - 1) / kColsPerBlock;
-  const int64_t items = static_cast<int64_t>(T) * chunks;
-  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
-    const int t = static_cast<int>(item / chunks);
-    const int c = static_cast<int>(item - static_cast<int64_t>(t) * chunks);
-    if (threadIdx.x < 32) {
-      const int lane = threadIdx.x;
-      int row = -1;
-      float w = 0.f;
-      if (lane < k) {
-        const int64_t q = static_cast<int64_t>(t) * k + lane;
-        row = row_of_pair[q];
-        w = topk_w[q];
-        if (row >= r_max) {
-          report_error(status, MOE_ERR_BOUNDS);
-          row = -1;
-        }
-        s_rows[lane] = row;
-        s_w[lane] = w;
-      }
-      const unsigned any = __ballot_sync(kFull, row >= 0);
-      if (lane == 0) s_any = any != 0;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int groups = (d + kCombCols - 1) / kCombCols;
+  const int64_t items = static_cast<int64_t>(T) * groups;
+  int64_t item = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int row_n = -1;
+  float w_n = 0.f;
+  if (item < items) combine_pair(row_of_pair, topk_w, item / groups, k, r_max, lane, status, row_n, w_n);
+  for (; item < items; item += nwarps) {
+    const int row = row_n;
+    const float w = w_n;
+    const int64_t next = item + nwarps;
+    if (next < items) combine_pair(row_of_pair, topk_w, next / groups, k, r_max, lane, status, row_n, w_n);
+    const int64_t t = item / groups;
+    const int g = static_cast<int>(item - t * groups);
+    int rows[8];
+    float ws[8];
+    bool any = false;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      rows[j] = __shfl_sync(kFull, row, j);
+      ws[j] = __shfl_sync(kFull, w, j);
+      if (j >= k) rows[j] = -1;
+      any |= rows[j] >= 0;
     }
-    __syncthreads();
-    const int qi = c * (kColsPerBlock / 4) + threadIdx.x;
-    if (qi < nq) {
+#pragma unroll 2
+    for (int i = 0; i < kCombCols / 128; ++i) {
+      const int col = g * kCombCols + i * 128 + lane * 4;
+      if (col >= d) continue;
       uint2 rbits = make_uint2(0u, 0u);
-      if (residual != nullptr) rbits = reinterpret_cast<const uint2*>(residual + static_cast<int64_t>(t) * d)[qi];
-      if (!s_any) {  // every choice dropped: the residual passes through unchanged
-        if (out_f32) {
-          reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<int64_t>(t) * d)[qi] =
-              make_float4(__uint_as_float(rbits.x << 16), __uint_as_float(rbits.x & 0xffff0000u),
-                          __uint_as_float(rbits.y << 16), __uint_as_float(rbits.y & 0xffff0000u));
-        } else {
-          reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + static_cast<int64_t>(t) * d)[qi] = rbits;
-        }
-      } else {
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        for (int j = 0; j < k; ++j) {  // ascending choice order
-          const int row = s_rows[j];
-          if (row < 0) continue;
-          const float wj = s_w[j];
-          const float4 v = reinterpret_cast<const float4*>(y + static_cast<int64_t>(row) * d)[qi];
-          a0 = fmaf(wj, v.x, a0);
-          a1 = fmaf(wj, v.y, a1);
-          a2 = fmaf(wj, v.z, a2);
-          a3 = fmaf(wj, v.w, a3);
-        }
-        const float o0 = __uint_as_float(rbits.x << 16) + a0;
-        const float o1 = __uint_as_float(rbits.x & 0xffff0000u) + a1;
-        const float o2 = __uint_as_float(rbits.y << 16) + a2;
-        const float o3 = __uint_as_float(rbits.y & 0xffff0000u) + a3;
-        if (out_f32) {
-          reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<int64_t>(t) * d)[qi] =
-              make_float4(o0, o1, o2, o3);
-        } else {
-          reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + static_cast<int64_t>(t) * d)[qi] =
-              make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
-        }
+      if (residual != nullptr) rbits = *reinterpret_cast<const uint2*>(residual + t * d + col);
+      const float r0 = __uint_as_float(rbits.x << 16), r1 = __uint_as_float(rbits.x & 0xffff0000u);
+      const float r2 = __uint_as_float(rbits.y << 16), r3 = __uint_as_float(rbits.y & 0xffff0000u);
+      if (!any) {  // every choice dropped: the residual passes through unchanged
+        if (out_f32)
+          *reinterpret_cast<float4*>(static_cast<float*>(out) + t * d + col) = make_float4(r0, r1, r2, r3);
+        else
+          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + t * d + col) = rbits;
+        continue;
       }
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {  // ascending choice order
+        if (rows[j] < 0) continue;
+        const float4 v = *reinterpret_cast<const float4*>(y + static_cast<int64_t>(rows[j]) * d + col);
+        a0 = fmaf(ws[j], v.x, a0);
+        a1 = fmaf(ws[j], v.y, a1);
+        a2 = fmaf(ws[j], v.z, a2);
+        a3 = fmaf(ws[j], v.w, a3);
+      }
+      const float o0 = r0 + a0, o1 = r1 + a1, o2 = r2 + a2, o3 = r3 + a3;
+      if (out_f32)
+        *reinterpret_cast<float4*>(static_cast<float*>(out) + t * d + col) = make_float4(o0, o1, o2, o3);
+      else
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + t * d + col) =
+            make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
     }
-    __syncthreads();
   }
 }
 
@@ -203,8 +220,8 @@ cudaError_t launch_combine(const float* y_perm, const int32_t* row_of_pair, cons
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  const int64_t items = static_cast<int64_t>(T) * ((d + kColsPerBlock - 1) / kColsPerBlock);
-  const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(items, di.sm_count * 16)));
+  const int64_t warps = static_cast<int64_t>(T) * ((d + kCombCols - 1) / kCombCols);
+  const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, di.sm_count * kCombBlocksPerSm)));
   return launch_pdl(combine_kernel, dim3(blocks), dim3(256), 0, s, y_perm, row_of_pair, topk_w,
                     residual, out, out_f32, T, d, k, r_max, status);
 }
