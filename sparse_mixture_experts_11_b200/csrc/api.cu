@@ -113,22 +113,18 @@ bool decode_ffn_for(const moe_dims* d) { return moe::use_decode_ffn(d->T, d->act
 
 size_t counters_bytes(const moe_dims* d) {
   const size_t decode =
-      decode_ffn_for(d) ? moe::decode_ffn_counter_bytes(d->n_experts, d->T, d->top_k, d->d_ff) : 0;
+      decode_ffn_for(d) ? moe::decode_ffn_counter_bytes(d->n_experts, d->T, d->top_k, d->d_ff, d->d_model) : 0;
   return round_up(std::max(ffn_plan(d).counter_bytes, decode), 256);
 }
 
 // The decode FFN's scratch in the shared region: after the decode router's partial dot products
 // (the launch that also routes reads them while other CTAs already store FFN partials), the
-// fp32 partials of y, then the gate/up partials passed between CTAs.
+// chunks' partials.
 size_t decode_ffn_part_offset(const moe_dims* d) { return decode_scratch_bytes(d); }
-size_t decode_ffn_part_gu_offset(const moe_dims* d) {
-  return decode_ffn_part_offset(d) +
-         round_up(moe::decode_ffn_part_bytes(max_rows(d), d->d_model, d->d_ff), 256);
-}
 size_t decode_ffn_scratch_bytes(const moe_dims* d) {
   if (!decode_ffn_for(d)) return 0;
-  return decode_ffn_part_gu_offset(d) +
-         round_up(moe::decode_ffn_part_gu_bytes(d->n_experts, d->T, d->top_k, d->d_ff), 256);
+  return decode_ffn_part_offset(d) +
+         round_up(moe::decode_ffn_part_bytes(d->n_experts, d->T, d->top_k, d->d_model, d->d_ff), 256);
 }
 
 // Router statistics emitted by the routing launches: the router's per-tile probability sums,
@@ -414,7 +410,6 @@ moe::DecodeFfnArgs decode_ffn_args(const moe_dims* dims, const uint16_t* x_perm,
   a.y_perm = y_perm;
   char* region = shared_region_of(dims, ws);
   a.part = reinterpret_cast<float*>(region + decode_ffn_part_offset(dims));
-  a.part_gu = reinterpret_cast<float*>(region + decode_ffn_part_gu_offset(dims));
   a.sync = reinterpret_cast<int*>(static_cast<char*>(ws) + moe::kStatusBytes);
   a.flags = a.sync + moe::kDecodeFfnSyncInts;
   a.N = dims->n_experts;
