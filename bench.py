@@ -176,25 +176,16 @@ def decode_route(T: int, n_experts: int, d_model: int) -> bool:
         math.ceil(d_model / 128) * T * n_experts * 4 <= DECODE_ROUTE_MAX_SCRATCH
 
 
-DECODE_FFN_MAX_T = 8  # SwiGLU batches up to this size take the d_ff-sliced decode FFN
-
-
-def launches_per_step(T: int, k: int, R_max: int, n_experts: int = 1, d_model: int = 1,
-                      act: str = "swiglu") -> int:
-    """Kernels one forward (moe_forward) launches. SwiGLU batches of at most 8 tokens: the decode
-    FFN, which also combines, and routes and sorts in the same launch while x_perm is at most
-    512 KB (else a routing launch and a permute launch before it). Other decode-sized batches
-    (decode_route): one routing launch (router, top-k and slots), which also sorts by expert
-    while x_perm is at most 512 KB, else a permute launch. Larger batches: router + top-k (plus
-    the W_r split kernel on the tensor-core path), capacity slots (1 pass, or 3 when the
-    arrivals span several chunks), permute. Then the grouped FFN (both GEMMs in one launch, when
-    rows can exist) and the combine."""
-    sorts = R_max * d_model * 2 <= DECODE_PERMUTE_MAX_BYTES
-    if act == "swiglu" and 1 <= T <= DECODE_FFN_MAX_T and R_max > 0:
-        return 1 if decode_route(T, n_experts, d_model) and sorts else 3
+def launches_per_step(T: int, k: int, R_max: int, n_experts: int = 1, d_model: int = 1) -> int:
+    """Kernels one forward (moe_forward) launches. Decode-sized batches (decode_route): one routing
+    launch (router, top-k and slots), which also sorts by expert while x_perm is at most
+    512 KB, else a permute launch. Larger batches: router + top-k (plus the W_r split kernel
+    on the tensor-core path), capacity slots (1 pass, or 3 when the arrivals span several
+    chunks), permute. Then the grouped FFN (both GEMMs in one launch, when rows can exist)
+    and the combine."""
     ffn = (1 if R_max > 0 else 0) + 1
     if decode_route(T, n_experts, d_model):
-        return 1 + (0 if sorts else 1) + ffn
+        return 1 + (0 if R_max * d_model * 2 <= DECODE_PERMUTE_MAX_BYTES else 1) + ffn
     chunks = max(1, math.ceil(T * k / SLOT_CHUNK))
     router = 2 if router_on_tensor_cores(T, n_experts, d_model) else 1
     return router + (1 if chunks == 1 else 3) + 1 + ffn
@@ -719,7 +710,7 @@ def sweep_entry(layer, spec: str, step_ms: list, stage_ms: dict, peaks: dict) ->
             "kept_rows": R, "active_experts": active, "capacity": layer.dims.capacity,
             "ffn": roof["ffn"], "layer": roof["layer"],
             "gpu_launches_per_step": launches_per_step(T, shape.top_k, layer.R_max,
-                                                       shape.n_experts, shape.d_model, shape.act)}
+                                                       shape.n_experts, shape.d_model)}
 
 
 def run_sweep(args, device, flush, peaks, headline=None) -> dict:
@@ -829,7 +820,7 @@ def run_gpu(args, rank, world, local_rank):
                 "h2d_bytes_per_step": T * shape.d_model * 2,
                 "d2h_bytes_per_step": T * shape.d_model * 2},
         "gpu_launches": launches_per_step(T, shape.top_k, layer.R_max, shape.n_experts,
-                                          shape.d_model, shape.act) * args.steps,
+                                          shape.d_model) * args.steps,
         "clocks": clk,
     }
     if args.sweep != "none" and world == 1:

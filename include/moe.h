@@ -39,8 +39,8 @@
  *       MOE_ERR_INVALID      null pointer where one is required, negative size, k > N, k < 1
  *       MOE_ERR_UNSUPPORTED  d_model or d_ff not a multiple of 64, N > 256, k > 8, a pointer
  *                            that is not 16-byte aligned, a device that is not sm_100, or a
- *                            grid whose CTAs wait on one another (the grouped and decode FFN)
- *                            that the device cannot hold resident at once
+ *                            grid whose CTAs wait on one another (the grouped FFN) that the
+ *                            device cannot hold resident at once
  *       MOE_ERR_WORKSPACE    ws_bytes below what moe_workspace_bytes() reports
  *       MOE_ERR_CUDA         a CUDA runtime or driver call failed while launching
  *     Nothing is launched when validation fails. T == 0 is valid and launches nothing.

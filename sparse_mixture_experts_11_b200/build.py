@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmoe.so")
-SOURCES = ["api.cu", "route.cu", "permute_combine.cu", "grouped_ffn.cu", "route_noalloc.cu", "router_tc.cu", "router_stats.cu", "backward.cu", "decode_ffn.cu"]
+SOURCES = ["api.cu", "route.cu", "permute_combine.cu", "grouped_ffn.cu", "route_noalloc.cu", "router_tc.cu", "router_stats.cu", "backward.cu"]
 GENCODE = "-gencode=arch=compute_100a,code=sm_100a"
 
 

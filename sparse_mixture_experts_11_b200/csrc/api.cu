@@ -109,23 +109,7 @@ moe::FfnScratchPlan ffn_plan(const moe_dims* d) {
 //   [shared region: routing scratch (capacity-scan chunk totals, router weight split, the
 //    decode router's partial dot products) or,
 //    later on the stream, the grouped FFN's stream-K partial tiles]
-bool decode_ffn_for(const moe_dims* d) { return moe::use_decode_ffn(d->T, d->act, max_rows(d)); }
-
-size_t counters_bytes(const moe_dims* d) {
-  const size_t decode =
-      decode_ffn_for(d) ? moe::decode_ffn_counter_bytes(d->n_experts, d->T, d->top_k, d->d_ff, d->d_model) : 0;
-  return round_up(std::max(ffn_plan(d).counter_bytes, decode), 256);
-}
-
-// The decode FFN's scratch in the shared region: after the decode router's partial dot products
-// (the launch that also routes reads them while other CTAs already store FFN partials), the
-// chunks' partials.
-size_t decode_ffn_part_offset(const moe_dims* d) { return decode_scratch_bytes(d); }
-size_t decode_ffn_scratch_bytes(const moe_dims* d) {
-  if (!decode_ffn_for(d)) return 0;
-  return decode_ffn_part_offset(d) +
-         round_up(moe::decode_ffn_part_bytes(d->n_experts, d->T, d->top_k, d->d_model, d->d_ff), 256);
-}
+size_t counters_bytes(const moe_dims* d) { return round_up(ffn_plan(d).counter_bytes, 256); }
 
 // Router statistics emitted by the routing launches: the router's per-tile probability sums,
 // after the routing scratch (both are live during the same call).
@@ -139,7 +123,7 @@ size_t route_stats_bytes(const moe_dims* d) {
 size_t shared_region_bytes(const moe_dims* d) {
   const size_t routing = slot_scratch_bytes(d) + split_scratch_bytes(d) + decode_scratch_bytes(d) +
                          route_stats_bytes(d);
-  const size_t ffn = round_up(std::max(ffn_plan(d).part_bytes, decode_ffn_scratch_bytes(d)), 256);
+  const size_t ffn = round_up(ffn_plan(d).part_bytes, 256);
   const size_t stats = round_up(moe::router_stats_scratch_bytes(d->T, d->n_experts), 256);
   const size_t redirect = round_up(moe::redirect_scratch_bytes(d->T, d->top_k), 256);
   return std::max(std::max(std::max(routing, ffn), stats), redirect);
@@ -397,32 +381,6 @@ Weights weights_of(const moe_mx_weights* w) {
   return Weights{w->fmt, w->gate_up, w->gate_up_scales, w->down, w->down_scales};
 }
 
-// The decode FFN's arguments for the stage call (no routing, no combine).
-moe::DecodeFfnArgs decode_ffn_args(const moe_dims* dims, const uint16_t* x_perm,
-                                   const int32_t* expert_offset, const Weights& w, uint16_t* h,
-                                   float* y_perm, void* ws) {
-  moe::DecodeFfnArgs a{};
-  a.x_perm = x_perm;
-  a.expert_offset = expert_offset;
-  a.w_gate_up = static_cast<const uint16_t*>(w.gate_up);
-  a.w_down = static_cast<const uint16_t*>(w.down);
-  a.h = h;
-  a.y_perm = y_perm;
-  char* region = shared_region_of(dims, ws);
-  a.part = reinterpret_cast<float*>(region + decode_ffn_part_offset(dims));
-  a.sync = reinterpret_cast<int*>(static_cast<char*>(ws) + moe::kStatusBytes);
-  a.flags = a.sync + moe::kDecodeFfnSyncInts;
-  a.N = dims->n_experts;
-  a.d = dims->d_model;
-  a.F = dims->d_ff;
-  a.T = dims->T;
-  a.k = dims->top_k;
-  a.r_max = max_rows(dims);
-  a.status = status_of(ws);
-  a.timeout_ns = moe::wait_timeout_ns();
-  return a;
-}
-
 moe_status grouped_ffn_impl(const moe_dims* dims, const uint16_t* x_perm,
                             const int32_t* expert_offset, const Weights& w, uint16_t* h,
                             float* y_perm, void* ws, size_t ws_bytes, void* stream) {
@@ -455,10 +413,6 @@ moe_status grouped_ffn_impl(const moe_dims* dims, const uint16_t* x_perm,
   a.status = status_of(ws);
   a.timeout_ns = moe::wait_timeout_ns();
   a.rows_per_expert = std::min(dims->capacity, dims->T);
-  if (w.fmt == MOE_WFMT_BF16 && decode_ffn_for(dims)) {
-    moe::DecodeFfnArgs da = decode_ffn_args(dims, x_perm, expert_offset, w, h, y_perm, ws);
-    return launch_status(moe::launch_decode_ffn(da, as_stream(stream)));
-  }
   const moe::FfnScratchPlan plan = ffn_plan(dims);
   a.counters = reinterpret_cast<int*>(static_cast<char*>(ws) + moe::kStatusBytes);
   if (plan.part_bytes > 0) a.part = reinterpret_cast<float*>(shared_region_of(dims, ws));
@@ -680,40 +634,6 @@ moe_status forward_impl(const moe_dims* dims, const uint16_t* x, const float* w_
   const int64_t rmax = max_rows(dims);
   const bool route_sorts = moe::use_decode_route(dims->T, dims->n_experts, dims->d_model) &&
                            rmax * dims->d_model * 2 <= moe::kDecodePermuteMaxBytes;
-  if (w.fmt == MOE_WFMT_BF16 && decode_ffn_for(dims)) {
-    // decode-sized batch: the FFN cut along d_ff, with the combine (and, when the router also
-    // sorts by expert, the routing) in the same launch
-    if (!aligned16(x) || !aligned16(w_router) || (logit_bias && !aligned16(logit_bias)) ||
-        !aligned16(out) || (residual && !aligned16(residual)))
-      return MOE_ERR_UNSUPPORTED;
-    if ((st = check_device()) != MOE_OK) return st;
-    if (!route_sorts) {
-      st = moe_route(dims, x, w_router, logit_bias, b.logits, b.topk_idx, b.topk_w, b.slot,
-                     b.expert_count, b.stage_ws, b.stage_ws_bytes, stream);
-      if (st != MOE_OK) return st;
-      st = moe_permute(dims, x, b.topk_idx, b.slot, b.expert_count, b.expert_offset,
-                       b.row_of_pair, b.pair_of_row, b.x_perm, b.stage_ws, b.stage_ws_bytes,
-                       stream);
-      if (st != MOE_OK) return st;
-    }
-    moe::DecodeFfnArgs da = decode_ffn_args(dims, b.x_perm, b.expert_offset, w, b.h, b.y_perm,
-                                            b.stage_ws);
-    da.row_of_pair = b.row_of_pair;
-    da.topk_w = b.topk_w;
-    da.residual = residual;
-    da.out = out;
-    da.out_f32 = 0;
-    if (route_sorts) {
-      da.route_in_kernel = true;
-      da.route = decode_route_args(dims, x, w_router, logit_bias, b.logits, b.topk_idx, b.topk_w,
-                                   b.slot, b.expert_count, b.stage_ws);
-      da.route.expert_offset = b.expert_offset;
-      da.route.row_of_pair = b.row_of_pair;
-      da.route.pair_of_row = b.pair_of_row;
-      da.route.x_perm = b.x_perm;
-    }
-    return launch_status(moe::launch_decode_ffn(da, as_stream(stream)));
-  }
   if (route_sorts) {
     // decode-sized batch: routing and the sort by expert in one launch
     if (!aligned16(x) || !aligned16(w_router) || (logit_bias && !aligned16(logit_bias)))

@@ -1,7 +1,6 @@
 // Routing of decode-sized batches in one pass over a few CTAs, and the warp-level top-k it
 // shares with the other routing kernels. Used by the decode router kernel (moe_route,
-// moe_forward, moe_route_noalloc) and by the fused decode layer kernel, which therefore route
-// bit for bit alike.
+// moe_forward, moe_route_noalloc).
 //
 // Page «Sparse Mixture-of-Experts» (bigdataschool wiki), «Роутер и top-k gating» (linear router,
 // softmax, top-k, renormalisation) and «Expert capacity и capacity factor» (capacity slots,
@@ -165,12 +164,10 @@ __device__ __forceinline__ bool decode_route_partials(const DecodeRouteArgs& a, 
 // order), top-k with the renormalised weights, the capacity slots in (choice, token) order, the
 // kept counts, the expert offsets and the rows of the kept pairs; all of it in shared memory
 // (sm). With `write` the CTA also stores the routing's outputs to global memory, and when the
-// permute outputs are given the offsets and row maps as well, with the x_perm copy unless
-// copy_rows is false.
+// permute outputs are given the offsets, the row maps and the x_perm copy as well.
 template <int TMAX, int EPT>
 __device__ __forceinline__ void decode_route_finish(const DecodeRouteArgs& a, int ctas,
-                                                    DecodeRouteSmem<TMAX, EPT>& sm, bool write,
-                                                    bool copy_rows = true) {
+                                                    DecodeRouteSmem<TMAX, EPT>& sm, bool write) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = a.T, N = a.N, d = a.d, k = a.k;
   const int S = ctas;
@@ -316,7 +313,7 @@ __device__ __forceinline__ void decode_route_finish(const DecodeRouteArgs& a, in
     sm.row[tid] = row;
   }
   __syncthreads();
-  if (permute && copy_rows) {
+  if (permute) {
     const int nv = d / 8;  // 16-byte vectors per row
     for (int i = tid; i < P * nv; i += kDrThreads) {
       const int p2 = i / nv, vv = i - p2 * nv;

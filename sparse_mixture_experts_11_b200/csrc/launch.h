@@ -255,90 +255,6 @@ struct GroupedFfnArgs {
 };
 cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s);
 
-// Expert FFN of decode-sized batches (SwiGLU, bf16 weights, T <= kDecodeFfnMaxT, so an expert
-// holds at most that many rows): the gate/up GEMM and then the down GEMM in tiles of 256 weight
-// rows, each tile cut into a fixed number of chunks of 64-k units that the CTAs take from a
-// global counter; each chunk's fp32 partial goes to the scratch and the CTA that finishes a
-// tile adds them in chunk order. h passes from the first GEMM to the second through global
-// memory, behind one flag per 128 columns of d_ff. Optionally the same launch first routes (the
-// decode router, as moe_route does) and finally combines with the residual. Every CTA of the
-// grid must be resident at once (one per SM).
-constexpr int kDecodeFfnMaxT = 8;
-constexpr int kDecodeFfnMaxRows = 8;    // rows per expert: at most T
-constexpr int kDecodeFfnSlice = 128;    // d_ff columns per gate/up tile
-constexpr int kDecodeFfnOutBlock = 256; // d rows per down tile
-constexpr int kDecodeFfnMaxCtas = 256;  // grid size at most (one CTA per SM)
-inline bool use_decode_ffn(int64_t T, int act, int64_t r_max) {
-  return act == MOE_ACT_SWIGLU && T >= 1 && T <= kDecodeFfnMaxT && r_max > 0;
-}
-inline int64_t decode_ffn_max_active(int64_t N, int64_t T, int64_t k) { return N < T * k ? N : T * k; }
-// gate/up tiles at most: the experts that can hold rows times ceil(F / 128)
-inline int64_t decode_ffn_max_slices(int64_t N, int64_t T, int64_t k, int64_t F) {
-  return decode_ffn_max_active(N, T, k) * ((F + kDecodeFfnSlice - 1) / kDecodeFfnSlice);
-}
-// down tiles at most: the experts that can hold rows times ceil(d / 256)
-inline int64_t decode_ffn_max_down_tiles(int64_t N, int64_t T, int64_t k, int64_t d) {
-  return decode_ffn_max_active(N, T, k) * ((d + kDecodeFfnOutBlock - 1) / kDecodeFfnOutBlock);
-}
-// Chunks per tile, from the shape only: about 1200 chunks when every expert that can hold rows
-// is active (some 8 per SM), of 2 to 64 units (64 KB to 2 MB of weights) each.
-struct DecodeFfnChunks {
-  int nca, ncb;  // chunks per gate/up tile (d / 64 units), per down tile (F / 64 units)
-};
-inline DecodeFfnChunks decode_ffn_chunks(int64_t N, int64_t T, int64_t k, int64_t d, int64_t F) {
-  const int64_t KB = d / 64, FB = F / 64;
-  const int64_t units = decode_ffn_max_slices(N, T, k, F) * KB + decode_ffn_max_down_tiles(N, T, k, d) * FB;
-  int64_t cu = units / 1200;
-  cu = cu < 2 ? 2 : (cu > 64 ? 64 : cu);
-  DecodeFfnChunks c;
-  c.nca = static_cast<int>((KB + cu - 1) / cu);
-  c.ncb = static_cast<int>((FB + cu - 1) / cu);
-  return c;
-}
-// Scratch: the fp32 partial of an 8 x 256 accumulator per chunk
-inline size_t decode_ffn_part_bytes(int64_t N, int64_t T, int64_t k, int64_t d, int64_t F) {
-  const DecodeFfnChunks c = decode_ffn_chunks(N, T, k, d, F);
-  const int64_t chunks = decode_ffn_max_slices(N, T, k, F) * c.nca + decode_ffn_max_down_tiles(N, T, k, d) * c.ncb;
-  return static_cast<size_t>(chunks) * kDecodeFfnMaxRows * 256 * sizeof(float);
-}
-// Counters, zero between calls: kDecodeFfnSyncInts (departures, the chunk counter), a flag per
-// gate/up tile (h stored), a finished-chunk count per gate/up tile and per down tile, a count per
-// 256 rows of d (down tiles finished)
-constexpr int kDecodeFfnSyncInts = 4;
-inline size_t decode_ffn_counter_bytes(int64_t N, int64_t T, int64_t k, int64_t F, int64_t d) {
-  return static_cast<size_t>(kDecodeFfnSyncInts + 2 * decode_ffn_max_slices(N, T, k, F) +
-                             decode_ffn_max_down_tiles(N, T, k, d) +
-                             (d + kDecodeFfnOutBlock - 1) / kDecodeFfnOutBlock) *
-         sizeof(int);
-}
-
-struct DecodeFfnArgs {
-  const uint16_t* x_perm;        // [r_max, d]
-  const int32_t* expert_offset;  // [N + 1]
-  const uint16_t* w_gate_up;     // [N, 2F, d]
-  const uint16_t* w_down;        // [N, d, F]
-  uint16_t* h;                   // [r_max, F]
-  float* y_perm;                 // [r_max, d]
-  float* part;                   // decode_ffn_part_bytes(): the chunks' partials
-  int* sync;                     // kDecodeFfnSyncInts, zero between calls
-  int* flags;                    // the rest of decode_ffn_counter_bytes(), zero between calls
-  int N, d, F, T, k;
-  int64_t r_max;
-  int* status;
-  uint64_t timeout_ns;
-  // combine (out non-null): out = residual + sum_j w_j y[row(t, j)], as moe_unpermute_combine
-  const int32_t* row_of_pair;
-  const float* topk_w;
-  const uint16_t* residual;  // may be null
-  void* out;
-  int out_f32;
-  // routing in the same launch (route_in_kernel): the decode router with its permute outputs;
-  // then x_perm and expert_offset above are the router's outputs
-  bool route_in_kernel;
-  DecodeRouteArgs route;
-};
-cudaError_t launch_decode_ffn(const DecodeFfnArgs& a, cudaStream_t s);
-
 // Backward pass (backward.cu). Saved from the forward: the routing, x_perm and y_perm.
 struct BackwardArgs {
   const uint16_t* d_out;          // [T, d] bf16

@@ -64,19 +64,12 @@ def test_workspace_sizes():
     assert moe.workspace_bytes(big) == (256 + counters(416, 0, 0) + 32 * 256 * 4
                                         + 3 * 256 * 7168 * 2 + 128 * 256 * 4)
     decode = moe.make_dims(4, 2880, 32, 4, 2880, "swiglu", 4)
-    # status word (+ the decode router's arrival counter) + the larger of the grouped FFN's
-    # counters (at most 1 + 16 m-tiles: 17 x 23 gate/up and 17 x 12 down tiles) and the decode
-    # FFN's (4 + for each of 16 experts x 23 gate/up tiles of 128 columns a flag and a chunk
-    # count + a chunk count for each of 16 x 12 down tiles of 256 rows + a count for each of
-    # the 12 row blocks) + the larger of the grouped FFN's two 4-row partial slots per CTA for
-    # each GEMM (148 + 148 CTAs) and the decode FFN's scratch: the decode router's partial dot
-    # products (23 slices x 4 tokens x 32 experts) and one 8 x 256 fp32 partial per chunk. The
-    # 25200 units of 64 k (16 x 23 x 45 + 16 x 12 x 45) make chunks of 21 units: 3 per tile.
-    decode_counters = -(-((4 + 2 * 16 * 23 + 16 * 12 + 12) * 4) // 256) * 256
-    chunks = (16 * 23 + 16 * 12) * 3
-    assert moe.workspace_bytes(decode) == (256 + max(counters(17, 17 * 23, 17 * 12), decode_counters)
-                                           + max(296 * 2 * 4 * 256 * 4,
-                                                 23 * 4 * 32 * 4 + chunks * 8 * 256 * 4))
+    # status word (+ the decode router's arrival counter) + counters (at most 1 + 16 m-tiles:
+    # 17 x 23 gate/up and 17 x 12 down tiles) + the larger of the decode router's partial dot
+    # products (23 slices x 4 tokens x 32 experts) and two 4-row partial slots per CTA for each
+    # GEMM (148 + 148 CTAs)
+    assert moe.workspace_bytes(decode) == (256 + counters(17, 17 * 23, 17 * 12)
+                                           + max(23 * 4 * 32 * 4, 296 * 2 * 4 * 256 * 4))
     fb = moe.forward_workspace_bytes(big)
     assert fb > 20480 * 7168 * 6
 

@@ -57,13 +57,11 @@ def test_launch_counts():
     assert bench.launches_per_step(16384, 8, 20480, 256, 7168) == 8
     # mid-size: per-token router, one slot pass, permute, grouped FFN, combine
     assert bench.launches_per_step(64, 4, 256, 32, 2880) == 5
-    # SwiGLU decode, at most 8 tokens: one launch routes, sorts, runs the FFN and combines
-    assert bench.launches_per_step(1, 2, 2, 8, 4096) == 1
-    assert bench.launches_per_step(8, 4, 32, 32, 2880) == 1
-    # ... unless x_perm exceeds 512 KB (8 tokens x 8 choices x 7168): routing, permute, FFN
-    assert bench.launches_per_step(8, 8, 64, 256, 7168) == 3
-    # GELU decode: one launch routes and sorts, grouped FFN, combine
-    assert bench.launches_per_step(1, 2, 2, 8, 4096, "gelu") == 3
+    # decode: one launch routes and sorts, grouped FFN, combine
+    assert bench.launches_per_step(1, 2, 2, 8, 4096) == 3
+    assert bench.launches_per_step(8, 4, 32, 32, 2880) == 3
+    # ... a separate permute when x_perm exceeds 512 KB (8 tokens x 8 choices x 7168)
+    assert bench.launches_per_step(8, 8, 64, 256, 7168) == 4
     # decode with an x_perm above 512 KB (16 tokens x 8 choices x 7168): separate permute
     assert bench.launches_per_step(16, 8, 128, 256, 7168) == 4
     # no rows can be kept: routing (and sort) and the combine only

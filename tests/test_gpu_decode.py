@@ -1,9 +1,9 @@
-"""The decode path (at most 8 tokens, SwiGLU): the expert FFN cut along d_ff into 64-column
-slices, each computed whole by one CTA, with y the sum of the slices' fp32 partials in a fixed
-order; in moe_forward also the routing and the combine in the same launch (GPU).
+"""The decode path (at most 8 tokens, SwiGLU): the one-launch decode router with the sort by
+expert, the grouped FFN with every expert's weights cut along d_ff over all SMs (stream-K, fp32
+partials added in a fixed order), the combine (GPU).
 
-Checked against the CPU oracle on the GPU's own logits, and the one-launch moe_forward against
-the four stage calls bit for bit (routing, permutation, h, y_perm and the output)."""
+Checked against the CPU oracle on the GPU's own logits, and moe_forward against the four stage
+calls bit for bit (routing, permutation, h, y_perm and the output)."""
 import numpy as np
 import pytest
 import torch
@@ -19,8 +19,8 @@ CASES = [
     (1, 2880, 32, 4, 2880, None, None, True),     # gpt-oss-shaped token, d not a multiple of 128
     (8, 512, 2, 2, 512, None, None, True),        # both experts hold exactly 8 rows
     (8, 256, 8, 2, 320, 1, 1.1, True),            # capacity 1: most pairs dropped, skewed loads
-    (6, 320, 6, 3, 64, 2, None, False),           # one slice per expert, no residual
-    (4, 1024, 64, 8, 2048, None, 1.1, True),      # many experts, 32 slices each
+    (6, 320, 6, 3, 64, 2, None, False),           # d_ff of one k block, no residual
+    (4, 1024, 64, 8, 2048, None, 1.1, True),      # many experts
     (7, 192, 5, 5, 128, None, None, True),        # k = N: every expert active
 ]
 
@@ -57,9 +57,9 @@ def test_decode_stage_parity(case):
 
 
 @pytest.mark.parametrize("case", CASES, ids=_ids)
-def test_decode_forward_one_launch_matches_stages(case):
-    """moe_forward routes, runs the FFN and combines in one launch; every buffer it writes
-    equals the stage calls' bit for bit, on two calls in a row (the counters return to zero)."""
+def test_decode_forward_matches_stages(case):
+    """Every buffer moe_forward writes equals the stage calls' bit for bit, on two calls in a row
+    (the counters return to zero)."""
     import sparse_mixture_experts_11_b200 as moe
     T, d, N, k, F, cap, zipf, residual = case
     inp = synthetic.make_custom_inputs(T, d, N, F, "swiglu", seed=17, device="cuda", zipf_s=zipf)
