@@ -52,6 +52,9 @@
 #include <algorithm>
 #include <mutex>
 
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "launch.h"
 #include "tma_host.h"
@@ -140,59 +143,39 @@ struct Cfg {
 };
 
 // Decoders of one MX row segment: 8 elements and the block scale X = 2^(s - 127) -> 8 bf16
-// (one 16-byte chunk), without conversion instructions (their throughput held the decode to
-// about 11 elements per clock per SM). Each element's value is formed in bf16 bits exactly, then
-// multiplied by the power-of-two scale in bf16x2 arithmetic, exact while the result is a normal
-// bf16 (a power of two only moves the exponent):
-//   E2M1: a byte permute looks up the high and the low byte of the bf16 of each of the eight
-//         magnitudes (0, 0.5, 1, 1.5, 2, 3, 4, 6), indexed by the code's three low bits; the
-//         sign bit moves to bit 15;
-//   E4M3: the code's exponent and mantissa bits placed at bf16 bits 4-14 (and its sign at 15)
-//         are the bf16 of value * 2^-120, normal or subnormal alike (both formats give 2^-6 and
-//         2^-126 the same subnormal steps relative to their biases); times 2^120 it is the value.
-//         The NaN codes S.1111.111 are set to NaN.
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
-  const __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&a),
-                                   *reinterpret_cast<const __nv_bfloat162*>(&b));
-  return *reinterpret_cast<const uint32_t*>(&r);
+// (one 16-byte chunk). Elements convert exactly to fp16 (CUDA's FP8/FP4 conversions), then
+// to fp32; the product with a power of two and the final bf16 rounding are exact while the
+// result stays in bf16's normal range.
+__device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
+  if (s == 255u) return __uint_as_float(0x7fc00000u);
+  if (s == 0u) return __uint_as_float(0x00400000u);  // 2^-127
+  return __uint_as_float(s << 23);
 }
 
-// E8M0 scale code -> 2^(s - 127) in both bf16 halves (s = 0: 2^-127, subnormal; 255: NaN).
-__device__ __forceinline__ uint32_t e8m0_to_bf16x2(uint32_t s) {
-  const uint32_t b = s == 255u ? 0x7FC0u : (s == 0u ? 0x0040u : (s << 7));
-  return b | (b << 16);
+__device__ __forceinline__ uint32_t half2raw_to_bf16x2(__half2_raw h, float x) {
+  __half_raw lo, hi;
+  lo.x = h.x;
+  hi.x = h.y;
+  return pack_bf16x2(__half2float(__half(lo)) * x, __half2float(__half(hi)) * x);
 }
 
-__device__ __forceinline__ uint4 decode8_e4m3(uint2 w, uint32_t sc2) {
-  constexpr uint32_t kTwo120 = 0x7B807B80u;  // bf16 2^120 in both halves
+__device__ __forceinline__ uint4 decode8_e4m3(uint2 w, float x) {
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t word = i < 2 ? w.x : w.y;
-    const uint32_t u = __byte_perm(word, 0u, (i & 1) ? 0x4342u : 0x4140u);  // two codes, one per half
-    const uint32_t em = u & 0x007F007Fu;
-    const uint32_t b = (em << 4) | ((u & 0x00800080u) << 8);
-    const uint32_t nan = __vcmpeq2(em, 0x007F007Fu) & 0x7FC07FC0u;
-    o[i] = bf16x2_mul(bf16x2_mul(b, kTwo120), sc2) | nan;
+    const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>(word >> (16 * (i & 1)));
+    o[i] = half2raw_to_bf16x2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3), x);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__device__ __forceinline__ uint4 decode8_e2m1(uint32_t w, uint32_t sc2) {
-  // bf16 bytes of the magnitudes, indexed by the three low code bits
-  constexpr uint32_t kHi03 = 0x3F3F3F00u, kHi47 = 0x40404040u;
-  constexpr uint32_t kLo03 = 0xC0800000u, kLo47 = 0xC0804000u;
+__device__ __forceinline__ uint4 decode8_e2m1(uint32_t w, float x) {
   uint32_t o[4];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {  // elements 4h .. 4h + 3: element 2i is the low nibble of byte i
-    const uint32_t n = (w >> (16 * h)) & 0xFFFFu;
-    const uint32_t sel = n & 0x7777u;
-    const uint32_t hi = __byte_perm(kHi03, kHi47, sel);
-    const uint32_t lo = __byte_perm(kLo03, kLo47, sel);
-    const uint32_t w0 = __byte_perm(lo, hi, 0x5140u) | ((n & 0x8u) << 12) | ((n & 0x80u) << 24);
-    const uint32_t w1 = __byte_perm(lo, hi, 0x7362u) | ((n & 0x800u) << 4) | ((n & 0x8000u) << 16);
-    o[2 * h] = bf16x2_mul(w0, sc2);
-    o[2 * h + 1] = bf16x2_mul(w1, sc2);
+  for (int i = 0; i < 4; ++i) {  // byte i holds elements 2i (low nibble) and 2i + 1
+    const __nv_fp4x2_storage_t pair = static_cast<__nv_fp4x2_storage_t>(w >> (8 * i));
+    o[i] = half2raw_to_bf16x2(__nv_cvt_fp4x2_to_halfraw2(pair, __NV_E2M1), x);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -901,8 +884,8 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
           }
           const uint8_t* stg = dyn_smem + (stg0 - smem_u32(dyn_smem)) + s2 * C::STG_BYTES;
           const uint8_t* scl = stg + kUmmaN * 128;
-          const uint32_t x0 = e8m0_to_bf16x2(scl[sc_base + (2 * j) * sc_step]);
-          const uint32_t x1 = e8m0_to_bf16x2(scl[sc_base + (2 * j + 1) * sc_step]);
+          const float x0 = e8m0_to_f32(scl[sc_base + (2 * j) * sc_step]);
+          const float x1 = e8m0_to_f32(scl[sc_base + (2 * j + 1) * sc_step]);
           // this k block's part of the packed row (64 or 32 bytes), then the eight chunks
           constexpr int kQ = C::ROW_BYTES / 16;
           uint4 raw[kQ];
@@ -913,7 +896,7 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
           uint8_t* bdst = dyn_smem + (b_addr(s) - smem_u32(dyn_smem)) + r * 128;
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
-            const uint32_t x = ch < 4 ? x0 : x1;  // elements 0..31: block 0; 32..63: block 1
+            const float x = ch < 4 ? x0 : x1;  // elements 0..31: block 0; 32..63: block 1
             uint4 v;
             if (WFMT == WFMT_MXFP8)
               v = decode8_e4m3(make_uint2(wd[2 * ch], wd[2 * ch + 1]), x);
