@@ -43,6 +43,7 @@ SWEEP = ("tiny_top2:64", "switch_top1:4096", "mixtral:1", "mixtral:16", "mixtral
          "mixtral:8192", "gpt_oss:1", "gpt_oss:8", "gpt_oss:64", "gpt_oss:16384",
          "fine_grained:16384")
 DECODE_MIN_STEPS = 100  # sweep points with T <= 64 time at least this many steps
+SWEEP_SETTLE_S = 2.0    # idle seconds before each sweep point
 METRIC = "MoE-layer fwd tokens/s on 1 B200; % of bf16 tensor peak / % of HBM BW"
 MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -732,6 +733,10 @@ def run_sweep(args, device, flush, peaks, headline=None) -> dict:
         steps = max(args.steps, DECODE_MIN_STEPS) if T <= 64 else args.steps
         layer = Layer(shape, T, device, wfmt=args.wfmt, weights=cache.get("weights"))
         cache["weights"] = layer.inp
+        # an idle pause first: a point timed right after a power-capped one (the large prefill
+        # GEMMs hold a 1 kW part at its power limit) otherwise starts at the capped clock
+        torch.cuda.synchronize()
+        time.sleep(SWEEP_SETTLE_S)
         clocks = ClockSampler(torch.cuda.current_device())
         step_ms, stage_ms, clk = measure_forward(layer, steps, args.warmup, flush, clocks=clocks)
         entry = sweep_entry(layer, spec, step_ms, stage_ms, peaks)
@@ -741,7 +746,7 @@ def run_sweep(args, device, flush, peaks, headline=None) -> dict:
     cache.clear()
     torch.cuda.empty_cache()
     return {"points": out,
-            "timing": "per point: the whole forward as one captured graph, L2 flushed before "
+            "timing": "per point, after a 2 s idle pause: the whole forward as one captured graph, L2 flushed before "
                       "every step; mean (and median) of the timed steps; grouped FFN from the "
                       "stage-by-stage pass; clocks sampled over each point's timed steps"}
 

@@ -47,6 +47,7 @@ __device__ __forceinline__ void block_offsets_256(const int32_t* __restrict__ co
 constexpr int kGroupCols = 256;  // columns per warp step: 8 per lane
 constexpr int kGroupsInFlight = 4;  // permute
 constexpr int kCombInFlight = 2;    // combine: its fp32 sums take the registers
+constexpr int kCopyInFlight = 6;    // combine of a token with no kept pair: a plain copy
 
 __device__ __forceinline__ void token_part(int64_t item, int parts, int groups, int& t, int& g0,
                                            int& g1) {
@@ -159,6 +160,34 @@ __global__ void __launch_bounds__(256, kCombBlocksPerSm) combine_kernel(
     }
     const int nkept = __popc(__ballot_sync(kFull, lane < k && row >= 0));
     const uint4* res = reinterpret_cast<const uint4*>(residual + static_cast<int64_t>(t) * d);
+    if (nkept == 0) {
+      // every choice dropped: the residual passes through unchanged, six groups in flight
+      for (int g = g0; g < g1; g += kCopyInFlight) {
+        uint4 rb[kCopyInFlight];
+#pragma unroll
+        for (int i = 0; i < kCopyInFlight; ++i) {
+          const int col = (g + i) * kGroupCols + lane * 8;
+          rb[i] = make_uint4(0u, 0u, 0u, 0u);
+          if (residual != nullptr && g + i < g1 && col < d) rb[i] = res[col / 8];
+        }
+#pragma unroll
+        for (int i = 0; i < kCopyInFlight; ++i) {
+          const int col = (g + i) * kGroupCols + lane * 8;
+          if (g + i >= g1 || col >= d) continue;
+          const int64_t o = static_cast<int64_t>(t) * d + col;
+          if (out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + o);
+            dst[0] = make_float4(__uint_as_float(rb[i].x << 16), __uint_as_float(rb[i].x & 0xffff0000u),
+                                 __uint_as_float(rb[i].y << 16), __uint_as_float(rb[i].y & 0xffff0000u));
+            dst[1] = make_float4(__uint_as_float(rb[i].z << 16), __uint_as_float(rb[i].z & 0xffff0000u),
+                                 __uint_as_float(rb[i].w << 16), __uint_as_float(rb[i].w & 0xffff0000u));
+          } else {
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + o) = rb[i];
+          }
+        }
+      }
+      continue;
+    }
     for (int g = g0; g < g1; g += kCombInFlight) {
       uint4 rb[kCombInFlight];
 #pragma unroll
