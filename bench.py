@@ -148,9 +148,10 @@ def roofline_of(shape, T: int, R: int, active: int, ffn_ms: float, step_ms: floa
         per_launch, src = f"{ab['weights']} B", peaks["source"] + " copy"
     ffn = {"bound": "tensor" if tensor else "hbm", "achieved": round(ach, 1), "peak": peak,
            "unit": unit, "frac": round(ach / peak, 4), "per_launch": per_launch,
-           "peak_source": src, "traffic": traffic,
-           "traffic_over_algorithmic": (round(traffic / ab["weights"], 3)
-                                        if traffic and not tensor else None)}
+           "peak_source": src, "traffic": int(traffic) if traffic else None,
+           # over the weights, each read once: HBM-bound points show re-reads; tensor-bound
+           # points add the activations (x_perm, h, y_perm) that spill out of L2
+           "traffic_over_weights": round(traffic / ab["weights"], 3) if traffic else None}
     layer_gbs = ab["layer"] / step_s / 1e9
     layer = {"achieved_gbs": round(layer_gbs, 1), "frac_hbm": round(layer_gbs / peaks["hbm_gbs"], 4),
              "algorithmic_bytes": ab["layer"]}
@@ -193,9 +194,21 @@ def launches_per_step(T: int, k: int, R_max: int, n_experts: int = 1, d_model: i
 
 
 # DRAM traffic of the grouped-FFN stage per forward (dram__bytes_read.sum +
-# dram__bytes_write.sum of its launch) from one ncu capture of the current kernel; workloads
-# without a capture of the current kernel report null.
-MEASURED_FFN_TRAFFIC = {("switch_top1", 4096): 1086589696 + 9595904}
+# dram__bytes_write.sum of one launch, as ncu prints them: three significant digits) from one
+# capture per workload of the current kernel; workloads without one report null.
+MEASURED_FFN_TRAFFIC = {
+    ("tiny_top2", 64): 1.67e6,
+    ("switch_top1", 4096): 1.09e9 + 10.68e6,
+    ("mixtral", 1): 709.46e6 + 3.15e6,
+    ("mixtral", 16): 2.82e9 + 4.78e6,
+    ("mixtral", 512): 2.86e9 + 45.51e6,
+    ("mixtral", 8192): 4.39e9 + 730.11e6,
+    ("gpt_oss", 1): 201.80e6 + 3.36e6,
+    ("gpt_oss", 8): 958.33e6 + 3.38e6,
+    ("gpt_oss", 64): 1.61e9 + 5.67e6,
+    ("gpt_oss", 16384): 2.35e9 + 1.09e9,
+    ("fine_grained", 16384): 19.44e9 + 181.11e6,
+}
 
 
 def load_peaks():
