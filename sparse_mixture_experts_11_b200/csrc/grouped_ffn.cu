@@ -121,9 +121,8 @@ struct Cfg {
   static constexpr int KG = MX ? 128 / ROW_BYTES : 1;
   static constexpr int STG_BYTES = MX ? kUmmaN * 128 + 2 * KG * kUmmaN : 0;
   static constexpr int STAGES_FIT = (kSmemBudget / STAGE_BYTES) > 8 ? 8 : (kSmemBudget / STAGE_BYTES);
-  // MX: three bf16 stages, so the decoders run a stage ahead of the MMA's round trip
-  // (decode, MMA, commit, stage free), and the rest of 224 KB for packed stages
-  // MX: two bf16 B stages (decoded from shared memory), a separate ring of SA A stages
+  // MX: two bf16 B stages (decoded from shared memory; a third measured no faster), a
+  // separate ring of SA A stages
   // (token rows, loaded ahead of the decoders: an A copy waits on L2 for about 1.7 us when
   // the weight streams load it), and the rest of 224 KB for packed stages
   static constexpr int kMxBudget = 224 * 1024;
