@@ -52,11 +52,14 @@ constexpr int kBK = 64;    // k per block (one 128-byte swizzle row of bf16)
 constexpr int kThreads = 256;
 constexpr int kConvThreads = 128;
 constexpr int kSmemLimit = 225 * 1024;
+constexpr uint64_t kPairDrainNs = 1000000;  // 1 ms
 
-template <int NP, bool PRESPLIT>
+template <int NP, bool PRESPLIT, bool PAIR = false>
 struct RCfg {
+  static_assert(!PAIR || PRESPLIT, "CTA pairs load the split terms by TMA");
   static constexpr int A_BYTES = kTok * kBK * 2;           // 16 KB per x tile
-  static constexpr int WT_BYTES = NP * kBK * 2;            // one split term tile
+  static constexpr int WROWS = PAIR ? NP / 2 : NP;         // term rows held by this CTA
+  static constexpr int WT_BYTES = WROWS * kBK * 2;         // one split term tile
   static constexpr int WBUF_BYTES = 3 * WT_BYTES;          // hi, mid, lo
   // PRESPLIT: each ring stage holds the x tile and the three term tiles.
   // in-kernel: a ring of x tiles plus two converter-written term buffers.
@@ -68,9 +71,11 @@ struct RCfg {
   static constexpr int SMEM_BYTES = FIXED_BYTES + STAGES * STAGE_BYTES + 1024;
   static_assert(STAGES >= 2, "router pipeline depth");
   static_assert(NP % 16 == 0 && NP >= 16 && NP <= 256, "UMMA N for M = 128");
+  static_assert(!PAIR || NP % 32 == 0, "UMMA N for a CTA pair (M = 256)");
   static_assert(kTok * (NP + 4) * 4 <= SMEM_BYTES - 1024, "logits staging fits the pipeline smem");
-  // with a k split: the staged partials plus the final rows of this CTA (at most 64)
-  static_assert((kTok + kTok / 2) * (NP + 4) * 4 <= SMEM_BYTES - 1024,
+  // with a k split (never with a CTA pair): the staged partials plus the final rows of this CTA
+  // (at most 64)
+  static_assert(PAIR || (kTok + kTok / 2) * (NP + 4) * 4 <= SMEM_BYTES - 1024,
                 "k-split staging (partials + final rows) fits the pipeline smem");
 };
 
@@ -238,14 +243,14 @@ __device__ __forceinline__ bool tile_prob_sums(float m, float* buf, int rows, in
   return true;
 }
 
-template <int NP, bool PRESPLIT, int KMAX>
+template <int NP, bool PRESPLIT, int KMAX, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ w, const float* __restrict__ bias,
                      float* __restrict__ logits, int32_t* __restrict__ topk_idx,
                      float* __restrict__ topk_w, int T, int d, int N, int k, int* status,
                      uint64_t timeout_ns, float* __restrict__ prob_part, int ksplit) {
-  using C = RCfg<NP, PRESPLIT>;
+  using C = RCfg<NP, PRESPLIT, PAIR>;
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t a_full[C::STAGES];
   __shared__ __align__(8) uint64_t a_empty[C::STAGES];
@@ -266,6 +271,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ksplit > 1: a cluster of ksplit CTAs shares one token tile, CTA `rank` taking k blocks
   // [kb_lo, kb_hi); the leader (rank 0) adds the partial logits in rank order
   const int rank = ksplit > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  // PAIR: the cluster's two CTAs take neighbouring token tiles, and the even CTA issues M = 256
+  // MMAs over both (its peer holds the other 128 tokens and the upper NP / 2 rows of each term)
+  const int prank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const bool mma_cta = prank == 0;
   const int t0 = (blockIdx.x / ksplit) * kTok;
   const int num_kb = d / kBK;
   const int kb_lo = rank * num_kb / ksplit, kb_hi = (rank + 1) * num_kb / ksplit;
@@ -294,8 +303,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 1) {
     __syncwarp();
-    tmem_alloc(smem_u32(&s_tmem), C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(&s_tmem), C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&s_tmem), C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   if (!PRESPLIT && warp >= 4 && NP > N) {
     // rows N..NP-1 of both term buffers stay zero for the whole kernel
@@ -311,7 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   pdl_wait();  // everything below reads the previous kernels' outputs or writes global memory
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();  // both CTAs' barriers and TMEM exist before either CTA uses the other's
+  else
+    __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = s_tmem;
 
@@ -331,25 +348,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t st = ring0 + s * C::STAGE_BYTES;
         const uint32_t fb = smem_u32(&a_full[s]);
-        mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-        tma_load_2d(st, &tmX, fb, kb * kBK, t0, pol_x);
-        if (PRESPLIT) {
+        if constexpr (PAIR) {
+          // both CTAs' bytes complete on the even CTA's barrier, which the even CTA arms
+          const uint32_t fb0 = map_smem_to_rank(fb, 0);
+          if (mma_cta) mbar_arrive_expect_tx(fb, 2 * C::STAGE_BYTES);
+          tma_load_2d_pair(st, &tmX, fb0, kb * kBK, t0, pol_x);
 #pragma unroll
           for (int term = 0; term < 3; ++term)
-            tma_load_3d(st + C::A_BYTES + term * C::WT_BYTES, &tmW, fb, kb * kBK, 0, term, pol_w);
+            tma_load_3d_pair(st + C::A_BYTES + term * C::WT_BYTES, &tmW, fb0, kb * kBK,
+                             prank * C::WROWS, term, pol_w);
+        } else {
+          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          tma_load_2d(st, &tmX, fb, kb * kBK, t0, pol_x);
+          if (PRESPLIT) {
+#pragma unroll
+            for (int term = 0; term < 3; ++term)
+              tma_load_3d(st + C::A_BYTES + term * C::WT_BYTES, &tmW, fb, kb * kBK, 0, term, pol_w);
+          }
         }
       }
       if (!ok) {
         s_abort = 1;
         report_error(status, MOE_ERR_TIMEOUT);
       }
-      for (int j = max(0, i - C::STAGES); j < i; ++j)
-        mbar_wait(smem_u32(&a_full[j % C::STAGES]), (j / C::STAGES) & 1, kDrainTimeoutNs, nullptr);
+      if (!PAIR || mma_cta) {
+        for (int j = max(0, i - C::STAGES); j < i; ++j)
+          mbar_wait(smem_u32(&a_full[j % C::STAGES]), (j / C::STAGES) & 1, kDrainTimeoutNs, nullptr);
+      } else {
+        // the odd CTA's copies complete on the even CTA's barriers: it waits until the MMAs have
+        // released its last stages (so they landed), within one overall limit that leaves any
+        // copy still in flight after a timeout ample time to land
+        const uint64_t t_end = globaltimer_ns() + kPairDrainNs;
+        for (int j = max(0, i - C::STAGES); j < i; ++j) {
+          const uint64_t now = globaltimer_ns();
+          mbar_wait(smem_u32(&a_empty[j % C::STAGES]), (j / C::STAGES) & 1,
+                    now < t_end ? t_end - now : 1, nullptr);
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kTok, NP);
+    if (lane == 0 && PAIR && !mma_cta) {
+      // the odd CTA of a pair issues nothing; its TMEM and shared memory stay in use until
+      // the even CTA's MMAs are done (the even CTA always signals this barrier at the end)
+      mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
+    } else if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * kTok : kTok, NP);
       bool ok = true, issued = false;
       for (int i = 0; i < n_it; ++i) {
         const int s = i % C::STAGES, b = i & 1;
@@ -365,23 +409,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int term = 0; term < 3; ++term) {
           const uint32_t bt = wt0 + term * C::WT_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            tc_mma_f16(tmem, smem_desc_k_sw128(a + kk * 32), smem_desc_k_sw128(bt + kk * 32), idesc,
-                       (i | term | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = smem_desc_k_sw128(a + kk * 32), bd = smem_desc_k_sw128(bt + kk * 32);
+            const uint32_t acc = (i | term | kk) != 0 ? 1u : 0u;
+            if constexpr (PAIR)
+              tc_mma_f16_pair(tmem, ad, bd, idesc, acc);
+            else
+              tc_mma_f16(tmem, ad, bd, idesc, acc);
+          }
         }
         issued = true;
-        tc_commit(smem_u32(&a_empty[s]));
-        if (!PRESPLIT) tc_commit(smem_u32(&w_empty[b]));
+        if constexpr (PAIR) {
+          tc_commit_pair(smem_u32(&a_empty[s]), 0x3);  // the stage is free in both CTAs
+        } else {
+          tc_commit(smem_u32(&a_empty[s]));
+          if (!PRESPLIT) tc_commit(smem_u32(&w_empty[b]));
+        }
       }
       if (ok) {
-        tc_commit(smem_u32(&acc_full));
+        if constexpr (PAIR)
+          tc_commit_pair(smem_u32(&acc_full), 0x3);
+        else
+          tc_commit(smem_u32(&acc_full));
       } else {
         s_abort = 1;
         report_error(status, MOE_ERR_TIMEOUT);
       }
       // every issued MMA has finished before TMEM is freed, also when the epilogue gave up
       // waiting for the accumulator
-      if (issued) {
+      if constexpr (PAIR) {
+        tc_commit_pair(smem_u32(&done_bar), 0x3);
+        mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
+      } else if (issued) {
         tc_commit(smem_u32(&done_bar));
         mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
       }
@@ -601,10 +660,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();  // neither CTA of a pair frees TMEM or exits while the other works
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -619,55 +684,79 @@ int router_ksplit(int tiles, int num_kb) {
   return ks;
 }
 
-template <int NP, bool PRESPLIT, int KMAX>
+// CTA pairs for the pre-split path when every tile has a CTA of its own and the tiles pair up:
+// the even CTA's M = 256 MMAs take half of each term tile from each CTA's shared memory, so a
+// CTA loads and its tensor core reads half the weight bytes per MMA (shared-memory bandwidth,
+// not the MMA rate, bounds the unpaired kernel at N = 256).
+bool router_pairs(int tiles, int num_kb, int np, bool presplit) {
+  return presplit && np >= 128 && tiles % 2 == 0 && router_ksplit(tiles, num_kb) == 1;
+}
+
+template <int NP, bool PRESPLIT, int KMAX, bool PAIR>
 cudaError_t launch_npk(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
                        const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
                        int d, int N, int k, int* status, uint64_t timeout_ns, float* prob_part, cudaStream_t s) {
-  using C = RCfg<NP, PRESPLIT>;
+  using C = RCfg<NP, PRESPLIT, PAIR>;
+  auto kernel = router_tc_kernel<NP, PRESPLIT, KMAX, PAIR>;
   static PerDeviceOnce once;
-  const cudaError_t attr = once.run([] {
-    return cudaFuncSetAttribute(router_tc_kernel<NP, PRESPLIT, KMAX>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  const cudaError_t attr = once.run([kernel] {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr != cudaSuccess) return attr;
   const int tiles = (T + kTok - 1) / kTok;
+  if constexpr (PAIR)
+    return launch_pdl_cluster(kernel, dim3(tiles), dim3(kThreads), C::SMEM_BYTES, s, 2u, mx, mw, w,
+                              bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns,
+                              prob_part, 1);
   const int ksplit = router_ksplit(tiles, d / kBK);
   if (ksplit == 1)
-    return launch_pdl(router_tc_kernel<NP, PRESPLIT, KMAX>, dim3(tiles), dim3(kThreads),
-                      C::SMEM_BYTES, s, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k,
-                      status, timeout_ns, prob_part, 1);
-  return launch_pdl_cluster(router_tc_kernel<NP, PRESPLIT, KMAX>, dim3(tiles * ksplit),
-                            dim3(kThreads), C::SMEM_BYTES, s, static_cast<unsigned>(ksplit), mx, mw,
-                            w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part,
-                            ksplit);
+    return launch_pdl(kernel, dim3(tiles), dim3(kThreads), C::SMEM_BYTES, s, mx, mw, w, bias,
+                      logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, 1);
+  return launch_pdl_cluster(kernel, dim3(tiles * ksplit), dim3(kThreads), C::SMEM_BYTES, s,
+                            static_cast<unsigned>(ksplit), mx, mw, w, bias, logits, topk_idx,
+                            topk_w, T, d, N, k, status, timeout_ns, prob_part, ksplit);
+}
+
+template <int NP, bool PRESPLIT, int KMAX>
+cudaError_t launch_npkp(bool pair, const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
+                        const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
+                        int d, int N, int k, int* status, uint64_t timeout_ns, float* prob_part,
+                        cudaStream_t s) {
+  if constexpr (PRESPLIT && NP >= 128) {
+    if (pair)
+      return launch_npk<NP, true, KMAX, true>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N,
+                                              k, status, timeout_ns, prob_part, s);
+  }
+  return launch_npk<NP, PRESPLIT, KMAX, false>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N,
+                                               k, status, timeout_ns, prob_part, s);
 }
 
 template <int NP, bool PRESPLIT>
-cudaError_t launch_np(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
+cudaError_t launch_np(bool pair, const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
                       const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
                       int d, int N, int k, int* status, uint64_t timeout_ns, float* prob_part, cudaStream_t s) {
   if (k <= 1)
-    return launch_npk<NP, PRESPLIT, 1>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+    return launch_npkp<NP, PRESPLIT, 1>(pair, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
   if (k <= 2)
-    return launch_npk<NP, PRESPLIT, 2>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+    return launch_npkp<NP, PRESPLIT, 2>(pair, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
   if (k <= 4)
-    return launch_npk<NP, PRESPLIT, 4>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
-  return launch_npk<NP, PRESPLIT, 8>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+    return launch_npkp<NP, PRESPLIT, 4>(pair, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+  return launch_npkp<NP, PRESPLIT, 8>(pair, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
 }
 
 template <bool PRESPLIT>
-cudaError_t launch_tc(const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
+cudaError_t launch_tc(bool pair, const CUtensorMap& mx, const CUtensorMap& mw, const float* w,
                       const float* bias, float* logits, int32_t* topk_idx, float* topk_w, int T,
                       int d, int N, int k, int* status, uint64_t timeout_ns, float* prob_part, cudaStream_t s) {
   if (N <= 16)
-    return launch_np<16, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+    return launch_np<16, PRESPLIT>(pair, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
   if (N <= 32)
-    return launch_np<32, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+    return launch_np<32, PRESPLIT>(pair, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
   if (N <= 64)
-    return launch_np<64, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+    return launch_np<64, PRESPLIT>(pair, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
   if (N <= 128)
-    return launch_np<128, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
-  return launch_np<256, PRESPLIT>(mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+    return launch_np<128, PRESPLIT>(pair, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
+  return launch_np<256, PRESPLIT>(pair, mx, mw, w, bias, logits, topk_idx, topk_w, T, d, N, k, status, timeout_ns, prob_part, s);
 }
 
 bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
@@ -703,13 +792,15 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const flo
   const int np = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
   if (split_scratch == nullptr) {
     memset(&mw, 0, sizeof(mw));  // unused by the in-kernel split
-    return launch_tc<false>(mx, mw, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status,
-                            timeout_ns, prob_part, s);
+    return launch_tc<false>(false, mx, mw, w_router, bias, logits, topk_idx, topk_w, T, d, N, k,
+                            status, timeout_ns, prob_part, s);
   }
+  const bool pair = router_pairs((T + kTok - 1) / kTok, d / kBK, np, true);
   {
+    // a CTA of a pair loads rows [rank * np / 2, rank * np / 2 + np / 2) of each term
     const cuuint64_t gd[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), 3};
     const cuuint64_t gs[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-    const cuuint32_t box[3] = {kBK, static_cast<cuuint32_t>(np), 1};
+    const cuuint32_t box[3] = {kBK, static_cast<cuuint32_t>(pair ? np / 2 : np), 1};
     if (!encode_bf16(&mw, split_scratch, 3, gd, gs, box)) return cudaErrorInvalidValue;
   }
   const int64_t n = static_cast<int64_t>(N) * d;
@@ -717,8 +808,8 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* w_router, const flo
   cudaError_t e = launch_pdl(split_router_weights_kernel, dim3(blocks), dim3(256), 0, s, w_router,
                              split_scratch, n);
   if (e != cudaSuccess) return e;
-  return launch_tc<true>(mx, mw, w_router, bias, logits, topk_idx, topk_w, T, d, N, k, status,
-                         timeout_ns, prob_part, s);
+  return launch_tc<true>(pair, mx, mw, w_router, bias, logits, topk_idx, topk_w, T, d, N, k,
+                         status, timeout_ns, prob_part, s);
 }
 
 }  // namespace moe
