@@ -53,6 +53,7 @@ constexpr int kThreads = 256;
 constexpr int kConvThreads = 128;
 constexpr int kSmemLimit = 225 * 1024;
 constexpr uint64_t kPairDrainNs = 1000000;  // 1 ms
+constexpr int kCand = 96;  // listed top-k candidates per token in the epilogue
 
 template <int NP, bool PRESPLIT, bool PAIR = false>
 struct RCfg {
@@ -73,6 +74,8 @@ struct RCfg {
   static_assert(NP % 16 == 0 && NP >= 16 && NP <= 256, "UMMA N for M = 128");
   static_assert(!PAIR || NP % 32 == 0, "UMMA N for a CTA pair (M = 256)");
   static_assert(kTok * (NP + 4) * 4 <= SMEM_BYTES - 1024, "logits staging fits the pipeline smem");
+  static_assert(kTok * (NP + 1) * 4 + kCand * kTok <= SMEM_BYTES - 1024,
+                "logits staging and the top-k candidate lists fit the pipeline smem");
   // with a k split (never with a CTA pair): the staged partials plus the final rows of this CTA
   // (at most 64)
   static_assert(PAIR || (kTok + kTok / 2) * (NP + 4) * 4 <= SMEM_BYTES - 1024,
@@ -143,6 +146,20 @@ struct TopK {
       e[r] = 0x7fffffff;
     }
   }
+  // add a candidate without branches: it takes the first slot whose entry it beats, and each
+  // entry it displaces moves down by one slot (the last one drops out)
+  __device__ __forceinline__ void insert(float key, int ex) {
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r) {
+      const bool b = better(key, ex, v[r], e[r]);
+      const float tv = v[r];
+      const int te = e[r];
+      v[r] = b ? key : tv;
+      e[r] = b ? ex : te;
+      key = b ? tv : key;
+      ex = b ? te : ex;
+    }
+  }
   // drop the best entry (the list moves up by one; the last slot empties)
   __device__ __forceinline__ void pop() {
 #pragma unroll
@@ -197,9 +214,33 @@ __device__ __forceinline__ bool finish_tile(const TopK<KMAX>& best, const float*
   if (!__all_sync(0xffffffffu, synced)) return false;
   const int rows = min(kTok, T - t0);
   float* dst = logits + static_cast<int64_t>(t0) * N;
-  for (int i = ct; i < rows * N; i += kConvThreads) {
-    const int r = i / N;
-    dst[i] = stage[r * NS + (i - r * N)];
+  if (N <= kConvThreads) {
+    // thread ct copies column ct mod N of rows ct / N, ct / N + 128 / N, ...
+    const int rstep = kConvThreads / N, r0 = ct / N, c = ct - r0 * N;
+    if (r0 < rstep) {
+      int r = r0;
+      for (; r + 3 * rstep < rows; r += 4 * rstep) {
+        float q[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) q[u] = stage[(r + u * rstep) * NS + c];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[(r + u * rstep) * N + c] = q[u];
+      }
+      for (; r < rows; r += rstep) dst[r * N + c] = stage[r * NS + c];
+    }
+  } else {
+    // thread ct copies columns ct and ct + 128 of every row
+    for (int c = ct; c < N; c += kConvThreads) {
+      int r = 0;
+      for (; r + 7 < rows; r += 8) {
+        float q[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) q[u] = stage[(r + u) * NS + c];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) dst[(r + u) * N + c] = q[u];
+      }
+      for (; r < rows; ++r) dst[r * N + c] = stage[r * NS + c];
+    }
   }
   return true;
 }
@@ -511,19 +552,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c0 + i < N4) stage[ct * NS + c0 + i] = __uint_as_float(v[i]);
         }
       } else {
-        TopK<KMAX> best;
+        // the token's logits into its staging row, and the largest key (NaN ranks as -inf) of
+        // each column class e mod KMAX: the smallest of these KMAX maxima, thr, is at most the
+        // KMAX-th largest key (each class holds a key >= thr), so every top-k column has a
+        // key >= thr
+        float gmax[KMAX];
+#pragma unroll
+        for (int r = 0; r < KMAX; ++r) gmax[r] = -INFINITY;
+        float* row = stage + ct * NS;
+        // 32 columns per TMEM load (columns past NP are never used: c0 + 32 <= NP or N <= 16);
+        // the chunk's bias values are loaded while the TMEM load is in flight
         for (int c0 = 0; c0 < N; c0 += 32) {
           uint32_t v[32];
-          tmem_ld_32x32b_x32(trow + c0, v);  // columns past NP are never used: c0 + 32 <= NP or N <= 16
+          tmem_ld_32x32b_x32(trow + c0, v);
+          float bv[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            bv[i] = (bias != nullptr && c0 + i < N) ? __ldg(bias + c0 + i) : 0.f;
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int e = c0 + i;
             if (e >= N) continue;
-            float L = __uint_as_float(v[i]);
-            if (bias != nullptr) L += __ldg(bias + e);
-            stage[ct * NS + e] = L;
-            best.offer(L, e);
+            const float L = __uint_as_float(v[i]) + bv[i];
+            row[e] = L;
+            gmax[i % KMAX] = fmaxf(gmax[i % KMAX], isnan(L) ? -INFINITY : L);
+          }
+        }
+        float thr = gmax[0];
+#pragma unroll
+        for (int r = 1; r < KMAX; ++r) thr = fminf(thr, gmax[r]);
+        // the columns with key >= thr, in column order, as bytes after the staging rows
+        // ([kCand][kTok]); then the top-k of just those, all lanes of the warp stepping through
+        // the longest list together. A token with more than kCand such columns (many equal
+        // keys) takes every column instead.
+        uint8_t* cand = reinterpret_cast<uint8_t*>(stage + kTok * NS);
+        int nc = 0;
+        for (int e0 = 0; e0 < N; e0 += 8) {
+          float q[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) q[u] = e0 + u < N ? row[e0 + u] : 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const bool c = e0 + u < N && (isnan(q[u]) ? -INFINITY : q[u]) >= thr;
+            if (c && nc < kCand) cand[nc * kTok + ct] = static_cast<uint8_t>(e0 + u);
+            nc += c ? 1 : 0;
+          }
+        }
+        const bool listed = nc <= kCand;
+        const int rounds = __reduce_max_sync(0xffffffffu, listed ? nc : 0);
+        TopK<KMAX> best;
+        for (int j = 0; j < rounds; ++j) {
+          float key = -INFINITY;
+          int ex = 0x7fffffff;
+          if (listed && j < nc) {
+            ex = cand[j * kTok + ct];
+            const float L = row[ex];
+            key = isnan(L) ? -INFINITY : L;
+          }
+          best.insert(key, ex);
+        }
+        if (__any_sync(0xffffffffu, !listed)) {
+          for (int e = 0; e < N; ++e) {
+            const float L = row[e];
+            if (!listed) best.insert(isnan(L) ? -INFINITY : L, e);
           }
         }
         ok = finish_tile<KMAX>(best, stage, t0, ct, T, N, NS, k, logits, topk_idx, topk_w,
