@@ -10,7 +10,8 @@ from .moe_oracle import (capacity_from_factor, router_logits, softmax_over_exper
                          expert_permutation, silu, gelu, expert_ffn, combine,
                          moe_layer_forward, router_statistics)
 from .mx_oracle import (MX_BLOCK, decode_e8m0, decode_e4m3, decode_e2m1,  # noqa: F401
-                        unpack_fp4, dequantize_mx)
+                        unpack_fp4, dequantize_mx, encode_e4m3, quantize_mxfp8,
+                        dequantize_mxfp8, mxfp8_round_trip, expert_ffn_mxfp8_act)
 from .moe_backward import (logistic, silu_derivative, gelu_derivative,  # noqa: F401
                            combine_backward, renormalise_backward, expert_backward, aux_loss_backward,
                            moe_layer_backward)

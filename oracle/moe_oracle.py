@@ -261,13 +261,17 @@ def _expert(weights: ExpertWeights, e: int) -> np.ndarray:
 #  residual pass-through from «Expert capacity и capacity factor»)
 # --------------------------------------------------------------------------
 def combine(x: np.ndarray, routing: dict, w_gate_up: ExpertWeights, w_down: ExpertWeights,
-            act: str, residual: Optional[np.ndarray], tokens: Optional[np.ndarray] = None) -> np.ndarray:
+            act: str, residual: Optional[np.ndarray], tokens: Optional[np.ndarray] = None,
+            ffn: Callable = None) -> np.ndarray:
     """out[t] = residual[t] + sum over kept choices j of w[t, j] * E_{idx[t, j]}(x[t]).
 
     The loop runs over choices j, then experts e, as in the pages' eager loop;
     dropped pairs are skipped. ``tokens`` restricts the output to a subset of
-    token indices (a token's output depends only on its own kept pairs).
+    token indices (a token's output depends only on its own kept pairs). ``ffn`` is the
+    expert (expert_ffn unless given; the MXFP8-activation variant passes its own).
     """
+    if ffn is None:
+        ffn = expert_ffn
     topk_idx, topk_w, slot = routing["topk_idx"], routing["topk_w"], routing["slot"]
     T, k = topk_idx.shape
     if tokens is None:
@@ -282,7 +286,7 @@ def combine(x: np.ndarray, routing: dict, w_gate_up: ExpertWeights, w_down: Expe
             mask = (idx_sub[:, j] == e) & (slot_sub[:, j] >= 0)
             if not mask.any():
                 continue
-            y = expert_ffn(x[tokens[mask]], _expert(w_gate_up, e), _expert(w_down, e), act)
+            y = ffn(x[tokens[mask]], _expert(w_gate_up, e), _expert(w_down, e), act)
             out[mask] += w_sub[mask, j][:, None] * y
     return out
 

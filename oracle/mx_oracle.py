@@ -87,3 +87,79 @@ def dequantize_mx(elements: np.ndarray, scales: np.ndarray, fmt: str) -> np.ndar
         raise ValueError("scales must be [K/32, rows]")
     x = decode_e8m0(scales).T  # [rows, K/32]
     return vals * np.repeat(x, MX_BLOCK, axis=1)
+
+
+# --------------------------------------------------------------------------
+# MXFP8 activations (the block-scaled tensor-core variant)
+# --------------------------------------------------------------------------
+# Reading (the pages fix no activation format): with the block-scaled formats the token rows
+# and h are quantised to MXFP8 along the reduction axis, following the OCP MX v1.0
+# conversion: per block of 32 the shared scale is X = 2^(floor(log2(amax)) - 8), 8 being the
+# exponent of E4M3's largest power of two (256), clamped to E8M0's range [-127, 127] (an
+# all-zero block takes 2^-127); each element is v / X rounded to the nearest E4M3 value,
+# ties to the even code, magnitudes above 448 saturating to 448.
+
+E4M3_EMAX = 8
+_E4M3_POS = decode_e4m3(np.arange(0x7F))  # codes 0x00..0x7E: 0 .. 448, increasing
+
+
+def encode_e4m3(v: np.ndarray) -> np.ndarray:
+    """Finite values -> E4M3 codes: nearest value (ties to the even code), |v| > 448 -> 448.
+
+    The sign bit is the value's (so -0.0 and negatives that round to zero give 0x80)."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.minimum(np.abs(v), 448.0)
+    hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 0, 126)
+    lo = np.clip(hi - 1, 0, 126)
+    d_lo = a - _E4M3_POS[lo]
+    d_hi = _E4M3_POS[hi] - a
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(take_hi, hi, lo).astype(np.int64)
+    return np.where(np.signbit(v), code | 0x80, code).astype(np.uint8)
+
+
+def quantize_mxfp8(x: np.ndarray):
+    """[..., K] values (K a multiple of 32) -> (codes [..., K] uint8 E4M3,
+    scales [..., K/32] uint8 E8M0), per block of 32 along the last axis."""
+    x = np.asarray(x, dtype=np.float64)
+    K = x.shape[-1]
+    if K % MX_BLOCK:
+        raise ValueError("K must be a multiple of 32")
+    blocks = x.reshape(x.shape[:-1] + (K // MX_BLOCK, MX_BLOCK))
+    amax = np.abs(blocks).max(axis=-1)
+    _, ex = np.frexp(amax)  # amax = m * 2^ex with m in [0.5, 1): floor(log2(amax)) = ex - 1
+    e = np.where(amax > 0, ex - 1 - E4M3_EMAX, -127)
+    e = np.clip(e, -127, 127).astype(np.int64)
+    codes = encode_e4m3(blocks * np.ldexp(1.0, -e)[..., None])
+    return codes.reshape(x.shape), (e + 127).astype(np.uint8)
+
+
+def dequantize_mxfp8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Inverse of quantize_mxfp8's storage: codes [..., K], scales [..., K/32] -> float64."""
+    vals = decode_e4m3(codes)
+    x = decode_e8m0(scales)
+    return vals * np.repeat(x, MX_BLOCK, axis=-1)
+
+
+def mxfp8_round_trip(x: np.ndarray) -> np.ndarray:
+    """x as the block-scaled tensor cores see it: quantised to MXFP8 and read back."""
+    return dequantize_mxfp8(*quantize_mxfp8(x))
+
+
+def expert_ffn_mxfp8_act(rows: np.ndarray, w_gate_up: np.ndarray, w_down: np.ndarray,
+                         act: str) -> np.ndarray:
+    """One expert with MXFP8 activations: the rows quantised along d, h (computed from the
+    quantised rows, then the activation) quantised along F, both products exact in float64.
+
+    SwiGLU: w_gate_up [2F, d] (gate rows, then up rows); GELU: w_gate_up [F, d]; w_down [d, F].
+    """
+    from .moe_oracle import gelu, silu
+    xq = mxfp8_round_trip(rows)
+    if act == "swiglu":
+        F = w_gate_up.shape[0] // 2
+        h = silu(xq @ w_gate_up[:F].T) * (xq @ w_gate_up[F:].T)
+    elif act == "gelu":
+        h = gelu(xq @ w_gate_up.T)
+    else:
+        raise ValueError(f"unknown activation {act!r}")
+    return mxfp8_round_trip(h) @ w_down.T

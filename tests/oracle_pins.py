@@ -402,8 +402,67 @@ def pin_dequantize_blocks(m):
     assert w4[1].tolist() == [4.0, 24.0] * 16 + [0.5, 3.0] * 16
 
 
+# MXFP8 activations (block-scaled variant): OCP MX v1.0 conversion, X = 2^(floor(log2 amax) - 8)
+def pin_mxfp8_quantize_closed_forms(m):
+    def q(block):
+        b = np.zeros(32)
+        b[:len(block)] = block
+        codes, scales = m.quantize_mxfp8(b[None, :])
+        return codes[0, :len(block)].tolist(), int(scales[0, 0])
+    assert q([1.0] * 32) == ([0x78] * 32, 119)          # amax 1: X = 2^-8, 256 = 1.0 * 2^8
+    assert q([448.0, 1.0]) == ([0x7E, 0x38], 127)        # amax 448: X = 1
+    assert q([480.0, -511.0]) == ([0x7E, 0xFE], 127)     # (448, 512) saturates to 448
+    assert q([256.0, 1.0625, 1.1875, -1.0625]) == ([0x78, 0x38, 0x3A, 0xB8], 127)  # ties to even
+    assert q([256.0, 3 / 512, 2.0 ** -10]) == ([0x78, 0x03, 0x00], 127)  # subnormal; half of 2^-9
+    assert q([0.0, 0.0]) == ([0, 0], 0)                  # all-zero block: X = 2^-127
+    assert q([2.0 ** -130]) == ([0x20], 0)               # X clamped to 2^-127: 2^-3 remains
+    assert q([2.0 ** 140]) == ([0x7E], 254)              # X clamped to 2^127: 2^13 saturates
+    assert q([20.0, 0.0])[1] == 123                      # floor(log2 20) = 4: X = 2^-4
+
+
+def pin_mxfp8_encode_against_torch(m):
+    import torch
+    rng = np.random.default_rng(7)
+    mags = np.ldexp(rng.uniform(1.0, 2.0, 4000), rng.integers(-12, 9, 4000))
+    v = (np.where(rng.random(4000) < 0.5, -1.0, 1.0) * mags).astype(np.float32)
+    v = v[np.abs(v) <= 448.0]
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(m.encode_e4m3(v.astype(np.float64)), ref)
+
+
+def pin_mxfp8_round_trip(m):
+    # blocks whose largest element lies in E4M3's top binade [256, 448] come back unchanged
+    rng = np.random.default_rng(11)
+    codes = rng.integers(0, 0x7F, size=(6, 64)) | (rng.integers(0, 2, size=(6, 64)) << 7)
+    codes[:, 0] = 0x7A
+    codes[:, 32] = 0xFC
+    scales = rng.integers(100, 150, size=(6, 2)).astype(np.uint8)
+    c2, s2 = m.quantize_mxfp8(m.dequantize_mxfp8(codes.astype(np.uint8), scales))
+    assert np.array_equal(c2, codes) and np.array_equal(s2, scales)
+
+
+def pin_mxfp8_act_ffn_hand_case(m):
+    # x = 1.0625 (a tie between 1.0 and 1.125 at X = 2^-8: 1.0 stays); SwiGLU gate 20 x, up x;
+    # h = silu(20) = 19.99999996 (X = 2^-4: 319.9999993 -> 320, so 20); y = [1, 0.5] h
+    d = F = 32
+    x = np.zeros((1, d))
+    x[0, 0] = 1.0625
+    wgu = np.zeros((2 * F, d))
+    wgu[0, 0], wgu[F, 0] = 20.0, 1.0
+    wd = np.zeros((d, F))
+    wd[0, 0], wd[1, 0] = 1.0, 0.5
+    y = m.expert_ffn_mxfp8_act(x, wgu, wd, "swiglu")
+    assert y[0, :2].tolist() == [20.0, 10.0] and not y[0, 2:].any()
+    # GELU: z = 4 x = 4.0, gelu(4) = 3.99987... (X = 2^-7: 511.98 saturates to 448 -> 3.5)
+    wg = np.zeros((F, d))
+    wg[0, 0] = 4.0
+    y = m.expert_ffn_mxfp8_act(x, wg, wd, "gelu")
+    assert y[0, :2].tolist() == [3.5, 1.75]
+
+
 MX_PINS = [pin_e8m0_closed_forms, pin_e4m3_closed_forms, pin_e4m3_against_torch, pin_e2m1_table,
-           pin_fp4_nibble_order, pin_dequantize_blocks]
+           pin_fp4_nibble_order, pin_dequantize_blocks, pin_mxfp8_quantize_closed_forms,
+           pin_mxfp8_encode_against_torch, pin_mxfp8_round_trip, pin_mxfp8_act_ffn_hand_case]
 
 
 # ---------------------------------------------------------------- reroute overflow policy

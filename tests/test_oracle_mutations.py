@@ -189,7 +189,59 @@ def _dequant_scales_not_transposed(elements, scales, fmt):
     return vals * np.repeat(x, mxo.MX_BLOCK, axis=1)
 
 
+def _quantize_scale_ceil(x):
+    x = np.asarray(x, dtype=np.float64)
+    blocks = x.reshape(x.shape[:-1] + (x.shape[-1] // 32, 32))
+    amax = np.abs(blocks).max(axis=-1)
+    e = np.where(amax > 0, np.ceil(np.log2(np.where(amax > 0, amax, 1.0))) - 8, -127)
+    e = np.clip(e, -127, 127).astype(np.int64)
+    codes = mxo.encode_e4m3(blocks * np.ldexp(1.0, -e)[..., None])
+    return codes.reshape(x.shape), (e + 127).astype(np.uint8)
+
+
+def _quantize_emax_7(x):
+    x = np.asarray(x, dtype=np.float64)
+    blocks = x.reshape(x.shape[:-1] + (x.shape[-1] // 32, 32))
+    amax = np.abs(blocks).max(axis=-1)
+    _, ex = np.frexp(amax)
+    e = np.clip(np.where(amax > 0, ex - 1 - 7, -127), -127, 127).astype(np.int64)
+    codes = mxo.encode_e4m3(blocks * np.ldexp(1.0, -e)[..., None])
+    return codes.reshape(x.shape), (e + 127).astype(np.uint8)
+
+
+def _encode_truncating(v):
+    v = np.asarray(v, dtype=np.float64)
+    a = np.minimum(np.abs(v), 448.0)
+    code = np.clip(np.searchsorted(mxo._E4M3_POS, a, side="right") - 1, 0, 126).astype(np.int64)
+    return np.where(np.signbit(v), code | 0x80, code).astype(np.uint8)
+
+
+def _encode_no_saturation(v):
+    v = np.asarray(v, dtype=np.float64)
+    out = mxo.__dict__["_encode_ref"](v).astype(np.int64)
+    return np.where(np.abs(v) > 448.0, out | 0x7F, out).astype(np.uint8)  # NaN code
+
+
+def _ffn_h_not_quantised(rows, wgu, wd, act):
+    xq = mxo.mxfp8_round_trip(rows)
+    F = wgu.shape[0] // 2
+    h = om.silu(xq @ wgu[:F].T) * (xq @ wgu[F:].T) if act == "swiglu" else om.gelu(xq @ wgu.T)
+    return h @ wd.T
+
+
+def _ffn_x_not_quantised(rows, wgu, wd, act):
+    F = wgu.shape[0] // 2
+    h = om.silu(rows @ wgu[:F].T) * (rows @ wgu[F:].T) if act == "swiglu" else om.gelu(rows @ wgu.T)
+    return mxo.mxfp8_round_trip(h) @ wd.T
+
+
 MX_MUTANTS = {
+    "mxfp8_scale_from_ceil": ("quantize_mxfp8", _quantize_scale_ceil),
+    "mxfp8_emax_7": ("quantize_mxfp8", _quantize_emax_7),
+    "e4m3_encode_truncates": ("encode_e4m3", _encode_truncating),
+    "e4m3_encode_no_saturation": ("encode_e4m3", _encode_no_saturation),
+    "act_ffn_h_not_quantised": ("expert_ffn_mxfp8_act", _ffn_h_not_quantised),
+    "act_ffn_x_not_quantised": ("expert_ffn_mxfp8_act", _ffn_x_not_quantised),
     "fp4_high_nibble_first": ("unpack_fp4", _unpack_high_first),
     "e4m3_bias_8": ("decode_e4m3", _e4m3_bias8),
     "e2m1_no_subnormal": ("decode_e2m1", _e2m1_no_subnormal),
@@ -201,6 +253,7 @@ MX_MUTANTS = {
 @pytest.mark.parametrize("name", sorted(MX_MUTANTS))
 def test_some_mx_pin_catches(name, monkeypatch):
     attr, fn = MX_MUTANTS[name]
+    monkeypatch.setitem(mxo.__dict__, "_encode_ref", mxo.encode_e4m3)
     monkeypatch.setattr(mxo, attr, fn)
     caught = []
     for pin in oracle_pins.MX_PINS:
