@@ -83,7 +83,7 @@ def weight_bytes(params: int, wfmt: str = "bf16") -> int:
     byte per 32 elements plus 1 B (MXFP8) or 1/2 B (MXFP4) per element."""
     if wfmt == "bf16":
         return params * 2
-    return (params if wfmt == "mxfp8" else params // 2) + params // 32
+    return (params if wfmt.startswith("mxfp8") else params // 2) + params // 32
 
 
 def algorithmic_bytes(shape, T: int, active_experts: int, R: int, wfmt: str = "bf16") -> dict:
@@ -322,7 +322,9 @@ class Layer:
         self.mx = None if wfmt == "bf16" else moe.mx_weights(
             self.dims, wfmt, i["w_gate_up_q"], i["w_gate_up_s"], i["w_down_q"], i["w_down_s"])
         self.R_max = moe.max_rows(self.dims)
-        self.fws = moe.new_workspace(self.dims, device, forward=True)
+        # block-scaled formats ("_bs"): the quantised activations follow the forward workspace
+        self.block_scaled = wfmt.endswith("_bs")
+        self.fws = moe.new_workspace(self.dims, device, forward=True, block_scaled=self.block_scaled)
         self.b = moe.forward_layout(self.dims, self.fws)
         self.out = torch.empty((T, shape.d_model), dtype=torch.bfloat16, device=device)
 
@@ -524,11 +526,15 @@ class Layer:
                                        P(b.x_perm), P(b.stage_ws), b.stage_ws_bytes,
                                        moe._stream(None)), "permute")
 
+        # the per-stage workspace is the forward layout's last region; the block-scaled formats
+        # find their activation region right after it
+        stage_ws_avail = self.fws.numel() - (b.stage_ws - self.fws.data_ptr())
+
         def ffn():
             if self.mx is not None:
                 moe._check(lib.moe_grouped_ffn_mx(d, P(b.x_perm), P(b.expert_offset),
                                                   moe.ctypes.byref(self.mx), P(b.h), P(b.y_perm),
-                                                  P(b.stage_ws), b.stage_ws_bytes,
+                                                  P(b.stage_ws), stage_ws_avail,
                                                   moe._stream(None)), "grouped_ffn_mx")
                 return
             moe._check(lib.moe_grouped_ffn(d, P(b.x_perm), P(b.expert_offset), ptr(i["w_gate_up"]),
@@ -957,8 +963,9 @@ def main(argv=None):
                     help="shape[:T], shapes: " + ", ".join(synthetic.SHAPES))
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--wfmt", choices=["bf16", "mxfp8", "mxfp4"], default="bf16",
-                    help="expert weight storage (MX formats: OCP microscaling, E8M0 block scales)")
+    ap.add_argument("--wfmt", choices=["bf16", "mxfp8", "mxfp4", "mxfp8_bs", "mxfp4_bs"], default="bf16",
+                    help="expert weight storage (MX formats: OCP microscaling, E8M0 block scales; "
+                         "_bs: on the block-scaled MMA with MXFP8-quantised activations)")
     ap.add_argument("--sweep", default="all",
                     help="'all' (every workload point), 'none', or a comma list of shape:T")
     ap.add_argument("--no-extras", action="store_true",

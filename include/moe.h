@@ -79,7 +79,19 @@ typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_GELU = 1 } moe_act;
  *   MOE_WFMT_MXFP8  elements FP8 E4M3 (bias 7, subnormals, max 448, S.1111.111 NaN), 1 byte
  *   MOE_WFMT_MXFP4  elements FP4 E2M1 (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), 2 per byte,
  *                   element 2i in the low nibble of byte i */
-typedef enum { MOE_WFMT_BF16 = 0, MOE_WFMT_MXFP8 = 1, MOE_WFMT_MXFP4 = 2 } moe_wfmt;
+/*   MOE_WFMT_MXFP8_BS, MOE_WFMT_MXFP4_BS  the same MXFP8 / MXFP4 weights read by the
+ *                   block-scaled tensor-core MMA (tcgen05 kind::mxf8f6f4): the token rows and h
+ *                   are quantised to MXFP8 (E4M3 elements, per 32 along K one E8M0 scale
+ *                   X = 2^(floor(log2 amax) - 8), nearest-even rounding, saturation at 448, as
+ *                   the OCP MX v1.0 conversion reads). MXFP4_BS needs d_model and d_ff to be
+ *                   multiples of 128. See moe_mx_act_workspace_bytes. */
+typedef enum {
+  MOE_WFMT_BF16 = 0,
+  MOE_WFMT_MXFP8 = 1,
+  MOE_WFMT_MXFP4 = 2,
+  MOE_WFMT_MXFP8_BS = 3,
+  MOE_WFMT_MXFP4_BS = 4
+} moe_wfmt;
 
 /* Shape of one layer invocation. */
 typedef struct {
@@ -339,6 +351,15 @@ typedef struct {
 moe_status moe_grouped_ffn_mx(const moe_dims* dims, const uint16_t* x_perm,
                               const int32_t* expert_offset, const moe_mx_weights* w, uint16_t* h,
                               float* y_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* Extra workspace of the block-scaled formats (MOE_WFMT_MXFP8_BS, MOE_WFMT_MXFP4_BS): the
+ * quantised token rows ([R_max, d_model] E4M3 codes) and the E8M0 scales of the rows and of h
+ * in the tensor-memory copy layout. moe_grouped_ffn_mx then needs ws_bytes >=
+ * round_up(moe_workspace_bytes, 256) + this, moe_forward_mx a forward workspace of
+ * round_up(moe_forward_workspace_bytes, 256) + this; the extra bytes follow the usual regions.
+ * With these formats h (the buffer passed in, or the forward layout's) receives h's E4M3 codes,
+ * [R_max, d_ff] bytes. Host-only. */
+moe_status moe_mx_act_workspace_bytes(const moe_dims* dims, size_t* bytes);
 
 /* moe_forward with MX expert weights (same workspace, layout and routing). */
 moe_status moe_forward_mx(const moe_dims* dims, const uint16_t* x, const float* w_router,

@@ -52,8 +52,10 @@ class ForwardBuffers(ctypes.Structure):
         "pair_of_row", "x_perm", "h", "y_perm", "stage_ws")] + [("stage_ws_bytes", ctypes.c_size_t)]
 
 
-WFMT_BF16, WFMT_MXFP8, WFMT_MXFP4 = 0, 1, 2
-_WFMT = {"mxfp8": WFMT_MXFP8, "mxfp4": WFMT_MXFP4}
+WFMT_BF16, WFMT_MXFP8, WFMT_MXFP4, WFMT_MXFP8_BS, WFMT_MXFP4_BS = 0, 1, 2, 3, 4
+# "_bs": the same weights on the block-scaled MMA, with MXFP8-quantised token rows and h
+_WFMT = {"mxfp8": WFMT_MXFP8, "mxfp4": WFMT_MXFP4, "mxfp8_bs": WFMT_MXFP8_BS,
+         "mxfp4_bs": WFMT_MXFP4_BS}
 
 
 class MxWeights(ctypes.Structure):
@@ -81,6 +83,7 @@ _SIGS = {
     "moe_unpermute_combine": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, ctypes.c_int32, _P,
                                              ctypes.c_size_t, _P]),
     "moe_forward_workspace_bytes": (ctypes.c_int, [_DIMS, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_mx_act_workspace_bytes": (ctypes.c_int, [_DIMS, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_forward_layout": (ctypes.c_int, [_DIMS, _P, ctypes.c_size_t, ctypes.POINTER(ForwardBuffers)]),
     "moe_forward": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_route_noalloc": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -176,9 +179,20 @@ def forward_workspace_bytes(dims: Dims) -> int:
     return int(n.value)
 
 
-def new_workspace(dims: Dims, device=None, forward: bool = False) -> torch.Tensor:
-    """A zeroed uint8 workspace tensor for the per-stage calls (or for moe_forward)."""
+def mx_act_workspace_bytes(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.moe_mx_act_workspace_bytes(ctypes.byref(dims), ctypes.byref(n)),
+           "moe_mx_act_workspace_bytes")
+    return int(n.value)
+
+
+def new_workspace(dims: Dims, device=None, forward: bool = False,
+                  block_scaled: bool = False) -> torch.Tensor:
+    """A zeroed uint8 workspace tensor for the per-stage calls (or for moe_forward); with
+    block_scaled, room for the block-scaled MX formats' quantised activations after it."""
     n = forward_workspace_bytes(dims) if forward else workspace_bytes(dims)
+    if block_scaled:
+        n = (n + 255) // 256 * 256 + mx_act_workspace_bytes(dims)
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
@@ -300,7 +314,7 @@ def mx_weights(dims: Dims, fmt: str, gate_up, gate_up_scales, down, down_scales)
     down [N, d_model, d_ff or d_ff/2] uint8, down_scales [N, d_ff/32, d_model] uint8."""
     d, N, F = dims.d_model, dims.n_experts, dims.d_ff
     rows = 2 * F if dims.act == ACT_SWIGLU else F
-    per = 1 if fmt == "mxfp8" else 2
+    per = 1 if fmt.startswith("mxfp8") else 2
     return MxWeights(_WFMT[fmt],
                      _ptr(gate_up, "gate_up", torch.uint8, (N, rows, d // per)),
                      _ptr(gate_up_scales, "gate_up_scales", torch.uint8, (N, d // 32, rows)),

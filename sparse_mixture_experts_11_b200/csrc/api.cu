@@ -365,8 +365,11 @@ struct Weights {
   const uint8_t* down_scales;
 };
 
+bool block_scaled(int fmt) { return fmt == MOE_WFMT_MXFP8_BS || fmt == MOE_WFMT_MXFP4_BS; }
+
 moe_status check_weights(const Weights& w) {
-  if (w.fmt != MOE_WFMT_BF16 && w.fmt != MOE_WFMT_MXFP8 && w.fmt != MOE_WFMT_MXFP4)
+  if (w.fmt != MOE_WFMT_BF16 && w.fmt != MOE_WFMT_MXFP8 && w.fmt != MOE_WFMT_MXFP4 &&
+      !block_scaled(w.fmt))
     return MOE_ERR_INVALID;
   if (!w.gate_up || !w.down) return MOE_ERR_INVALID;
   if (w.fmt != MOE_WFMT_BF16 && (!w.gate_up_scales || !w.down_scales)) return MOE_ERR_INVALID;
@@ -381,14 +384,21 @@ Weights weights_of(const moe_mx_weights* w) {
   return Weights{w->fmt, w->gate_up, w->gate_up_scales, w->down, w->down_scales};
 }
 
+// act_ws: the block-scaled formats' activation region (moe_mx_act_workspace_bytes), or null.
 moe_status grouped_ffn_impl(const moe_dims* dims, const uint16_t* x_perm,
                             const int32_t* expert_offset, const Weights& w, uint16_t* h,
-                            float* y_perm, void* ws, size_t ws_bytes, void* stream) {
+                            float* y_perm, void* ws, size_t ws_bytes, void* stream,
+                            void* act_ws = nullptr) {
   moe_status st = check_dims(dims);
   if (st != MOE_OK) return st;
   const int64_t rmax = max_rows(dims);
   if (dims->T == 0 || rmax == 0) return MOE_OK;
   if ((st = check_weights(w)) != MOE_OK) return st;
+  if (block_scaled(w.fmt)) {
+    if (act_ws == nullptr || !aligned16(act_ws)) return MOE_ERR_WORKSPACE;
+    if (w.fmt == MOE_WFMT_MXFP4_BS && (dims->d_model % 128 != 0 || dims->d_ff % 128 != 0))
+      return MOE_ERR_UNSUPPORTED;
+  }
   if (!x_perm || !expert_offset || !h || !y_perm || !ws) return MOE_ERR_INVALID;
   if (!aligned16(x_perm) || !aligned16(expert_offset) || !aligned16(h) || !aligned16(y_perm) ||
       !aligned16(ws))
@@ -416,6 +426,7 @@ moe_status grouped_ffn_impl(const moe_dims* dims, const uint16_t* x_perm,
   const moe::FfnScratchPlan plan = ffn_plan(dims);
   a.counters = reinterpret_cast<int*>(static_cast<char*>(ws) + moe::kStatusBytes);
   if (plan.part_bytes > 0) a.part = reinterpret_cast<float*>(shared_region_of(dims, ws));
+  a.act_ws = act_ws;
   return launch_status(moe::launch_grouped_ffn(a, as_stream(stream)));
 }
 }  // namespace
@@ -429,12 +440,28 @@ moe_status moe_grouped_ffn(const moe_dims* dims, const uint16_t* x_perm,
                           ws, ws_bytes, stream);
 }
 
+moe_status moe_mx_act_workspace_bytes(const moe_dims* dims, size_t* bytes) {
+  const moe_status st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if (bytes == nullptr) return MOE_ERR_INVALID;
+  *bytes = moe::mx_act_layout(dims->n_experts, dims->d_model, dims->d_ff, max_rows(dims)).total;
+  return MOE_OK;
+}
+
 moe_status moe_grouped_ffn_mx(const moe_dims* dims, const uint16_t* x_perm,
                               const int32_t* expert_offset, const moe_mx_weights* w, uint16_t* h,
                               float* y_perm, void* ws, size_t ws_bytes, void* stream) {
   if (w == nullptr || w->fmt == MOE_WFMT_BF16) return MOE_ERR_INVALID;
+  void* act_ws = nullptr;
+  if (block_scaled(w->fmt) && check_dims(dims) == MOE_OK && ws != nullptr) {
+    const size_t base = round_up(stage_ws_bytes(dims), 256);
+    size_t extra = 0;
+    moe_mx_act_workspace_bytes(dims, &extra);
+    if (ws_bytes < base + extra) return MOE_ERR_WORKSPACE;
+    act_ws = static_cast<char*>(ws) + base;
+  }
   return grouped_ffn_impl(dims, x_perm, expert_offset, weights_of(w), h, y_perm, ws, ws_bytes,
-                          stream);
+                          stream, act_ws);
 }
 
 moe_status moe_unpermute_combine(const moe_dims* dims, const float* y_perm,
@@ -628,6 +655,15 @@ moe_status forward_impl(const moe_dims* dims, const uint16_t* x, const float* w_
   moe_forward_buffers b;
   moe_status st = moe_forward_layout(dims, ws, ws_bytes, &b);
   if (st != MOE_OK) return st;
+  void* act_ws = nullptr;
+  if (block_scaled(w.fmt)) {  // the activation region follows the forward layout
+    size_t base = 0, extra = 0;
+    moe_forward_workspace_bytes(dims, &base);
+    moe_mx_act_workspace_bytes(dims, &extra);
+    base = round_up(base, 256);
+    if (ws_bytes < base + extra) return MOE_ERR_WORKSPACE;
+    act_ws = static_cast<char*>(ws) + base;
+  }
   if (dims->T == 0) return MOE_OK;
   if (!x || !w_router || !out) return MOE_ERR_INVALID;
   if ((st = check_weights(w)) != MOE_OK) return st;
@@ -656,7 +692,7 @@ moe_status forward_impl(const moe_dims* dims, const uint16_t* x, const float* w_
   }
   if (st != MOE_OK) return st;
   st = grouped_ffn_impl(dims, b.x_perm, b.expert_offset, w, b.h, b.y_perm, b.stage_ws,
-                        b.stage_ws_bytes, stream);
+                        b.stage_ws_bytes, stream, act_ws);
   if (st != MOE_OK) return st;
   return moe_unpermute_combine(dims, b.y_perm, b.row_of_pair, b.topk_w, residual, out, 0,
                                b.stage_ws, b.stage_ws_bytes, stream);

@@ -212,6 +212,15 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
+// Plain bulk copy global -> shared (both 16-byte aligned, bytes a multiple of 16) completing
+// its bytes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // Shared -> global tiled stores (bulk-group completion). The source is read asynchronously:
 // wait with tma_store_wait_read before writing it again, and with tma_store_wait_all before
 // the CTA exits.
@@ -332,6 +341,28 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t cta_mask) 
       : "memory");
 }
 
+// Block-scaled MMA (kind::mxf8f6f4, 8-, 6- or 4-bit A and B from shared memory, E8M0 scale
+// factors of A's rows and B's rows in TMEM at sfa / sfb; each address's bits 31:30 pick the
+// byte of the scale word, i.e. the 32-element K block): D[tmem] (+)= (A * SA)(B * SB)^T.
+__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Shared memory -> TMEM copy of a 32-row x 16-byte matrix, repeated in the four 32-lane
+// quarters (the scale-factor layout of the block-scaled MMA). One thread issues it; it is
+// ordered with the same thread's tcgen05.mma.
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+               : "memory");
+}
+
 // 32 lanes x 32-bit, 16 consecutive columns per thread (thread i <- TMEM lane base+i).
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -372,6 +403,26 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t smem_addr) {
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
+}
+
+// Descriptor of a shared-memory matrix without swizzle, K-major: core matrices of 8 rows x
+// 16 bytes stored contiguously (128 bytes), stride byte offset 128 between 8-row groups.
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with E8M0 scales (bit 23): A and B formats at bits
+// 7-9 and 10-12 (0 E4M3, 5 E2M1), B's and A's scale byte at bits 4-5 and 29-30, N >> 3 at
+// 17-22, M >> 4 at 24-28, both K-major.
+__host__ __device__ constexpr uint32_t idesc_mx(int M, int N, int a_fmt, int b_fmt, int sf_id) {
+  return (static_cast<uint32_t>(sf_id) << 4) | (static_cast<uint32_t>(a_fmt) << 7) |
+         (static_cast<uint32_t>(b_fmt) << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(sf_id) << 29);
 }
 
 // Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), A and B bf16

@@ -88,6 +88,10 @@ struct PhaseParams {
 
 struct FfnParams {
   const int32_t* expert_offset;  // [N+1]
+  // block-scaled formats: E8M0 scales of the quantised token rows (x) and of h, one 512-byte
+  // atom per (m-tile, k block) in the TMEM copy layout (row r, block q at 16 (r % 32) + 4 (r / 32) + q)
+  const uint8_t* x_atoms;
+  uint8_t* h_atoms;
   int64_t r_max;
   int64_t rows_per_expert;       // no expert may hold more rows (partial slots are this tall)
   int n_experts;
@@ -102,14 +106,20 @@ struct FfnParams {
 };
 
 // Weight storage: bf16, or an MX format (blocks of 32 elements along K sharing one E8M0
-// scale) with E4M3 or E2M1 elements, decoded exactly to bf16 in shared memory.
-enum { WFMT_BF16 = 0, WFMT_MXFP8 = 1, WFMT_MXFP4 = 2 };
+// scale) with E4M3 or E2M1 elements, decoded exactly to bf16 in shared memory; or, block-scaled
+// (BS8, BS4), the same MX weights read by the block-scaled MMA (kind::mxf8f6f4) against token
+// rows and h quantised to MXFP8.
+enum { WFMT_BF16 = 0, WFMT_MXFP8 = 1, WFMT_MXFP4 = 2, WFMT_BS8 = 3, WFMT_BS4 = 4 };
+constexpr int kBsK = 128;        // block-scaled: k per stage (128 one-byte elements = 128 bytes)
+constexpr int kBsSfStage = 2560; // per stage: A scale atom 512 B, raw B scales 1 KB, B atoms 1 KB
+constexpr int kBsBudget = 216 * 1024;
 constexpr int kConvThreads = 256;  // MX decoders (warps 7-14)
 constexpr int kConvWarps = kConvThreads / 32;
 
 template <int BM, int WFMT>
 struct Cfg {
-  static constexpr bool MX = WFMT != WFMT_BF16;
+  static constexpr bool MX = WFMT == WFMT_MXFP8 || WFMT == WFMT_MXFP4;  // decoded in smem
+  static constexpr bool BS = WFMT == WFMT_BS8 || WFMT == WFMT_BS4;      // block-scaled MMA
   static constexpr int THREADS = MX ? kThreads + 32 + kConvThreads : kThreads;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = kUmmaN * BK * 2;
@@ -120,7 +130,9 @@ struct Cfg {
   static constexpr int ROW_BYTES = WFMT == WFMT_MXFP8 ? BK : BK / 2;  // per row and k block
   static constexpr int KG = MX ? 128 / ROW_BYTES : 1;
   static constexpr int STG_BYTES = MX ? kUmmaN * 128 + 2 * KG * kUmmaN : 0;
-  static constexpr int STAGES_FIT = (kSmemBudget / STAGE_BYTES) > 8 ? 8 : (kSmemBudget / STAGE_BYTES);
+  static constexpr int SF_STAGE = BS ? kBsSfStage : 0;
+  static constexpr int STAGES_RAW = BS ? kBsBudget / (STAGE_BYTES + kBsSfStage) : kSmemBudget / STAGE_BYTES;
+  static constexpr int STAGES_FIT = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   // MX: two bf16 B stages (decoded from shared memory; a third measured no faster), a
   // separate ring of SA A stages
   // (token rows, loaded ahead of the decoders: an A copy waits on L2 for about 1.7 us when
@@ -133,7 +145,12 @@ struct Cfg {
   static constexpr int SST_FIT = MX ? (kMxBudget - B_RING - A_RING) / STG_BYTES : 0;
   static constexpr int SST = SST_FIT > 16 ? 16 : SST_FIT;
   static constexpr int TMEM_COLS = 2 * kUmmaN;
-  static constexpr int SMEM_BYTES = B_RING + A_RING + SST * STG_BYTES + 1024;  // + alignment slack
+  // accumulator buffers in TMEM: two (the epilogue of one tile overlaps the next tile's MMAs),
+  // or one for BS, whose scale factors take TMEM columns 256 (A) and 264-271 (B)
+  static constexpr int NACC = BS ? 1 : 2;
+  static constexpr int SF_RING = STAGES * SF_STAGE;
+  static constexpr int SMEM_BYTES = B_RING + A_RING + SST * STG_BYTES + SF_RING + 1024;  // + alignment slack
+  static_assert(!BS || BM == 128, "block-scaled MMA: M = 128");
   static_assert(TMEM_COLS <= 512, "two accumulators must fit in TMEM");
   static_assert(STAGES >= 2, "pipeline depth");
   static_assert(!MX || SST >= 2, "MX staging depth");
@@ -372,11 +389,60 @@ __device__ __forceinline__ void store_final16(const PhaseParams& p, int64_t row,
   }
 }
 
+// One MX block of 32 fp32 values -> E4M3 codes of v / X with X = 2^(floor(log2 amax) - 8),
+// X clamped to [2^-127, 2^127] (OCP MX v1.0 conversion: 8 is the exponent of E4M3's largest
+// power of two; the elements round to nearest even and saturate at 448). Returns X's E8M0
+// code; the codes of elements 0-15 go to lo, 16-31 to hi (element i in byte i).
+__device__ __forceinline__ uint32_t mxfp8_block(const float (&v)[32], uint4& lo, uint4& hi) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int ebits = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);  // 0: zero or subnormal
+  const int e = max(ebits - 127 - 8, -127);
+  const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e exactly
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t p0 = __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i] * inv, v[4 * i + 1] * inv),
+                                                 __NV_SATFINITE, __NV_E4M3);
+    const uint32_t p1 = __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i + 2] * inv, v[4 * i + 3] * inv),
+                                                 __NV_SATFINITE, __NV_E4M3);
+    w[i] = p0 | (p1 << 16);
+  }
+  lo = make_uint4(w[0], w[1], w[2], w[3]);
+  hi = make_uint4(w[4], w[5], w[6], w[7]);
+  return static_cast<uint32_t>(e + 127);
+}
+
+// Byte of the scale of row r (of a 128-row tile) and 32-column block q (of a 128-column k
+// block) in a 512-byte scale atom.
+__device__ __forceinline__ int sf_atom_byte(int r, int q) { return 16 * (r & 31) + 4 * (r >> 5) + q; }
+
+// h of 32 columns of one row as MXFP8: codes to h (bytes, row stride ld) and the scale into
+// the h atom of (m-tile gm, k block col / 128) for the down projection's MMA.
+template <int EPI>
+__device__ __forceinline__ void store_h_mx32(const FfnParams& fp, const PhaseParams& p,
+                                             int64_t row, int col, int gm, int r_local,
+                                             const float (&a)[32], const float (&b)[32]) {
+  float hv[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) hv[i] = EPI == EPI_SWIGLU ? silu_f(a[i]) * b[i] : gelu_f(a[i]);
+  uint4 lo, hi;
+  const uint32_t sc = mxfp8_block(hv, lo, hi);
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + row * p.ld_out + col);
+  dst[0] = lo;
+  dst[1] = hi;
+  fp.h_atoms[(static_cast<int64_t>(gm) * fp.ph[1].num_kb + col / kBsK) * 512 +
+             sf_atom_byte(r_local, (col >> 5) & 3)] = static_cast<uint8_t>(sc);
+}
+
 // Epilogue of one segment (all 128 epilogue threads): read the accumulator from TMEM, store
 // the final tile or this segment's partial, hand the TMEM buffer back; for a partial, count the
 // arrival and, if last, add the partials in order and store the tile. Returns whether this CTA
 // wrote the tile's final values in *finished; false on a timed-out wait.
-template <int EPI, int BN, int BM>
+// NACC: TMEM accumulator buffers (segment tc uses buffer tc % NACC). QH: h is stored as MXFP8
+// (codes and scale atoms) instead of bf16.
+template <int EPI, int BN, int BM, int NACC, bool QH>
 __device__ __forceinline__ bool epilogue_segment(const FfnParams& fp, const PhaseParams& p,
                                                  const Sched& sched, const Seg& sg,
                                                  const TileCoord& c, uint32_t tmem_base, int tc,
@@ -387,8 +453,8 @@ __device__ __forceinline__ bool epilogue_segment(const FfnParams& fp, const Phas
   const int q = warp & 3;  // TMEM lane quadrant this warp may access
   // tile row held by this thread's TMEM lane (M = 64 uses lanes 0-15 of each quadrant)
   const int r_local = BM == 128 ? q * 32 + lane : (lane < 16 ? q * 16 + lane : BM);
-  const int buf = tc & 1;
-  const uint32_t tph = (tc >> 1) & 1;
+  const int buf = NACC == 2 ? tc & 1 : 0;
+  const uint32_t tph = NACC == 2 ? (tc >> 1) & 1 : tc & 1;
   const bool got = mbar_wait(tfull, tph, fp.timeout_ns, s_abort);
   if (!__all_sync(0xffffffffu, got)) return false;
   tc_fence_after_sync();
@@ -402,8 +468,29 @@ __device__ __forceinline__ bool epilogue_segment(const FfnParams& fp, const Phas
                          static_cast<uint32_t>(buf * kUmmaN);
   const bool row_ok = r_local < c.rows;
   const int64_t row = static_cast<int64_t>(c.m0) + r_local;
+  if (QH && whole) {
 #pragma unroll 1
-  for (int cc = 0; cc < BN; cc += 16) {
+    for (int cc = 0; cc < BN; cc += 32) {
+      if (c.n0 + cc >= p.n_out) break;  // warp-uniform: ragged last n-tile (F % 32 == 0)
+      float a[32], b[32];
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(t_row + cc, v);
+      if (EPI == EPI_SWIGLU) {
+        uint32_t u[32];
+        tmem_ld_32x32b_x32(t_row + BN + cc, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) b[i] = __uint_as_float(u[i]);
+      } else {
+        tmem_ld_wait();
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(v[i]);
+      if (row_ok) store_h_mx32<EPI>(fp, p, row, c.n0 + cc, c.gm, r_local, a, b);
+    }
+  }
+#pragma unroll 1
+  for (int cc = 0; cc < BN && !(QH && whole); cc += 16) {
     if (c.n0 + cc >= p.n_out) break;  // warp-uniform: ragged last n-tile
     float a[16], b[16];
     uint32_t v[16];
@@ -457,11 +544,44 @@ __device__ __forceinline__ bool epilogue_segment(const FfnParams& fp, const Phas
   }
   if (!__all_sync(0xffffffffu, epilogue_sync(ebar, epi_phase, fp.timeout_ns, s_abort))) return false;
   if (!*s_fixup) return false;
+  const int cols = min(BN, p.n_out - c.n0);
+  const int et = threadIdx.x - 64;  // 0..127
+  if (QH) {
+    // MXFP8 h: item i is (tile row i / G32, 32-column block i % G32), one MX block per item
+    constexpr int G32 = BN / 32;
+    for (int i = et; i < c.rows * G32; i += kEpiThreads) {
+      const int r = i / G32, c32 = (i - r * G32) * 32;
+      if (c32 >= cols) continue;
+      float ga[32], ub[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        ga[q] = 0.f;
+        ub[q] = 0.f;
+      }
+#pragma unroll 1
+      for (int j = 0; j < n_seg; ++j) {  // fixed order (CTA index): deterministic sums
+        const int b2 = first_cta + j;
+        const int slot2 = sk_begin(sched, b2) >= t_it0 ? 0 : 1;
+        const float* src =
+            p.part + (static_cast<int64_t>(b2 * 2 + slot2) * fp.slot_rows + r) * kUmmaN + c32;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(src) + q);
+          ga[4 * q] += v.x; ga[4 * q + 1] += v.y; ga[4 * q + 2] += v.z; ga[4 * q + 3] += v.w;
+          if (EPI == EPI_SWIGLU) {
+            const float4 u = __ldcg(reinterpret_cast<const float4*>(src + BN) + q);
+            ub[4 * q] += u.x; ub[4 * q + 1] += u.y; ub[4 * q + 2] += u.z; ub[4 * q + 3] += u.w;
+          }
+        }
+      }
+      store_h_mx32<EPI>(fp, p, static_cast<int64_t>(c.m0) + r, c.n0 + c32, c.gm, r, ga, ub);
+    }
+    *finished = true;
+    return true;
+  }
   // All 128 epilogue threads share the reduction: item i is (tile row i / G, float4 column
   // group i % G), so neighbouring threads touch neighbouring columns.
   constexpr int G = BN / 4;
-  const int cols = min(BN, p.n_out - c.n0);
-  const int et = threadIdx.x - 64;  // 0..127
   for (int i = et; i < c.rows * G; i += kEpiThreads) {
     const int r = i / G, c4 = (i - r * G) * 4;
     if (c4 >= cols) continue;
@@ -533,6 +653,14 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
     return C::MX ? tiles + i * C::B_BYTES : tiles + i * C::STAGE_BYTES + C::A_BYTES;
   };
   constexpr int AST = C::MX ? C::SA : C::STAGES;  // stages of the A operand's ring
+  // BS: per stage [A scale atom 512 B | raw B scales [2][4][128] | B scale atoms [2][512]]
+  const uint32_t sf0 = stg0 + C::SST * C::STG_BYTES;
+  auto sf_addr = [&](int i) -> uint32_t { return sf0 + i * C::SF_STAGE; };
+  // BS: the A scale atom of (m-tile gm, k block kb) of phase ph
+  auto a_atom = [&](int ph, int gm, int kb) -> const uint8_t* {
+    return (ph == 0 ? p.x_atoms : p.h_atoms) + (static_cast<int64_t>(gm) * p.ph[ph].num_kb + kb) * 512;
+  };
+  constexpr int KX = C::BS ? kBsK : BK;  // A / B column coordinate step per k block
   uint64_t* const a_full = C::MX ? afull_bar : full_bar;
   uint64_t* const a_empty = C::MX ? aempty_bar : empty_bar;
 
@@ -541,9 +669,11 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
     prefetch_tensormap(&tmB1);
     prefetch_tensormap(&tmA2);
     prefetch_tensormap(&tmB2);
-    if (C::MX) {
+    if (C::MX || C::BS) {
       prefetch_tensormap(&tmS1);
       prefetch_tensormap(&tmS2);
+    }
+    if (C::MX) {
       for (int s = 0; s < C::SST; ++s) {
         mbar_init(smem_u32(&sfull_bar[s]), 1);
         mbar_init(smem_u32(&sempty_bar[s]), kConvWarps);
@@ -662,8 +792,28 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
             const uint32_t fb = smem_u32(&a_full[s]);
             const uint32_t a_dst = a_addr(s);
             const uint32_t b_dst = b_addr(s);
-            mbar_arrive_expect_tx(fb, C::MX ? C::A_BYTES : C::STAGE_BYTES);
-            if (!C::MX) {  // MX: the decoders fill the B half
+            // (E2M1 through the padded 4-bit type counts its packed bytes, half the smem it fills)
+            mbar_arrive_expect_tx(fb, C::MX ? C::A_BYTES
+                                            : C::STAGE_BYTES + (C::BS ? 1536 : 0) -
+                                                  (WFMT == WFMT_BS4 ? C::B_BYTES / 2 : 0));
+            if (C::BS) {
+              // weights and their raw scales ([half][4 blocks][128 rows] bytes); the token
+              // rows' scale atom goes with the A tile
+              const uint32_t sfr = sf_addr(s) + 512;
+              const int kx = kb * kBsK;
+              if (ph == 0 && EPI1 == EPI_SWIGLU) {
+                tma_load_4d(b_dst, &tmB1, fb, kx, c.n0, 0, c.e, pol_b);
+                tma_load_4d(b_dst + BN1 * 128, &tmB1, fb, kx, c.n0, 1, c.e, pol_b);
+                tma_load_4d(sfr, &tmS1, fb, c.n0, 0, 4 * kb, c.e, pol_b);
+                tma_load_4d(sfr + 512, &tmS1, fb, c.n0, 1, 4 * kb, c.e, pol_b);
+              } else {
+                const CUtensorMap* tb = ph == 0 ? &tmB1 : &tmB2;
+                const CUtensorMap* ts = ph == 0 ? &tmS1 : &tmS2;
+                tma_load_3d(b_dst, tb, fb, kx, c.n0, c.e, pol_b);
+                tma_load_3d(sfr, ts, fb, c.n0, 4 * kb, c.e, pol_b);
+                tma_load_3d(sfr + 512, ts, fb, c.n0 + 128, 4 * kb, c.e, pol_b);
+              }
+            } else if (!C::MX) {  // MX: the decoders fill the B half
               if (ph == 0) {
                 if (EPI1 == EPI_SWIGLU) {
                   tma_load_4d(b_dst, &tmB1, fb, kb * BK, c.n0, 0, c.e, pol_b);
@@ -676,7 +826,8 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
               }
             }
             if (ready) {
-              tma_load_2d(a_dst, tA, fb, kb * BK, c.m0, pol_a);
+              tma_load_2d(a_dst, tA, fb, kb * KX, c.m0, pol_a);
+              if (C::BS) bulk_load(sf_addr(s), a_atom(ph, c.gm, kb), 512, fb);
               ++it;
               continue;
             }
@@ -688,8 +839,9 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
               fence_proxy_async_global();
               for (int j = pend_from; j <= it; ++j) {
                 const int sj = j % AST;
-                tma_load_2d(a_addr(sj), tA, smem_u32(&a_full[sj]),
-                            (sg.kb0 + (j - seg_it0)) * BK, c.m0, pol_a);
+                const int kbj = sg.kb0 + (j - seg_it0);
+                tma_load_2d(a_addr(sj), tA, smem_u32(&a_full[sj]), kbj * KX, c.m0, pol_a);
+                if (C::BS) bulk_load(sf_addr(sj), a_atom(ph, c.gm, kbj), 512, smem_u32(&a_full[sj]));
               }
               pend_from = -1;
               ready = true;
@@ -709,7 +861,79 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if constexpr (C::BS) {
+      // Block-scaled: the whole warp turns each stage's raw weight scales ([half][block][row])
+      // into the two 512-byte atoms of the TMEM copy layout; lane 0 copies the A and B atoms
+      // into TMEM (A at column 256, B at 264-271) and issues the four K = 32 MMAs. TMEM copies
+      // and MMAs of one thread run in issue order, so one scale area serves every stage.
+      constexpr int kBFmt = WFMT == WFMT_BS4 ? 5 : 0;  // E2M1 or E4M3 weights; A is E4M3
+      const uint32_t t_sfa = tmem_base + kUmmaN, t_sfb = tmem_base + kUmmaN + 8;
+      int it = 0, tc = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        const Sched sc = s_sched[ph];
+        SegCursor cur(sc);
+        Seg sg;
+        for (; ok && cur.next(sc, sg); ++tc) {
+          // one accumulator: the epilogue has read the previous segment's
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&tempty_bar[0]), (tc & 1) ^ 1u, p.timeout_ns, &s_abort));
+          if (!ok) break;
+          tc_fence_after_sync();
+          for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+            const int s = it % C::STAGES;
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[s]), (it / C::STAGES) & 1,
+                                                    p.timeout_ns, &s_abort));
+            if (!ok) break;
+            {
+              const uint8_t* raw = dyn_smem + (sf_addr(s) + 512 - smem_u32(dyn_smem));
+              uint8_t* atoms = dyn_smem + (sf_addr(s) + 1536 - smem_u32(dyn_smem));
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                uint32_t w[4];
+#pragma unroll
+                for (int r1 = 0; r1 < 4; ++r1) {
+                  const uint8_t* src = raw + j * 512 + r1 * 32 + lane;
+                  w[r1] = static_cast<uint32_t>(src[0]) | (static_cast<uint32_t>(src[128]) << 8) |
+                          (static_cast<uint32_t>(src[256]) << 16) | (static_cast<uint32_t>(src[384]) << 24);
+                }
+                *reinterpret_cast<uint4*>(atoms + j * 512 + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
+            fence_proxy_async_smem();  // generic stores -> visible to the tensor core's copy
+            __syncwarp();
+            if (lane == 0) {
+              tc_fence_after_sync();
+              const uint32_t a_base = a_addr(s), b_base = b_addr(s);
+              tc_cp_32x128b_x4(t_sfa, smem_desc_plain(sf_addr(s)));
+              tc_cp_32x128b_x4(t_sfb, smem_desc_plain(sf_addr(s) + 1536));
+              tc_cp_32x128b_x4(t_sfb + 4, smem_desc_plain(sf_addr(s) + 2048));
+#pragma unroll
+              for (int kk = 0; kk < kBsK / 32; ++kk)
+                tc_mma_mx(tmem_base, smem_desc_k_sw128(a_base + kk * 32),
+                          smem_desc_k_sw128(b_base + kk * 32), idesc_mx(BM, kUmmaN, 0, kBFmt, kk),
+                          t_sfa | (static_cast<uint32_t>(kk) << 30),
+                          t_sfb | (static_cast<uint32_t>(kk) << 30),
+                          (kb != sg.kb0 || kk != 0) ? 1u : 0u);
+              tc_commit(smem_u32(&empty_bar[s]));
+            }
+            issued = true;
+          }
+          if (!ok) break;
+          if (lane == 0) tc_commit(smem_u32(&tfull_bar[0]));
+        }
+      }
+      if (lane == 0) {
+        if (!ok) {
+          s_abort = 1;
+          report_error(p.status, MOE_ERR_TIMEOUT);
+        }
+        if (issued) {
+          tc_commit(smem_u32(&done_bar));
+          mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
+        }
+      }
+    } else if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(BM, kUmmaN);
       int it = 0, tc = 0;
       bool ok = true;
@@ -775,16 +999,17 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
       Seg sg;
       for (; cur.next(sc, sg); ++tc) {
         const TileCoord c = decode_tile<BM>(sg.tile, N, bn, p.ph[ph].n_tiles_n, s_mt, s_off);
-        const uint32_t tf = smem_u32(&tfull_bar[tc & 1]), te = smem_u32(&tempty_bar[tc & 1]);
+        const int bi = C::NACC == 2 ? (tc & 1) : 0;
+        const uint32_t tf = smem_u32(&tfull_bar[bi]), te = smem_u32(&tempty_bar[bi]);
         bool finished = false;
         if (ph == 0)
-          ok = epilogue_segment<EPI1, BN1, BM>(p, p.ph[0], sc, sg, c, tmem_base, tc, tf, te,
-                                               smem_u32(&epi_bar), epi_phase, &s_abort,
-                                               &s_fixup, &finished);
+          ok = epilogue_segment<EPI1, BN1, BM, C::NACC, C::BS>(p, p.ph[0], sc, sg, c, tmem_base, tc,
+                                                               tf, te, smem_u32(&epi_bar), epi_phase,
+                                                               &s_abort, &s_fixup, &finished);
         else
-          ok = epilogue_segment<EPI_STORE_F32, kDnBn, BM>(p, p.ph[1], sc, sg, c, tmem_base, tc,
-                                                          tf, te, smem_u32(&epi_bar), epi_phase,
-                                                          &s_abort, &s_fixup, &finished);
+          ok = epilogue_segment<EPI_STORE_F32, kDnBn, BM, C::NACC, false>(
+              p, p.ph[1], sc, sg, c, tmem_base, tc, tf, te, smem_u32(&epi_bar), epi_phase,
+              &s_abort, &s_fixup, &finished);
         if (!ok) break;
         if (ph == 0 && finished) {
           // this CTA wrote the tile's h: order it before TMA loads, then count it (one fenced
@@ -939,6 +1164,98 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
   }
 }
 
+// Block-scaled formats: the token rows x_perm as MXFP8 (the A operand of the gate/up GEMM).
+// Slot (gm, r) is row r of m-tile gm (the tiles of the grouped FFN: experts in order, 128
+// rows each, the last one of an expert partial). A valid row's 32-column blocks become E4M3
+// codes in xq [r_max, d] (bytes) and their scales go to the tile's atoms; rows past the
+// expert's end and blocks past d get scale code 0 (2^-127). The h atoms (filled by the
+// gate/up epilogue for valid rows) are zeroed first.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t* __restrict__ x,
+                                                            const int32_t* __restrict__ expert_offset,
+                                                            int N, int d, int num_kb, int64_t r_max,
+                                                            int m_tiles_cap, uint8_t* __restrict__ xq,
+                                                            uint8_t* __restrict__ x_atoms,
+                                                            uint8_t* __restrict__ h_atoms,
+                                                            int64_t h_atom_bytes, int* status) {
+  __shared__ int s_mt[257], s_off[257];
+  pdl_trigger();
+  pdl_wait();
+  const int tid = threadIdx.x, lane = tid & 31;
+  // zero the h atoms (16-byte stores; the region is a multiple of 512 bytes)
+  for (int64_t i = blockIdx.x * 256ll + tid; i < h_atom_bytes / 16; i += static_cast<int64_t>(gridDim.x) * 256)
+    reinterpret_cast<uint4*>(h_atoms)[i] = make_uint4(0u, 0u, 0u, 0u);
+  // per-expert m-tiles (one warp, serial over the <= 256 experts: tiny)
+  if (tid < 32) {
+    int acc = 0;
+    bool bad = false;
+    for (int e0 = 0; e0 < N; e0 += 32) {
+      const int e = e0 + lane;
+      int cnt = 0;
+      if (e < N) {
+        const int a = expert_offset[e], b = expert_offset[e + 1];
+        s_off[e] = a;
+        if (a < 0 || b < a || b > r_max) bad = true;
+        else cnt = (b - a + 127) / 128;
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (e < N) s_mt[e] = acc + incl - cnt;
+      acc += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      s_off[N] = expert_offset[N];
+      s_mt[N] = acc;
+    }
+    if (__any_sync(0xffffffffu, bad) || acc > m_tiles_cap) {
+      if (lane == 0) {
+        s_mt[N] = 0;  // no tiles: the grouped FFN reports the same offsets
+        if (blockIdx.x == 0) report_error(status, MOE_ERR_BOUNDS);
+      }
+    }
+  }
+  __syncthreads();
+  const int warp_g = blockIdx.x * 8 + (tid >> 5), warps = gridDim.x * 8;
+  const int64_t slots = static_cast<int64_t>(s_mt[N]) * 128;
+  for (int64_t sl = warp_g; sl < slots; sl += warps) {
+    const int gm = static_cast<int>(sl >> 7), r = static_cast<int>(sl & 127);
+    int lo = 0, hi = N - 1;  // expert of m-tile gm: the largest e with s_mt[e] <= gm
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_mt[mid] <= gm) lo = mid; else hi = mid - 1;
+    }
+    const int64_t row = s_off[lo] + static_cast<int64_t>(gm - s_mt[lo]) * 128 + r;
+    const bool valid = row < s_off[lo + 1] && row < r_max;
+    for (int q = lane; q < num_kb * 4; q += 32) {
+      uint32_t sc = 0;
+      if (valid && q * 32 < d) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + row * d + q * 32);
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 w = __ldg(src + j);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            v[8 * j + 2 * t] = __uint_as_float(ww[t] << 16);
+            v[8 * j + 2 * t + 1] = __uint_as_float(ww[t] & 0xffff0000u);
+          }
+        }
+        uint4 lo4, hi4;
+        sc = mxfp8_block(v, lo4, hi4);
+        uint4* dst = reinterpret_cast<uint4*>(xq + row * d + q * 32);
+        dst[0] = lo4;
+        dst[1] = hi4;
+      }
+      x_atoms[(static_cast<int64_t>(gm) * num_kb + q / 4) * 512 + sf_atom_byte(r, q & 3)] =
+          static_cast<uint8_t>(sc);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ host side
 template <int EPI1, int BN1, int BM, int WFMT>
 cudaError_t launch_one(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
@@ -992,19 +1309,21 @@ constexpr int kGuBnGelu = 256;
 }  // namespace
 
 FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max,
-                                int64_t rows_per_expert) {
+                                int64_t rows_per_expert, bool block_scaled) {
   FfnScratchPlan pl{};
   pl.bm = 128;
   if (r_max <= 0) return pl;
-  pl.bm = rows_per_expert <= 64 ? 64 : 128;
+  pl.bm = (rows_per_expert <= 64 && !block_scaled) ? 64 : 128;
+  const int kbe = block_scaled ? kBsK : BK;  // k per block
+  const int nkb1 = (d + kbe - 1) / kbe, nkb2 = (F + kbe - 1) / kbe;
   pl.slot_rows = static_cast<int>(std::min<int64_t>(pl.bm, std::max<int64_t>(1, rows_per_expert)));
   const int bn1 = act == MOE_ACT_SWIGLU ? kGuBnSwiglu : kGuBnGelu;
   pl.m_tiles_ub = m_tiles_upper_bound(r_max, N, pl.bm);
   pl.tiles1_ub = pl.m_tiles_ub * ((F + bn1 - 1) / bn1);
   pl.tiles2_ub = pl.m_tiles_ub * ((d + kDnBn - 1) / kDnBn);
   if (pl.slot_rows <= kSkMaxSlotRows) {
-    const int64_t by1 = pl.tiles1_ub * (d / BK) / std::min(kSkMinKb, d / BK);
-    const int64_t by2 = pl.tiles2_ub * (F / BK) / std::min(kSkMinKb, F / BK);
+    const int64_t by1 = pl.tiles1_ub * nkb1 / std::min(kSkMinKb, nkb1);
+    const int64_t by2 = pl.tiles2_ub * nkb2 / std::min(kSkMinKb, nkb2);
     pl.sk_ctas1 = static_cast<int>(std::min<int64_t>(kSkMaxCtas, by1));
     pl.sk_ctas2 = static_cast<int>(std::min<int64_t>(kSkMaxCtas, by2));
   }
@@ -1014,6 +1333,17 @@ FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max,
   pl.part_bytes = static_cast<size_t>(pl.sk_ctas1 + pl.sk_ctas2) * 2 * pl.slot_rows * kUmmaN *
                   sizeof(float);
   return pl;
+}
+
+MxActLayout mx_act_layout(int N, int d, int F, int64_t r_max) {
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  MxActLayout l{};
+  const int64_t mt = r_max > 0 ? m_tiles_upper_bound(r_max, N, 128) : 0;
+  l.xq_bytes = up(static_cast<size_t>(std::max<int64_t>(r_max, 0)) * d);
+  l.x_atom_bytes = up(static_cast<size_t>(mt) * ((d + kBsK - 1) / kBsK) * 512);
+  l.h_atom_bytes = up(static_cast<size_t>(mt) * ((F + kBsK - 1) / kBsK) * 512);
+  l.total = l.xq_bytes + l.x_atom_bytes + l.h_atom_bytes;
+  return l;
 }
 
 cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
@@ -1027,8 +1357,15 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   const uint64_t N = static_cast<uint64_t>(a.N), R = static_cast<uint64_t>(a.r_max);
   const bool swiglu = a.act == MOE_ACT_SWIGLU;
   const int bn_gu = swiglu ? kGuBnSwiglu : kGuBnGelu;
+  const bool bs = a.wfmt == MOE_WFMT_MXFP8_BS || a.wfmt == MOE_WFMT_MXFP4_BS;
   const FfnScratchPlan plan =
-      ffn_scratch_plan(a.N, a.d, a.F, a.act, a.r_max, a.rows_per_expert);
+      ffn_scratch_plan(a.N, a.d, a.F, a.act, a.r_max, a.rows_per_expert, bs);
+  if (bs) {  // the workspace regions were sized by the default plan
+    const FfnScratchPlan std_plan = ffn_scratch_plan(a.N, a.d, a.F, a.act, a.r_max, a.rows_per_expert);
+    if (plan.counter_bytes > std_plan.counter_bytes || plan.part_bytes > std_plan.part_bytes ||
+        a.act_ws == nullptr)
+      return cudaErrorInvalidValue;
+  }
   const int bm = plan.bm;
   // weights are read once per m-tile; when every expert has at most one m-tile (decode-sized
   // batches) they are pure streams and should not displace the activations in L2
@@ -1037,6 +1374,65 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   CUtensorMap mA1, mB1, mA2, mB2, mS1, mS2;
   memset(&mS1, 0, sizeof(mS1));  // bf16 weights: the scale maps are not read
   memset(&mS2, 0, sizeof(mS2));
+  const MxActLayout al = mx_act_layout(a.N, a.d, a.F, a.r_max);
+  uint8_t* const xq = static_cast<uint8_t*>(a.act_ws);
+  uint8_t* const x_atoms = bs ? xq + al.xq_bytes : nullptr;
+  uint8_t* const h_atoms = bs ? x_atoms + al.x_atom_bytes : nullptr;
+  if (bs) {
+    // A: the quantised rows and h as bytes [R][K], 128-byte boxes of 128 rows (128B swizzle)
+    {
+      const uint64_t dims[2] = {d, R};
+      const uint64_t str[1] = {d};
+      const uint32_t box[2] = {128, 128};
+      if (!make_map_u8(&mA1, xq, 2, dims, str, box, true)) return cudaErrorInvalidValue;
+    }
+    {
+      const uint64_t dims[2] = {F, R};
+      const uint64_t str[1] = {F};
+      const uint32_t box[2] = {128, 128};
+      if (!make_map_u8(&mA2, a.h, 2, dims, str, box, true)) return cudaErrorInvalidValue;
+    }
+    // B: the MX elements, one k block (128 elements) of 128 or 256 rows a box; E4M3 as bytes,
+    // E2M1 through the padded 4-bit type (k a multiple of 128). Scales: boxes of 4 blocks x
+    // 128 rows from [N][K/32][rows].
+    const bool fp4 = a.wfmt == MOE_WFMT_MXFP4_BS;
+    if (fp4 && (d % 128 != 0 || F % 128 != 0)) return cudaErrorInvalidValue;
+    const uint64_t db = fp4 ? d / 2 : d, fb = fp4 ? F / 2 : F;  // bytes per row
+    auto emap = [&](CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* str, const uint32_t* box) {
+      return fp4 ? make_map_fp4_padded(m, base, rank, dims, str, box)
+                 : make_map_u8(m, base, rank, dims, str, box, true);
+    };
+    if (swiglu) {
+      const uint64_t dims[4] = {d, F, 2, N};
+      const uint64_t str[3] = {db, F * db, 2 * F * db};
+      const uint32_t box[4] = {128, 128, 1, 1};
+      if (!emap(&mB1, a.w_gate_up, 4, dims, str, box)) return cudaErrorInvalidValue;
+      const uint64_t sd[4] = {F, 2, d / 32, N};
+      const uint64_t ss[3] = {F, 2 * F, (d / 32) * 2 * F};
+      const uint32_t sb[4] = {128, 1, 4, 1};
+      if (!make_map_u8(&mS1, a.w_gate_up_scales, 4, sd, ss, sb, false)) return cudaErrorInvalidValue;
+    } else {
+      const uint64_t dims[3] = {d, F, N};
+      const uint64_t str[2] = {db, F * db};
+      const uint32_t box[3] = {128, 256, 1};
+      if (!emap(&mB1, a.w_gate_up, 3, dims, str, box)) return cudaErrorInvalidValue;
+      const uint64_t sd[3] = {F, d / 32, N};
+      const uint64_t ss[2] = {F, (d / 32) * F};
+      const uint32_t sb[3] = {128, 4, 1};
+      if (!make_map_u8(&mS1, a.w_gate_up_scales, 3, sd, ss, sb, false)) return cudaErrorInvalidValue;
+    }
+    {
+      const uint64_t dims[3] = {F, d, N};
+      const uint64_t str[2] = {fb, d * fb};
+      const uint32_t box[3] = {128, 256, 1};
+      if (!emap(&mB2, a.w_down, 3, dims, str, box)) return cudaErrorInvalidValue;
+      const uint64_t sd[3] = {d, F / 32, N};
+      const uint64_t ss[2] = {d, (F / 32) * d};
+      const uint32_t sb[3] = {128, 4, 1};
+      if (!make_map_u8(&mS2, a.w_down_scales, 3, sd, ss, sb, false)) return cudaErrorInvalidValue;
+    }
+  } else {
   {
     const uint64_t dims[2] = {d, R};
     const uint64_t str[1] = {d * 2};
@@ -1101,6 +1497,7 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
     const uint32_t box[3] = {BK, static_cast<uint32_t>(kDnBn), 1};
     if (!make_map(&mB2, a.w_down, 3, dims, str, box)) return cudaErrorInvalidValue;
   }
+  }  // not block-scaled
 
   const bool stream_k = a.part != nullptr;
   FfnParams fp{};
@@ -1118,13 +1515,15 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   fp.status = a.status;
   fp.timeout_ns = a.timeout_ns;
   fp.weight_policy = wpol;
+  fp.x_atoms = x_atoms;
+  fp.h_atoms = h_atoms;
 
   PhaseParams& p1 = fp.ph[0];
   p1.out = a.h;
   p1.ld_out = a.F;
   p1.n_out = a.F;
   p1.n_tiles_n = (a.F + bn_gu - 1) / bn_gu;
-  p1.num_kb = a.d / BK;
+  p1.num_kb = bs ? (a.d + kBsK - 1) / kBsK : a.d / BK;
   p1.sk_ctas = stream_k ? plan.sk_ctas1 : 0;
   p1.part = a.part;
   p1.tile_counters = cnt;
@@ -1135,7 +1534,7 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   p2.ld_out = a.d;
   p2.n_out = a.d;
   p2.n_tiles_n = (a.d + kDnBn - 1) / kDnBn;
-  p2.num_kb = a.F / BK;
+  p2.num_kb = bs ? (a.F + kBsK - 1) / kBsK : a.F / BK;
   p2.sk_ctas = stream_k ? plan.sk_ctas2 : 0;
   p2.part = stream_k ? a.part + static_cast<size_t>(plan.sk_ctas1) * 2 * plan.slot_rows * kUmmaN
                      : nullptr;
@@ -1144,6 +1543,18 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   const int64_t useful = std::max(useful_ctas(plan.tiles1_ub, p1.num_kb, p1.sk_ctas),
                                   useful_ctas(plan.tiles2_ub, p2.num_kb, p2.sk_ctas));
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(useful, di.sm_count)));
+  if (bs) {
+    const int qgrid = static_cast<int>(std::min<int64_t>(
+        std::max<int64_t>(1, (plan.m_tiles_ub * 128 + 7) / 8), static_cast<int64_t>(di.sm_count) * 8));
+    cudaError_t qe = launch_pdl(quantize_rows_kernel, dim3(qgrid), dim3(256), 0, s, a.x_perm,
+                                a.expert_offset, a.N, a.d, p1.num_kb, a.r_max,
+                                static_cast<int>(plan.m_tiles_ub), xq, x_atoms, h_atoms,
+                                static_cast<int64_t>(al.h_atom_bytes), a.status);
+    if (qe != cudaSuccess) return qe;
+    if (a.wfmt == MOE_WFMT_MXFP8_BS)
+      return launch_fmt<WFMT_BS8>(swiglu, 128, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
+    return launch_fmt<WFMT_BS4>(swiglu, 128, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
+  }
   if (a.wfmt == MOE_WFMT_MXFP8)
     return launch_fmt<WFMT_MXFP8>(swiglu, bm, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
   if (a.wfmt == MOE_WFMT_MXFP4)
@@ -1156,9 +1567,14 @@ template <int WFMT>
 cudaError_t launch_fmt(bool swiglu, int bm, const CUtensorMap& a1, const CUtensorMap& b1,
                        const CUtensorMap& a2, const CUtensorMap& b2, const CUtensorMap& s1,
                        const CUtensorMap& s2, const FfnParams& fp, int grid, cudaStream_t s) {
-  if (bm == 64)
-    return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 64, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s)
-                  : launch_one<EPI_GELU, kGuBnGelu, 64, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s);
+  if constexpr (WFMT == WFMT_BS8 || WFMT == WFMT_BS4) {  // 128-row tiles only
+    return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s)
+                  : launch_one<EPI_GELU, kGuBnGelu, 128, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s);
+  } else {
+    if (bm == 64)
+      return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 64, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s)
+                    : launch_one<EPI_GELU, kGuBnGelu, 64, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s);
+  }
   return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s)
                 : launch_one<EPI_GELU, kGuBnGelu, 128, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s);
 }

@@ -231,9 +231,18 @@ struct FfnScratchPlan {
   size_t counter_bytes;
   size_t part_bytes;       // shares the workspace region with the routing scratch
 };
-// rows_per_expert: the most rows any one expert can receive, min(capacity, T).
+// rows_per_expert: the most rows any one expert can receive, min(capacity, T). block_scaled:
+// the plan of the block-scaled formats (128-row tiles, k blocks of 128); it never needs more
+// counter or partial bytes than the default plan of the same shape.
 FfnScratchPlan ffn_scratch_plan(int N, int d, int F, int act, int64_t r_max,
-                                int64_t rows_per_expert);
+                                int64_t rows_per_expert, bool block_scaled = false);
+// Bytes the block-scaled formats need besides the per-stage workspace: the quantised token
+// rows [r_max, d] (1 byte each) and the scale atoms of the rows and of h (512 bytes per m-tile
+// and k block of 128), each region rounded up to 256 bytes.
+struct MxActLayout {
+  size_t xq_bytes, x_atom_bytes, h_atom_bytes, total;
+};
+MxActLayout mx_act_layout(int N, int d, int F, int64_t r_max);
 
 struct GroupedFfnArgs {
   const uint16_t* x_perm;
@@ -252,6 +261,7 @@ struct GroupedFfnArgs {
   int* counters;            // ffn_scratch_plan().counter_bytes, zero between calls
   float* part;              // ffn_scratch_plan().part_bytes, or null: whole tiles only
   int64_t rows_per_expert;  // min(capacity, T)
+  void* act_ws;             // block-scaled formats: mx_act_layout().total bytes; else unused
 };
 cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s);
 

@@ -73,6 +73,32 @@ inline bool make_map_u8(CUtensorMap* m, const void* base, int rank, const uint64
   return r == CUDA_SUCCESS;
 }
 
+// FP4 elements stored packed (two per byte, element 2i in the low nibble) loaded into the
+// layout the block-scaled MMA reads for a 4-bit operand: every 16 elements (8 bytes) followed by
+// 8 bytes of padding, so a k block of 128 elements takes 128 bytes of shared memory (128B
+// swizzle). dims[0] counts elements (a multiple of 128), strides are in bytes (multiples of 32),
+// box[0] is 128 and the base 32-byte aligned.
+inline bool make_map_fp4_padded(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                                const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t gd[5];
+  cuuint64_t gs[4];
+  cuuint32_t bx[5];
+  cuuint32_t es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) gs[i] = strides_bytes[i];
+  }
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, static_cast<cuuint32_t>(rank),
+                        const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // fp32 tensor map with 128-byte swizzle (boxes of 32 elements along dims[0]), for stores.
 inline bool make_map_f32(CUtensorMap* m, void* base, int rank, const uint64_t* dims,
                          const uint64_t* strides_bytes, const uint32_t* box) {

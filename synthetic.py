@@ -203,9 +203,11 @@ def make_mx_matrix_stack(n_experts: int, rows: int, K: int, fmt: str, *, seed: i
 
 def make_mx_layer_inputs(shape: LayerShape, T: int, fmt: str, *, seed: int = 0, device="cpu") -> dict:
     """Hidden states and router as in make_layer_inputs; expert weights in an MX format:
-    w_gate_up_q/_s for the packed gate_up rows ([N, 2F or F, d]) and w_down_q/_s ([N, d, F])."""
+    w_gate_up_q/_s for the packed gate_up rows ([N, 2F or F, d]) and w_down_q/_s ([N, d, F]).
+    fmt "mxfp8_bs" / "mxfp4_bs" (block-scaled path) draws the same weights as "mxfp8" / "mxfp4"."""
     dev = torch.device(device)
     N, d, F = shape.n_experts, shape.d_model, shape.d_ff
+    wfmt, fmt = fmt, fmt[:-3] if fmt.endswith("_bs") else fmt
     w_router = _normal((N, d), 1.0 / math.sqrt(d), dev, seed, _WR)
     bias = zipf_logit_bias(N, shape.zipf_s).to(dev) if shape.zipf_s is not None else None
     gq, gs = make_mx_matrix_stack(N, shape.gate_up_rows(), d, fmt, seed=seed, tensor_id=_WGU_Q,
@@ -213,7 +215,7 @@ def make_mx_layer_inputs(shape: LayerShape, T: int, fmt: str, *, seed: int = 0, 
     dq, ds = make_mx_matrix_stack(N, d, F, fmt, seed=seed, tensor_id=_WD_Q, scale_tensor_id=_WD_S,
                                   device=dev)
     return {"x": make_hidden(T, d, seed=seed, device=dev), "w_router": w_router, "logit_bias": bias,
-            "wfmt": fmt, "w_gate_up_q": gq, "w_gate_up_s": gs, "w_down_q": dq, "w_down_s": ds}
+            "wfmt": wfmt, "w_gate_up_q": gq, "w_gate_up_s": gs, "w_down_q": dq, "w_down_s": ds}
 
 
 def make_mx_custom_inputs(T: int, d_model: int, n_experts: int, d_ff: int, act: str, fmt: str, *,

@@ -69,7 +69,9 @@ class StageRun:
         R = moe.max_rows(self.dims)
         self.R_max = R
         dev = device
-        self.ws = moe.new_workspace(self.dims, dev)
+        # block-scaled MX formats: quantised activations, room for them after the workspace
+        self.block_scaled = str(inp.get("wfmt", "")).endswith("_bs")
+        self.ws = moe.new_workspace(self.dims, dev, block_scaled=self.block_scaled)
         z = lambda shape, dt: torch.full(shape, -7, dtype=dt, device=dev) if dt == torch.int32 \
             else torch.full(shape, float("nan"), dtype=dt, device=dev)
         self.logits = z((T, N), torch.float32)
@@ -171,6 +173,7 @@ def expert_weights_f64(w: torch.Tensor):
 def mx_weight_getters(inp):
     """Lazy per-expert float64 weights decoded from MX storage by the oracle."""
     fmt = inp["wfmt"]
+    fmt = fmt[:-3] if fmt.endswith("_bs") else fmt
 
     def make(q, sc):
         cache = {}
@@ -183,11 +186,16 @@ def mx_weight_getters(inp):
     return make(inp["w_gate_up_q"], inp["w_gate_up_s"]), make(inp["w_down_q"], inp["w_down_s"])
 
 
+def expert_ffn_of(run: StageRun):
+    """The oracle's expert for this run: MXFP8-quantised activations on the block-scaled path."""
+    return oracle.expert_ffn_mxfp8_act if getattr(run, "block_scaled", False) else oracle.expert_ffn
+
+
 def check_outputs(run: StageRun, routing: dict, act: str, tokens=None, residual=True):
     i = run.inp
     x = f64(i["x"])
     res = x if residual else None
-    want = oracle.combine(x, routing, run.gu, run.dn, act, res, tokens)
+    want = oracle.combine(x, routing, run.gu, run.dn, act, res, tokens, ffn=expert_ffn_of(run))
     sel = slice(None) if tokens is None else torch.from_numpy(np.asarray(tokens)).long().cuda()
     g32 = f64(run.out32[sel])
     g16 = f64(run.out[sel])
@@ -234,7 +242,7 @@ def check_expert_rows(run: StageRun, routing: dict, act: str, rows: np.ndarray):
     for n, r in enumerate(rows):
         e = int(np.searchsorted(off, r, side="right") - 1)
         t = int(por[r]) // k
-        want = oracle.expert_ffn(f64(x[t:t + 1]), gu(e), dn(e), act)[0]
+        want = expert_ffn_of(run)(f64(x[t:t + 1]), gu(e), dn(e), act)[0]
         err = np.abs(y[n] - want)
         assert err.max() <= y_row_max_abs(want), f"row {r} (expert {e}, token {t}) max-abs {err.max()}"
         assert mean_rel(y[n], want) <= OUT_MEAN_REL
