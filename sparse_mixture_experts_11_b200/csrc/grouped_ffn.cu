@@ -111,8 +111,9 @@ struct FfnParams {
 // rows and h quantised to MXFP8.
 enum { WFMT_BF16 = 0, WFMT_MXFP8 = 1, WFMT_MXFP4 = 2, WFMT_BS8 = 3, WFMT_BS4 = 4 };
 constexpr int kBsK = 128;        // block-scaled: k per stage (128 one-byte elements = 128 bytes)
-constexpr int kBsSfStage = 2560; // per stage: A scale atom 512 B, raw B scales 1 KB, B atoms 1 KB
-constexpr int kBsBudget = 216 * 1024;
+constexpr int kBsSfB = 2048;      // per B stage: raw B scales 1 KB, their atoms 1 KB
+constexpr int kBsBudget = 226 * 1024;
+constexpr int kBsSmallRows = 32;  // BS tiles with at most this many rows load only those rows
 constexpr int kConvThreads = 256;  // MX decoders (warps 7-14)
 constexpr int kConvWarps = kConvThreads / 32;
 
@@ -120,7 +121,9 @@ template <int BM, int WFMT>
 struct Cfg {
   static constexpr bool MX = WFMT == WFMT_MXFP8 || WFMT == WFMT_MXFP4;  // decoded in smem
   static constexpr bool BS = WFMT == WFMT_BS8 || WFMT == WFMT_BS4;      // block-scaled MMA
-  static constexpr int THREADS = MX ? kThreads + 32 + kConvThreads : kThreads;
+  // MX: + the packed-ring producer and 8 decoder warps; BS: + a warp that lays out the weight
+  // scales of each stage for the TMEM copy (6) and the weight producer (7)
+  static constexpr int THREADS = MX ? kThreads + 32 + kConvThreads : (BS ? kThreads + 64 : kThreads);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = kUmmaN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -130,8 +133,11 @@ struct Cfg {
   static constexpr int ROW_BYTES = WFMT == WFMT_MXFP8 ? BK : BK / 2;  // per row and k block
   static constexpr int KG = MX ? 128 / ROW_BYTES : 1;
   static constexpr int STG_BYTES = MX ? kUmmaN * 128 + 2 * KG * kUmmaN : 0;
-  static constexpr int SF_STAGE = BS ? kBsSfStage : 0;
-  static constexpr int STAGES_RAW = BS ? kBsBudget / (STAGE_BYTES + kBsSfStage) : kSmemBudget / STAGE_BYTES;
+  // BS: weight stages (B tile + raw and laid-out scales) beside a ring of SA token-row stages
+  // (A tile + its scale atom): rows come from L2, weights from HBM, so the weights get the depth
+  static constexpr int SA_BS = 3;
+  static constexpr int STAGES_RAW = BS ? (kBsBudget - SA_BS * (A_BYTES + 512)) / (B_BYTES + kBsSfB)
+                                       : kSmemBudget / STAGE_BYTES;
   static constexpr int STAGES_FIT = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   // MX: two bf16 B stages (decoded from shared memory; a third measured no faster), a
   // separate ring of SA A stages
@@ -139,8 +145,8 @@ struct Cfg {
   // the weight streams load it), and the rest of 224 KB for packed stages
   static constexpr int kMxBudget = 224 * 1024;
   static constexpr int STAGES = MX ? 2 : STAGES_FIT;
-  static constexpr int SA = MX ? (BM == 64 ? 6 : 3) : 0;
-  static constexpr int B_RING = MX ? STAGES * B_BYTES : STAGES * STAGE_BYTES;  // bytes
+  static constexpr int SA = MX ? (BM == 64 ? 6 : 3) : (BS ? SA_BS : 0);
+  static constexpr int B_RING = (MX || BS) ? STAGES * B_BYTES : STAGES * STAGE_BYTES;  // bytes
   static constexpr int A_RING = SA * A_BYTES;
   static constexpr int SST_FIT = MX ? (kMxBudget - B_RING - A_RING) / STG_BYTES : 0;
   static constexpr int SST = SST_FIT > 16 ? 16 : SST_FIT;
@@ -148,7 +154,7 @@ struct Cfg {
   // accumulator buffers in TMEM: two (the epilogue of one tile overlaps the next tile's MMAs),
   // or one for BS, whose scale factors take TMEM columns 256 (A) and 264-271 (B)
   static constexpr int NACC = BS ? 1 : 2;
-  static constexpr int SF_RING = STAGES * SF_STAGE;
+  static constexpr int SF_RING = BS ? STAGES * kBsSfB + SA * 512 : 0;
   static constexpr int SMEM_BYTES = B_RING + A_RING + SST * STG_BYTES + SF_RING + 1024;  // + alignment slack
   static_assert(!BS || BM == 128, "block-scaled MMA: M = 128");
   static_assert(TMEM_COLS <= 512, "two accumulators must fit in TMEM");
@@ -616,7 +622,9 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
                        const __grid_constant__ CUtensorMap tmA2,
                        const __grid_constant__ CUtensorMap tmB2,
                        const __grid_constant__ CUtensorMap tmS1,
-                       const __grid_constant__ CUtensorMap tmS2, const FfnParams p) {
+                       const __grid_constant__ CUtensorMap tmS2,
+                       const __grid_constant__ CUtensorMap tmA1s,
+                       const __grid_constant__ CUtensorMap tmA2s, const FfnParams p) {
   using C = Cfg<BM, WFMT>;
   static_assert(EPI1 != EPI_SWIGLU || 2 * BN1 == kUmmaN, "SwiGLU tile: gate | up halves");
   static_assert(EPI1 == EPI_SWIGLU || BN1 == kUmmaN, "GELU tile");
@@ -636,8 +644,9 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
   __shared__ int s_last_cta;
   __shared__ __align__(8) uint64_t sfull_bar[C::MX ? C::SST : 1];
   __shared__ __align__(8) uint64_t sempty_bar[C::MX ? C::SST : 1];
-  __shared__ __align__(8) uint64_t afull_bar[C::MX ? C::SA : 1];
-  __shared__ __align__(8) uint64_t aempty_bar[C::MX ? C::SA : 1];
+  __shared__ __align__(8) uint64_t afull_bar[(C::MX || C::BS) ? C::SA : 1];
+  __shared__ __align__(8) uint64_t aempty_bar[(C::MX || C::BS) ? C::SA : 1];
+  __shared__ __align__(8) uint64_t sfready_bar[C::BS ? C::STAGES : 1];  // BS: stage's scale atoms laid out
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5;
@@ -646,23 +655,26 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
   const uint32_t tiles = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   // bf16: stage s = [A | B]; MX: B stages, then the A ring, then the packed ring
   const uint32_t stg0 = tiles + C::B_RING + C::A_RING;
+  constexpr bool kSplitA = C::MX || C::BS;  // the A operand has its own ring
   auto a_addr = [&](int i) -> uint32_t {
-    return C::MX ? tiles + C::B_RING + i * C::A_BYTES : tiles + i * C::STAGE_BYTES;
+    return kSplitA ? tiles + C::B_RING + i * C::A_BYTES : tiles + i * C::STAGE_BYTES;
   };
   auto b_addr = [&](int i) -> uint32_t {
-    return C::MX ? tiles + i * C::B_BYTES : tiles + i * C::STAGE_BYTES + C::A_BYTES;
+    return kSplitA ? tiles + i * C::B_BYTES : tiles + i * C::STAGE_BYTES + C::A_BYTES;
   };
-  constexpr int AST = C::MX ? C::SA : C::STAGES;  // stages of the A operand's ring
-  // BS: per stage [A scale atom 512 B | raw B scales [2][4][128] | B scale atoms [2][512]]
+  constexpr int AST = kSplitA ? C::SA : C::STAGES;  // stages of the A operand's ring
+  // BS: per weight stage [raw B scales [2][4][128] | B scale atoms [2][512]], then per A stage
+  // the rows' scale atom (512 B)
   const uint32_t sf0 = stg0 + C::SST * C::STG_BYTES;
-  auto sf_addr = [&](int i) -> uint32_t { return sf0 + i * C::SF_STAGE; };
+  auto sf_addr = [&](int i) -> uint32_t { return sf0 + i * kBsSfB; };
+  auto sfa_addr = [&](int i) -> uint32_t { return sf0 + C::STAGES * kBsSfB + i * 512; };
   // BS: the A scale atom of (m-tile gm, k block kb) of phase ph
   auto a_atom = [&](int ph, int gm, int kb) -> const uint8_t* {
     return (ph == 0 ? p.x_atoms : p.h_atoms) + (static_cast<int64_t>(gm) * p.ph[ph].num_kb + kb) * 512;
   };
   constexpr int KX = C::BS ? kBsK : BK;  // A / B column coordinate step per k block
-  uint64_t* const a_full = C::MX ? afull_bar : full_bar;
-  uint64_t* const a_empty = C::MX ? aempty_bar : empty_bar;
+  uint64_t* const a_full = kSplitA ? afull_bar : full_bar;
+  uint64_t* const a_empty = kSplitA ? aempty_bar : empty_bar;
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmA1);
@@ -688,6 +700,8 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
       mbar_init(smem_u32(&afull_bar[s]), 1);
       mbar_init(smem_u32(&aempty_bar[s]), 1);
     }
+    if (C::BS)
+      for (int s = 0; s < C::STAGES; ++s) mbar_init(smem_u32(&sfready_bar[s]), 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tfull_bar[b]), 1);
       mbar_init(smem_u32(&tempty_bar[b]), kEpiThreads);
@@ -772,11 +786,15 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
       for (int ph = 0; ph < 2 && ok; ++ph) {
         const Sched sc = s_sched[ph];
         const int bn = ph == 0 ? BN1 : kDnBn;
-        const CUtensorMap* tA = ph == 0 ? &tmA1 : &tmA2;
         SegCursor cur(sc);
         Seg sg;
         while (ok && cur.next(sc, sg)) {
           const TileCoord c = decode_tile<BM>(sg.tile, N, bn, p.ph[ph].n_tiles_n, s_mt, s_off);
+          // BS: a tile of at most 32 rows loads just those (the MMA's other rows read stale
+          // shared memory; their results are never stored)
+          const bool small_a = C::BS && c.rows <= kBsSmallRows;
+          const CUtensorMap* tA = small_a ? (ph == 0 ? &tmA1s : &tmA2s) : (ph == 0 ? &tmA1 : &tmA2);
+          const uint32_t a_bytes = small_a ? kBsSmallRows * 128 : C::A_BYTES;
           // phase 1: the W_d blocks go out at once; the h blocks once the rows' h is complete
           // (one poll here: an acquire load stalls this thread for an L2 round trip)
           bool ready = ph == 0 || ld_acquire_gpu(p.h_ready + c.gm) >= h_target;
@@ -792,28 +810,8 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
             const uint32_t fb = smem_u32(&a_full[s]);
             const uint32_t a_dst = a_addr(s);
             const uint32_t b_dst = b_addr(s);
-            // (E2M1 through the padded 4-bit type counts its packed bytes, half the smem it fills)
-            mbar_arrive_expect_tx(fb, C::MX ? C::A_BYTES
-                                            : C::STAGE_BYTES + (C::BS ? 1536 : 0) -
-                                                  (WFMT == WFMT_BS4 ? C::B_BYTES / 2 : 0));
-            if (C::BS) {
-              // weights and their raw scales ([half][4 blocks][128 rows] bytes); the token
-              // rows' scale atom goes with the A tile
-              const uint32_t sfr = sf_addr(s) + 512;
-              const int kx = kb * kBsK;
-              if (ph == 0 && EPI1 == EPI_SWIGLU) {
-                tma_load_4d(b_dst, &tmB1, fb, kx, c.n0, 0, c.e, pol_b);
-                tma_load_4d(b_dst + BN1 * 128, &tmB1, fb, kx, c.n0, 1, c.e, pol_b);
-                tma_load_4d(sfr, &tmS1, fb, c.n0, 0, 4 * kb, c.e, pol_b);
-                tma_load_4d(sfr + 512, &tmS1, fb, c.n0, 1, 4 * kb, c.e, pol_b);
-              } else {
-                const CUtensorMap* tb = ph == 0 ? &tmB1 : &tmB2;
-                const CUtensorMap* ts = ph == 0 ? &tmS1 : &tmS2;
-                tma_load_3d(b_dst, tb, fb, kx, c.n0, c.e, pol_b);
-                tma_load_3d(sfr, ts, fb, c.n0, 4 * kb, c.e, pol_b);
-                tma_load_3d(sfr + 512, ts, fb, c.n0 + 128, 4 * kb, c.e, pol_b);
-              }
-            } else if (!C::MX) {  // MX: the decoders fill the B half
+            mbar_arrive_expect_tx(fb, C::MX ? C::A_BYTES : (C::BS ? a_bytes + 512 : C::STAGE_BYTES));
+            if (!C::MX && !C::BS) {  // MX: the decoders fill the B half; BS: warp 7 loads it
               if (ph == 0) {
                 if (EPI1 == EPI_SWIGLU) {
                   tma_load_4d(b_dst, &tmB1, fb, kb * BK, c.n0, 0, c.e, pol_b);
@@ -827,7 +825,7 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
             }
             if (ready) {
               tma_load_2d(a_dst, tA, fb, kb * KX, c.m0, pol_a);
-              if (C::BS) bulk_load(sf_addr(s), a_atom(ph, c.gm, kb), 512, fb);
+              if (C::BS) bulk_load(sfa_addr(s), a_atom(ph, c.gm, kb), 512, fb);
               ++it;
               continue;
             }
@@ -841,7 +839,7 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
                 const int sj = j % AST;
                 const int kbj = sg.kb0 + (j - seg_it0);
                 tma_load_2d(a_addr(sj), tA, smem_u32(&a_full[sj]), kbj * KX, c.m0, pol_a);
-                if (C::BS) bulk_load(sf_addr(sj), a_atom(ph, c.gm, kbj), 512, smem_u32(&a_full[sj]));
+                if (C::BS) bulk_load(sfa_addr(sj), a_atom(ph, c.gm, kbj), 512, smem_u32(&a_full[sj]));
               }
               pend_from = -1;
               ready = true;
@@ -862,52 +860,39 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if constexpr (C::BS) {
-      // Block-scaled: the whole warp turns each stage's raw weight scales ([half][block][row])
-      // into the two 512-byte atoms of the TMEM copy layout; lane 0 copies the A and B atoms
-      // into TMEM (A at column 256, B at 264-271) and issues the four K = 32 MMAs. TMEM copies
-      // and MMAs of one thread run in issue order, so one scale area serves every stage.
-      constexpr int kBFmt = WFMT == WFMT_BS4 ? 5 : 0;  // E2M1 or E4M3 weights; A is E4M3
-      const uint32_t t_sfa = tmem_base + kUmmaN, t_sfb = tmem_base + kUmmaN + 8;
-      int it = 0, tc = 0;
-      bool ok = true;
-      bool issued = false;
-      for (int ph = 0; ph < 2 && ok; ++ph) {
-        const Sched sc = s_sched[ph];
-        SegCursor cur(sc);
-        Seg sg;
-        for (; ok && cur.next(sc, sg); ++tc) {
-          // one accumulator: the epilogue has read the previous segment's
-          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&tempty_bar[0]), (tc & 1) ^ 1u, p.timeout_ns, &s_abort));
-          if (!ok) break;
-          tc_fence_after_sync();
-          for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
-            const int s = it % C::STAGES;
-            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[s]), (it / C::STAGES) & 1,
-                                                    p.timeout_ns, &s_abort));
-            if (!ok) break;
-            {
-              const uint8_t* raw = dyn_smem + (sf_addr(s) + 512 - smem_u32(dyn_smem));
-              uint8_t* atoms = dyn_smem + (sf_addr(s) + 1536 - smem_u32(dyn_smem));
-#pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                uint32_t w[4];
-#pragma unroll
-                for (int r1 = 0; r1 < 4; ++r1) {
-                  const uint8_t* src = raw + j * 512 + r1 * 32 + lane;
-                  w[r1] = static_cast<uint32_t>(src[0]) | (static_cast<uint32_t>(src[128]) << 8) |
-                          (static_cast<uint32_t>(src[256]) << 16) | (static_cast<uint32_t>(src[384]) << 24);
-                }
-                *reinterpret_cast<uint4*>(atoms + j * 512 + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-              }
+      // Block-scaled: once warp 6 has laid out a stage's scale atoms (which implies the stage's
+      // loads have landed), lane 0 copies the A and B atoms into TMEM (A at column 256, B at
+      // 264-271) and issues the four K = 32 MMAs. TMEM copies and MMAs of one thread run in
+      // issue order, so one scale area in TMEM serves every stage.
+      if (lane == 0) {
+        constexpr int kBFmt = WFMT == WFMT_BS4 ? 5 : 0;  // E2M1 or E4M3 weights; A is E4M3
+        const uint32_t t_sfa = tmem_base + kUmmaN, t_sfb = tmem_base + kUmmaN + 8;
+        int it = 0, tc = 0;
+        bool ok = true;
+        bool issued = false;
+        for (int ph = 0; ph < 2 && ok; ++ph) {
+          const Sched sc = s_sched[ph];
+          SegCursor cur(sc);
+          Seg sg;
+          for (; ok && cur.next(sc, sg); ++tc) {
+            // one accumulator: the epilogue has read the previous segment's
+            if (!mbar_wait(smem_u32(&tempty_bar[0]), (tc & 1) ^ 1u, p.timeout_ns, &s_abort)) {
+              ok = false;
+              break;
             }
-            fence_proxy_async_smem();  // generic stores -> visible to the tensor core's copy
-            __syncwarp();
-            if (lane == 0) {
+            tc_fence_after_sync();
+            for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+              const int s = it % C::STAGES, sa = it % C::SA;
+              if (!mbar_wait(smem_u32(&sfready_bar[s]), (it / C::STAGES) & 1, p.timeout_ns, &s_abort) ||
+                  !mbar_wait(smem_u32(&afull_bar[sa]), (it / C::SA) & 1, p.timeout_ns, &s_abort)) {
+                ok = false;
+                break;
+              }
               tc_fence_after_sync();
-              const uint32_t a_base = a_addr(s), b_base = b_addr(s);
-              tc_cp_32x128b_x4(t_sfa, smem_desc_plain(sf_addr(s)));
-              tc_cp_32x128b_x4(t_sfb, smem_desc_plain(sf_addr(s) + 1536));
-              tc_cp_32x128b_x4(t_sfb + 4, smem_desc_plain(sf_addr(s) + 2048));
+              const uint32_t a_base = a_addr(sa), b_base = b_addr(s);
+              tc_cp_32x128b_x4(t_sfa, smem_desc_plain(sfa_addr(sa)));
+              tc_cp_32x128b_x4(t_sfb, smem_desc_plain(sf_addr(s) + 1024));
+              tc_cp_32x128b_x4(t_sfb + 4, smem_desc_plain(sf_addr(s) + 1536));
 #pragma unroll
               for (int kk = 0; kk < kBsK / 32; ++kk)
                 tc_mma_mx(tmem_base, smem_desc_k_sw128(a_base + kk * 32),
@@ -916,14 +901,13 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
                           t_sfb | (static_cast<uint32_t>(kk) << 30),
                           (kb != sg.kb0 || kk != 0) ? 1u : 0u);
               tc_commit(smem_u32(&empty_bar[s]));
+              tc_commit(smem_u32(&aempty_bar[sa]));
+              issued = true;
             }
-            issued = true;
+            if (!ok) break;
+            tc_commit(smem_u32(&tfull_bar[0]));
           }
-          if (!ok) break;
-          if (lane == 0) tc_commit(smem_u32(&tfull_bar[0]));
         }
-      }
-      if (lane == 0) {
         if (!ok) {
           s_abort = 1;
           report_error(p.status, MOE_ERR_TIMEOUT);
@@ -1029,6 +1013,95 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
     if (!ok) {
       s_abort = 1;
       report_error(p.status, MOE_ERR_TIMEOUT);
+    }
+  } else if (C::BS && warp == 6) {
+    // ---------------------------------------------------------------- BS scale layout (warp 6)
+    // Each stage's raw weight scales ([half][4 blocks][128 rows] bytes, as TMA loaded them)
+    // become the two 512-byte atoms of the TMEM copy layout: row r = r0 + 32 r1 of half j and
+    // block q at byte 16 r0 + 4 r1 + q of atom j; lane r0 writes its 16 bytes of each atom.
+    // The stage is written again only after its MMAs (and their TMEM copies) have finished.
+    int it = 0;
+    bool ok = true;
+    for (int ph = 0; ph < 2 && ok; ++ph) {
+      const Sched sc = s_sched[ph];
+      SegCursor cur(sc);
+      Seg sg;
+      while (ok && cur.next(sc, sg)) {
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[s]), (it / C::STAGES) & 1,
+                                                  p.timeout_ns, &s_abort));
+          if (!ok) break;
+          const uint8_t* raw = dyn_smem + (sf_addr(s) - smem_u32(dyn_smem));
+          uint8_t* atoms = dyn_smem + (sf_addr(s) + 1024 - smem_u32(dyn_smem));
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            uint32_t w[4];
+#pragma unroll
+            for (int r1 = 0; r1 < 4; ++r1) {
+              const uint8_t* src = raw + j * 512 + r1 * 32 + lane;
+              w[r1] = static_cast<uint32_t>(src[0]) | (static_cast<uint32_t>(src[128]) << 8) |
+                      (static_cast<uint32_t>(src[256]) << 16) | (static_cast<uint32_t>(src[384]) << 24);
+            }
+            *reinterpret_cast<uint4*>(atoms + j * 512 + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          fence_proxy_async_smem();  // generic stores -> visible to the tensor core's copy
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sfready_bar[s]));
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      s_abort = 1;
+      report_error(p.status, MOE_ERR_TIMEOUT);
+    }
+  } else if (C::BS && warp == 7) {
+    // ---------------------------------------------------------------- BS weight producer (warp 7)
+    // Weight tiles and their raw scales ([half][4 blocks][128 rows] bytes) into the weight ring,
+    // running ahead of the token rows (warp 0), which come from L2.
+    if (lane == 0) {
+      const uint64_t pol_b = make_policy(p.weight_policy);
+      int it = 0;
+      bool ok = true;
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        const Sched sc = s_sched[ph];
+        const int bn = ph == 0 ? BN1 : kDnBn;
+        SegCursor cur(sc);
+        Seg sg;
+        while (ok && cur.next(sc, sg)) {
+          const TileCoord c = decode_tile<BM>(sg.tile, N, bn, p.ph[ph].n_tiles_n, s_mt, s_off);
+          for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+            const int s = it % C::STAGES;
+            if (!mbar_wait(smem_u32(&empty_bar[s]), ((it / C::STAGES) & 1) ^ 1u, p.timeout_ns, &s_abort)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = smem_u32(&full_bar[s]);
+            const uint32_t b_dst = b_addr(s), sfr = sf_addr(s);
+            // E2M1 through the padded 4-bit type counts its packed bytes, half the smem it fills
+            mbar_arrive_expect_tx(fb, (WFMT == WFMT_BS4 ? C::B_BYTES / 2 : C::B_BYTES) + 1024);
+            const int kx = kb * kBsK;
+            if (ph == 0 && EPI1 == EPI_SWIGLU) {
+              tma_load_4d(b_dst, &tmB1, fb, kx, c.n0, 0, c.e, pol_b);
+              tma_load_4d(b_dst + BN1 * 128, &tmB1, fb, kx, c.n0, 1, c.e, pol_b);
+              tma_load_4d(sfr, &tmS1, fb, c.n0, 0, 4 * kb, c.e, pol_b);
+              tma_load_4d(sfr + 512, &tmS1, fb, c.n0, 1, 4 * kb, c.e, pol_b);
+            } else {
+              const CUtensorMap* tb = ph == 0 ? &tmB1 : &tmB2;
+              const CUtensorMap* ts = ph == 0 ? &tmS1 : &tmS2;
+              tma_load_3d(b_dst, tb, fb, kx, c.n0, c.e, pol_b);
+              tma_load_3d(sfr, ts, fb, c.n0, 4 * kb, c.e, pol_b);
+              tma_load_3d(sfr + 512, ts, fb, c.n0 + 128, 4 * kb, c.e, pol_b);
+            }
+          }
+        }
+      }
+      if (!ok) {
+        s_abort = 1;
+        report_error(p.status, MOE_ERR_TIMEOUT);
+      }
+      for (int i = max(0, it - C::STAGES); i < it; ++i)
+        mbar_wait(smem_u32(&full_bar[i % C::STAGES]), (i / C::STAGES) & 1, kDrainTimeoutNs, nullptr);
     }
   } else if (C::MX && warp == 6) {
     // ---------------------------------------------------------------- MX packed-ring producer
@@ -1260,6 +1333,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t* __re
 template <int EPI1, int BN1, int BM, int WFMT>
 cudaError_t launch_one(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
                        const CUtensorMap& b2, const CUtensorMap& s1, const CUtensorMap& s2,
+                       const CUtensorMap& a1s, const CUtensorMap& a2s,
                        const FfnParams& fp, int grid, cudaStream_t s) {
   using C = Cfg<BM, WFMT>;
   static PerDeviceOnce once;
@@ -1278,13 +1352,14 @@ cudaError_t launch_one(const CUtensorMap& a1, const CUtensorMap& b1, const CUten
   if (de != cudaSuccess) return de;
   if (static_cast<int64_t>(per_sm) * di.sm_count < grid) return cudaErrorInvalidConfiguration;
   return launch_pdl(grouped_ffn_kernel<EPI1, BN1, BM, WFMT>, dim3(grid), dim3(C::THREADS),
-                    C::SMEM_BYTES, s, a1, b1, a2, b2, s1, s2, fp);
+                    C::SMEM_BYTES, s, a1, b1, a2, b2, s1, s2, a1s, a2s, fp);
 }
 
 template <int WFMT>
 cudaError_t launch_fmt(bool swiglu, int bm, const CUtensorMap& a1, const CUtensorMap& b1,
                        const CUtensorMap& a2, const CUtensorMap& b2, const CUtensorMap& s1,
-                       const CUtensorMap& s2, const FfnParams& fp, int grid, cudaStream_t s);
+                       const CUtensorMap& s2, const CUtensorMap& a1s, const CUtensorMap& a2s,
+                       const FfnParams& fp, int grid, cudaStream_t s);
 
 // sum_e ceil(m_e / bm) <= ceil(R / bm) + (experts with rows)
 int64_t m_tiles_upper_bound(int64_t r_max, int N, int bm) {
@@ -1371,9 +1446,11 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   // batches) they are pure streams and should not displace the activations in L2
   const int wpol = (a.rows_per_expert <= bm) ? 1 : 0;
 
-  CUtensorMap mA1, mB1, mA2, mB2, mS1, mS2;
+  CUtensorMap mA1, mB1, mA2, mB2, mS1, mS2, mA1s, mA2s;
   memset(&mS1, 0, sizeof(mS1));  // bf16 weights: the scale maps are not read
   memset(&mS2, 0, sizeof(mS2));
+  memset(&mA1s, 0, sizeof(mA1s));  // only the block-scaled formats read the 32-row maps
+  memset(&mA2s, 0, sizeof(mA2s));
   const MxActLayout al = mx_act_layout(a.N, a.d, a.F, a.r_max);
   uint8_t* const xq = static_cast<uint8_t*>(a.act_ws);
   uint8_t* const x_atoms = bs ? xq + al.xq_bytes : nullptr;
@@ -1385,12 +1462,16 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
       const uint64_t str[1] = {d};
       const uint32_t box[2] = {128, 128};
       if (!make_map_u8(&mA1, xq, 2, dims, str, box, true)) return cudaErrorInvalidValue;
+      const uint32_t box_s[2] = {128, static_cast<uint32_t>(kBsSmallRows)};
+      if (!make_map_u8(&mA1s, xq, 2, dims, str, box_s, true)) return cudaErrorInvalidValue;
     }
     {
       const uint64_t dims[2] = {F, R};
       const uint64_t str[1] = {F};
       const uint32_t box[2] = {128, 128};
       if (!make_map_u8(&mA2, a.h, 2, dims, str, box, true)) return cudaErrorInvalidValue;
+      const uint32_t box_s[2] = {128, static_cast<uint32_t>(kBsSmallRows)};
+      if (!make_map_u8(&mA2s, a.h, 2, dims, str, box_s, true)) return cudaErrorInvalidValue;
     }
     // B: the MX elements, one k block (128 elements) of 128 or 256 rows a box; E4M3 as bytes,
     // E2M1 through the padded 4-bit type (k a multiple of 128). Scales: boxes of 4 blocks x
@@ -1552,31 +1633,32 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
                                 static_cast<int64_t>(al.h_atom_bytes), a.status);
     if (qe != cudaSuccess) return qe;
     if (a.wfmt == MOE_WFMT_MXFP8_BS)
-      return launch_fmt<WFMT_BS8>(swiglu, 128, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
-    return launch_fmt<WFMT_BS4>(swiglu, 128, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
+      return launch_fmt<WFMT_BS8>(swiglu, 128, mA1, mB1, mA2, mB2, mS1, mS2, mA1s, mA2s, fp, grid, s);
+    return launch_fmt<WFMT_BS4>(swiglu, 128, mA1, mB1, mA2, mB2, mS1, mS2, mA1s, mA2s, fp, grid, s);
   }
   if (a.wfmt == MOE_WFMT_MXFP8)
-    return launch_fmt<WFMT_MXFP8>(swiglu, bm, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
+    return launch_fmt<WFMT_MXFP8>(swiglu, bm, mA1, mB1, mA2, mB2, mS1, mS2, mA1s, mA2s, fp, grid, s);
   if (a.wfmt == MOE_WFMT_MXFP4)
-    return launch_fmt<WFMT_MXFP4>(swiglu, bm, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
-  return launch_fmt<WFMT_BF16>(swiglu, bm, mA1, mB1, mA2, mB2, mS1, mS2, fp, grid, s);
+    return launch_fmt<WFMT_MXFP4>(swiglu, bm, mA1, mB1, mA2, mB2, mS1, mS2, mA1s, mA2s, fp, grid, s);
+  return launch_fmt<WFMT_BF16>(swiglu, bm, mA1, mB1, mA2, mB2, mS1, mS2, mA1s, mA2s, fp, grid, s);
 }
 
 namespace {
 template <int WFMT>
 cudaError_t launch_fmt(bool swiglu, int bm, const CUtensorMap& a1, const CUtensorMap& b1,
                        const CUtensorMap& a2, const CUtensorMap& b2, const CUtensorMap& s1,
-                       const CUtensorMap& s2, const FfnParams& fp, int grid, cudaStream_t s) {
+                       const CUtensorMap& s2, const CUtensorMap& a1s, const CUtensorMap& a2s,
+                       const FfnParams& fp, int grid, cudaStream_t s) {
   if constexpr (WFMT == WFMT_BS8 || WFMT == WFMT_BS4) {  // 128-row tiles only
-    return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s)
-                  : launch_one<EPI_GELU, kGuBnGelu, 128, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s);
+    return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128, WFMT>(a1, b1, a2, b2, s1, s2, a1s, a2s, fp, grid, s)
+                  : launch_one<EPI_GELU, kGuBnGelu, 128, WFMT>(a1, b1, a2, b2, s1, s2, a1s, a2s, fp, grid, s);
   } else {
     if (bm == 64)
-      return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 64, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s)
-                    : launch_one<EPI_GELU, kGuBnGelu, 64, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s);
+      return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 64, WFMT>(a1, b1, a2, b2, s1, s2, a1s, a2s, fp, grid, s)
+                    : launch_one<EPI_GELU, kGuBnGelu, 64, WFMT>(a1, b1, a2, b2, s1, s2, a1s, a2s, fp, grid, s);
   }
-  return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s)
-                : launch_one<EPI_GELU, kGuBnGelu, 128, WFMT>(a1, b1, a2, b2, s1, s2, fp, grid, s);
+  return swiglu ? launch_one<EPI_SWIGLU, kGuBnSwiglu, 128, WFMT>(a1, b1, a2, b2, s1, s2, a1s, a2s, fp, grid, s)
+                : launch_one<EPI_GELU, kGuBnGelu, 128, WFMT>(a1, b1, a2, b2, s1, s2, a1s, a2s, fp, grid, s);
 }
 }  // namespace
 
