@@ -137,12 +137,17 @@ def roofline_of(shape, T: int, R: int, active: int, ffn_ms: float, step_ms: floa
     targets are stated on. Tensor-bound points also report the layer's TFLOP/s."""
     ab = algorithmic_bytes(shape, T, active, R, wfmt)
     flops = ffn_flops(shape, R)
-    ridge = (peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9)
+    # the block-scaled formats run FP8 MMAs: their tensor peak is the bf16 one times the
+    # nominal FP8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense)
+    fp8 = wfmt.endswith("_bs")
+    t_peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+    ridge = (t_peak * 1e12) / (peaks["hbm_gbs"] * 1e9)
     tensor = ab["weights"] > 0 and flops / ab["weights"] > ridge
     ffn_s, step_s = ffn_ms * 1e-3, step_ms * 1e-3
     if tensor:
-        ach, peak, unit = flops / ffn_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-        per_launch, src = f"{flops} FLOP", peaks["source"] + " bf16 burst"
+        ach, peak, unit = flops / ffn_s / 1e12, t_peak, "TFLOP/s"
+        per_launch = f"{flops} FLOP"
+        src = peaks["source"] + (" bf16 burst x 2 (fp8)" if fp8 else " bf16 burst")
     else:
         ach, peak, unit = ab["weights"] / ffn_s / 1e9, peaks["hbm_gbs"], "GB/s"
         per_launch, src = f"{ab['weights']} B", peaks["source"] + " copy"
@@ -954,6 +959,45 @@ def run_reference(args, rank, world):
 
 
 # ----------------------------------------------------------------------------- main
+def run_route_only(args) -> dict:
+    """moe_route on the workload's tokens and router (synthetic, as in the layer), timed as a
+    captured graph between L2 flushes."""
+    import sparse_mixture_experts_11_b200 as moe
+    device = torch.device("cuda")
+    shape, T = parse_workload(args.workload)
+    r = synthetic.make_router_weights(shape, device=device)
+    x = synthetic.make_hidden(T, shape.d_model, device=device)
+    N, k = shape.n_experts, shape.top_k
+    dims = moe.make_dims(T, shape.d_model, N, k, shape.d_ff, shape.act, capacity_of(shape, T))
+    ws = moe.new_workspace(dims, device)
+    logits = torch.empty(T, N, device=device)
+    idx = torch.empty(T, k, dtype=torch.int32, device=device)
+    tw = torch.empty(T, k, device=device)
+    slot = torch.empty(T, k, dtype=torch.int32, device=device)
+    cnt = torch.empty(N, dtype=torch.int32, device=device)
+    call = lambda: moe.route(dims, x, r["w_router"], r.get("logit_bias"), logits, idx, tw, slot, cnt, ws)
+    flush = (torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device),
+             torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device))
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    ts = []
+    for _ in range(args.steps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    del g
+    return {"metric": "route_ms", "value": round(statistics.median(ts), 4), "unit": "ms",
+            "workload": shape.describe(T), "steps": args.steps, "warmup": args.warmup}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -970,6 +1014,9 @@ def main(argv=None):
                     help="'all' (every workload point), 'none', or a comma list of shape:T")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the router-statistics, backward and redirect timings")
+    ap.add_argument("--route-only", action="store_true",
+                    help="time moe_route alone on the workload's tokens (no expert weights on "
+                         "the device; for profiling the routing kernels)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -982,6 +1029,10 @@ def main(argv=None):
         line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
+        return 0
+
+    if args.route_only:
+        print(json.dumps(run_route_only(args)), flush=True)
         return 0
 
     if world > 1:
