@@ -1237,6 +1237,363 @@ __global__ void __launch_bounds__(Cfg<BM, WFMT>::THREADS, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair kernel
+// bf16 weights in batches whose experts hold many 128-row m-tiles (the tensor-bound regime): a
+// cluster of two CTAs takes two neighbouring m-tiles of one expert and the same output
+// columns. The even CTA issues M = 256 MMAs (cta_group::2); each CTA holds its own 128 token
+// rows and half of the 256 weight rows (SwiGLU: the gate rows in the even CTA, the up rows in
+// the odd one). Each SM's tensor core then reads 8 KB of operands per MMA instead of 12 KB, so
+// the TMA writes and MMA reads of shared memory stay within its bandwidth. Whole tiles only;
+// the down projection waits on the same per-m-tile h counters as the one-CTA kernel. A pair
+// whose odd m-tile lies past its expert's rows computes it (from whatever rows TMA returns)
+// and stores nothing.
+constexpr int kPairStageBytes = 128 * BK * 2 * 2;           // A 16 KB + half of B 16 KB
+constexpr int kPairStages = kSmemBudget / kPairStageBytes;  // 6
+constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + 1024;
+
+struct PairTile {
+  int e, m0, rows, n0, gm;
+  bool valid;  // this CTA's m-tile exists (else rows = 0)
+};
+
+// Pair tile `tile` of a phase with ntn n-tiles; s_mp[e] = first m-tile pair of expert e.
+__device__ __forceinline__ PairTile decode_pair_tile(int tile, int N, int bn, int ntn, int rank,
+                                                     const int* s_mp, const int* s_mt,
+                                                     const int* s_off) {
+  int lo = 0, hi = N - 1;  // largest e with s_mp[e] * ntn <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_mp[mid] * ntn <= tile)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  PairTile c;
+  c.e = lo;
+  const int local = tile - s_mp[lo] * ntn;
+  const int np = s_mp[lo + 1] - s_mp[lo];
+  const int nt = local / np;
+  const int mi = 2 * (local - nt * np) + rank;
+  c.valid = mi < s_mt[lo + 1] - s_mt[lo];
+  c.m0 = s_off[lo] + mi * 128;
+  c.rows = c.valid ? min(128, s_off[lo + 1] - c.m0) : 0;
+  c.n0 = nt * bn;
+  c.gm = s_mt[lo] + mi;
+  return c;
+}
+
+template <int EPI1, int BN1>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_ffn_pair_kernel(const __grid_constant__ CUtensorMap tmA1,
+                            const __grid_constant__ CUtensorMap tmB1,
+                            const __grid_constant__ CUtensorMap tmA2,
+                            const __grid_constant__ CUtensorMap tmB2, const FfnParams p) {
+  static_assert(EPI1 != EPI_SWIGLU || 2 * BN1 == kUmmaN, "SwiGLU tile: gate | up halves");
+  static_assert(EPI1 == EPI_SWIGLU || BN1 == kUmmaN, "GELU tile");
+  extern __shared__ __align__(1024) uint8_t dyn_smem[];
+  __shared__ __align__(8) uint64_t full_bar[kPairStages];   // even CTA: both CTAs' bytes
+  __shared__ __align__(8) uint64_t empty_bar[kPairStages];  // both CTAs (multicast commit)
+  __shared__ __align__(8) uint64_t tfull_bar[2];            // both CTAs (multicast commit)
+  __shared__ __align__(8) uint64_t tempty_bar[2];           // even CTA: both epilogues
+  __shared__ __align__(8) uint64_t done_bar;
+  __shared__ __align__(8) uint64_t epi_bar;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ volatile int s_abort;
+  __shared__ int s_mt[257], s_mp[257], s_off[257];
+  __shared__ int s_tiles[2];
+  __shared__ int s_last_cta;
+
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = p.n_experts;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const bool lead = rank == 0;
+  const int cl = static_cast<int>(blockIdx.x) >> 1, ncl = static_cast<int>(gridDim.x) >> 1;
+  const uint32_t tiles0 = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  auto a_addr = [&](int s) -> uint32_t { return tiles0 + s * kPairStageBytes; };
+  auto b_addr = [&](int s) -> uint32_t { return tiles0 + s * kPairStageBytes + 128 * BK * 2; };
+
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tmA1);
+    prefetch_tensormap(&tmB1);
+    prefetch_tensormap(&tmA2);
+    prefetch_tensormap(&tmB2);
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&tfull_bar[b]), 1);
+      mbar_init(smem_u32(&tempty_bar[b]), 2 * kEpiThreads);
+    }
+    mbar_init(smem_u32(&done_bar), 1);
+    mbar_init(smem_u32(&epi_bar), kEpiThreads);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tmem_alloc_pair(smem_u32(&s_tmem_base), 2 * kUmmaN);
+    tmem_relinquish_pair();
+  }
+  pdl_wait();  // below: reads of the previous kernels' outputs and writes to global memory
+  if (warp == 2) {
+    // per-expert m-tiles and m-tile pairs, and their exclusive prefixes (serial over experts
+    // in steps of 32)
+    int acc_t = 0, acc_p = 0;
+    bool bad = false;
+    for (int e0 = 0; e0 < N; e0 += 32) {
+      const int e = e0 + lane;
+      int ct = 0;
+      if (e < N) {
+        const int a = p.expert_offset[e], b = p.expert_offset[e + 1];
+        s_off[e] = a;
+        if (a < 0 || b < a || b > p.r_max || b - a > p.rows_per_expert)
+          bad = true;
+        else
+          ct = (b - a + 127) / 128;
+      }
+      const int cp = (ct + 1) / 2;
+      int it = ct, ip = cp;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ut = __shfl_up_sync(0xffffffffu, it, o);
+        const int up = __shfl_up_sync(0xffffffffu, ip, o);
+        if (lane >= o) {
+          it += ut;
+          ip += up;
+        }
+      }
+      if (e < N) {
+        s_mt[e] = acc_t + it - ct;
+        s_mp[e] = acc_p + ip - cp;
+      }
+      acc_t += __shfl_sync(0xffffffffu, it, 31);
+      acc_p += __shfl_sync(0xffffffffu, ip, 31);
+    }
+    bad = __any_sync(0xffffffffu, bad) || acc_t > p.m_tiles_cap;
+    if (lane == 0) {
+      s_off[N] = p.expert_offset[N];
+      s_mt[N] = acc_t;
+      s_mp[N] = bad ? 0 : acc_p;  // bad offsets: no tiles
+      for (int ph = 0; ph < 2; ++ph) s_tiles[ph] = s_mp[N] * p.ph[ph].n_tiles_n;
+      if (bad) report_error(p.status, MOE_ERR_BOUNDS);
+    }
+  }
+  tc_fence_before_sync();
+  cluster_sync_all();  // both CTAs' barriers and TMEM exist before either uses the other's
+  tc_fence_after_sync();
+  const uint32_t tmem_base = s_tmem_base;
+  const int h_target = p.ph[0].n_tiles_n;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer (each CTA)
+    if (lane == 0) {
+      const uint64_t pol_a = make_policy(2);
+      const uint64_t pol_b = make_policy(p.weight_policy);
+      int it = 0;
+      bool ok = true;
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        const int bn = ph == 0 ? BN1 : kDnBn;
+        const CUtensorMap* tA = ph == 0 ? &tmA1 : &tmA2;
+        const int nkb = p.ph[ph].num_kb;
+        for (int tile = cl; ok && tile < s_tiles[ph]; tile += ncl) {
+          const PairTile c = decode_pair_tile(tile, N, bn, p.ph[ph].n_tiles_n, rank, s_mp, s_mt, s_off);
+          bool ready = ph == 0 || !c.valid || ld_acquire_gpu(p.h_ready + c.gm) >= h_target;
+          int pend_from = -1;
+          const int it0 = it;
+          for (int kb = 0; kb < nkb; ++kb) {
+            const int s = it % kPairStages;
+            if (!mbar_wait(smem_u32(&empty_bar[s]), ((it / kPairStages) & 1) ^ 1u, p.timeout_ns, &s_abort)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = smem_u32(&full_bar[s]);
+            const uint32_t fb0 = map_smem_to_rank(fb, 0);
+            if (lead) mbar_arrive_expect_tx(fb, 2 * kPairStageBytes);
+            // this CTA's half of the 256 weight rows
+            if (ph == 0 && EPI1 == EPI_SWIGLU)
+              tma_load_4d_pair(b_addr(s), &tmB1, fb0, kb * BK, c.n0, rank, c.e, pol_b);
+            else
+              tma_load_3d_pair(b_addr(s), ph == 0 ? &tmB1 : &tmB2, fb0, kb * BK, c.n0 + 128 * rank,
+                               c.e, pol_b);
+            if (ready) {
+              tma_load_2d_pair(a_addr(s), tA, fb0, kb * BK, c.m0, pol_a);
+              ++it;
+              continue;
+            }
+            if (pend_from < 0) pend_from = it;
+            if (it - pend_from + 1 == kPairStages || kb + 1 == nkb) {
+              // every stage holds a W_d block (or the tile ends): wait for the rows' h
+              if (!wait_counter_at_least(p.h_ready + c.gm, h_target, p.timeout_ns, &s_abort))
+                ok = false;  // the h loads below still complete the armed stages
+              fence_proxy_async_global();
+              for (int j = pend_from; j <= it; ++j) {
+                const int sj = j % kPairStages;
+                tma_load_2d_pair(a_addr(sj), tA, map_smem_to_rank(smem_u32(&full_bar[sj]), 0),
+                                 (j - it0) * BK, c.m0, pol_a);
+              }
+              pend_from = -1;
+              ready = true;
+            }
+            ++it;
+            if (!ok) break;
+          }
+        }
+      }
+      if (!ok) {
+        s_abort = 1;
+        report_error(p.status, MOE_ERR_TIMEOUT);
+      }
+      if (lead) {
+        for (int i = max(0, it - kPairStages); i < it; ++i)
+          mbar_wait(smem_u32(&full_bar[i % kPairStages]), (i / kPairStages) & 1, kDrainTimeoutNs, nullptr);
+      } else {
+        // the odd CTA's copies complete on the even CTA's barriers: wait until the MMAs have
+        // released its last stages, within one overall limit
+        const uint64_t t_end = globaltimer_ns() + 1000000ull;
+        for (int i = max(0, it - kPairStages); i < it; ++i) {
+          const uint64_t now = globaltimer_ns();
+          mbar_wait(smem_u32(&empty_bar[i % kPairStages]), (i / kPairStages) & 1,
+                    now < t_end ? t_end - now : 1, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (even CTA)
+    if (lane == 0 && lead) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, kUmmaN);
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        const int nkb = p.ph[ph].num_kb;
+        for (int tile = cl; ok && tile < s_tiles[ph]; tile += ncl, ++tc) {
+          const int buf = tc & 1;
+          if (!mbar_wait(smem_u32(&tempty_bar[buf]), ((tc >> 1) & 1) ^ 1u, p.timeout_ns, &s_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kUmmaN);
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = it % kPairStages;
+            if (!mbar_wait(smem_u32(&full_bar[s]), (it / kPairStages) & 1, p.timeout_ns, &s_abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              tc_mma_f16_pair(d_tmem, smem_desc_k_sw128(a_addr(s) + kk * 32),
+                              smem_desc_k_sw128(b_addr(s) + kk * 32), idesc,
+                              (kb | kk) != 0 ? 1u : 0u);
+            tc_commit_pair(smem_u32(&empty_bar[s]), 0x3);
+          }
+          if (!ok) break;
+          tc_commit_pair(smem_u32(&tfull_bar[buf]), 0x3);
+        }
+      }
+      if (!ok) {
+        s_abort = 1;
+        report_error(p.status, MOE_ERR_TIMEOUT);
+      }
+      // always signalled, so the odd CTA's wait below ends with the MMAs
+      tc_commit_pair(smem_u32(&done_bar), 0x3);
+      mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
+    } else if (lane == 0) {
+      mbar_wait(smem_u32(&done_bar), 0, kDrainTimeoutNs, nullptr);
+    }
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;
+    const int r_local = q * 32 + lane;
+    int tc = 0;
+    uint32_t epi_phase = 0;
+    bool ok = true;
+    for (int ph = 0; ph < 2 && ok; ++ph) {
+      const int bn = ph == 0 ? BN1 : kDnBn;
+      const PhaseParams& pp = p.ph[ph];
+      for (int tile = cl; tile < s_tiles[ph]; tile += ncl, ++tc) {
+        const PairTile c = decode_pair_tile(tile, N, bn, pp.n_tiles_n, rank, s_mp, s_mt, s_off);
+        const int buf = tc & 1;
+        const bool got = mbar_wait(smem_u32(&tfull_bar[buf]), (tc >> 1) & 1, p.timeout_ns, &s_abort);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(buf * kUmmaN);
+        const bool row_ok = r_local < c.rows;
+        const int64_t row = static_cast<int64_t>(c.m0) + r_local;
+#pragma unroll 1
+        for (int cc = 0; cc < bn; cc += 16) {
+          if (c.n0 + cc >= pp.n_out) break;  // warp-uniform: ragged last n-tile
+          float a[16], b[16];
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_row + cc, v);
+          if (ph == 0 && EPI1 == EPI_SWIGLU) {
+            uint32_t u[16];
+            tmem_ld_32x32b_x16(t_row + BN1 + cc, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) b[i] = __uint_as_float(u[i]);
+          } else {
+            tmem_ld_wait();
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(v[i]);
+          if (!row_ok) continue;
+          if (ph == 0)
+            store_final16<EPI1>(pp, row, c.n0 + cc, a, b);
+          else
+            store_final16<EPI_STORE_F32>(pp, row, c.n0 + cc, a, b);
+        }
+        tc_fence_before_sync();
+        // the accumulator buffer is free once both CTAs' epilogues have read it
+        if (lead)
+          mbar_arrive(smem_u32(&tempty_bar[buf]));
+        else
+          mbar_arrive_cluster(map_smem_to_rank(smem_u32(&tempty_bar[buf]), 0));
+        if (ph == 0 && c.valid) {
+          // this CTA wrote the tile's h: order it before TMA loads, then count it
+          fence_proxy_async_global();
+          if (!__all_sync(0xffffffffu, epilogue_sync(smem_u32(&epi_bar), epi_phase, p.timeout_ns, &s_abort))) {
+            ok = false;
+            break;
+          }
+          if (threadIdx.x == 64) {
+            __threadfence();
+            atomicAdd(p.h_ready + c.gm, 1);
+          }
+        }
+      }
+    }
+    if (!ok) {
+      s_abort = 1;
+      report_error(p.status, MOE_ERR_TIMEOUT);
+    }
+  }
+
+  tc_fence_before_sync();
+  cluster_sync_all();  // neither CTA of a pair frees TMEM or exits while the other works
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc_pair(tmem_base, 2 * kUmmaN);
+  }
+  // the last CTA to finish zeroes the m-tile counters for the next call
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last_cta = atomicAdd(p.done_ctas, 1) == static_cast<int>(gridDim.x) - 1;
+  }
+  __syncthreads();
+  if (s_last_cta) {
+    __threadfence();
+    for (int i = threadIdx.x; i < s_mt[N]; i += kThreads) p.h_ready[i] = 0;
+    if (threadIdx.x == 0) *p.done_ctas = 0;
+  }
+}
+
 // Block-scaled formats: the token rows x_perm as MXFP8 (the A operand of the gate/up GEMM).
 // Slot (gm, r) is row r of m-tile gm (the tiles of the grouped FFN: experts in order, 128
 // rows each, the last one of an expert partial). A valid row's 32-column blocks become E4M3
@@ -1330,6 +1687,19 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t* __re
 }
 
 // ------------------------------------------------------------------ host side
+template <int EPI1, int BN1>
+cudaError_t launch_pair(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
+                        const CUtensorMap& b2, const FfnParams& fp, int grid, cudaStream_t s) {
+  static PerDeviceOnce once;
+  const cudaError_t attr_err = once.run([] {
+    return cudaFuncSetAttribute(grouped_ffn_pair_kernel<EPI1, BN1>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  return launch_pdl_cluster(grouped_ffn_pair_kernel<EPI1, BN1>, dim3(grid), dim3(kThreads),
+                            kPairSmemBytes, s, 2u, a1, b1, a2, b2, fp);
+}
+
 template <int EPI1, int BN1, int BM, int WFMT>
 cudaError_t launch_one(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
                        const CUtensorMap& b2, const CUtensorMap& s1, const CUtensorMap& s2,
@@ -1580,7 +1950,22 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   }
   }  // not block-scaled
 
-  const bool stream_k = a.part != nullptr;
+  // CTA pairs for bf16 weights when the experts average at least four 128-row m-tiles (the
+  // tensor-bound regime): whole tiles, weight boxes of 128 rows
+  const bool pair = a.wfmt == MOE_WFMT_BF16 && bm == 128 && a.r_max >= 512LL * a.N;
+  if (pair) {
+    if (!swiglu) {
+      const uint64_t dims[3] = {d, F, N};
+      const uint64_t str[2] = {d * 2, F * d * 2};
+      const uint32_t box[3] = {BK, 128, 1};
+      if (!make_map(&mB1, a.w_gate_up, 3, dims, str, box)) return cudaErrorInvalidValue;
+    }
+    const uint64_t dims[3] = {F, d, N};
+    const uint64_t str[2] = {F * 2, d * F * 2};
+    const uint32_t box[3] = {BK, 128, 1};
+    if (!make_map(&mB2, a.w_down, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  const bool stream_k = a.part != nullptr && !pair;
   FfnParams fp{};
   fp.expert_offset = a.expert_offset;
   fp.r_max = a.r_max;
@@ -1624,6 +2009,11 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   const int64_t useful = std::max(useful_ctas(plan.tiles1_ub, p1.num_kb, p1.sk_ctas),
                                   useful_ctas(plan.tiles2_ub, p2.num_kb, p2.sk_ctas));
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(useful, di.sm_count)));
+  if (pair) {
+    const int pgrid = 2 * std::max(1, std::min(di.sm_count / 2, static_cast<int>((useful + 1) / 2)));
+    return swiglu ? launch_pair<EPI_SWIGLU, kGuBnSwiglu>(mA1, mB1, mA2, mB2, fp, pgrid, s)
+                  : launch_pair<EPI_GELU, kGuBnGelu>(mA1, mB1, mA2, mB2, fp, pgrid, s);
+  }
   if (bs) {
     const int qgrid = static_cast<int>(std::min<int64_t>(
         std::max<int64_t>(1, (plan.m_tiles_ub * 128 + 7) / 8), static_cast<int64_t>(di.sm_count) * 8));
