@@ -1950,9 +1950,10 @@ cudaError_t launch_grouped_ffn(const GroupedFfnArgs& a, cudaStream_t s) {
   }
   }  // not block-scaled
 
-  // CTA pairs for bf16 weights when the experts average at least four 128-row m-tiles (the
-  // tensor-bound regime): whole tiles, weight boxes of 128 rows
-  const bool pair = a.wfmt == MOE_WFMT_BF16 && bm == 128 && a.r_max >= 512LL * a.N;
+  // CTA pairs for bf16 weights when the experts average at least eight 128-row m-tiles (the
+  // tensor-bound regime): whole tiles, weight boxes of 128 rows. An expert's odd last m-tile
+  // costs a whole pair tile, which at four m-tiles per expert outweighs the gain.
+  const bool pair = a.wfmt == MOE_WFMT_BF16 && bm == 128 && a.r_max >= 1024LL * a.N;
   if (pair) {
     if (!swiglu) {
       const uint64_t dims[3] = {d, F, N};
