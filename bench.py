@@ -12,7 +12,8 @@ write-back. A second pass replays the stages as separate graphs with events betw
 the per-stage breakdown and the grouped FFN's roofline. The end-to-end figure (e2e) calls
 moe_forward eagerly, with the H2D copy of the tokens and the D2H copy of the output of every
 step inside its timed region; the copies run on their own streams and overlap the
-neighbouring steps' compute. Under torchrun every rank runs its own replica of the workload
+neighbouring steps' compute. Its `copies_only` entry times the same copies with no forward
+between them, the host link's floor under the end-to-end figure. Under torchrun every rank runs its own replica of the workload
 (weak scaling, no collective on the data path). Rank 0 prints the line, with the time taken
 as the max over ranks.
 
@@ -601,6 +602,36 @@ class Layer:
             g.replay()
             ev[n + 1].record()
 
+    def e2e_copies(self, steps: int, warmup: int):
+        """The copies of e2e_pipeline alone: per step the H2D of the tokens and the D2H of an
+        output buffer, on the same two copy streams and pinned buffers, with no forward between
+        them. Returns the elapsed ms of `steps` steps, first H2D to last D2H on the device: the
+        floor under the end-to-end figure that the host link sets."""
+        i = self.inp
+        T, d = self.T, self.shape.d_model
+        x_host = [i["x"].cpu().pin_memory() for _ in range(2)]
+        out_host = [torch.empty((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        x_dev = [torch.empty_like(i["x"]) for _ in range(2)]
+        out_dev = [torch.zeros_like(i["x"]) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        s_in.wait_stream(torch.cuda.current_stream())
+        s_out.wait_stream(torch.cuda.current_stream())
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for n in range(warmup + steps):
+            b = n % 2
+            if n == warmup:
+                s_in.wait_stream(s_out)
+                s_out.wait_stream(s_in)
+                t0.record(s_in)
+            with torch.cuda.stream(s_in):
+                x_dev[b].copy_(x_host[b], non_blocking=True)
+            with torch.cuda.stream(s_out):
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+        s_in.wait_stream(s_out)
+        t1.record(s_in)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
+
     def e2e_pipeline(self, steps: int, warmup: int):
         """End to end through the public call, as a serving loop would run it: every step
         copies its tokens from pinned host memory (H2D), runs moe_forward, and copies the
@@ -643,6 +674,19 @@ class Layer:
         t1.record(s_comp)
         torch.cuda.synchronize()
         return t0.elapsed_time(t1)
+
+
+def e2e_entry(T: int, d: int, steps: int, world: int, e2e_ms: float, copies_ms: float) -> dict:
+    """The end-to-end figure and its bound: the same steps' host copies alone (H2D of x and
+    D2H of out, both directions at once), as tokens/s and as the copies' rate in GB/s."""
+    nbytes = T * d * 2
+    e2e = tokens_per_second(T, steps, world, e2e_ms)
+    floor = tokens_per_second(T, steps, world, copies_ms)
+    return {"value": round(e2e, 1), "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+            "d2h_bytes_per_step": nbytes,
+            "copies_only": {"value": round(floor, 1), "unit": "tokens/s",
+                            "gbs_per_direction": round(nbytes * steps / (copies_ms * 1e-3) / 1e9, 1),
+                            "frac": round(e2e / floor, 4)}}
 
 
 def reduce_max(values, world: int, device) -> list:
@@ -806,8 +850,9 @@ def run_gpu(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     e2e_ms = layer.e2e_pipeline(args.steps, args.warmup)
+    copies_ms = layer.e2e_copies(args.steps, args.warmup)
 
-    total_ms, e2e_ms = reduce_max([total_ms, e2e_ms], world, device)
+    total_ms, e2e_ms, copies_ms = reduce_max([total_ms, e2e_ms, copies_ms], world, device)
 
     R, active = routing_counts(layer)
     traffic = MEASURED_FFN_TRAFFIC.get((shape.name, T)) if args.wfmt == "bf16" else None
@@ -845,9 +890,7 @@ def run_gpu(args, rank, world, local_rank):
         "backward": backward,
         "roofline": roof,
         "layer": roof_all["layer"],
-        "e2e": {"value": round(tokens_per_second(T, args.steps, world, e2e_ms), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": T * shape.d_model * 2,
-                "d2h_bytes_per_step": T * shape.d_model * 2},
+        "e2e": e2e_entry(T, shape.d_model, args.steps, world, e2e_ms, copies_ms),
         "gpu_launches": launches_per_step(T, shape.top_k, layer.R_max, shape.n_experts,
                                           shape.d_model) * args.steps,
         "clocks": clk,
