@@ -25,6 +25,9 @@ SMALL_CASES = [
     ("splitk_decode_gelu", 5, 256, 16, 1, 2048, "gelu", None, None),
     ("splitk_decode_deep_k", 2, 4096, 8, 2, 2048, "swiglu", None, None),
     ("splitk_decode_ragged_n", 7, 2880, 32, 4, 2880, "swiglu", None, None),
+    # at most two rows per expert, GELU and both tokens in both experts
+    ("gemv_decode_gelu", 2, 384, 16, 2, 1088, "gelu", None, None),
+    ("gemv_two_rows_per_expert", 2, 576, 2, 2, 768, "swiglu", None, None),
     # large enough that the router runs on tensor cores (T*N*d*4 bytes > 256 MiB);
     # expert counts padded to 16, 32, 64, 128 (N=100) and 256 tensor-core columns
     ("tc_router_n8_bias", 20000, 512, 8, 2, 128, "swiglu", 1.25, 1.1),

@@ -21,10 +21,10 @@ def _forward(dims, inp, ws, out):
 
 # per-token router, decode-sized one-launch router, tensor-core router (T * N * d * 4 > 256 MiB),
 # the tensor-core router on CTA pairs (76 tiles, 256 experts), the grouped FFN on CTA pairs
-# (R_max >= 512 N)
+# (R_max >= 1024 N), and a single token (one-launch router, stream-K grouped FFN)
 @pytest.mark.parametrize("T,d,N,k,F", [(512, 1024, 8, 2, 2048), (3, 512, 8, 2, 1024),
                                        (4096, 1024, 64, 1, 1024), (9728, 512, 256, 8, 256),
-                                       (4096, 512, 4, 2, 512)])
+                                       (4096, 512, 4, 2, 512), (1, 512, 8, 2, 1024)])
 def test_wait_timeout_reported_and_context_survives(T, d, N, k, F):
     inp = synthetic.make_custom_inputs(T, d, N, F, "swiglu", seed=4, device="cuda")
     dims = moe.make_dims(T, d, N, k, F, "swiglu", T)
