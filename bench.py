@@ -208,11 +208,11 @@ MEASURED_FFN_TRAFFIC = {
     ("mixtral", 1): 709.46e6 + 3.15e6,
     ("mixtral", 16): 2.82e9 + 4.78e6,
     ("mixtral", 512): 2.86e9 + 45.51e6,
-    ("mixtral", 8192): 4.39e9 + 730.11e6,
+    ("mixtral", 8192): 5.83e9 + 726.43e6,  # the CTA-pair kernel
     ("gpt_oss", 1): 201.80e6 + 3.36e6,
     ("gpt_oss", 8): 958.33e6 + 3.38e6,
     ("gpt_oss", 64): 1.61e9 + 5.67e6,
-    ("gpt_oss", 16384): 2.35e9 + 1.09e9,
+    ("gpt_oss", 16384): 2.64e9 + 1.10e9,  # the CTA-pair kernel
     ("fine_grained", 16384): 19.44e9 + 181.11e6,
 }
 
