@@ -551,7 +551,10 @@ __global__ void __launch_bounds__(256) act_bwd_kernel(const float* __restrict__ 
 // ------------------------------------------------------------------ router weight gradient
 // dW_r = dL^T x in fp32, in two passes with a fixed summation order: chunk c of the tokens
 // adds its tokens in order into part[c][n][col] (thread = column, 16 experts a block), then
-// the chunks are added in order. db[n] = sum_t dL[t, n]: warp w of a block adds tokens
+// the chunks are added in order. dL is zero except on each token's k chosen experts (the
+// renormalised weights depend on those logits only), so a block adds only the tokens with a
+// chosen expert among its 16: the same sums in the same order, without the terms that are
+// exactly zero. db[n] = sum_t dL[t, n]: warp w of a block adds tokens
 // t = w mod 32 in order for 32 experts, and the 32 warp sums are added in warp order.
 constexpr int kRwExperts = 16;
 constexpr int kRwTokens = 64;
@@ -560,6 +563,8 @@ __global__ void __launch_bounds__(256) router_wgrad_partial_kernel(
     const float* __restrict__ d_logits, const uint16_t* __restrict__ x, float* __restrict__ part,
     int T, int d, int N, int chunk) {
   __shared__ float s_dl[kRwTokens][kRwExperts];
+  __shared__ int s_list[kRwTokens];  // the staged tokens with a nonzero dL here, in order
+  __shared__ int s_nz;
   pdl_wait();
   pdl_trigger();
   const int col = blockIdx.x * 256 + threadIdx.x;
@@ -576,19 +581,36 @@ __global__ void __launch_bounds__(256) router_wgrad_partial_kernel(
           (tt < t1 && n < N) ? d_logits[static_cast<int64_t>(tt) * N + n] : 0.f;
     }
     __syncthreads();
+    if (threadIdx.x < 32) {  // staged dL rows past the chunk's end are zero: never listed
+      const int lane = threadIdx.x;
+      int base = 0;
+      for (int h = 0; h < kRwTokens; h += 32) {
+        bool nz = false;
+#pragma unroll
+        for (int i = 0; i < kRwExperts; ++i) nz |= s_dl[h + lane][i] != 0.f;
+        const unsigned m = __ballot_sync(0xffffffffu, nz);
+        if (nz) s_list[base + __popc(m & ((1u << lane) - 1u))] = h + lane;
+        base += __popc(m);
+      }
+      if (lane == 0) s_nz = base;
+    }
+    __syncthreads();
     if (col < d) {
-      const int nt = min(kRwTokens, t1 - tb);
-      // eight tokens' loads in flight at once; the additions keep token order (staged dL rows
-      // past the chunk's end are zero)
-      for (int tt = 0; tt < nt; tt += 8) {
+      const int nz = s_nz;
+      // eight listed tokens' loads in flight at once; the additions keep token order
+      for (int u0 = 0; u0 < nz; u0 += 8) {
+        int tl[8];
         float xv[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          xv[u] = tt + u < nt ? bf16_bits_to_float(x[static_cast<int64_t>(tb + tt + u) * d + col]) : 0.f;
+        for (int u = 0; u < 8; ++u) {
+          tl[u] = u0 + u < nz ? s_list[u0 + u] : -1;
+          xv[u] = tl[u] >= 0 ? bf16_bits_to_float(x[static_cast<int64_t>(tb + tl[u]) * d + col]) : 0.f;
+        }
 #pragma unroll
         for (int u = 0; u < 8; ++u)
+          if (tl[u] >= 0)
 #pragma unroll
-          for (int i = 0; i < kRwExperts; ++i) acc[i] += s_dl[tt + u][i] * xv[u];
+            for (int i = 0; i < kRwExperts; ++i) acc[i] += s_dl[tl[u]][i] * xv[u];
       }
     }
   }
